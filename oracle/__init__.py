@@ -1,0 +1,138 @@
+"""fp64 CPU oracle for the gated delta rule (TEST INFRASTRUCTURE).
+
+Only ``tests/``, ``__graft_entry__.smoke()`` and the CPU-baseline leg of
+``bench.py`` may import this package. The CUDA library and its Python binding
+never import it. The arithmetic lives in ``gdn_oracle.c`` (plain sequential fp64
+loops, one token at a time; see its header for the definition it follows); this
+module only compiles it with gcc, converts arrays to fp64 and marshals pointers.
+
+Parity pins: the oracle is checked, in ``tests/test_oracle_pins.py``, against
+exact rational brute force (explicit products of the per-token update matrices),
+closed forms (single token, alpha = 0, key overwrite), invariants (beta = 0 and
+alpha = 1 leave S unchanged; Householder reflection preserves the Frobenius
+norm; the norm bound of a contraction), an independent fp64 chunked (WY) form,
+and decode/prefill/varlen consistency identities.
+"""
+from __future__ import annotations
+
+import ctypes
+import os
+import subprocess
+import threading
+
+import numpy as np
+
+_HERE = os.path.dirname(os.path.abspath(__file__))
+_SRC = os.path.join(_HERE, "gdn_oracle.c")
+_LIB_PATH = os.path.join(_HERE, "libgdn_oracle.so")
+_lib = None
+_lock = threading.Lock()
+
+
+def build(force: bool = False) -> str:
+    """Compile gdn_oracle.c into oracle/libgdn_oracle.so with gcc (-O2, pthreads)."""
+    if force or not os.path.exists(_LIB_PATH) or os.path.getmtime(_LIB_PATH) < os.path.getmtime(_SRC):
+        cmd = ["gcc", "-O2", "-fPIC", "-shared", "-std=c99", "-D_POSIX_C_SOURCE=200809L",
+               "-o", _LIB_PATH, _SRC, "-lm", "-lpthread"]
+        subprocess.check_call(cmd)
+    return _LIB_PATH
+
+
+def load_library(path: str):
+    """Load an oracle build from an explicit path (used by the mutation tests)."""
+    lib = ctypes.CDLL(path)
+    _declare(lib)
+    return lib
+
+
+def _declare(lib):
+    dp = ctypes.POINTER(ctypes.c_double)
+    lib.gdn_oracle_prefill.restype = ctypes.c_int
+    lib.gdn_oracle_prefill.argtypes = [dp, dp, dp, dp, dp, ctypes.POINTER(ctypes.c_int64),
+                                       ctypes.c_int, ctypes.c_int, ctypes.c_int, ctypes.c_int,
+                                       ctypes.c_double, dp, dp, dp, ctypes.c_int]
+    lib.gdn_oracle_decode.restype = ctypes.c_int
+    lib.gdn_oracle_decode.argtypes = [dp, dp, dp, dp, dp, dp, ctypes.c_int,
+                                      ctypes.POINTER(ctypes.c_int32), dp,
+                                      ctypes.c_int, ctypes.c_int, ctypes.c_int, ctypes.c_int,
+                                      ctypes.c_int, ctypes.c_int, ctypes.c_double, ctypes.c_int]
+
+
+def _load():
+    global _lib
+    with _lock:
+        if _lib is None:
+            build()
+            lib = ctypes.CDLL(_LIB_PATH)
+            _declare(lib)
+            _lib = lib
+    return _lib
+
+
+def f64(x) -> np.ndarray:
+    """Exact fp64 copy of a numpy array or torch tensor (bf16/fp32 upcast exactly)."""
+    if x is None:
+        return None
+    try:
+        import torch
+        if isinstance(x, torch.Tensor):
+            return np.ascontiguousarray(x.detach().to("cpu", torch.float64).numpy())
+    except ImportError:  # pragma: no cover
+        pass
+    return np.ascontiguousarray(np.asarray(x, dtype=np.float64))
+
+
+def _ptr(a, ctype=ctypes.c_double):
+    if a is None:
+        return None
+    return a.ctypes.data_as(ctypes.POINTER(ctype))
+
+
+def prefill(q, k, v, g, beta, cu_seqlens, initial_state=None, scale=None, nthreads=0, lib=None):
+    """Sequential fp64 prefill over packed sequences.
+
+    q, k: [total_T, H, dk]; v: [total_T, H, dv]; g, beta: [total_T, H];
+    cu_seqlens: [N + 1]; initial_state: [N, H, dv, dk] or None (zero state).
+    Returns (o [total_T, H, dv], final_state [N, H, dv, dk], threads_used), fp64.
+    """
+    lib = lib or _load()
+    q, k, v, g, beta = (f64(a) for a in (q, k, v, g, beta))
+    cu = np.ascontiguousarray(np.asarray(f64(cu_seqlens), dtype=np.int64))
+    init = f64(initial_state)
+    total_T, H, dk = q.shape
+    dv = v.shape[-1]
+    N = cu.shape[0] - 1
+    if scale is None:
+        scale = 1.0 / np.sqrt(dk)
+    o = np.zeros((total_T, H, dv), np.float64)
+    fin = np.zeros((N, H, dv, dk), np.float64)
+    rc = lib.gdn_oracle_prefill(_ptr(q), _ptr(k), _ptr(v), _ptr(g), _ptr(beta),
+                                _ptr(cu, ctypes.c_int64), N, H, dk, dv, float(scale), _ptr(init),
+                                _ptr(o), _ptr(fin), int(nthreads))
+    if rc < 0:
+        raise ValueError("gdn_oracle_prefill: bad arguments")
+    return o, fin, rc
+
+
+def decode(q, k, v, g, beta, pool, slot_ids, scale=None, nthreads=0, lib=None):
+    """Sequential fp64 decode over a slot-indexed pool (the pool copy is updated).
+
+    q: [B, T, H, dk]; k: [B, T, H, nh, dk]; v: [B, T, H, nh, dv]; g: [B, T, H];
+    beta: [B, T, H, nh]; pool: [num_slots, H, dv, dk]; slot_ids: [B].
+    Returns (o [B, T, H, dv], new_pool, threads_used), fp64.
+    """
+    lib = lib or _load()
+    q, k, v, g, beta = (f64(a) for a in (q, k, v, g, beta))
+    pool = f64(pool).copy()
+    slots = np.ascontiguousarray(np.asarray(f64(slot_ids), dtype=np.int32))
+    B, T, H, dk = q.shape
+    nh, dv = v.shape[3], v.shape[4]
+    if scale is None:
+        scale = 1.0 / np.sqrt(dk)
+    o = np.zeros((B, T, H, dv), np.float64)
+    rc = lib.gdn_oracle_decode(_ptr(q), _ptr(k), _ptr(v), _ptr(g), _ptr(beta), _ptr(pool),
+                               pool.shape[0], _ptr(slots, ctypes.c_int32), _ptr(o),
+                               B, T, H, dk, dv, nh, float(scale), int(nthreads))
+    if rc < 0:
+        raise ValueError("gdn_oracle_decode: bad arguments")
+    return o, pool, rc

@@ -1,0 +1,216 @@
+/*
+ * Gated delta rule: plain, sequential, fp64 CPU oracle.
+ *
+ * TEST INFRASTRUCTURE. Only the tests, the package's smoke check and the
+ * benchmark's CPU-baseline leg may load this library. The CUDA library never
+ * links, calls or includes anything from here, and this file includes nothing
+ * from the CUDA sources.
+ *
+ * What it computes (per sequence or slot, per head, tokens in order):
+ *
+ *   gated delta rule (Yang, Kautz, Hatamizadeh, "Gated Delta Networks:
+ *   Improving Mamba2 with Delta Rule", ICLR 2025, eq. for the gated delta
+ *   update):
+ *       S_t = alpha_t (I - beta_t k_t k_t^T) S_{t-1} + beta_t k_t v_t^T,
+ *       o_t = scale * S_t^T q_t,          alpha_t = exp(g_t),
+ *   with S_t of shape dk x dv.
+ *
+ *   gated delta product (the multi-Householder variant named by the kernel
+ *   family cake_gated_delta_product_mtp on the FlashInfer PR #7156 page,
+ *   "Cake GDP kernel: shared-memory reduction and direct register loads",
+ *   introduction): per token one gate, then n_h Householder updates in order
+ *   j = 1..n_h, then one output:
+ *       S <- alpha_t S
+ *       S <- (I - beta_{t,j} k_{t,j} k_{t,j}^T) S + beta_{t,j} k_{t,j} v_{t,j}^T
+ *       o_t = scale * S^T q_t
+ *   With n_h = 1 this is the gated delta rule above, since
+ *   (I - b k k^T)(a S) = a (I - b k k^T) S.
+ *
+ * Storage: states are kept K-last, i.e. S^T row-major [dv][dk], the layout the
+ * FlashInfer PR #7156 page (section 1) indexes as state + row + k_col and the
+ * FlashInfer PR #3866 page (section 2, accumulate_state_fragment) contracts over
+ * the second index. Everything here is fp64; inputs arrive as fp64 copies of the
+ * exact values the GPU reads.
+ */
+#include <math.h>
+#include <pthread.h>
+#include <stdint.h>
+#include <stdlib.h>
+#include <string.h>
+#include <unistd.h>
+
+/* ---- the three steps of one token, on one head, state St = S^T [dv][dk] ---- */
+
+/* S <- alpha S */
+static void apply_gate(double* St, double alpha, int dk, int dv) {
+  for (int j = 0; j < dv; ++j)
+    for (int i = 0; i < dk; ++i) St[(size_t)j * dk + i] *= alpha;
+}
+
+/* S <- (I - beta k k^T) S + beta k v^T, one column S[:, j] (= row j of St) at a
+ * time: p = k^T S[:, j];  S[:, j] <- S[:, j] - beta k p + beta k v_j. */
+static void apply_householder(double* St, const double* k, const double* v, double beta,
+                              int dk, int dv) {
+  for (int j = 0; j < dv; ++j) {
+    double* col = St + (size_t)j * dk;
+    double p = 0.0;
+    for (int i = 0; i < dk; ++i) p += k[i] * col[i];
+    for (int i = 0; i < dk; ++i) col[i] = col[i] - beta * k[i] * p + beta * k[i] * v[j];
+  }
+}
+
+/* o = scale * S^T q */
+static void emit_output(const double* St, const double* q, double scale, double* o,
+                        int dk, int dv) {
+  for (int j = 0; j < dv; ++j) {
+    const double* col = St + (size_t)j * dk;
+    double acc = 0.0;
+    for (int i = 0; i < dk; ++i) acc += col[i] * q[i];
+    o[j] = scale * acc;
+  }
+}
+
+/* ---- a tiny work queue over independent (sequence or slot, head) pairs ---- */
+
+typedef struct {
+  int n_items;
+  int next;
+  pthread_mutex_t lock;
+  void (*fn)(void* ctx, int item);
+  void* ctx;
+} queue_t;
+
+static void* worker(void* arg) {
+  queue_t* q = (queue_t*)arg;
+  for (;;) {
+    pthread_mutex_lock(&q->lock);
+    int item = q->next++;
+    pthread_mutex_unlock(&q->lock);
+    if (item >= q->n_items) break;
+    q->fn(q->ctx, item);
+  }
+  return NULL;
+}
+
+static int run_items(int n_items, int nthreads, void (*fn)(void*, int), void* ctx) {
+  if (nthreads <= 0) nthreads = (int)sysconf(_SC_NPROCESSORS_ONLN);
+  if (nthreads < 1) nthreads = 1;
+  if (nthreads > n_items) nthreads = n_items > 0 ? n_items : 1;
+  queue_t q;
+  q.n_items = n_items;
+  q.next = 0;
+  q.fn = fn;
+  q.ctx = ctx;
+  pthread_mutex_init(&q.lock, NULL);
+  if (nthreads == 1) {
+    worker(&q);
+  } else {
+    pthread_t* th = (pthread_t*)malloc(sizeof(pthread_t) * (size_t)nthreads);
+    if (!th) return -2;
+    for (int i = 0; i < nthreads; ++i) pthread_create(&th[i], NULL, worker, &q);
+    for (int i = 0; i < nthreads; ++i) pthread_join(th[i], NULL);
+    free(th);
+  }
+  pthread_mutex_destroy(&q.lock);
+  return nthreads;
+}
+
+/* ---- prefill: packed varlen sequences ---- */
+
+typedef struct {
+  const double *q, *k, *v, *g, *beta;
+  const int64_t* cu;
+  int H, dk, dv;
+  double scale;
+  const double* init;
+  double* o;
+  double* fin;
+} prefill_ctx;
+
+static void prefill_item(void* vctx, int item) {
+  prefill_ctx* c = (prefill_ctx*)vctx;
+  const int H = c->H, dk = c->dk, dv = c->dv;
+  const int n = item / H, h = item % H;
+  const size_t ssz = (size_t)dk * dv;
+  double* St = (double*)malloc(ssz * sizeof(double));
+  if (c->init)
+    memcpy(St, c->init + ((size_t)n * H + h) * ssz, ssz * sizeof(double));
+  else
+    memset(St, 0, ssz * sizeof(double));
+  for (int64_t t = c->cu[n]; t < c->cu[n + 1]; ++t) {
+    const size_t th = (size_t)t * H + h;
+    apply_gate(St, exp(c->g[th]), dk, dv);
+    apply_householder(St, c->k + th * dk, c->v + th * dv, c->beta[th], dk, dv);
+    emit_output(St, c->q + th * dk, c->scale, c->o + th * dv, dk, dv);
+  }
+  if (c->fin) memcpy(c->fin + ((size_t)n * H + h) * ssz, St, ssz * sizeof(double));
+  free(St);
+}
+
+/*
+ * q, k: [total_T, H, dk]; v: [total_T, H, dv]; g, beta: [total_T, H];
+ * cu_seqlens: [N + 1] (cu[0] = 0, non-decreasing); init: [N, H, dv, dk] or NULL
+ * (zero state); o: [total_T, H, dv]; final_state: [N, H, dv, dk] or NULL.
+ * Returns the number of threads used, or a negative value on bad arguments.
+ */
+int gdn_oracle_prefill(const double* q, const double* k, const double* v, const double* g,
+                       const double* beta, const int64_t* cu_seqlens, int N, int H, int dk,
+                       int dv, double scale, const double* init, double* o, double* final_state,
+                       int nthreads) {
+  if (N < 0 || H <= 0 || dk <= 0 || dv <= 0 || !cu_seqlens) return -1;
+  if (cu_seqlens[0] != 0) return -1;
+  for (int n = 0; n < N; ++n)
+    if (cu_seqlens[n + 1] < cu_seqlens[n]) return -1;
+  prefill_ctx c = {q, k, v, g, beta, cu_seqlens, H, dk, dv, scale, init, o, final_state};
+  return run_items(N * H, nthreads, prefill_item, &c);
+}
+
+/* ---- decode: slot-indexed state pool, updated in place ---- */
+
+typedef struct {
+  const double *q, *k, *v, *g, *beta;
+  double* pool;
+  int num_slots;
+  const int32_t* slot_ids;
+  double* o;
+  int T, H, dk, dv, nh;
+  double scale;
+} decode_ctx;
+
+static void decode_item(void* vctx, int item) {
+  decode_ctx* c = (decode_ctx*)vctx;
+  const int H = c->H, T = c->T, dk = c->dk, dv = c->dv, nh = c->nh;
+  const int b = item / H, h = item % H;
+  const int slot = c->slot_ids[b];
+  if (slot < 0 || slot >= c->num_slots) {
+    for (int t = 0; t < T; ++t)
+      memset(c->o + (((size_t)b * T + t) * H + h) * dv, 0, (size_t)dv * sizeof(double));
+    return;
+  }
+  double* St = c->pool + ((size_t)slot * H + h) * (size_t)dk * dv;
+  for (int t = 0; t < T; ++t) {
+    const size_t bth = ((size_t)b * T + t) * H + h;
+    apply_gate(St, exp(c->g[bth]), dk, dv);
+    for (int m = 0; m < nh; ++m) {
+      const size_t km = bth * nh + m;
+      apply_householder(St, c->k + km * dk, c->v + km * dv, c->beta[km], dk, dv);
+    }
+    emit_output(St, c->q + bth * dk, c->scale, c->o + bth * dv, dk, dv);
+  }
+}
+
+/*
+ * q: [B, T, H, dk]; k: [B, T, H, nh, dk]; v: [B, T, H, nh, dv]; g: [B, T, H];
+ * beta: [B, T, H, nh]; pool: [num_slots, H, dv, dk], updated in place for the
+ * slots named by slot_ids[B] (a negative or out-of-range id leaves the pool
+ * untouched and writes zeros to that row of o); o: [B, T, H, dv].
+ * Returns the number of threads used, or a negative value on bad arguments.
+ */
+int gdn_oracle_decode(const double* q, const double* k, const double* v, const double* g,
+                      const double* beta, double* pool, int num_slots, const int32_t* slot_ids,
+                      double* o, int B, int T, int H, int dk, int dv, int nh, double scale,
+                      int nthreads) {
+  if (B < 0 || T <= 0 || H <= 0 || dk <= 0 || dv <= 0 || nh <= 0 || num_slots < 0) return -1;
+  decode_ctx c = {q, k, v, g, beta, pool, num_slots, slot_ids, o, T, H, dk, dv, nh, scale};
+  return run_items(B * H, nthreads, decode_item, &c);
+}
