@@ -1,0 +1,497 @@
+"""Benchmark of the gated delta rule library on B200.
+
+    python bench.py [--gpus N] [--steps K] [--warmup W] [--impl ours|reference] [--parts ...]
+
+Headline (one JSON line on rank 0): the T=1 decode step on B=64 sequences x
+H=32 heads, dk=dv=128, fp32 state pool of 256 slots, as state GB/s (state bytes
+read + written per second). A step is one decode launch over one batch; steps
+rotate over 4 disjoint slot sets of the 512 MiB pool so that each step reads
+state that is not in the 126 MB L2. The other workloads (chunked prefill
+B=4 x 8192 x H=16; varlen prefill 32 seqs x H=32; long sequence B=1 x 65536 x
+H=4; gated delta product B=128 x T=4 x n_h=2; tiny fp32) are measured in the
+same run and reported under "parts".
+
+With torchrun (N > 1) every rank runs the same per-GPU workload on its own
+device (weak scaling, no collective on the data path); times are the max over
+ranks. `--impl reference` times the fp64 CPU oracle on the same workload.
+"""
+from __future__ import annotations
+
+import argparse
+import hashlib
+import json
+import math
+import os
+import statistics
+import subprocess
+import sys
+import threading
+import time
+
+import torch
+
+ROOT = os.path.dirname(os.path.abspath(__file__))
+if ROOT not in sys.path:
+    sys.path.insert(0, ROOT)
+
+METRIC = "GDN decode state GB/s (% of 8 TB/s); chunked prefill tokens/s (% roofline)"
+NOMINAL_HBM_GBS = 8000.0
+FALLBACK_PEAKS = {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "bf16_tflops_sustained": 1400.0}
+
+
+# ---------------------------------------------------------------- environment
+
+def load_peaks():
+    path = os.path.join(ROOT, "MEASURED_PEAKS.json")
+    if os.path.exists(path):
+        with open(path) as f:
+            d = json.load(f)
+        return d, "measured"
+    return dict(FALLBACK_PEAKS), "fallback"
+
+
+def dist_setup():
+    ws = int(os.environ.get("WORLD_SIZE", "1"))
+    rank = int(os.environ.get("RANK", "0"))
+    local = int(os.environ.get("LOCAL_RANK", "0"))
+    if ws > 1:
+        import datetime
+        import torch.distributed as dist
+        os.environ.setdefault("MASTER_ADDR", "127.0.0.1")
+        torch.cuda.set_device(local)
+        dist.init_process_group("nccl", timeout=datetime.timedelta(seconds=120),
+                                device_id=torch.device("cuda", local))
+    else:
+        torch.cuda.set_device(0)
+    return ws, rank, local
+
+
+def barrier(ws):
+    if ws > 1:
+        import torch.distributed as dist
+        dist.barrier()
+
+
+def max_over_ranks(x: float, ws: int) -> float:
+    if ws == 1:
+        return x
+    import torch.distributed as dist
+    t = torch.tensor([x], dtype=torch.float64, device="cuda")
+    dist.all_reduce(t, op=dist.ReduceOp.MAX)
+    return float(t.item())
+
+
+class ClockSampler:
+    """Samples nvidia-smi SM clocks and throttle reasons while the timed region runs."""
+    FIELDS = ("index,clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.active,"
+              "clocks_event_reasons.hw_slowdown,clocks_event_reasons.hw_thermal_slowdown,"
+              "clocks_event_reasons.sw_thermal_slowdown,clocks_event_reasons.sw_power_cap")
+
+    def __init__(self, gpu_index: int):
+        self.gpu = gpu_index
+        self.rows = []
+        self._stop = threading.Event()
+        self._th = None
+
+    def _run(self):
+        while not self._stop.is_set():
+            try:
+                out = subprocess.run(["nvidia-smi", "-i", str(self.gpu), f"--query-gpu={self.FIELDS}",
+                                      "--format=csv,noheader,nounits"], capture_output=True, text=True,
+                                     timeout=5).stdout.strip()
+                if out:
+                    self.rows.append([x.strip() for x in out.split(",")])
+            except Exception:
+                pass
+            self._stop.wait(0.2)
+
+    def __enter__(self):
+        self._th = threading.Thread(target=self._run, daemon=True)
+        self._th.start()
+        return self
+
+    def __exit__(self, *exc):
+        self._stop.set()
+        self._th.join(timeout=10)
+
+    def summary(self):
+        if not self.rows:
+            return {"sm_mhz": None, "sm_max_mhz": None, "reasons": [], "samples": 0}
+        sm = [float(r[1]) for r in self.rows if r[1].replace(".", "").isdigit()]
+        mx = [float(r[2]) for r in self.rows if r[2].replace(".", "").isdigit()]
+        names = ["hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap"]
+        reasons = sorted({names[i] for r in self.rows for i in range(4)
+                          if len(r) > 5 + i and r[5 + i].lower() == "active"})
+        return {"sm_mhz": statistics.median(sm) if sm else None, "sm_max_mhz": max(mx) if mx else None,
+                "reasons": reasons, "samples": len(self.rows)}
+
+
+def source_sha(*rel_paths) -> str:
+    h = hashlib.sha256()
+    for p in rel_paths:
+        with open(os.path.join(ROOT, p), "rb") as f:
+            h.update(f.read())
+    return h.hexdigest()[:16]
+
+
+def ncu_traffic(kernel_key: str, sources):
+    """DRAM bytes per launch from the committed ncu summary, if the kernel source is unchanged."""
+    path = os.path.join(ROOT, "profiles", "ncu_traffic.json")
+    if not os.path.exists(path):
+        return None
+    with open(path) as f:
+        d = json.load(f)
+    e = d.get(kernel_key)
+    if not e or e.get("source_sha") != source_sha(*sources):
+        return None
+    return e.get("dram_bytes_per_launch")
+
+
+# ---------------------------------------------------------------- timing helpers
+
+def time_launches(fn, steps, warmup, ws, stream=None):
+    """Runs fn(i) warmup times, then `steps` times bracketed by barrier + synchronize;
+    returns (max-over-ranks total ms, list of per-launch ms from CUDA events)."""
+    stream = stream or torch.cuda.current_stream()
+    for i in range(warmup):
+        fn(i)
+    torch.cuda.synchronize()
+    evs = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)) for _ in range(steps)]
+    start, stop = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    barrier(ws)
+    torch.cuda.synchronize()
+    start.record(stream)
+    for i in range(steps):
+        evs[i][0].record(stream)
+        fn(warmup + i)
+        evs[i][1].record(stream)
+    stop.record(stream)
+    torch.cuda.synchronize()
+    barrier(ws)
+    total = max_over_ranks(start.elapsed_time(stop), ws)
+    per = [a.elapsed_time(b) for a, b in evs]
+    return total, per
+
+
+# ---------------------------------------------------------------- decode workloads
+
+DECODE_CFGS = {
+    "decode": dict(B=64, T=1, H=32, d=128, nh=1, slots=256,
+                   name="decode T=1, B=64, H=32, dk=dv=128, fp32 pool of 256 slots, bf16 q/k/v"),
+    "gdp": dict(B=128, T=4, H=32, d=128, nh=2, slots=512,
+                name="gated delta product decode, B=128, H=32, T=4, n_h=2, dk=dv=128, pool of 512 slots"),
+}
+
+
+def decode_bytes(c):
+    """Algorithmic HBM bytes of one decode step: state read + write, q/k/v (bf16),
+    g and beta (fp32), o (bf16), slot ids."""
+    B, T, H, d, nh = c["B"], c["T"], c["H"], c["d"], c["nh"]
+    heads = B * H
+    state = 2 * heads * d * d * 4
+    qkv = heads * T * (d + nh * d + nh * d) * 2
+    gb = heads * T * (1 + nh) * 4
+    o = heads * T * d * 2
+    return state, state + qkv + gb + o + B * 4
+
+
+def bench_decode(key, steps, warmup, ws, rank, peaks, e2e=True):
+    import gated_delta_rule_58_b200 as gdn
+    from gated_delta_rule_58_b200 import inputs
+    c = DECODE_CFGS[key]
+    dev = torch.device("cuda", torch.cuda.current_device())
+    inp = inputs.decode_inputs(c["B"], c["T"], c["H"], c["d"], c["d"], c["nh"], c["slots"],
+                               seed=rank, device=dev)
+    nsets = c["slots"] // c["B"]
+    perm = torch.randperm(c["slots"], generator=torch.Generator().manual_seed(rank)).to(torch.int32)
+    slot_sets = [perm[i * c["B"]:(i + 1) * c["B"]].to(dev) for i in range(nsets)]
+    o = torch.empty((c["B"], c["T"], c["H"], c["d"]), dtype=torch.bfloat16, device=dev)
+    pool = inp.pool
+
+    def step(i):
+        gdn.gdn_decode(inp.q, inp.k, inp.v, inp.g, inp.beta, pool, slot_sets[i % nsets], o, scale=inp.scale)
+
+    total_ms, per = time_launches(step, steps, warmup, ws)
+    state_b, alg_b = decode_bytes(c)
+    ms = total_ms / steps
+    res = {
+        "workload": c["name"],
+        "ms_per_step": ms,
+        "state_gbs": state_b / (ms * 1e-3) / 1e9 * ws,
+        "launch_ms_mean": statistics.fmean(per),
+        "launches_per_step": 1,
+        "alg_bytes_per_launch": alg_b,
+        "state_bytes_per_launch": state_b,
+    }
+    if e2e:
+        # end to end through the public API with host buffers: pinned H2D of the step's
+        # inputs, the call, and D2H of o, all inside the timed region
+        host = {n: getattr(inp, n).cpu().pin_memory() for n in ("q", "k", "v", "g", "beta")}
+        host_slots = [s.cpu().pin_memory() for s in slot_sets]
+        dev_bufs = {n: torch.empty_like(getattr(inp, n)) for n in host}
+        dslots = torch.empty_like(slot_sets[0])
+        o_host = torch.empty(o.shape, dtype=o.dtype).pin_memory()
+        h2d = sum(t.numel() * t.element_size() for t in host.values()) + host_slots[0].numel() * 4
+        d2h = o.numel() * o.element_size()
+
+        def e2e_step(i):
+            for n, t in host.items():
+                dev_bufs[n].copy_(t, non_blocking=True)
+            dslots.copy_(host_slots[i % nsets], non_blocking=True)
+            gdn.gdn_decode(dev_bufs["q"], dev_bufs["k"], dev_bufs["v"], dev_bufs["g"], dev_bufs["beta"],
+                           pool, dslots, o, scale=inp.scale)
+            o_host.copy_(o, non_blocking=True)
+
+        e2e_total, _ = time_launches(e2e_step, steps, warmup, ws)
+        e_ms = e2e_total / steps
+        res["e2e"] = {"value": state_b / (e_ms * 1e-3) / 1e9 * ws, "unit": "GB/s",
+                      "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h, "ms_per_step": e_ms}
+    achieved = alg_b / (res["launch_ms_mean"] * 1e-3) / 1e9
+    peak = peaks["hbm_gbs"]
+    res["roofline"] = {"bound": "hbm", "achieved": achieved, "peak": peak, "unit": "GB/s",
+                       "frac": achieved / peak,
+                       "traffic": ncu_traffic(f"gdn_decode_kernel:{key}",
+                                              ["gated_delta_rule_58_b200/csrc/decode.cu"])}
+    res["pct_of_8tbs_state"] = res["state_gbs"] / ws / NOMINAL_HBM_GBS * 100
+    return res
+
+
+# ---------------------------------------------------------------- prefill workloads
+
+def prefill_cfg(key, device, seed):
+    from gated_delta_rule_58_b200 import inputs
+    if key == "prefill":
+        return inputs.prefill_b4_t8192_h16(device=device, seed=seed), 64, \
+            "chunked prefill, B=4 x T=8192, H=16, dk=dv=128, chunk 64, bf16 q/k/v, fp32 initial state"
+    if key == "varlen":
+        return inputs.varlen32_h32(device=device, seed=seed), 64, \
+            "varlen prefill, 32 seqs L~U[64,16384], H=32, dk=dv=128, chunk 64"
+    if key == "longseq":
+        return inputs.longseq_b1_t65536_h4(device=device, seed=seed), 64, \
+            "low-parallelism prefill, B=1 x T=65536, H=4, dk=dv=128, chunk 64"
+    if key == "tiny":
+        return inputs.tiny_prefill(device=device, seed=seed), 16, \
+            "tiny prefill, B=1, H=2, T=64, dk=dv=32, fp32, chunk 16"
+    raise KeyError(key)
+
+
+def prefill_alg_bytes(inp):
+    total, H, dk = inp.q.shape
+    dv = inp.v.shape[-1]
+    N = inp.cu_seqlens.numel() - 1
+    es = inp.q.element_size()
+    per_tok = H * ((2 * dk + dv) * es + 8 + dv * 2)
+    states = N * H * dk * dv * 4 * (2 if inp.initial_state is not None else 1)
+    return total * per_tok + states
+
+
+def prefill_flops(inp, chunk):
+    """Algorithmic flops of the chunked form per (sequence, head) chunk, summed."""
+    total, H, d = inp.q.shape
+    lens = inp.seqlens
+    f = 0
+    for L in lens:
+        full, rem = divmod(L, chunk)
+        for C in [chunk] * full + ([rem] if rem else []):
+            f += 5 * 2 * C * C * d + 3 * 2 * C * d * d + 2 * C ** 3 // 3
+    return f * H
+
+
+def bench_prefill(key, steps, warmup, ws, rank, peaks, algo=None):
+    import gated_delta_rule_58_b200 as gdn
+    dev = torch.device("cuda", torch.cuda.current_device())
+    inp, chunk, name = prefill_cfg(key, dev, rank)
+    algo = gdn.GDN_PREFILL_AUTO if algo is None else algo
+    total, H, dk = inp.q.shape
+    dv = inp.v.shape[-1]
+    N = inp.cu_seqlens.numel() - 1
+    o = torch.empty((total, H, dv), dtype=torch.bfloat16, device=dev)
+    fin = torch.empty((N, H, dv, dk), dtype=torch.float32, device=dev)
+    ws_bytes = gdn.gdn_chunk_prefill_workspace_size(N, total, H, dk, dv, chunk, algo)
+    work = torch.empty(max(ws_bytes, 1), dtype=torch.uint8, device=dev)
+
+    def step(i):
+        gdn.gdn_chunk_prefill(inp.q, inp.k, inp.v, inp.g, inp.beta, inp.cu_seqlens, o,
+                              initial_state=inp.initial_state, final_state=fin, chunk=chunk,
+                              scale=inp.scale, algo=algo, workspace=work)
+
+    total_ms, per = time_launches(step, steps, warmup, ws)
+    ms = total_ms / steps
+    alg_b = prefill_alg_bytes(inp)
+    flops = prefill_flops(inp, chunk)
+    t = ms * 1e-3
+    hbm_t = alg_b / (peaks["hbm_gbs"] * 1e9)
+    tc_t = flops / (peaks["bf16_tflops"] * 1e12)
+    bound = "hbm" if hbm_t >= tc_t else "tensor"
+    res = {
+        "workload": name,
+        "algo": {0: "auto", 1: "fused", 2: "transfer", 3: "sequential"}[algo],
+        "ms_per_step": ms,
+        "tokens_per_s": total / t * ws,
+        "roofline": {"bound": bound,
+                     "achieved": alg_b / t / 1e9 if bound == "hbm" else flops / t / 1e12,
+                     "peak": peaks["hbm_gbs"] if bound == "hbm" else peaks["bf16_tflops"],
+                     "unit": "GB/s" if bound == "hbm" else "TFLOP/s",
+                     "frac": max(hbm_t, tc_t) / t,
+                     "traffic": None},
+        "pct_of_nominal_roofline": max(alg_b / (NOMINAL_HBM_GBS * 1e9), flops / 2.25e15) / t * 100,
+        "alg_bytes": alg_b,
+        "flops": flops,
+        "workspace_bytes": ws_bytes,
+    }
+    del inp, o, fin, work
+    torch.cuda.empty_cache()
+    return res
+
+
+# ---------------------------------------------------------------- CPU oracle (baseline / reference arm)
+
+def oracle_decode_rate(key, budget_s=10.0, seed=0):
+    """Times the fp64 oracle on the decode workload (full batch) for ~budget_s;
+    returns state GB/s-equivalent, threads used and the sample description."""
+    import oracle
+    from gated_delta_rule_58_b200 import inputs
+    c = DECODE_CFGS[key]
+    inp = inputs.decode_inputs(c["B"], c["T"], c["H"], c["d"], c["d"], c["nh"], c["slots"], seed=seed)
+    args = [oracle.f64(x) for x in (inp.q, inp.k, inp.v, inp.g, inp.beta)]
+    pool = oracle.f64(inp.pool)
+    state_b, _ = decode_bytes(c)
+    n = 0
+    t0 = time.perf_counter()
+    threads = 0
+    while True:
+        _, pool, threads = oracle.decode(*args, pool, inp.slot_ids, scale=inp.scale)
+        n += 1
+        if time.perf_counter() - t0 >= budget_s:
+            break
+    dt = time.perf_counter() - t0
+    return state_b * n / dt / 1e9, threads, f"{n} full decode steps ({c['name']}) in {dt:.1f} s"
+
+
+def run_reference(args, ws, rank):
+    """The reference arm: the fp64 CPU oracle on the headline workload."""
+    if rank != 0:
+        return
+    steps, warmup = args.steps, args.warmup
+    budget = max(1.0, min(20.0, 120.0 / max(steps + warmup, 1)))
+    for _ in range(warmup):
+        oracle_decode_rate("decode", budget_s=0.1)
+    rates = []
+    threads = 0
+    sample = ""
+    t0 = time.perf_counter()
+    for _ in range(steps):
+        r, threads, sample = oracle_decode_rate("decode", budget_s=budget)
+        rates.append(r)
+    elapsed = time.perf_counter() - t0
+    value = statistics.fmean(rates)
+    c = DECODE_CFGS["decode"]
+    state_b, _ = decode_bytes(c)
+    line = {
+        "impl": "reference", "metric": METRIC, "value": value, "unit": "GB/s", "n_gpus": 1,
+        "steps": steps, "warmup": warmup, "ms_per_step": state_b / (value * 1e9) * 1e3,
+        "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "f64",
+        "data": "synthetic", "config": {"workload": c["name"], "l2": "n/a (CPU)"},
+        "cpu_baseline": {"value": value, "unit": "GB/s", "cores": threads, "kind": "oracle",
+                         "sample": f"per step: {sample}; total {elapsed:.1f} s"},
+        "e2e": {"value": value, "unit": "GB/s", "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0},
+    }
+    print(json.dumps(line), flush=True)
+
+
+# ---------------------------------------------------------------- main
+
+def main():
+    ap = argparse.ArgumentParser()
+    ap.add_argument("--gpus", type=int, default=1)
+    ap.add_argument("--steps", type=int, default=2000)
+    ap.add_argument("--warmup", type=int, default=20)
+    ap.add_argument("--impl", default="ours", choices=["ours", "reference"])
+    ap.add_argument("--parts", default="gdp,prefill,varlen,longseq,tiny",
+                    help="comma list of extra workloads to measure (empty for none)")
+    ap.add_argument("--part-steps", type=int, default=5)
+    ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--prefill-algo", default=None, help="force fused|transfer|sequential for the parts")
+    args = ap.parse_args()
+    if args.warmup < 3:
+        args.warmup = 3
+
+    ws, rank, local = dist_setup()
+    if args.impl == "reference":
+        run_reference(args, ws, rank)
+        if ws > 1:
+            import torch.distributed as dist
+            dist.destroy_process_group()
+        return
+
+    import gated_delta_rule_58_b200 as gdn
+    gdn.lib()  # fails loudly if the CUDA library is missing
+    peaks, peak_src = load_peaks()
+    vis = os.environ.get("CUDA_VISIBLE_DEVICES", "")
+    vis_list = [x for x in vis.split(",") if x]
+    gpu_index = vis_list[local] if local < len(vis_list) else str(local)
+
+    with ClockSampler(gpu_index) as clk:
+        head = bench_decode("decode", args.steps, args.warmup, ws, rank, peaks)
+        parts = []
+        algo = None
+        if args.prefill_algo:
+            algo = {"fused": gdn.GDN_PREFILL_FUSED, "transfer": gdn.GDN_PREFILL_TRANSFER,
+                    "sequential": gdn.GDN_PREFILL_SEQUENTIAL}[args.prefill_algo]
+        for key in [p for p in args.parts.split(",") if p]:
+            try:
+                if key == "gdp":
+                    r = bench_decode("gdp", max(args.part_steps * 20, 20), args.warmup, ws, rank, peaks,
+                                     e2e=False)
+                    r["metric"] = "GDP decode state GB/s"
+                else:
+                    r = bench_prefill(key, args.part_steps, 3, ws, rank, peaks, algo=algo)
+                    r["metric"] = "prefill tokens/s"
+                r["key"] = key
+            except Exception as e:  # a part that is not supported is reported, not fatal
+                r = {"key": key, "error": f"{type(e).__name__}: {e}"}
+            parts.append(r)
+
+    if ws > 1:
+        import torch.distributed as dist
+        dist.barrier()
+
+    if rank == 0:
+        cpu = None
+        if not args.no_cpu_baseline and ws == 1:
+            v, threads, sample = oracle_decode_rate("decode", budget_s=10.0)
+            cpu = {"value": v, "unit": "GB/s", "cores": threads, "kind": "oracle", "sample": sample}
+        clocks = clk.summary()
+        line = {
+            "metric": METRIC,
+            "value": head["state_gbs"],
+            "unit": "GB/s",
+            "n_gpus": ws,
+            "steps": args.steps,
+            "warmup": args.warmup,
+            "ms_per_step": head["ms_per_step"],
+            "higher_is_better": True,
+            "scaling": "weak",
+            "vs_baseline": None,
+            "dtype": "f32",
+            "data": "synthetic",
+            "config": {"workload": head["workload"],
+                       "l2": "inputs larger than L2: steps rotate over 4 disjoint 64-slot sets of a 512 MiB pool",
+                       "parallelism": f"dp{ws} (independent sequences per GPU)",
+                       "pct_of_8tbs_state": head["pct_of_8tbs_state"],
+                       "peaks": peak_src},
+            "roofline": head["roofline"],
+            "cpu_baseline": cpu,
+            "e2e": head.get("e2e"),
+            "gpu_launches": args.steps,
+            "clocks": clocks,
+            "parts": parts,
+        }
+        print(json.dumps(line), flush=True)
+    if ws > 1:
+        import torch.distributed as dist
+        dist.destroy_process_group()
+
+
+if __name__ == "__main__":
+    main()

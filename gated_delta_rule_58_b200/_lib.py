@@ -1,0 +1,177 @@
+"""ctypes binding of libgdn.so (include/gdn.h). Argument marshalling only.
+
+Every compute step runs in the CUDA library; this module turns torch tensors
+into device pointers and sizes, passes the current CUDA stream, and raises
+GdnError on a non-OK status. There is no CPU fallback: if libgdn.so is missing
+the first call raises.
+"""
+from __future__ import annotations
+
+import ctypes
+import os
+import re
+import threading
+
+PKG = os.path.dirname(os.path.abspath(__file__))
+LIB_PATH = os.path.join(PKG, "libgdn.so")
+HEADER = os.path.join(os.path.dirname(PKG), "include", "gdn.h")
+
+GDN_OK = 0
+GDN_ERR_INVALID_ARG = 1
+GDN_ERR_UNSUPPORTED = 2
+GDN_ERR_WORKSPACE = 3
+GDN_ERR_CUDA = 4
+GDN_ERR_DEVICE_DATA = 5
+
+GDN_BF16 = 0
+GDN_F32 = 1
+
+GDN_PREFILL_AUTO = 0
+GDN_PREFILL_FUSED = 1
+GDN_PREFILL_TRANSFER = 2
+GDN_PREFILL_SEQUENTIAL = 3
+
+GDN_DEVERR_SLOT_OUT_OF_RANGE = 0x1
+GDN_DEVERR_BAD_CU_SEQLENS = 0x2
+GDN_DEVERR_TIMEOUT = 0x4
+
+_lib = None
+_lock = threading.Lock()
+
+
+class GdnError(RuntimeError):
+    def __init__(self, status: int, message: str):
+        super().__init__(f"gdn status {status}: {message}")
+        self.status = status
+
+
+def declared_functions(header: str = HEADER):
+    """Names of the functions include/gdn.h declares."""
+    text = open(header).read()
+    text = re.sub(r"/\*.*?\*/", "", text, flags=re.S)
+    return sorted(set(re.findall(r"\b(gdn_\w+)\s*\(", text)))
+
+
+def lib() -> ctypes.CDLL:
+    """Load libgdn.so (raises if it has not been built)."""
+    global _lib
+    with _lock:
+        if _lib is None:
+            if not os.path.exists(LIB_PATH):
+                raise RuntimeError(
+                    f"{LIB_PATH} is missing: build it with `python -m gated_delta_rule_58_b200.build` "
+                    "(the library has no CPU fallback)")
+            L = ctypes.CDLL(LIB_PATH)
+            vp, i32, i64, f32, sz = (ctypes.c_void_p, ctypes.c_int, ctypes.c_int64, ctypes.c_float,
+                                     ctypes.c_size_t)
+            L.gdn_decode.restype = i32
+            L.gdn_decode.argtypes = [vp, vp, vp, vp, vp, vp, i32, vp, vp, i32, i32, i32, i32, i32, i32,
+                                     f32, i32, i32, vp]
+            L.gdn_chunk_prefill_workspace_size.restype = sz
+            L.gdn_chunk_prefill_workspace_size.argtypes = [i32, i64, i32, i32, i32, i32, i32]
+            L.gdn_chunk_prefill.restype = i32
+            L.gdn_chunk_prefill.argtypes = [vp, vp, vp, vp, vp, vp, i32, i64, vp, vp, vp, i32, i32, i32,
+                                            i32, f32, i32, i32, i32, vp, sz, vp]
+            L.gdn_last_error.restype = ctypes.c_char_p
+            L.gdn_last_error.argtypes = []
+            L.gdn_get_device_error.restype = i32
+            L.gdn_get_device_error.argtypes = [ctypes.POINTER(ctypes.c_uint32)]
+            L.gdn_version.restype = ctypes.c_char_p
+            L.gdn_version.argtypes = []
+            _lib = L
+    return _lib
+
+
+def gdn_last_error() -> str:
+    return lib().gdn_last_error().decode()
+
+
+def gdn_version() -> str:
+    return lib().gdn_version().decode()
+
+
+def _check(status: int):
+    if status != GDN_OK:
+        raise GdnError(status, gdn_last_error())
+
+
+def gdn_get_device_error() -> int:
+    """Read and clear the sticky device error word (synchronises the device)."""
+    flags = ctypes.c_uint32(0)
+    st = lib().gdn_get_device_error(ctypes.byref(flags))
+    if st not in (GDN_OK, GDN_ERR_DEVICE_DATA):
+        _check(st)
+    return int(flags.value)
+
+
+# ---------------------------------------------------------------- torch marshalling
+
+def _dtype_code(t) -> int:
+    import torch
+    if t.dtype == torch.bfloat16:
+        return GDN_BF16
+    if t.dtype == torch.float32:
+        return GDN_F32
+    raise TypeError(f"unsupported dtype {t.dtype} (bf16 or fp32)")
+
+
+def _ptr(t):
+    if t is None:
+        return None
+    if not t.is_contiguous():
+        raise ValueError("tensors must be contiguous")
+    return t.data_ptr()
+
+
+def _stream_ptr(stream, device):
+    import torch
+    if stream is None:
+        stream = torch.cuda.current_stream(device)
+    return stream.cuda_stream if hasattr(stream, "cuda_stream") else int(stream)
+
+
+def gdn_decode(q, k, v, g, beta, state_pool, slot_ids, o, scale=None, stream=None):
+    """One decode step (see include/gdn.h). Shapes:
+    q [B,T,H,dk], k [B,T,H,n_h,dk], v [B,T,H,n_h,dv], g [B,T,H], beta [B,T,H,n_h],
+    state_pool [num_slots,H,dv,dk] fp32 (updated in place), slot_ids [B] int32, o [B,T,H,dv]."""
+    B, T, H, dk = q.shape
+    n_h, dv = k.shape[3], v.shape[4]
+    if scale is None:
+        scale = dk ** -0.5
+    st = lib().gdn_decode(_ptr(q), _ptr(k), _ptr(v), _ptr(g), _ptr(beta), _ptr(state_pool),
+                          state_pool.shape[0], _ptr(slot_ids), _ptr(o), B, T, H, dk, dv, n_h,
+                          float(scale), _dtype_code(q), _dtype_code(o), _stream_ptr(stream, q.device))
+    _check(st)
+    return o
+
+
+def gdn_chunk_prefill_workspace_size(N, total_T, H, dk, dv, chunk, algo=GDN_PREFILL_AUTO) -> int:
+    n = lib().gdn_chunk_prefill_workspace_size(N, total_T, H, dk, dv, chunk, algo)
+    if n == ctypes.c_size_t(-1).value:
+        raise GdnError(GDN_ERR_INVALID_ARG, gdn_last_error())
+    return int(n)
+
+
+def gdn_chunk_prefill(q, k, v, g, beta, cu_seqlens, o, initial_state=None, final_state=None,
+                      chunk=64, scale=None, algo=GDN_PREFILL_AUTO, workspace=None, stream=None):
+    """Chunked varlen prefill (see include/gdn.h). Shapes: q,k [total_T,H,dk], v [total_T,H,dv],
+    g,beta [total_T,H] fp32, cu_seqlens [N+1] int32 (device), initial/final_state [N,H,dv,dk] fp32,
+    o [total_T,H,dv]. `workspace` is a uint8 CUDA tensor; when None one of the required size is
+    allocated through torch for this call."""
+    import torch
+    total_T, H, dk = q.shape
+    dv = v.shape[-1]
+    N = cu_seqlens.numel() - 1
+    if scale is None:
+        scale = dk ** -0.5
+    need = gdn_chunk_prefill_workspace_size(N, total_T, H, dk, dv, chunk, algo)
+    if workspace is None and need > 0:
+        workspace = torch.empty(need, dtype=torch.uint8, device=q.device)
+    ws_ptr = _ptr(workspace)
+    ws_bytes = workspace.numel() if workspace is not None else 0
+    st = lib().gdn_chunk_prefill(_ptr(q), _ptr(k), _ptr(v), _ptr(g), _ptr(beta), _ptr(cu_seqlens), N,
+                                 total_T, _ptr(initial_state), _ptr(final_state), _ptr(o), H, dk, dv,
+                                 chunk, float(scale), _dtype_code(q), _dtype_code(o), algo, ws_ptr,
+                                 ws_bytes, _stream_ptr(stream, q.device))
+    _check(st)
+    return o

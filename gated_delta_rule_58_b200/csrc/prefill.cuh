@@ -1,0 +1,58 @@
+// Internal prefill interfaces shared by the prefill translation units.
+#pragma once
+
+#include "common.cuh"
+
+namespace gdn {
+
+struct PrefillShape {
+  int N;            // sequences
+  int64_t total_T;  // packed tokens
+  int H, dk, dv, chunk;
+};
+
+struct PrefillArgs {
+  const void* q;
+  const void* k;
+  const void* v;
+  const float* g;
+  const float* beta;
+  const int32_t* cu_seqlens;
+  const float* initial_state;
+  float* final_state;
+  void* o;
+  float scale;
+  gdn_dtype_t in_dtype, out_dtype;
+  void* workspace;
+  unsigned int* err;
+};
+
+// Validates the shape for `requested` and resolves GDN_PREFILL_AUTO.
+gdn_status_t prefill_resolve(const PrefillShape& s, gdn_dtype_t in, gdn_prefill_algo_t requested,
+                             gdn_prefill_algo_t* resolved);
+// AUTO choice between the two tensor-core algorithms (dk == dv == 128, chunk == 64).
+gdn_prefill_algo_t prefill_auto_tensor_core(const PrefillShape& s);
+size_t prefill_workspace_bytes(const PrefillShape& s, gdn_prefill_algo_t resolved);
+gdn_status_t prefill_launch(const PrefillShape& s, const PrefillArgs& a, gdn_prefill_algo_t resolved,
+                            cudaStream_t stream);
+
+gdn_status_t prefill_sequential_launch(const PrefillShape& s, const PrefillArgs& a, cudaStream_t stream);
+gdn_status_t prefill_fused_launch(const PrefillShape& s, const PrefillArgs& a, cudaStream_t stream);
+size_t prefill_transfer_workspace_bytes(const PrefillShape& s);
+gdn_status_t prefill_transfer_launch(const PrefillShape& s, const PrefillArgs& a, cudaStream_t stream);
+
+// Reads cu_seqlens[n], cu_seqlens[n+1] and validates them against total_T; on a bad
+// pair sets GDN_DEVERR_BAD_CU_SEQLENS and returns false (the caller skips the unit).
+__device__ __forceinline__ bool seq_bounds(const int32_t* cu, int n, int64_t total_T,
+                                           unsigned int* err, int64_t* bos, int64_t* eos) {
+  const int32_t a = __ldg(cu + n), b = __ldg(cu + n + 1);
+  if (a < 0 || b < a || (int64_t)b > total_T || (n == 0 && a != 0)) {
+    raise_device_error(err, GDN_DEVERR_BAD_CU_SEQLENS);
+    return false;
+  }
+  *bos = a;
+  *eos = b;
+  return true;
+}
+
+}  // namespace gdn

@@ -1,0 +1,172 @@
+/*
+ * gdn.h — C ABI of the B200 (sm_100a) gated delta rule library, libgdn.so.
+ *
+ * The method. Per head, an fp32 recurrent state S (dk x dv) evolves token by
+ * token as the gated delta rule (Yang, Kautz, Hatamizadeh, "Gated Delta
+ * Networks: Improving Mamba2 with Delta Rule", ICLR 2025):
+ *
+ *     S_t = alpha_t (I - beta_t k_t k_t^T) S_{t-1} + beta_t k_t v_t^T
+ *     o_t = scale * S_t^T q_t,                alpha_t = exp(g_t)
+ *
+ * The gated delta product (kernel family cake_gated_delta_product_mtp on the
+ * FlashInfer PR #7156 page, "Cake GDP kernel: shared-memory reduction and
+ * direct register loads", introduction and section 1) applies, per token, the
+ * gate once and then n_h Householder updates (I - beta_j k_j k_j^T) S +
+ * beta_j k_j v_j^T in order j = 1..n_h, then emits one output.
+ *
+ * Conventions shared by every entry point:
+ *  - All tensor pointers are DEVICE pointers (cudaMalloc'd or equivalent) unless
+ *    stated otherwise, densely packed, innermost dimension contiguous, 16-byte
+ *    aligned. No stride arguments: the layouts are the ones documented here.
+ *  - States are stored K-last: S^T row-major, [.., dv, dk] (fp32), the layout the
+ *    FlashInfer PR #7156 page (section 1) loads as float4 rows over k, and the
+ *    FlashInfer PR #3866 page ("CP delta-rule precompute at ultra-low
+ *    parallelism", section 2) contracts over the second index.
+ *  - The caller owns every buffer. The library never allocates, frees or
+ *    synchronises; it only enqueues kernels on `stream` (a cudaStream_t passed as
+ *    void*, NULL = legacy default stream). Calls are therefore capturable into CUDA
+ *    graphs once the workspace size is known (the "prepare before capture" pattern
+ *    of the FlashInfer PR #6291 page, section 3).
+ *  - Every host-checkable error (null or misaligned pointer, bad size, unsupported
+ *    combination, small workspace) returns a non-OK status BEFORE anything is
+ *    launched; gdn_last_error() then gives a message (thread-local). Errors that
+ *    only the data can show (slot id out of range, non-monotone cu_seqlens) are
+ *    detected on the device: the offending unit is skipped (never an out-of-bounds
+ *    access) and a sticky device error word is set, read by gdn_get_device_error().
+ *  - Input dtype: q, k, v are GDN_BF16 or GDN_F32 (same dtype for all three); g
+ *    and beta are always fp32; o is GDN_BF16 (round-to-nearest-even) or GDN_F32.
+ */
+#ifndef GDN_H_
+#define GDN_H_
+
+#include <stddef.h>
+#include <stdint.h>
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+typedef enum {
+  GDN_OK = 0,
+  GDN_ERR_INVALID_ARG = 1,   /* null/misaligned pointer, negative or inconsistent sizes */
+  GDN_ERR_UNSUPPORTED = 2,   /* valid but not implemented (dims, dtype, chunk, algorithm) */
+  GDN_ERR_WORKSPACE = 3,     /* workspace pointer null or smaller than required */
+  GDN_ERR_CUDA = 4,          /* a CUDA runtime call failed (message has the CUDA error) */
+  GDN_ERR_DEVICE_DATA = 5    /* returned by gdn_get_device_error when the device flagged data */
+} gdn_status_t;
+
+typedef enum { GDN_BF16 = 0, GDN_F32 = 1 } gdn_dtype_t;
+
+/* Bits of the sticky device error word (gdn_get_device_error). */
+#define GDN_DEVERR_SLOT_OUT_OF_RANGE 0x1u  /* a slot id >= num_slots was skipped */
+#define GDN_DEVERR_BAD_CU_SEQLENS 0x2u     /* cu_seqlens not 0-based / non-decreasing / > total_T */
+#define GDN_DEVERR_TIMEOUT 0x4u            /* a bounded inter-CTA wait gave up */
+
+/*
+ * gdn_decode — one decode step over a slot-indexed state pool, updated in place.
+ *
+ * Computes, for every batch row b with slot s = slot_ids[b] and every head h,
+ * T tokens in order, each: S <- alpha_t S, then n_h Householder updates, then
+ * o[b,t,h,:] = scale * S^T q[b,t,h,:]; the final S is written back to the pool
+ * slot. n_h = 1, T = 1 is the gated delta rule decode step (the T=1 split-V
+ * variant of the FlashInfer PR #7156 page); n_h > 1 and/or T > 1 is the gated
+ * delta product multi-token step of the same page.
+ *
+ *   q          [B, T, H, dk]        in_dtype
+ *   k          [B, T, H, n_h, dk]   in_dtype
+ *   v          [B, T, H, n_h, dv]   in_dtype
+ *   g          [B, T, H]            fp32, log-space gate (alpha = exp(g); -inf allowed)
+ *   beta       [B, T, H, n_h]       fp32
+ *   state_pool [num_slots, H, dv, dk] fp32, K-last; read and written in place
+ *   slot_ids   [B] int32. Negative id: row skipped (pool untouched, o rows set to 0).
+ *              Id >= num_slots: same, and GDN_DEVERR_SLOT_OUT_OF_RANGE is set.
+ *              Ids must be distinct (duplicates race: undefined result).
+ *   o          [B, T, H, dv]        out_dtype
+ *
+ * Supported: dk == dv in {32, 64, 128}; T in {1, 2, 4, 8}, n_h in {1, 2, 4}, T * n_h <= 8.
+ * scale: usually 1/sqrt(dk). Returns GDN_OK after enqueueing one kernel.
+ */
+gdn_status_t gdn_decode(const void* q, const void* k, const void* v, const float* g,
+                        const float* beta, float* state_pool, int num_slots,
+                        const int32_t* slot_ids, void* o, int B, int T, int H, int dk, int dv,
+                        int n_h, float scale, gdn_dtype_t in_dtype, gdn_dtype_t out_dtype,
+                        void* stream);
+
+/* Prefill algorithm selection (gdn_chunk_prefill / gdn_chunk_prefill_workspace_size). */
+typedef enum {
+  GDN_PREFILL_AUTO = 0,       /* library picks from (N, H, total_T, dims) */
+  GDN_PREFILL_FUSED = 1,      /* tcgen05 chunk pipeline, state kept on chip across chunks;
+                                 dk == dv == 128, chunk == 64 */
+  GDN_PREFILL_TRANSFER = 2,   /* chunk-parallel local states + transfer matrices, then the
+                                 inter-chunk fixup scan, then outputs (the CP precompute
+                                 structure of the FlashInfer PR #3866 page, section 2);
+                                 for few (sequence, head) pairs with long sequences;
+                                 dk == dv == 128, chunk == 64 */
+  GDN_PREFILL_SEQUENTIAL = 3  /* token-sequential SIMT kernel, any dk == dv in {32, 64,
+                                 128}; the chunk size does not change its arithmetic */
+} gdn_prefill_algo_t;
+
+/*
+ * gdn_chunk_prefill_workspace_size — bytes of device workspace gdn_chunk_prefill
+ * needs for these sizes and this algorithm (0 is a valid answer). Host-only, no
+ * CUDA call: call it before stream capture. Returns (size_t)-1 for arguments
+ * gdn_chunk_prefill would reject (see gdn_last_error).
+ */
+size_t gdn_chunk_prefill_workspace_size(int N, int64_t total_T, int H, int dk, int dv, int chunk,
+                                        gdn_prefill_algo_t algo);
+
+/*
+ * gdn_chunk_prefill — chunked prefill over varlen sequences packed by cu_seqlens.
+ *
+ * For each sequence n (tokens cu_seqlens[n] .. cu_seqlens[n+1]-1) and head h,
+ * runs the recurrence from initial_state[n,h] (or zero) over the sequence,
+ * writes o for every token and the state after the last token to
+ * final_state[n,h]. Internally the sequence is cut into chunks of `chunk` tokens
+ * starting at the sequence start (the last chunk may be partial); within a chunk
+ * the WY/UT form with T = (I + tril(diag(beta) decay * K K^T))^{-1} is used, and
+ * the chunk states are passed along as S_{c+1} = M_c S_c + H_c (transfer M_c,
+ * local state H_c; FlashInfer PR #3866 page, section 2). An empty sequence
+ * copies its initial state (or zeros) to final_state.
+ *
+ *   q, k          [total_T, H, dk]   in_dtype
+ *   v             [total_T, H, dv]   in_dtype
+ *   g, beta       [total_T, H]       fp32 (g finite)
+ *   cu_seqlens    [N + 1] int32, DEVICE; cu[0] = 0, non-decreasing, cu[N] = total_T
+ *   initial_state [N, H, dv, dk] fp32 or NULL (zero state)
+ *   final_state   [N, H, dv, dk] fp32 or NULL (not written); may alias initial_state
+ *   o             [total_T, H, dv]   out_dtype
+ *   workspace     device buffer of >= gdn_chunk_prefill_workspace_size(...) bytes
+ *                 (may be NULL when that size is 0), 256-byte aligned, owned by the
+ *                 caller; must not be shared by calls that overlap on the GPU.
+ *
+ * Numerics: tensor-core products use fp16 operands with fp32 accumulation; the
+ * state is carried in fp32. Inputs must therefore lie within the fp16 range
+ * (|x| < 65504) on the FUSED and TRANSFER algorithms.
+ */
+gdn_status_t gdn_chunk_prefill(const void* q, const void* k, const void* v, const float* g,
+                               const float* beta, const int32_t* cu_seqlens, int N,
+                               int64_t total_T, const float* initial_state, float* final_state,
+                               void* o, int H, int dk, int dv, int chunk, float scale,
+                               gdn_dtype_t in_dtype, gdn_dtype_t out_dtype,
+                               gdn_prefill_algo_t algo, void* workspace, size_t workspace_bytes,
+                               void* stream);
+
+/* Message for the last non-OK status returned on this host thread ("" if none). */
+const char* gdn_last_error(void);
+
+/*
+ * gdn_get_device_error — read and clear the sticky device error word of the
+ * current CUDA device (GDN_DEVERR_* bits). Synchronous: waits for all prior work
+ * on the device. Returns GDN_OK when the word was 0, GDN_ERR_DEVICE_DATA when a
+ * bit was set (*flags gets the word), GDN_ERR_CUDA on a CUDA failure.
+ */
+gdn_status_t gdn_get_device_error(uint32_t* flags);
+
+/* Library version, e.g. "gdn 0.1.0 sm_100a". */
+const char* gdn_version(void);
+
+#ifdef __cplusplus
+}
+#endif
+
+#endif /* GDN_H_ */

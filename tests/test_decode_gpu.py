@@ -1,0 +1,140 @@
+"""GPU parity of gdn_decode (gated delta rule T=1 and the gated delta product)
+against the fp64 oracle, through the C ABI."""
+import numpy as np
+import pytest
+import torch
+
+import oracle
+import gated_delta_rule_58_b200 as gdn
+from gated_delta_rule_58_b200 import inputs
+from tests.util import assert_close, to64
+
+pytestmark = pytest.mark.gpu
+DEV = "cuda"
+
+
+def _run(inp, out_dtype=torch.bfloat16):
+    pool = inp.pool.to(DEV).clone()
+    q, k, v = inp.q.to(DEV), inp.k.to(DEV), inp.v.to(DEV)
+    g, beta = inp.g.to(DEV), inp.beta.to(DEV)
+    slots = inp.slot_ids.to(DEV)
+    B, T, H, dk = q.shape
+    o = torch.empty((B, T, H, v.shape[-1]), dtype=out_dtype, device=DEV)
+    gdn.gdn_decode(q, k, v, g, beta, pool, slots, o, scale=inp.scale)
+    torch.cuda.synchronize()
+    return o, pool
+
+
+def _check_against_oracle(inp, o, pool, what):
+    o_ref, pool_ref, _ = oracle.decode(inp.q, inp.k, inp.v, inp.g, inp.beta, inp.pool, inp.slot_ids,
+                                       scale=inp.scale)
+    assert_close(o, o_ref, what=f"{what} o")
+    used = sorted(set(int(s) for s in inp.slot_ids.tolist() if 0 <= s < inp.pool.shape[0]))
+    assert_close(pool[used], pool_ref[used], what=f"{what} state")
+    untouched = [s for s in range(inp.pool.shape[0]) if s not in used]
+    assert torch.equal(pool[untouched].cpu(), inp.pool[untouched]), "untouched slots changed"
+
+
+def test_decode_b64_h32_full_size():
+    """T=1 decode at the benchmark size: B=64, H=32, dk=dv=128, 256 slots, every head checked."""
+    inp = inputs.decode_b64_h32()
+    o, pool = _run(inp)
+    _check_against_oracle(inp, o, pool, "decode B64 H32")
+
+
+def test_gdp_b128_h32_t4_nh2_full_size():
+    """Gated delta product at the benchmark size: B=128, H=32, T=4, n_h=2, 512 slots."""
+    inp = inputs.gdp_b128_h32_t4_nh2()
+    o, pool = _run(inp)
+    _check_against_oracle(inp, o, pool, "GDP B128 T4 nh2")
+
+
+@pytest.mark.parametrize("d", [32, 64, 128])
+@pytest.mark.parametrize("T,nh", [(1, 1), (2, 1), (4, 1), (8, 1), (1, 2), (2, 2), (4, 2), (1, 4), (2, 4)])
+def test_decode_shapes(d, T, nh):
+    inp = inputs.decode_inputs(5, T, 3, d, d, nh, 9, seed=d + 10 * T + nh)
+    o, pool = _run(inp, out_dtype=torch.float32)
+    _check_against_oracle(inp, o, pool, f"d={d} T={T} nh={nh}")
+
+
+@pytest.mark.parametrize("dtype", [torch.float32, torch.bfloat16])
+def test_decode_input_dtypes(dtype):
+    inp = inputs.decode_inputs(7, 2, 4, 128, 128, 2, 10, seed=3, dtype=dtype)
+    for out in (torch.float32, torch.bfloat16):
+        o, pool = _run(inp, out_dtype=out)
+        _check_against_oracle(inp, o, pool, f"in={dtype} out={out}")
+
+
+def test_decode_weak_and_zero_decay():
+    for g_range in ((0.0, 0.0), (0.0, 0.01)):
+        inp = inputs.decode_inputs(8, 4, 4, 128, 128, 2, 16, seed=5, g_range=g_range)
+        o, pool = _run(inp, out_dtype=torch.float32)
+        _check_against_oracle(inp, o, pool, f"g_range={g_range}")
+
+
+def test_decode_alpha_zero():
+    """g = -inf (alpha = 0): the old state is dropped exactly."""
+    inp = inputs.decode_inputs(4, 1, 2, 128, 128, 1, 6, seed=6)
+    inp.g.fill_(float("-inf"))
+    o, pool = _run(inp, out_dtype=torch.float32)
+    _check_against_oracle(inp, o, pool, "alpha=0")
+    s = int(inp.slot_ids[0])
+    exp = inp.beta[0, 0, 0, 0] * torch.outer(inp.v[0, 0, 0, 0].float(), inp.k[0, 0, 0, 0].float())
+    assert torch.allclose(pool[s, 0].cpu(), exp, rtol=1e-6, atol=1e-7)
+
+
+def test_negative_slot_skips_row():
+    inp = inputs.decode_inputs(4, 2, 2, 64, 64, 1, 8, seed=7)
+    inp.slot_ids[1] = -1
+    o, pool = _run(inp, out_dtype=torch.float32)
+    assert torch.all(o[1] == 0)
+    _check_against_oracle(inp, o, pool, "negative slot")
+    assert gdn.gdn_get_device_error() == 0
+
+
+def test_out_of_range_slot_is_flagged_and_skipped():
+    inp = inputs.decode_inputs(3, 1, 2, 128, 128, 1, 6, seed=8)
+    gdn.gdn_get_device_error()  # clear
+    inp.slot_ids[2] = 6  # == num_slots
+    o, pool = _run(inp, out_dtype=torch.float32)
+    assert torch.all(o[2] == 0)
+    flags = gdn.gdn_get_device_error()
+    assert flags & gdn.GDN_DEVERR_SLOT_OUT_OF_RANGE
+    assert gdn.gdn_get_device_error() == 0  # read clears
+    _check_against_oracle(inp, o, pool, "slot out of range")
+
+
+def test_decode_deterministic_and_permutation_equivariant():
+    inp = inputs.decode_b64_h32(seed=11)
+    o1, p1 = _run(inp)
+    o2, p2 = _run(inp)
+    assert torch.equal(o1, o2) and torch.equal(p1, p2)
+    perm = torch.randperm(64, generator=torch.Generator().manual_seed(0))
+    inp_p = inputs.DecodeInputs(inp.q[perm], inp.k[perm], inp.v[perm], inp.g[perm], inp.beta[perm],
+                                inp.pool, inp.slot_ids[perm], inp.scale)
+    o3, p3 = _run(inp_p)
+    assert torch.equal(o3, o1[perm.to(DEV)]) and torch.equal(p3, p1)
+
+
+def test_decode_T_steps_equal_sequential_prefill_on_gpu():
+    """Decode applied token by token == the sequential GPU prefill over the same tokens."""
+    T, H, d = 6, 2, 64
+    pin = inputs.prefill_inputs([T], H, d, d, seed=12)
+    pool = torch.zeros((2, H, d, d), device=DEV)
+    pool[1] = pin.initial_state[0].to(DEV)
+    slots = torch.tensor([1], dtype=torch.int32, device=DEV)
+    outs = []
+    for t in range(T):
+        o = torch.empty((1, 1, H, d), device=DEV)
+        gdn.gdn_decode(pin.q[t][None, None].to(DEV), pin.k[t][None, None, :, None].to(DEV),
+                       pin.v[t][None, None, :, None].to(DEV), pin.g[t][None, None].to(DEV),
+                       pin.beta[t][None, None, :, None].to(DEV), pool, slots, o, scale=pin.scale)
+        outs.append(o[0, 0])
+    o_p = torch.empty((T, H, d), device=DEV)
+    fin = torch.empty((1, H, d, d), device=DEV)
+    gdn.gdn_chunk_prefill(pin.q.to(DEV), pin.k.to(DEV), pin.v.to(DEV), pin.g.to(DEV),
+                          pin.beta.to(DEV), pin.cu_seqlens.to(DEV), o_p,
+                          initial_state=pin.initial_state.to(DEV), final_state=fin, chunk=16,
+                          scale=pin.scale, algo=gdn.GDN_PREFILL_SEQUENTIAL)
+    assert_close(torch.stack(outs), o_p, tol=1e-5, what="decode vs prefill o")
+    assert_close(pool[1], fin[0], tol=1e-5, what="decode vs prefill state")

@@ -1,0 +1,104 @@
+"""The C-ABI library loads on a machine without a GPU, exports every symbol the
+header declares, and rejects bad arguments on the host before any CUDA call."""
+import ctypes
+
+import pytest
+
+import gated_delta_rule_58_b200 as gdn
+from gated_delta_rule_58_b200 import _lib
+
+
+@pytest.fixture(scope="module")
+def L():
+    from gated_delta_rule_58_b200 import build
+    build.build()
+    return _lib.lib()
+
+
+def test_exports_every_declared_symbol(L):
+    names = _lib.declared_functions()
+    assert {"gdn_decode", "gdn_chunk_prefill", "gdn_chunk_prefill_workspace_size",
+            "gdn_last_error", "gdn_get_device_error", "gdn_version"} <= set(names)
+    for n in names:
+        assert hasattr(L, n), f"libgdn.so does not export {n}"
+
+
+def test_version(L):
+    assert "sm_100a" in gdn.gdn_version()
+
+
+FAKE = 0x10000  # an aligned, never-dereferenced address: validation fails before any use
+
+
+def _decode(L, **kw):
+    a = dict(q=FAKE, k=FAKE, v=FAKE, g=FAKE, beta=FAKE, pool=FAKE, num_slots=4, slots=FAKE, o=FAKE,
+             B=2, T=1, H=2, dk=128, dv=128, nh=1, scale=0.1, din=0, dout=0, stream=None)
+    a.update(kw)
+    return L.gdn_decode(a["q"], a["k"], a["v"], a["g"], a["beta"], a["pool"], a["num_slots"], a["slots"],
+                        a["o"], a["B"], a["T"], a["H"], a["dk"], a["dv"], a["nh"], a["scale"], a["din"],
+                        a["dout"], a["stream"])
+
+
+@pytest.mark.parametrize("kw,status", [
+    (dict(dk=48, dv=48), gdn.GDN_ERR_UNSUPPORTED),
+    (dict(dk=128, dv=64), gdn.GDN_ERR_UNSUPPORTED),
+    (dict(T=0), gdn.GDN_ERR_INVALID_ARG),
+    (dict(H=0), gdn.GDN_ERR_INVALID_ARG),
+    (dict(nh=0), gdn.GDN_ERR_INVALID_ARG),
+    (dict(din=7), gdn.GDN_ERR_INVALID_ARG),
+    (dict(q=None), gdn.GDN_ERR_INVALID_ARG),
+    (dict(pool=FAKE + 4), gdn.GDN_ERR_INVALID_ARG),
+    (dict(slots=None), gdn.GDN_ERR_INVALID_ARG),
+])
+def test_decode_rejects_on_host(L, kw, status):
+    assert _decode(L, **kw) == status
+    assert gdn.gdn_last_error() != ""
+
+
+def test_decode_empty_batch_is_ok_without_gpu(L):
+    assert _decode(L, B=0, q=None, k=None, v=None) == gdn.GDN_OK
+
+
+def test_workspace_size_queries(L):
+    ws = gdn.gdn_chunk_prefill_workspace_size
+    assert ws(4, 32768, 16, 128, 128, 64, gdn.GDN_PREFILL_SEQUENTIAL) == 0
+    assert ws(1, 64, 2, 32, 32, 16, gdn.GDN_PREFILL_AUTO) == 0
+    with pytest.raises(gdn.GdnError):
+        ws(1, 64, 2, 48, 48, 16, gdn.GDN_PREFILL_AUTO)
+    with pytest.raises(gdn.GdnError):
+        ws(1, 64, 2, 128, 128, 32, gdn.GDN_PREFILL_FUSED)
+    assert L.gdn_chunk_prefill_workspace_size(-1, 0, 1, 32, 32, 16, 0) == ctypes.c_size_t(-1).value
+
+
+def _prefill(L, **kw):
+    a = dict(q=FAKE, k=FAKE, v=FAKE, g=FAKE, beta=FAKE, cu=FAKE, N=1, total=64, init=None, fin=FAKE,
+             o=FAKE, H=2, dk=32, dv=32, chunk=16, scale=0.1, din=1, dout=1, algo=0, ws=None, wsb=0,
+             stream=None)
+    a.update(kw)
+    return L.gdn_chunk_prefill(a["q"], a["k"], a["v"], a["g"], a["beta"], a["cu"], a["N"], a["total"],
+                               a["init"], a["fin"], a["o"], a["H"], a["dk"], a["dv"], a["chunk"],
+                               a["scale"], a["din"], a["dout"], a["algo"], a["ws"], a["wsb"], a["stream"])
+
+
+@pytest.mark.parametrize("kw,status", [
+    (dict(dk=48, dv=48), gdn.GDN_ERR_UNSUPPORTED),
+    (dict(N=-1), gdn.GDN_ERR_INVALID_ARG),
+    (dict(total=-5), gdn.GDN_ERR_INVALID_ARG),
+    (dict(chunk=0), gdn.GDN_ERR_INVALID_ARG),
+    (dict(cu=None), gdn.GDN_ERR_INVALID_ARG),
+    (dict(q=FAKE + 2), gdn.GDN_ERR_INVALID_ARG),
+    (dict(init=FAKE + 8), gdn.GDN_ERR_INVALID_ARG),
+    (dict(algo=9), gdn.GDN_ERR_INVALID_ARG),
+    (dict(dk=128, dv=128, chunk=32, algo=gdn.GDN_PREFILL_FUSED), gdn.GDN_ERR_UNSUPPORTED),
+    (dict(dout=5), gdn.GDN_ERR_INVALID_ARG),
+])
+def test_prefill_rejects_on_host(L, kw, status):
+    assert _prefill(L, **kw) == status
+    assert gdn.gdn_last_error() != ""
+
+
+def test_binding_fails_loudly_without_library(monkeypatch, tmp_path):
+    monkeypatch.setattr(_lib, "_lib", None)
+    monkeypatch.setattr(_lib, "LIB_PATH", str(tmp_path / "missing.so"))
+    with pytest.raises(RuntimeError, match="no CPU fallback"):
+        _lib.lib()
