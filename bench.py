@@ -360,7 +360,7 @@ def oracle_decode_rate(key, budget_s=10.0, seed=0):
     t0 = time.perf_counter()
     threads = 0
     while True:
-        _, pool, threads = oracle.decode(*args, pool, inp.slot_ids, scale=inp.scale)
+        _, pool, threads = oracle.decode(*args, pool, inp.slot_ids, scale=inp.scale, copy_pool=False)
         n += 1
         if time.perf_counter() - t0 >= budget_s:
             break

@@ -5,12 +5,12 @@
 
 namespace gdn {
 
-// Set once the tensor-core algorithms are built; until then AUTO takes the
-// sequential SIMT path for every shape.
-constexpr bool kTensorCorePrefillBuilt = false;
+// Set once the transfer (chunk-parallel fixup) algorithm is built; until then AUTO
+// takes the fused path for every tensor-core shape.
+constexpr bool kTransferPrefillBuilt = false;
 
 gdn_prefill_algo_t prefill_auto_tensor_core(const PrefillShape& s) {
-  if (!kTensorCorePrefillBuilt) return GDN_PREFILL_SEQUENTIAL;
+  if (!kTransferPrefillBuilt) return GDN_PREFILL_FUSED;
   // Few (sequence, head) pairs with long sequences leave most SMs idle on the fused
   // path (one chain of chunks per pair); the transfer path spreads the chunks of a
   // chain over all SMs and leaves only the short fixup scan serial.

@@ -114,16 +114,19 @@ def prefill(q, k, v, g, beta, cu_seqlens, initial_state=None, scale=None, nthrea
     return o, fin, rc
 
 
-def decode(q, k, v, g, beta, pool, slot_ids, scale=None, nthreads=0, lib=None):
+def decode(q, k, v, g, beta, pool, slot_ids, scale=None, nthreads=0, lib=None, copy_pool=True):
     """Sequential fp64 decode over a slot-indexed pool (the pool copy is updated).
 
     q: [B, T, H, dk]; k: [B, T, H, nh, dk]; v: [B, T, H, nh, dv]; g: [B, T, H];
     beta: [B, T, H, nh]; pool: [num_slots, H, dv, dk]; slot_ids: [B].
-    Returns (o [B, T, H, dv], new_pool, threads_used), fp64.
+    Returns (o [B, T, H, dv], new_pool, threads_used), fp64. With copy_pool=False an
+    fp64 C-contiguous numpy pool is updated in place (no copy).
     """
     lib = lib or _load()
     q, k, v, g, beta = (f64(a) for a in (q, k, v, g, beta))
-    pool = f64(pool).copy()
+    if copy_pool or not (isinstance(pool, np.ndarray) and pool.dtype == np.float64
+                         and pool.flags.c_contiguous):
+        pool = f64(pool).copy()
     slots = np.ascontiguousarray(np.asarray(f64(slot_ids), dtype=np.int32))
     B, T, H, dk = q.shape
     nh, dv = v.shape[3], v.shape[4]

@@ -79,3 +79,91 @@ def test_bad_cu_seqlens_flagged():
     inp.cu_seqlens[1] = 25  # > total
     run_prefill(inp, SEQ)
     assert gdn.gdn_get_device_error() & gdn.GDN_DEVERR_BAD_CU_SEQLENS
+
+
+# ---------------------------------------------------------------- fused tensor-core path
+
+FUSED = gdn.GDN_PREFILL_FUSED
+
+
+@pytest.mark.parametrize("g_range", [(0.01, 0.5), (0.0, 0.01), (0.0, 0.0)])
+def test_fused_varlen_edges(g_range):
+    """Lengths around the chunk size, an empty and a one-token sequence; weak and zero
+    decay make the state passing between chunks visible in the outputs."""
+    lens = [1, 0, 63, 64, 65, 130, 200, 7]
+    inp = inputs.prefill_inputs(lens, 3, 128, 128, seed=21, g_range=g_range)
+    check(inp, FUSED, what=f"fused {g_range}")
+
+
+@pytest.mark.parametrize("in_dtype", [torch.bfloat16, torch.float32])
+@pytest.mark.parametrize("out_dtype", [torch.bfloat16, torch.float32])
+def test_fused_dtypes(in_dtype, out_dtype):
+    inp = inputs.prefill_inputs([300, 65], 2, 128, 128, seed=22, dtype=in_dtype, g_range=(0.0, 0.05))
+    check(inp, FUSED, what="fused dtypes", out_dtype=out_dtype)
+
+
+def test_fused_no_initial_state_and_alias():
+    inp = inputs.prefill_inputs([129, 64], 2, 128, 128, seed=23, with_initial_state=False)
+    check(inp, FUSED, what="fused no init")
+    inp2 = inputs.prefill_inputs([129, 64], 2, 128, 128, seed=24, g_range=(0.0, 0.02))
+    check(inp2, FUSED, what="fused alias", alias=True)
+
+
+def test_fused_resume_equals_one_call():
+    """prefill(T1) then prefill(T2, init=final) equals prefill(T1 + T2), on the GPU."""
+    inp = inputs.prefill_inputs([320], 2, 128, 128, seed=25, g_range=(0.0, 0.01))
+    o_all, f_all = run_prefill(inp, FUSED)
+    a = inputs.PrefillInputs(inp.q[:192], inp.k[:192], inp.v[:192], inp.g[:192], inp.beta[:192],
+                             torch.tensor([0, 192], dtype=torch.int32), inp.initial_state, inp.scale)
+    o1, f1 = run_prefill(a, FUSED)
+    b = inputs.PrefillInputs(inp.q[192:], inp.k[192:], inp.v[192:], inp.g[192:], inp.beta[192:],
+                             torch.tensor([0, 128], dtype=torch.int32), f1.cpu(), inp.scale)
+    o2, f2 = run_prefill(b, FUSED)
+    assert_close(torch.cat([o1, o2]), o_all, tol=1e-5, what="resume o")
+    assert_close(f2, f_all, tol=1e-5, what="resume state")
+
+
+def test_fused_varlen_bitwise_equals_single_sequence_calls():
+    lens = [100, 37, 256]
+    inp = inputs.prefill_inputs(lens, 2, 128, 128, seed=26, g_range=(0.0, 0.02))
+    o, fin = run_prefill(inp, FUSED)
+    cu = inp.cu_seqlens.tolist()
+    for n in range(len(lens)):
+        sl = slice(cu[n], cu[n + 1])
+        one = inputs.PrefillInputs(inp.q[sl], inp.k[sl], inp.v[sl], inp.g[sl], inp.beta[sl],
+                                   torch.tensor([0, lens[n]], dtype=torch.int32),
+                                   inp.initial_state[n:n + 1], inp.scale)
+        o_n, f_n = run_prefill(one, FUSED)
+        assert torch.equal(o_n, o[sl]) and torch.equal(f_n[0], fin[n])
+    o2, fin2 = run_prefill(inp, FUSED)
+    assert torch.equal(o, o2) and torch.equal(fin, fin2)  # deterministic
+
+
+def test_fused_b4_t8192_h16_full_size():
+    """Chunked prefill at the benchmark size (B=4 x 8192, H=16), every (sequence, head)."""
+    inp = inputs.prefill_b4_t8192_h16()
+    check(inp, FUSED, what="B4 T8192 H16", out_dtype=torch.bfloat16)
+
+
+def _sampled_pairs_check(inp, algo, pairs, chunk=64):
+    o, fin = run_prefill(inp, algo, chunk=chunk, out_dtype=torch.bfloat16)
+    cu = inp.cu_seqlens.tolist()
+    for n, h in pairs:
+        sl = slice(cu[n], cu[n + 1])
+        L = cu[n + 1] - cu[n]
+        o_r, f_r, _ = oracle.prefill(inp.q[sl, h:h + 1], inp.k[sl, h:h + 1], inp.v[sl, h:h + 1],
+                                     inp.g[sl, h:h + 1], inp.beta[sl, h:h + 1], [0, L],
+                                     inp.initial_state[n:n + 1, h:h + 1], scale=inp.scale)
+        assert_close(o[sl, h:h + 1], o_r, what=f"pair ({n},{h}) o")
+        assert_close(fin[n:n + 1, h:h + 1], f_r, what=f"pair ({n},{h}) state")
+
+
+def test_fused_varlen32_h32_sampled():
+    """Varlen 32 sequences x H=32 at full size; the oracle checks a seeded sample of
+    (sequence, head) pairs, including the longest and the shortest sequence."""
+    inp = inputs.varlen32_h32(device=DEV)
+    lens = inp.seqlens
+    longest, shortest = int(np.argmax(lens)), int(np.argmin(lens))
+    rng = np.random.default_rng(0)
+    pairs = [(longest, 0), (shortest, 31)] + [(int(rng.integers(32)), int(rng.integers(32))) for _ in range(4)]
+    _sampled_pairs_check(inp, FUSED, pairs)
