@@ -13,18 +13,32 @@
 //   O^T = scale [ S^T Q^T diag(gamma) + U^T P^T ],  P = tril(exp(G_r - G_i) Q K^T)
 //   S^T <- gamma_C S^T + U^T diag(exp(G_C - G_i)) K
 //
-// Every product is written with the value dimension (dv = 128) or the key
-// dimension on the MMA's M side, so all MMAs are M = 128 (cta_group::1) with
-// fp16 operands in 128-byte-swizzled shared memory and fp32 accumulators in
-// TMEM. fp16 (10-bit mantissa) keeps the result within the 2e-3 tolerance where
-// bf16 operands do not; bf16 inputs are converted on load. The decay factors
-// exp(G_i - G_j) are taken on differences of cumulative gates (the cumulative
-// decay idiom of the FlashInfer PR #6291 page, section 2), never as a ratio.
+// Every product is written with the value or key dimension on the MMA's M side,
+// so all MMAs are M = 128 (cta_group::1) with fp16 operands in 128-byte-swizzled
+// shared memory (the fp16 copy of the state is read straight from TMEM as the A
+// operand) and fp32 accumulators in TMEM. fp16 (10-bit mantissa) keeps the
+// result within the 2e-3 tolerance where bf16 operands do not; bf16 inputs are
+// converted in shared memory. The decay factors exp(G_i - G_j) are taken on
+// differences of cumulative gates (the cumulative decay idiom of the FlashInfer
+// PR #6291 page, section 2), never as a ratio. The chunk step is the local-state /
+// transfer update S_{c+1} = M_c S_c + H_c of the FlashInfer PR #3866 page
+// (section 2) evaluated without materialising M_c or H_c.
 //
-// The local-state / transfer view of the same chunk step (S_{c+1} = M_c S_c +
-// H_c, FlashInfer PR #3866 page, section 2) is what this kernel evaluates
-// without materialising M_c or H_c: H_c = K~^T U~ and -K~^T W S_c are the two
-// halves of the accumulate into the state.
+// Warp specialisation (13 warps) and the chunk pipeline:
+//   loader  (warps 8-11): cp.async of chunk c's q/k/v rows straight into the
+//            swizzled fp16 tiles (bf16 bits converted in place), g/beta, the
+//            cumulative gates and decays. Runs up to one chunk ahead.
+//   prep    (warps 4-7):  A and P from [K;Q]K^T, the triangular solve, the fp16
+//            T diag(beta gamma) / T diag(beta) tiles, then W^T -> fp16 tile.
+//            Works on chunk c+1 while the state warps finish chunk c.
+//   state   (warps 0-3):  U^T -> fp16 tiles, the new state -> fp16 TMEM operand
+//            (and the gamma_C rescale of the fp32 TMEM state), outputs -> HBM.
+//   mma     (warp 12):    one thread issues every tcgen05.mma in dependency order.
+// Hand-offs are mbarriers: tcgen05.commit for MMA completion, one elected arrive
+// per warpgroup (after a named barrier) for thread-produced tiles. Every wait is
+// bounded; a timeout sets GDN_DEVERR_TIMEOUT and unwinds all roles.
+#include <type_traits>
+
 #include "prefill.cuh"
 #include "tcgen05.cuh"
 
@@ -33,48 +47,64 @@ namespace {
 
 constexpr int C = 64;      // chunk
 constexpr int D = 128;     // dk = dv
-constexpr int kThreads = 128;
-constexpr uint64_t kWaitNs = 2000000000ull;  // bounded MMA waits: 2 s
+constexpr int kThreads = 13 * 32;
+constexpr int kPrepWarp0 = 4, kLoadWarp0 = 8, kMmaWarp = 12;  // state warps are 0-3
+constexpr uint32_t kBarState = 1, kBarPrep = 2, kBarLoad = 3;  // named barrier ids
+constexpr uint64_t kWaitNs = 2000000000ull;                     // 2 s
 
-// Shared memory map (bytes from a 1024-aligned base). fp16 operand tiles use the
-// SWIZZLE_128B canonical layouts (see tcgen05.cuh).
-constexpr uint32_t OFF_KQ = 0;          // [2 dk halves][128 rows: K tokens 0-63, Q tokens 64-127][64] fp16
+// Shared memory map (bytes from a 1024-aligned base).
+constexpr uint32_t OFF_KQ = 0;          // 2 buffers: [2 dk halves][128 rows: K 0-63, Q 64-127][64] fp16
+constexpr uint32_t KQ_BUF = 32768;
 constexpr uint32_t KQ_HALF = 16384;
-constexpr uint32_t OFF_V = 32768;       // [2 dv halves][64 tokens][64] fp16
+constexpr uint32_t OFF_V = 65536;       // 2 buffers: [2 dv halves][64 tokens][64] fp16
+constexpr uint32_t V_BUF = 16384;
 constexpr uint32_t V_HALF = 8192;
-constexpr uint32_t OFF_S16 = 49152;     // S^T [2 dk halves][128 dv rows][64] fp16 (K-major A)
-constexpr uint32_t S16_HALF = 16384;
-constexpr uint32_t OFF_W16 = 81920;     // W^T [128 dk rows][64 tokens] fp16 (MN-major B)
-constexpr uint32_t OFF_U16 = 98304;     // U^T [128 dv rows][64 tokens] fp16 (K-major A)
-constexpr uint32_t OFF_UDD = 114688;    // U^T diag(exp(G_C - G_i)), same layout
-constexpr uint32_t OFF_TP = 131072;     // T diag(beta gamma)  [64 rows][64] fp16 (K-major B)
-constexpr uint32_t OFF_TPP = 139264;    // T diag(beta)        [64 rows][64] fp16
-constexpr uint32_t OFF_P16 = 147456;    // P                   [64 rows][64] fp16
-constexpr int LDA = C + 1;              // padded fp32 row stride
-constexpr uint32_t OFF_A = 155648;      // A fp32 [64][65]
-constexpr uint32_t OFF_T = OFF_A + C * LDA * 4;   // T fp32 [64][65]
-constexpr uint32_t OFF_X = OFF_T + C * LDA * 4;   // 3 x 16x16 fp32 scratch
-constexpr uint32_t OFF_VEC = OFF_X + 3 * 256 * 4; // G, gamma, dd, beta, beta*gamma (5 x 64 fp32)
-constexpr uint32_t OFF_BAR = OFF_VEC + 5 * C * 4; // mbarrier, TMEM base, abort flag
-constexpr uint32_t SMEM_USED = OFF_BAR + 64;
-constexpr uint32_t SMEM_BYTES = SMEM_USED + 1024;  // slack for 1024-byte alignment
+constexpr uint32_t OFF_W16 = 98304;     // W^T [128 dk rows][64 tokens] fp16 (MN-major B)
+constexpr uint32_t OFF_U16 = 114688;    // U^T [128 dv rows][64 tokens] fp16 (K-major A)
+constexpr uint32_t OFF_UDD = 131072;    // U^T diag(exp(G_C - G_i))
+constexpr uint32_t OFF_TP = 147456;     // T diag(beta gamma) [64][64] fp16 (K-major B)
+constexpr uint32_t OFF_TPP = 155648;    // T diag(beta)
+constexpr uint32_t OFF_P16 = 163840;    // 2 buffers: P [64][64] fp16 (K-major B)
+constexpr uint32_t P_BUF = 8192;
+constexpr uint32_t OFF_A = 180224;      // A fp32 [64][64], 16-byte chunks XOR-swizzled by row
+constexpr uint32_t OFF_T = 196608;      // T fp32 [64][64], same swizzle
+constexpr uint32_t OFF_VEC = 212992;    // 2 buffers x {G, gamma, dd, beta, beta*gamma} x 64 fp32
+constexpr uint32_t VEC_BUF = 5 * C * 4;
+constexpr uint32_t OFF_BAR = OFF_VEC + 2 * VEC_BUF;
+constexpr uint32_t SMEM_USED = OFF_BAR + 256;
+constexpr uint32_t SMEM_BYTES = SMEM_USED + 1024;  // slack for the 1024-byte alignment
 
-// TMEM columns (fp32 accumulators, 128 lanes)
-constexpr uint32_t COL_S = 0;     // S^T: lane = dv row, 128 columns = dk
-constexpr uint32_t COL_D1 = 128;  // [K;Q] K^T: lanes 0-63 K K^T, 64-127 Q K^T
-constexpr uint32_t COL_W = 192;   // W^T: lane = dk, column = token
-constexpr uint32_t COL_U = 256;   // U~^T then U^T: lane = dv, column = token
-constexpr uint32_t COL_O1 = 320;  // S^T Q^T
-constexpr uint32_t COL_O2 = 384;  // U^T P^T
+// TMEM columns (fp32, 128 lanes)
+constexpr uint32_t COL_S = 0;     // S^T: lane = dv row, columns = dk
+constexpr uint32_t COL_D1 = 128;  // [K;Q] K^T (lanes 0-63 K K^T, 64-127 Q K^T)
+constexpr uint32_t COL_SH = 192;  // fp16 S^T as the MMA A operand: two halves per column
+constexpr uint32_t COL_W = 256;   // W^T: lane = dk, column = token
+constexpr uint32_t COL_U = 320;   // U~^T then U^T: lane = dv, column = token
+constexpr uint32_t COL_O1 = 384;  // S^T Q^T
+constexpr uint32_t COL_O2 = 448;  // U^T P^T
 constexpr uint32_t TMEM_COLS = 512;
+
+// mbarrier slots
+enum Bar : int {
+  B_L0 = 0, B_L1,      // loader -> chunk tiles ready (per buffer)
+  B_M1,                // MMA: D1 ready
+  B_M2,                // MMA: W^T, U~^T ready
+  B_M3A,               // MMA: U^T ready (S16, W16 consumed)
+  B_M4B,               // MMA: new state ready
+  B_M4A,               // MMA: O2 ready (all chunk MMAs done)
+  B_E2,                // prep: T', T'', P ready, D1 buffer consumed
+  B_E3,                // prep: W16 ready, W region consumed
+  B_E5,                // state: U16/UDD ready, U region consumed
+  B_E6A,               // state: S16 ready, TMEM state rescaled
+  B_E6B,               // state: O1/O2 consumed
+  B_COUNT
+};
 
 __device__ __forceinline__ uint32_t pack_half2(float a, float b) {
   __half2 h = __floats2half2_rn(a, b);
   return *reinterpret_cast<uint32_t*>(&h);
 }
 
-// Writes 8 fp32 values as fp16 into 16-byte chunk `chunk` of row `row` of a
-// swizzled tile at byte address `tile` (8-row groups 1024 bytes apart).
 __device__ __forceinline__ void st_sw128_chunk(uint8_t* tile, uint32_t row, uint32_t chunk, const float* v) {
   uint4 u;
   u.x = pack_half2(v[0], v[1]);
@@ -84,207 +114,361 @@ __device__ __forceinline__ void st_sw128_chunk(uint8_t* tile, uint32_t row, uint
   *reinterpret_cast<uint4*>(tile + tc::sw128_offset(row, chunk, 1024)) = u;
 }
 
+// [64][64] fp32 matrices: element (i, j) lives at i*64 + (j ^ ((i & 7) << 2)), i.e.
+// the 16-byte chunks of a row are XOR-swizzled so that row-wise float4 accesses by
+// consecutive rows and column-wise scalar accesses are both bank-conflict free.
+__device__ __forceinline__ int sidx(int i, int j) { return i * 64 + (j ^ ((i & 7) << 2)); }
+
 struct Smem {
   uint8_t* base;
   __device__ float* A() const { return reinterpret_cast<float*>(base + OFF_A); }
   __device__ float* T() const { return reinterpret_cast<float*>(base + OFF_T); }
-  __device__ float* X() const { return reinterpret_cast<float*>(base + OFF_X); }
-  __device__ float* G() const { return reinterpret_cast<float*>(base + OFF_VEC); }
-  __device__ float* gam() const { return G() + C; }
-  __device__ float* dd() const { return G() + 2 * C; }
-  __device__ float* beta() const { return G() + 3 * C; }
-  __device__ float* bg() const { return G() + 4 * C; }
-  __device__ uint64_t* bar() const { return reinterpret_cast<uint64_t*>(base + OFF_BAR); }
-  __device__ uint32_t* tmem_slot() const { return reinterpret_cast<uint32_t*>(base + OFF_BAR + 8); }
-  __device__ int* abort_flag() const { return reinterpret_cast<int*>(base + OFF_BAR + 12); }
+  __device__ float* vec(int b) const { return reinterpret_cast<float*>(base + OFF_VEC + b * VEC_BUF); }
+  __device__ uint64_t* bar(int i) const { return reinterpret_cast<uint64_t*>(base + OFF_BAR) + i; }
+  __device__ uint32_t* tmem_slot() const { return reinterpret_cast<uint32_t*>(base + OFF_BAR + 8 * B_COUNT); }
+  __device__ volatile int* abort_flag() const {
+    return reinterpret_cast<volatile int*>(base + OFF_BAR + 8 * B_COUNT + 4);
+  }
   __device__ uint32_t u32(uint32_t off) const { return tc::smem_u32(base + off); }
 };
+// vec(b) layout: [0,64) G, [64,128) gamma, [128,192) dd, [192,256) beta, [256,320) beta*gamma
+constexpr int V_G = 0, V_GAM = 64, V_DD = 128, V_BETA = 192, V_BG = 256;
 
-// Thread 0 waits for the committed MMAs; everyone then learns whether they finished.
-__device__ __forceinline__ bool wait_mma(const Smem& sm, uint32_t& phase, unsigned int* err) {
-  if (threadIdx.x == 0) {
-    if (!tc::mbar_wait(sm.bar(), phase, kWaitNs)) {
-      *sm.abort_flag() = 1;
-      raise_device_error(err, GDN_DEVERR_TIMEOUT);
-    }
-  }
-  phase ^= 1u;
-  __syncthreads();
-  tc::fence_after_sync();
-  return *sm.abort_flag() == 0;
+__device__ __forceinline__ bool wait_bar(const Smem& sm, int b, uint32_t parity, unsigned int* err) {
+  if (tc::mbar_wait(sm.bar(b), parity, kWaitNs, sm.abort_flag())) return true;
+  if (*sm.abort_flag() == 0) raise_device_error(err, GDN_DEVERR_TIMEOUT);
+  *sm.abort_flag() = 1;
+  return false;
 }
 
-// Barrier after threads wrote operand tiles (generic proxy) and/or touched TMEM,
-// before the MMA issuer reads them.
-__device__ __forceinline__ void publish_to_mma() {
+// Warpgroup hand-off: writers' smem visible to the async proxy and TMEM accesses
+// ordered, the group synchronised, then one elected arrive.
+__device__ __forceinline__ void group_signal(const Smem& sm, uint32_t bar_id, int b) {
   tc::fence_proxy_async_smem();
   tc::fence_before_sync();
-  __syncthreads();
+  tc::named_sync(bar_id, 128);
+  if ((threadIdx.x & 127) == 0) tc::mbar_arrive(sm.bar(b));
 }
+
+// ---------------------------------------------------------------- loader role
 
 template <typename TIn>
-__device__ __forceinline__ void load_chunk(const Smem& sm, const PrefillShape& s, const PrefillArgs& a, int h,
-                                           int64_t t0, int Lc) {
-  const int tid = threadIdx.x;
-  if (tid < C) {
-    float gv = 0.f, bv = 0.f;
-    if (tid < Lc) {
-      const size_t th = (size_t)(t0 + tid) * s.H + h;
-      gv = __ldg(a.g + th);
-      bv = __ldg(a.beta + th);
-    }
-    sm.G()[tid] = gv;
-    sm.beta()[tid] = bv;
-  }
-  const TIn* srcs[3] = {static_cast<const TIn*>(a.k), static_cast<const TIn*>(a.q), static_cast<const TIn*>(a.v)};
+__device__ void loader_role(const Smem& sm, const PrefillShape& s, const PrefillArgs& a, int h, int64_t bos,
+                            int64_t eos, int nchunks) {
+  const int t = threadIdx.x - kLoadWarp0 * 32;  // 0..127
+  for (int c = 0; c < nchunks; ++c) {
+    const int b = c & 1;
+    // chunk c-2 (same buffers) fully consumed: its outputs were read, so every
+    // MMA of that chunk, including the ones reading K, Q and V, has completed
+    if (c >= 2 && !wait_bar(sm, B_E6B, (c - 2) & 1, a.err)) return;
+    const int64_t t0 = bos + (int64_t)c * C;
+    const int Lc = (int)((eos - t0) < C ? (eos - t0) : C);
+    float* vec = sm.vec(b);
+#pragma unroll
+    for (int mat = 0; mat < 3; ++mat) {
+      const TIn* src0 = static_cast<const TIn*>(mat == 0 ? a.k : (mat == 1 ? a.q : a.v));
+      uint8_t* base = (mat == 2) ? sm.base + OFF_V + b * V_BUF : sm.base + OFF_KQ + b * KQ_BUF;
+      const uint32_t half = (mat == 2) ? V_HALF : KQ_HALF;
+      const int roff = (mat == 1) ? C : 0;
 #pragma unroll 4
-  for (int i = tid; i < 3 * C * 16; i += kThreads) {
-    const int mat = i / (C * 16);
-    const int rem = i - mat * (C * 16);
-    const int row = rem >> 4;
-    const int ch = rem & 15;  // 8-element chunk of the 128-wide row
-    float v8[8];
-    if (row < Lc) {
-      load8_f32(srcs[mat] + ((size_t)(t0 + row) * s.H + h) * D + ch * 8, v8);
-    } else {
+      for (int i = t; i < C * 16; i += 128) {
+        const int row = i >> 4, ch = i & 15;
+        uint8_t* tile = base + (ch >> 3) * half;
+        const uint32_t off = tc::sw128_offset(row + roff, ch & 7, 1024);
+        const TIn* src = src0 + ((size_t)(t0 + (row < Lc ? row : 0)) * s.H + h) * D + ch * 8;
+        if constexpr (std::is_same<TIn, __nv_bfloat16>::value) {
+          tc::cp_async16(tc::smem_u32(tile + off), src, row < Lc ? 16u : 0u);
+        } else {
+          float v8[8];
+          if (row < Lc) {
+            load8_f32(src, v8);
+          } else {
 #pragma unroll
-      for (int x = 0; x < 8; ++x) v8[x] = 0.f;
+            for (int x = 0; x < 8; ++x) v8[x] = 0.f;
+          }
+          st_sw128_chunk(tile, row + roff, ch & 7, v8);
+        }
+      }
     }
-    uint8_t* tile;
-    uint32_t r;
-    if (mat == 2) {
-      tile = sm.base + OFF_V + (ch >> 3) * V_HALF;
-      r = row;
-    } else {
-      tile = sm.base + OFF_KQ + (ch >> 3) * KQ_HALF;
-      r = row + (mat == 1 ? C : 0);
+    if (t < C) {  // g and beta (scalar loads, issued behind the async copies)
+      float gv = 0.f, bv = 0.f;
+      if (t < Lc) {
+        const size_t th = (size_t)(t0 + t) * s.H + h;
+        gv = __ldg(a.g + th);
+        bv = __ldg(a.beta + th);
+      }
+      vec[V_G + t] = gv;
+      vec[V_BETA + t] = bv;
     }
-    st_sw128_chunk(tile, r, ch & 7, v8);
+    if constexpr (std::is_same<TIn, __nv_bfloat16>::value) {
+      tc::cp_async_commit();
+      tc::cp_async_wait_all();
+      // bf16 -> fp16 in place: each thread converts the chunks it copied
+#pragma unroll
+      for (int mat = 0; mat < 3; ++mat) {
+        uint8_t* base = (mat == 2) ? sm.base + OFF_V + b * V_BUF : sm.base + OFF_KQ + b * KQ_BUF;
+        const uint32_t half = (mat == 2) ? V_HALF : KQ_HALF;
+        const int roff = (mat == 1) ? C : 0;
+#pragma unroll 4
+        for (int i = t; i < C * 16; i += 128) {
+          const int row = i >> 4, ch = i & 15;
+          uint4* p = reinterpret_cast<uint4*>(base + (ch >> 3) * half + tc::sw128_offset(row + roff, ch & 7, 1024));
+          const uint4 raw = *p;
+          const __nv_bfloat162* hb = reinterpret_cast<const __nv_bfloat162*>(&raw);
+          uint4 u;
+          float2 f0 = __bfloat1622float2(hb[0]), f1 = __bfloat1622float2(hb[1]);
+          float2 f2 = __bfloat1622float2(hb[2]), f3 = __bfloat1622float2(hb[3]);
+          u.x = pack_half2(f0.x, f0.y);
+          u.y = pack_half2(f1.x, f1.y);
+          u.z = pack_half2(f2.x, f2.y);
+          u.w = pack_half2(f3.x, f3.y);
+          *p = u;
+        }
+      }
+    }
+    tc::named_sync(kBarLoad, 128);
+    if (t < 32) {
+      // inclusive cumulative sum of the chunk's log gates (two per lane), decays
+      const float x0 = vec[V_G + 2 * t], x1 = vec[V_G + 2 * t + 1];
+      float pre = x0 + x1;
+#pragma unroll
+      for (int off = 1; off < 32; off <<= 1) {
+        const float y = __shfl_up_sync(0xffffffffu, pre, off);
+        if (t >= off) pre += y;
+      }
+      const float Gc = __shfl_sync(0xffffffffu, pre, 31);
+#pragma unroll
+      for (int e = 0; e < 2; ++e) {
+        const int i = 2 * t + e;
+        const float Gi = e ? pre : pre - x1;
+        const float gm = __expf(Gi);
+        vec[V_G + i] = Gi;
+        vec[V_GAM + i] = gm;
+        vec[V_DD + i] = __expf(Gc - Gi);
+        vec[V_BG + i] = vec[V_BETA + i] * gm;
+      }
+    }
+    group_signal(sm, kBarLoad, B_L0 + b);
   }
-  __syncthreads();
-  if (tid < 32) {
-    // inclusive cumulative sum of the chunk's log gates (two per lane)
-    const float x0 = sm.G()[2 * tid], x1 = sm.G()[2 * tid + 1];
-    float pre = x0 + x1;
-#pragma unroll
-    for (int off = 1; off < 32; off <<= 1) {
-      const float y = __shfl_up_sync(0xffffffffu, pre, off);
-      if (tid >= off) pre += y;
-    }
-    __syncwarp();
-    sm.G()[2 * tid] = pre - x1;
-    sm.G()[2 * tid + 1] = pre;
-    __syncwarp();
-    const float Gc = __shfl_sync(0xffffffffu, pre, 31);
-#pragma unroll
-    for (int e = 0; e < 2; ++e) {
-      const int i = 2 * tid + e;
-      const float Gi = e ? pre : pre - x1;
-      const float gm = __expf(Gi);
-      sm.gam()[i] = gm;
-      sm.dd()[i] = __expf(Gc - Gi);
-      sm.bg()[i] = sm.beta()[i] * gm;
-    }
-  }
-  publish_to_mma();
 }
 
-// T = (I + A)^{-1} for the strictly lower 64x64 A in shared memory (fp32):
-// 16x16 diagonal blocks by forward substitution, then the off-diagonal blocks
-// by diagonals: T_ij = -T_ii sum_{k=j}^{i-1} A_ik T_kj.
-__device__ __forceinline__ void solve_unit_lower(const Smem& sm) {
-  const int tid = threadIdx.x;
+// ---------------------------------------------------------------- prep role
+
+// 16-byte chunk q of row i of a [64][64] fp32 matrix (chunks XOR-swizzled by row).
+__device__ __forceinline__ float4* row_chunk(float* M, int i, int q) {
+  return reinterpret_cast<float4*>(M + i * 64 + 4 * (q ^ (i & 7)));
+}
+
+__device__ __forceinline__ uint32_t to_tf32(float x) {
+  uint32_t r;
+  asm("cvt.rna.tf32.f32 %0, %1;" : "=r"(r) : "f"(x));
+  return r;
+}
+
+// Warp-level D(16x8) += A(16x8) B(8x8) on tf32 tensor cores, fp32 accumulate.
+__device__ __forceinline__ void mma_tf32_16x8x8(float* d, const uint32_t* a, const uint32_t* b) {
+  asm volatile("mma.sync.aligned.m16n8k8.row.col.f32.tf32.tf32.f32 {%0,%1,%2,%3}, {%4,%5,%6,%7}, {%8,%9}, "
+               "{%0,%1,%2,%3};"
+               : "+f"(d[0]), "+f"(d[1]), "+f"(d[2]), "+f"(d[3])
+               : "r"(a[0]), "r"(a[1]), "r"(a[2]), "r"(a[3]), "r"(b[0]), "r"(b[1]));
+}
+
+// acc (16x16 block, two m16n8 fragments) += M1[r1.., c1..] (16x16) * M2[r2.., c2..] (16x16),
+// both [64][64] fp32 swizzled tiles in shared memory. Fragment layout of
+// m16n8k8: g = lane / 4, t = lane % 4; A: (g, t), (g+8, t), (g, t+4), (g+8, t+4);
+// B: (t, g), (t+4, g); C: (g, 2t), (g, 2t+1), (g+8, 2t), (g+8, 2t+1).
+__device__ __forceinline__ void warp_block_mma(float (*acc)[4], const float* M1, int r1, int c1, const float* M2,
+                                               int r2, int c2, int lane) {
+  const int g = lane >> 2, t = lane & 3;
+#pragma unroll
+  for (int ks = 0; ks < 2; ++ks) {
+    uint32_t a[4];
+    a[0] = to_tf32(M1[sidx(r1 + g, c1 + 8 * ks + t)]);
+    a[1] = to_tf32(M1[sidx(r1 + g + 8, c1 + 8 * ks + t)]);
+    a[2] = to_tf32(M1[sidx(r1 + g, c1 + 8 * ks + t + 4)]);
+    a[3] = to_tf32(M1[sidx(r1 + g + 8, c1 + 8 * ks + t + 4)]);
+#pragma unroll
+    for (int nt = 0; nt < 2; ++nt) {
+      uint32_t b[2];
+      b[0] = to_tf32(M2[sidx(r2 + 8 * ks + t, c2 + 8 * nt + g)]);
+      b[1] = to_tf32(M2[sidx(r2 + 8 * ks + t + 4, c2 + 8 * nt + g)]);
+      mma_tf32_16x8x8(acc[nt], a, b);
+    }
+  }
+}
+
+// Writes a 16x16 accumulator (two m16n8 fragments) times `sign` into a swizzled tile.
+__device__ __forceinline__ void warp_block_store(float* M, int r0, int c0, float (*acc)[4], float sign, int lane) {
+  const int g = lane >> 2, t = lane & 3;
+#pragma unroll
+  for (int nt = 0; nt < 2; ++nt) {
+    M[sidx(r0 + g, c0 + 8 * nt + 2 * t)] = sign * acc[nt][0];
+    M[sidx(r0 + g, c0 + 8 * nt + 2 * t + 1)] = sign * acc[nt][1];
+    M[sidx(r0 + g + 8, c0 + 8 * nt + 2 * t)] = sign * acc[nt][2];
+    M[sidx(r0 + g + 8, c0 + 8 * nt + 2 * t + 1)] = sign * acc[nt][3];
+  }
+}
+
+// T = (I + A)^{-1} for the strictly lower 64x64 A (fp32). The four 16x16 diagonal
+// blocks are inverted by forward substitution (one thread per column); the
+// off-diagonal blocks follow level by level, T_ij = -T_ii sum_{k=j}^{i-1} A_ik T_kj,
+// one warp per block, on tf32 warp MMAs. X_ij is parked in the diagonal block
+// A_ii, which the solve no longer reads.
+__device__ __forceinline__ void solve_unit_lower(const Smem& sm, int t) {
   float* A = sm.A();
   float* T = sm.T();
-  float* X = sm.X();
-  if (tid < C) {
-    const int b = tid >> 4, c = tid & 15;
-    float t[16];
+  if (t < C) {
+    const int b = t >> 4, c = t & 15;
+    float x[16];
 #pragma unroll
     for (int r = 0; r < 16; ++r) {
-      float acc = 0.f;
+      float acc0 = 0.f, acc1 = 0.f;
 #pragma unroll
-      for (int k = 0; k < r; ++k) acc = fmaf(A[(16 * b + r) * LDA + 16 * b + k], t[k], acc);
-      t[r] = (r < c) ? 0.f : ((r == c) ? 1.f : -acc);
-    }
-#pragma unroll
-    for (int r = 0; r < 16; ++r) T[(16 * b + r) * LDA + 16 * b + c] = t[r];
-  }
-  __syncthreads();
-  for (int d = 1; d < 4; ++d) {
-    const int nb = 4 - d;
-    for (int o = threadIdx.x; o < nb * 256; o += kThreads) {
-      const int bi = o >> 8, i = d + bi, j = i - d, r = (o >> 4) & 15, cc = o & 15;
-      float acc = 0.f;
-      for (int k = j; k < i; ++k) {
-#pragma unroll
-        for (int m = 0; m < 16; ++m)
-          acc = fmaf(A[(16 * i + r) * LDA + 16 * k + m], T[(16 * k + m) * LDA + 16 * j + cc], acc);
+      for (int k = 0; k < r; ++k) {
+        if (k & 1) acc1 = fmaf(A[sidx(16 * b + r, 16 * b + k)], x[k], acc1);
+        else acc0 = fmaf(A[sidx(16 * b + r, 16 * b + k)], x[k], acc0);
       }
-      X[bi * 256 + r * 16 + cc] = acc;
+      x[r] = (r < c) ? 0.f : ((r == c) ? 1.f : -(acc0 + acc1));
     }
-    __syncthreads();
-    for (int o = threadIdx.x; o < nb * 256; o += kThreads) {
-      const int bi = o >> 8, i = d + bi, j = i - d, r = (o >> 4) & 15, cc = o & 15;
-      float acc = 0.f;
 #pragma unroll
-      for (int m = 0; m < 16; ++m) acc = fmaf(T[(16 * i + r) * LDA + 16 * i + m], X[bi * 256 + m * 16 + cc], acc);
-      T[(16 * i + r) * LDA + 16 * j + cc] = -acc;
+    for (int r = 0; r < 16; ++r) T[sidx(16 * b + r, 16 * b + c)] = x[r];
+  }
+  tc::named_sync(kBarPrep, 128);
+  const int w = t >> 5, lane = t & 31;
+#pragma unroll 1
+  for (int d = 1; d < 4; ++d) {
+    if (w < 4 - d) {
+      const int i = d + w, j = i - d;
+      float acc[2][4] = {{0.f, 0.f, 0.f, 0.f}, {0.f, 0.f, 0.f, 0.f}};
+      for (int k = j; k < i; ++k) warp_block_mma(acc, A, 16 * i, 16 * k, T, 16 * k, 16 * j, lane);
+      warp_block_store(A, 16 * i, 16 * i, acc, 1.f, lane);  // X_ij parked in A_ii
+      __syncwarp();
+      float y[2][4] = {{0.f, 0.f, 0.f, 0.f}, {0.f, 0.f, 0.f, 0.f}};
+      warp_block_mma(y, T, 16 * i, 16 * i, A, 16 * i, 16 * i, lane);
+      warp_block_store(T, 16 * i, 16 * j, y, -1.f, lane);
     }
-    __syncthreads();
+    tc::named_sync(kBarPrep, 128);
   }
 }
 
-template <typename TIn, typename TOut>
-__global__ void __launch_bounds__(kThreads, 1)
-gdn_prefill_fused_kernel(const PrefillShape s, const PrefillArgs a) {
-  extern __shared__ uint8_t smem_raw[];
-  Smem sm;
-  sm.base = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
-  const int tid = threadIdx.x;
-  const int warp = tid >> 5;
-  const int n = blockIdx.x / s.H;
-  const int h = blockIdx.x - n * s.H;
-  int64_t bos, eos;
-  if (!seq_bounds(a.cu_seqlens, n, s.total_T, a.err, &bos, &eos)) return;
-
-  const size_t state_off = ((size_t)n * s.H + h) * (size_t)D * D;
-  const int64_t L = eos - bos;
-  const int nchunks = (int)((L + C - 1) / C);
-  if (nchunks == 0) {  // empty sequence: the state passes through
-    if (a.final_state) {
-      for (int i = tid; i < D * D / 4; i += kThreads) {
-        const float4 x = a.initial_state ? reinterpret_cast<const float4*>(a.initial_state + state_off)[i]
-                                         : make_float4(0.f, 0.f, 0.f, 0.f);
-        reinterpret_cast<float4*>(a.final_state + state_off)[i] = x;
+__device__ void prep_role(const Smem& sm, uint32_t tmem, int nchunks, unsigned int* err) {
+  const int t = threadIdx.x - kPrepWarp0 * 32;  // 0..127 == TMEM lane
+  const int warp = threadIdx.x >> 5;
+  const uint32_t tl = tmem + ((uint32_t)((warp & 3) * 32) << 16);
+  for (int c = 0; c < nchunks; ++c) {
+    const int b = c & 1;
+    if (!wait_bar(sm, B_L0 + b, (c >> 1) & 1, err)) return;
+    if (!wait_bar(sm, B_M1, c & 1, err)) return;
+    tc::fence_after_sync();
+    const float* vec = sm.vec(b);
+    const float* G = vec + V_G;
+    if (t < C) {
+      // A row t (rows 0-63 of D1): beta_t exp(G_t - G_j) k_t.k_j for j < t; the
+      // chunks right of the diagonal are never read by the solve and are skipped
+      const float Gi = G[t], bi = vec[V_BETA + t];
+#pragma unroll
+      for (int hq = 0; hq < 2; ++hq) {
+        // tcgen05.ld is warp-collective: the condition must be uniform across the
+        // warp, so it uses the warp's largest row (t | 31)
+        if (32 * hq < (t | 31)) {
+          float x[32];
+          tc::tmem_ld16(tl + COL_D1 + hq * 32, x);
+          tc::tmem_ld16(tl + COL_D1 + hq * 32 + 16, x + 16);
+          tc::wait_ld();
+#pragma unroll
+          for (int q = 0; q < 8; ++q) {
+            const int j0 = 32 * hq + 4 * q;
+            if (j0 < t) {
+              float4 v;
+              v.x = (j0 + 0 < t) ? bi * __expf(Gi - G[j0 + 0]) * x[4 * q + 0] : 0.f;
+              v.y = (j0 + 1 < t) ? bi * __expf(Gi - G[j0 + 1]) * x[4 * q + 1] : 0.f;
+              v.z = (j0 + 2 < t) ? bi * __expf(Gi - G[j0 + 2]) * x[4 * q + 2] : 0.f;
+              v.w = (j0 + 3 < t) ? bi * __expf(Gi - G[j0 + 3]) * x[4 * q + 3] : 0.f;
+              *row_chunk(sm.A(), t, j0 >> 2) = v;
+            }
+          }
+        }
+      }
+    } else {
+      // P row r (rows 64-127 of D1) into P16[b]; its previous reader (chunk c-2's O2
+      // MMA) completed before this chunk's D1 MMA, whose completion was waited on
+      const int r = t - C;
+      const float Gr = G[r];
+#pragma unroll
+      for (int hq = 0; hq < 2; ++hq) {
+        float x[32];
+        tc::tmem_ld16(tl + COL_D1 + hq * 32, x);
+        tc::tmem_ld16(tl + COL_D1 + hq * 32 + 16, x + 16);
+        tc::wait_ld();
+#pragma unroll
+        for (int cc = 0; cc < 4; ++cc) {
+          float v[8];
+#pragma unroll
+          for (int m = 0; m < 8; ++m) {
+            const int i = 32 * hq + cc * 8 + m;
+            v[m] = (i <= r) ? __expf(Gr - G[i]) * x[cc * 8 + m] : 0.f;  // zeros above the diagonal
+          }
+          st_sw128_chunk(sm.base + OFF_P16 + b * P_BUF, r, 4 * hq + cc, v);
+        }
       }
     }
-    return;
+    tc::named_sync(kBarPrep, 128);
+    solve_unit_lower(sm, t);
+    // T diag(beta gamma) and T diag(beta) as fp16 (the previous chunk's W/U~ MMA
+    // finished reading them: B_M2 of chunk c-1 was waited before E3 of chunk c-1)
+    {
+      const int mat = t >> 6, i = t & 63;
+      const float* colscale = vec + (mat ? V_BETA : V_BG);
+      uint8_t* tile = sm.base + (mat ? OFF_TPP : OFF_TP);
+#pragma unroll
+      for (int cc = 0; cc < 8; ++cc) {
+        const float4 lo = *row_chunk(sm.T(), i, 2 * cc), hi = *row_chunk(sm.T(), i, 2 * cc + 1);
+        const float tv[8] = {lo.x, lo.y, lo.z, lo.w, hi.x, hi.y, hi.z, hi.w};
+        float v[8];
+#pragma unroll
+        for (int m = 0; m < 8; ++m) {
+          const int j = cc * 8 + m;
+          v[m] = (j <= i) ? tv[m] * colscale[j] : 0.f;
+        }
+        st_sw128_chunk(tile, i, cc, v);
+      }
+    }
+    group_signal(sm, kBarPrep, B_E2);
+    // W^T -> fp16 once the W MMA is done and the previous chunk's M3a read W16
+    if (!wait_bar(sm, B_M2, c & 1, err)) return;
+    if (c >= 1 && !wait_bar(sm, B_M3A, (c - 1) & 1, err)) return;
+    tc::fence_after_sync();
+#pragma unroll
+    for (int hq = 0; hq < 2; ++hq) {
+      float w[32];
+      tc::tmem_ld16(tl + COL_W + hq * 32, w);
+      tc::tmem_ld16(tl + COL_W + hq * 32 + 16, w + 16);
+      tc::wait_ld();
+#pragma unroll
+      for (int q = 0; q < 4; ++q) st_sw128_chunk(sm.base + OFF_W16, t, 4 * hq + q, w + 8 * q);
+    }
+    group_signal(sm, kBarPrep, B_E3);
   }
+}
 
-  if (warp == 0) {
-    tc::tmem_alloc(sm.tmem_slot(), TMEM_COLS);
-    tc::tmem_relinquish();
-  }
-  if (tid == 0) {
-    tc::mbar_init(sm.bar(), 1);
-    tc::fence_mbar_init();
-    *sm.abort_flag() = 0;
-  }
-  tc::fence_before_sync();
-  __syncthreads();
-  tc::fence_after_sync();
-  const uint32_t tmem = *sm.tmem_slot();
-  const uint32_t tl = tmem + ((uint32_t)(warp * 32) << 16);  // this warp's TMEM lane quarter
-  uint32_t phase = 0;
+// ---------------------------------------------------------------- state role
 
-  const uint32_t kq = sm.u32(OFF_KQ), v16 = sm.u32(OFF_V), s16 = sm.u32(OFF_S16), w16 = sm.u32(OFF_W16);
-  const uint32_t u16 = sm.u32(OFF_U16), udd = sm.u32(OFF_UDD), tp = sm.u32(OFF_TP), tpp = sm.u32(OFF_TPP);
-  const uint32_t p16 = sm.u32(OFF_P16);
+template <typename TOut>
+__device__ void state_role(const Smem& sm, const PrefillShape& s, const PrefillArgs& a, uint32_t tmem, int h,
+                           int64_t bos, int64_t eos, int nchunks, size_t state_off) {
+  const int j = threadIdx.x;  // TMEM lane == dv row of S^T
+  const int warp = threadIdx.x >> 5;
+  const uint32_t tl = tmem + ((uint32_t)((warp & 3) * 32) << 16);
+  TOut* op = static_cast<TOut*>(a.o);
+  // outputs of a chunk are staged row-major [64 tokens][128 dv] in the U16/UDD
+  // tiles (free between the chunk's last MMA and the next chunk's U epilogue)
+  TOut* stage = reinterpret_cast<TOut*>(sm.base + OFF_U16);
+  constexpr uint32_t kRowBytes = D * sizeof(TOut);
 
-  // ---- initial state: row j = tid of S^T into TMEM (fp32) and S16 (fp16)
+  // initial state: fp16 TMEM operand = S_0; fp32 TMEM state = gamma_C(0) * S_0
+  if (!wait_bar(sm, B_L0, 0, a.err)) return;
   {
-    const int j = tid;
+    const float gC = sm.vec(0)[V_GAM + C - 1];
     for (int q = 0; q < D / 16; ++q) {
       float v[16];
       if (a.initial_state) {
@@ -298,229 +482,255 @@ gdn_prefill_fused_kernel(const PrefillShape s, const PrefillArgs a) {
 #pragma unroll
         for (int x = 0; x < 16; ++x) v[x] = 0.f;
       }
+      uint32_t hv[8];
+#pragma unroll
+      for (int x = 0; x < 8; ++x) hv[x] = tc::half2_bits(v[2 * x], v[2 * x + 1]);
+      tc::tmem_st8_bits(tl + COL_SH + q * 8, hv);
+#pragma unroll
+      for (int x = 0; x < 16; ++x) v[x] *= gC;
       tc::tmem_st16(tl + COL_S + q * 16, v);
-      uint8_t* tile = sm.base + OFF_S16 + (q >> 2) * S16_HALF;
-      st_sw128_chunk(tile, j, (q & 3) * 2, v);
-      st_sw128_chunk(tile, j, (q & 3) * 2 + 1, v + 8);
     }
     tc::wait_st();
   }
-  publish_to_mma();
-
-  const TOut* dummy = nullptr;
-  (void)dummy;
-  TOut* op = static_cast<TOut*>(a.o);
+  group_signal(sm, kBarState, B_E6A);
 
   for (int c = 0; c < nchunks; ++c) {
+    const int b = c & 1;
+    const float* vec = sm.vec(b);
     const int64_t t0 = bos + (int64_t)c * C;
     const int Lc = (int)((eos - t0) < C ? (eos - t0) : C);
-
-    // P0: inputs of the chunk -> fp16 tiles; cumulative gates
-    load_chunk<TIn>(sm, s, a, h, t0, Lc);
-
-    // P1: [K;Q] K^T -> TMEM D1 (M=128 rows K then Q, N=64, K=dk)
-    if (tid == 0) {
-      tc::fence_after_sync();
-      const uint32_t id = tc::idesc_f16(128, 64, 0, 0);
-#pragma unroll
-      for (int ks = 0; ks < 8; ++ks) {
-        const uint32_t off = (ks >> 2) * KQ_HALF + (ks & 3) * 32;
-        tc::mma_f16(tmem + COL_D1, tc::sw128_desc(kq + off, 16, 1024), tc::sw128_desc(kq + off, 16, 1024), id,
-                    ks > 0);
-      }
-      tc::mma_commit(sm.bar());
+    // E5: U^T -> fp16 tiles (after the previous chunk's output stores read the stage)
+    if (!wait_bar(sm, B_M3A, c & 1, a.err)) return;
+    if (c >= 1) {
+      if (j < 32) tc::bulk_wait_read();
+      tc::named_sync(kBarState, 128);
     }
-    if (!wait_mma(sm, phase, a.err)) break;
-
-    // P2: A (fp32) from the K K^T rows, P (fp16) from the Q K^T rows
-    {
-      float x[64];
+    tc::fence_after_sync();
 #pragma unroll
-      for (int q = 0; q < 4; ++q) tc::tmem_ld16(tl + COL_D1 + q * 16, x + 16 * q);
+    for (int hq = 0; hq < 2; ++hq) {
+      float u[32];
+      tc::tmem_ld16(tl + COL_U + hq * 32, u);
+      tc::tmem_ld16(tl + COL_U + hq * 32 + 16, u + 16);
       tc::wait_ld();
-      const float* G = sm.G();
-      if (tid < C) {
-        const int i = tid;
-        const float Gi = G[i], bi = sm.beta()[i];
-        float* Arow = sm.A() + i * LDA;
-#pragma unroll
-        for (int j = 0; j < C; ++j) Arow[j] = (j < i) ? bi * __expf(Gi - G[j]) * x[j] : 0.f;
-      } else {
-        const int r = tid - C;
-        const float Gr = G[r];
-#pragma unroll
-        for (int cc = 0; cc < 8; ++cc) {
-          float v[8];
-#pragma unroll
-          for (int m = 0; m < 8; ++m) {
-            const int i = cc * 8 + m;
-            v[m] = (i <= r) ? __expf(Gr - G[i]) * x[i] : 0.f;
-          }
-          st_sw128_chunk(sm.base + OFF_P16, r, cc, v);
-        }
-      }
-    }
-    __syncthreads();
-
-    // P3: T = (I + A)^{-1}; T diag(beta gamma) and T diag(beta) as fp16 B operands
-    solve_unit_lower(sm);
-    {
-      const int mat = tid >> 6, i = tid & 63;
-      const float* colscale = mat ? sm.beta() : sm.bg();
-      uint8_t* tile = sm.base + (mat ? OFF_TPP : OFF_TP);
-      const float* Trow = sm.T() + i * LDA;
-#pragma unroll
-      for (int cc = 0; cc < 8; ++cc) {
-        float v[8];
-#pragma unroll
-        for (int m = 0; m < 8; ++m) {
-          const int j = cc * 8 + m;
-          v[m] = (j <= i) ? Trow[j] * colscale[j] : 0.f;
-        }
-        st_sw128_chunk(tile, i, cc, v);
-      }
-    }
-    publish_to_mma();
-
-    // P4: W^T = K^T T'^T and U~^T = V^T T''^T (A MN-major from the token tiles)
-    if (tid == 0) {
-      tc::fence_after_sync();
-      const uint32_t id = tc::idesc_f16(128, 64, 1, 0);
-#pragma unroll
-      for (int ks = 0; ks < 4; ++ks) {
-        tc::mma_f16(tmem + COL_W, tc::sw128_desc(kq + ks * 2048, KQ_HALF, 1024),
-                    tc::sw128_desc(tp + ks * 32, 16, 1024), id, ks > 0);
-      }
-#pragma unroll
-      for (int ks = 0; ks < 4; ++ks) {
-        tc::mma_f16(tmem + COL_U, tc::sw128_desc(v16 + ks * 2048, V_HALF, 1024),
-                    tc::sw128_desc(tpp + ks * 32, 16, 1024), id, ks > 0);
-      }
-      tc::mma_commit(sm.bar());
-    }
-    if (!wait_mma(sm, phase, a.err)) break;
-
-    // P5: W^T -> fp16 MN-major B tile; scale the resident state by gamma_C
-    {
-      const int i = tid;
 #pragma unroll
       for (int q = 0; q < 4; ++q) {
-        float w[16];
-        tc::tmem_ld16(tl + COL_W + q * 16, w);
-        tc::wait_ld();
-        st_sw128_chunk(sm.base + OFF_W16, i, 2 * q, w);
-        st_sw128_chunk(sm.base + OFF_W16, i, 2 * q + 1, w + 8);
-      }
-      const float gC = sm.gam()[C - 1];
+        float ud[8];
 #pragma unroll
-      for (int q = 0; q < D / 16; ++q) {
-        float v[16];
-        tc::tmem_ld16(tl + COL_S + q * 16, v);
-        tc::wait_ld();
-#pragma unroll
-        for (int x = 0; x < 16; ++x) v[x] *= gC;
-        tc::tmem_st16(tl + COL_S + q * 16, v);
+        for (int x = 0; x < 8; ++x) ud[x] = u[8 * q + x] * vec[V_DD + 32 * hq + 8 * q + x];
+        st_sw128_chunk(sm.base + OFF_U16, j, 4 * hq + q, u + 8 * q);
+        st_sw128_chunk(sm.base + OFF_UDD, j, 4 * hq + q, ud);
       }
-      tc::wait_st();
     }
-    publish_to_mma();
+    group_signal(sm, kBarState, B_E5);
+    // E6a: new state -> fp16 operand; rescale by the next chunk's gamma_C; final state
+    if (!wait_bar(sm, B_M4B, c & 1, a.err)) return;
+    tc::fence_after_sync();
+    const bool last = (c == nchunks - 1);
+    float gnext = 1.f;
+    if (!last) {
+      if (!wait_bar(sm, B_L0 + (b ^ 1), ((c + 1) >> 1) & 1, a.err)) return;
+      gnext = sm.vec(b ^ 1)[V_GAM + C - 1];
+    }
+#pragma unroll
+    for (int hq = 0; hq < 4; ++hq) {
+      float v[32];
+      tc::tmem_ld16(tl + COL_S + hq * 32, v);
+      tc::tmem_ld16(tl + COL_S + hq * 32 + 16, v + 16);
+      tc::wait_ld();
+      if (!last) {
+        uint32_t hv[16];
+#pragma unroll
+        for (int x = 0; x < 16; ++x) hv[x] = tc::half2_bits(v[2 * x], v[2 * x + 1]);
+        tc::tmem_st16_bits(tl + COL_SH + hq * 16, hv);
+#pragma unroll
+        for (int x = 0; x < 32; ++x) v[x] *= gnext;
+        tc::tmem_st16(tl + COL_S + hq * 32, v);
+        tc::tmem_st16(tl + COL_S + hq * 32 + 16, v + 16);
+      } else if (a.final_state) {
+        float4* dst = reinterpret_cast<float4*>(a.final_state + state_off + (size_t)j * D + hq * 32);
+#pragma unroll
+        for (int x = 0; x < 8; ++x) dst[x] = make_float4(v[4 * x], v[4 * x + 1], v[4 * x + 2], v[4 * x + 3]);
+      }
+    }
+    tc::wait_st();
+    group_signal(sm, kBarState, B_E6A);
+    // E6b: outputs of the chunk -> staging rows -> bulk stores
+    if (!wait_bar(sm, B_M4A, c & 1, a.err)) return;
+    tc::fence_after_sync();
+    const float sc = a.scale;
+#pragma unroll
+    for (int hq = 0; hq < 2; ++hq) {
+      float o1[32], o2[32];
+#pragma unroll
+      for (int q = 0; q < 2; ++q) {
+        tc::tmem_ld16(tl + COL_O1 + hq * 32 + q * 16, o1 + 16 * q);
+        tc::tmem_ld16(tl + COL_O2 + hq * 32 + q * 16, o2 + 16 * q);
+      }
+      tc::wait_ld();
+#pragma unroll
+      for (int x = 0; x < 32; ++x) {
+        const int r = hq * 32 + x;
+        store_out(stage + r * D + j, sc * fmaf(vec[V_GAM + r], o1[x], o2[x]));
+      }
+    }
+    tc::fence_proxy_async_smem();
+    tc::fence_before_sync();
+    tc::named_sync(kBarState, 128);
+    if (j < 32) {
+      for (int r = j; r < Lc; r += 32)
+        tc::bulk_store(op + ((size_t)(t0 + r) * s.H + h) * D, tc::smem_u32(stage + r * D), kRowBytes);
+      tc::bulk_commit();
+    }
+    if (j == 0) tc::mbar_arrive(sm.bar(B_E6B));
+  }
+  if (j < 32) tc::bulk_wait_all();
+}
 
-    // P6: U^T = U~^T - S^T W^T (accumulate with negated A); O1 = S^T Q^T
-    if (tid == 0) {
+// ---------------------------------------------------------------- mma role
+
+// D1 = [K;Q] K^T for chunk buffer b.
+__device__ __forceinline__ void issue_m1(const Smem& sm, uint32_t tmem, int b) {
+  const uint32_t kq = sm.u32(OFF_KQ + b * KQ_BUF);
+  const uint32_t id = tc::idesc_f16(128, 64, 0, 0);
+#pragma unroll
+  for (int ks = 0; ks < 8; ++ks) {
+    const uint32_t off = (ks >> 2) * KQ_HALF + (ks & 3) * 32;
+    tc::mma_f16(tmem + COL_D1, tc::sw128_desc(kq + off, 16, 1024), tc::sw128_desc(kq + off, 16, 1024), id, ks > 0);
+  }
+  tc::mma_commit(sm.bar(B_M1));
+}
+
+// W^T = K^T T'^T and U~^T = V^T T''^T for chunk buffer b (A MN-major from the token tiles).
+__device__ __forceinline__ void issue_m2(const Smem& sm, uint32_t tmem, int b) {
+  const uint32_t kq = sm.u32(OFF_KQ + b * KQ_BUF), v16 = sm.u32(OFF_V + b * V_BUF);
+  const uint32_t tp = sm.u32(OFF_TP), tpp = sm.u32(OFF_TPP);
+  const uint32_t id = tc::idesc_f16(128, 64, 1, 0);
+#pragma unroll
+  for (int ks = 0; ks < 4; ++ks)
+    tc::mma_f16(tmem + COL_W, tc::sw128_desc(kq + ks * 2048, KQ_HALF, 1024), tc::sw128_desc(tp + ks * 32, 16, 1024),
+                id, ks > 0);
+#pragma unroll
+  for (int ks = 0; ks < 4; ++ks)
+    tc::mma_f16(tmem + COL_U, tc::sw128_desc(v16 + ks * 2048, V_HALF, 1024), tc::sw128_desc(tpp + ks * 32, 16, 1024),
+                id, ks > 0);
+  tc::mma_commit(sm.bar(B_M2));
+}
+
+__device__ void mma_role(const Smem& sm, uint32_t tmem, int nchunks, unsigned int* err) {
+  const uint32_t w16 = sm.u32(OFF_W16), u16 = sm.u32(OFF_U16), udd = sm.u32(OFF_UDD);
+  const uint32_t p16 = sm.u32(OFF_P16);
+  const uint32_t id_u = tc::idesc_f16(128, 64, 0, 1, 1);
+  const uint32_t id_o = tc::idesc_f16(128, 64, 0, 0);
+  const uint32_t id_s = tc::idesc_f16(128, 128, 0, 1);
+
+  if (!wait_bar(sm, B_L0, 0, err)) return;
+  tc::fence_after_sync();
+  issue_m1(sm, tmem, 0);
+  if (!wait_bar(sm, B_E2, 0, err)) return;
+  tc::fence_after_sync();
+  issue_m2(sm, tmem, 0);
+  for (int c = 0; c < nchunks; ++c) {
+    const int b = c & 1;
+    const uint32_t kq = sm.u32(OFF_KQ + b * KQ_BUF);
+    if (c + 1 < nchunks) {
+      if (!wait_bar(sm, B_L0 + (b ^ 1), ((c + 1) >> 1) & 1, err)) return;
       tc::fence_after_sync();
-      const uint32_t idu = tc::idesc_f16(128, 64, 0, 1, 1);
-      const uint32_t ido = tc::idesc_f16(128, 64, 0, 0);
-#pragma unroll
-      for (int ks = 0; ks < 8; ++ks) {
-        const uint64_t ad = tc::sw128_desc(s16 + (ks >> 2) * S16_HALF + (ks & 3) * 32, 16, 1024);
-        tc::mma_f16(tmem + COL_U, ad, tc::sw128_desc(w16 + ks * 2048, 16384, 1024), idu, 1);
-      }
-#pragma unroll
-      for (int ks = 0; ks < 8; ++ks) {
-        const uint64_t ad = tc::sw128_desc(s16 + (ks >> 2) * S16_HALF + (ks & 3) * 32, 16, 1024);
-        const uint64_t bd = tc::sw128_desc(kq + 8 * 1024 + (ks >> 2) * KQ_HALF + (ks & 3) * 32, 16, 1024);
-        tc::mma_f16(tmem + COL_O1, ad, bd, ido, ks > 0);
-      }
-      tc::mma_commit(sm.bar());
+      issue_m1(sm, tmem, b ^ 1);
     }
-    if (!wait_mma(sm, phase, a.err)) break;
-
-    // P7: U^T -> fp16 A tiles (plain and decayed to the chunk end)
-    {
-      const int j = tid;
+    // M3a: U^T -= S^T W^T (A = fp16 state from TMEM)
+    if (!wait_bar(sm, B_E3, c & 1, err)) return;
+    if (!wait_bar(sm, B_E6A, c & 1, err)) return;
+    tc::fence_after_sync();
 #pragma unroll
-      for (int q = 0; q < 4; ++q) {
-        float u[16], ud[16];
-        tc::tmem_ld16(tl + COL_U + q * 16, u);
-        tc::wait_ld();
+    for (int ks = 0; ks < 8; ++ks)
+      tc::mma_f16_ts(tmem + COL_U, tmem + COL_SH + ks * 8, tc::sw128_desc(w16 + ks * 2048, 16384, 1024), id_u, 1);
+    tc::mma_commit(sm.bar(B_M3A));
+    // M3b: O1 = S^T Q^T (after the previous chunk's outputs were read)
+    if (c >= 1 && !wait_bar(sm, B_E6B, (c - 1) & 1, err)) return;
+    tc::fence_after_sync();
 #pragma unroll
-        for (int x = 0; x < 16; ++x) ud[x] = u[x] * sm.dd()[q * 16 + x];
-        st_sw128_chunk(sm.base + OFF_U16, j, 2 * q, u);
-        st_sw128_chunk(sm.base + OFF_U16, j, 2 * q + 1, u + 8);
-        st_sw128_chunk(sm.base + OFF_UDD, j, 2 * q, ud);
-        st_sw128_chunk(sm.base + OFF_UDD, j, 2 * q + 1, ud + 8);
-      }
+    for (int ks = 0; ks < 8; ++ks) {
+      const uint64_t bd = tc::sw128_desc(kq + 8 * 1024 + (ks >> 2) * KQ_HALF + (ks & 3) * 32, 16, 1024);
+      tc::mma_f16_ts(tmem + COL_O1, tmem + COL_SH + ks * 8, bd, id_o, ks > 0);
     }
-    publish_to_mma();
-
-    // P8: O2 = U^T P^T; S^T += (U^T diag(dd)) K
-    if (tid == 0) {
+    // M4b: S^T += (U^T diag(dd)) K ; M4a: O2 = U^T P^T
+    if (!wait_bar(sm, B_E5, c & 1, err)) return;
+    tc::fence_after_sync();
+#pragma unroll
+    for (int ks = 0; ks < 4; ++ks)
+      tc::mma_f16(tmem + COL_S, tc::sw128_desc(udd + ks * 32, 16, 1024),
+                  tc::sw128_desc(kq + ks * 2048, KQ_HALF, 1024), id_s, 1);
+    tc::mma_commit(sm.bar(B_M4B));
+#pragma unroll
+    for (int ks = 0; ks < 4; ++ks)
+      tc::mma_f16(tmem + COL_O2, tc::sw128_desc(u16 + ks * 32, 16, 1024),
+                  tc::sw128_desc(p16 + b * P_BUF + ks * 32, 16, 1024), id_o, ks > 0);
+    tc::mma_commit(sm.bar(B_M4A));
+    // M2 of the next chunk
+    if (c + 1 < nchunks) {
+      if (!wait_bar(sm, B_E2, (c + 1) & 1, err)) return;
       tc::fence_after_sync();
-      const uint32_t ido = tc::idesc_f16(128, 64, 0, 0);
-      const uint32_t ids = tc::idesc_f16(128, 128, 0, 1);
-#pragma unroll
-      for (int ks = 0; ks < 4; ++ks)
-        tc::mma_f16(tmem + COL_O2, tc::sw128_desc(u16 + ks * 32, 16, 1024),
-                    tc::sw128_desc(p16 + ks * 32, 16, 1024), ido, ks > 0);
-#pragma unroll
-      for (int ks = 0; ks < 4; ++ks)
-        tc::mma_f16(tmem + COL_S, tc::sw128_desc(udd + ks * 32, 16, 1024),
-                    tc::sw128_desc(kq + ks * 2048, KQ_HALF, 1024), ids, 1);
-      tc::mma_commit(sm.bar());
+      issue_m2(sm, tmem, b ^ 1);
     }
-    if (!wait_mma(sm, phase, a.err)) break;
+  }
+}
 
-    // P9: outputs of the chunk; new state -> fp16 operand (and fp32 final state)
-    {
-      const int j = tid;
-      const float sc = a.scale;
-#pragma unroll
-      for (int q = 0; q < 4; ++q) {
-        float o1[16], o2[16];
-        tc::tmem_ld16(tl + COL_O1 + q * 16, o1);
-        tc::tmem_ld16(tl + COL_O2 + q * 16, o2);
-        tc::wait_ld();
-#pragma unroll
-        for (int x = 0; x < 16; ++x) {
-          const int r = q * 16 + x;
-          if (r < Lc)
-            store_out(op + ((size_t)(t0 + r) * s.H + h) * D + j, sc * fmaf(sm.gam()[r], o1[x], o2[x]));
-        }
-      }
-      const bool last = (c == nchunks - 1);
-#pragma unroll
-      for (int q = 0; q < D / 16; ++q) {
-        float v[16];
-        tc::tmem_ld16(tl + COL_S + q * 16, v);
-        tc::wait_ld();
-        uint8_t* tile = sm.base + OFF_S16 + (q >> 2) * S16_HALF;
-        st_sw128_chunk(tile, j, (q & 3) * 2, v);
-        st_sw128_chunk(tile, j, (q & 3) * 2 + 1, v + 8);
-        if (last && a.final_state) {
-          float4* dst = reinterpret_cast<float4*>(a.final_state + state_off + (size_t)j * D + q * 16);
-#pragma unroll
-          for (int x = 0; x < 4; ++x) dst[x] = make_float4(v[4 * x], v[4 * x + 1], v[4 * x + 2], v[4 * x + 3]);
-        }
+// ---------------------------------------------------------------- kernel
+
+template <typename TIn, typename TOut>
+__global__ void __launch_bounds__(kThreads, 1)
+gdn_prefill_fused_kernel(const PrefillShape s, const PrefillArgs a) {
+  extern __shared__ uint8_t smem_raw[];
+  Smem sm;
+  sm.base = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
+  const int warp = threadIdx.x >> 5;
+  const int n = blockIdx.x / s.H;
+  const int h = blockIdx.x - n * s.H;
+  int64_t bos, eos;
+  if (!seq_bounds(a.cu_seqlens, n, s.total_T, a.err, &bos, &eos)) return;
+
+  const size_t state_off = ((size_t)n * s.H + h) * (size_t)D * D;
+  const int nchunks = (int)((eos - bos + C - 1) / C);
+  if (nchunks == 0) {  // empty sequence: the state passes through
+    if (a.final_state) {
+      for (int i = threadIdx.x; i < D * D / 4; i += kThreads) {
+        const float4 x = a.initial_state ? reinterpret_cast<const float4*>(a.initial_state + state_off)[i]
+                                         : make_float4(0.f, 0.f, 0.f, 0.f);
+        reinterpret_cast<float4*>(a.final_state + state_off)[i] = x;
       }
     }
-    publish_to_mma();
+    return;
   }
 
-  // teardown: every MMA has completed (each phase waited), TMEM can be released
+  if (warp == kMmaWarp) {
+    tc::tmem_alloc(sm.tmem_slot(), TMEM_COLS);
+    tc::tmem_relinquish();
+  }
+  if (threadIdx.x == 0) {
+    for (int i = 0; i < B_COUNT; ++i) tc::mbar_init(sm.bar(i), 1);
+    *sm.abort_flag() = 0;
+    tc::fence_mbar_init();
+  }
   tc::fence_before_sync();
   __syncthreads();
   tc::fence_after_sync();
-  if (warp == 0) tc::tmem_dealloc(tmem, TMEM_COLS);
+  const uint32_t tmem = *sm.tmem_slot();
+
+  if (warp < kPrepWarp0) {
+    state_role<TOut>(sm, s, a, tmem, h, bos, eos, nchunks, state_off);
+  } else if (warp < kLoadWarp0) {
+    prep_role(sm, tmem, nchunks, a.err);
+  } else if (warp < kMmaWarp) {
+    loader_role<TIn>(sm, s, a, h, bos, eos, nchunks);
+  } else if ((threadIdx.x & 31) == 0) {
+    mma_role(sm, tmem, nchunks, a.err);
+  }
+
+  // teardown: every role finished (all MMAs were waited on by the state role)
+  tc::fence_before_sync();
+  __syncthreads();
+  tc::fence_after_sync();
+  if (warp == kMmaWarp) tc::tmem_dealloc(tmem, TMEM_COLS);
 }
 
 template <typename TIn, typename TOut>
