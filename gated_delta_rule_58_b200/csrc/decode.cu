@@ -2,36 +2,42 @@
 // fp32 state pool, updated in place.
 //
 // Design (B200). The step is HBM-bound: every (slot, head) state of dk x dv fp32
-// is read once and written once. Following the T=1 split-V variant of the
-// FlashInfer PR #7156 page ("Cake GDP kernel: shared-memory reduction and direct
-// register loads", sections 1-2), the state is streamed straight from HBM into
-// registers with 16-byte vector loads (no shared-memory staging), and the value
-// dimension is split across CTAs so that small batches still fill the 148 SMs.
+// is read once and written once. The T=1 split-V variant on the FlashInfer PR
+// #7156 page ("Cake GDP kernel: shared-memory reduction and direct register
+// loads", sections 1-2) streams the state straight into registers; here each
+// state instead moves as ONE bulk TMA copy (cp.async.bulk) into a shared-memory
+// stage and back out with one bulk store, so the bytes in flight per SM no longer
+// depend on how many registers the math needs:
 //
-// Mapping. State rows are K-last rows S^T[j, :] (one value column j of S, dk
-// contiguous fp32). A group of LPR lanes shares one row: lane `sub` holds the
-// float4 chunks sub, sub+LPR, sub+2*LPR, ... so that each warp-wide load covers
-// LPR*16 contiguous bytes of 32/LPR rows. Each thread owns R rows.
+//   persistent grid, one CTA per SM, items = (batch row, head) pairs
+//   producer warp : per item, slot id, gates and betas (scalar loads), then bulk
+//                   copies of the state (64 KiB at dk = 128) and of the item's
+//                   k, q, v rows into a free stage (2-3 stages), tracked by an
+//                   mbarrier's transaction count
+//   consumer warps: two threads per state row load its halves from shared
+//                   memory into registers, do the arithmetic below, write the
+//                   row back, and one thread bulk-stores the stage to the pool
 //
-// Arithmetic. Per row j the step is M = T*n_h sub-steps (gate on the first
-// sub-step of each token, then a Householder update) and T outputs. Writing the
-// row after sub-step m as s_m = Gamma_m s_0 + sum_{l<=m} c_l k_l, every quantity
-// the recurrence needs is a dot product of the OLD row s_0 with a key or a query
-// plus per-head Gram entries:
+// Arithmetic. Per row j (value column j of S, stored K-last as S^T[j, :]) the
+// step is M = T*n_h sub-steps (gate on the first sub-step of each token, then a
+// Householder update) and T outputs. Writing the row after sub-step m as
+// s_m = Gamma_m s_0 + sum_{l<=m} c_l k_l, every quantity the recurrence needs is
+// a dot product of the OLD row s_0 with a key or a query plus per-head Gram
+// entries:
 //     u_m   = k_m . (gated s) = Gamma_m (k_m . s_0) + sum_{l<m} c_l (k_m . k_l)
 //     c_m   = beta_m (v_m[j] - u_m)
 //     o_t   = scale (Gamma (q_t . s_0) + sum_{l<=m_t} c_l (q_t . k_l))
 //     s_new = Gamma_M s_0 + sum_m c_m k_m
-// so one pass of FMAs over the resident row, one shuffle reduction of all M + T
-// dot products, a scalar recurrence of O(M^2) per row, and one pass of FMAs for
-// the update. For T = n_h = 1 this is u = k.s, c = beta (v - alpha u),
-// s' = alpha s + c k, o = scale (alpha q.s + c q.k).
+// so one pass over the resident row for all dot products, one partner shuffle,
+// an O(M^2) scalar recurrence and one pass for the update. For T = n_h = 1 this
+// is u = k.s, c = beta (v - alpha u), s' = alpha s + c k, o = scale (alpha q.s + c q.k).
 #include "common.cuh"
+#include "tcgen05.cuh"
 
 namespace gdn {
 namespace {
 
-constexpr int kDecodeThreads = 128;
+constexpr uint64_t kDecodeWaitNs = 2000000000ull;
 
 struct DecodeParams {
   const void* q;
@@ -43,241 +49,325 @@ struct DecodeParams {
   const int32_t* slot_ids;
   void* o;
   unsigned int* err;
-  int B, H, dv, num_slots;
-  int row_blocks;  // CTAs per (b, h)
+  int B, H, num_slots;
+  int n_items;
   float scale;
 };
 
+// Stage layout for one item (all offsets 16-byte aligned):
+//   [state DK x DK fp32][keys M x DK][queries TT x DK][values M x DK][header]
+// header: slot (int), alpha[TT], beta[M], gram[M][M], qk[TT][M] (fp32)
+template <int DK, int TT, int NH, typename TIn>
+struct StageLayout {
+  static constexpr int M = TT * NH;
+  static constexpr uint32_t kState = DK * DK * 4;
+  static constexpr uint32_t kRow = DK * sizeof(TIn);
+  static constexpr uint32_t kKeys = kState;
+  static constexpr uint32_t kQueries = kKeys + M * kRow;
+  static constexpr uint32_t kValues = kQueries + TT * kRow;
+  static constexpr uint32_t kHeader = kValues + M * kRow;
+  static constexpr uint32_t kAlpha = kHeader + 16;
+  static constexpr uint32_t kBeta = kAlpha + 4 * TT;
+  static constexpr uint32_t kGram = kBeta + 4 * M;
+  static constexpr uint32_t kQK = kGram + 4 * M * M;
+  static constexpr uint32_t kBytes = ((kQK + 4 * TT * M) + 127) / 128 * 128;
+  static constexpr uint32_t kVecBytes = (2 * M + TT) * kRow;
+  // keys and queries as fp32 (one buffer shared by all stages); T = n_h = 1 reads
+  // the raw vectors instead and needs none
+  static constexpr uint32_t kVecF32 = (M > 1) ? (M + TT) * DK * 4 : 0;
+  static constexpr int kStages = (3 * kBytes + kVecF32 <= 215 * 1024) ? 3 : 2;
+  static constexpr uint32_t kSmem = kStages * kBytes + kVecF32 + 64 + 128;  // + barriers + alignment
+};
+
 template <typename TIn>
-__device__ __forceinline__ float ld_in(const TIn* p) { return to_f32(*p); }
+__device__ __forceinline__ void load4_f32(const uint8_t* p, float* out);
+template <>
+__device__ __forceinline__ void load4_f32<__nv_bfloat16>(const uint8_t* p, float* out) {
+  const uint2 raw = *reinterpret_cast<const uint2*>(p);
+  const float2 a = __bfloat1622float2(*reinterpret_cast<const __nv_bfloat162*>(&raw.x));
+  const float2 b = __bfloat1622float2(*reinterpret_cast<const __nv_bfloat162*>(&raw.y));
+  out[0] = a.x; out[1] = a.y; out[2] = b.x; out[3] = b.y;
+}
+template <>
+__device__ __forceinline__ void load4_f32<float>(const uint8_t* p, float* out) {
+  const float4 f = *reinterpret_cast<const float4*>(p);
+  out[0] = f.x; out[1] = f.y; out[2] = f.z; out[3] = f.w;
+}
 
-// DK: head key dim; LPR: lanes per row; R: rows per thread; TT tokens, NH keys per token.
-template <int DK, int LPR, int R, int TT, int NH, typename TIn, typename TOut>
-__global__ void __launch_bounds__(kDecodeThreads, (TT * NH + TT > 2) ? 3 : 4)
+template <int DK, int TT, int NH, typename TIn, typename TOut>
+__global__ void __launch_bounds__(2 * DK + 32, 1)
 gdn_decode_kernel(const DecodeParams p) {
-  constexpr int M = TT * NH;            // sub-steps
-  constexpr int NV = M + TT;            // vectors dotted with the old row: keys then queries
-  constexpr int CPL = DK / (4 * LPR);   // float4 chunks per lane per row
-  constexpr int SLOTS = 32 / LPR;       // row slots per warp
-  constexpr int WARPS = kDecodeThreads / 32;
-  constexpr int RPC = WARPS * SLOTS * R;  // rows per CTA
-  static_assert(CPL >= 1 && DK % (4 * LPR) == 0, "bad DK/LPR");
+  using L = StageLayout<DK, TT, NH, TIn>;
+  constexpr int M = L::M;
+  constexpr int NV = M + TT;                 // vectors dotted with the old row: keys then queries
+  constexpr int NS = L::kStages;
+  constexpr int kConsumers = 2 * DK;         // two threads per state row
+  constexpr int CPH = DK / 8;                // float4 chunks per half row
+  constexpr uint32_t kBarConsumers = 1;
 
-  __shared__ __align__(16) float s_vec[NV][DK];   // k_1..k_M, q_1..q_T (fp32)
-  __shared__ float s_vals[M][RPC];                // v_m[j] for this CTA's rows
-  __shared__ float s_gram[M][M];                  // k_m . k_l
-  __shared__ float s_qk[TT][M];                   // q_t . k_l
-  __shared__ float s_beta[M];
-  __shared__ float s_alpha[TT];
+  extern __shared__ uint8_t smem_raw[];
+  uint8_t* base = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 127) & ~uintptr_t(127));
+  float* vecf = reinterpret_cast<float*>(base + NS * L::kBytes);  // [NV][DK] fp32 of the current item
+  uint64_t* full = reinterpret_cast<uint64_t*>(base + NS * L::kBytes + L::kVecF32);
+  uint64_t* empty = full + NS;
 
   const int tid = threadIdx.x;
-  const int lane = tid & 31;
-  const int warp = tid >> 5;
-  const int sub = lane % LPR;
-  const int slot_in_warp = lane / LPR;
+  if (tid == 0) {
+    for (int s = 0; s < NS; ++s) {
+      tc::mbar_init(&full[s], 1);
+      tc::mbar_init(&empty[s], 1);
+    }
+    tc::fence_mbar_init();
+  }
+  __syncthreads();
 
-  const int bh = blockIdx.x / p.row_blocks;
-  const int rb = blockIdx.x - bh * p.row_blocks;
-  const int b = bh / p.H;
-  const int h = bh - b * p.H;
-  const int row0 = rb * RPC;
-
-  const TIn* qp = static_cast<const TIn*>(p.q);
-  const TIn* kp = static_cast<const TIn*>(p.k);
-  const TIn* vp = static_cast<const TIn*>(p.v);
-  TOut* op = static_cast<TOut*>(p.o);
-
-  const int slot = __ldg(p.slot_ids + b);
-  if (slot < 0 || slot >= p.num_slots) {
-    if (slot >= p.num_slots && tid == 0 && rb == 0) raise_device_error(p.err, GDN_DEVERR_SLOT_OUT_OF_RANGE);
-    for (int i = tid; i < TT * RPC; i += kDecodeThreads) {
-      const int t = i / RPC, j = row0 + (i - t * RPC);
-      if (j < p.dv) store_out(op + (((size_t)b * TT + t) * p.H + h) * p.dv + j, 0.f);
+  if (tid >= kConsumers) {
+    // ---------------- producer (one thread)
+    if (tid != kConsumers) return;
+    const TIn* kp = static_cast<const TIn*>(p.k);
+    const TIn* qp = static_cast<const TIn*>(p.q);
+    const TIn* vp = static_cast<const TIn*>(p.v);
+    int it = 0;
+    for (int item = blockIdx.x; item < p.n_items; item += gridDim.x, ++it) {
+      const int s = it % NS;
+      if (it >= NS && !tc::mbar_wait(&empty[s], ((it / NS) & 1) ^ 1, kDecodeWaitNs)) {
+        raise_device_error(p.err, GDN_DEVERR_TIMEOUT);
+        return;
+      }
+      uint8_t* st = base + s * L::kBytes;
+      const int b = item / p.H, h = item - (item / p.H) * p.H;
+      int slot = __ldg(p.slot_ids + b);
+      if (slot >= p.num_slots) {
+        raise_device_error(p.err, GDN_DEVERR_SLOT_OUT_OF_RANGE);
+        slot = -1;
+      }
+      if (slot < 0) slot = -1;
+      *reinterpret_cast<int*>(st + L::kHeader) = slot;
+#pragma unroll
+      for (int t = 0; t < TT; ++t)
+        reinterpret_cast<float*>(st + L::kAlpha)[t] = expf(__ldg(p.g + ((size_t)b * TT + t) * p.H + h));
+#pragma unroll
+      for (int m = 0; m < M; ++m) {
+        const int t = m / NH, mm = m - t * NH;
+        reinterpret_cast<float*>(st + L::kBeta)[m] = __ldg(p.beta + (((size_t)b * TT + t) * p.H + h) * NH + mm);
+      }
+      if (slot < 0) {
+        tc::mbar_arrive(&full[s]);
+        continue;
+      }
+      tc::mbar_arrive_expect_tx(&full[s], L::kState + L::kVecBytes);
+      const uint32_t sst = tc::smem_u32(st);
+      tc::bulk_load(sst, p.pool + ((size_t)slot * p.H + h) * (size_t)DK * DK, L::kState, &full[s]);
+#pragma unroll
+      for (int t = 0; t < TT; ++t) {
+        const size_t bth = ((size_t)b * TT + t) * p.H + h;
+        tc::bulk_load(sst + L::kKeys + t * NH * L::kRow, kp + bth * NH * DK, NH * L::kRow, &full[s]);
+        tc::bulk_load(sst + L::kQueries + t * L::kRow, qp + bth * DK, L::kRow, &full[s]);
+        tc::bulk_load(sst + L::kValues + t * NH * L::kRow, vp + bth * NH * DK, NH * L::kRow, &full[s]);
+      }
     }
     return;
   }
 
-  // 1) Stream this thread's state rows HBM -> registers first, so the loads are
-  //    in flight while the per-head vectors are staged and the Gram is built.
-  float* state = p.pool + ((size_t)slot * p.H + h) * (size_t)p.dv * DK;
-  int rows[R];
-  bool live[R];  // rows past dv (small dv, last row block) are computed on zeros, never stored
-  float4 s[R][CPL];
+  // ---------------- consumers: thread -> (row, half)
+  const int lane = tid & 31, warp = tid >> 5;
+  const int row = warp * 16 + (lane & 15);
+  const int half = lane >> 4;
+  TOut* op = static_cast<TOut*>(p.o);
+  int it = 0;
+  int prev_stage = -1;
+  for (int item = blockIdx.x; item < p.n_items; item += gridDim.x, ++it) {
+    const int s = it % NS;
+    uint8_t* st = base + s * L::kBytes;
+    if (!tc::mbar_wait(&full[s], (it / NS) & 1, kDecodeWaitNs)) {
+      if (tid == 0) raise_device_error(p.err, GDN_DEVERR_TIMEOUT);
+      break;
+    }
+    const int b = item / p.H, h = item - (item / p.H) * p.H;
+    const int slot = *reinterpret_cast<const int*>(st + L::kHeader);
+    const float* alpha = reinterpret_cast<const float*>(st + L::kAlpha);
+    const float* betas = reinterpret_cast<const float*>(st + L::kBeta);
+    float* gram = reinterpret_cast<float*>(st + L::kGram);
+    float* qk = reinterpret_cast<float*>(st + L::kQK);
+    if (slot >= 0 && M == 1) {
+      // T = n_h = 1: k.s, q.s and the Gram entry q.k in one pass over the half row
+      float* srow = reinterpret_cast<float*>(st) + (size_t)row * DK + half * (DK / 2);
+      float4 sv[CPH];
 #pragma unroll
-  for (int r = 0; r < R; ++r) {
-    rows[r] = row0 + (warp * R + r) * SLOTS + slot_in_warp;
-    live[r] = rows[r] < p.dv;
-    const float4* src = reinterpret_cast<const float4*>(state + (size_t)rows[r] * DK);
+      for (int c = 0; c < CPH; ++c) sv[c] = reinterpret_cast<const float4*>(srow)[(c + row) & (CPH - 1)];
+      float ks = 0.f, qs = 0.f, qkv = 0.f;
 #pragma unroll
-    for (int c = 0; c < CPL; ++c)
-      s[r][c] = live[r] ? __ldcs(src + c * LPR + sub) : make_float4(0.f, 0.f, 0.f, 0.f);
-  }
+      for (int c = 0; c < CPH; ++c) {
+        const int e = half * (DK / 2) + 4 * ((c + row) & (CPH - 1));
+        float wk[4], wq[4];
+        load4_f32<TIn>(st + L::kKeys + e * sizeof(TIn), wk);
+        load4_f32<TIn>(st + L::kQueries + e * sizeof(TIn), wq);
+        ks = fmaf(sv[c].x, wk[0], fmaf(sv[c].y, wk[1], fmaf(sv[c].z, wk[2], fmaf(sv[c].w, wk[3], ks))));
+        qs = fmaf(sv[c].x, wq[0], fmaf(sv[c].y, wq[1], fmaf(sv[c].z, wq[2], fmaf(sv[c].w, wq[3], qs))));
+        qkv = fmaf(wq[0], wk[0], fmaf(wq[1], wk[1], fmaf(wq[2], wk[2], fmaf(wq[3], wk[3], qkv))));
+      }
+      ks += __shfl_xor_sync(0xffffffffu, ks, 16);
+      qs += __shfl_xor_sync(0xffffffffu, qs, 16);
+      qkv += __shfl_xor_sync(0xffffffffu, qkv, 16);
+      const float a = alpha[0];
+      const float vj = to_f32(reinterpret_cast<const TIn*>(st + L::kValues)[row]);
+      const float cm = betas[0] * (vj - a * ks);
+      if (half == 0) store_out(op + ((size_t)b * p.H + h) * DK + row, p.scale * fmaf(cm, qkv, a * qs));
+#pragma unroll
+      for (int c = 0; c < CPH; ++c) {
+        const int e = half * (DK / 2) + 4 * ((c + row) & (CPH - 1));
+        float wk[4];
+        load4_f32<TIn>(st + L::kKeys + e * sizeof(TIn), wk);
+        float4 x = sv[c];
+        x.x = fmaf(cm, wk[0], a * x.x);
+        x.y = fmaf(cm, wk[1], a * x.y);
+        x.z = fmaf(cm, wk[2], a * x.z);
+        x.w = fmaf(cm, wk[3], a * x.w);
+        reinterpret_cast<float4*>(srow)[(c + row) & (CPH - 1)] = x;
+      }
+    } else if (slot >= 0) {
+      // keys and queries of the item -> fp32 once (every FMA below reads them)
+      for (int e = tid * 4; e < NV * DK; e += kConsumers * 4)
+        load4_f32<TIn>(st + L::kKeys + e * sizeof(TIn), vecf + e);
+      tc::named_sync(kBarConsumers, kConsumers);
+      // per-head Gram entries k_m.k_l (l < m) and q_t.k_l, one warp per pair
+      constexpr int kPairsKK = M * (M - 1) / 2;
+      constexpr int kPairs = kPairsKK + TT * M;
+      for (int pair = warp; pair < kPairs; pair += kConsumers / 32) {
+        int va, vb;
+        if (pair < kPairsKK) {
+          va = 1;
+          int rem = pair;
+          while (rem >= va) { rem -= va; ++va; }
+          vb = rem;
+        } else {
+          const int x = pair - kPairsKK;
+          va = M + x / M;
+          vb = x - (x / M) * M;
+        }
+        const float* pa = vecf + va * DK;  // the queries follow the keys
+        const float* pb = vecf + vb * DK;
+        float acc = 0.f;
+        for (int e = lane * 4; e < DK; e += 128) {
+          const float4 xa = *reinterpret_cast<const float4*>(pa + e);
+          const float4 xb = *reinterpret_cast<const float4*>(pb + e);
+          acc = fmaf(xa.x, xb.x, fmaf(xa.y, xb.y, fmaf(xa.z, xb.z, fmaf(xa.w, xb.w, acc))));
+        }
+#pragma unroll
+        for (int off = 16; off > 0; off >>= 1) acc += __shfl_xor_sync(0xffffffffu, acc, off);
+        if (lane == 0) {
+          if (pair < kPairsKK) gram[va * M + vb] = acc;
+          else qk[(va - M) * M + vb] = acc;
+        }
+      }
+      tc::named_sync(kBarConsumers, kConsumers);
 
-  // 2) Stage keys and queries of this (b, h) as fp32, the values of this CTA's
-  //    rows, beta and the gates.
-  {
-    constexpr int kChunks = NV * DK / 8;
-    for (int i = tid; i < kChunks; i += kDecodeThreads) {
-      const int vec = i / (DK / 8);
-      const int e = (i - vec * (DK / 8)) * 8;
-      const TIn* src;
-      if (vec < M) {
-        const int t = vec / NH, m = vec - t * NH;
-        src = kp + ((((size_t)b * TT + t) * p.H + h) * NH + m) * DK + e;
-      } else {
-        const int t = vec - M;
-        src = qp + (((size_t)b * TT + t) * p.H + h) * DK + e;
-      }
-      float tmp[8];
-      load8_f32(src, tmp);
+      // my half row: its chunks are visited in rotated order (c + row) so that eight
+      // consecutive rows hit eight different shared-memory bank groups
+      float* srow = reinterpret_cast<float*>(st) + (size_t)row * DK + half * (DK / 2);
+      float4 sv[CPH];
 #pragma unroll
-      for (int x = 0; x < 8; ++x) s_vec[vec][e + x] = tmp[x];
-    }
-    for (int i = tid; i < M * RPC; i += kDecodeThreads) {
-      const int m = i / RPC, jj = i - m * RPC;
-      const int t = m / NH, mm = m - t * NH;
-      s_vals[m][jj] = (row0 + jj < p.dv)
-          ? ld_in(vp + ((((size_t)b * TT + t) * p.H + h) * NH + mm) * p.dv + row0 + jj)
-          : 0.f;
-    }
-    if (tid < M) {
-      const int t = tid / NH, mm = tid - t * NH;
-      s_beta[tid] = __ldg(p.beta + (((size_t)b * TT + t) * p.H + h) * NH + mm);
-    }
-    if (tid >= 32 && tid < 32 + TT) {
-      const int t = tid - 32;
-      s_alpha[t] = expf(__ldg(p.g + ((size_t)b * TT + t) * p.H + h));
-    }
-  }
-  __syncthreads();
+      for (int c = 0; c < CPH; ++c) sv[c] = reinterpret_cast<const float4*>(srow)[(c + row) & (CPH - 1)];
+      float dots[NV];
+#pragma unroll
+      for (int vec = 0; vec < NV; ++vec) dots[vec] = 0.f;
+#pragma unroll
+      for (int c = 0; c < CPH; ++c) {
+        const int e = half * (DK / 2) + 4 * ((c + row) & (CPH - 1));
+#pragma unroll
+        for (int vec = 0; vec < NV; ++vec) {
+          const float4 w = *reinterpret_cast<const float4*>(vecf + vec * DK + e);
+          float a = dots[vec];
+          a = fmaf(sv[c].x, w.x, a);
+          a = fmaf(sv[c].y, w.y, a);
+          a = fmaf(sv[c].z, w.z, a);
+          a = fmaf(sv[c].w, w.w, a);
+          dots[vec] = a;
+        }
+      }
+#pragma unroll
+      for (int vec = 0; vec < NV; ++vec) dots[vec] += __shfl_xor_sync(0xffffffffu, dots[vec], 16);
 
-  // 3) Per-head Gram entries k_m.k_l (l < m) and q_t.k_l, one warp per pair.
-  {
-    constexpr int kPairsKK = M * (M - 1) / 2;
-    constexpr int kPairs = kPairsKK + TT * M;
-    for (int pair = warp; pair < kPairs; pair += WARPS) {
-      int a, c;
-      if (pair < kPairsKK) {
-        a = 1;
-        int rem = pair;
-        while (rem >= a) { rem -= a; ++a; }
-        c = rem;  // (a, c) with c < a
-      } else {
-        const int x = pair - kPairsKK;
-        a = M + x / M;  // query index into s_vec
-        c = x - (x / M) * M;
+      // scalar recurrence for this row (both halves, redundantly)
+      float coef[M];
+      float G = 1.f;
+#pragma unroll
+      for (int t = 0; t < TT; ++t) {
+        const float a = alpha[t];
+        G *= a;
+#pragma unroll
+        for (int l = 0; l < t * NH; ++l) coef[l] *= a;
+#pragma unroll
+        for (int x = 0; x < NH; ++x) {
+          const int m = t * NH + x;
+          float u = G * dots[m];
+#pragma unroll
+          for (int l = 0; l < m; ++l) u = fmaf(coef[l], gram[m * M + l], u);
+          const float vj = to_f32(reinterpret_cast<const TIn*>(st + L::kValues + m * L::kRow)[row]);
+          coef[m] = betas[m] * (vj - u);
+        }
+        float out = G * dots[M + t];
+#pragma unroll
+        for (int l = 0; l < (t + 1) * NH; ++l) out = fmaf(coef[l], qk[t * M + l], out);
+        if (half == 0) store_out(op + (((size_t)b * TT + t) * p.H + h) * DK + row, p.scale * out);
       }
-      float acc = 0.f;
-      for (int e = lane; e < DK; e += 32) acc = fmaf(s_vec[a][e], s_vec[c][e], acc);
+      // s_new = Gamma s_0 + sum_m c_m k_m, written back in place (same rotated chunks)
 #pragma unroll
-      for (int off = 16; off > 0; off >>= 1) acc += __shfl_xor_sync(0xffffffffu, acc, off);
-      if (lane == 0) {
-        if (pair < kPairsKK) s_gram[a][c] = acc;
-        else s_qk[a - M][c] = acc;
+      for (int c = 0; c < CPH; ++c) {
+        const int e = half * (DK / 2) + 4 * ((c + row) & (CPH - 1));
+        float4 x = sv[c];
+        x.x *= G; x.y *= G; x.z *= G; x.w *= G;
+#pragma unroll
+        for (int m = 0; m < M; ++m) {
+          const float4 w = *reinterpret_cast<const float4*>(vecf + m * DK + e);
+          x.x = fmaf(coef[m], w.x, x.x);
+          x.y = fmaf(coef[m], w.y, x.y);
+          x.z = fmaf(coef[m], w.z, x.z);
+          x.w = fmaf(coef[m], w.w, x.w);
+        }
+        reinterpret_cast<float4*>(srow)[(c + row) & (CPH - 1)] = x;
       }
+    } else {
+      // skipped row of the batch: o = 0, pool untouched
+#pragma unroll
+      for (int t = 0; t < TT; ++t)
+        if (half == 0) store_out(op + (((size_t)b * TT + t) * p.H + h) * DK + row, 0.f);
     }
-  }
-  __syncthreads();
-
-  // 4) Dot products of the old rows with every key and query.
-  float dots[NV][R];
-#pragma unroll
-  for (int vec = 0; vec < NV; ++vec)
-#pragma unroll
-    for (int r = 0; r < R; ++r) dots[vec][r] = 0.f;
-#pragma unroll
-  for (int c = 0; c < CPL; ++c) {
-#pragma unroll
-    for (int vec = 0; vec < NV; ++vec) {
-      const float4 w = *reinterpret_cast<const float4*>(&s_vec[vec][(c * LPR + sub) * 4]);
-#pragma unroll
-      for (int r = 0; r < R; ++r) {
-        float a = dots[vec][r];
-        a = fmaf(s[r][c].x, w.x, a);
-        a = fmaf(s[r][c].y, w.y, a);
-        a = fmaf(s[r][c].z, w.z, a);
-        a = fmaf(s[r][c].w, w.w, a);
-        dots[vec][r] = a;
-      }
+    // stage -> pool (one bulk store); the previous item's stage is handed back to
+    // the producer once its store has finished reading shared memory
+    tc::fence_proxy_async_smem();
+    tc::named_sync(kBarConsumers, kConsumers);
+    if (tid == 0) {
+      if (slot >= 0)
+        tc::bulk_store(p.pool + ((size_t)slot * p.H + h) * (size_t)DK * DK, tc::smem_u32(st), L::kState);
+      tc::bulk_commit();
+      tc::bulk_wait_read_1();
+      if (prev_stage >= 0) tc::mbar_arrive(&empty[prev_stage]);
     }
+    prev_stage = s;
   }
-#pragma unroll
-  for (int off = 1; off < LPR; off <<= 1)
-#pragma unroll
-    for (int vec = 0; vec < NV; ++vec)
-#pragma unroll
-      for (int r = 0; r < R; ++r) dots[vec][r] += __shfl_xor_sync(0xffffffffu, dots[vec][r], off);
-
-  // 5) Scalar recurrence per row (every lane of the row group, redundantly).
-  float coef[R][M];
-  float gam[R];
-#pragma unroll
-  for (int r = 0; r < R; ++r) {
-    const int jj = rows[r] - row0;
-    float G = 1.f;
-#pragma unroll
-    for (int t = 0; t < TT; ++t) {
-      const float a = s_alpha[t];
-      G *= a;
-#pragma unroll
-      for (int l = 0; l < t * NH; ++l) coef[r][l] *= a;
-#pragma unroll
-      for (int x = 0; x < NH; ++x) {
-        const int m = t * NH + x;
-        float u = G * dots[m][r];
-#pragma unroll
-        for (int l = 0; l < m; ++l) u = fmaf(coef[r][l], s_gram[m][l], u);
-        coef[r][m] = s_beta[m] * (s_vals[m][jj] - u);
-      }
-      float out = G * dots[M + t][r];
-#pragma unroll
-      for (int l = 0; l < (t + 1) * NH; ++l) out = fmaf(coef[r][l], s_qk[t][l], out);
-      if (live[r] && sub == (t % LPR))
-        store_out(op + (((size_t)b * TT + t) * p.H + h) * p.dv + rows[r], p.scale * out);
-    }
-    gam[r] = G;
-  }
-
-  // 6) s_new = Gamma s_0 + sum_m c_m k_m, written back in place.
-#pragma unroll
-  for (int c = 0; c < CPL; ++c) {
-#pragma unroll
-    for (int r = 0; r < R; ++r) {
-      s[r][c].x *= gam[r];
-      s[r][c].y *= gam[r];
-      s[r][c].z *= gam[r];
-      s[r][c].w *= gam[r];
-    }
-#pragma unroll
-    for (int m = 0; m < M; ++m) {
-      const float4 w = *reinterpret_cast<const float4*>(&s_vec[m][(c * LPR + sub) * 4]);
-#pragma unroll
-      for (int r = 0; r < R; ++r) {
-        s[r][c].x = fmaf(coef[r][m], w.x, s[r][c].x);
-        s[r][c].y = fmaf(coef[r][m], w.y, s[r][c].y);
-        s[r][c].z = fmaf(coef[r][m], w.z, s[r][c].z);
-        s[r][c].w = fmaf(coef[r][m], w.w, s[r][c].w);
-      }
-    }
-  }
-#pragma unroll
-  for (int r = 0; r < R; ++r) {
-    if (!live[r]) continue;
-    float4* dst = reinterpret_cast<float4*>(state + (size_t)rows[r] * DK);
-#pragma unroll
-    for (int c = 0; c < CPL; ++c) __stcs(dst + c * LPR + sub, s[r][c]);
-  }
+  if (tid == 0) tc::bulk_wait_all();
 }
 
 template <int DK, int TT, int NH, typename TIn, typename TOut>
 gdn_status_t launch_typed(DecodeParams p, cudaStream_t stream) {
-  constexpr int LPR = 4;
-  constexpr int R = (TT * NH + TT > 2) ? 1 : 2;  // 32 or 64 state floats per thread
-  constexpr int RPC = (kDecodeThreads / 32) * (32 / LPR) * R;
-  p.row_blocks = (p.dv + RPC - 1) / RPC;
-  const long long grid = (long long)p.B * p.H * p.row_blocks;
-  if (grid == 0) return ok();
-  gdn_decode_kernel<DK, LPR, R, TT, NH, TIn, TOut><<<(unsigned)grid, kDecodeThreads, 0, stream>>>(p);
+  using L = StageLayout<DK, TT, NH, TIn>;
+  static int sm_count = 0;
+  static bool configured = false;
+  if (!configured) {
+    int dev = 0;
+    cudaError_t e = cudaGetDevice(&dev);
+    if (e == cudaSuccess) e = cudaDeviceGetAttribute(&sm_count, cudaDevAttrMultiProcessorCount, dev);
+    if (e == cudaSuccess)
+      e = cudaFuncSetAttribute(gdn_decode_kernel<DK, TT, NH, TIn, TOut>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                               L::kSmem);
+    if (e != cudaSuccess) return fail(GDN_ERR_CUDA, std::string("gdn_decode: setup: ") + cudaGetErrorString(e));
+    configured = true;
+  }
+  p.n_items = p.B * p.H;
+  if (p.n_items == 0) return ok();
+  const int grid = p.n_items < sm_count ? p.n_items : sm_count;
+  gdn_decode_kernel<DK, TT, NH, TIn, TOut><<<grid, 2 * DK + 32, L::kSmem, stream>>>(p);
   return check_launch("gdn_decode");
 }
 
@@ -292,8 +382,7 @@ gdn_status_t launch_dtypes(DecodeParams p, gdn_dtype_t in, gdn_dtype_t out, cuda
 }
 
 template <int DK>
-gdn_status_t launch_steps(DecodeParams p, int T, int nh, gdn_dtype_t in, gdn_dtype_t out,
-                          cudaStream_t s) {
+gdn_status_t launch_steps(DecodeParams p, int T, int nh, gdn_dtype_t in, gdn_dtype_t out, cudaStream_t s) {
 #define GDN_DECODE_CASE(TT_, NH_) \
   if (T == TT_ && nh == NH_) return launch_dtypes<DK, TT_, NH_>(p, in, out, s);
   GDN_DECODE_CASE(1, 1)
@@ -317,7 +406,8 @@ gdn_status_t decode_launch(const void* q, const void* k, const void* v, const fl
                            const float* beta, float* pool, int num_slots, const int32_t* slot_ids,
                            void* o, int B, int T, int H, int dk, int dv, int nh, float scale,
                            gdn_dtype_t in, gdn_dtype_t out, unsigned int* err, cudaStream_t stream) {
-  DecodeParams p{q, k, v, g, beta, pool, slot_ids, o, err, B, H, dv, num_slots, 0, scale};
+  (void)dv;
+  DecodeParams p{q, k, v, g, beta, pool, slot_ids, o, err, B, H, num_slots, 0, scale};
   switch (dk) {
     case 32: return launch_steps<32>(p, T, nh, in, out, stream);
     case 64: return launch_steps<64>(p, T, nh, in, out, stream);
