@@ -14,9 +14,10 @@
 //                   copies of the state (64 KiB at dk = 128) and of the item's
 //                   k, q, v rows into a free stage (2-3 stages), tracked by an
 //                   mbarrier's transaction count
-//   consumer warps: two threads per state row load its halves from shared
-//                   memory into registers, do the arithmetic below, write the
-//                   row back, and one thread bulk-stores the stage to the pool
+//   consumer warps: two (single token) or four (multi-token) threads per state
+//                   row load its parts from shared memory into registers, do the
+//                   arithmetic below, write the row back, and one thread
+//                   bulk-stores the stage to the pool
 //
 // Arithmetic. Per row j (value column j of S, stored K-last as S^T[j, :]) the
 // step is M = T*n_h sub-steps (gate on the first sub-step of each token, then a
@@ -94,15 +95,23 @@ __device__ __forceinline__ void load4_f32<float>(const uint8_t* p, float* out) {
   out[0] = f.x; out[1] = f.y; out[2] = f.z; out[3] = f.w;
 }
 
+// Threads per state row (2 or 4; the consumer mapping below supports both).
+// Measured on B200, 4 threads per row gained nothing for the multi-token product
+// (its 96-register cap spills), so both step shapes use 2.
+template <int TT, int NH>
+__host__ __device__ constexpr int threads_per_row() { return 2; }
+
 template <int DK, int TT, int NH, typename TIn, typename TOut>
-__global__ void __launch_bounds__(2 * DK + 32, 1)
+__global__ void __launch_bounds__(threads_per_row<TT, NH>() * DK + 32, 1)
 gdn_decode_kernel(const DecodeParams p) {
   using L = StageLayout<DK, TT, NH, TIn>;
   constexpr int M = L::M;
   constexpr int NV = M + TT;                 // vectors dotted with the old row: keys then queries
   constexpr int NS = L::kStages;
-  constexpr int kConsumers = 2 * DK;         // two threads per state row
-  constexpr int CPH = DK / 8;                // float4 chunks per half row
+  constexpr int TPR = threads_per_row<TT, NH>();
+  constexpr int kConsumers = TPR * DK;
+  constexpr int CPH = DK / (4 * TPR);        // float4 chunks per thread's part of a row
+  constexpr int RPW = 32 / TPR;              // rows per warp
   constexpr uint32_t kBarConsumers = 1;
 
   extern __shared__ uint8_t smem_raw[];
@@ -169,10 +178,11 @@ gdn_decode_kernel(const DecodeParams p) {
     return;
   }
 
-  // ---------------- consumers: thread -> (row, half)
+  // ---------------- consumers: thread -> (row, part); the parts of a row are lanes
+  // that differ in their top bits, so partial sums combine with xor shuffles
   const int lane = tid & 31, warp = tid >> 5;
-  const int row = warp * 16 + (lane & 15);
-  const int half = lane >> 4;
+  const int row = warp * RPW + (lane & (RPW - 1));
+  const int half = lane / RPW;  // which part of the row (0..TPR-1)
   TOut* op = static_cast<TOut*>(p.o);
   int it = 0;
   int prev_stage = -1;
@@ -191,14 +201,14 @@ gdn_decode_kernel(const DecodeParams p) {
     float* qk = reinterpret_cast<float*>(st + L::kQK);
     if (slot >= 0 && M == 1) {
       // T = n_h = 1: k.s, q.s and the Gram entry q.k in one pass over the half row
-      float* srow = reinterpret_cast<float*>(st) + (size_t)row * DK + half * (DK / 2);
+      float* srow = reinterpret_cast<float*>(st) + (size_t)row * DK + half * (DK / TPR);
       float4 sv[CPH];
 #pragma unroll
       for (int c = 0; c < CPH; ++c) sv[c] = reinterpret_cast<const float4*>(srow)[(c + row) & (CPH - 1)];
       float ks = 0.f, qs = 0.f, qkv = 0.f;
 #pragma unroll
       for (int c = 0; c < CPH; ++c) {
-        const int e = half * (DK / 2) + 4 * ((c + row) & (CPH - 1));
+        const int e = half * (DK / TPR) + 4 * ((c + row) & (CPH - 1));
         float wk[4], wq[4];
         load4_f32<TIn>(st + L::kKeys + e * sizeof(TIn), wk);
         load4_f32<TIn>(st + L::kQueries + e * sizeof(TIn), wq);
@@ -215,7 +225,7 @@ gdn_decode_kernel(const DecodeParams p) {
       if (half == 0) store_out(op + ((size_t)b * p.H + h) * DK + row, p.scale * fmaf(cm, qkv, a * qs));
 #pragma unroll
       for (int c = 0; c < CPH; ++c) {
-        const int e = half * (DK / 2) + 4 * ((c + row) & (CPH - 1));
+        const int e = half * (DK / TPR) + 4 * ((c + row) & (CPH - 1));
         float wk[4];
         load4_f32<TIn>(st + L::kKeys + e * sizeof(TIn), wk);
         float4 x = sv[c];
@@ -233,7 +243,7 @@ gdn_decode_kernel(const DecodeParams p) {
       // per-head Gram entries k_m.k_l (l < m) and q_t.k_l, one warp per pair
       constexpr int kPairsKK = M * (M - 1) / 2;
       constexpr int kPairs = kPairsKK + TT * M;
-      for (int pair = warp; pair < kPairs; pair += kConsumers / 32) {
+      for (int pair = warp; pair < kPairs; pair += kConsumers / 32) {  // one warp per pair
         int va, vb;
         if (pair < kPairsKK) {
           va = 1;
@@ -262,9 +272,9 @@ gdn_decode_kernel(const DecodeParams p) {
       }
       tc::named_sync(kBarConsumers, kConsumers);
 
-      // my half row: its chunks are visited in rotated order (c + row) so that eight
-      // consecutive rows hit eight different shared-memory bank groups
-      float* srow = reinterpret_cast<float*>(st) + (size_t)row * DK + half * (DK / 2);
+      // my part of the row: its chunks are visited in rotated order (c + row) so
+      // that eight consecutive rows hit eight different shared-memory bank groups
+      float* srow = reinterpret_cast<float*>(st) + (size_t)row * DK + half * (DK / TPR);
       float4 sv[CPH];
 #pragma unroll
       for (int c = 0; c < CPH; ++c) sv[c] = reinterpret_cast<const float4*>(srow)[(c + row) & (CPH - 1)];
@@ -273,7 +283,7 @@ gdn_decode_kernel(const DecodeParams p) {
       for (int vec = 0; vec < NV; ++vec) dots[vec] = 0.f;
 #pragma unroll
       for (int c = 0; c < CPH; ++c) {
-        const int e = half * (DK / 2) + 4 * ((c + row) & (CPH - 1));
+        const int e = half * (DK / TPR) + 4 * ((c + row) & (CPH - 1));
 #pragma unroll
         for (int vec = 0; vec < NV; ++vec) {
           const float4 w = *reinterpret_cast<const float4*>(vecf + vec * DK + e);
@@ -286,7 +296,9 @@ gdn_decode_kernel(const DecodeParams p) {
         }
       }
 #pragma unroll
-      for (int vec = 0; vec < NV; ++vec) dots[vec] += __shfl_xor_sync(0xffffffffu, dots[vec], 16);
+      for (int off = RPW; off < 32; off <<= 1)
+#pragma unroll
+        for (int vec = 0; vec < NV; ++vec) dots[vec] += __shfl_xor_sync(0xffffffffu, dots[vec], off);
 
       // scalar recurrence for this row (both halves, redundantly)
       float coef[M];
@@ -314,7 +326,7 @@ gdn_decode_kernel(const DecodeParams p) {
       // s_new = Gamma s_0 + sum_m c_m k_m, written back in place (same rotated chunks)
 #pragma unroll
       for (int c = 0; c < CPH; ++c) {
-        const int e = half * (DK / 2) + 4 * ((c + row) & (CPH - 1));
+        const int e = half * (DK / TPR) + 4 * ((c + row) & (CPH - 1));
         float4 x = sv[c];
         x.x *= G; x.y *= G; x.z *= G; x.w *= G;
 #pragma unroll
@@ -367,7 +379,8 @@ gdn_status_t launch_typed(DecodeParams p, cudaStream_t stream) {
   p.n_items = p.B * p.H;
   if (p.n_items == 0) return ok();
   const int grid = p.n_items < sm_count ? p.n_items : sm_count;
-  gdn_decode_kernel<DK, TT, NH, TIn, TOut><<<grid, 2 * DK + 32, L::kSmem, stream>>>(p);
+  gdn_decode_kernel<DK, TT, NH, TIn, TOut>
+      <<<grid, threads_per_row<TT, NH>() * DK + 32, L::kSmem, stream>>>(p);
   return check_launch("gdn_decode");
 }
 

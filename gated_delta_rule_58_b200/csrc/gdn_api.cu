@@ -177,7 +177,7 @@ gdn_status_t gdn_chunk_prefill(const void* q, const void* k, const void* v, cons
   st = gdn::device_error_word(&err);
   if (st != GDN_OK) return st;
   gdn::PrefillArgs a{q, k, v, g, beta, cu_seqlens, initial_state, final_state, o, scale,
-                     in_dtype, out_dtype, workspace, err};
+                     in_dtype, out_dtype, workspace, err, gdn::kPrefillOutputs};
   return gdn::prefill_launch(s, a, resolved, gdn::as_stream(stream));
 }
 

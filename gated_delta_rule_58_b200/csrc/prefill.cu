@@ -5,9 +5,8 @@
 
 namespace gdn {
 
-// Set once the transfer (chunk-parallel fixup) algorithm is built; until then AUTO
-// takes the fused path for every tensor-core shape.
-constexpr bool kTransferPrefillBuilt = false;
+// AUTO may pick the transfer (chunk-parallel fixup) algorithm.
+constexpr bool kTransferPrefillBuilt = true;
 
 gdn_prefill_algo_t prefill_auto_tensor_core(const PrefillShape& s) {
   if (!kTransferPrefillBuilt) return GDN_PREFILL_FUSED;

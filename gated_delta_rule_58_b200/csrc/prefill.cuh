@@ -25,7 +25,16 @@ struct PrefillArgs {
   gdn_dtype_t in_dtype, out_dtype;
   void* workspace;
   unsigned int* err;
+  // Fused-kernel mode. kPrefillOutputs: the normal prefill. kPrefillLocalState:
+  // zero initial state, no outputs (final state = the local state H of each
+  // sequence). kPrefillTransfer: identity initial state, values taken as zero, no
+  // outputs (final state = the transfer matrix M^T of each sequence, K-last).
+  int mode;
 };
+
+constexpr int kPrefillOutputs = 0;
+constexpr int kPrefillLocalState = 1;
+constexpr int kPrefillTransfer = 2;
 
 // Validates the shape for `requested` and resolves GDN_PREFILL_AUTO.
 gdn_status_t prefill_resolve(const PrefillShape& s, gdn_dtype_t in, gdn_prefill_algo_t requested,

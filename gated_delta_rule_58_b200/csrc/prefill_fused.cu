@@ -156,6 +156,7 @@ template <typename TIn>
 __device__ void loader_role(const Smem& sm, const PrefillShape& s, const PrefillArgs& a, int h, int64_t bos,
                             int64_t eos, int nchunks) {
   const int t = threadIdx.x - kLoadWarp0 * 32;  // 0..127
+  const bool zero_values = (a.mode == kPrefillTransfer);  // transfer run: V taken as 0
   for (int c = 0; c < nchunks; ++c) {
     const int b = c & 1;
     // chunk c-2 (same buffers) fully consumed: its outputs were read, so every
@@ -176,11 +177,12 @@ __device__ void loader_role(const Smem& sm, const PrefillShape& s, const Prefill
         uint8_t* tile = base + (ch >> 3) * half;
         const uint32_t off = tc::sw128_offset(row + roff, ch & 7, 1024);
         const TIn* src = src0 + ((size_t)(t0 + (row < Lc ? row : 0)) * s.H + h) * D + ch * 8;
+        const bool live = row < Lc && !(mat == 2 && zero_values);
         if constexpr (std::is_same<TIn, __nv_bfloat16>::value) {
-          tc::cp_async16(tc::smem_u32(tile + off), src, row < Lc ? 16u : 0u);
+          tc::cp_async16(tc::smem_u32(tile + off), src, live ? 16u : 0u);
         } else {
           float v8[8];
-          if (row < Lc) {
+          if (live) {
             load8_f32(src, v8);
           } else {
 #pragma unroll
@@ -471,7 +473,10 @@ __device__ void state_role(const Smem& sm, const PrefillShape& s, const PrefillA
     const float gC = sm.vec(0)[V_GAM + C - 1];
     for (int q = 0; q < D / 16; ++q) {
       float v[16];
-      if (a.initial_state) {
+      if (a.mode == kPrefillTransfer) {  // S_0 = I: row j of S^T is e_j
+#pragma unroll
+        for (int x = 0; x < 16; ++x) v[x] = (q * 16 + x == j) ? 1.f : 0.f;
+      } else if (a.initial_state) {
         const float4* src = reinterpret_cast<const float4*>(a.initial_state + state_off + (size_t)j * D + q * 16);
 #pragma unroll
         for (int x = 0; x < 4; ++x) {
@@ -554,9 +559,16 @@ __device__ void state_role(const Smem& sm, const PrefillShape& s, const PrefillA
     }
     tc::wait_st();
     group_signal(sm, kBarState, B_E6A);
-    // E6b: outputs of the chunk -> staging rows -> bulk stores
+    // E6b: outputs of the chunk -> staging rows -> bulk stores (skipped when the
+    // run produces states only)
     if (!wait_bar(sm, B_M4A, c & 1, a.err)) return;
     tc::fence_after_sync();
+    if (op == nullptr) {
+      tc::fence_before_sync();
+      tc::named_sync(kBarState, 128);
+      if (j == 0) tc::mbar_arrive(sm.bar(B_E6B));
+      continue;
+    }
     const float sc = a.scale;
 #pragma unroll
     for (int hq = 0; hq < 2; ++hq) {
@@ -694,8 +706,12 @@ gdn_prefill_fused_kernel(const PrefillShape s, const PrefillArgs a) {
   if (nchunks == 0) {  // empty sequence: the state passes through
     if (a.final_state) {
       for (int i = threadIdx.x; i < D * D / 4; i += kThreads) {
-        const float4 x = a.initial_state ? reinterpret_cast<const float4*>(a.initial_state + state_off)[i]
-                                         : make_float4(0.f, 0.f, 0.f, 0.f);
+        float4 x = a.initial_state ? reinterpret_cast<const float4*>(a.initial_state + state_off)[i]
+                                   : make_float4(0.f, 0.f, 0.f, 0.f);
+        if (a.mode == kPrefillTransfer) {  // identity (row r of the K-last layout is e_r)
+          const int r = (4 * i) / D, c0 = (4 * i) % D;
+          x = make_float4(c0 == r, c0 + 1 == r, c0 + 2 == r, c0 + 3 == r);
+        }
         reinterpret_cast<float4*>(a.final_state + state_off)[i] = x;
       }
     }

@@ -167,3 +167,49 @@ def test_fused_varlen32_h32_sampled():
     rng = np.random.default_rng(0)
     pairs = [(longest, 0), (shortest, 31)] + [(int(rng.integers(32)), int(rng.integers(32))) for _ in range(4)]
     _sampled_pairs_check(inp, FUSED, pairs)
+
+
+# ---------------------------------------------------------------- transfer (chunk-parallel fixup) path
+
+TRANSFER = gdn.GDN_PREFILL_TRANSFER
+
+
+@pytest.mark.parametrize("g_range", [(0.01, 0.5), (0.0, 0.01), (0.0, 0.0)])
+def test_transfer_varlen_edges(g_range):
+    lens = [1, 0, 63, 64, 65, 130, 200, 7]
+    inp = inputs.prefill_inputs(lens, 3, 128, 128, seed=31, g_range=g_range)
+    check(inp, TRANSFER, what=f"transfer {g_range}")
+
+
+def test_transfer_no_initial_state_and_alias():
+    inp = inputs.prefill_inputs([129, 0, 64], 2, 128, 128, seed=32, with_initial_state=False)
+    check(inp, TRANSFER, what="transfer no init")
+    inp2 = inputs.prefill_inputs([400, 64], 2, 128, 128, seed=33, g_range=(0.0, 0.02))
+    check(inp2, TRANSFER, what="transfer alias", alias=True)
+
+
+def test_transfer_multi_chunk_segments_weak_decay():
+    """20000 tokens x 8 heads: segments of several chunks (G > 1) and a long fixup chain."""
+    inp = inputs.prefill_inputs([20000], 8, 128, 128, seed=34, g_range=(0.0, 0.02))
+    check(inp, TRANSFER, what="transfer long weak decay")
+
+
+def test_transfer_matches_fused():
+    inp = inputs.prefill_inputs([3000, 500, 1], 4, 128, 128, seed=35, g_range=(0.0, 0.05))
+    o_f, f_f = run_prefill(inp, FUSED)
+    o_t, f_t = run_prefill(inp, TRANSFER)
+    assert_close(o_t, o_f, what="transfer vs fused o")
+    assert_close(f_t, f_f, what="transfer vs fused state")
+
+
+def test_transfer_b1_t65536_h4_full_size():
+    """Low-parallelism prefill at the benchmark size (B=1 x 65536, H=4), every head."""
+    inp = inputs.longseq_b1_t65536_h4()
+    check(inp, TRANSFER, what="B1 T65536 H4", out_dtype=torch.bfloat16)
+
+
+def test_auto_picks_transfer_for_long_low_parallelism():
+    ws = gdn.gdn_chunk_prefill_workspace_size
+    assert ws(1, 65536, 4, 128, 128, 64, gdn.GDN_PREFILL_AUTO) == \
+        ws(1, 65536, 4, 128, 128, 64, gdn.GDN_PREFILL_TRANSFER) > 0
+    assert ws(4, 32768, 16, 128, 128, 64, gdn.GDN_PREFILL_AUTO) == 0
