@@ -51,17 +51,23 @@ def load_peaks():
 
 
 def dist_setup():
+    """One process per GPU under torchrun (env RANK/LOCAL_RANK/WORLD_SIZE/MASTER_*).
+    NCCL on GPUs; gloo when CUDA is absent (the CPU-only reference arm and tests)."""
     ws = int(os.environ.get("WORLD_SIZE", "1"))
     rank = int(os.environ.get("RANK", "0"))
     local = int(os.environ.get("LOCAL_RANK", "0"))
+    cuda = torch.cuda.is_available()
     if ws > 1:
         import datetime
         import torch.distributed as dist
         os.environ.setdefault("MASTER_ADDR", "127.0.0.1")
-        torch.cuda.set_device(local)
-        dist.init_process_group("nccl", timeout=datetime.timedelta(seconds=120),
-                                device_id=torch.device("cuda", local))
-    else:
+        timeout = datetime.timedelta(seconds=120)
+        if cuda:
+            torch.cuda.set_device(local)
+            dist.init_process_group("nccl", timeout=timeout, device_id=torch.device("cuda", local))
+        else:
+            dist.init_process_group("gloo", timeout=timeout)
+    elif cuda:
         torch.cuda.set_device(0)
     return ws, rank, local
 
@@ -76,7 +82,8 @@ def max_over_ranks(x: float, ws: int) -> float:
     if ws == 1:
         return x
     import torch.distributed as dist
-    t = torch.tensor([x], dtype=torch.float64, device="cuda")
+    dev = "cuda" if dist.get_backend() == "nccl" else "cpu"
+    t = torch.tensor([x], dtype=torch.float64, device=dev)
     dist.all_reduce(t, op=dist.ReduceOp.MAX)
     return float(t.item())
 
@@ -381,54 +388,80 @@ def bench_prefill(key, steps, warmup, ws, rank, peaks, algo=None):
 
 # ---------------------------------------------------------------- CPU oracle (baseline / reference arm)
 
+class OracleDecode:
+    """The fp64 CPU oracle on a decode workload, timed on the host cores. A sample is
+    the first `rows` batch rows of one full step (all heads), so its cost is bounded."""
+
+    def __init__(self, key, seed=0):
+        import oracle
+        from gated_delta_rule_58_b200 import inputs
+        self.oracle = oracle
+        self.c = DECODE_CFGS[key]
+        c = self.c
+        inp = inputs.decode_inputs(c["B"], c["T"], c["H"], c["d"], c["d"], c["nh"], c["slots"], seed=seed)
+        self.args = [oracle.f64(x) for x in (inp.q, inp.k, inp.v, inp.g, inp.beta)]
+        self.pool = oracle.f64(inp.pool)
+        self.slots = inp.slot_ids
+        self.scale = inp.scale
+        self.threads = 0
+
+    def step(self, rows):
+        """One oracle call on `rows` batch rows; returns its wall time in seconds."""
+        sub = [a[:rows] for a in self.args]
+        t0 = time.perf_counter()
+        _, self.pool, self.threads = self.oracle.decode(*sub, self.pool, self.slots[:rows], scale=self.scale,
+                                                        copy_pool=False)
+        return time.perf_counter() - t0
+
+    def state_bytes(self, rows):
+        c = self.c
+        return 2 * rows * c["H"] * c["d"] * c["d"] * 4
+
+    def rows_for(self, seconds):
+        """Batch rows whose oracle step takes about `seconds` (at least one row)."""
+        B = self.c["B"]
+        t_full = self.step(B)
+        return B if t_full <= seconds else max(1, int(B * seconds / t_full))
+
+
 def oracle_decode_rate(key, budget_s=10.0, seed=0):
-    """Times the fp64 oracle on the decode workload (full batch) for ~budget_s;
-    returns state GB/s-equivalent, threads used and the sample description."""
-    import oracle
-    from gated_delta_rule_58_b200 import inputs
-    c = DECODE_CFGS[key]
-    inp = inputs.decode_inputs(c["B"], c["T"], c["H"], c["d"], c["d"], c["nh"], c["slots"], seed=seed)
-    args = [oracle.f64(x) for x in (inp.q, inp.k, inp.v, inp.g, inp.beta)]
-    pool = oracle.f64(inp.pool)
-    state_b, _ = decode_bytes(c)
-    n = 0
-    t0 = time.perf_counter()
-    threads = 0
-    while True:
-        _, pool, threads = oracle.decode(*args, pool, inp.slot_ids, scale=inp.scale, copy_pool=False)
+    """cpu_baseline: the oracle on the decode workload for about budget_s; returns
+    state GB/s-equivalent, threads used and the sample description."""
+    od = OracleDecode(key, seed)
+    rows = od.rows_for(budget_s / 10)
+    n, dt = 0, 0.0
+    while dt < budget_s:
+        dt += od.step(rows)
         n += 1
-        if time.perf_counter() - t0 >= budget_s:
-            break
-    dt = time.perf_counter() - t0
-    return state_b * n / dt / 1e9, threads, f"{n} full decode steps ({c['name']}) in {dt:.1f} s"
+    return (od.state_bytes(rows) * n / dt / 1e9, od.threads,
+            f"{n} oracle steps of {rows} of {od.c['B']} batch rows x {od.c['H']} heads ({od.c['name']}), "
+            f"{dt:.1f} s")
 
 
 def run_reference(args, ws, rank):
-    """The reference arm: the fp64 CPU oracle on the headline workload."""
+    """The reference arm: the fp64 CPU oracle on the headline workload, on rank 0 only.
+    Each step is a bounded sample (the first rows of the batch, all heads), sized so the
+    whole run takes about --reference-seconds (two minutes) whatever --steps/--warmup are."""
     if rank != 0:
         return
     steps, warmup = args.steps, args.warmup
-    budget = max(1.0, min(20.0, 120.0 / max(steps + warmup, 1)))
+    od = OracleDecode("decode")
+    per_step = args.reference_seconds / (steps + warmup)
+    rows = od.rows_for(per_step)
     for _ in range(warmup):
-        oracle_decode_rate("decode", budget_s=0.1)
-    rates = []
-    threads = 0
-    sample = ""
-    t0 = time.perf_counter()
-    for _ in range(steps):
-        r, threads, sample = oracle_decode_rate("decode", budget_s=budget)
-        rates.append(r)
-    elapsed = time.perf_counter() - t0
-    value = statistics.fmean(rates)
-    c = DECODE_CFGS["decode"]
-    state_b, _ = decode_bytes(c)
+        od.step(rows)
+    t = sum(od.step(rows) for _ in range(steps))
+    value = od.state_bytes(rows) * steps / t / 1e9
+    c = od.c
+    sample = (f"each step: the oracle on {rows} of {c['B']} batch rows x {c['H']} heads of one decode "
+              f"step; {steps} timed steps in {t:.3f} s")
     line = {
-        "impl": "reference", "metric": METRIC, "value": value, "unit": "GB/s", "n_gpus": 1,
-        "steps": steps, "warmup": warmup, "ms_per_step": state_b / (value * 1e9) * 1e3,
+        "impl": "reference", "metric": METRIC, "value": value, "unit": "GB/s", "n_gpus": ws,
+        "steps": steps, "warmup": warmup, "ms_per_step": t / steps * 1e3,
         "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "f64",
         "data": "synthetic", "config": {"workload": c["name"], "l2": "n/a (CPU)"},
-        "cpu_baseline": {"value": value, "unit": "GB/s", "cores": threads, "kind": "oracle",
-                         "sample": f"per step: {sample}; total {elapsed:.1f} s"},
+        "cpu_baseline": {"value": value, "unit": "GB/s", "cores": od.threads, "kind": "oracle",
+                         "sample": sample},
         "e2e": {"value": value, "unit": "GB/s", "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0},
     }
     print(json.dumps(line), flush=True)
@@ -446,6 +479,8 @@ def main():
                     help="comma list of extra workloads to measure (empty for none)")
     ap.add_argument("--part-steps", type=int, default=5)
     ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--reference-seconds", type=float, default=120.0,
+                    help="wall-time budget of the --impl reference run")
     ap.add_argument("--prefill-algo", default=None, help="force fused|transfer|sequential for the parts")
     args = ap.parse_args()
     if args.warmup < 3:
