@@ -72,6 +72,9 @@ def lib() -> ctypes.CDLL:
             L.gdn_chunk_prefill.restype = i32
             L.gdn_chunk_prefill.argtypes = [vp, vp, vp, vp, vp, vp, i32, i64, vp, vp, vp, i32, i32, i32,
                                             i32, f32, i32, i32, i32, vp, sz, vp]
+            L.gdn_chunk_prefill_static_scratch.restype = i32
+            L.gdn_chunk_prefill_static_scratch.argtypes = [vp, vp, vp, vp, vp, vp, i32, i64, vp, vp, vp, i32,
+                                                           i32, i32, i32, f32, i32, i32, vp]
             L.gdn_last_error.restype = ctypes.c_char_p
             L.gdn_last_error.argtypes = []
             L.gdn_get_device_error.restype = i32
@@ -173,5 +176,23 @@ def gdn_chunk_prefill(q, k, v, g, beta, cu_seqlens, o, initial_state=None, final
                                  total_T, _ptr(initial_state), _ptr(final_state), _ptr(o), H, dk, dv,
                                  chunk, float(scale), _dtype_code(q), _dtype_code(o), algo, ws_ptr,
                                  ws_bytes, _stream_ptr(stream, q.device))
+    _check(st)
+    return o
+
+
+def gdn_chunk_prefill_static_scratch(q, k, v, g, beta, cu_seqlens, o, initial_state=None, final_state=None,
+                                     chunk=64, scale=None, stream=None):
+    """Transfer prefill whose scratch is the library's own 32 MiB device array, for
+    callers that cannot allocate device memory at call time (see include/gdn.h).
+    Same shapes as gdn_chunk_prefill; nothing is allocated, here or in the library."""
+    total_T, H, dk = q.shape
+    dv = v.shape[-1]
+    N = cu_seqlens.numel() - 1
+    if scale is None:
+        scale = dk ** -0.5
+    st = lib().gdn_chunk_prefill_static_scratch(
+        _ptr(q), _ptr(k), _ptr(v), _ptr(g), _ptr(beta), _ptr(cu_seqlens), N, total_T, _ptr(initial_state),
+        _ptr(final_state), _ptr(o), H, dk, dv, chunk, float(scale), _dtype_code(q), _dtype_code(o),
+        _stream_ptr(stream, q.device))
     _check(st)
     return o

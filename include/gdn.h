@@ -151,6 +151,32 @@ gdn_status_t gdn_chunk_prefill(const void* q, const void* k, const void* v, cons
                                gdn_prefill_algo_t algo, void* workspace, size_t workspace_bytes,
                                void* stream);
 
+/*
+ * gdn_chunk_prefill_static_scratch — gdn_chunk_prefill with GDN_PREFILL_TRANSFER,
+ * for callers that cannot allocate device memory when they call (a plugin whose
+ * host framework owns every device allocation, a serving engine that has
+ * reserved the whole device for its own pool, a loop that may not block on the
+ * allocator). It allocates nothing: the transfer algorithm's scratch lives in a
+ * 32 MiB array the library places in device memory, held on every GPU that loads
+ * the library until the process exits. The pages have no counterpart of this
+ * entry point; it is an addition of this library.
+ *
+ * Arguments, layouts and numerics are those of gdn_chunk_prefill (no workspace
+ * arguments). A shape whose transfer workspace
+ * (gdn_chunk_prefill_workspace_size(..., GDN_PREFILL_TRANSFER)) exceeds 32 MiB is
+ * rejected with GDN_ERR_WORKSPACE before anything is launched. All calls on a
+ * device share the one scratch array, which keeps the previous call's contents
+ * (nothing in it needs clearing); calls that overlap on the GPU race on it and
+ * must be serialised by the caller. The first call on each device looks up the
+ * array's device address; make it before any stream capture.
+ */
+gdn_status_t gdn_chunk_prefill_static_scratch(const void* q, const void* k, const void* v, const float* g,
+                                              const float* beta, const int32_t* cu_seqlens, int N,
+                                              int64_t total_T, const float* initial_state,
+                                              float* final_state, void* o, int H, int dk, int dv,
+                                              int chunk, float scale, gdn_dtype_t in_dtype,
+                                              gdn_dtype_t out_dtype, void* stream);
+
 /* Message for the last non-OK status returned on this host thread ("" if none). */
 const char* gdn_last_error(void);
 
