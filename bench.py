@@ -476,7 +476,7 @@ def main():
     ap.add_argument("--warmup", type=int, default=20)
     ap.add_argument("--impl", default="ours", choices=["ours", "reference"])
     ap.add_argument("--parts", default="gdp,prefill,varlen,longseq,tiny",
-                    help="comma list of extra workloads to measure (empty for none)")
+                    help="comma list of extra workloads to measure ('none' for none)")
     ap.add_argument("--part-steps", type=int, default=5)
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--reference-seconds", type=float, default=120.0,
@@ -502,13 +502,15 @@ def main():
     gpu_index = vis_list[local] if local < len(vis_list) else str(local)
 
     with ClockSampler(gpu_index) as clk:
-        head = bench_decode("decode", args.steps, args.warmup, ws, rank, peaks)
+        with torch.cuda.nvtx.range("decode"):  # NVTX ranges let ncu select one workload
+            head = bench_decode("decode", args.steps, args.warmup, ws, rank, peaks)
         parts = []
         algo = None
         if args.prefill_algo:
             algo = {"fused": gdn.GDN_PREFILL_FUSED, "transfer": gdn.GDN_PREFILL_TRANSFER,
                     "sequential": gdn.GDN_PREFILL_SEQUENTIAL}[args.prefill_algo]
-        for key in [p for p in args.parts.split(",") if p]:
+        for key in [p for p in args.parts.split(",") if p and p != "none"]:
+            torch.cuda.nvtx.range_push(key)
             try:
                 if key == "gdp":
                     r = bench_decode("gdp", max(args.part_steps * 20, 20), args.warmup, ws, rank, peaks,
@@ -520,6 +522,7 @@ def main():
                 r["key"] = key
             except Exception as e:  # a part that is not supported is reported, not fatal
                 r = {"key": key, "error": f"{type(e).__name__}: {e}"}
+            torch.cuda.nvtx.range_pop()
             parts.append(r)
 
     if ws > 1:

@@ -32,8 +32,11 @@
 // so one pass over the resident row for all dot products, one partner shuffle,
 // an O(M^2) scalar recurrence and one pass for the update. For T = n_h = 1 this
 // is u = k.s, c = beta (v - alpha u), s' = alpha s + c k, o = scale (alpha q.s + c q.k).
+#include <cstring>
+
 #include "common.cuh"
 #include "tcgen05.cuh"
+#include "tensor_map.cuh"
 
 namespace gdn {
 namespace {
@@ -58,9 +61,18 @@ struct DecodeParams {
 // Stage layout for one item (all offsets 16-byte aligned):
 //   [state DK x DK fp32][keys M x DK][queries TT x DK][values M x DK][header]
 // header: slot (int), alpha[TT], beta[M], gram[M][M], qk[TT][M] (fp32)
+//
+// Single-token steps copy the state linearly (row j of S^T at j * DK * 4). Multi-
+// token steps load and store it as DK/32 tiles of [DK rows][32 fp32] through a
+// tensor map with the 128-byte swizzle: tile x holds columns 32x..32x+31, row j
+// at j * 128 bytes, its 16-byte chunk c at ((c ^ (j & 7)) * 16). Eight consecutive
+// rows then read one chunk index from eight different bank groups while every
+// thread of a warp reads the same key / query chunk (a broadcast).
 template <int DK, int TT, int NH, typename TIn>
 struct StageLayout {
   static constexpr int M = TT * NH;
+  static constexpr bool kSwizzled = M > 1;
+  static constexpr uint32_t kAlign = kSwizzled ? 1024 : 128;  // the swizzle follows address bits 4-9
   static constexpr uint32_t kState = DK * DK * 4;
   static constexpr uint32_t kRow = DK * sizeof(TIn);
   static constexpr uint32_t kKeys = kState;
@@ -71,13 +83,13 @@ struct StageLayout {
   static constexpr uint32_t kBeta = kAlpha + 4 * TT;
   static constexpr uint32_t kGram = kBeta + 4 * M;
   static constexpr uint32_t kQK = kGram + 4 * M * M;
-  static constexpr uint32_t kBytes = ((kQK + 4 * TT * M) + 127) / 128 * 128;
+  static constexpr uint32_t kBytes = ((kQK + 4 * TT * M) + kAlign - 1) / kAlign * kAlign;
   static constexpr uint32_t kVecBytes = (2 * M + TT) * kRow;
   // keys and queries as fp32 (one buffer shared by all stages); T = n_h = 1 reads
   // the raw vectors instead and needs none
   static constexpr uint32_t kVecF32 = (M > 1) ? (M + TT) * DK * 4 : 0;
-  static constexpr int kStages = (3 * kBytes + kVecF32 <= 215 * 1024) ? 3 : 2;
-  static constexpr uint32_t kSmem = kStages * kBytes + kVecF32 + 64 + 128;  // + barriers + alignment
+  static constexpr int kStages = (3 * kBytes + kVecF32 + 64 + kAlign <= 226 * 1024) ? 3 : 2;
+  static constexpr uint32_t kSmem = kStages * kBytes + kVecF32 + 64 + kAlign;  // + barriers + alignment
 };
 
 template <typename TIn>
@@ -103,7 +115,7 @@ __host__ __device__ constexpr int threads_per_row() { return 2; }
 
 template <int DK, int TT, int NH, typename TIn, typename TOut>
 __global__ void __launch_bounds__(threads_per_row<TT, NH>() * DK + 32, 1)
-gdn_decode_kernel(const DecodeParams p) {
+gdn_decode_kernel(const DecodeParams p, const __grid_constant__ CUtensorMap pool_map) {
   using L = StageLayout<DK, TT, NH, TIn>;
   constexpr int M = L::M;
   constexpr int NV = M + TT;                 // vectors dotted with the old row: keys then queries
@@ -115,7 +127,8 @@ gdn_decode_kernel(const DecodeParams p) {
   constexpr uint32_t kBarConsumers = 1;
 
   extern __shared__ uint8_t smem_raw[];
-  uint8_t* base = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 127) & ~uintptr_t(127));
+  uint8_t* base = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + L::kAlign - 1) &
+                                             ~uintptr_t(L::kAlign - 1));
   float* vecf = reinterpret_cast<float*>(base + NS * L::kBytes);  // [NV][DK] fp32 of the current item
   uint64_t* full = reinterpret_cast<uint64_t*>(base + NS * L::kBytes + L::kVecF32);
   uint64_t* empty = full + NS;
@@ -166,7 +179,12 @@ gdn_decode_kernel(const DecodeParams p) {
       }
       tc::mbar_arrive_expect_tx(&full[s], L::kState + L::kVecBytes);
       const uint32_t sst = tc::smem_u32(st);
-      tc::bulk_load(sst, p.pool + ((size_t)slot * p.H + h) * (size_t)DK * DK, L::kState, &full[s]);
+      if constexpr (L::kSwizzled) {
+#pragma unroll
+        for (int x = 0; x < DK / 32; ++x) tc::tma_load_3d(sst + x * DK * 128, &pool_map, 32 * x, 0, slot * p.H + h, &full[s]);
+      } else {
+        tc::bulk_load(sst, p.pool + ((size_t)slot * p.H + h) * (size_t)DK * DK, L::kState, &full[s]);
+      }
 #pragma unroll
       for (int t = 0; t < TT; ++t) {
         const size_t bth = ((size_t)b * TT + t) * p.H + h;
@@ -272,18 +290,21 @@ gdn_decode_kernel(const DecodeParams p) {
       }
       tc::named_sync(kBarConsumers, kConsumers);
 
-      // my part of the row: its chunks are visited in rotated order (c + row) so
-      // that eight consecutive rows hit eight different shared-memory bank groups
-      float* srow = reinterpret_cast<float*>(st) + (size_t)row * DK + half * (DK / TPR);
+      // my part of the row: global float4 chunk gc = half * CPH + c sits in tile gc / 8,
+      // swizzled position (gc % 8) ^ (row % 8); the key / query chunk is gc itself
+      uint8_t* srow = st + (size_t)row * 128;
       float4 sv[CPH];
 #pragma unroll
-      for (int c = 0; c < CPH; ++c) sv[c] = reinterpret_cast<const float4*>(srow)[(c + row) & (CPH - 1)];
+      for (int c = 0; c < CPH; ++c) {
+        const int gc = half * CPH + c;
+        sv[c] = *reinterpret_cast<const float4*>(srow + (gc >> 3) * (DK * 128) + (((gc & 7) ^ (row & 7)) << 4));
+      }
       float dots[NV];
 #pragma unroll
       for (int vec = 0; vec < NV; ++vec) dots[vec] = 0.f;
 #pragma unroll
       for (int c = 0; c < CPH; ++c) {
-        const int e = half * (DK / TPR) + 4 * ((c + row) & (CPH - 1));
+        const int e = 4 * (half * CPH + c);
 #pragma unroll
         for (int vec = 0; vec < NV; ++vec) {
           const float4 w = *reinterpret_cast<const float4*>(vecf + vec * DK + e);
@@ -323,10 +344,11 @@ gdn_decode_kernel(const DecodeParams p) {
         for (int l = 0; l < (t + 1) * NH; ++l) out = fmaf(coef[l], qk[t * M + l], out);
         if (half == 0) store_out(op + (((size_t)b * TT + t) * p.H + h) * DK + row, p.scale * out);
       }
-      // s_new = Gamma s_0 + sum_m c_m k_m, written back in place (same rotated chunks)
+      // s_new = Gamma s_0 + sum_m c_m k_m, written back in place (same swizzled chunks)
 #pragma unroll
       for (int c = 0; c < CPH; ++c) {
-        const int e = half * (DK / TPR) + 4 * ((c + row) & (CPH - 1));
+        const int gc = half * CPH + c;
+        const int e = 4 * gc;
         float4 x = sv[c];
         x.x *= G; x.y *= G; x.z *= G; x.w *= G;
 #pragma unroll
@@ -337,7 +359,7 @@ gdn_decode_kernel(const DecodeParams p) {
           x.z = fmaf(coef[m], w.z, x.z);
           x.w = fmaf(coef[m], w.w, x.w);
         }
-        reinterpret_cast<float4*>(srow)[(c + row) & (CPH - 1)] = x;
+        *reinterpret_cast<float4*>(srow + (gc >> 3) * (DK * 128) + (((gc & 7) ^ (row & 7)) << 4)) = x;
       }
     } else {
       // skipped row of the batch: o = 0, pool untouched
@@ -350,8 +372,15 @@ gdn_decode_kernel(const DecodeParams p) {
     tc::fence_proxy_async_smem();
     tc::named_sync(kBarConsumers, kConsumers);
     if (tid == 0) {
-      if (slot >= 0)
-        tc::bulk_store(p.pool + ((size_t)slot * p.H + h) * (size_t)DK * DK, tc::smem_u32(st), L::kState);
+      if (slot >= 0) {
+        if constexpr (L::kSwizzled) {
+#pragma unroll
+          for (int x = 0; x < DK / 32; ++x)
+            tc::tma_store_3d(&pool_map, 32 * x, 0, slot * p.H + h, tc::smem_u32(st) + x * DK * 128);
+        } else {
+          tc::bulk_store(p.pool + ((size_t)slot * p.H + h) * (size_t)DK * DK, tc::smem_u32(st), L::kState);
+        }
+      }
       tc::bulk_commit();
       tc::bulk_wait_read_1();
       if (prev_stage >= 0) tc::mbar_arrive(&empty[prev_stage]);
@@ -359,6 +388,16 @@ gdn_decode_kernel(const DecodeParams p) {
     prev_stage = s;
   }
   if (tid == 0) tc::bulk_wait_all();
+}
+
+// The pool as a 3-D fp32 tensor {DK columns, DK rows, num_slots * H states}; a box
+// is one 32-column tile of one state, 128-byte swizzled.
+template <int DK>
+gdn_status_t pool_tensor_map(const DecodeParams& p, CUtensorMap* map) {
+  const uint64_t dims[3] = {(uint64_t)DK, (uint64_t)DK, (uint64_t)p.num_slots * (uint64_t)p.H};
+  const uint64_t strides[2] = {(uint64_t)DK * 4, (uint64_t)DK * DK * 4};
+  const uint32_t box[3] = {32, (uint32_t)DK, 1};
+  return make_tensor_map_3d(map, CU_TENSOR_MAP_DATA_TYPE_FLOAT32, p.pool, dims, strides, box, "gdn_decode");
 }
 
 template <int DK, int TT, int NH, typename TIn, typename TOut>
@@ -379,8 +418,16 @@ gdn_status_t launch_typed(DecodeParams p, cudaStream_t stream) {
   p.n_items = p.B * p.H;
   if (p.n_items == 0) return ok();
   const int grid = p.n_items < sm_count ? p.n_items : sm_count;
+  CUtensorMap map;
+  memset(&map, 0, sizeof(map));
+  if constexpr (L::kSwizzled) {
+    if ((long long)p.num_slots * p.H >= (1LL << 31))
+      return fail(GDN_ERR_UNSUPPORTED, "gdn_decode: num_slots * H must be below 2^31 for multi-token steps");
+    const gdn_status_t st = pool_tensor_map<DK>(p, &map);
+    if (st != GDN_OK) return st;
+  }
   gdn_decode_kernel<DK, TT, NH, TIn, TOut>
-      <<<grid, threads_per_row<TT, NH>() * DK + 32, L::kSmem, stream>>>(p);
+      <<<grid, threads_per_row<TT, NH>() * DK + 32, L::kSmem, stream>>>(p, map);
   return check_launch("gdn_decode");
 }
 

@@ -164,6 +164,19 @@ __device__ __forceinline__ void bulk_store(void* gdst, uint32_t ssrc, uint32_t b
   asm volatile("cp.async.bulk.global.shared::cta.bulk_group [%0], [%1], %2;"
                :: "l"(gdst), "r"(ssrc), "r"(bytes) : "memory");
 }
+// Tiled tensor copies (TMA) of a 3-D box, coordinates {x, y, z} in elements of the
+// tensor map (x innermost; x * element size must be a multiple of 16 bytes). The
+// map is a kernel parameter (__grid_constant__), passed by its generic address.
+// Loads complete on `bar` (transaction bytes); stores join the bulk groups.
+__device__ __forceinline__ void tma_load_3d(uint32_t sdst, const void* tmap, int x, int y, int z, uint64_t* bar) {
+  asm volatile(
+      "cp.async.bulk.tensor.3d.shared::cta.global.tile.mbarrier::complete_tx::bytes [%0], [%1, {%2, %3, %4}], [%5];"
+      :: "r"(sdst), "l"(tmap), "r"(x), "r"(y), "r"(z), "r"(smem_u32(bar)) : "memory");
+}
+__device__ __forceinline__ void tma_store_3d(const void* tmap, int x, int y, int z, uint32_t ssrc) {
+  asm volatile("cp.async.bulk.tensor.3d.global.shared::cta.tile.bulk_group [%0, {%1, %2, %3}], [%4];"
+               :: "l"(tmap), "r"(x), "r"(y), "r"(z), "r"(ssrc) : "memory");
+}
 __device__ __forceinline__ void bulk_commit() { asm volatile("cp.async.bulk.commit_group;" ::: "memory"); }
 // Waits until every committed bulk store has finished reading shared memory.
 __device__ __forceinline__ void bulk_wait_read() { asm volatile("cp.async.bulk.wait_group.read 0;" ::: "memory"); }

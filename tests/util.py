@@ -1,4 +1,10 @@
-"""Comparison helpers shared by the GPU parity tests."""
+"""Comparison helpers shared by the GPU parity tests.
+
+With GDN_PARITY_LOG set to a file path, every comparison appends one JSON line
+(what, normwise relative error, max abs error, tolerance) to that file."""
+import json
+import os
+
 import numpy as np
 import torch
 
@@ -29,6 +35,11 @@ def assert_close(x, ref, tol=TOL, what=""):
     if not ra.size:
         return
     scale = max(float(np.abs(ra).max()), 1e-30)
+    log = os.environ.get("GDN_PARITY_LOG")
+    if log:
+        with open(log, "a") as f:
+            f.write(json.dumps({"what": what, "relerr": relerr(xa, ra), "max_abs": float(np.abs(xa - ra).max()),
+                                "tol": tol, "bf16": is_bf16, "n": int(ra.size)}) + "\n")
     if is_bf16:
         ulp = np.maximum(np.abs(ra), 1e-38)
         ulp = 2.0 ** (np.floor(np.log2(ulp)) - 7)
