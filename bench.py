@@ -375,7 +375,8 @@ def bench_prefill(key, steps, warmup, ws, rank, peaks, algo=None):
                      "peak": peaks["hbm_gbs"] if bound == "hbm" else peaks["bf16_tflops"],
                      "unit": "GB/s" if bound == "hbm" else "TFLOP/s",
                      "frac": max(hbm_t, tc_t) / t,
-                     "traffic": None},
+                     "traffic": ncu_traffic(f"gdn_prefill_fused_kernel:{key}",
+                                            ["gated_delta_rule_58_b200/csrc/prefill_fused.cu"])},
         "pct_of_nominal_roofline": max(alg_b / (NOMINAL_HBM_GBS * 1e9), flops / 2.25e15) / t * 100,
         "alg_bytes": alg_b,
         "flops": flops,
