@@ -25,9 +25,11 @@
 // (section 2) evaluated without materialising M_c or H_c.
 //
 // Warp specialisation (13 warps) and the chunk pipeline:
-//   loader  (warps 8-11): cp.async of chunk c's q/k/v rows straight into the
-//            swizzled fp16 tiles (bf16 bits converted in place), g/beta, the
-//            cumulative gates and decays. Runs up to one chunk ahead.
+//   loader  (warps 8-11): TMA tensor loads of chunk c's q/k/v rows (bf16) straight
+//            into the 128-byte-swizzled MMA tiles, g/beta, the cumulative gates
+//            and decays, then the in-place conversion to fp16. fp32 inputs are
+//            loaded and converted by the threads instead.
+//            Runs up to one chunk ahead.
 //   prep    (warps 4-7):  A and P from [K;Q]K^T, the triangular solve, the fp16
 //            T diag(beta gamma) / T diag(beta) tiles, then W^T -> fp16 tile.
 //            Works on chunk c+1 while the state warps finish chunk c.
@@ -37,10 +39,12 @@
 // Hand-offs are mbarriers: tcgen05.commit for MMA completion, one elected arrive
 // per warpgroup (after a named barrier) for thread-produced tiles. Every wait is
 // bounded; a timeout sets GDN_DEVERR_TIMEOUT and unwinds all roles.
+#include <cstring>
 #include <type_traits>
 
 #include "prefill.cuh"
 #include "tcgen05.cuh"
+#include "tensor_map.cuh"
 
 namespace gdn {
 namespace {
@@ -87,6 +91,7 @@ constexpr uint32_t TMEM_COLS = 512;
 // mbarrier slots
 enum Bar : int {
   B_L0 = 0, B_L1,      // loader -> chunk tiles ready (per buffer)
+  B_T0, B_T1,          // TMA -> raw bf16 tiles landed (per buffer)
   B_M1,                // MMA: D1 ready
   B_M2,                // MMA: W^T, U~^T ready
   B_M3A,               // MMA: U^T ready (S16, W16 consumed)
@@ -152,11 +157,35 @@ __device__ __forceinline__ void group_signal(const Smem& sm, uint32_t bar_id, in
 
 // ---------------------------------------------------------------- loader role
 
+struct QkvMaps {
+  CUtensorMap q, k, v;  // bf16 [total_T][H][128] as {128, H, total_T}; box {64, 1, 64}
+};
+
+// bf16 -> fp16 of one 16-byte chunk (8 elements) in place.
+__device__ __forceinline__ void convert_chunk_bf16(uint8_t* p) {
+  uint4* q = reinterpret_cast<uint4*>(p);
+  const uint4 raw = *q;
+  const __nv_bfloat162* hb = reinterpret_cast<const __nv_bfloat162*>(&raw);
+  uint4 u;
+  const float2 f0 = __bfloat1622float2(hb[0]), f1 = __bfloat1622float2(hb[1]);
+  const float2 f2 = __bfloat1622float2(hb[2]), f3 = __bfloat1622float2(hb[3]);
+  u.x = pack_half2(f0.x, f0.y);
+  u.y = pack_half2(f1.x, f1.y);
+  u.z = pack_half2(f2.x, f2.y);
+  u.w = pack_half2(f3.x, f3.y);
+  *q = u;
+}
+
 template <typename TIn>
-__device__ void loader_role(const Smem& sm, const PrefillShape& s, const PrefillArgs& a, int h, int64_t bos,
-                            int64_t eos, int nchunks) {
+__device__ void loader_role(const Smem& sm, const PrefillShape& s, const PrefillArgs& a, const QkvMaps& maps,
+                            int h, int64_t bos, int64_t eos, int nchunks) {
+  constexpr bool kTma = std::is_same<TIn, __nv_bfloat16>::value;
   const int t = threadIdx.x - kLoadWarp0 * 32;  // 0..127
   const bool zero_values = (a.mode == kPrefillTransfer);  // transfer run: V taken as 0
+  if (zero_values) {  // both V buffers stay zero for the whole run
+    for (int i = t; i < 2 * V_BUF / 16; i += 128)
+      *reinterpret_cast<uint4*>(sm.base + OFF_V + 16 * i) = make_uint4(0u, 0u, 0u, 0u);
+  }
   for (int c = 0; c < nchunks; ++c) {
     const int b = c & 1;
     // chunk c-2 (same buffers) fully consumed: its outputs were read, so every
@@ -165,34 +194,24 @@ __device__ void loader_role(const Smem& sm, const PrefillShape& s, const Prefill
     const int64_t t0 = bos + (int64_t)c * C;
     const int Lc = (int)((eos - t0) < C ? (eos - t0) : C);
     float* vec = sm.vec(b);
+    uint8_t* kq = sm.base + OFF_KQ + b * KQ_BUF;
+    uint8_t* v16 = sm.base + OFF_V + b * V_BUF;
+    if constexpr (kTma) {
+      // rows past the sequence end load the next tokens (or zeros past the tensor);
+      // their beta and g are set to 0 below, which removes them from every product
+      if (t == 0) {
+        tc::fence_proxy_async_smem();  // the previous generic writes of these tiles precede the copies
+        tc::mbar_arrive_expect_tx(sm.bar(B_T0 + b), (zero_values ? 2u : 3u) * 16384u);
 #pragma unroll
-    for (int mat = 0; mat < 3; ++mat) {
-      const TIn* src0 = static_cast<const TIn*>(mat == 0 ? a.k : (mat == 1 ? a.q : a.v));
-      uint8_t* base = (mat == 2) ? sm.base + OFF_V + b * V_BUF : sm.base + OFF_KQ + b * KQ_BUF;
-      const uint32_t half = (mat == 2) ? V_HALF : KQ_HALF;
-      const int roff = (mat == 1) ? C : 0;
-#pragma unroll 4
-      for (int i = t; i < C * 16; i += 128) {
-        const int row = i >> 4, ch = i & 15;
-        uint8_t* tile = base + (ch >> 3) * half;
-        const uint32_t off = tc::sw128_offset(row + roff, ch & 7, 1024);
-        const TIn* src = src0 + ((size_t)(t0 + (row < Lc ? row : 0)) * s.H + h) * D + ch * 8;
-        const bool live = row < Lc && !(mat == 2 && zero_values);
-        if constexpr (std::is_same<TIn, __nv_bfloat16>::value) {
-          tc::cp_async16(tc::smem_u32(tile + off), src, live ? 16u : 0u);
-        } else {
-          float v8[8];
-          if (live) {
-            load8_f32(src, v8);
-          } else {
-#pragma unroll
-            for (int x = 0; x < 8; ++x) v8[x] = 0.f;
-          }
-          st_sw128_chunk(tile, row + roff, ch & 7, v8);
+        for (int hf = 0; hf < 2; ++hf) {
+          tc::tma_load_3d(tc::smem_u32(kq + hf * KQ_HALF), &maps.k, 64 * hf, h, (int)t0, sm.bar(B_T0 + b));
+          tc::tma_load_3d(tc::smem_u32(kq + hf * KQ_HALF + C * 128), &maps.q, 64 * hf, h, (int)t0, sm.bar(B_T0 + b));
+          if (!zero_values)
+            tc::tma_load_3d(tc::smem_u32(v16 + hf * V_HALF), &maps.v, 64 * hf, h, (int)t0, sm.bar(B_T0 + b));
         }
       }
     }
-    if (t < C) {  // g and beta (scalar loads, issued behind the async copies)
+    if (t < C) {  // g and beta (zero past the sequence end)
       float gv = 0.f, bv = 0.f;
       if (t < Lc) {
         const size_t th = (size_t)(t0 + t) * s.H + h;
@@ -201,32 +220,6 @@ __device__ void loader_role(const Smem& sm, const PrefillShape& s, const Prefill
       }
       vec[V_G + t] = gv;
       vec[V_BETA + t] = bv;
-    }
-    if constexpr (std::is_same<TIn, __nv_bfloat16>::value) {
-      tc::cp_async_commit();
-      tc::cp_async_wait_all();
-      // bf16 -> fp16 in place: each thread converts the chunks it copied
-#pragma unroll
-      for (int mat = 0; mat < 3; ++mat) {
-        uint8_t* base = (mat == 2) ? sm.base + OFF_V + b * V_BUF : sm.base + OFF_KQ + b * KQ_BUF;
-        const uint32_t half = (mat == 2) ? V_HALF : KQ_HALF;
-        const int roff = (mat == 1) ? C : 0;
-#pragma unroll 4
-        for (int i = t; i < C * 16; i += 128) {
-          const int row = i >> 4, ch = i & 15;
-          uint4* p = reinterpret_cast<uint4*>(base + (ch >> 3) * half + tc::sw128_offset(row + roff, ch & 7, 1024));
-          const uint4 raw = *p;
-          const __nv_bfloat162* hb = reinterpret_cast<const __nv_bfloat162*>(&raw);
-          uint4 u;
-          float2 f0 = __bfloat1622float2(hb[0]), f1 = __bfloat1622float2(hb[1]);
-          float2 f2 = __bfloat1622float2(hb[2]), f3 = __bfloat1622float2(hb[3]);
-          u.x = pack_half2(f0.x, f0.y);
-          u.y = pack_half2(f1.x, f1.y);
-          u.z = pack_half2(f2.x, f2.y);
-          u.w = pack_half2(f3.x, f3.y);
-          *p = u;
-        }
-      }
     }
     tc::named_sync(kBarLoad, 128);
     if (t < 32) {
@@ -248,6 +241,41 @@ __device__ void loader_role(const Smem& sm, const PrefillShape& s, const Prefill
         vec[V_GAM + i] = gm;
         vec[V_DD + i] = __expf(Gc - Gi);
         vec[V_BG + i] = vec[V_BETA + i] * gm;
+      }
+    }
+    tc::named_sync(kBarLoad, 128);
+    if constexpr (kTma) {
+      if (!wait_bar(sm, B_T0 + b, (c >> 1) & 1, a.err)) return;
+      // in place to fp16 (the queries stay unscaled: P is taken from Q K^T)
+#pragma unroll 4
+      for (int i = t; i < 3 * C * 16; i += 128) {
+        const int mat = i >> 10, rem = i & 1023;  // 0 K, 1 Q, 2 V; 64 rows x 16 chunks each
+        const int row = rem >> 4, ch = rem & 15;
+        if (mat == 2 && zero_values) continue;
+        uint8_t* tile = (mat == 2) ? v16 + (ch >> 3) * V_HALF : kq + (ch >> 3) * KQ_HALF;
+        const int trow = row + (mat == 1 ? C : 0);
+        convert_chunk_bf16(tile + tc::sw128_offset(trow, ch & 7, 1024));
+      }
+    } else {
+#pragma unroll
+      for (int mat = 0; mat < 3; ++mat) {
+        if (mat == 2 && zero_values) continue;
+        const TIn* src0 = static_cast<const TIn*>(mat == 0 ? a.k : (mat == 1 ? a.q : a.v));
+        uint8_t* base = (mat == 2) ? v16 : kq;
+        const uint32_t half = (mat == 2) ? V_HALF : KQ_HALF;
+        const int roff = (mat == 1) ? C : 0;
+#pragma unroll 4
+        for (int i = t; i < C * 16; i += 128) {
+          const int row = i >> 4, ch = i & 15;
+          float v8[8];
+          if (row < Lc) {
+            load8_f32(src0 + ((size_t)(t0 + row) * s.H + h) * D + ch * 8, v8);
+          } else {
+#pragma unroll
+            for (int x = 0; x < 8; ++x) v8[x] = 0.f;
+          }
+          st_sw128_chunk(base + (ch >> 3) * half, row + roff, ch & 7, v8);
+        }
       }
     }
     group_signal(sm, kBarLoad, B_L0 + b);
@@ -691,7 +719,7 @@ __device__ void mma_role(const Smem& sm, uint32_t tmem, int nchunks, unsigned in
 
 template <typename TIn, typename TOut>
 __global__ void __launch_bounds__(kThreads, 1)
-gdn_prefill_fused_kernel(const PrefillShape s, const PrefillArgs a) {
+gdn_prefill_fused_kernel(const PrefillShape s, const PrefillArgs a, const __grid_constant__ QkvMaps maps) {
   extern __shared__ uint8_t smem_raw[];
   Smem sm;
   sm.base = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
@@ -737,7 +765,7 @@ gdn_prefill_fused_kernel(const PrefillShape s, const PrefillArgs a) {
   } else if (warp < kLoadWarp0) {
     prep_role(sm, tmem, nchunks, a.err);
   } else if (warp < kMmaWarp) {
-    loader_role<TIn>(sm, s, a, h, bos, eos, nchunks);
+    loader_role<TIn>(sm, s, a, maps, h, bos, eos, nchunks);
   } else if ((threadIdx.x & 31) == 0) {
     mma_role(sm, tmem, nchunks, a.err);
   }
@@ -760,7 +788,22 @@ gdn_status_t launch(const PrefillShape& s, const PrefillArgs& a, cudaStream_t st
     configured = true;
   }
   const unsigned grid = (unsigned)((long long)s.N * s.H);
-  gdn_prefill_fused_kernel<TIn, TOut><<<grid, kThreads, SMEM_BYTES, stream>>>(s, a);
+  QkvMaps maps;
+  memset(&maps, 0, sizeof(maps));
+  if (std::is_same<TIn, __nv_bfloat16>::value && s.total_T > 0) {
+    // q, k, v as {128, H, total_T} bf16; one box = 64 features x 64 tokens of one head
+    const uint64_t dims[3] = {(uint64_t)D, (uint64_t)s.H, (uint64_t)s.total_T};
+    const uint64_t strides[2] = {(uint64_t)D * 2, (uint64_t)s.H * D * 2};
+    const uint32_t box[3] = {64, 1, (uint32_t)C};
+    const void* src[3] = {a.q, a.k, a.v};
+    CUtensorMap* dst[3] = {&maps.q, &maps.k, &maps.v};
+    for (int i = 0; i < 3; ++i) {
+      const gdn_status_t st = make_tensor_map_3d(dst[i], CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, src[i], dims, strides, box,
+                                                 "fused prefill");
+      if (st != GDN_OK) return st;
+    }
+  }
+  gdn_prefill_fused_kernel<TIn, TOut><<<grid, kThreads, SMEM_BYTES, stream>>>(s, a, maps);
   return check_launch("gdn_chunk_prefill (fused)");
 }
 

@@ -14,18 +14,20 @@
 //      a zero state, final state = H_seg (K-last, i.e. H_seg^T);
 //   3. transfers: the same kernel from the identity state with the values taken
 //      as zero, final state = M_seg (stored K-last, i.e. M_seg^T row-major);
-//   4. fixup scan (SIMT): per (sequence, head), the state rows split across CTAs,
-//      fixed[s] = S; S^T <- S^T M_seg^T + H_seg^T over the sequence's segments,
-//      then the final state (the serial part; the PR #3866 page's SIMT fixup
-//      loop, with the next segment's transfer rows preloaded);
+//   4. fixup scan (SIMT, fp32): per (sequence, head), the state rows split across
+//      CTAs, fixed[s] = S; S^T <- S^T M_seg^T + H_seg^T over the sequence's
+//      segments, then the final state (the serial part; the PR #3866 page's SIMT
+//      fixup loop, with the next segment's transfer matrix staged ahead);
 //   5. outputs: the fused kernel over all segments, each from its fixed state.
 //
 // Steps 2, 3 and 5 use every SM even for a single sequence; only step 4 is
-// serial, with G times fewer steps than there are chunks. G is picked so that
-// steps 2/3/5 have about four segment CTAs per SM.
+// serial, with G times fewer steps than there are chunks. G is the smallest
+// power of two that fits steps 2/3/5 into about one wave of CTAs (one per SM):
+// more segments would add fixup steps without shortening those passes.
 #include <string>
 
 #include "prefill.cuh"
+#include "tcgen05.cuh"
 
 namespace gdn {
 namespace {
@@ -33,7 +35,7 @@ namespace {
 constexpr int C = 64;
 constexpr int D = 128;
 constexpr int kFixRows = 8;       // state rows (value indices) per fixup CTA
-constexpr int kFixThreads = 128;  // one thread per key column
+constexpr int kFixThreads = 128;  // 4 warps; each thread a 2 x 4 tile of the 8 x 128 block
 
 size_t align256(size_t x) { return (x + 255) / 256 * 256; }
 
@@ -43,9 +45,9 @@ struct TransferLayout {
   size_t off_seg_cu, off_seg_of_seq, off_local, off_transfer, off_fixed, total;
 };
 
-// Segment CTAs wanted per state run: about four per SM of a B200 (148 SMs). A
-// constant, so that the workspace size is a pure function of the shape.
-constexpr long long kTargetSegmentCtas = 4LL * 148;
+// Segment CTAs wanted per state run: one per SM of a B200 (148 SMs). A constant,
+// so that the workspace size is a pure function of the shape.
+constexpr long long kTargetSegmentCtas = 148;
 
 TransferLayout layout_for(const PrefillShape& s) {
   TransferLayout L{};
@@ -114,7 +116,7 @@ gdn_segment_map_kernel(const int32_t* cu, int N, int64_t total_T, int seg_len, i
     const int excl = carry + (warp > 0 ? warp_sums[warp - 1] : 0) + x - cnt;
     if (n < N) {
       seg_of_seq[n] = excl;
-      const int32_t a = cu[n], b = cu[n + 1];
+      const int32_t a = cu[n];
       for (int k = 0; k < cnt && excl + k < max_segments; ++k) seg_cu[excl + k] = a + k * seg_len;
     }
     __syncthreads();
@@ -129,58 +131,124 @@ gdn_segment_map_kernel(const int32_t* cu, int N, int64_t total_T, int seg_len, i
 }
 
 // 4. Fixup scan over the segments of one (sequence, head), kFixRows rows of S^T
-//    per CTA: fixed[s] = S, then S^T <- S^T M^T + H^T. Thread l owns column l.
+//    per CTA: fixed[s] = S, then S^T <- S^T M^T + H^T, in fp32 (the products
+//    compose along the whole sequence, so no reduced-precision operands here).
+//    Each segment's transfer matrix (64 KiB) and local-state rows are staged in
+//    shared memory by one bulk copy, one segment ahead (two buffers). Thread
+//    (warp w, lane = 8 rg + cg) owns rows 2rg, 2rg+1 and columns 32w + 4cg .. +3
+//    of the block; the state block is kept transposed in shared memory (sT[i][j])
+//    for the products and in registers (the thread's own tile) for the stores.
+constexpr uint32_t kFixMtBytes = D * D * 4;
+constexpr uint32_t kFixLocBytes = kFixRows * D * 4;
+constexpr uint32_t kFixSmem = 2 * kFixMtBytes + 2 * kFixLocBytes + D * kFixRows * 4 + 64;
+constexpr uint64_t kFixWaitNs = 2000000000ull;
+
+__device__ __forceinline__ void fixup_issue(float* mt, float* loc, uint64_t* bar, const float* transfer,
+                                            const float* local, size_t off, int r0) {
+  tc::fence_proxy_async_smem();  // earlier generic reads of this buffer precede the copy
+  tc::mbar_arrive_expect_tx(bar, kFixMtBytes + kFixLocBytes);
+  tc::bulk_load(tc::smem_u32(mt), transfer + off, kFixMtBytes, bar);
+  tc::bulk_load(tc::smem_u32(loc), local + off + (size_t)r0 * D, kFixLocBytes, bar);
+}
+
 __global__ void __launch_bounds__(kFixThreads)
 gdn_fixup_scan_kernel(const int32_t* seg_of_seq, int H, const float* local, const float* transfer,
-                      float* fixed, const float* initial_state, float* final_state) {
-  __shared__ __align__(16) float srow[kFixRows][D];
-  const int l = threadIdx.x;
+                      float* fixed, const float* initial_state, float* final_state, unsigned int* err) {
+  extern __shared__ __align__(16) uint8_t fsm[];
+  float* mt = reinterpret_cast<float*>(fsm);                 // [2][D][D]
+  float* loc = mt + 2 * D * D;                                // [2][kFixRows][D]
+  float* sT = loc + 2 * kFixRows * D;                         // [D][kFixRows]
+  uint64_t* full = reinterpret_cast<uint64_t*>(sT + D * kFixRows);
+  const int tid = threadIdx.x, w = tid >> 5, lane = tid & 31;
+  const int rg = lane >> 3, cg = lane & 7;
+  const int jr = 2 * rg;                 // first of my two rows (within the block)
+  const int l0 = 32 * w + 4 * cg;        // first of my four columns
   const int rblocks = D / kFixRows;
   const int rb = blockIdx.x % rblocks;
   const int nh = blockIdx.x / rblocks;
   const int n = nh / H, h = nh - (nh / H) * H;
   const int r0 = rb * kFixRows;
   const size_t ssz = (size_t)D * D;
-#pragma unroll
-  for (int j = 0; j < kFixRows; ++j)
-    srow[j][l] = initial_state ? initial_state[((size_t)n * H + h) * ssz + (size_t)(r0 + j) * D + l] : 0.f;
-  __syncthreads();
+  const size_t soff = ((size_t)n * H + h) * ssz;
   const int s0 = seg_of_seq[n], s1 = seg_of_seq[n + 1];
-  for (int sg = s0; sg < s1; ++sg) {
-    const size_t off = ((size_t)sg * H + h) * ssz;
-    float acc[kFixRows];
+
+  if (tid == 0) {
+    tc::mbar_init(&full[0], 1);
+    tc::mbar_init(&full[1], 1);
+    tc::fence_mbar_init();
+  }
+  // my tile of the initial state (registers) and the transposed block (shared)
+  float cur[2][4];
 #pragma unroll
-    for (int j = 0; j < kFixRows; ++j) {
-      acc[j] = local[off + (size_t)(r0 + j) * D + l];
-      fixed[off + (size_t)(r0 + j) * D + l] = srow[j][l];  // state at the segment start
+  for (int a = 0; a < 2; ++a) {
+    float4 x = make_float4(0.f, 0.f, 0.f, 0.f);
+    if (initial_state) x = *reinterpret_cast<const float4*>(initial_state + soff + (size_t)(r0 + jr + a) * D + l0);
+    cur[a][0] = x.x; cur[a][1] = x.y; cur[a][2] = x.z; cur[a][3] = x.w;
+#pragma unroll
+    for (int x4 = 0; x4 < 4; ++x4) sT[(l0 + x4) * kFixRows + jr + a] = cur[a][x4];
+  }
+  __syncthreads();
+  if (tid == 0 && s0 < s1)
+    fixup_issue(mt, loc, &full[0], transfer, local, ((size_t)s0 * H + h) * ssz, r0);
+
+  int it = 0;
+  bool pending_other = false;  // a prefetch into the other buffer is in flight
+  for (int sg = s0; sg < s1; ++sg, ++it) {
+    const int b = it & 1;
+    pending_other = false;
+    if (tid == 0 && sg + 1 < s1) {
+      fixup_issue(mt + (b ^ 1) * D * D, loc + (b ^ 1) * kFixRows * D, &full[b ^ 1], transfer, local,
+                  ((size_t)(sg + 1) * H + h) * ssz, r0);
+      pending_other = true;
     }
-    // acc[j] += sum_i S^T[j][i] * M^T[i][l], transfer rows streamed 16 at a time
-    const float* mt = transfer + off + l;
-    for (int i0 = 0; i0 < D; i0 += 16) {
-      float m[16];
-#pragma unroll
-      for (int i = 0; i < 16; ++i) m[i] = mt[(size_t)(i0 + i) * D];
-#pragma unroll
-      for (int j = 0; j < kFixRows; ++j) {
-#pragma unroll
-        for (int q = 0; q < 4; ++q) {
-          const float4 sv = *reinterpret_cast<const float4*>(&srow[j][i0 + 4 * q]);
-          acc[j] = fmaf(sv.x, m[4 * q], acc[j]);
-          acc[j] = fmaf(sv.y, m[4 * q + 1], acc[j]);
-          acc[j] = fmaf(sv.z, m[4 * q + 2], acc[j]);
-          acc[j] = fmaf(sv.w, m[4 * q + 3], acc[j]);
-        }
+    const bool got = tc::mbar_wait(&full[b], (it >> 1) & 1, kFixWaitNs);
+    if (!__syncthreads_and(got)) {
+      if (tid == 0) {
+        raise_device_error(err, GDN_DEVERR_TIMEOUT);
+        if (pending_other) tc::mbar_wait(&full[b ^ 1], ((it + 1) >> 1) & 1, kFixWaitNs);
       }
+      return;
     }
-    __syncthreads();
+    const size_t off = ((size_t)sg * H + h) * ssz;
+    const float* m = mt + b * D * D;
+    const float* lr = loc + b * kFixRows * D;
+    float acc[2][4];
 #pragma unroll
-    for (int j = 0; j < kFixRows; ++j) srow[j][l] = acc[j];
+    for (int a = 0; a < 2; ++a) {
+      // the state at the segment start, then the local state as the accumulator
+      *reinterpret_cast<float4*>(fixed + off + (size_t)(r0 + jr + a) * D + l0) =
+          make_float4(cur[a][0], cur[a][1], cur[a][2], cur[a][3]);
+      const float4 x = *reinterpret_cast<const float4*>(lr + (jr + a) * D + l0);
+      acc[a][0] = x.x; acc[a][1] = x.y; acc[a][2] = x.z; acc[a][3] = x.w;
+    }
+#pragma unroll 8
+    for (int i = 0; i < D; ++i) {
+      const float2 sv = *reinterpret_cast<const float2*>(sT + i * kFixRows + jr);
+      const float4 mv = *reinterpret_cast<const float4*>(m + i * D + l0);
+      acc[0][0] = fmaf(sv.x, mv.x, acc[0][0]);
+      acc[0][1] = fmaf(sv.x, mv.y, acc[0][1]);
+      acc[0][2] = fmaf(sv.x, mv.z, acc[0][2]);
+      acc[0][3] = fmaf(sv.x, mv.w, acc[0][3]);
+      acc[1][0] = fmaf(sv.y, mv.x, acc[1][0]);
+      acc[1][1] = fmaf(sv.y, mv.y, acc[1][1]);
+      acc[1][2] = fmaf(sv.y, mv.z, acc[1][2]);
+      acc[1][3] = fmaf(sv.y, mv.w, acc[1][3]);
+    }
+    __syncthreads();  // every read of sT and of this buffer is done
+#pragma unroll
+    for (int a = 0; a < 2; ++a)
+#pragma unroll
+      for (int x4 = 0; x4 < 4; ++x4) {
+        cur[a][x4] = acc[a][x4];
+        sT[(l0 + x4) * kFixRows + jr + a] = acc[a][x4];
+      }
     __syncthreads();
   }
   if (final_state) {
 #pragma unroll
-    for (int j = 0; j < kFixRows; ++j)
-      final_state[((size_t)n * H + h) * ssz + (size_t)(r0 + j) * D + l] = srow[j][l];
+    for (int a = 0; a < 2; ++a)
+      *reinterpret_cast<float4*>(final_state + soff + (size_t)(r0 + jr + a) * D + l0) =
+          make_float4(cur[a][0], cur[a][1], cur[a][2], cur[a][3]);
   }
 }
 
@@ -220,8 +288,16 @@ gdn_status_t prefill_transfer_launch(const PrefillShape& s, const PrefillArgs& a
   st = prefill_fused_launch(seg, tr, stream);
   if (st != GDN_OK) return st;
 
-  gdn_fixup_scan_kernel<<<(unsigned)((long long)s.N * s.H * (D / kFixRows)), kFixThreads, 0, stream>>>(
-      seg_of_seq, s.H, local, transfer, fixed, a.initial_state, a.final_state);
+  static bool fix_configured = false;
+  if (!fix_configured) {
+    const cudaError_t e =
+        cudaFuncSetAttribute(gdn_fixup_scan_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, kFixSmem);
+    if (e != cudaSuccess)
+      return fail(GDN_ERR_CUDA, std::string("transfer prefill: cudaFuncSetAttribute: ") + cudaGetErrorString(e));
+    fix_configured = true;
+  }
+  gdn_fixup_scan_kernel<<<(unsigned)((long long)s.N * s.H * (D / kFixRows)), kFixThreads, kFixSmem, stream>>>(
+      seg_of_seq, s.H, local, transfer, fixed, a.initial_state, a.final_state, a.err);
   st = check_launch("transfer prefill: fixup scan");
   if (st != GDN_OK) return st;
 
