@@ -136,8 +136,19 @@ struct Smem {
   }
   __device__ uint32_t u32(uint32_t off) const { return tc::smem_u32(base + off); }
 };
-// vec(b) layout: [0,64) G, [64,128) gamma, [128,192) dd, [192,256) beta, [256,320) beta*gamma
+// vec(b) layout: [0,64) G log2(e) (cumulative log gate in base 2), [64,128) gamma,
+// [128,192) dd, [192,256) beta, [256,320) beta*gamma
 constexpr int V_G = 0, V_GAM = 64, V_DD = 128, V_BETA = 192, V_BG = 256;
+constexpr float kLog2e = 1.4426950408889634f;
+
+// 2^x on the special-function unit (exp(y) = 2^(y log2 e)); results below the
+// normal range flush to zero, which only drops decays under 1e-38. Not volatile,
+// so independent calls can be scheduled back to back.
+__device__ __forceinline__ float exp2_approx(float x) {
+  float y;
+  asm("ex2.approx.ftz.f32 %0, %1;" : "=f"(y) : "f"(x));
+  return y;
+}
 
 __device__ __forceinline__ bool wait_bar(const Smem& sm, int b, uint32_t parity, unsigned int* err) {
   if (tc::mbar_wait(sm.bar(b), parity, kWaitNs, sm.abort_flag())) return true;
@@ -159,6 +170,7 @@ __device__ __forceinline__ void group_signal(const Smem& sm, uint32_t bar_id, in
 
 struct QkvMaps {
   CUtensorMap q, k, v;  // bf16 [total_T][H][128] as {128, H, total_T}; box {64, 1, 64}
+  CUtensorMap o;        // o [total_T][H][128] as {128, H, total_T}; box {128, 1, 64}, not swizzled
 };
 
 // bf16 -> fp16 of one 16-byte chunk (8 elements) in place.
@@ -231,15 +243,15 @@ __device__ void loader_role(const Smem& sm, const PrefillShape& s, const Prefill
         const float y = __shfl_up_sync(0xffffffffu, pre, off);
         if (t >= off) pre += y;
       }
-      const float Gc = __shfl_sync(0xffffffffu, pre, 31);
+      const float Gc = __shfl_sync(0xffffffffu, pre, 31) * kLog2e;
 #pragma unroll
       for (int e = 0; e < 2; ++e) {
         const int i = 2 * t + e;
-        const float Gi = e ? pre : pre - x1;
-        const float gm = __expf(Gi);
+        const float Gi = (e ? pre : pre - x1) * kLog2e;
+        const float gm = exp2_approx(Gi);
         vec[V_G + i] = Gi;
         vec[V_GAM + i] = gm;
-        vec[V_DD + i] = __expf(Gc - Gi);
+        vec[V_DD + i] = exp2_approx(Gc - Gi);
         vec[V_BG + i] = vec[V_BETA + i] * gm;
       }
     }
@@ -348,17 +360,17 @@ __device__ __forceinline__ void solve_unit_lower(const Smem& sm, int t) {
   float* A = sm.A();
   float* T = sm.T();
   if (t < C) {
+    // column c of the inverse of diagonal block b, column-oriented: once x_k is
+    // known it is folded into every later row, so each step waits on one FMA
     const int b = t >> 4, c = t & 15;
-    float x[16];
+    float x[16], acc[16];
 #pragma unroll
-    for (int r = 0; r < 16; ++r) {
-      float acc0 = 0.f, acc1 = 0.f;
+    for (int r = 0; r < 16; ++r) acc[r] = 0.f;
 #pragma unroll
-      for (int k = 0; k < r; ++k) {
-        if (k & 1) acc1 = fmaf(A[sidx(16 * b + r, 16 * b + k)], x[k], acc1);
-        else acc0 = fmaf(A[sidx(16 * b + r, 16 * b + k)], x[k], acc0);
-      }
-      x[r] = (r < c) ? 0.f : ((r == c) ? 1.f : -(acc0 + acc1));
+    for (int k = 0; k < 16; ++k) {
+      x[k] = (k < c) ? 0.f : ((k == c) ? 1.f : -acc[k]);
+#pragma unroll
+      for (int r = k + 1; r < 16; ++r) acc[r] = fmaf(A[sidx(16 * b + r, 16 * b + k)], x[k], acc[r]);
     }
 #pragma unroll
     for (int r = 0; r < 16; ++r) T[sidx(16 * b + r, 16 * b + c)] = x[r];
@@ -385,6 +397,9 @@ __device__ void prep_role(const Smem& sm, uint32_t tmem, int nchunks, unsigned i
   const int t = threadIdx.x - kPrepWarp0 * 32;  // 0..127 == TMEM lane
   const int warp = threadIdx.x >> 5;
   const uint32_t tl = tmem + ((uint32_t)((warp & 3) * 32) << 16);
+  // both P tiles start as zeros: the strictly upper 16-byte chunks are never written
+  for (int i = t; i < 2 * P_BUF / 16; i += 128)
+    *reinterpret_cast<uint4*>(sm.base + OFF_P16 + 16 * i) = make_uint4(0u, 0u, 0u, 0u);
   for (int c = 0; c < nchunks; ++c) {
     const int b = c & 1;
     if (!wait_bar(sm, B_L0 + b, (c >> 1) & 1, err)) return;
@@ -404,41 +419,66 @@ __device__ void prep_role(const Smem& sm, uint32_t tmem, int nchunks, unsigned i
           float x[32];
           tc::tmem_ld16(tl + COL_D1 + hq * 32, x);
           tc::tmem_ld16(tl + COL_D1 + hq * 32 + 16, x + 16);
+          float4 gj[8];  // G of the 32 columns, loaded up front (no loads inside the masked loop)
+#pragma unroll
+          for (int q = 0; q < 8; ++q) gj[q] = *reinterpret_cast<const float4*>(G + 32 * hq + 4 * q);
+          // the 32 decays first, unconditionally (independent, so they pipeline);
+          // entries right of the diagonal may overflow and are masked below
+          float e[32];
+#pragma unroll
+          for (int q = 0; q < 8; ++q) {
+            e[4 * q + 0] = exp2_approx(Gi - gj[q].x);
+            e[4 * q + 1] = exp2_approx(Gi - gj[q].y);
+            e[4 * q + 2] = exp2_approx(Gi - gj[q].z);
+            e[4 * q + 3] = exp2_approx(Gi - gj[q].w);
+          }
           tc::wait_ld();
 #pragma unroll
           for (int q = 0; q < 8; ++q) {
             const int j0 = 32 * hq + 4 * q;
-            if (j0 < t) {
-              float4 v;
-              v.x = (j0 + 0 < t) ? bi * __expf(Gi - G[j0 + 0]) * x[4 * q + 0] : 0.f;
-              v.y = (j0 + 1 < t) ? bi * __expf(Gi - G[j0 + 1]) * x[4 * q + 1] : 0.f;
-              v.z = (j0 + 2 < t) ? bi * __expf(Gi - G[j0 + 2]) * x[4 * q + 2] : 0.f;
-              v.w = (j0 + 3 < t) ? bi * __expf(Gi - G[j0 + 3]) * x[4 * q + 3] : 0.f;
-              *row_chunk(sm.A(), t, j0 >> 2) = v;
-            }
+            float4 v;
+            v.x = (j0 + 0 < t) ? bi * e[4 * q + 0] * x[4 * q + 0] : 0.f;
+            v.y = (j0 + 1 < t) ? bi * e[4 * q + 1] * x[4 * q + 1] : 0.f;
+            v.z = (j0 + 2 < t) ? bi * e[4 * q + 2] * x[4 * q + 2] : 0.f;
+            v.w = (j0 + 3 < t) ? bi * e[4 * q + 3] * x[4 * q + 3] : 0.f;
+            if (j0 < t) *row_chunk(sm.A(), t, j0 >> 2) = v;
           }
         }
       }
     } else {
       // P row r (rows 64-127 of D1) into P16[b]; its previous reader (chunk c-2's O2
-      // MMA) completed before this chunk's D1 MMA, whose completion was waited on
+      // MMA) completed before this chunk's D1 MMA, whose completion was waited on.
+      // 16-byte chunks entirely above the diagonal keep the zeros written at start.
       const int r = t - C;
       const float Gr = G[r];
 #pragma unroll
       for (int hq = 0; hq < 2; ++hq) {
-        float x[32];
-        tc::tmem_ld16(tl + COL_D1 + hq * 32, x);
-        tc::tmem_ld16(tl + COL_D1 + hq * 32 + 16, x + 16);
-        tc::wait_ld();
+        if (32 * hq <= (r | 31)) {  // warp-uniform (tcgen05.ld is warp-collective)
+          float x[32];
+          tc::tmem_ld16(tl + COL_D1 + hq * 32, x);
+          tc::tmem_ld16(tl + COL_D1 + hq * 32 + 16, x + 16);
+          float4 gi[8];
 #pragma unroll
-        for (int cc = 0; cc < 4; ++cc) {
-          float v[8];
+          for (int q = 0; q < 8; ++q) gi[q] = *reinterpret_cast<const float4*>(G + 32 * hq + 4 * q);
+          float e[32];
 #pragma unroll
-          for (int m = 0; m < 8; ++m) {
-            const int i = 32 * hq + cc * 8 + m;
-            v[m] = (i <= r) ? __expf(Gr - G[i]) * x[cc * 8 + m] : 0.f;  // zeros above the diagonal
+          for (int q = 0; q < 8; ++q) {
+            e[4 * q + 0] = exp2_approx(Gr - gi[q].x);
+            e[4 * q + 1] = exp2_approx(Gr - gi[q].y);
+            e[4 * q + 2] = exp2_approx(Gr - gi[q].z);
+            e[4 * q + 3] = exp2_approx(Gr - gi[q].w);
           }
-          st_sw128_chunk(sm.base + OFF_P16 + b * P_BUF, r, 4 * hq + cc, v);
+          tc::wait_ld();
+#pragma unroll
+          for (int cc = 0; cc < 4; ++cc) {
+            float v[8];
+#pragma unroll
+            for (int m = 0; m < 8; ++m) {
+              const int i = 32 * hq + cc * 8 + m;
+              v[m] = (i <= r) ? e[cc * 8 + m] * x[cc * 8 + m] : 0.f;
+            }
+            if (32 * hq + cc * 8 <= r) st_sw128_chunk(sm.base + OFF_P16 + b * P_BUF, r, 4 * hq + cc, v);
+          }
         }
       }
     }
@@ -484,8 +524,8 @@ __device__ void prep_role(const Smem& sm, uint32_t tmem, int nchunks, unsigned i
 // ---------------------------------------------------------------- state role
 
 template <typename TOut>
-__device__ void state_role(const Smem& sm, const PrefillShape& s, const PrefillArgs& a, uint32_t tmem, int h,
-                           int64_t bos, int64_t eos, int nchunks, size_t state_off) {
+__device__ void state_role(const Smem& sm, const PrefillShape& s, const PrefillArgs& a, const QkvMaps& maps,
+                           uint32_t tmem, int h, int64_t bos, int64_t eos, int nchunks, size_t state_off) {
   const int j = threadIdx.x;  // TMEM lane == dv row of S^T
   const int warp = threadIdx.x >> 5;
   const uint32_t tl = tmem + ((uint32_t)((warp & 3) * 32) << 16);
@@ -606,17 +646,28 @@ __device__ void state_role(const Smem& sm, const PrefillShape& s, const PrefillA
         tc::tmem_ld16(tl + COL_O1 + hq * 32 + q * 16, o1 + 16 * q);
         tc::tmem_ld16(tl + COL_O2 + hq * 32 + q * 16, o2 + 16 * q);
       }
+      float4 gm[8];
+#pragma unroll
+      for (int q = 0; q < 8; ++q) gm[q] = *reinterpret_cast<const float4*>(vec + V_GAM + hq * 32 + 4 * q);
       tc::wait_ld();
 #pragma unroll
-      for (int x = 0; x < 32; ++x) {
-        const int r = hq * 32 + x;
-        store_out(stage + r * D + j, sc * fmaf(vec[V_GAM + r], o1[x], o2[x]));
+      for (int q = 0; q < 8; ++q) {
+        const int r = hq * 32 + 4 * q;
+        store_out(stage + (r + 0) * D + j, sc * fmaf(gm[q].x, o1[4 * q + 0], o2[4 * q + 0]));
+        store_out(stage + (r + 1) * D + j, sc * fmaf(gm[q].y, o1[4 * q + 1], o2[4 * q + 1]));
+        store_out(stage + (r + 2) * D + j, sc * fmaf(gm[q].z, o1[4 * q + 2], o2[4 * q + 2]));
+        store_out(stage + (r + 3) * D + j, sc * fmaf(gm[q].w, o1[4 * q + 3], o2[4 * q + 3]));
       }
     }
     tc::fence_proxy_async_smem();
     tc::fence_before_sync();
     tc::named_sync(kBarState, 128);
-    if (j < 32) {
+    if (Lc == C) {  // a full chunk: one tensor store of the [64 tokens][128] tile
+      if (j == 0) {
+        tc::tma_store_3d(&maps.o, 0, h, (int)t0, tc::smem_u32(stage));
+        tc::bulk_commit();
+      }
+    } else if (j < 32) {  // the last, partial chunk: row by row
       for (int r = j; r < Lc; r += 32)
         tc::bulk_store(op + ((size_t)(t0 + r) * s.H + h) * D, tc::smem_u32(stage + r * D), kRowBytes);
       tc::bulk_commit();
@@ -761,7 +812,7 @@ gdn_prefill_fused_kernel(const PrefillShape s, const PrefillArgs a, const __grid
   const uint32_t tmem = *sm.tmem_slot();
 
   if (warp < kPrepWarp0) {
-    state_role<TOut>(sm, s, a, tmem, h, bos, eos, nchunks, state_off);
+    state_role<TOut>(sm, s, a, maps, tmem, h, bos, eos, nchunks, state_off);
   } else if (warp < kLoadWarp0) {
     prep_role(sm, tmem, nchunks, a.err);
   } else if (warp < kMmaWarp) {
@@ -802,6 +853,16 @@ gdn_status_t launch(const PrefillShape& s, const PrefillArgs& a, cudaStream_t st
                                                  "fused prefill");
       if (st != GDN_OK) return st;
     }
+  }
+  if (a.o != nullptr && s.total_T > 0) {
+    constexpr bool kBf16Out = std::is_same<TOut, __nv_bfloat16>::value;
+    const uint64_t dims[3] = {(uint64_t)D, (uint64_t)s.H, (uint64_t)s.total_T};
+    const uint64_t strides[2] = {(uint64_t)D * sizeof(TOut), (uint64_t)s.H * D * sizeof(TOut)};
+    const uint32_t box[3] = {(uint32_t)D, 1, (uint32_t)C};
+    const gdn_status_t st =
+        make_tensor_map_3d(&maps.o, kBf16Out ? CU_TENSOR_MAP_DATA_TYPE_BFLOAT16 : CU_TENSOR_MAP_DATA_TYPE_FLOAT32, a.o,
+                           dims, strides, box, "fused prefill", CU_TENSOR_MAP_SWIZZLE_NONE);
+    if (st != GDN_OK) return st;
   }
   gdn_prefill_fused_kernel<TIn, TOut><<<grid, kThreads, SMEM_BYTES, stream>>>(s, a, maps);
   return check_launch("gdn_chunk_prefill (fused)");

@@ -32,7 +32,7 @@ gdn_status_t encode_tiled(EncodeTiledFn* fn) {
 
 gdn_status_t make_tensor_map_3d(CUtensorMap* map, CUtensorMapDataType type, const void* base,
                                 const uint64_t dims[3], const uint64_t strides[2], const uint32_t box[3],
-                                const char* what) {
+                                const char* what, CUtensorMapSwizzle swizzle) {
   EncodeTiledFn encode = nullptr;
   const gdn_status_t st = encode_tiled(&encode);
   if (st != GDN_OK) return st;
@@ -41,7 +41,7 @@ gdn_status_t make_tensor_map_3d(CUtensorMap* map, CUtensorMapDataType type, cons
   const cuuint32_t b[3] = {box[0], box[1], box[2]};
   const cuuint32_t e[3] = {1, 1, 1};
   const CUresult r = encode(map, type, 3, const_cast<void*>(base), d, s, b, e, CU_TENSOR_MAP_INTERLEAVE_NONE,
-                            CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
+                            swizzle, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
                             CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
   if (r != CUDA_SUCCESS)
     return fail(GDN_ERR_CUDA, std::string(what) + ": cuTensorMapEncodeTiled failed (CUresult " +
