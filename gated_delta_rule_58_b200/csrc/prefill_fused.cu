@@ -351,46 +351,77 @@ __device__ __forceinline__ void warp_block_store(float* M, int r0, int c0, float
   }
 }
 
-// T = (I + A)^{-1} for the strictly lower 64x64 A (fp32). The four 16x16 diagonal
-// blocks are inverted by forward substitution (one thread per column); the
-// off-diagonal blocks follow level by level, T_ij = -T_ii sum_{k=j}^{i-1} A_ik T_kj,
-// one warp per block, on tf32 warp MMAs. X_ij is parked in the diagonal block
-// A_ii, which the solve no longer reads.
-__device__ __forceinline__ void solve_unit_lower(const Smem& sm, int t) {
+// T = (I + A)^{-1} for the strictly lower 64x64 A (fp32), in two parts.
+//
+// solve_local (warps 4 and 5, right after each wrote its 32 rows of A): the two
+// 16x16 diagonal blocks of the warp's rows are inverted by forward substitution,
+// then merged into the inverse of the warp's 32x32 diagonal block,
+// T_10 = -T_11 (A_10 T_00) (or T_32 for warp 5), on tf32 warp MMAs. Only the
+// warp's own rows are read, so __syncwarp orders the steps.
+//
+// Forward substitution by rows, in registers: thread t owns row r = t % 16 of
+// block b = t / 16 (its A row), starting from e_r. At step k row k is final; its
+// first k+1 entries (the rest are zero) are broadcast by shuffles from lane k of
+// the half-warp and every later row subtracts A_rk times it.
+__device__ __forceinline__ void solve_local(const Smem& sm, int t) {
   float* A = sm.A();
   float* T = sm.T();
-  if (t < C) {
-    // column c of the inverse of diagonal block b, column-oriented: once x_k is
-    // known it is folded into every later row, so each step waits on one FMA
-    const int b = t >> 4, c = t & 15;
-    float x[16], acc[16];
+  {
+    const int b = t >> 4, r = t & 15, hl = threadIdx.x & 16;
+    float arow[16], trow[16];
 #pragma unroll
-    for (int r = 0; r < 16; ++r) acc[r] = 0.f;
-#pragma unroll
-    for (int k = 0; k < 16; ++k) {
-      x[k] = (k < c) ? 0.f : ((k == c) ? 1.f : -acc[k]);
-#pragma unroll
-      for (int r = k + 1; r < 16; ++r) acc[r] = fmaf(A[sidx(16 * b + r, 16 * b + k)], x[k], acc[r]);
+    for (int q = 0; q < 4; ++q) {
+      const float4 a4 = *row_chunk(A, 16 * b + r, 4 * b + q);
+      arow[4 * q + 0] = a4.x; arow[4 * q + 1] = a4.y; arow[4 * q + 2] = a4.z; arow[4 * q + 3] = a4.w;
     }
 #pragma unroll
-    for (int r = 0; r < 16; ++r) T[sidx(16 * b + r, 16 * b + c)] = x[r];
+    for (int m = 0; m < 16; ++m) trow[m] = (m == r) ? 1.f : 0.f;
+#pragma unroll
+    for (int k = 0; k < 15; ++k) {
+      const float lk = (k < r) ? arow[k] : 0.f;  // A_rk for the later rows only
+#pragma unroll
+      for (int m = 0; m <= k; ++m) {
+        const float rk = __shfl_sync(0xffffffffu, trow[m], hl | k);
+        trow[m] = fmaf(-lk, rk, trow[m]);
+      }
+    }
+#pragma unroll
+    for (int q = 0; q < 4; ++q)
+      *row_chunk(T, 16 * b + r, 4 * b + q) =
+          make_float4(trow[4 * q + 0], trow[4 * q + 1], trow[4 * q + 2], trow[4 * q + 3]);
   }
-  tc::named_sync(kBarPrep, 128);
+  __syncwarp();
+  const int wl = t >> 5, lane = t & 31;
+  const int i = 2 * wl + 1, j = 2 * wl;
+  float acc[2][4] = {{0.f, 0.f, 0.f, 0.f}, {0.f, 0.f, 0.f, 0.f}};
+  warp_block_mma(acc, A, 16 * i, 16 * j, T, 16 * j, 16 * j, lane);
+  warp_block_store(A, 16 * i, 16 * i, acc, 1.f, lane);  // X = A_ij T_jj parked in A_ii (no longer read)
+  __syncwarp();
+  float y[2][4] = {{0.f, 0.f, 0.f, 0.f}, {0.f, 0.f, 0.f, 0.f}};
+  warp_block_mma(y, T, 16 * i, 16 * i, A, 16 * i, 16 * i, lane);
+  warp_block_store(T, 16 * i, 16 * j, y, -1.f, lane);
+}
+
+// solve_merge (all four prep warps, after a barrier): the bottom-left 32x32 block,
+// T_BL = -T_bot (A_BL T_top), one 16x16 output block per warp and stage. The
+// intermediate Y = A_BL T_top is parked in the four diagonal blocks of A.
+__device__ __forceinline__ void solve_merge(const Smem& sm, int t) {
+  float* A = sm.A();
+  float* T = sm.T();
   const int w = t >> 5, lane = t & 31;
-#pragma unroll 1
-  for (int d = 1; d < 4; ++d) {
-    if (w < 4 - d) {
-      const int i = d + w, j = i - d;
-      float acc[2][4] = {{0.f, 0.f, 0.f, 0.f}, {0.f, 0.f, 0.f, 0.f}};
-      for (int k = j; k < i; ++k) warp_block_mma(acc, A, 16 * i, 16 * k, T, 16 * k, 16 * j, lane);
-      warp_block_store(A, 16 * i, 16 * i, acc, 1.f, lane);  // X_ij parked in A_ii
-      __syncwarp();
-      float y[2][4] = {{0.f, 0.f, 0.f, 0.f}, {0.f, 0.f, 0.f, 0.f}};
-      warp_block_mma(y, T, 16 * i, 16 * i, A, 16 * i, 16 * i, lane);
-      warp_block_store(T, 16 * i, 16 * j, y, -1.f, lane);
-    }
-    tc::named_sync(kBarPrep, 128);
+  const int i = 2 + (w >> 1), j = w & 1;
+  float acc[2][4] = {{0.f, 0.f, 0.f, 0.f}, {0.f, 0.f, 0.f, 0.f}};
+  for (int k = j; k < 2; ++k) warp_block_mma(acc, A, 16 * i, 16 * k, T, 16 * k, 16 * j, lane);  // Y_ij
+  const int p = 2 * (i - 2) + j;
+  warp_block_store(A, 16 * p, 16 * p, acc, 1.f, lane);
+  tc::named_sync(kBarPrep, 128);
+  float y[2][4] = {{0.f, 0.f, 0.f, 0.f}, {0.f, 0.f, 0.f, 0.f}};
+  for (int k = 2; k <= i; ++k) {
+    const int pk = 2 * (k - 2) + j;
+    warp_block_mma(y, T, 16 * i, 16 * k, A, 16 * pk, 16 * pk, lane);  // T_ik Y_kj
   }
+  warp_block_store(T, 16 * i, 16 * j, y, -1.f, lane);
+  tc::named_sync(kBarPrep, 128);
 }
 
 __device__ void prep_role(const Smem& sm, uint32_t tmem, int nchunks, unsigned int* err) {
@@ -482,8 +513,9 @@ __device__ void prep_role(const Smem& sm, uint32_t tmem, int nchunks, unsigned i
         }
       }
     }
+    if (t < C) solve_local(sm, t);  // warps 4 and 5: their own 32x32 diagonal blocks
     tc::named_sync(kBarPrep, 128);
-    solve_unit_lower(sm, t);
+    solve_merge(sm, t);
     // T diag(beta gamma) and T diag(beta) as fp16 (the previous chunk's W/U~ MMA
     // finished reading them: B_M2 of chunk c-1 was waited before E3 of chunk c-1)
     {
