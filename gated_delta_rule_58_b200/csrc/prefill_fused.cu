@@ -72,9 +72,9 @@ constexpr uint32_t OFF_P16 = 163840;    // 2 buffers: P [64][64] fp16 (K-major B
 constexpr uint32_t P_BUF = 8192;
 constexpr uint32_t OFF_A = 180224;      // A fp32 [64][64], 16-byte chunks XOR-swizzled by row
 constexpr uint32_t OFF_T = 196608;      // T fp32 [64][64], same swizzle
-constexpr uint32_t OFF_VEC = 212992;    // 2 buffers x {G, gamma, dd, beta, beta*gamma} x 64 fp32
+constexpr uint32_t OFF_VEC = 212992;    // 3 buffers (chunk % 3) x {G, gamma, dd, beta, beta*gamma} x 64 fp32
 constexpr uint32_t VEC_BUF = 5 * C * 4;
-constexpr uint32_t OFF_BAR = OFF_VEC + 2 * VEC_BUF;
+constexpr uint32_t OFF_BAR = OFF_VEC + 3 * VEC_BUF;
 constexpr uint32_t SMEM_USED = OFF_BAR + 256;
 constexpr uint32_t SMEM_BYTES = SMEM_USED + 1024;  // slack for the 1024-byte alignment
 
@@ -92,6 +92,7 @@ constexpr uint32_t TMEM_COLS = 512;
 enum Bar : int {
   B_L0 = 0, B_L1,      // loader -> chunk tiles ready (per buffer)
   B_T0, B_T1,          // TMA -> raw bf16 tiles landed (per buffer)
+  B_LC0, B_LC1,        // loader -> fp16 tiles converted (per buffer)
   B_M1,                // MMA: D1 ready
   B_M2,                // MMA: W^T, U~^T ready
   B_M3A,               // MMA: U^T ready (S16, W16 consumed)
@@ -200,12 +201,12 @@ __device__ void loader_role(const Smem& sm, const PrefillShape& s, const Prefill
   }
   for (int c = 0; c < nchunks; ++c) {
     const int b = c & 1;
-    // chunk c-2 (same buffers) fully consumed: its outputs were read, so every
-    // MMA of that chunk, including the ones reading K, Q and V, has completed
-    if (c >= 2 && !wait_bar(sm, B_E6B, (c - 2) & 1, a.err)) return;
+    // chunk c-2 (same tile buffers) no longer reads K, Q or V: its state update,
+    // the last MMA to read them, has completed (so have the earlier ones)
+    if (c >= 2 && !wait_bar(sm, B_M4B, (c - 2) & 1, a.err)) return;
     const int64_t t0 = bos + (int64_t)c * C;
     const int Lc = (int)((eos - t0) < C ? (eos - t0) : C);
-    float* vec = sm.vec(b);
+    float* vec = sm.vec(c % 3);  // three gate buffers: chunk c-2's output epilogue may still read its own
     uint8_t* kq = sm.base + OFF_KQ + b * KQ_BUF;
     uint8_t* v16 = sm.base + OFF_V + b * V_BUF;
     if constexpr (kTma) {
@@ -257,8 +258,12 @@ __device__ void loader_role(const Smem& sm, const PrefillShape& s, const Prefill
     }
     tc::named_sync(kBarLoad, 128);
     if constexpr (kTma) {
+      // the raw bf16 tiles feed [K;Q] K^T directly (bf16 MMA, exact inputs); they
+      // are converted to fp16 in place once that MMA has read them
       if (!wait_bar(sm, B_T0 + b, (c >> 1) & 1, a.err)) return;
-      // in place to fp16 (the queries stay unscaled: P is taken from Q K^T)
+      group_signal(sm, kBarLoad, B_L0 + b);
+      if (!wait_bar(sm, B_M1, c & 1, a.err)) return;
+      tc::fence_after_sync();
 #pragma unroll 4
       for (int i = t; i < 3 * C * 16; i += 128) {
         const int mat = i >> 10, rem = i & 1023;  // 0 K, 1 Q, 2 V; 64 rows x 16 chunks each
@@ -289,8 +294,9 @@ __device__ void loader_role(const Smem& sm, const PrefillShape& s, const Prefill
           st_sw128_chunk(base + (ch >> 3) * half, row + roff, ch & 7, v8);
         }
       }
+      group_signal(sm, kBarLoad, B_L0 + b);
     }
-    group_signal(sm, kBarLoad, B_L0 + b);
+    group_signal(sm, kBarLoad, B_LC0 + b);
   }
 }
 
@@ -436,7 +442,7 @@ __device__ void prep_role(const Smem& sm, uint32_t tmem, int nchunks, unsigned i
     if (!wait_bar(sm, B_L0 + b, (c >> 1) & 1, err)) return;
     if (!wait_bar(sm, B_M1, c & 1, err)) return;
     tc::fence_after_sync();
-    const float* vec = sm.vec(b);
+    const float* vec = sm.vec(c % 3);
     const float* G = vec + V_G;
     if (t < C) {
       // A row t (rows 0-63 of D1): beta_t exp(G_t - G_j) k_t.k_j for j < t; the
@@ -601,7 +607,7 @@ __device__ void state_role(const Smem& sm, const PrefillShape& s, const PrefillA
 
   for (int c = 0; c < nchunks; ++c) {
     const int b = c & 1;
-    const float* vec = sm.vec(b);
+    const float* vec = sm.vec(c % 3);
     const int64_t t0 = bos + (int64_t)c * C;
     const int Lc = (int)((eos - t0) < C ? (eos - t0) : C);
     // E5: U^T -> fp16 tiles (after the previous chunk's output stores read the stage)
@@ -634,7 +640,7 @@ __device__ void state_role(const Smem& sm, const PrefillShape& s, const PrefillA
     float gnext = 1.f;
     if (!last) {
       if (!wait_bar(sm, B_L0 + (b ^ 1), ((c + 1) >> 1) & 1, a.err)) return;
-      gnext = sm.vec(b ^ 1)[V_GAM + C - 1];
+      gnext = sm.vec((c + 1) % 3)[V_GAM + C - 1];
     }
 #pragma unroll
     for (int hq = 0; hq < 4; ++hq) {
@@ -711,10 +717,10 @@ __device__ void state_role(const Smem& sm, const PrefillShape& s, const PrefillA
 
 // ---------------------------------------------------------------- mma role
 
-// D1 = [K;Q] K^T for chunk buffer b.
-__device__ __forceinline__ void issue_m1(const Smem& sm, uint32_t tmem, int b) {
+// D1 = [K;Q] K^T for chunk buffer b (raw bf16 tiles, or fp16 ones for fp32 inputs).
+__device__ __forceinline__ void issue_m1(const Smem& sm, uint32_t tmem, int b, int raw_bf16) {
   const uint32_t kq = sm.u32(OFF_KQ + b * KQ_BUF);
-  const uint32_t id = tc::idesc_f16(128, 64, 0, 0);
+  const uint32_t id = tc::idesc_f16(128, 64, 0, 0, 0, raw_bf16);
 #pragma unroll
   for (int ks = 0; ks < 8; ++ks) {
     const uint32_t off = (ks >> 2) * KQ_HALF + (ks & 3) * 32;
@@ -739,7 +745,7 @@ __device__ __forceinline__ void issue_m2(const Smem& sm, uint32_t tmem, int b) {
   tc::mma_commit(sm.bar(B_M2));
 }
 
-__device__ void mma_role(const Smem& sm, uint32_t tmem, int nchunks, unsigned int* err) {
+__device__ void mma_role(const Smem& sm, uint32_t tmem, int nchunks, int raw_bf16, unsigned int* err) {
   const uint32_t w16 = sm.u32(OFF_W16), u16 = sm.u32(OFF_U16), udd = sm.u32(OFF_UDD);
   const uint32_t p16 = sm.u32(OFF_P16);
   const uint32_t id_u = tc::idesc_f16(128, 64, 0, 1, 1);
@@ -748,8 +754,9 @@ __device__ void mma_role(const Smem& sm, uint32_t tmem, int nchunks, unsigned in
 
   if (!wait_bar(sm, B_L0, 0, err)) return;
   tc::fence_after_sync();
-  issue_m1(sm, tmem, 0);
+  issue_m1(sm, tmem, 0, raw_bf16);
   if (!wait_bar(sm, B_E2, 0, err)) return;
+  if (!wait_bar(sm, B_LC0, 0, err)) return;
   tc::fence_after_sync();
   issue_m2(sm, tmem, 0);
   for (int c = 0; c < nchunks; ++c) {
@@ -758,7 +765,7 @@ __device__ void mma_role(const Smem& sm, uint32_t tmem, int nchunks, unsigned in
     if (c + 1 < nchunks) {
       if (!wait_bar(sm, B_L0 + (b ^ 1), ((c + 1) >> 1) & 1, err)) return;
       tc::fence_after_sync();
-      issue_m1(sm, tmem, b ^ 1);
+      issue_m1(sm, tmem, b ^ 1, raw_bf16);
     }
     // M3a: U^T -= S^T W^T (A = fp16 state from TMEM)
     if (!wait_bar(sm, B_E3, c & 1, err)) return;
@@ -792,6 +799,7 @@ __device__ void mma_role(const Smem& sm, uint32_t tmem, int nchunks, unsigned in
     // M2 of the next chunk
     if (c + 1 < nchunks) {
       if (!wait_bar(sm, B_E2, (c + 1) & 1, err)) return;
+      if (!wait_bar(sm, B_LC0 + (b ^ 1), ((c + 1) >> 1) & 1, err)) return;
       tc::fence_after_sync();
       issue_m2(sm, tmem, b ^ 1);
     }
@@ -850,7 +858,7 @@ gdn_prefill_fused_kernel(const PrefillShape s, const PrefillArgs a, const __grid
   } else if (warp < kMmaWarp) {
     loader_role<TIn>(sm, s, a, maps, h, bos, eos, nchunks);
   } else if ((threadIdx.x & 31) == 0) {
-    mma_role(sm, tmem, nchunks, a.err);
+    mma_role(sm, tmem, nchunks, std::is_same<TIn, __nv_bfloat16>::value ? 1 : 0, a.err);
   }
 
   // teardown: every role finished (all MMAs were waited on by the state role)

@@ -95,11 +95,11 @@ __device__ __forceinline__ uint32_t sw128_offset(uint32_t row, uint32_t chunk, u
   return (row >> 3) * sbo + (row & 7u) * 128u + ((chunk ^ (row & 7u)) << 4);
 }
 
-// Instruction descriptor, kind::f16 with fp16 A/B and fp32 D.
+// Instruction descriptor, kind::f16 with fp16 (or, with ab_bf16, bf16) A and B and fp32 D.
 // a_mn / b_mn: operand is MN-major (1) or K-major (0); neg_a negates A.
-__host__ __device__ constexpr uint32_t idesc_f16(int M, int N, int a_mn, int b_mn, int neg_a = 0) {
-  return (1u << 4)                      // D format: f32
-         | (0u << 7) | (0u << 10)       // A, B format: f16
+__host__ __device__ constexpr uint32_t idesc_f16(int M, int N, int a_mn, int b_mn, int neg_a = 0, int ab_bf16 = 0) {
+  return (1u << 4)                                              // D format: f32
+         | ((uint32_t)ab_bf16 << 7) | ((uint32_t)ab_bf16 << 10)  // A, B format: f16 (0) or bf16 (1)
          | ((uint32_t)neg_a << 13)
          | ((uint32_t)a_mn << 15) | ((uint32_t)b_mn << 16)
          | ((uint32_t)(N >> 3) << 17)
