@@ -27,15 +27,18 @@
 // Warp specialisation (13 warps) and the chunk pipeline:
 //   loader  (warps 8-11): TMA tensor loads of chunk c's q/k/v rows (bf16) straight
 //            into the 128-byte-swizzled MMA tiles, g/beta, the cumulative gates
-//            and decays, then the in-place conversion to fp16. fp32 inputs are
-//            loaded and converted by the threads instead.
-//            Runs up to one chunk ahead.
+//            and decays; once [K;Q]K^T has read the raw tiles, their in-place
+//            conversion to fp16. fp32 inputs are loaded and converted by the
+//            threads instead. Runs up to two chunks ahead.
 //   prep    (warps 4-7):  A and P from [K;Q]K^T, the triangular solve, the fp16
-//            T diag(beta gamma) / T diag(beta) tiles, then W^T -> fp16 tile.
-//            Works on chunk c+1 while the state warps finish chunk c.
-//   state   (warps 0-3):  U^T -> fp16 tiles, the new state -> fp16 TMEM operand
-//            (and the gamma_C rescale of the fp32 TMEM state), outputs -> HBM.
-//   mma     (warp 12):    one thread issues every tcgen05.mma in dependency order.
+//            T diag(beta gamma) / T diag(beta) tiles. Works on chunk c+1 while
+//            the state warps finish chunk c.
+//   state   (warps 0-3):  W^T -> fp16 tile, U^T -> fp16 tiles, the new state ->
+//            fp16 TMEM operand (and the gamma_C rescale of the fp32 TMEM state),
+//            outputs -> HBM.
+//   mma     (warp 12):    one thread issues every tcgen05.mma in dependency order;
+//            the next chunk's [K;Q]K^T goes first, as soon as its tiles are in and
+//            the prep warps have read this chunk's.
 // Hand-offs are mbarriers: tcgen05.commit for MMA completion, one elected arrive
 // per warpgroup (after a named barrier) for thread-produced tiles. Every wait is
 // bounded; a timeout sets GDN_DEVERR_TIMEOUT and unwinds all roles.
@@ -98,8 +101,9 @@ enum Bar : int {
   B_M3A,               // MMA: U^T ready (S16, W16 consumed)
   B_M4B,               // MMA: new state ready
   B_M4A,               // MMA: O2 ready (all chunk MMAs done)
-  B_E2,                // prep: T', T'', P ready, D1 buffer consumed
-  B_E3,                // prep: W16 ready, W region consumed
+  B_E1,                // prep: D1 consumed (one arrival per prep warp)
+  B_E2,                // prep: T', T'', P ready
+  B_E3,                // state: W16 ready, W region consumed
   B_E5,                // state: U16/UDD ready, U region consumed
   B_E6A,               // state: S16 ready, TMEM state rescaled
   B_E6B,               // state: O1/O2 consumed
@@ -519,11 +523,16 @@ __device__ void prep_role(const Smem& sm, uint32_t tmem, int nchunks, unsigned i
         }
       }
     }
+    // this warp's reads of D1 are complete: the next chunk's [K;Q]K^T may overwrite it
+    tc::fence_before_sync();
+    __syncwarp();
+    if ((t & 31) == 0) tc::mbar_arrive(sm.bar(B_E1));
     if (t < C) solve_local(sm, t);  // warps 4 and 5: their own 32x32 diagonal blocks
     tc::named_sync(kBarPrep, 128);
     solve_merge(sm, t);
-    // T diag(beta gamma) and T diag(beta) as fp16 (the previous chunk's W/U~ MMA
-    // finished reading them: B_M2 of chunk c-1 was waited before E3 of chunk c-1)
+    // T diag(beta gamma) and T diag(beta) as fp16, once the previous chunk's W/U~
+    // MMA has read the old ones
+    if (c >= 1 && !wait_bar(sm, B_M2, (c - 1) & 1, err)) return;
     {
       const int mat = t >> 6, i = t & 63;
       const float* colscale = vec + (mat ? V_BETA : V_BG);
@@ -542,20 +551,6 @@ __device__ void prep_role(const Smem& sm, uint32_t tmem, int nchunks, unsigned i
       }
     }
     group_signal(sm, kBarPrep, B_E2);
-    // W^T -> fp16 once the W MMA is done and the previous chunk's M3a read W16
-    if (!wait_bar(sm, B_M2, c & 1, err)) return;
-    if (c >= 1 && !wait_bar(sm, B_M3A, (c - 1) & 1, err)) return;
-    tc::fence_after_sync();
-#pragma unroll
-    for (int hq = 0; hq < 2; ++hq) {
-      float w[32];
-      tc::tmem_ld16(tl + COL_W + hq * 32, w);
-      tc::tmem_ld16(tl + COL_W + hq * 32 + 16, w + 16);
-      tc::wait_ld();
-#pragma unroll
-      for (int q = 0; q < 4; ++q) st_sw128_chunk(sm.base + OFF_W16, t, 4 * hq + q, w + 8 * q);
-    }
-    group_signal(sm, kBarPrep, B_E3);
   }
 }
 
@@ -610,6 +605,20 @@ __device__ void state_role(const Smem& sm, const PrefillShape& s, const PrefillA
     const float* vec = sm.vec(c % 3);
     const int64_t t0 = bos + (int64_t)c * C;
     const int Lc = (int)((eos - t0) < C ? (eos - t0) : C);
+    // E3: W^T -> fp16 tile once the W MMA is done (W16's previous reader, chunk
+    // c-1's U MMA, completed before E5 of chunk c-1)
+    if (!wait_bar(sm, B_M2, c & 1, a.err)) return;
+    tc::fence_after_sync();
+#pragma unroll
+    for (int hq = 0; hq < 2; ++hq) {
+      float w[32];
+      tc::tmem_ld16(tl + COL_W + hq * 32, w);
+      tc::tmem_ld16(tl + COL_W + hq * 32 + 16, w + 16);
+      tc::wait_ld();
+#pragma unroll
+      for (int q = 0; q < 4; ++q) st_sw128_chunk(sm.base + OFF_W16, j, 4 * hq + q, w + 8 * q);
+    }
+    group_signal(sm, kBarState, B_E3);
     // E5: U^T -> fp16 tiles (after the previous chunk's output stores read the stage)
     if (!wait_bar(sm, B_M3A, c & 1, a.err)) return;
     if (c >= 1) {
@@ -755,18 +764,21 @@ __device__ void mma_role(const Smem& sm, uint32_t tmem, int nchunks, int raw_bf1
   if (!wait_bar(sm, B_L0, 0, err)) return;
   tc::fence_after_sync();
   issue_m1(sm, tmem, 0, raw_bf16);
-  if (!wait_bar(sm, B_E2, 0, err)) return;
-  if (!wait_bar(sm, B_LC0, 0, err)) return;
-  tc::fence_after_sync();
-  issue_m2(sm, tmem, 0);
   for (int c = 0; c < nchunks; ++c) {
     const int b = c & 1;
     const uint32_t kq = sm.u32(OFF_KQ + b * KQ_BUF);
+    // M1 of the next chunk as soon as its tiles are in and this chunk's D1 was read
     if (c + 1 < nchunks) {
       if (!wait_bar(sm, B_L0 + (b ^ 1), ((c + 1) >> 1) & 1, err)) return;
+      if (!wait_bar(sm, B_E1, c & 1, err)) return;
       tc::fence_after_sync();
       issue_m1(sm, tmem, b ^ 1, raw_bf16);
     }
+    // M2: W^T, U~^T of this chunk
+    if (!wait_bar(sm, B_E2, c & 1, err)) return;
+    if (!wait_bar(sm, B_LC0 + b, (c >> 1) & 1, err)) return;
+    tc::fence_after_sync();
+    issue_m2(sm, tmem, b);
     // M3a: U^T -= S^T W^T (A = fp16 state from TMEM)
     if (!wait_bar(sm, B_E3, c & 1, err)) return;
     if (!wait_bar(sm, B_E6A, c & 1, err)) return;
@@ -796,13 +808,6 @@ __device__ void mma_role(const Smem& sm, uint32_t tmem, int nchunks, int raw_bf1
       tc::mma_f16(tmem + COL_O2, tc::sw128_desc(u16 + ks * 32, 16, 1024),
                   tc::sw128_desc(p16 + b * P_BUF + ks * 32, 16, 1024), id_o, ks > 0);
     tc::mma_commit(sm.bar(B_M4A));
-    // M2 of the next chunk
-    if (c + 1 < nchunks) {
-      if (!wait_bar(sm, B_E2, (c + 1) & 1, err)) return;
-      if (!wait_bar(sm, B_LC0 + (b ^ 1), ((c + 1) >> 1) & 1, err)) return;
-      tc::fence_after_sync();
-      issue_m2(sm, tmem, b ^ 1);
-    }
   }
 }
 
@@ -842,7 +847,7 @@ gdn_prefill_fused_kernel(const PrefillShape s, const PrefillArgs a, const __grid
     tc::tmem_relinquish();
   }
   if (threadIdx.x == 0) {
-    for (int i = 0; i < B_COUNT; ++i) tc::mbar_init(sm.bar(i), 1);
+    for (int i = 0; i < B_COUNT; ++i) tc::mbar_init(sm.bar(i), i == B_E1 ? 4 : 1);
     *sm.abort_flag() = 0;
     tc::fence_mbar_init();
   }
