@@ -127,8 +127,7 @@ gdn_decode_kernel(const DecodeParams p, const __grid_constant__ CUtensorMap pool
   constexpr uint32_t kBarConsumers = 1;
 
   extern __shared__ uint8_t smem_raw[];
-  uint8_t* base = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + L::kAlign - 1) &
-                                             ~uintptr_t(L::kAlign - 1));
+  uint8_t* base = tc::align_smem<L::kAlign>(smem_raw);
   float* vecf = reinterpret_cast<float*>(base + NS * L::kBytes);  // [NV][DK] fp32 of the current item
   uint64_t* full = reinterpret_cast<uint64_t*>(base + NS * L::kBytes + L::kVecF32);
   uint64_t* empty = full + NS;

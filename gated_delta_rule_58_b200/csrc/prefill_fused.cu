@@ -534,19 +534,25 @@ __device__ void prep_role(const Smem& sm, uint32_t tmem, int nchunks, unsigned i
     // MMA has read the old ones
     if (c >= 1 && !wait_bar(sm, B_M2, (c - 1) & 1, err)) return;
     {
+      // row i of T times the column scales; the row and the scales are loaded
+      // up front (independent loads), the upper part is written as zeros
       const int mat = t >> 6, i = t & 63;
       const float* colscale = vec + (mat ? V_BETA : V_BG);
       uint8_t* tile = sm.base + (mat ? OFF_TPP : OFF_TP);
+      float4 tr[16], cs[16];
+#pragma unroll
+      for (int q = 0; q < 16; ++q) {
+        tr[q] = *row_chunk(sm.T(), i, q);
+        cs[q] = *reinterpret_cast<const float4*>(colscale + 4 * q);
+      }
 #pragma unroll
       for (int cc = 0; cc < 8; ++cc) {
-        const float4 lo = *row_chunk(sm.T(), i, 2 * cc), hi = *row_chunk(sm.T(), i, 2 * cc + 1);
-        const float tv[8] = {lo.x, lo.y, lo.z, lo.w, hi.x, hi.y, hi.z, hi.w};
+        const float4 a0 = tr[2 * cc], a1 = tr[2 * cc + 1], s0 = cs[2 * cc], s1 = cs[2 * cc + 1];
+        const float prod[8] = {a0.x * s0.x, a0.y * s0.y, a0.z * s0.z, a0.w * s0.w,
+                               a1.x * s1.x, a1.y * s1.y, a1.z * s1.z, a1.w * s1.w};
         float v[8];
 #pragma unroll
-        for (int m = 0; m < 8; ++m) {
-          const int j = cc * 8 + m;
-          v[m] = (j <= i) ? tv[m] * colscale[j] : 0.f;
-        }
+        for (int m = 0; m < 8; ++m) v[m] = (cc * 8 + m <= i) ? prod[m] : 0.f;
         st_sw128_chunk(tile, i, cc, v);
       }
     }
@@ -818,7 +824,7 @@ __global__ void __launch_bounds__(kThreads, 1)
 gdn_prefill_fused_kernel(const PrefillShape s, const PrefillArgs a, const __grid_constant__ QkvMaps maps) {
   extern __shared__ uint8_t smem_raw[];
   Smem sm;
-  sm.base = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
+  sm.base = tc::align_smem<1024>(smem_raw);
   const int warp = threadIdx.x >> 5;
   const int n = blockIdx.x / s.H;
   const int h = blockIdx.x - n * s.H;

@@ -13,6 +13,15 @@ __device__ __forceinline__ uint32_t smem_u32(const void* p) {
   return static_cast<uint32_t>(__cvta_generic_to_shared(p));
 }
 
+// The dynamic shared-memory array advanced to the next `align`-byte boundary by
+// pointer arithmetic on the array itself (not through an integer), so that the
+// compiler still sees a shared-memory pointer and emits shared-memory accesses.
+template <uint32_t kAlign>
+__device__ __forceinline__ uint8_t* align_smem(uint8_t* smem) {
+  const uint32_t a = smem_u32(smem);
+  return smem + ((kAlign - (a & (kAlign - 1u))) & (kAlign - 1u));
+}
+
 __device__ __forceinline__ uint64_t globaltimer_ns() {
   uint64_t t;
   asm volatile("mov.u64 %0, %%globaltimer;" : "=l"(t));
