@@ -58,6 +58,7 @@ constexpr int kThreads = 13 * 32;
 constexpr int kPrepWarp0 = 4, kLoadWarp0 = 8, kMmaWarp = 12;  // state warps are 0-3
 constexpr uint32_t kBarState = 1, kBarPrep = 2, kBarLoad = 3;  // named barrier ids
 constexpr uint64_t kWaitNs = 2000000000ull;                     // 2 s
+constexpr int kLptMaxSeqs = 64;  // longest-first launch order up to this many sequences
 
 // Shared memory map (bytes from a 1024-aligned base).
 constexpr uint32_t OFF_KQ = 0;          // 2 buffers: [2 dk halves][128 rows: K 0-63, Q 64-127][64] fp16
@@ -826,8 +827,40 @@ gdn_prefill_fused_kernel(const PrefillShape s, const PrefillArgs a, const __grid
   Smem sm;
   sm.base = tc::align_smem<1024>(smem_raw);
   const int warp = threadIdx.x >> 5;
-  const int n = blockIdx.x / s.H;
-  const int h = blockIdx.x - n * s.H;
+  const int rank = blockIdx.x / s.H;
+  const int h = blockIdx.x - rank * s.H;
+  // Longest sequence first: the CTAs of the rank-th longest sequence (ties by
+  // index) have the rank-th block indices, so long sequences start in the first
+  // wave and the last wave holds short ones. Each CTA ranks the lengths itself
+  // (one warp, O(N^2) compares on a shared-memory copy), so only for small N;
+  // beyond that the order is the sequence index. Results do not depend on it.
+  int n = rank;
+  if (s.N > 1 && s.N <= kLptMaxSeqs) {
+    int* lens = reinterpret_cast<int*>(sm.A());  // the A tile is free until the first chunk
+    for (int i = threadIdx.x; i < s.N; i += blockDim.x) {
+      const int32_t l = __ldg(a.cu_seqlens + i + 1) - __ldg(a.cu_seqlens + i);
+      lens[i] = l > 0 ? l : 0;
+    }
+    __syncthreads();
+    if (warp == 0) {
+      int found = -1;
+      for (int i = threadIdx.x; i < s.N; i += 32) {
+        const int li = lens[i];
+        int r = 0;
+        for (int j = 0; j < s.N; ++j) {
+          const int lj = lens[j];
+          r += (lj > li || (lj == li && j < i)) ? 1 : 0;
+        }
+        if (r == rank) found = i;
+      }
+#pragma unroll
+      for (int off = 16; off > 0; off >>= 1) found = max(found, __shfl_xor_sync(0xffffffffu, found, off));
+      if (threadIdx.x == 0) lens[kLptMaxSeqs] = found;
+    }
+    __syncthreads();
+    n = lens[kLptMaxSeqs];
+    __syncthreads();  // the A tile is reused below
+  }
   int64_t bos, eos;
   if (!seq_bounds(a.cu_seqlens, n, s.total_T, a.err, &bos, &eos)) return;
 
