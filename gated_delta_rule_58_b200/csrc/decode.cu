@@ -257,34 +257,54 @@ gdn_decode_kernel(const DecodeParams p, const __grid_constant__ CUtensorMap pool
       for (int e = tid * 4; e < NV * DK; e += kConsumers * 4)
         load4_f32<TIn>(st + L::kKeys + e * sizeof(TIn), vecf + e);
       tc::named_sync(kBarConsumers, kConsumers);
-      // per-head Gram entries k_m.k_l (l < m) and q_t.k_l, one warp per pair
+      // per-head Gram entries k_m.k_l (l < m) and q_t.k_l: warp w takes pairs w,
+      // w + W, ...; their partial sums are reduced together (independent shuffles)
       constexpr int kPairsKK = M * (M - 1) / 2;
       constexpr int kPairs = kPairsKK + TT * M;
-      for (int pair = warp; pair < kPairs; pair += kConsumers / 32) {  // one warp per pair
-        int va, vb;
-        if (pair < kPairsKK) {
-          va = 1;
-          int rem = pair;
-          while (rem >= va) { rem -= va; ++va; }
-          vb = rem;
-        } else {
-          const int x = pair - kPairsKK;
-          va = M + x / M;
-          vb = x - (x / M) * M;
-        }
-        const float* pa = vecf + va * DK;  // the queries follow the keys
-        const float* pb = vecf + vb * DK;
-        float acc = 0.f;
-        for (int e = lane * 4; e < DK; e += 128) {
-          const float4 xa = *reinterpret_cast<const float4*>(pa + e);
-          const float4 xb = *reinterpret_cast<const float4*>(pb + e);
-          acc = fmaf(xa.x, xb.x, fmaf(xa.y, xb.y, fmaf(xa.z, xb.z, fmaf(xa.w, xb.w, acc))));
-        }
+      constexpr int kWarps = kConsumers / 32;
+      constexpr int kPPW = (kPairs + kWarps - 1) / kWarps;
+      float gacc[kPPW];
 #pragma unroll
-        for (int off = 16; off > 0; off >>= 1) acc += __shfl_xor_sync(0xffffffffu, acc, off);
-        if (lane == 0) {
-          if (pair < kPairsKK) gram[va * M + vb] = acc;
-          else qk[(va - M) * M + vb] = acc;
+      for (int q = 0; q < kPPW; ++q) {
+        const int pair = warp + q * kWarps;
+        gacc[q] = 0.f;
+        if (pair < kPairs) {  // warp-uniform
+          int va, vb;
+          if (pair < kPairsKK) {
+            va = 1;
+            int rem = pair;
+            while (rem >= va) { rem -= va; ++va; }
+            vb = rem;
+          } else {
+            const int x = pair - kPairsKK;
+            va = M + x / M;
+            vb = x - (x / M) * M;
+          }
+          const float* pa = vecf + va * DK;  // the queries follow the keys
+          const float* pb = vecf + vb * DK;
+          for (int e = lane * 4; e < DK; e += 128) {
+            const float4 xa = *reinterpret_cast<const float4*>(pa + e);
+            const float4 xb = *reinterpret_cast<const float4*>(pb + e);
+            gacc[q] = fmaf(xa.x, xb.x, fmaf(xa.y, xb.y, fmaf(xa.z, xb.z, fmaf(xa.w, xb.w, gacc[q]))));
+          }
+        }
+      }
+#pragma unroll
+      for (int off = 16; off > 0; off >>= 1)
+#pragma unroll
+        for (int q = 0; q < kPPW; ++q) gacc[q] += __shfl_xor_sync(0xffffffffu, gacc[q], off);
+      if (lane == 0) {
+#pragma unroll
+        for (int q = 0; q < kPPW; ++q) {
+          const int pair = warp + q * kWarps;
+          if (pair < kPairsKK) {
+            int va = 1, rem = pair;
+            while (rem >= va) { rem -= va; ++va; }
+            gram[va * M + rem] = gacc[q];
+          } else if (pair < kPairs) {
+            const int x = pair - kPairsKK;
+            qk[(x / M) * M + (x - (x / M) * M)] = gacc[q];
+          }
         }
       }
       tc::named_sync(kBarConsumers, kConsumers);
