@@ -10,13 +10,26 @@ constexpr bool kTransferPrefillBuilt = true;
 
 gdn_prefill_algo_t prefill_auto_tensor_core(const PrefillShape& s) {
   if (!kTransferPrefillBuilt) return GDN_PREFILL_FUSED;
-  // Few (sequence, head) pairs with long sequences leave most SMs idle on the fused
-  // path (one chain of chunks per pair); the transfer path spreads the chunks of a
-  // chain over all SMs and leaves only the short fixup scan serial.
+  // Cost model in units of one chunk step of one CTA (the fused kernel's period).
+  // Fused: one CTA per (sequence, head) walks its chunks, so the time is the
+  // chunks per sequence (times the waves when the pairs exceed the SMs). Transfer:
+  // three passes of the same kernel over segments of G chunks (one wave of
+  // segment CTAs, or more when G is capped), plus a serial fixup scan whose step
+  // costs about 0.7 of a chunk step, plus the launches. The constants were
+  // measured on B200 (148 SMs). The average sequence length stands in for
+  // the lengths (they are on the device); transfer is taken only when it is
+  // clearly cheaper.
+  constexpr long long kSms = 148;
   const long long pairs = (long long)s.N * s.H;
-  const long long avg_len = s.N > 0 ? s.total_T / s.N : 0;
-  if (pairs <= 16 && avg_len >= 8192) return GDN_PREFILL_TRANSFER;
-  return GDN_PREFILL_FUSED;
+  if (pairs <= 0 || pairs > kSms || s.total_T <= 0) return GDN_PREFILL_FUSED;
+  const long long chunks = (s.total_T / s.N + 63) / 64;  // per sequence, average
+  const long long g = prefill_transfer_segment_chunks(s);
+  const long long seg_per_seq = (chunks + g - 1) / g;
+  const long long waves = (pairs * seg_per_seq + kSms - 1) / kSms;
+  // + about 7 chunk steps of fixed cost: the segment map and three kernel launches
+  const double transfer = 3.0 * (double)g * (double)waves + 0.7 * (double)seg_per_seq + 7.0;
+  const double fused = (double)chunks;
+  return transfer < 0.8 * fused ? GDN_PREFILL_TRANSFER : GDN_PREFILL_FUSED;
 }
 
 gdn_status_t prefill_resolve(const PrefillShape& s, gdn_dtype_t in, gdn_prefill_algo_t requested,

@@ -48,6 +48,8 @@ gdn_status_t prefill_launch(const PrefillShape& s, const PrefillArgs& a, gdn_pre
 gdn_status_t prefill_sequential_launch(const PrefillShape& s, const PrefillArgs& a, cudaStream_t stream);
 gdn_status_t prefill_fused_launch(const PrefillShape& s, const PrefillArgs& a, cudaStream_t stream);
 size_t prefill_transfer_workspace_bytes(const PrefillShape& s);
+// Chunks per segment (G) the transfer algorithm uses for this shape.
+int prefill_transfer_segment_chunks(const PrefillShape& s);
 gdn_status_t prefill_transfer_launch(const PrefillShape& s, const PrefillArgs& a, cudaStream_t stream);
 
 // Reads cu_seqlens[n], cu_seqlens[n+1] and validates them against total_T; on a bad

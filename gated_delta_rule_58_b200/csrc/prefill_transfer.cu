@@ -256,6 +256,8 @@ gdn_fixup_scan_kernel(const int32_t* seg_of_seq, int H, const float* local, cons
 
 size_t prefill_transfer_workspace_bytes(const PrefillShape& s) { return layout_for(s).total; }
 
+int prefill_transfer_segment_chunks(const PrefillShape& s) { return layout_for(s).seg_chunks; }
+
 gdn_status_t prefill_transfer_launch(const PrefillShape& s, const PrefillArgs& a, cudaStream_t stream) {
   const TransferLayout L = layout_for(s);
   uint8_t* ws = static_cast<uint8_t*>(a.workspace);

@@ -80,6 +80,20 @@ def _prefill(L, **kw):
                                a["scale"], a["din"], a["dout"], a["algo"], a["ws"], a["wsb"], a["stream"])
 
 
+def test_auto_choice_between_fused_and_transfer():
+    """AUTO follows the chunk-step cost model: transfer for few long chains, fused
+    when the pairs fill the GPU or the sequences are too short to pay for three
+    passes. The choice shows in the workspace query (0 for fused)."""
+    ws = gdn.gdn_chunk_prefill_workspace_size
+    A, T = gdn.GDN_PREFILL_AUTO, gdn.GDN_PREFILL_TRANSFER
+    for shape in [(1, 65536, 4), (1, 16384, 8), (2, 32768, 8), (1, 8192, 16)]:
+        N, total, H = shape
+        assert ws(N, total, H, 128, 128, 64, A) == ws(N, total, H, 128, 128, 64, T) > 0, shape
+    for shape in [(4, 32768, 16), (8, 8192, 8), (32, 263000, 32), (1, 2048, 1), (0, 0, 4)]:
+        N, total, H = shape
+        assert ws(N, total, H, 128, 128, 64, A) == 0, shape
+
+
 @pytest.mark.parametrize("kw,status", [
     (dict(dk=48, dv=48), gdn.GDN_ERR_UNSUPPORTED),
     (dict(N=-1), gdn.GDN_ERR_INVALID_ARG),

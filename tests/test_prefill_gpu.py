@@ -207,9 +207,3 @@ def test_transfer_b1_t65536_h4_full_size():
     inp = inputs.longseq_b1_t65536_h4()
     check(inp, TRANSFER, what="B1 T65536 H4", out_dtype=torch.bfloat16)
 
-
-def test_auto_picks_transfer_for_long_low_parallelism():
-    ws = gdn.gdn_chunk_prefill_workspace_size
-    assert ws(1, 65536, 4, 128, 128, 64, gdn.GDN_PREFILL_AUTO) == \
-        ws(1, 65536, 4, 128, 128, 64, gdn.GDN_PREFILL_TRANSFER) > 0
-    assert ws(4, 32768, 16, 128, 128, 64, gdn.GDN_PREFILL_AUTO) == 0
