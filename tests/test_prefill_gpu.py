@@ -139,6 +139,28 @@ def test_fused_varlen_bitwise_equals_single_sequence_calls():
     assert torch.equal(o, o2) and torch.equal(fin, fin2)  # deterministic
 
 
+@pytest.mark.parametrize("nseq", [64, 70])
+def test_fused_many_sequences_launch_order(nseq):
+    """The fused kernel launches the longest sequences first when there are at most
+    64 of them and in index order beyond; both must give the oracle's results, and
+    a sequence's results must not depend on its neighbours (ties and empty
+    sequences included)."""
+    rng = np.random.default_rng(nseq)
+    lens = [int(x) for x in rng.integers(0, 200, size=nseq)]
+    lens[3] = lens[5] = 150  # a tie
+    lens[7] = 0
+    inp = inputs.prefill_inputs(lens, 2, 128, 128, seed=40 + nseq, g_range=(0.0, 0.05))
+    o, fin = check(inp, FUSED, what=f"{nseq} sequences")
+    cu = inp.cu_seqlens.tolist()
+    for n in (3, 5, 7, nseq - 1):
+        sl = slice(cu[n], cu[n + 1])
+        one = inputs.PrefillInputs(inp.q[sl], inp.k[sl], inp.v[sl], inp.g[sl], inp.beta[sl],
+                                   torch.tensor([0, lens[n]], dtype=torch.int32),
+                                   inp.initial_state[n:n + 1], inp.scale)
+        o_n, f_n = run_prefill(one, FUSED)
+        assert torch.equal(o_n, o[sl]) and torch.equal(f_n[0], fin[n])
+
+
 def test_fused_b4_t8192_h16_full_size():
     """Chunked prefill at the benchmark size (B=4 x 8192, H=16), every (sequence, head)."""
     inp = inputs.prefill_b4_t8192_h16()
