@@ -34,8 +34,9 @@ namespace {
 
 constexpr int C = 64;
 constexpr int D = 128;
-constexpr int kFixRows = 8;       // state rows (value indices) per fixup CTA
-constexpr int kFixThreads = 128;  // 4 warps; each thread a 2 x 4 tile of the 8 x 128 block
+constexpr int kFixRows = 4;       // state rows (value indices) per fixup CTA
+constexpr int kFixRPT = kFixRows / 4;  // rows per thread (four row groups per warp)
+constexpr int kFixThreads = 128;  // 4 warps; each thread a kFixRPT x 4 tile of the block
 
 size_t align256(size_t x) { return (x + 255) / 256 * 256; }
 
@@ -135,7 +136,8 @@ gdn_segment_map_kernel(const int32_t* cu, int N, int64_t total_T, int seg_len, i
 //    compose along the whole sequence, so no reduced-precision operands here).
 //    Each segment's transfer matrix (64 KiB) and local-state rows are staged in
 //    shared memory by one bulk copy, one segment ahead (two buffers). Thread
-//    (warp w, lane = 8 rg + cg) owns rows 2rg, 2rg+1 and columns 32w + 4cg .. +3
+//    (warp w, lane = 8 rg + cg) owns kFixRPT rows from kFixRPT * rg and columns
+//    32w + 4cg .. +3
 //    of the block; the state block is kept transposed in shared memory (sT[i][j])
 //    for the products and in registers (the thread's own tile) for the stores.
 constexpr uint32_t kFixMtBytes = D * D * 4;
@@ -161,7 +163,7 @@ gdn_fixup_scan_kernel(const int32_t* seg_of_seq, int H, const float* local, cons
   uint64_t* full = reinterpret_cast<uint64_t*>(sT + D * kFixRows);
   const int tid = threadIdx.x, w = tid >> 5, lane = tid & 31;
   const int rg = lane >> 3, cg = lane & 7;
-  const int jr = 2 * rg;                 // first of my two rows (within the block)
+  const int jr = kFixRPT * rg;           // first of my rows (within the block)
   const int l0 = 32 * w + 4 * cg;        // first of my four columns
   const int rblocks = D / kFixRows;
   const int rb = blockIdx.x % rblocks;
@@ -178,9 +180,9 @@ gdn_fixup_scan_kernel(const int32_t* seg_of_seq, int H, const float* local, cons
     tc::fence_mbar_init();
   }
   // my tile of the initial state (registers) and the transposed block (shared)
-  float cur[2][4];
+  float cur[kFixRPT][4];
 #pragma unroll
-  for (int a = 0; a < 2; ++a) {
+  for (int a = 0; a < kFixRPT; ++a) {
     float4 x = make_float4(0.f, 0.f, 0.f, 0.f);
     if (initial_state) x = *reinterpret_cast<const float4*>(initial_state + soff + (size_t)(r0 + jr + a) * D + l0);
     cur[a][0] = x.x; cur[a][1] = x.y; cur[a][2] = x.z; cur[a][3] = x.w;
@@ -212,9 +214,9 @@ gdn_fixup_scan_kernel(const int32_t* seg_of_seq, int H, const float* local, cons
     const size_t off = ((size_t)sg * H + h) * ssz;
     const float* m = mt + b * D * D;
     const float* lr = loc + b * kFixRows * D;
-    float acc[2][4];
+    float acc[kFixRPT][4];
 #pragma unroll
-    for (int a = 0; a < 2; ++a) {
+    for (int a = 0; a < kFixRPT; ++a) {
       // the state at the segment start, then the local state as the accumulator
       *reinterpret_cast<float4*>(fixed + off + (size_t)(r0 + jr + a) * D + l0) =
           make_float4(cur[a][0], cur[a][1], cur[a][2], cur[a][3]);
@@ -223,20 +225,19 @@ gdn_fixup_scan_kernel(const int32_t* seg_of_seq, int H, const float* local, cons
     }
 #pragma unroll 8
     for (int i = 0; i < D; ++i) {
-      const float2 sv = *reinterpret_cast<const float2*>(sT + i * kFixRows + jr);
       const float4 mv = *reinterpret_cast<const float4*>(m + i * D + l0);
-      acc[0][0] = fmaf(sv.x, mv.x, acc[0][0]);
-      acc[0][1] = fmaf(sv.x, mv.y, acc[0][1]);
-      acc[0][2] = fmaf(sv.x, mv.z, acc[0][2]);
-      acc[0][3] = fmaf(sv.x, mv.w, acc[0][3]);
-      acc[1][0] = fmaf(sv.y, mv.x, acc[1][0]);
-      acc[1][1] = fmaf(sv.y, mv.y, acc[1][1]);
-      acc[1][2] = fmaf(sv.y, mv.z, acc[1][2]);
-      acc[1][3] = fmaf(sv.y, mv.w, acc[1][3]);
+#pragma unroll
+      for (int a = 0; a < kFixRPT; ++a) {
+        const float sv = sT[i * kFixRows + jr + a];
+        acc[a][0] = fmaf(sv, mv.x, acc[a][0]);
+        acc[a][1] = fmaf(sv, mv.y, acc[a][1]);
+        acc[a][2] = fmaf(sv, mv.z, acc[a][2]);
+        acc[a][3] = fmaf(sv, mv.w, acc[a][3]);
+      }
     }
     __syncthreads();  // every read of sT and of this buffer is done
 #pragma unroll
-    for (int a = 0; a < 2; ++a)
+    for (int a = 0; a < kFixRPT; ++a)
 #pragma unroll
       for (int x4 = 0; x4 < 4; ++x4) {
         cur[a][x4] = acc[a][x4];
@@ -246,7 +247,7 @@ gdn_fixup_scan_kernel(const int32_t* seg_of_seq, int H, const float* local, cons
   }
   if (final_state) {
 #pragma unroll
-    for (int a = 0; a < 2; ++a)
+    for (int a = 0; a < kFixRPT; ++a)
       *reinterpret_cast<float4*>(final_state + soff + (size_t)(r0 + jr + a) * D + l0) =
           make_float4(cur[a][0], cur[a][1], cur[a][2], cur[a][3]);
   }
