@@ -435,6 +435,43 @@ __device__ __forceinline__ void solve_merge(const Smem& sm, int t) {
   tc::named_sync(kBarPrep, 128);
 }
 
+// Columns 32 hq .. 32 hq + 31 of A row t: beta_t 2^(G_t - G_j) x_j for j < t (base-2
+// cumulative gates), 16-byte chunks right of the diagonal skipped (the solve never
+// reads them). The decays are computed unconditionally (independent, so they
+// pipeline); entries right of the diagonal may overflow and are masked.
+__device__ __forceinline__ void a_row_half(float* A, int t, int hq, float bi, float Gi, const float* G,
+                                           const float* x) {
+#pragma unroll
+  for (int q = 0; q < 8; ++q) {
+    const int j0 = 32 * hq + 4 * q;
+    const float4 g4 = *reinterpret_cast<const float4*>(G + j0);
+    float4 v;
+    v.x = (j0 + 0 < t) ? bi * exp2_approx(Gi - g4.x) * x[4 * q + 0] : 0.f;
+    v.y = (j0 + 1 < t) ? bi * exp2_approx(Gi - g4.y) * x[4 * q + 1] : 0.f;
+    v.z = (j0 + 2 < t) ? bi * exp2_approx(Gi - g4.z) * x[4 * q + 2] : 0.f;
+    v.w = (j0 + 3 < t) ? bi * exp2_approx(Gi - g4.w) * x[4 * q + 3] : 0.f;
+    if (j0 < t) *row_chunk(A, t, j0 >> 2) = v;
+  }
+}
+
+// Columns 32 hq .. 32 hq + 31 of P row r into the fp16 tile: 2^(G_r - G_i) x_i for
+// i <= r; chunks entirely above the diagonal are left as they are (zeros).
+__device__ __forceinline__ void p_row_half(uint8_t* p16, int r, int hq, float Gr, const float* G, const float* x) {
+#pragma unroll
+  for (int cc = 0; cc < 4; ++cc) {
+    const float4 g0 = *reinterpret_cast<const float4*>(G + 32 * hq + 8 * cc);
+    const float4 g1 = *reinterpret_cast<const float4*>(G + 32 * hq + 8 * cc + 4);
+    const float gv[8] = {g0.x, g0.y, g0.z, g0.w, g1.x, g1.y, g1.z, g1.w};
+    float v[8];
+#pragma unroll
+    for (int m = 0; m < 8; ++m) {
+      const int i = 32 * hq + cc * 8 + m;
+      v[m] = (i <= r) ? exp2_approx(Gr - gv[m]) * x[cc * 8 + m] : 0.f;
+    }
+    if (32 * hq + cc * 8 <= r) st_sw128_chunk(p16, r, 4 * hq + cc, v);
+  }
+}
+
 __device__ void prep_role(const Smem& sm, uint32_t tmem, int nchunks, unsigned int* err) {
   const int t = threadIdx.x - kPrepWarp0 * 32;  // 0..127 == TMEM lane
   const int warp = threadIdx.x >> 5;
@@ -450,42 +487,23 @@ __device__ void prep_role(const Smem& sm, uint32_t tmem, int nchunks, unsigned i
     const float* vec = sm.vec(c % 3);
     const float* G = vec + V_G;
     if (t < C) {
-      // A row t (rows 0-63 of D1): beta_t exp(G_t - G_j) k_t.k_j for j < t; the
-      // chunks right of the diagonal are never read by the solve and are skipped
+      // A row t (rows 0-63 of D1): beta_t exp(G_t - G_j) k_t.k_j for j < t. Warp 5
+      // (rows 32-63) needs both 32-column halves: the second half's TMEM load is
+      // issued before the first half is processed, so its latency is hidden.
       const float Gi = G[t], bi = vec[V_BETA + t];
-#pragma unroll
-      for (int hq = 0; hq < 2; ++hq) {
-        // tcgen05.ld is warp-collective: the condition must be uniform across the
-        // warp, so it uses the warp's largest row (t | 31)
-        if (32 * hq < (t | 31)) {
-          float x[32];
-          tc::tmem_ld16(tl + COL_D1 + hq * 32, x);
-          tc::tmem_ld16(tl + COL_D1 + hq * 32 + 16, x + 16);
-          float4 gj[8];  // G of the 32 columns, loaded up front (no loads inside the masked loop)
-#pragma unroll
-          for (int q = 0; q < 8; ++q) gj[q] = *reinterpret_cast<const float4*>(G + 32 * hq + 4 * q);
-          // the 32 decays first, unconditionally (independent, so they pipeline);
-          // entries right of the diagonal may overflow and are masked below
-          float e[32];
-#pragma unroll
-          for (int q = 0; q < 8; ++q) {
-            e[4 * q + 0] = exp2_approx(Gi - gj[q].x);
-            e[4 * q + 1] = exp2_approx(Gi - gj[q].y);
-            e[4 * q + 2] = exp2_approx(Gi - gj[q].z);
-            e[4 * q + 3] = exp2_approx(Gi - gj[q].w);
-          }
-          tc::wait_ld();
-#pragma unroll
-          for (int q = 0; q < 8; ++q) {
-            const int j0 = 32 * hq + 4 * q;
-            float4 v;
-            v.x = (j0 + 0 < t) ? bi * e[4 * q + 0] * x[4 * q + 0] : 0.f;
-            v.y = (j0 + 1 < t) ? bi * e[4 * q + 1] * x[4 * q + 1] : 0.f;
-            v.z = (j0 + 2 < t) ? bi * e[4 * q + 2] * x[4 * q + 2] : 0.f;
-            v.w = (j0 + 3 < t) ? bi * e[4 * q + 3] * x[4 * q + 3] : 0.f;
-            if (j0 < t) *row_chunk(sm.A(), t, j0 >> 2) = v;
-          }
-        }
+      const bool two = (t | 31) > 32;  // warp-uniform (tcgen05.ld is warp-collective)
+      float x0[32], x1[32];
+      tc::tmem_ld16(tl + COL_D1, x0);
+      tc::tmem_ld16(tl + COL_D1 + 16, x0 + 16);
+      tc::wait_ld();
+      if (two) {
+        tc::tmem_ld16(tl + COL_D1 + 32, x1);
+        tc::tmem_ld16(tl + COL_D1 + 48, x1 + 16);
+      }
+      a_row_half(sm.A(), t, 0, bi, Gi, G, x0);
+      if (two) {
+        tc::wait_ld();
+        a_row_half(sm.A(), t, 1, bi, Gi, G, x1);
       }
     } else {
       // P row r (rows 64-127 of D1) into P16[b]; its previous reader (chunk c-2's O2
@@ -493,35 +511,20 @@ __device__ void prep_role(const Smem& sm, uint32_t tmem, int nchunks, unsigned i
       // 16-byte chunks entirely above the diagonal keep the zeros written at start.
       const int r = t - C;
       const float Gr = G[r];
-#pragma unroll
-      for (int hq = 0; hq < 2; ++hq) {
-        if (32 * hq <= (r | 31)) {  // warp-uniform (tcgen05.ld is warp-collective)
-          float x[32];
-          tc::tmem_ld16(tl + COL_D1 + hq * 32, x);
-          tc::tmem_ld16(tl + COL_D1 + hq * 32 + 16, x + 16);
-          float4 gi[8];
-#pragma unroll
-          for (int q = 0; q < 8; ++q) gi[q] = *reinterpret_cast<const float4*>(G + 32 * hq + 4 * q);
-          float e[32];
-#pragma unroll
-          for (int q = 0; q < 8; ++q) {
-            e[4 * q + 0] = exp2_approx(Gr - gi[q].x);
-            e[4 * q + 1] = exp2_approx(Gr - gi[q].y);
-            e[4 * q + 2] = exp2_approx(Gr - gi[q].z);
-            e[4 * q + 3] = exp2_approx(Gr - gi[q].w);
-          }
-          tc::wait_ld();
-#pragma unroll
-          for (int cc = 0; cc < 4; ++cc) {
-            float v[8];
-#pragma unroll
-            for (int m = 0; m < 8; ++m) {
-              const int i = 32 * hq + cc * 8 + m;
-              v[m] = (i <= r) ? e[cc * 8 + m] * x[cc * 8 + m] : 0.f;
-            }
-            if (32 * hq + cc * 8 <= r) st_sw128_chunk(sm.base + OFF_P16 + b * P_BUF, r, 4 * hq + cc, v);
-          }
-        }
+      const bool two = (r | 31) >= 32;  // warp 7: both halves (warp-uniform)
+      uint8_t* p16 = sm.base + OFF_P16 + b * P_BUF;
+      float x0[32], x1[32];
+      tc::tmem_ld16(tl + COL_D1, x0);
+      tc::tmem_ld16(tl + COL_D1 + 16, x0 + 16);
+      tc::wait_ld();
+      if (two) {
+        tc::tmem_ld16(tl + COL_D1 + 32, x1);
+        tc::tmem_ld16(tl + COL_D1 + 48, x1 + 16);
+      }
+      p_row_half(p16, r, 0, Gr, G, x0);
+      if (two) {
+        tc::wait_ld();
+        p_row_half(p16, r, 1, Gr, G, x1);
       }
     }
     // this warp's reads of D1 are complete: the next chunk's [K;Q]K^T may overwrite it
