@@ -14,10 +14,11 @@
 //                   copies of the state (64 KiB at dk = 128) and of the item's
 //                   k, q, v rows into a free stage (2-3 stages), tracked by an
 //                   mbarrier's transaction count
-//   consumer warps: two (single token) or four (multi-token) threads per state
-//                   row load its parts from shared memory into registers, do the
-//                   arithmetic below, write the row back, and one thread
-//                   bulk-stores the stage to the pool
+//   consumer warps: single token: two threads per state row load its halves from
+//                   shared memory into registers, do the arithmetic below and
+//                   write the row back; multi-token: two groups take alternate
+//                   items, a thread owning half of two rows; one thread per group
+//                   stores the stage to the pool
 //
 // Arithmetic. Per row j (value column j of S, stored K-last as S^T[j, :]) the
 // step is M = T*n_h sub-steps (gate on the first sub-step of each token, then a
@@ -85,9 +86,11 @@ struct StageLayout {
   static constexpr uint32_t kQK = kGram + 4 * M * M;
   static constexpr uint32_t kBytes = ((kQK + 4 * TT * M) + kAlign - 1) / kAlign * kAlign;
   static constexpr uint32_t kVecBytes = (2 * M + TT) * kRow;
-  // keys and queries as fp32 (one buffer shared by all stages); T = n_h = 1 reads
-  // the raw vectors instead and needs none
-  static constexpr uint32_t kVecF32 = (M > 1) ? (M + TT) * DK * 4 : 0;
+  // consumer groups (items in flight per CTA)
+  static constexpr int kGroups = (M > 1) ? 2 : 1;
+  // keys and queries as fp32 (one buffer per consumer group, shared by the stages);
+  // T = n_h = 1 reads the raw vectors instead and needs none
+  static constexpr uint32_t kVecF32 = (M > 1) ? kGroups * (M + TT) * DK * 4 : 0;
   static constexpr int kStages = (3 * kBytes + kVecF32 + 64 + kAlign <= 226 * 1024) ? 3 : 2;
   static constexpr uint32_t kSmem = kStages * kBytes + kVecF32 + 64 + kAlign;  // + barriers + alignment
 };
@@ -107,18 +110,76 @@ __device__ __forceinline__ void load4_f32<float>(const uint8_t* p, float* out) {
   out[0] = f.x; out[1] = f.y; out[2] = f.z; out[3] = f.w;
 }
 
-// Threads per state row (2 or 4; the consumer mapping below supports both).
-// Measured on B200, 4 threads per row gained nothing for the multi-token product
-// (its 96-register cap spills), so both step shapes use 2.
+// Threads per state row of the single-token kernel (2 or 4; its consumer mapping
+// supports both). 2 measured best on B200.
 template <int TT, int NH>
 __host__ __device__ constexpr int threads_per_row() { return 2; }
 
+// Producer (one thread of the last warp): for each item of the CTA, in order, the
+// slot id, gates and betas go into the stage header and the state and the item's
+// k, q, v rows are bulk-copied into the stage; the stage's full barrier counts the
+// bytes. A stage is refilled once its previous item released it (empty barrier).
+template <int DK, int TT, int NH, typename TIn>
+__device__ __forceinline__ void decode_producer(const DecodeParams& p, const CUtensorMap* pool_map, uint8_t* base,
+                                                uint64_t* full, uint64_t* empty) {
+  using L = StageLayout<DK, TT, NH, TIn>;
+  constexpr int M = L::M;
+  constexpr int NS = L::kStages;
+  const TIn* kp = static_cast<const TIn*>(p.k);
+  const TIn* qp = static_cast<const TIn*>(p.q);
+  const TIn* vp = static_cast<const TIn*>(p.v);
+  int it = 0;
+  for (int item = blockIdx.x; item < p.n_items; item += gridDim.x, ++it) {
+    const int s = it % NS;
+    if (it >= NS && !tc::mbar_wait(&empty[s], ((it / NS) & 1) ^ 1, kDecodeWaitNs)) {
+      raise_device_error(p.err, GDN_DEVERR_TIMEOUT);
+      return;
+    }
+    uint8_t* st = base + s * L::kBytes;
+    const int b = item / p.H, h = item - (item / p.H) * p.H;
+    int slot = __ldg(p.slot_ids + b);
+    if (slot >= p.num_slots) {
+      raise_device_error(p.err, GDN_DEVERR_SLOT_OUT_OF_RANGE);
+      slot = -1;
+    }
+    if (slot < 0) slot = -1;
+    *reinterpret_cast<int*>(st + L::kHeader) = slot;
+#pragma unroll
+    for (int t = 0; t < TT; ++t)
+      reinterpret_cast<float*>(st + L::kAlpha)[t] = expf(__ldg(p.g + ((size_t)b * TT + t) * p.H + h));
+#pragma unroll
+    for (int m = 0; m < M; ++m) {
+      const int t = m / NH, mm = m - t * NH;
+      reinterpret_cast<float*>(st + L::kBeta)[m] = __ldg(p.beta + (((size_t)b * TT + t) * p.H + h) * NH + mm);
+    }
+    if (slot < 0) {
+      tc::mbar_arrive(&full[s]);
+      continue;
+    }
+    tc::mbar_arrive_expect_tx(&full[s], L::kState + L::kVecBytes);
+    const uint32_t sst = tc::smem_u32(st);
+    if constexpr (L::kSwizzled) {
+#pragma unroll
+      for (int x = 0; x < DK / 32; ++x) tc::tma_load_3d(sst + x * DK * 128, pool_map, 32 * x, 0, slot * p.H + h, &full[s]);
+    } else {
+      tc::bulk_load(sst, p.pool + ((size_t)slot * p.H + h) * (size_t)DK * DK, L::kState, &full[s]);
+    }
+#pragma unroll
+    for (int t = 0; t < TT; ++t) {
+      const size_t bth = ((size_t)b * TT + t) * p.H + h;
+      tc::bulk_load(sst + L::kKeys + t * NH * L::kRow, kp + bth * NH * DK, NH * L::kRow, &full[s]);
+      tc::bulk_load(sst + L::kQueries + t * L::kRow, qp + bth * DK, L::kRow, &full[s]);
+      tc::bulk_load(sst + L::kValues + t * NH * L::kRow, vp + bth * NH * DK, NH * L::kRow, &full[s]);
+    }
+  }
+}
+
+// Single-token step (T = n_h = 1): 2 threads per state row, all consumers on one item.
 template <int DK, int TT, int NH, typename TIn, typename TOut>
 __global__ void __launch_bounds__(threads_per_row<TT, NH>() * DK + 32, 1)
 gdn_decode_kernel(const DecodeParams p, const __grid_constant__ CUtensorMap pool_map) {
   using L = StageLayout<DK, TT, NH, TIn>;
-  constexpr int M = L::M;
-  constexpr int NV = M + TT;                 // vectors dotted with the old row: keys then queries
+  static_assert(L::M == 1, "single-token step");
   constexpr int NS = L::kStages;
   constexpr int TPR = threads_per_row<TT, NH>();
   constexpr int kConsumers = TPR * DK;
@@ -128,7 +189,6 @@ gdn_decode_kernel(const DecodeParams p, const __grid_constant__ CUtensorMap pool
 
   extern __shared__ uint8_t smem_raw[];
   uint8_t* base = tc::align_smem<L::kAlign>(smem_raw);
-  float* vecf = reinterpret_cast<float*>(base + NS * L::kBytes);  // [NV][DK] fp32 of the current item
   uint64_t* full = reinterpret_cast<uint64_t*>(base + NS * L::kBytes + L::kVecF32);
   uint64_t* empty = full + NS;
 
@@ -143,55 +203,7 @@ gdn_decode_kernel(const DecodeParams p, const __grid_constant__ CUtensorMap pool
   __syncthreads();
 
   if (tid >= kConsumers) {
-    // ---------------- producer (one thread)
-    if (tid != kConsumers) return;
-    const TIn* kp = static_cast<const TIn*>(p.k);
-    const TIn* qp = static_cast<const TIn*>(p.q);
-    const TIn* vp = static_cast<const TIn*>(p.v);
-    int it = 0;
-    for (int item = blockIdx.x; item < p.n_items; item += gridDim.x, ++it) {
-      const int s = it % NS;
-      if (it >= NS && !tc::mbar_wait(&empty[s], ((it / NS) & 1) ^ 1, kDecodeWaitNs)) {
-        raise_device_error(p.err, GDN_DEVERR_TIMEOUT);
-        return;
-      }
-      uint8_t* st = base + s * L::kBytes;
-      const int b = item / p.H, h = item - (item / p.H) * p.H;
-      int slot = __ldg(p.slot_ids + b);
-      if (slot >= p.num_slots) {
-        raise_device_error(p.err, GDN_DEVERR_SLOT_OUT_OF_RANGE);
-        slot = -1;
-      }
-      if (slot < 0) slot = -1;
-      *reinterpret_cast<int*>(st + L::kHeader) = slot;
-#pragma unroll
-      for (int t = 0; t < TT; ++t)
-        reinterpret_cast<float*>(st + L::kAlpha)[t] = expf(__ldg(p.g + ((size_t)b * TT + t) * p.H + h));
-#pragma unroll
-      for (int m = 0; m < M; ++m) {
-        const int t = m / NH, mm = m - t * NH;
-        reinterpret_cast<float*>(st + L::kBeta)[m] = __ldg(p.beta + (((size_t)b * TT + t) * p.H + h) * NH + mm);
-      }
-      if (slot < 0) {
-        tc::mbar_arrive(&full[s]);
-        continue;
-      }
-      tc::mbar_arrive_expect_tx(&full[s], L::kState + L::kVecBytes);
-      const uint32_t sst = tc::smem_u32(st);
-      if constexpr (L::kSwizzled) {
-#pragma unroll
-        for (int x = 0; x < DK / 32; ++x) tc::tma_load_3d(sst + x * DK * 128, &pool_map, 32 * x, 0, slot * p.H + h, &full[s]);
-      } else {
-        tc::bulk_load(sst, p.pool + ((size_t)slot * p.H + h) * (size_t)DK * DK, L::kState, &full[s]);
-      }
-#pragma unroll
-      for (int t = 0; t < TT; ++t) {
-        const size_t bth = ((size_t)b * TT + t) * p.H + h;
-        tc::bulk_load(sst + L::kKeys + t * NH * L::kRow, kp + bth * NH * DK, NH * L::kRow, &full[s]);
-        tc::bulk_load(sst + L::kQueries + t * L::kRow, qp + bth * DK, L::kRow, &full[s]);
-        tc::bulk_load(sst + L::kValues + t * NH * L::kRow, vp + bth * NH * DK, NH * L::kRow, &full[s]);
-      }
-    }
+    if (tid == kConsumers) decode_producer<DK, TT, NH, TIn>(p, &pool_map, base, full, empty);
     return;
   }
 
@@ -214,10 +226,8 @@ gdn_decode_kernel(const DecodeParams p, const __grid_constant__ CUtensorMap pool
     const int slot = *reinterpret_cast<const int*>(st + L::kHeader);
     const float* alpha = reinterpret_cast<const float*>(st + L::kAlpha);
     const float* betas = reinterpret_cast<const float*>(st + L::kBeta);
-    float* gram = reinterpret_cast<float*>(st + L::kGram);
-    float* qk = reinterpret_cast<float*>(st + L::kQK);
-    if (slot >= 0 && M == 1) {
-      // T = n_h = 1: k.s, q.s and the Gram entry q.k in one pass over the half row
+    if (slot >= 0) {
+      // k.s, q.s and the Gram entry q.k in one pass over the half row
       float* srow = reinterpret_cast<float*>(st) + (size_t)row * DK + half * (DK / TPR);
       float4 sv[CPH];
 #pragma unroll
@@ -252,154 +262,16 @@ gdn_decode_kernel(const DecodeParams p, const __grid_constant__ CUtensorMap pool
         x.w = fmaf(cm, wk[3], a * x.w);
         reinterpret_cast<float4*>(srow)[(c + row) & (CPH - 1)] = x;
       }
-    } else if (slot >= 0) {
-      // keys and queries of the item -> fp32 once (every FMA below reads them)
-      for (int e = tid * 4; e < NV * DK; e += kConsumers * 4)
-        load4_f32<TIn>(st + L::kKeys + e * sizeof(TIn), vecf + e);
-      tc::named_sync(kBarConsumers, kConsumers);
-      // per-head Gram entries k_m.k_l (l < m) and q_t.k_l: warp w takes pairs w,
-      // w + W, ...; their partial sums are reduced together (independent shuffles)
-      constexpr int kPairsKK = M * (M - 1) / 2;
-      constexpr int kPairs = kPairsKK + TT * M;
-      constexpr int kWarps = kConsumers / 32;
-      constexpr int kPPW = (kPairs + kWarps - 1) / kWarps;
-      float gacc[kPPW];
-#pragma unroll
-      for (int q = 0; q < kPPW; ++q) {
-        const int pair = warp + q * kWarps;
-        gacc[q] = 0.f;
-        if (pair < kPairs) {  // warp-uniform
-          int va, vb;
-          if (pair < kPairsKK) {
-            va = 1;
-            int rem = pair;
-            while (rem >= va) { rem -= va; ++va; }
-            vb = rem;
-          } else {
-            const int x = pair - kPairsKK;
-            va = M + x / M;
-            vb = x - (x / M) * M;
-          }
-          const float* pa = vecf + va * DK;  // the queries follow the keys
-          const float* pb = vecf + vb * DK;
-          for (int e = lane * 4; e < DK; e += 128) {
-            const float4 xa = *reinterpret_cast<const float4*>(pa + e);
-            const float4 xb = *reinterpret_cast<const float4*>(pb + e);
-            gacc[q] = fmaf(xa.x, xb.x, fmaf(xa.y, xb.y, fmaf(xa.z, xb.z, fmaf(xa.w, xb.w, gacc[q]))));
-          }
-        }
-      }
-#pragma unroll
-      for (int off = 16; off > 0; off >>= 1)
-#pragma unroll
-        for (int q = 0; q < kPPW; ++q) gacc[q] += __shfl_xor_sync(0xffffffffu, gacc[q], off);
-      if (lane == 0) {
-#pragma unroll
-        for (int q = 0; q < kPPW; ++q) {
-          const int pair = warp + q * kWarps;
-          if (pair < kPairsKK) {
-            int va = 1, rem = pair;
-            while (rem >= va) { rem -= va; ++va; }
-            gram[va * M + rem] = gacc[q];
-          } else if (pair < kPairs) {
-            const int x = pair - kPairsKK;
-            qk[(x / M) * M + (x - (x / M) * M)] = gacc[q];
-          }
-        }
-      }
-      tc::named_sync(kBarConsumers, kConsumers);
-
-      // my part of the row: global float4 chunk gc = half * CPH + c sits in tile gc / 8,
-      // swizzled position (gc % 8) ^ (row % 8); the key / query chunk is gc itself
-      uint8_t* srow = st + (size_t)row * 128;
-      float4 sv[CPH];
-#pragma unroll
-      for (int c = 0; c < CPH; ++c) {
-        const int gc = half * CPH + c;
-        sv[c] = *reinterpret_cast<const float4*>(srow + (gc >> 3) * (DK * 128) + (((gc & 7) ^ (row & 7)) << 4));
-      }
-      float dots[NV];
-#pragma unroll
-      for (int vec = 0; vec < NV; ++vec) dots[vec] = 0.f;
-#pragma unroll
-      for (int c = 0; c < CPH; ++c) {
-        const int e = 4 * (half * CPH + c);
-#pragma unroll
-        for (int vec = 0; vec < NV; ++vec) {
-          const float4 w = *reinterpret_cast<const float4*>(vecf + vec * DK + e);
-          float a = dots[vec];
-          a = fmaf(sv[c].x, w.x, a);
-          a = fmaf(sv[c].y, w.y, a);
-          a = fmaf(sv[c].z, w.z, a);
-          a = fmaf(sv[c].w, w.w, a);
-          dots[vec] = a;
-        }
-      }
-#pragma unroll
-      for (int off = RPW; off < 32; off <<= 1)
-#pragma unroll
-        for (int vec = 0; vec < NV; ++vec) dots[vec] += __shfl_xor_sync(0xffffffffu, dots[vec], off);
-
-      // scalar recurrence for this row (both halves, redundantly)
-      float coef[M];
-      float G = 1.f;
-#pragma unroll
-      for (int t = 0; t < TT; ++t) {
-        const float a = alpha[t];
-        G *= a;
-#pragma unroll
-        for (int l = 0; l < t * NH; ++l) coef[l] *= a;
-#pragma unroll
-        for (int x = 0; x < NH; ++x) {
-          const int m = t * NH + x;
-          float u = G * dots[m];
-#pragma unroll
-          for (int l = 0; l < m; ++l) u = fmaf(coef[l], gram[m * M + l], u);
-          const float vj = to_f32(reinterpret_cast<const TIn*>(st + L::kValues + m * L::kRow)[row]);
-          coef[m] = betas[m] * (vj - u);
-        }
-        float out = G * dots[M + t];
-#pragma unroll
-        for (int l = 0; l < (t + 1) * NH; ++l) out = fmaf(coef[l], qk[t * M + l], out);
-        if (half == 0) store_out(op + (((size_t)b * TT + t) * p.H + h) * DK + row, p.scale * out);
-      }
-      // s_new = Gamma s_0 + sum_m c_m k_m, written back in place (same swizzled chunks)
-#pragma unroll
-      for (int c = 0; c < CPH; ++c) {
-        const int gc = half * CPH + c;
-        const int e = 4 * gc;
-        float4 x = sv[c];
-        x.x *= G; x.y *= G; x.z *= G; x.w *= G;
-#pragma unroll
-        for (int m = 0; m < M; ++m) {
-          const float4 w = *reinterpret_cast<const float4*>(vecf + m * DK + e);
-          x.x = fmaf(coef[m], w.x, x.x);
-          x.y = fmaf(coef[m], w.y, x.y);
-          x.z = fmaf(coef[m], w.z, x.z);
-          x.w = fmaf(coef[m], w.w, x.w);
-        }
-        *reinterpret_cast<float4*>(srow + (gc >> 3) * (DK * 128) + (((gc & 7) ^ (row & 7)) << 4)) = x;
-      }
-    } else {
+    } else if (half == 0) {
       // skipped row of the batch: o = 0, pool untouched
-#pragma unroll
-      for (int t = 0; t < TT; ++t)
-        if (half == 0) store_out(op + (((size_t)b * TT + t) * p.H + h) * DK + row, 0.f);
+      store_out(op + ((size_t)b * p.H + h) * DK + row, 0.f);
     }
     // stage -> pool (one bulk store); the previous item's stage is handed back to
     // the producer once its store has finished reading shared memory
     tc::fence_proxy_async_smem();
     tc::named_sync(kBarConsumers, kConsumers);
     if (tid == 0) {
-      if (slot >= 0) {
-        if constexpr (L::kSwizzled) {
-#pragma unroll
-          for (int x = 0; x < DK / 32; ++x)
-            tc::tma_store_3d(&pool_map, 32 * x, 0, slot * p.H + h, tc::smem_u32(st) + x * DK * 128);
-        } else {
-          tc::bulk_store(p.pool + ((size_t)slot * p.H + h) * (size_t)DK * DK, tc::smem_u32(st), L::kState);
-        }
-      }
+      if (slot >= 0) tc::bulk_store(p.pool + ((size_t)slot * p.H + h) * (size_t)DK * DK, tc::smem_u32(st), L::kState);
       tc::bulk_commit();
       tc::bulk_wait_read_1();
       if (prev_stage >= 0) tc::mbar_arrive(&empty[prev_stage]);
@@ -407,6 +279,256 @@ gdn_decode_kernel(const DecodeParams p, const __grid_constant__ CUtensorMap pool
     prev_stage = s;
   }
   if (tid == 0) tc::bulk_wait_all();
+}
+
+// Multi-token / product step (M = T n_h > 1). Two consumer groups of DK threads
+// take the CTA's items alternately (group g its items g, g + 2, ...), so one
+// group's phases, which are separated by group barriers, overlap the other's.
+// In a group a thread owns one half (16-byte chunks half*DK/8 .. ) of two state
+// rows, j and j + DK/2: each key / query chunk it reads from shared memory (a
+// broadcast across its half-warp) feeds both rows, which halves the shared-memory
+// wavefronts per row against one row per thread. Per item:
+//   keys and queries -> fp32 (the group's buffer); the Gram entries k_m.k_l (l < m)
+//   and q_t.k_l, one warp per pair; the row pass (all NV dot products of the two
+//   old rows, halves combined by one xor shuffle); the scalar recurrence of each
+//   row; the update pass s_new = Gamma s_0 + sum_m c_m k_m written back in place;
+//   the stage stored to the pool and released.
+template <int DK, int TT, int NH, typename TIn, typename TOut>
+__global__ void __launch_bounds__(2 * DK + 32, 1)
+gdn_decode_multi_kernel(const DecodeParams p, const __grid_constant__ CUtensorMap pool_map) {
+  using L = StageLayout<DK, TT, NH, TIn>;
+  static_assert(L::M > 1 && L::kGroups == 2, "multi-token step");
+  constexpr int M = L::M;
+  constexpr int NV = M + TT;                 // vectors dotted with the old rows: keys then queries
+  constexpr int NS = L::kStages;
+  constexpr int kGroupThreads = DK;          // DK/2 row pairs x 2 halves
+  constexpr int kConsumers = 2 * kGroupThreads;
+  constexpr int CPH = DK / 8;                // float4 chunks in half a row
+  constexpr int kPairsKK = M * (M - 1) / 2;
+  constexpr int kPairs = kPairsKK + TT * M;
+  constexpr int kGroupWarps = kGroupThreads / 32;
+  constexpr int kBatch = 8;                  // Gram pairs per warp reduced together
+
+  extern __shared__ uint8_t smem_raw[];
+  uint8_t* base = tc::align_smem<L::kAlign>(smem_raw);
+  uint64_t* full = reinterpret_cast<uint64_t*>(base + NS * L::kBytes + L::kVecF32);
+  uint64_t* empty = full + NS;
+
+  const int tid = threadIdx.x;
+  if (tid == 0) {
+    for (int s = 0; s < NS; ++s) {
+      tc::mbar_init(&full[s], 1);
+      tc::mbar_init(&empty[s], 1);
+    }
+    tc::fence_mbar_init();
+  }
+  __syncthreads();
+
+  if (tid >= kConsumers) {
+    if (tid == kConsumers) decode_producer<DK, TT, NH, TIn>(p, &pool_map, base, full, empty);
+    return;
+  }
+
+  const int grp = tid / kGroupThreads, gt = tid - grp * kGroupThreads;
+  const uint32_t bar_id = 1 + grp;
+  float* vecf = reinterpret_cast<float*>(base + NS * L::kBytes) + grp * NV * DK;  // [NV][DK] fp32
+  const int lane = gt & 31, gw = gt >> 5;
+  const int half = lane >> 4;
+  const int r0 = gw * 16 + (lane & 15), r1 = r0 + DK / 2;
+  // chunk gc of row r sits in tile gc / 8 at the swizzled position (gc % 8) ^ (r % 8);
+  // r1 % 8 == r0 % 8, so both rows use the same offsets
+  TOut* op = static_cast<TOut*>(p.o);
+  for (int it = grp, item = blockIdx.x + grp * gridDim.x; item < p.n_items; it += 2, item += 2 * gridDim.x) {
+    const int s = it % NS;
+    uint8_t* st = base + s * L::kBytes;
+    // The stage's previous item (it - NS) must have been released before this fill
+    // is waited for, so that full[s]'s parity names this fill and not the last one.
+    if (it >= NS && !tc::mbar_wait(&empty[s], ((it - NS) / NS) & 1, kDecodeWaitNs)) {
+      if (gt == 0) raise_device_error(p.err, GDN_DEVERR_TIMEOUT);
+      break;
+    }
+    if (!tc::mbar_wait(&full[s], (it / NS) & 1, kDecodeWaitNs)) {
+      if (gt == 0) raise_device_error(p.err, GDN_DEVERR_TIMEOUT);
+      break;
+    }
+    const int b = item / p.H, h = item - (item / p.H) * p.H;
+    const int slot = *reinterpret_cast<const int*>(st + L::kHeader);
+    const float* alpha = reinterpret_cast<const float*>(st + L::kAlpha);
+    const float* betas = reinterpret_cast<const float*>(st + L::kBeta);
+    float* gram = reinterpret_cast<float*>(st + L::kGram);
+    float* qk = reinterpret_cast<float*>(st + L::kQK);
+    if (slot >= 0) {
+      // keys and queries of the item -> fp32 once (every FMA below reads them)
+      for (int e = gt * 4; e < NV * DK; e += kGroupThreads * 4)
+        load4_f32<TIn>(st + L::kKeys + e * sizeof(TIn), vecf + e);
+      tc::named_sync(bar_id, kGroupThreads);
+      // Gram entries: warp w takes pairs w, w + W, ...; a batch of kBatch pairs has
+      // its partial sums reduced together (independent shuffles)
+      for (int p0 = gw; p0 < kPairs; p0 += kGroupWarps * kBatch) {
+        float gacc[kBatch];
+#pragma unroll
+        for (int q = 0; q < kBatch; ++q) {
+          const int pair = p0 + q * kGroupWarps;
+          gacc[q] = 0.f;
+          if (pair < kPairs) {  // warp-uniform
+            int va, vb;
+            if (pair < kPairsKK) {
+              va = 1;
+              int rem = pair;
+              while (rem >= va) { rem -= va; ++va; }
+              vb = rem;
+            } else {
+              const int x = pair - kPairsKK;
+              va = M + x / M;
+              vb = x - (x / M) * M;
+            }
+            const float* pa = vecf + va * DK;  // the queries follow the keys
+            const float* pb = vecf + vb * DK;
+            for (int e = lane * 4; e < DK; e += 128) {
+              const float4 xa = *reinterpret_cast<const float4*>(pa + e);
+              const float4 xb = *reinterpret_cast<const float4*>(pb + e);
+              gacc[q] = fmaf(xa.x, xb.x, fmaf(xa.y, xb.y, fmaf(xa.z, xb.z, fmaf(xa.w, xb.w, gacc[q]))));
+            }
+          }
+        }
+#pragma unroll
+        for (int off = 16; off > 0; off >>= 1)
+#pragma unroll
+          for (int q = 0; q < kBatch; ++q) gacc[q] += __shfl_xor_sync(0xffffffffu, gacc[q], off);
+        if (lane == 0) {
+#pragma unroll
+          for (int q = 0; q < kBatch; ++q) {
+            const int pair = p0 + q * kGroupWarps;
+            if (pair < kPairsKK) {
+              int va = 1, rem = pair;
+              while (rem >= va) { rem -= va; ++va; }
+              gram[va * M + rem] = gacc[q];
+            } else if (pair < kPairs) {
+              const int x = pair - kPairsKK;
+              qk[(x / M) * M + (x - (x / M) * M)] = gacc[q];
+            }
+          }
+        }
+      }
+      tc::named_sync(bar_id, kGroupThreads);
+
+      // row pass: dot products of both old rows with every key and query
+      const uint8_t* srow0 = st + (size_t)r0 * 128;
+      const uint8_t* srow1 = st + (size_t)r1 * 128;
+      float d0[NV], d1[NV];
+#pragma unroll
+      for (int v = 0; v < NV; ++v) d0[v] = d1[v] = 0.f;
+#pragma unroll 4
+      for (int c = 0; c < CPH; ++c) {
+        const int gc = half * CPH + c;
+        const uint32_t off = (gc >> 3) * (DK * 128) + (((gc & 7) ^ (r0 & 7)) << 4);
+        const float4 x0 = *reinterpret_cast<const float4*>(srow0 + off);
+        const float4 x1 = *reinterpret_cast<const float4*>(srow1 + off);
+        const float* w = vecf + 4 * gc;
+#pragma unroll
+        for (int v = 0; v < NV; ++v) {
+          const float4 wv = *reinterpret_cast<const float4*>(w + v * DK);
+          float a0 = d0[v], a1 = d1[v];
+          a0 = fmaf(x0.x, wv.x, a0); a1 = fmaf(x1.x, wv.x, a1);
+          a0 = fmaf(x0.y, wv.y, a0); a1 = fmaf(x1.y, wv.y, a1);
+          a0 = fmaf(x0.z, wv.z, a0); a1 = fmaf(x1.z, wv.z, a1);
+          a0 = fmaf(x0.w, wv.w, a0); a1 = fmaf(x1.w, wv.w, a1);
+          d0[v] = a0;
+          d1[v] = a1;
+        }
+      }
+#pragma unroll
+      for (int v = 0; v < NV; ++v) {
+        d0[v] += __shfl_xor_sync(0xffffffffu, d0[v], 16);
+        d1[v] += __shfl_xor_sync(0xffffffffu, d1[v], 16);
+      }
+
+      // scalar recurrence of both rows (both halves, redundantly); half 0 writes the
+      // outputs of row r0, half 1 those of row r1
+      float c0[M], c1[M];
+      float G = 1.f;
+#pragma unroll
+      for (int t = 0; t < TT; ++t) {
+        const float a = alpha[t];
+        G *= a;
+#pragma unroll
+        for (int l = 0; l < t * NH; ++l) {
+          c0[l] *= a;
+          c1[l] *= a;
+        }
+#pragma unroll
+        for (int x = 0; x < NH; ++x) {
+          const int m = t * NH + x;
+          float u0 = G * d0[m], u1 = G * d1[m];
+#pragma unroll
+          for (int l = 0; l < m; ++l) {
+            const float gv = gram[m * M + l];
+            u0 = fmaf(c0[l], gv, u0);
+            u1 = fmaf(c1[l], gv, u1);
+          }
+          const TIn* vrow = reinterpret_cast<const TIn*>(st + L::kValues + m * L::kRow);
+          c0[m] = betas[m] * (to_f32(vrow[r0]) - u0);
+          c1[m] = betas[m] * (to_f32(vrow[r1]) - u1);
+        }
+        float o0 = G * d0[M + t], o1 = G * d1[M + t];
+#pragma unroll
+        for (int l = 0; l < (t + 1) * NH; ++l) {
+          const float qv = qk[t * M + l];
+          o0 = fmaf(c0[l], qv, o0);
+          o1 = fmaf(c1[l], qv, o1);
+        }
+        TOut* orow = op + (((size_t)b * TT + t) * p.H + h) * DK;
+        if (half == 0) store_out(orow + r0, p.scale * o0);
+        else store_out(orow + r1, p.scale * o1);
+      }
+
+      // update pass: s_new = Gamma s_0 + sum_m c_m k_m, in place (same swizzled chunks)
+      uint8_t* wrow0 = st + (size_t)r0 * 128;
+      uint8_t* wrow1 = st + (size_t)r1 * 128;
+#pragma unroll 4
+      for (int c = 0; c < CPH; ++c) {
+        const int gc = half * CPH + c;
+        const uint32_t off = (gc >> 3) * (DK * 128) + (((gc & 7) ^ (r0 & 7)) << 4);
+        float4 x0 = *reinterpret_cast<const float4*>(wrow0 + off);
+        float4 x1 = *reinterpret_cast<const float4*>(wrow1 + off);
+        x0.x *= G; x0.y *= G; x0.z *= G; x0.w *= G;
+        x1.x *= G; x1.y *= G; x1.z *= G; x1.w *= G;
+        const float* w = vecf + 4 * gc;
+#pragma unroll
+        for (int m = 0; m < M; ++m) {
+          const float4 wv = *reinterpret_cast<const float4*>(w + m * DK);
+          x0.x = fmaf(c0[m], wv.x, x0.x); x1.x = fmaf(c1[m], wv.x, x1.x);
+          x0.y = fmaf(c0[m], wv.y, x0.y); x1.y = fmaf(c1[m], wv.y, x1.y);
+          x0.z = fmaf(c0[m], wv.z, x0.z); x1.z = fmaf(c1[m], wv.z, x1.z);
+          x0.w = fmaf(c0[m], wv.w, x0.w); x1.w = fmaf(c1[m], wv.w, x1.w);
+        }
+        *reinterpret_cast<float4*>(wrow0 + off) = x0;
+        *reinterpret_cast<float4*>(wrow1 + off) = x1;
+      }
+    } else {
+      // skipped row of the batch: o = 0, pool untouched
+#pragma unroll
+      for (int t = 0; t < TT; ++t) {
+        TOut* orow = op + (((size_t)b * TT + t) * p.H + h) * DK;
+        store_out(orow + (half == 0 ? r0 : r1), 0.f);
+      }
+    }
+    // stage -> pool (tensor stores of the swizzled tiles); the stage goes back to
+    // the producer as soon as the stores have read it
+    tc::fence_proxy_async_smem();
+    tc::named_sync(bar_id, kGroupThreads);
+    if (gt == 0) {
+      if (slot >= 0) {
+#pragma unroll
+        for (int x = 0; x < DK / 32; ++x)
+          tc::tma_store_3d(&pool_map, 32 * x, 0, slot * p.H + h, tc::smem_u32(st) + x * DK * 128);
+        tc::bulk_commit();
+        tc::bulk_wait_read();
+      }
+      tc::mbar_arrive(&empty[s]);
+    }
+  }
+  if (gt == 0) tc::bulk_wait_all();
 }
 
 // The pool as a 3-D fp32 tensor {DK columns, DK rows, num_slots * H states}; a box
@@ -428,9 +550,14 @@ gdn_status_t launch_typed(DecodeParams p, cudaStream_t stream) {
     int dev = 0;
     cudaError_t e = cudaGetDevice(&dev);
     if (e == cudaSuccess) e = cudaDeviceGetAttribute(&sm_count, cudaDevAttrMultiProcessorCount, dev);
-    if (e == cudaSuccess)
-      e = cudaFuncSetAttribute(gdn_decode_kernel<DK, TT, NH, TIn, TOut>, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                               L::kSmem);
+    if (e == cudaSuccess) {
+      if constexpr (L::kSwizzled)
+        e = cudaFuncSetAttribute(gdn_decode_multi_kernel<DK, TT, NH, TIn, TOut>,
+                                 cudaFuncAttributeMaxDynamicSharedMemorySize, L::kSmem);
+      else
+        e = cudaFuncSetAttribute(gdn_decode_kernel<DK, TT, NH, TIn, TOut>,
+                                 cudaFuncAttributeMaxDynamicSharedMemorySize, L::kSmem);
+    }
     if (e != cudaSuccess) return fail(GDN_ERR_CUDA, std::string("gdn_decode: setup: ") + cudaGetErrorString(e));
     configured = true;
   }
@@ -445,8 +572,11 @@ gdn_status_t launch_typed(DecodeParams p, cudaStream_t stream) {
     const gdn_status_t st = pool_tensor_map<DK>(p, &map);
     if (st != GDN_OK) return st;
   }
-  gdn_decode_kernel<DK, TT, NH, TIn, TOut>
-      <<<grid, threads_per_row<TT, NH>() * DK + 32, L::kSmem, stream>>>(p, map);
+  if constexpr (L::kSwizzled)
+    gdn_decode_multi_kernel<DK, TT, NH, TIn, TOut><<<grid, 2 * DK + 32, L::kSmem, stream>>>(p, map);
+  else
+    gdn_decode_kernel<DK, TT, NH, TIn, TOut>
+        <<<grid, threads_per_row<TT, NH>() * DK + 32, L::kSmem, stream>>>(p, map);
   return check_launch("gdn_decode");
 }
 
