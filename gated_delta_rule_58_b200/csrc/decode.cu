@@ -119,7 +119,11 @@ __host__ __device__ constexpr int threads_per_row() { return 2; }
 // slot id, gates and betas go into the stage header and the state and the item's
 // k, q, v rows are bulk-copied into the stage; the stage's full barrier counts the
 // bytes. A stage is refilled once its previous item released it (empty barrier).
-template <int DK, int TT, int NH, typename TIn>
+// With kStores the consumers release a stage as soon as their arithmetic is done
+// and the producer writes the stage's state back to the pool (tensor stores of
+// the swizzled tiles) before it refills the stage, so the consumers never wait
+// for a store to drain.
+template <int DK, int TT, int NH, typename TIn, bool kStores>
 __device__ __forceinline__ void decode_producer(const DecodeParams& p, const CUtensorMap* pool_map, uint8_t* base,
                                                 uint64_t* full, uint64_t* empty) {
   using L = StageLayout<DK, TT, NH, TIn>;
@@ -128,6 +132,17 @@ __device__ __forceinline__ void decode_producer(const DecodeParams& p, const CUt
   const TIn* kp = static_cast<const TIn*>(p.k);
   const TIn* qp = static_cast<const TIn*>(p.q);
   const TIn* vp = static_cast<const TIn*>(p.v);
+  // state of the stage's finished item `prev` -> pool
+  auto store_stage = [&](int prev, uint8_t* st) {
+    const int prev_item = blockIdx.x + prev * gridDim.x;
+    const int ph = prev_item - (prev_item / p.H) * p.H;
+    const int pslot = *reinterpret_cast<const int*>(st + L::kHeader);
+    if (pslot < 0) return;
+#pragma unroll
+    for (int x = 0; x < DK / 32; ++x)
+      tc::tma_store_3d(pool_map, 32 * x, 0, pslot * p.H + ph, tc::smem_u32(st) + x * DK * 128);
+    tc::bulk_commit();
+  };
   int it = 0;
   for (int item = blockIdx.x; item < p.n_items; item += gridDim.x, ++it) {
     const int s = it % NS;
@@ -136,6 +151,12 @@ __device__ __forceinline__ void decode_producer(const DecodeParams& p, const CUt
       return;
     }
     uint8_t* st = base + s * L::kBytes;
+    if constexpr (kStores) {
+      if (it >= NS) {
+        store_stage(it - NS, st);
+        tc::bulk_wait_read();  // the stores have read the stage: it may be refilled
+      }
+    }
     const int b = item / p.H, h = item - (item / p.H) * p.H;
     int slot = __ldg(p.slot_ids + b);
     if (slot >= p.num_slots) {
@@ -172,6 +193,18 @@ __device__ __forceinline__ void decode_producer(const DecodeParams& p, const CUt
       tc::bulk_load(sst + L::kValues + t * NH * L::kRow, vp + bth * NH * DK, NH * L::kRow, &full[s]);
     }
   }
+  if constexpr (kStores) {
+    // the last items' states: each once its consumers are done with it
+    for (int prev = (it > NS ? it - NS : 0); prev < it; ++prev) {
+      const int s = prev % NS;
+      if (!tc::mbar_wait(&empty[s], (prev / NS) & 1, kDecodeWaitNs)) {
+        raise_device_error(p.err, GDN_DEVERR_TIMEOUT);
+        break;
+      }
+      store_stage(prev, base + s * L::kBytes);
+    }
+    tc::bulk_wait_all();
+  }
 }
 
 // Single-token step (T = n_h = 1): 2 threads per state row, all consumers on one item.
@@ -203,7 +236,7 @@ gdn_decode_kernel(const DecodeParams p, const __grid_constant__ CUtensorMap pool
   __syncthreads();
 
   if (tid >= kConsumers) {
-    if (tid == kConsumers) decode_producer<DK, TT, NH, TIn>(p, &pool_map, base, full, empty);
+    if (tid == kConsumers) decode_producer<DK, TT, NH, TIn, false>(p, &pool_map, base, full, empty);
     return;
   }
 
@@ -325,7 +358,7 @@ gdn_decode_multi_kernel(const DecodeParams p, const __grid_constant__ CUtensorMa
   __syncthreads();
 
   if (tid >= kConsumers) {
-    if (tid == kConsumers) decode_producer<DK, TT, NH, TIn>(p, &pool_map, base, full, empty);
+    if (tid == kConsumers) decode_producer<DK, TT, NH, TIn, true>(p, &pool_map, base, full, empty);
     return;
   }
 
@@ -513,22 +546,12 @@ gdn_decode_multi_kernel(const DecodeParams p, const __grid_constant__ CUtensorMa
         store_out(orow + (half == 0 ? r0 : r1), 0.f);
       }
     }
-    // stage -> pool (tensor stores of the swizzled tiles); the stage goes back to
-    // the producer as soon as the stores have read it
+    // the stage goes back to the producer, which stores the state to the pool
+    // (the writes are made visible to its tensor stores first)
     tc::fence_proxy_async_smem();
     tc::named_sync(bar_id, kGroupThreads);
-    if (gt == 0) {
-      if (slot >= 0) {
-#pragma unroll
-        for (int x = 0; x < DK / 32; ++x)
-          tc::tma_store_3d(&pool_map, 32 * x, 0, slot * p.H + h, tc::smem_u32(st) + x * DK * 128);
-        tc::bulk_commit();
-        tc::bulk_wait_read();
-      }
-      tc::mbar_arrive(&empty[s]);
-    }
+    if (gt == 0) tc::mbar_arrive(&empty[s]);
   }
-  if (gt == 0) tc::bulk_wait_all();
 }
 
 // The pool as a 3-D fp32 tensor {DK columns, DK rows, num_slots * H states}; a box
