@@ -146,6 +146,17 @@ __device__ __forceinline__ void decode_producer(const DecodeParams& p, const CUt
   int it = 0;
   for (int item = blockIdx.x; item < p.n_items; item += gridDim.x, ++it) {
     const int s = it % NS;
+    // the item's scalars are loaded before the stage wait, which hides their latency
+    const int b = item / p.H, h = item - (item / p.H) * p.H;
+    int slot = __ldg(p.slot_ids + b);
+    float gv[TT], bv[M];
+#pragma unroll
+    for (int t = 0; t < TT; ++t) gv[t] = __ldg(p.g + ((size_t)b * TT + t) * p.H + h);
+#pragma unroll
+    for (int m = 0; m < M; ++m) {
+      const int t = m / NH, mm = m - t * NH;
+      bv[m] = __ldg(p.beta + (((size_t)b * TT + t) * p.H + h) * NH + mm);
+    }
     if (it >= NS && !tc::mbar_wait(&empty[s], ((it / NS) & 1) ^ 1, kDecodeWaitNs)) {
       raise_device_error(p.err, GDN_DEVERR_TIMEOUT);
       return;
@@ -157,8 +168,6 @@ __device__ __forceinline__ void decode_producer(const DecodeParams& p, const CUt
         tc::bulk_wait_read();  // the stores have read the stage: it may be refilled
       }
     }
-    const int b = item / p.H, h = item - (item / p.H) * p.H;
-    int slot = __ldg(p.slot_ids + b);
     if (slot >= p.num_slots) {
       raise_device_error(p.err, GDN_DEVERR_SLOT_OUT_OF_RANGE);
       slot = -1;
@@ -166,13 +175,9 @@ __device__ __forceinline__ void decode_producer(const DecodeParams& p, const CUt
     if (slot < 0) slot = -1;
     *reinterpret_cast<int*>(st + L::kHeader) = slot;
 #pragma unroll
-    for (int t = 0; t < TT; ++t)
-      reinterpret_cast<float*>(st + L::kAlpha)[t] = expf(__ldg(p.g + ((size_t)b * TT + t) * p.H + h));
+    for (int t = 0; t < TT; ++t) reinterpret_cast<float*>(st + L::kAlpha)[t] = expf(gv[t]);
 #pragma unroll
-    for (int m = 0; m < M; ++m) {
-      const int t = m / NH, mm = m - t * NH;
-      reinterpret_cast<float*>(st + L::kBeta)[m] = __ldg(p.beta + (((size_t)b * TT + t) * p.H + h) * NH + mm);
-    }
+    for (int m = 0; m < M; ++m) reinterpret_cast<float*>(st + L::kBeta)[m] = bv[m];
     if (slot < 0) {
       tc::mbar_arrive(&full[s]);
       continue;
