@@ -22,6 +22,7 @@ import hashlib
 import json
 import math
 import os
+import re
 import statistics
 import subprocess
 import sys
@@ -133,11 +134,19 @@ class ClockSampler:
                 "reasons": reasons, "samples": len(self.rows)}
 
 
+def source_code(text: str) -> str:
+    """The code of a C++/CUDA source: // and /* */ comments, trailing blanks and
+    empty lines removed, so an edit of comments alone keeps the hash."""
+    text = re.sub(r"/\*.*?\*/", "", text, flags=re.S)
+    lines = (re.sub(r"//.*$", "", l).rstrip() for l in text.splitlines())
+    return "\n".join(l for l in lines if l)
+
+
 def source_sha(*rel_paths) -> str:
     h = hashlib.sha256()
     for p in rel_paths:
-        with open(os.path.join(ROOT, p), "rb") as f:
-            h.update(f.read())
+        with open(os.path.join(ROOT, p), encoding="utf-8") as f:
+            h.update(source_code(f.read()).encode())
     return h.hexdigest()[:16]
 
 

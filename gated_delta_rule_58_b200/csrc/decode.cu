@@ -10,15 +10,17 @@
 // depend on how many registers the math needs:
 //
 //   persistent grid, one CTA per SM, items = (batch row, head) pairs
-//   producer warp : per item, slot id, gates and betas (scalar loads), then bulk
-//                   copies of the state (64 KiB at dk = 128) and of the item's
-//                   k, q, v rows into a free stage (2-3 stages), tracked by an
-//                   mbarrier's transaction count
+//   producer warp : per item, slot id, gates and betas (scalar loads issued
+//                   before it waits for a free stage), then bulk copies of the
+//                   state (64 KiB at dk = 128) and of the item's k, q, v rows into
+//                   the stage (2-3 stages), tracked by an mbarrier's transaction
+//                   count
 //   consumer warps: single token: two threads per state row load its halves from
 //                   shared memory into registers, do the arithmetic below and
-//                   write the row back; multi-token: two groups take alternate
-//                   items, a thread owning half of two rows; one thread per group
-//                   stores the stage to the pool
+//                   write the row back, and one consumer thread bulk-stores the
+//                   stage to the pool; multi-token: two groups take alternate
+//                   items, a thread owning half of two rows, and the producer
+//                   stores each finished stage to the pool before refilling it
 //
 // Arithmetic. Per row j (value column j of S, stored K-last as S^T[j, :]) the
 // step is M = T*n_h sub-steps (gate on the first sub-step of each token, then a
@@ -67,8 +69,8 @@ struct DecodeParams {
 // token steps load and store it as DK/32 tiles of [DK rows][32 fp32] through a
 // tensor map with the 128-byte swizzle: tile x holds columns 32x..32x+31, row j
 // at j * 128 bytes, its 16-byte chunk c at ((c ^ (j & 7)) * 16). Eight consecutive
-// rows then read one chunk index from eight different bank groups while every
-// thread of a warp reads the same key / query chunk (a broadcast).
+// rows then read one chunk index from eight different bank groups while the
+// threads of a half-warp read the same key / query chunk (a broadcast).
 template <int DK, int TT, int NH, typename TIn>
 struct StageLayout {
   static constexpr int M = TT * NH;
