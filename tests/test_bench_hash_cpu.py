@@ -1,0 +1,36 @@
+"""The kernel-code hash that keeps committed ncu traffic figures attached to a
+kernel: comments and blank lines do not change it, code does."""
+import os
+import sys
+
+ROOT = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
+sys.path.insert(0, ROOT)
+
+import bench  # noqa: E402
+
+
+def test_comments_and_blank_lines_do_not_change_the_code():
+    a = "int f(int x) {\n  return x + 1;  // one more\n}\n"
+    b = "// header\n/* block\n   comment */\nint f(int x) {\n\n  return x + 1;\n}\n"
+    assert bench.source_code(a) == bench.source_code(b)
+
+
+def test_a_code_change_changes_the_code():
+    a = "int f(int x) {\n  return x + 1;\n}\n"
+    b = "int f(int x) {\n  return x + 2;\n}\n"
+    assert bench.source_code(a) != bench.source_code(b)
+
+
+def test_committed_traffic_entries_match_the_sources():
+    """Every entry of profiles/ncu_traffic.json names a kernel whose source hashes
+    to the recorded value (else bench.py reports traffic as null)."""
+    import json
+    with open(os.path.join(ROOT, "profiles", "ncu_traffic.json")) as f:
+        entries = {k: v for k, v in json.load(f).items() if not k.startswith("_")}
+    src = {"gdn_decode_kernel": "decode.cu", "gdn_decode_multi_kernel": "decode.cu",
+           "gdn_prefill_fused_kernel": "prefill_fused.cu"}
+    for key, e in entries.items():
+        path = "gated_delta_rule_58_b200/csrc/" + src[key.split(":")[0]]
+        assert bench.source_sha(path) == e["source_sha"], key
+        assert bench.ncu_traffic(key, [path]) == e["dram_bytes_per_launch"]
+        assert os.path.exists(os.path.join(ROOT, "profiles", e["profile"]))

@@ -65,6 +65,20 @@ def test_decode_input_dtypes(dtype):
         _check_against_oracle(inp, o, pool, f"in={dtype} out={out}")
 
 
+@pytest.mark.parametrize("T,nh,dtype", [(4, 2, torch.float32), (8, 1, torch.bfloat16), (4, 2, torch.bfloat16)])
+def test_multi_token_many_items_per_cta(T, nh, dtype):
+    """Several items per CTA (B*H = 151*3 over at most 148 CTAs), so both consumer
+    groups cycle through the stages more than once, with skipped rows in between;
+    fp32 inputs and T=8 run with two stages, bf16 T=4 n_h=2 with three."""
+    inp = inputs.decode_inputs(151, T, 3, 128, 128, nh, 160, seed=21 + T + nh, dtype=dtype)
+    inp.slot_ids[5] = -1
+    inp.slot_ids[77] = -1
+    o, pool = _run(inp, out_dtype=torch.float32)
+    assert torch.all(o[5] == 0) and torch.all(o[77] == 0)
+    _check_against_oracle(inp, o, pool, f"many items T={T} nh={nh} {dtype}")
+    assert gdn.gdn_get_device_error() == 0
+
+
 def test_decode_weak_and_zero_decay():
     for g_range in ((0.0, 0.0), (0.0, 0.01)):
         inp = inputs.decode_inputs(8, 4, 4, 128, 128, 2, 16, seed=5, g_range=g_range)
