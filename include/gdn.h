@@ -60,7 +60,7 @@ typedef enum { GDN_BF16 = 0, GDN_F32 = 1 } gdn_dtype_t;
 /* Bits of the sticky device error word (gdn_get_device_error). */
 #define GDN_DEVERR_SLOT_OUT_OF_RANGE 0x1u  /* a slot id >= num_slots was skipped */
 #define GDN_DEVERR_BAD_CU_SEQLENS 0x2u     /* cu_seqlens not 0-based / non-decreasing / > total_T */
-#define GDN_DEVERR_TIMEOUT 0x4u            /* a bounded inter-CTA wait gave up */
+#define GDN_DEVERR_TIMEOUT 0x4u            /* a bounded wait inside a kernel gave up (2 s); the kernel unwound */
 
 /*
  * gdn_decode — one decode step over a slot-indexed state pool, updated in place.
