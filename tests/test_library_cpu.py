@@ -70,6 +70,18 @@ def test_workspace_size_queries(L):
     assert L.gdn_chunk_prefill_workspace_size(-1, 0, 1, 32, 32, 16, 0) == ctypes.c_size_t(-1).value
 
 
+
+def test_prefill_raw_stream_handle_needs_an_explicit_workspace(L):
+    """With a raw stream handle the binding cannot tie a workspace it allocates to
+    that stream, so it refuses before allocating or launching anything."""
+    import torch
+    q = torch.empty((128, 4, 128), dtype=torch.bfloat16)
+    g = torch.empty((128, 4))
+    cu = torch.tensor([0, 128], dtype=torch.int32)
+    assert gdn.gdn_chunk_prefill_workspace_size(1, 128, 4, 128, 128, 64, gdn.GDN_PREFILL_TRANSFER) > 0
+    with pytest.raises(ValueError, match="raw handle"):
+        gdn.gdn_chunk_prefill(q, q, q, g, g, cu, q, algo=gdn.GDN_PREFILL_TRANSFER, stream=12345)
+
 def _prefill(L, **kw):
     a = dict(q=FAKE, k=FAKE, v=FAKE, g=FAKE, beta=FAKE, cu=FAKE, N=1, total=64, init=None, fin=FAKE,
              o=FAKE, H=2, dk=32, dv=32, chunk=16, scale=0.1, din=1, dout=1, algo=0, ws=None, wsb=0,
