@@ -160,9 +160,9 @@ def gdn_chunk_prefill(q, k, v, g, beta, cu_seqlens, o, initial_state=None, final
     """Chunked varlen prefill (see include/gdn.h). Shapes: q,k [total_T,H,dk], v [total_T,H,dv],
     g,beta [total_T,H] fp32, cu_seqlens [N+1] int32 (device), initial/final_state [N,H,dv,dk] fp32,
     o [total_T,H,dv]. `workspace` is a uint8 CUDA tensor; when None one of the required size is
-    allocated through torch for this call (and tied to `stream` when one is given, so torch does
-    not hand the memory out again before the call's kernels are done; a raw stream handle needs
-    an explicit `workspace`)."""
+    allocated through torch for this call, on `stream` when one is given, so torch orders any
+    reuse of that memory after the call's kernels; a raw stream handle needs an explicit
+    `workspace`."""
     import torch
     total_T, H, dk = q.shape
     dv = v.shape[-1]
@@ -171,11 +171,13 @@ def gdn_chunk_prefill(q, k, v, g, beta, cu_seqlens, o, initial_state=None, final
         scale = dk ** -0.5
     need = gdn_chunk_prefill_workspace_size(N, total_T, H, dk, dv, chunk, algo)
     if workspace is None and need > 0:
-        if stream is not None and not isinstance(stream, torch.cuda.Stream):
+        if stream is None:
+            workspace = torch.empty(need, dtype=torch.uint8, device=q.device)
+        elif isinstance(stream, torch.cuda.Stream):
+            with torch.cuda.stream(stream):  # the caching allocator orders reuse on this stream
+                workspace = torch.empty(need, dtype=torch.uint8, device=q.device)
+        else:
             raise ValueError("gdn_chunk_prefill: pass `workspace` when `stream` is a raw handle")
-        workspace = torch.empty(need, dtype=torch.uint8, device=q.device)
-        if stream is not None:
-            workspace.record_stream(stream)
     ws_ptr = _ptr(workspace)
     ws_bytes = workspace.numel() if workspace is not None else 0
     st = lib().gdn_chunk_prefill(_ptr(q), _ptr(k), _ptr(v), _ptr(g), _ptr(beta), _ptr(cu_seqlens), N,
