@@ -38,6 +38,7 @@
 #include <cstring>
 
 #include "common.cuh"
+#include "device_once.h"
 #include "tcgen05.cuh"
 #include "tensor_map.cuh"
 
@@ -574,12 +575,13 @@ gdn_status_t pool_tensor_map(const DecodeParams& p, CUtensorMap* map) {
 template <int DK, int TT, int NH, typename TIn, typename TOut>
 gdn_status_t launch_typed(DecodeParams p, cudaStream_t stream) {
   using L = StageLayout<DK, TT, NH, TIn>;
-  static int sm_count = 0;
-  static bool configured = false;
-  if (!configured) {
-    int dev = 0;
-    cudaError_t e = cudaGetDevice(&dev);
-    if (e == cudaSuccess) e = cudaDeviceGetAttribute(&sm_count, cudaDevAttrMultiProcessorCount, dev);
+  // per device: the SM count (grid size) and the shared-memory opt-in
+  static PerDeviceOnce once;
+  int dev = 0, sm_count = 0;
+  cudaError_t e = cudaGetDevice(&dev);
+  if (e != cudaSuccess) return fail(GDN_ERR_CUDA, std::string("gdn_decode: cudaGetDevice: ") + cudaGetErrorString(e));
+  const bool ready = run_once_per_device(once, dev, [&](int d, int* sms) {
+    e = cudaDeviceGetAttribute(sms, cudaDevAttrMultiProcessorCount, d);
     if (e == cudaSuccess) {
       if constexpr (L::kSwizzled)
         e = cudaFuncSetAttribute(gdn_decode_multi_kernel<DK, TT, NH, TIn, TOut>,
@@ -588,9 +590,11 @@ gdn_status_t launch_typed(DecodeParams p, cudaStream_t stream) {
         e = cudaFuncSetAttribute(gdn_decode_kernel<DK, TT, NH, TIn, TOut>,
                                  cudaFuncAttributeMaxDynamicSharedMemorySize, L::kSmem);
     }
-    if (e != cudaSuccess) return fail(GDN_ERR_CUDA, std::string("gdn_decode: setup: ") + cudaGetErrorString(e));
-    configured = true;
-  }
+    return e == cudaSuccess;
+  }, &sm_count);
+  if (!ready)
+    return fail(e != cudaSuccess ? GDN_ERR_CUDA : GDN_ERR_UNSUPPORTED,
+                std::string("gdn_decode: setup: ") + (e != cudaSuccess ? cudaGetErrorString(e) : "device index too large"));
   p.n_items = p.B * p.H;
   if (p.n_items == 0) return ok();
   const int grid = p.n_items < sm_count ? p.n_items : sm_count;

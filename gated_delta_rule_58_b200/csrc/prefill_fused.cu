@@ -45,6 +45,7 @@
 #include <cstring>
 #include <type_traits>
 
+#include "device_once.h"
 #include "prefill.cuh"
 #include "tcgen05.cuh"
 #include "tensor_map.cuh"
@@ -216,7 +217,7 @@ __device__ void loader_role(const Smem& sm, const PrefillShape& s, const Prefill
     uint8_t* v16 = sm.base + OFF_V + b * V_BUF;
     if constexpr (kTma) {
       // rows past the sequence end load the next tokens (or zeros past the tensor);
-      // their beta and g are set to 0 below, which removes them from every product
+      // they are zeroed once the copies have landed, and their beta and g are 0
       if (t == 0) {
         tc::fence_proxy_async_smem();  // the previous generic writes of these tiles precede the copies
         tc::mbar_arrive_expect_tx(sm.bar(B_T0 + b), (zero_values ? 2u : 3u) * 16384u);
@@ -266,6 +267,23 @@ __device__ void loader_role(const Smem& sm, const PrefillShape& s, const Prefill
       // the raw bf16 tiles feed [K;Q] K^T directly (bf16 MMA, exact inputs); they
       // are converted to fp16 in place once that MMA has read them
       if (!wait_bar(sm, B_T0 + b, (c >> 1) & 1, a.err)) return;
+      if (Lc < C) {
+        // Rows past the sequence end hold the next sequence's tokens (or zeros past
+        // the tensor). They are zeroed before any product reads them: beta = g = 0
+        // alone would leave 0 * x in the products, which is NaN for a non-finite x
+        // of the neighbour (or one outside the fp16 range after the conversion).
+        // In the 128-byte-swizzled tiles row r is the 128 bytes at r * 128.
+        const int nrows = C - Lc;
+        const int per_tile = nrows * 8;  // 16-byte chunks of the padded rows of one half tile
+        const int n_tiles = zero_values ? 4 : 6;  // K and Q halves, then V halves
+        for (int i = t; i < n_tiles * per_tile; i += 128) {
+          const int tile = i / per_tile, rem = i - tile * per_tile;
+          const int row = Lc + (rem >> 3), ch = rem & 7;
+          uint8_t* base = (tile < 4) ? kq + (tile >> 1) * KQ_HALF + (tile & 1) * (C * 128)
+                                     : v16 + (tile - 4) * V_HALF;
+          *reinterpret_cast<uint4*>(base + row * 128 + ch * 16) = make_uint4(0u, 0u, 0u, 0u);
+        }
+      }
       group_signal(sm, kBarLoad, B_L0 + b);
       if (!wait_bar(sm, B_M1, c & 1, a.err)) return;
       tc::fence_after_sync();
@@ -917,14 +935,17 @@ gdn_prefill_fused_kernel(const PrefillShape s, const PrefillArgs a, const __grid
 
 template <typename TIn, typename TOut>
 gdn_status_t launch(const PrefillShape& s, const PrefillArgs& a, cudaStream_t stream) {
-  static bool configured = false;
-  if (!configured) {
-    const cudaError_t e = cudaFuncSetAttribute(gdn_prefill_fused_kernel<TIn, TOut>,
-                                               cudaFuncAttributeMaxDynamicSharedMemorySize, SMEM_BYTES);
-    if (e != cudaSuccess)
-      return fail(GDN_ERR_CUDA, std::string("fused prefill: cudaFuncSetAttribute: ") + cudaGetErrorString(e));
-    configured = true;
-  }
+  static PerDeviceOnce once;  // the shared-memory opt-in applies to the current device only
+  int dev = 0;
+  cudaError_t e = cudaGetDevice(&dev);
+  if (e != cudaSuccess) return fail(GDN_ERR_CUDA, std::string("fused prefill: cudaGetDevice: ") + cudaGetErrorString(e));
+  if (!run_once_per_device(once, dev, [&](int, int*) {
+        e = cudaFuncSetAttribute(gdn_prefill_fused_kernel<TIn, TOut>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                 SMEM_BYTES);
+        return e == cudaSuccess;
+      }))
+    return fail(e != cudaSuccess ? GDN_ERR_CUDA : GDN_ERR_UNSUPPORTED,
+                std::string("fused prefill: setup: ") + (e != cudaSuccess ? cudaGetErrorString(e) : "device index too large"));
   const unsigned grid = (unsigned)((long long)s.N * s.H);
   QkvMaps maps;
   memset(&maps, 0, sizeof(maps));

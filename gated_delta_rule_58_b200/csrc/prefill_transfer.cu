@@ -26,6 +26,7 @@
 // more segments would add fixup steps without shortening those passes.
 #include <string>
 
+#include "device_once.h"
 #include "prefill.cuh"
 #include "tcgen05.cuh"
 
@@ -291,14 +292,17 @@ gdn_status_t prefill_transfer_launch(const PrefillShape& s, const PrefillArgs& a
   st = prefill_fused_launch(seg, tr, stream);
   if (st != GDN_OK) return st;
 
-  static bool fix_configured = false;
-  if (!fix_configured) {
-    const cudaError_t e =
-        cudaFuncSetAttribute(gdn_fixup_scan_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, kFixSmem);
-    if (e != cudaSuccess)
-      return fail(GDN_ERR_CUDA, std::string("transfer prefill: cudaFuncSetAttribute: ") + cudaGetErrorString(e));
-    fix_configured = true;
-  }
+  static PerDeviceOnce once;  // the shared-memory opt-in applies to the current device only
+  int dev = 0;
+  cudaError_t e = cudaGetDevice(&dev);
+  if (e != cudaSuccess) return fail(GDN_ERR_CUDA, std::string("transfer prefill: cudaGetDevice: ") + cudaGetErrorString(e));
+  if (!run_once_per_device(once, dev, [&](int, int*) {
+        e = cudaFuncSetAttribute(gdn_fixup_scan_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, kFixSmem);
+        return e == cudaSuccess;
+      }))
+    return fail(e != cudaSuccess ? GDN_ERR_CUDA : GDN_ERR_UNSUPPORTED,
+                std::string("transfer prefill: setup: ") +
+                    (e != cudaSuccess ? cudaGetErrorString(e) : "device index too large"));
   gdn_fixup_scan_kernel<<<(unsigned)((long long)s.N * s.H * (D / kFixRows)), kFixThreads, kFixSmem, stream>>>(
       seg_of_seq, s.H, local, transfer, fixed, a.initial_state, a.final_state, a.err);
   st = check_launch("transfer prefill: fixup scan");

@@ -6,7 +6,7 @@ import torch
 import oracle
 import gated_delta_rule_58_b200 as gdn
 from gated_delta_rule_58_b200 import inputs
-from tests.util import assert_close
+from tests.util import assert_close, cached
 
 pytestmark = pytest.mark.gpu
 DEV = "cuda"
@@ -161,34 +161,78 @@ def test_fused_many_sequences_launch_order(nseq):
         assert torch.equal(o_n, o[sl]) and torch.equal(f_n[0], fin[n])
 
 
-def test_fused_b4_t8192_h16_full_size():
-    """Chunked prefill at the benchmark size (B=4 x 8192, H=16), every (sequence, head)."""
-    inp = inputs.prefill_b4_t8192_h16()
-    check(inp, FUSED, what="B4 T8192 H16", out_dtype=torch.bfloat16)
+def _full_size(name):
+    """The named benchmark workload and its oracle results, computed once per process."""
+    def make():
+        inp = getattr(inputs, name)()
+        return inp, oracle_prefill(inp)
+    return cached(name, make)
 
 
-def _sampled_pairs_check(inp, algo, pairs, chunk=64):
-    o, fin = run_prefill(inp, algo, chunk=chunk, out_dtype=torch.bfloat16)
+@pytest.mark.parametrize("algo", [gdn.GDN_PREFILL_AUTO, FUSED])
+@pytest.mark.parametrize("out_dtype", [torch.float32, torch.bfloat16])
+def test_b4_t8192_h16_full_size(algo, out_dtype):
+    """Chunked prefill at the benchmark size (B=4 x 8192, H=16), every (sequence, head);
+    fp32 outputs are held to the 2e-3 normwise bar directly."""
+    inp, (o_ref, f_ref) = _full_size("prefill_b4_t8192_h16")
+    o, fin = run_prefill(inp, algo, out_dtype=out_dtype)
+    assert_close(o, o_ref, what=f"B4 T8192 H16 o ({out_dtype})")
+    assert_close(fin, f_ref, what=f"B4 T8192 H16 final state ({out_dtype})")
+
+
+@pytest.mark.parametrize("algo", [gdn.GDN_PREFILL_AUTO, FUSED])
+def test_varlen32_h32_every_pair(algo):
+    """Varlen 32 sequences x H=32 at full size (lengths ~U[64, 16384]), every
+    (sequence, head) against the oracle: fp32 outputs at 2e-3 normwise, bf16 outputs
+    element-wise, final states at 2e-3. The oracle runs one sequence at a time."""
+    inp = cached("varlen32_h32", inputs.varlen32_h32)
+    o32, fin = run_prefill(inp, algo, out_dtype=torch.float32)
+    o16, fin16 = run_prefill(inp, algo, out_dtype=torch.bfloat16)
+    assert torch.equal(fin, fin16)  # the state path does not depend on the output dtype
     cu = inp.cu_seqlens.tolist()
-    for n, h in pairs:
+    for n in range(len(cu) - 1):
         sl = slice(cu[n], cu[n + 1])
         L = cu[n + 1] - cu[n]
-        o_r, f_r, _ = oracle.prefill(inp.q[sl, h:h + 1], inp.k[sl, h:h + 1], inp.v[sl, h:h + 1],
-                                     inp.g[sl, h:h + 1], inp.beta[sl, h:h + 1], [0, L],
-                                     inp.initial_state[n:n + 1, h:h + 1], scale=inp.scale)
-        assert_close(o[sl, h:h + 1], o_r, what=f"pair ({n},{h}) o")
-        assert_close(fin[n:n + 1, h:h + 1], f_r, what=f"pair ({n},{h}) state")
+        o_r, f_r, _ = oracle.prefill(inp.q[sl], inp.k[sl], inp.v[sl], inp.g[sl], inp.beta[sl], [0, L],
+                                     inp.initial_state[n:n + 1], scale=inp.scale)
+        assert_close(o32[sl], o_r, what=f"varlen seq {n} (L={L}) o fp32")
+        assert_close(o16[sl], o_r, what=f"varlen seq {n} (L={L}) o bf16")
+        assert_close(fin[n:n + 1], f_r, what=f"varlen seq {n} (L={L}) state")
 
 
-def test_fused_varlen32_h32_sampled():
-    """Varlen 32 sequences x H=32 at full size; the oracle checks a seeded sample of
-    (sequence, head) pairs, including the longest and the shortest sequence."""
-    inp = inputs.varlen32_h32(device=DEV)
-    lens = inp.seqlens
-    longest, shortest = int(np.argmax(lens)), int(np.argmin(lens))
-    rng = np.random.default_rng(0)
-    pairs = [(longest, 0), (shortest, 31)] + [(int(rng.integers(32)), int(rng.integers(32))) for _ in range(4)]
-    _sampled_pairs_check(inp, FUSED, pairs)
+def _poisoned(inp, n, value):
+    """A copy of the packed inputs with every token of sequence n set to `value`
+    (q, k, v; g and beta too)."""
+    cu = inp.cu_seqlens.tolist()
+    sl = slice(cu[n], cu[n + 1])
+    out = inputs.PrefillInputs(inp.q.clone(), inp.k.clone(), inp.v.clone(), inp.g.clone(), inp.beta.clone(),
+                               inp.cu_seqlens.clone(), inp.initial_state.clone(), inp.scale)
+    for t in (out.q, out.k, out.v, out.g, out.beta):
+        t[sl] = value
+    return out
+
+
+@pytest.mark.parametrize("algo", [FUSED, gdn.GDN_PREFILL_TRANSFER])
+@pytest.mark.parametrize("value", [float("nan"), 1.0e5, float("inf")])
+def test_neighbour_data_cannot_leak_into_a_sequence(algo, value):
+    """The last, partial chunk of a sequence is loaded together with the first tokens
+    of the next sequence. Whatever those tokens hold (NaN, inf, or a value beyond the
+    fp16 range), the sequence's outputs and final state must be bitwise those of a
+    call with clean neighbours."""
+    lens = [100, 37, 256, 65]
+    inp = inputs.prefill_inputs(lens, 2, 128, 128, seed=27, g_range=(0.0, 0.02))
+    o_ref, f_ref = run_prefill(inp, algo)
+    cu = inp.cu_seqlens.tolist()
+    for bad in (1, 2, 3):  # poison sequence `bad`; sequence bad-1 ends in a partial chunk
+        o, fin = run_prefill(_poisoned(inp, bad, value), algo)
+        good = bad - 1
+        sl = slice(cu[good], cu[good + 1])
+        assert torch.equal(o[sl], o_ref[sl]), f"sequence {good} outputs changed by its neighbour ({value})"
+        assert torch.equal(fin[good], f_ref[good]), f"sequence {good} state changed by its neighbour ({value})"
+        for other in range(len(lens)):
+            if other != bad:
+                slo = slice(cu[other], cu[other + 1])
+                assert torch.equal(o[slo], o_ref[slo]) and torch.equal(fin[other], f_ref[other])
 
 
 # ---------------------------------------------------------------- transfer (chunk-parallel fixup) path
@@ -224,8 +268,13 @@ def test_transfer_matches_fused():
     assert_close(f_t, f_f, what="transfer vs fused state")
 
 
-def test_transfer_b1_t65536_h4_full_size():
-    """Low-parallelism prefill at the benchmark size (B=1 x 65536, H=4), every head."""
-    inp = inputs.longseq_b1_t65536_h4()
-    check(inp, TRANSFER, what="B1 T65536 H4", out_dtype=torch.bfloat16)
-
+@pytest.mark.parametrize("algo,out_dtype", [(gdn.GDN_PREFILL_AUTO, torch.float32),
+                                             (gdn.GDN_PREFILL_AUTO, torch.bfloat16),
+                                             (FUSED, torch.float32)])
+def test_b1_t65536_h4_full_size(algo, out_dtype):
+    """Low-parallelism prefill at the benchmark size (B=1 x 65536, H=4), every head;
+    AUTO takes the transfer (chunk-parallel fixup) path here."""
+    inp, (o_ref, f_ref) = _full_size("longseq_b1_t65536_h4")
+    o, fin = run_prefill(inp, algo, out_dtype=out_dtype)
+    assert_close(o, o_ref, what=f"B1 T65536 H4 o ({out_dtype})")
+    assert_close(fin, f_ref, what=f"B1 T65536 H4 final state ({out_dtype})")

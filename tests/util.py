@@ -49,3 +49,14 @@ def assert_close(x, ref, tol=TOL, what=""):
     else:
         e = relerr(xa, ra)
         assert e <= tol, f"{what}: normwise relative error {e:.3e} > {tol}"
+
+
+_CACHE = {}
+
+
+def cached(key, fn):
+    """fn() once per test process under `key` (the oracle's full-size results and
+    the inputs they were computed from are reused by several tests)."""
+    if key not in _CACHE:
+        _CACHE[key] = fn()
+    return _CACHE[key]
