@@ -505,6 +505,53 @@ def oracle_decode_rate(key, budget_s=10.0, seed=0):
             f"{dt:.1f} s")
 
 
+def oracle_prefill_rate(key, budget_s=4.0, seed=0):
+    """cpu_baseline of a prefill part: the fp64 oracle on the first L tokens of every
+    sequence of the workload (all heads), L chosen from a short calibration run so
+    the timed call takes about budget_s. Returns tokens/s (a token = all H heads of
+    one position, as in the GPU metric), the threads used and the sample."""
+    import numpy as np
+    import oracle
+    gen_dev = "cuda" if torch.cuda.is_available() else "cpu"  # the sample is copied to the host
+    inp, _, name = prefill_cfg(key, gen_dev, seed)
+    cu = inp.cu_seqlens.tolist()
+    N = len(cu) - 1
+    H = inp.q.shape[1]
+    longest = max(cu[n + 1] - cu[n] for n in range(N))
+
+    def sample(L):
+        lens = [min(L, cu[n + 1] - cu[n]) for n in range(N)]
+        idx = torch.cat([torch.arange(cu[n], cu[n] + lens[n]) for n in range(N)])
+        new_cu = np.concatenate([[0], np.cumsum(lens)]).astype(np.int64)
+        idx_dev = idx.to(inp.q.device)
+        args = [oracle.f64(t[idx_dev]) for t in (inp.q, inp.k, inp.v, inp.g, inp.beta)]
+        return args, new_cu, int(new_cu[-1])
+
+    init = oracle.f64(inp.initial_state)
+
+    def timed(L, reps=1):
+        args, new_cu, tokens = sample(L)
+        t0 = time.perf_counter()
+        for _ in range(reps):
+            _, _, threads = oracle.prefill(*args, new_cu, init, scale=inp.scale)
+        return time.perf_counter() - t0, threads, tokens * reps
+
+    L = min(64, longest)
+    dt, threads, tokens = timed(L)
+    reps = 1
+    if L < longest:
+        L = max(L, min(longest, int(L * budget_s / max(dt, 1e-3)) // 64 * 64))
+        dt, threads, tokens = timed(L)
+    else:  # the whole workload is short: repeat it
+        reps = max(1, int(budget_s / max(dt, 1e-4)))
+        dt, threads, tokens = timed(L, reps)
+    note = f" ({N * H} (sequence, head) chains: at most {N * H} threads)" if N * H < 16 else ""
+    rep = f", {reps} calls" if reps > 1 else ""
+    return (tokens / dt, threads,
+            f"oracle on the first {L} tokens of each of the {N} sequences x {H} heads "
+            f"({tokens // reps} tokens{rep}) of '{name}', {dt:.1f} s{note}")
+
+
 def run_reference(args, ws, rank):
     """The reference arm: the fp64 CPU oracle on the headline workload, on rank 0 only.
     Each step is a bounded sample (the first rows of the batch, all heads), sized so the
@@ -601,6 +648,17 @@ def main():
         if not args.no_cpu_baseline and ws == 1:
             v, threads, sample = oracle_decode_rate("decode", budget_s=10.0)
             cpu = {"value": v, "unit": "GB/s", "cores": threads, "kind": "oracle", "sample": sample}
+            for r in parts:  # every part gets the oracle's rate in the part's own unit
+                if "error" in r:
+                    continue
+                if r["key"] == "gdp":
+                    v, threads, sample = oracle_decode_rate("gdp", budget_s=4.0)
+                    r["cpu_baseline"] = {"value": v, "unit": "GB/s", "cores": threads, "kind": "oracle",
+                                         "sample": sample}
+                else:
+                    v, threads, sample = oracle_prefill_rate(r["key"], budget_s=4.0)
+                    r["cpu_baseline"] = {"value": v, "unit": "tokens/s", "cores": threads, "kind": "oracle",
+                                         "sample": sample}
         clocks = clk.summary()
         line = {
             "metric": METRIC,
