@@ -223,6 +223,13 @@ def time_graph(fn, steps, warmup, ws):
 DECODE_CFGS = {
     "decode": dict(B=64, T=1, H=32, d=128, nh=1, slots=256,
                    name="decode T=1, B=64, H=32, dk=dv=128, fp32 pool of 256 slots, bf16 q/k/v"),
+    # small batches: the T=1 step splits each head's state rows over several CTAs
+    "decode_b1": dict(B=1, T=1, H=32, d=128, nh=1, slots=512,
+                      name="decode T=1, B=1, H=32, dk=dv=128, fp32 pool of 512 slots (split along V)"),
+    "decode_b4": dict(B=4, T=1, H=32, d=128, nh=1, slots=512,
+                      name="decode T=1, B=4, H=32, dk=dv=128, fp32 pool of 512 slots (split along V)"),
+    "decode_b16": dict(B=16, T=1, H=32, d=128, nh=1, slots=512,
+                       name="decode T=1, B=16, H=32, dk=dv=128, fp32 pool of 512 slots (split along V)"),
     "gdp": dict(B=128, T=4, H=32, d=128, nh=2, slots=512,
                 name="gated delta product decode, B=128, H=32, T=4, n_h=2, dk=dv=128, pool of 512 slots"),
 }
@@ -589,7 +596,7 @@ def main():
     ap.add_argument("--steps", type=int, default=2000)
     ap.add_argument("--warmup", type=int, default=20)
     ap.add_argument("--impl", default="ours", choices=["ours", "reference"])
-    ap.add_argument("--parts", default="gdp,prefill,varlen,longseq,tiny",
+    ap.add_argument("--parts", default="gdp,decode_b1,decode_b4,decode_b16,prefill,varlen,longseq,tiny",
                     help="comma list of extra workloads to measure ('none' for none)")
     ap.add_argument("--part-steps", type=int, default=5)
     ap.add_argument("--no-cpu-baseline", action="store_true")
@@ -626,10 +633,10 @@ def main():
         for key in [p for p in args.parts.split(",") if p and p != "none"]:
             torch.cuda.nvtx.range_push(key)
             try:
-                if key == "gdp":
-                    r = bench_decode("gdp", max(args.part_steps * 20, 20), args.warmup, ws, rank, peaks,
+                if key in DECODE_CFGS:
+                    r = bench_decode(key, max(args.part_steps * 20, 20), args.warmup, ws, rank, peaks,
                                      e2e=False)
-                    r["metric"] = "GDP decode state GB/s"
+                    r["metric"] = "GDP decode state GB/s" if key == "gdp" else "decode state GB/s"
                 else:
                     r = bench_prefill(key, args.part_steps, 3, ws, rank, peaks, algo=algo)
                     r["metric"] = "prefill tokens/s"
@@ -651,8 +658,8 @@ def main():
             for r in parts:  # every part gets the oracle's rate in the part's own unit
                 if "error" in r:
                     continue
-                if r["key"] == "gdp":
-                    v, threads, sample = oracle_decode_rate("gdp", budget_s=4.0)
+                if r["key"] in DECODE_CFGS:
+                    v, threads, sample = oracle_decode_rate(r["key"], budget_s=2.0 if r["key"] != "gdp" else 4.0)
                     r["cpu_baseline"] = {"value": v, "unit": "GB/s", "cores": threads, "kind": "oracle",
                                          "sample": sample}
                 else:

@@ -72,12 +72,15 @@ struct DecodeParams {
 // at j * 128 bytes, its 16-byte chunk c at ((c ^ (j & 7)) * 16). Eight consecutive
 // rows then read one chunk index from eight different bank groups while the
 // threads of a half-warp read the same key / query chunk (a broadcast).
-template <int DK, int TT, int NH, typename TIn>
+template <int DK, int TT, int NH, typename TIn, int ROWS = DK>
 struct StageLayout {
   static constexpr int M = TT * NH;
   static constexpr bool kSwizzled = M > 1;
   static constexpr uint32_t kAlign = kSwizzled ? 1024 : 128;  // the swizzle follows address bits 4-9
-  static constexpr uint32_t kState = DK * DK * 4;
+  static constexpr int kRows = ROWS;                           // state rows (value indices) per item
+  static constexpr int kParts = DK / ROWS;                     // items per (batch row, head)
+  static_assert(!kSwizzled || ROWS == DK, "multi-token steps take whole heads");
+  static constexpr uint32_t kState = kRows * DK * 4;
   static constexpr uint32_t kRow = DK * sizeof(TIn);
   static constexpr uint32_t kKeys = kState;
   static constexpr uint32_t kQueries = kKeys + M * kRow;
@@ -126,10 +129,10 @@ __host__ __device__ constexpr int threads_per_row() { return 2; }
 // and the producer writes the stage's state back to the pool (tensor stores of
 // the swizzled tiles) before it refills the stage, so the consumers never wait
 // for a store to drain.
-template <int DK, int TT, int NH, typename TIn, bool kStores>
+template <int DK, int TT, int NH, typename TIn, bool kStores, int ROWS = DK>
 __device__ __forceinline__ void decode_producer(const DecodeParams& p, const CUtensorMap* pool_map, uint8_t* base,
                                                 uint64_t* full, uint64_t* empty) {
-  using L = StageLayout<DK, TT, NH, TIn>;
+  using L = StageLayout<DK, TT, NH, TIn, ROWS>;
   constexpr int M = L::M;
   constexpr int NS = L::kStages;
   const TIn* kp = static_cast<const TIn*>(p.k);
@@ -150,7 +153,8 @@ __device__ __forceinline__ void decode_producer(const DecodeParams& p, const CUt
   for (int item = blockIdx.x; item < p.n_items; item += gridDim.x, ++it) {
     const int s = it % NS;
     // the item's scalars are loaded before the stage wait, which hides their latency
-    const int b = item / p.H, h = item - (item / p.H) * p.H;
+    const int bh = item / L::kParts, part = item - bh * L::kParts;
+    const int b = bh / p.H, h = bh - (bh / p.H) * p.H;
     int slot = __ldg(p.slot_ids + b);
     float gv[TT], bv[M];
 #pragma unroll
@@ -191,7 +195,8 @@ __device__ __forceinline__ void decode_producer(const DecodeParams& p, const CUt
 #pragma unroll
       for (int x = 0; x < DK / 32; ++x) tc::tma_load_3d(sst + x * DK * 128, pool_map, 32 * x, 0, slot * p.H + h, &full[s]);
     } else {
-      tc::bulk_load(sst, p.pool + ((size_t)slot * p.H + h) * (size_t)DK * DK, L::kState, &full[s]);
+      tc::bulk_load(sst, p.pool + (((size_t)slot * p.H + h) * DK + (size_t)part * L::kRows) * DK, L::kState,
+                    &full[s]);
     }
 #pragma unroll
     for (int t = 0; t < TT; ++t) {
@@ -216,14 +221,19 @@ __device__ __forceinline__ void decode_producer(const DecodeParams& p, const CUt
 }
 
 // Single-token step (T = n_h = 1): 2 threads per state row, all consumers on one item.
-template <int DK, int TT, int NH, typename TIn, typename TOut>
-__global__ void __launch_bounds__(threads_per_row<TT, NH>() * DK + 32, 1)
+// An item is ROWS consecutive state rows (value indices) of one (batch row, head):
+// the whole head when there are enough heads to fill the GPU, a part of it (the
+// split along V) otherwise. Rows are independent in this step (each needs only the
+// head's k, q and its own v entry), so every row gets the same arithmetic in the
+// same order whatever ROWS is.
+template <int DK, int TT, int NH, typename TIn, typename TOut, int ROWS>
+__global__ void __launch_bounds__(threads_per_row<TT, NH>() * ROWS + 32, 1)
 gdn_decode_kernel(const DecodeParams p, const __grid_constant__ CUtensorMap pool_map) {
-  using L = StageLayout<DK, TT, NH, TIn>;
+  using L = StageLayout<DK, TT, NH, TIn, ROWS>;
   static_assert(L::M == 1, "single-token step");
   constexpr int NS = L::kStages;
   constexpr int TPR = threads_per_row<TT, NH>();
-  constexpr int kConsumers = TPR * DK;
+  constexpr int kConsumers = TPR * ROWS;
   constexpr int CPH = DK / (4 * TPR);        // float4 chunks per thread's part of a row
   constexpr int RPW = 32 / TPR;              // rows per warp
   constexpr uint32_t kBarConsumers = 1;
@@ -244,7 +254,7 @@ gdn_decode_kernel(const DecodeParams p, const __grid_constant__ CUtensorMap pool
   __syncthreads();
 
   if (tid >= kConsumers) {
-    if (tid == kConsumers) decode_producer<DK, TT, NH, TIn, false>(p, &pool_map, base, full, empty);
+    if (tid == kConsumers) decode_producer<DK, TT, NH, TIn, false, ROWS>(p, &pool_map, base, full, empty);
     return;
   }
 
@@ -263,20 +273,23 @@ gdn_decode_kernel(const DecodeParams p, const __grid_constant__ CUtensorMap pool
       if (tid == 0) raise_device_error(p.err, GDN_DEVERR_TIMEOUT);
       break;
     }
-    const int b = item / p.H, h = item - (item / p.H) * p.H;
+    const int bh = item / L::kParts, part = item - bh * L::kParts;
+    const int b = bh / p.H, h = bh - (bh / p.H) * p.H;
+    const int grow = part * ROWS + row;  // the row's value index in the head
     const int slot = *reinterpret_cast<const int*>(st + L::kHeader);
     const float* alpha = reinterpret_cast<const float*>(st + L::kAlpha);
     const float* betas = reinterpret_cast<const float*>(st + L::kBeta);
     if (slot >= 0) {
-      // k.s, q.s and the Gram entry q.k in one pass over the half row
+      // k.s, q.s and the Gram entry q.k in one pass over the half row (the chunk
+      // order is rotated by the row, which spreads a warp's loads over the banks)
       float* srow = reinterpret_cast<float*>(st) + (size_t)row * DK + half * (DK / TPR);
       float4 sv[CPH];
 #pragma unroll
-      for (int c = 0; c < CPH; ++c) sv[c] = reinterpret_cast<const float4*>(srow)[(c + row) & (CPH - 1)];
+      for (int c = 0; c < CPH; ++c) sv[c] = reinterpret_cast<const float4*>(srow)[(c + grow) & (CPH - 1)];
       float ks = 0.f, qs = 0.f, qkv = 0.f;
 #pragma unroll
       for (int c = 0; c < CPH; ++c) {
-        const int e = half * (DK / TPR) + 4 * ((c + row) & (CPH - 1));
+        const int e = half * (DK / TPR) + 4 * ((c + grow) & (CPH - 1));
         float wk[4], wq[4];
         load4_f32<TIn>(st + L::kKeys + e * sizeof(TIn), wk);
         load4_f32<TIn>(st + L::kQueries + e * sizeof(TIn), wq);
@@ -288,12 +301,12 @@ gdn_decode_kernel(const DecodeParams p, const __grid_constant__ CUtensorMap pool
       qs += __shfl_xor_sync(0xffffffffu, qs, 16);
       qkv += __shfl_xor_sync(0xffffffffu, qkv, 16);
       const float a = alpha[0];
-      const float vj = to_f32(reinterpret_cast<const TIn*>(st + L::kValues)[row]);
+      const float vj = to_f32(reinterpret_cast<const TIn*>(st + L::kValues)[grow]);
       const float cm = betas[0] * (vj - a * ks);
-      if (half == 0) store_out(op + ((size_t)b * p.H + h) * DK + row, p.scale * fmaf(cm, qkv, a * qs));
+      if (half == 0) store_out(op + ((size_t)b * p.H + h) * DK + grow, p.scale * fmaf(cm, qkv, a * qs));
 #pragma unroll
       for (int c = 0; c < CPH; ++c) {
-        const int e = half * (DK / TPR) + 4 * ((c + row) & (CPH - 1));
+        const int e = half * (DK / TPR) + 4 * ((c + grow) & (CPH - 1));
         float wk[4];
         load4_f32<TIn>(st + L::kKeys + e * sizeof(TIn), wk);
         float4 x = sv[c];
@@ -301,18 +314,20 @@ gdn_decode_kernel(const DecodeParams p, const __grid_constant__ CUtensorMap pool
         x.y = fmaf(cm, wk[1], a * x.y);
         x.z = fmaf(cm, wk[2], a * x.z);
         x.w = fmaf(cm, wk[3], a * x.w);
-        reinterpret_cast<float4*>(srow)[(c + row) & (CPH - 1)] = x;
+        reinterpret_cast<float4*>(srow)[(c + grow) & (CPH - 1)] = x;
       }
     } else if (half == 0) {
       // skipped row of the batch: o = 0, pool untouched
-      store_out(op + ((size_t)b * p.H + h) * DK + row, 0.f);
+      store_out(op + ((size_t)b * p.H + h) * DK + grow, 0.f);
     }
     // stage -> pool (one bulk store); the previous item's stage is handed back to
     // the producer once its store has finished reading shared memory
     tc::fence_proxy_async_smem();
     tc::named_sync(kBarConsumers, kConsumers);
     if (tid == 0) {
-      if (slot >= 0) tc::bulk_store(p.pool + ((size_t)slot * p.H + h) * (size_t)DK * DK, tc::smem_u32(st), L::kState);
+      if (slot >= 0)
+        tc::bulk_store(p.pool + (((size_t)slot * p.H + h) * DK + (size_t)part * ROWS) * DK, tc::smem_u32(st),
+                       L::kState);
       tc::bulk_commit();
       tc::bulk_wait_read_1();
       if (prev_stage >= 0) tc::mbar_arrive(&empty[prev_stage]);
@@ -572,8 +587,9 @@ gdn_status_t pool_tensor_map(const DecodeParams& p, CUtensorMap* map) {
   return make_tensor_map_3d(map, CU_TENSOR_MAP_DATA_TYPE_FLOAT32, p.pool, dims, strides, box, "gdn_decode");
 }
 
+// Multi-token / product step: one CTA per SM, whole heads.
 template <int DK, int TT, int NH, typename TIn, typename TOut>
-gdn_status_t launch_typed(DecodeParams p, cudaStream_t stream) {
+gdn_status_t launch_multi(DecodeParams p, cudaStream_t stream) {
   using L = StageLayout<DK, TT, NH, TIn>;
   // per device: the SM count (grid size) and the shared-memory opt-in
   static PerDeviceOnce once;
@@ -582,14 +598,9 @@ gdn_status_t launch_typed(DecodeParams p, cudaStream_t stream) {
   if (e != cudaSuccess) return fail(GDN_ERR_CUDA, std::string("gdn_decode: cudaGetDevice: ") + cudaGetErrorString(e));
   const bool ready = run_once_per_device(once, dev, [&](int d, int* sms) {
     e = cudaDeviceGetAttribute(sms, cudaDevAttrMultiProcessorCount, d);
-    if (e == cudaSuccess) {
-      if constexpr (L::kSwizzled)
-        e = cudaFuncSetAttribute(gdn_decode_multi_kernel<DK, TT, NH, TIn, TOut>,
-                                 cudaFuncAttributeMaxDynamicSharedMemorySize, L::kSmem);
-      else
-        e = cudaFuncSetAttribute(gdn_decode_kernel<DK, TT, NH, TIn, TOut>,
-                                 cudaFuncAttributeMaxDynamicSharedMemorySize, L::kSmem);
-    }
+    if (e == cudaSuccess)
+      e = cudaFuncSetAttribute(gdn_decode_multi_kernel<DK, TT, NH, TIn, TOut>,
+                               cudaFuncAttributeMaxDynamicSharedMemorySize, L::kSmem);
     return e == cudaSuccess;
   }, &sm_count);
   if (!ready)
@@ -598,20 +609,85 @@ gdn_status_t launch_typed(DecodeParams p, cudaStream_t stream) {
   p.n_items = p.B * p.H;
   if (p.n_items == 0) return ok();
   const int grid = p.n_items < sm_count ? p.n_items : sm_count;
+  if ((long long)p.num_slots * p.H >= (1LL << 31))
+    return fail(GDN_ERR_UNSUPPORTED, "gdn_decode: num_slots * H must be below 2^31 for multi-token steps");
   CUtensorMap map;
   memset(&map, 0, sizeof(map));
-  if constexpr (L::kSwizzled) {
-    if ((long long)p.num_slots * p.H >= (1LL << 31))
-      return fail(GDN_ERR_UNSUPPORTED, "gdn_decode: num_slots * H must be below 2^31 for multi-token steps");
-    const gdn_status_t st = pool_tensor_map<DK>(p, &map);
-    if (st != GDN_OK) return st;
-  }
-  if constexpr (L::kSwizzled)
-    gdn_decode_multi_kernel<DK, TT, NH, TIn, TOut><<<grid, 2 * DK + 32, L::kSmem, stream>>>(p, map);
-  else
-    gdn_decode_kernel<DK, TT, NH, TIn, TOut>
-        <<<grid, threads_per_row<TT, NH>() * DK + 32, L::kSmem, stream>>>(p, map);
+  const gdn_status_t st = pool_tensor_map<DK>(p, &map);
+  if (st != GDN_OK) return st;
+  gdn_decode_multi_kernel<DK, TT, NH, TIn, TOut><<<grid, 2 * DK + 32, L::kSmem, stream>>>(p, map);
   return check_launch("gdn_decode");
+}
+
+// Single-token step with ROWS state rows per item; persistent grid of as many CTAs
+// as fit on the device at once (one per SM for whole heads, several for parts).
+template <int DK, typename TIn, typename TOut, int ROWS>
+gdn_status_t launch_single_rows(DecodeParams p, cudaStream_t stream) {
+  using L = StageLayout<DK, 1, 1, TIn, ROWS>;
+  constexpr int kThreadsPerCta = threads_per_row<1, 1>() * ROWS + 32;
+  auto kernel = gdn_decode_kernel<DK, 1, 1, TIn, TOut, ROWS>;
+  static PerDeviceOnce once;  // per device: SMs x resident CTAs, and the shared-memory opt-in
+  int dev = 0, slots = 0;
+  cudaError_t e = cudaGetDevice(&dev);
+  if (e != cudaSuccess) return fail(GDN_ERR_CUDA, std::string("gdn_decode: cudaGetDevice: ") + cudaGetErrorString(e));
+  const bool ready = run_once_per_device(once, dev, [&](int d, int* out) {
+    int sms = 0, per_sm = 0;
+    e = cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, d);
+    if (e == cudaSuccess) e = cudaFuncSetAttribute(kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, L::kSmem);
+    if (e == cudaSuccess)
+      e = cudaOccupancyMaxActiveBlocksPerMultiprocessor(&per_sm, kernel, kThreadsPerCta, L::kSmem);
+    *out = sms * (per_sm > 0 ? per_sm : 1);
+    return e == cudaSuccess;
+  }, &slots);
+  if (!ready)
+    return fail(e != cudaSuccess ? GDN_ERR_CUDA : GDN_ERR_UNSUPPORTED,
+                std::string("gdn_decode: setup: ") + (e != cudaSuccess ? cudaGetErrorString(e) : "device index too large"));
+  p.n_items = p.B * p.H * L::kParts;
+  if (p.n_items == 0) return ok();
+  const int grid = p.n_items < slots ? p.n_items : slots;
+  CUtensorMap map;  // unused by the single-token step (linear bulk copies)
+  memset(&map, 0, sizeof(map));
+  kernel<<<grid, kThreadsPerCta, L::kSmem, stream>>>(p, map);
+  return check_launch("gdn_decode");
+}
+
+// Parts per head for the single-token step: whole heads when there are at least
+// four per SM, else the smallest power-of-two split (rows per part >= 16) that
+// reaches four items per SM, so that every SM streams state even at small batch
+// (the T=1 split-V idea of the FlashInfer PR #7156 page, introduction).
+inline int decode_parts(long long heads, int sm_count, int dk) {
+  int parts = 1;
+  while (parts * 2 <= dk / 16 && heads * parts < 4LL * sm_count) parts *= 2;
+  return parts;
+}
+
+template <int DK, typename TIn, typename TOut>
+gdn_status_t launch_single(DecodeParams p, cudaStream_t stream) {
+  static PerDeviceOnce once;
+  int dev = 0, sms = 0;
+  cudaError_t e = cudaGetDevice(&dev);
+  if (e == cudaSuccess && !run_once_per_device(once, dev, [&](int d, int* out) {
+        e = cudaDeviceGetAttribute(out, cudaDevAttrMultiProcessorCount, d);
+        return e == cudaSuccess;
+      }, &sms))
+    if (e == cudaSuccess) return fail(GDN_ERR_UNSUPPORTED, "gdn_decode: device index too large");
+  if (e != cudaSuccess) return fail(GDN_ERR_CUDA, std::string("gdn_decode: ") + cudaGetErrorString(e));
+  switch (decode_parts((long long)p.B * p.H, sms, DK)) {
+    case 1: return launch_single_rows<DK, TIn, TOut, DK>(p, stream);
+    case 2: if constexpr (DK / 2 >= 16) return launch_single_rows<DK, TIn, TOut, DK / 2>(p, stream); break;
+    case 4: if constexpr (DK / 4 >= 16) return launch_single_rows<DK, TIn, TOut, DK / 4>(p, stream); break;
+    case 8: if constexpr (DK / 8 >= 16) return launch_single_rows<DK, TIn, TOut, DK / 8>(p, stream); break;
+    default: break;
+  }
+  return fail(GDN_ERR_UNSUPPORTED, "gdn_decode: no split for this head size");
+}
+
+template <int DK, int TT, int NH, typename TIn, typename TOut>
+gdn_status_t launch_typed(DecodeParams p, cudaStream_t stream) {
+  if constexpr (TT == 1 && NH == 1)
+    return launch_single<DK, TIn, TOut>(p, stream);
+  else
+    return launch_multi<DK, TT, NH, TIn, TOut>(p, stream);
 }
 
 template <int DK, int TT, int NH>

@@ -49,13 +49,13 @@ def _declare(lib):
     dp = ctypes.POINTER(ctypes.c_double)
     lib.gdn_oracle_prefill.restype = ctypes.c_int
     lib.gdn_oracle_prefill.argtypes = [dp, dp, dp, dp, dp, ctypes.POINTER(ctypes.c_int64),
-                                       ctypes.c_int, ctypes.c_int, ctypes.c_int, ctypes.c_int,
-                                       ctypes.c_double, dp, dp, dp, ctypes.c_int]
+                                       ctypes.c_int, ctypes.c_int, ctypes.c_int, ctypes.c_int, ctypes.c_int,
+                                       ctypes.c_double, ctypes.c_int, dp, dp, dp, ctypes.c_int]
     lib.gdn_oracle_decode.restype = ctypes.c_int
     lib.gdn_oracle_decode.argtypes = [dp, dp, dp, dp, dp, dp, ctypes.c_int,
                                       ctypes.POINTER(ctypes.c_int32), dp,
-                                      ctypes.c_int, ctypes.c_int, ctypes.c_int, ctypes.c_int,
-                                      ctypes.c_int, ctypes.c_int, ctypes.c_double, ctypes.c_int]
+                                      ctypes.c_int, ctypes.c_int, ctypes.c_int, ctypes.c_int, ctypes.c_int,
+                                      ctypes.c_int, ctypes.c_int, ctypes.c_double, ctypes.c_int, ctypes.c_int]
 
 
 def _load():
@@ -88,36 +88,40 @@ def _ptr(a, ctype=ctypes.c_double):
     return a.ctypes.data_as(ctypes.POINTER(ctype))
 
 
-def prefill(q, k, v, g, beta, cu_seqlens, initial_state=None, scale=None, nthreads=0, lib=None):
+def prefill(q, k, v, g, beta, cu_seqlens, initial_state=None, scale=None, nthreads=0, lib=None,
+            l2norm=False):
     """Sequential fp64 prefill over packed sequences.
 
-    q, k: [total_T, H, dk]; v: [total_T, H, dv]; g, beta: [total_T, H];
+    q, k: [total_T, H_qk, dk] (H a multiple of H_qk; value head h reads q/k head
+    h // (H // H_qk)); v: [total_T, H, dv]; g, beta: [total_T, H];
     cu_seqlens: [N + 1]; initial_state: [N, H, dv, dk] or None (zero state).
+    l2norm: scale q and k to unit length per token (in fp64) before use.
     Returns (o [total_T, H, dv], final_state [N, H, dv, dk], threads_used), fp64.
     """
     lib = lib or _load()
     q, k, v, g, beta = (f64(a) for a in (q, k, v, g, beta))
     cu = np.ascontiguousarray(np.asarray(f64(cu_seqlens), dtype=np.int64))
     init = f64(initial_state)
-    total_T, H, dk = q.shape
-    dv = v.shape[-1]
+    total_T, Hqk, dk = q.shape
+    H, dv = v.shape[1], v.shape[-1]
     N = cu.shape[0] - 1
     if scale is None:
         scale = 1.0 / np.sqrt(dk)
     o = np.zeros((total_T, H, dv), np.float64)
     fin = np.zeros((N, H, dv, dk), np.float64)
     rc = lib.gdn_oracle_prefill(_ptr(q), _ptr(k), _ptr(v), _ptr(g), _ptr(beta),
-                                _ptr(cu, ctypes.c_int64), N, H, dk, dv, float(scale), _ptr(init),
-                                _ptr(o), _ptr(fin), int(nthreads))
+                                _ptr(cu, ctypes.c_int64), N, H, Hqk, dk, dv, float(scale), int(bool(l2norm)),
+                                _ptr(init), _ptr(o), _ptr(fin), int(nthreads))
     if rc < 0:
         raise ValueError("gdn_oracle_prefill: bad arguments")
     return o, fin, rc
 
 
-def decode(q, k, v, g, beta, pool, slot_ids, scale=None, nthreads=0, lib=None, copy_pool=True):
+def decode(q, k, v, g, beta, pool, slot_ids, scale=None, nthreads=0, lib=None, copy_pool=True,
+           l2norm=False):
     """Sequential fp64 decode over a slot-indexed pool (the pool copy is updated).
 
-    q: [B, T, H, dk]; k: [B, T, H, nh, dk]; v: [B, T, H, nh, dv]; g: [B, T, H];
+    q: [B, T, H_qk, dk]; k: [B, T, H_qk, nh, dk]; v: [B, T, H, nh, dv]; g: [B, T, H];
     beta: [B, T, H, nh]; pool: [num_slots, H, dv, dk]; slot_ids: [B].
     Returns (o [B, T, H, dv], new_pool, threads_used), fp64. With copy_pool=False an
     fp64 C-contiguous numpy pool is updated in place (no copy).
@@ -128,14 +132,14 @@ def decode(q, k, v, g, beta, pool, slot_ids, scale=None, nthreads=0, lib=None, c
                          and pool.flags.c_contiguous):
         pool = f64(pool).copy()
     slots = np.ascontiguousarray(np.asarray(f64(slot_ids), dtype=np.int32))
-    B, T, H, dk = q.shape
-    nh, dv = v.shape[3], v.shape[4]
+    B, T, Hqk, dk = q.shape
+    H, nh, dv = v.shape[2], v.shape[3], v.shape[4]
     if scale is None:
         scale = 1.0 / np.sqrt(dk)
     o = np.zeros((B, T, H, dv), np.float64)
     rc = lib.gdn_oracle_decode(_ptr(q), _ptr(k), _ptr(v), _ptr(g), _ptr(beta), _ptr(pool),
                                pool.shape[0], _ptr(slots, ctypes.c_int32), _ptr(o),
-                               B, T, H, dk, dv, nh, float(scale), int(nthreads))
+                               B, T, H, Hqk, dk, dv, nh, float(scale), int(bool(l2norm)), int(nthreads))
     if rc < 0:
         raise ValueError("gdn_oracle_decode: bad arguments")
     return o, pool, rc

@@ -26,6 +26,14 @@
  *   With n_h = 1 this is the gated delta rule above, since
  *   (I - b k k^T)(a S) = a (I - b k k^T) S.
  *
+ * Heads (grouped value attention): q and k may have fewer heads (H_qk) than
+ * v, g, beta, o and the state (H, a multiple of H_qk). Value head h then reads
+ * query/key head h / (H / H_qk): consecutive value heads share one q/k head, the
+ * grouping of repeating each q/k head H / H_qk times in place. H_qk = H is the
+ * plain one-to-one case. With l2norm set, q and k are first scaled to unit
+ * Euclidean length per token (per q/k head and, for k, per Householder), in
+ * fp64; a zero vector stays zero.
+ *
  * Storage: states are kept K-last, i.e. S^T row-major [dv][dk], the layout the
  * FlashInfer PR #7156 page (section 1) indexes as state + row + k_col and the
  * FlashInfer PR #3866 page (section 2, accumulate_state_fragment) contracts over
@@ -68,6 +76,16 @@ static void emit_output(const double* St, const double* q, double scale, double*
     for (int i = 0; i < dk; ++i) acc += col[i] * q[i];
     o[j] = scale * acc;
   }
+}
+
+/* q/k of one token, optionally scaled to unit length (into `buf`) */
+static const double* maybe_unit(const double* x, int n, int l2norm, double* buf) {
+  if (!l2norm) return x;
+  double ss = 0.0;
+  for (int i = 0; i < n; ++i) ss += x[i] * x[i];
+  const double inv = ss > 0.0 ? 1.0 / sqrt(ss) : 0.0;
+  for (int i = 0; i < n; ++i) buf[i] = x[i] * inv;
+  return buf;
 }
 
 /* ---- a tiny work queue over independent (sequence or slot, head) pairs ---- */
@@ -120,7 +138,7 @@ static int run_items(int n_items, int nthreads, void (*fn)(void*, int), void* ct
 typedef struct {
   const double *q, *k, *v, *g, *beta;
   const int64_t* cu;
-  int H, dk, dv;
+  int H, Hqk, dk, dv, l2norm;
   double scale;
   const double* init;
   double* o;
@@ -129,39 +147,46 @@ typedef struct {
 
 static void prefill_item(void* vctx, int item) {
   prefill_ctx* c = (prefill_ctx*)vctx;
-  const int H = c->H, dk = c->dk, dv = c->dv;
+  const int H = c->H, Hqk = c->Hqk, dk = c->dk, dv = c->dv;
   const int n = item / H, h = item % H;
+  const int hq = h / (H / Hqk); /* the value head's query/key head */
   const size_t ssz = (size_t)dk * dv;
   double* St = (double*)malloc(ssz * sizeof(double));
+  double* buf = (double*)malloc(2 * (size_t)dk * sizeof(double));
   if (c->init)
     memcpy(St, c->init + ((size_t)n * H + h) * ssz, ssz * sizeof(double));
   else
     memset(St, 0, ssz * sizeof(double));
   for (int64_t t = c->cu[n]; t < c->cu[n + 1]; ++t) {
-    const size_t th = (size_t)t * H + h;
+    const size_t th = (size_t)t * H + h;   /* v, g, beta, o */
+    const size_t tq = (size_t)t * Hqk + hq; /* q, k */
+    const double* kt = maybe_unit(c->k + tq * dk, dk, c->l2norm, buf);
+    const double* qt = maybe_unit(c->q + tq * dk, dk, c->l2norm, buf + dk);
     apply_gate(St, exp(c->g[th]), dk, dv);
-    apply_householder(St, c->k + th * dk, c->v + th * dv, c->beta[th], dk, dv);
-    emit_output(St, c->q + th * dk, c->scale, c->o + th * dv, dk, dv);
+    apply_householder(St, kt, c->v + th * dv, c->beta[th], dk, dv);
+    emit_output(St, qt, c->scale, c->o + th * dv, dk, dv);
   }
   if (c->fin) memcpy(c->fin + ((size_t)n * H + h) * ssz, St, ssz * sizeof(double));
+  free(buf);
   free(St);
 }
 
 /*
- * q, k: [total_T, H, dk]; v: [total_T, H, dv]; g, beta: [total_T, H];
+ * q, k: [total_T, Hqk, dk]; v: [total_T, H, dv]; g, beta: [total_T, H];
  * cu_seqlens: [N + 1] (cu[0] = 0, non-decreasing); init: [N, H, dv, dk] or NULL
  * (zero state); o: [total_T, H, dv]; final_state: [N, H, dv, dk] or NULL.
+ * H must be a multiple of Hqk; l2norm != 0 normalises q and k per token.
  * Returns the number of threads used, or a negative value on bad arguments.
  */
 int gdn_oracle_prefill(const double* q, const double* k, const double* v, const double* g,
-                       const double* beta, const int64_t* cu_seqlens, int N, int H, int dk,
-                       int dv, double scale, const double* init, double* o, double* final_state,
-                       int nthreads) {
-  if (N < 0 || H <= 0 || dk <= 0 || dv <= 0 || !cu_seqlens) return -1;
+                       const double* beta, const int64_t* cu_seqlens, int N, int H, int Hqk,
+                       int dk, int dv, double scale, int l2norm, const double* init, double* o,
+                       double* final_state, int nthreads) {
+  if (N < 0 || H <= 0 || Hqk <= 0 || H % Hqk != 0 || dk <= 0 || dv <= 0 || !cu_seqlens) return -1;
   if (cu_seqlens[0] != 0) return -1;
   for (int n = 0; n < N; ++n)
     if (cu_seqlens[n + 1] < cu_seqlens[n]) return -1;
-  prefill_ctx c = {q, k, v, g, beta, cu_seqlens, H, dk, dv, scale, init, o, final_state};
+  prefill_ctx c = {q, k, v, g, beta, cu_seqlens, H, Hqk, dk, dv, l2norm, scale, init, o, final_state};
   return run_items(N * H, nthreads, prefill_item, &c);
 }
 
@@ -173,14 +198,15 @@ typedef struct {
   int num_slots;
   const int32_t* slot_ids;
   double* o;
-  int T, H, dk, dv, nh;
+  int T, H, Hqk, dk, dv, nh, l2norm;
   double scale;
 } decode_ctx;
 
 static void decode_item(void* vctx, int item) {
   decode_ctx* c = (decode_ctx*)vctx;
-  const int H = c->H, T = c->T, dk = c->dk, dv = c->dv, nh = c->nh;
+  const int H = c->H, Hqk = c->Hqk, T = c->T, dk = c->dk, dv = c->dv, nh = c->nh;
   const int b = item / H, h = item % H;
+  const int hq = h / (H / Hqk); /* the value head's query/key head */
   const int slot = c->slot_ids[b];
   if (slot < 0 || slot >= c->num_slots) {
     for (int t = 0; t < T; ++t)
@@ -188,29 +214,36 @@ static void decode_item(void* vctx, int item) {
     return;
   }
   double* St = c->pool + ((size_t)slot * H + h) * (size_t)dk * dv;
+  double* buf = (double*)malloc(2 * (size_t)dk * sizeof(double));
   for (int t = 0; t < T; ++t) {
-    const size_t bth = ((size_t)b * T + t) * H + h;
+    const size_t bth = ((size_t)b * T + t) * H + h;   /* v, g, beta, o */
+    const size_t btq = ((size_t)b * T + t) * Hqk + hq; /* q, k */
     apply_gate(St, exp(c->g[bth]), dk, dv);
     for (int m = 0; m < nh; ++m) {
       const size_t km = bth * nh + m;
-      apply_householder(St, c->k + km * dk, c->v + km * dv, c->beta[km], dk, dv);
+      const double* kt = maybe_unit(c->k + (btq * nh + m) * dk, dk, c->l2norm, buf);
+      apply_householder(St, kt, c->v + km * dv, c->beta[km], dk, dv);
     }
-    emit_output(St, c->q + bth * dk, c->scale, c->o + bth * dv, dk, dv);
+    emit_output(St, maybe_unit(c->q + btq * dk, dk, c->l2norm, buf + dk), c->scale, c->o + bth * dv, dk, dv);
   }
+  free(buf);
 }
 
 /*
- * q: [B, T, H, dk]; k: [B, T, H, nh, dk]; v: [B, T, H, nh, dv]; g: [B, T, H];
+ * q: [B, T, Hqk, dk]; k: [B, T, Hqk, nh, dk]; v: [B, T, H, nh, dv]; g: [B, T, H];
  * beta: [B, T, H, nh]; pool: [num_slots, H, dv, dk], updated in place for the
  * slots named by slot_ids[B] (a negative or out-of-range id leaves the pool
- * untouched and writes zeros to that row of o); o: [B, T, H, dv].
+ * untouched and writes zeros to that row of o); o: [B, T, H, dv]. H must be a
+ * multiple of Hqk; l2norm != 0 normalises q and every k per token.
  * Returns the number of threads used, or a negative value on bad arguments.
  */
 int gdn_oracle_decode(const double* q, const double* k, const double* v, const double* g,
                       const double* beta, double* pool, int num_slots, const int32_t* slot_ids,
-                      double* o, int B, int T, int H, int dk, int dv, int nh, double scale,
-                      int nthreads) {
-  if (B < 0 || T <= 0 || H <= 0 || dk <= 0 || dv <= 0 || nh <= 0 || num_slots < 0) return -1;
-  decode_ctx c = {q, k, v, g, beta, pool, num_slots, slot_ids, o, T, H, dk, dv, nh, scale};
+                      double* o, int B, int T, int H, int Hqk, int dk, int dv, int nh, double scale,
+                      int l2norm, int nthreads) {
+  if (B < 0 || T <= 0 || H <= 0 || Hqk <= 0 || H % Hqk != 0 || dk <= 0 || dv <= 0 || nh <= 0 ||
+      num_slots < 0)
+    return -1;
+  decode_ctx c = {q, k, v, g, beta, pool, num_slots, slot_ids, o, T, H, Hqk, dk, dv, nh, l2norm, scale};
   return run_items(B * H, nthreads, decode_item, &c);
 }

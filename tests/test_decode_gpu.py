@@ -155,3 +155,28 @@ def test_decode_T_steps_equal_sequential_prefill_on_gpu():
                           scale=pin.scale, algo=gdn.GDN_PREFILL_SEQUENTIAL)
     assert_close(torch.stack(outs), o_p, tol=1e-5, what="decode vs prefill o")
     assert_close(pool[1], fin[0], tol=1e-5, what="decode vs prefill state")
+
+
+@pytest.mark.parametrize("B", [1, 4, 16])
+def test_split_v_small_batch_bitwise_equals_whole_heads(B):
+    """With few heads the T=1 step splits each head's state rows over several items
+    (the split along V). Each row gets the same arithmetic in the same order, so the
+    first B batch rows of a B=64 x H=32 step (whole heads per item) must come out
+    bitwise identical when they are run alone (split heads)."""
+    inp = inputs.decode_b64_h32(seed=13)
+    o_full, p_full = _run(inp, out_dtype=torch.float32)
+    sub = inputs.DecodeInputs(inp.q[:B], inp.k[:B], inp.v[:B], inp.g[:B], inp.beta[:B], inp.pool,
+                              inp.slot_ids[:B], inp.scale)
+    o, p = _run(sub, out_dtype=torch.float32)
+    used = sub.slot_ids.long().to(DEV)
+    assert torch.equal(o, o_full[:B])
+    assert torch.equal(p[used], p_full[used])
+    _check_against_oracle(sub, o, p, f"split-V B={B}")
+
+
+def test_split_v_b1_h4_against_oracle():
+    """B=1, H=4: four heads, each split into parts of 16 state rows."""
+    for out_dtype in (torch.float32, torch.bfloat16):
+        inp = inputs.decode_inputs(1, 1, 4, 128, 128, 1, 3, seed=14)
+        o, pool = _run(inp, out_dtype=out_dtype)
+        _check_against_oracle(inp, o, pool, f"split-V B=1 H=4 ({out_dtype})")

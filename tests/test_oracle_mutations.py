@@ -15,8 +15,8 @@ from tests.test_oracle_pins import PIN_CHECKS
 SRC = os.path.join(os.path.dirname(oracle.__file__), "gdn_oracle.c")
 
 PREFILL_GATE = "    apply_gate(St, exp(c->g[th]), dk, dv);\n"
-PREFILL_HH = "    apply_householder(St, c->k + th * dk, c->v + th * dv, c->beta[th], dk, dv);\n"
-PREFILL_OUT = "    emit_output(St, c->q + th * dk, c->scale, c->o + th * dv, dk, dv);\n"
+PREFILL_HH = "    apply_householder(St, kt, c->v + th * dv, c->beta[th], dk, dv);\n"
+PREFILL_OUT = "    emit_output(St, qt, c->scale, c->o + th * dv, dk, dv);\n"
 
 MUTANTS = {
     # the gate scales the token's own write (gate after the update)
@@ -46,8 +46,21 @@ MUTANTS = {
     # gated delta product: Householder updates applied in reverse order
     "gdp_reverse_order": [("      const size_t km = bth * nh + m;", "      const size_t km = bth * nh + (nh - 1 - m);")],
     # the projection uses the previous token's key
-    "stale_key": [("apply_householder(St, c->k + th * dk,",
-                   "apply_householder(St, c->k + (t > c->cu[n] ? th - H : th) * dk,")],
+    "stale_key": [("const double* kt = maybe_unit(c->k + tq * dk,",
+                   "const double* kt = maybe_unit(c->k + (t > c->cu[n] ? tq - Hqk : tq) * dk,")],
+    # grouped heads: value head h reads q/k head h % H_qk instead of h / (H / H_qk)
+    "grouped_heads_modulo": [("  const int hq = h / (H / Hqk); /* the value head's query/key head */\n"
+                              "  const size_t ssz",
+                              "  const int hq = h % Hqk;\n  const size_t ssz"),
+                             ("  const int hq = h / (H / Hqk); /* the value head's query/key head */\n"
+                              "  const int slot",
+                              "  const int hq = h % Hqk;\n  const int slot")],
+    # the q/k normalisation applied to the query only
+    "l2norm_query_only": [("const double* kt = maybe_unit(c->k + tq * dk, dk, c->l2norm, buf);",
+                           "const double* kt = c->k + tq * dk;")],
+    # the normalisation divides by the squared norm
+    "l2norm_squared": [("const double inv = ss > 0.0 ? 1.0 / sqrt(ss) : 0.0;",
+                        "const double inv = ss > 0.0 ? 1.0 / ss : 0.0;")],
 }
 
 

@@ -457,4 +457,90 @@ def test_oracle_rejects_bad_cu_seqlens():
         oracle.prefill(q, q, q, np.zeros((4, 1)), np.zeros((4, 1)), [1, 4])
 
 
+# ---------------------------------------------------------------- grouped heads, q/k normalisation
+
+def check_grouped_heads_equal_repeated_qk_heads(lib=None):
+    """H value heads over H_qk q/k heads (value head h reads q/k head h // (H // H_qk))
+    give exactly the results of the one-to-one call whose q/k heads are repeated in
+    place H // H_qk times; prefill and (multi-Householder) decode."""
+    rng = _rng(31)
+    T, Hqk, r, dk, dv = 9, 2, 3, 4, 3
+    H = Hqk * r
+    q = _unit(rng.standard_normal((T, Hqk, dk)))
+    k = _unit(rng.standard_normal((T, Hqk, dk)))
+    v = rng.standard_normal((T, H, dv))
+    beta = 1 / (1 + np.exp(-rng.standard_normal((T, H))))
+    g = -rng.uniform(0.0, 0.3, (T, H))
+    init = 0.1 * rng.standard_normal((2, H, dv, dk))
+    cu = [0, 4, T]
+    o, fin, _ = _prefill(lib)(q, k, v, g, beta, cu, init, scale=0.7)
+    o1, fin1, _ = _prefill(lib)(np.repeat(q, r, axis=1), np.repeat(k, r, axis=1), v, g, beta, cu, init, scale=0.7)
+    assert np.array_equal(o, o1) and np.array_equal(fin, fin1)
+    B, TT, nh, slots = 2, 2, 2, 3
+    qd = _unit(rng.standard_normal((B, TT, Hqk, dk)))
+    kd = _unit(rng.standard_normal((B, TT, Hqk, nh, dk)))
+    vd = rng.standard_normal((B, TT, H, nh, dv))
+    bd = 1 / (1 + np.exp(-rng.standard_normal((B, TT, H, nh))))
+    gd = -rng.uniform(0.0, 0.3, (B, TT, H))
+    pool = 0.1 * rng.standard_normal((slots, H, dv, dk))
+    sid = np.array([2, 0], np.int32)
+    od, pd, _ = _decode(lib)(qd, kd, vd, gd, bd, pool, sid, scale=0.7)
+    od1, pd1, _ = _decode(lib)(np.repeat(qd, r, axis=2), np.repeat(kd, r, axis=2), vd, gd, bd, pool, sid, scale=0.7)
+    assert np.array_equal(od, od1) and np.array_equal(pd, pd1)
+
+
+def check_l2norm_is_scale_invariant(lib=None):
+    """With the q/k normalisation on, positive per-token scalings of q and k change
+    nothing (up to rounding), and the result equals the plain recurrence on q and k
+    normalised beforehand; prefill and decode."""
+    rng = _rng(32)
+    T, H, dk, dv = 7, 2, 5, 3
+    q = rng.standard_normal((T, H, dk))
+    k = rng.standard_normal((T, H, dk))
+    v = rng.standard_normal((T, H, dv))
+    beta = 1 / (1 + np.exp(-rng.standard_normal((T, H))))
+    g = -rng.uniform(0.0, 0.3, (T, H))
+    init = 0.1 * rng.standard_normal((1, H, dv, dk))
+    sq = rng.uniform(0.1, 10.0, (T, H, 1))
+    sk = rng.uniform(0.1, 10.0, (T, H, 1))
+    o, fin, _ = _prefill(lib)(q, k, v, g, beta, [0, T], init, scale=0.5, l2norm=True)
+    o2, fin2, _ = _prefill(lib)(q * sq, k * sk, v, g, beta, [0, T], init, scale=0.5, l2norm=True)
+    o3, fin3, _ = _prefill(lib)(_unit(q), _unit(k), v, g, beta, [0, T], init, scale=0.5)
+    for x, y in ((o, o2), (fin, fin2), (o, o3), (fin, fin3)):
+        assert _relerr(x, y) < 1e-13
+    # the normalisation matters: un-normalised keys give a different state
+    o4, _, _ = _prefill(lib)(q * sq, k * sk, v, g, beta, [0, T], init, scale=0.5)
+    assert _relerr(o4, o) > 1e-3
+    B, TT, nh = 2, 2, 2
+    qd = rng.standard_normal((B, TT, H, dk))
+    kd = rng.standard_normal((B, TT, H, nh, dk))
+    vd = rng.standard_normal((B, TT, H, nh, dv))
+    bd = 1 / (1 + np.exp(-rng.standard_normal((B, TT, H, nh))))
+    gd = -rng.uniform(0.0, 0.3, (B, TT, H))
+    pool = 0.1 * rng.standard_normal((2, H, dv, dk))
+    sid = np.array([1, 0], np.int32)
+    od, pd, _ = _decode(lib)(qd, kd, vd, gd, bd, pool, sid, scale=0.5, l2norm=True)
+    od2, pd2, _ = _decode(lib)(qd * 3.0, kd * rng.uniform(0.1, 10.0, (B, TT, H, nh, 1)), vd, gd, bd, pool, sid,
+                               scale=0.5, l2norm=True)
+    od3, pd3, _ = _decode(lib)(_unit(qd), _unit(kd), vd, gd, bd, pool, sid, scale=0.5)
+    for x, y in ((od, od2), (pd, pd2), (od, od3), (pd, pd3)):
+        assert _relerr(x, y) < 1e-13
+
+
+def test_grouped_heads_equal_repeated_qk_heads():
+    check_grouped_heads_equal_repeated_qk_heads()
+
+
+def test_l2norm_is_scale_invariant():
+    check_l2norm_is_scale_invariant()
+
+
+def test_oracle_rejects_head_counts_that_do_not_divide():
+    rng = _rng(33)
+    q = rng.standard_normal((3, 2, 4))
+    v = rng.standard_normal((3, 3, 4))
+    with pytest.raises(ValueError):
+        oracle.prefill(q, q, v, np.zeros((3, 3)), np.ones((3, 3)), [0, 3])
+
+
 PIN_CHECKS.extend(v for k, v in sorted(globals().items()) if k.startswith("check_"))
