@@ -36,9 +36,10 @@
 //   state   (warps 0-3):  W^T -> fp16 tile, U^T -> fp16 tiles, the new state ->
 //            fp16 TMEM operand (and the gamma_C rescale of the fp32 TMEM state),
 //            outputs -> HBM.
-//   mma     (warp 12):    one thread issues every tcgen05.mma in dependency order;
-//            the next chunk's [K;Q]K^T goes first, as soon as its tiles are in and
-//            the prep warps have read this chunk's.
+//   mma     (warp 12):    one thread issues the chunk's tcgen05.mma products in
+//            dependency order. [K;Q]K^T is issued by the loader's first thread
+//            instead, as soon as its tiles are in and the prep warps have read the
+//            previous chunk's, so the chain's MMAs never wait on future tiles.
 // Hand-offs are mbarriers: tcgen05.commit for MMA completion, one elected arrive
 // per warpgroup (after a named barrier) for thread-produced tiles. Every wait is
 // bounded; a timeout sets GDN_DEVERR_TIMEOUT and unwinds all roles.
@@ -180,6 +181,24 @@ struct QkvMaps {
   CUtensorMap o;        // o [total_T][H][128] as {128, H, total_T}; box {128, 1, 64}, not swizzled
 };
 
+// TMA loads of the raw bf16 K, Q (and V) tiles of the chunk starting at token t0
+// into tile buffer b, completing on B_T0 + b. Issued by one thread, once the
+// buffer's previous chunk (two chunks back) has had its last MMA complete.
+__device__ __forceinline__ void issue_tile_loads(const Smem& sm, const QkvMaps& maps, int b, int h, int64_t t0,
+                                                 bool zero_values) {
+  uint8_t* kq = sm.base + OFF_KQ + b * KQ_BUF;
+  uint8_t* v16 = sm.base + OFF_V + b * V_BUF;
+  tc::fence_proxy_async_smem();  // the previous generic writes of these tiles precede the copies
+  tc::mbar_arrive_expect_tx(sm.bar(B_T0 + b), (zero_values ? 2u : 3u) * 16384u);
+#pragma unroll
+  for (int hf = 0; hf < 2; ++hf) {
+    tc::tma_load_3d(tc::smem_u32(kq + hf * KQ_HALF), &maps.k, 64 * hf, h, (int)t0, sm.bar(B_T0 + b));
+    tc::tma_load_3d(tc::smem_u32(kq + hf * KQ_HALF + C * 128), &maps.q, 64 * hf, h, (int)t0, sm.bar(B_T0 + b));
+    if (!zero_values)
+      tc::tma_load_3d(tc::smem_u32(v16 + hf * V_HALF), &maps.v, 64 * hf, h, (int)t0, sm.bar(B_T0 + b));
+  }
+}
+
 // bf16 -> fp16 of one 16-byte chunk (8 elements) in place.
 __device__ __forceinline__ void convert_chunk_bf16(uint8_t* p) {
   uint4* q = reinterpret_cast<uint4*>(p);
@@ -195,9 +214,31 @@ __device__ __forceinline__ void convert_chunk_bf16(uint8_t* p) {
   *q = u;
 }
 
+// D1 = [K;Q] K^T for chunk buffer b (raw bf16 tiles, or fp16 ones for fp32 inputs).
+__device__ __forceinline__ void issue_m1(const Smem& sm, uint32_t tmem, int b, int raw_bf16) {
+  const uint32_t kq = sm.u32(OFF_KQ + b * KQ_BUF);
+  const uint32_t id = tc::idesc_f16(128, 64, 0, 0, 0, raw_bf16);
+#pragma unroll
+  for (int ks = 0; ks < 8; ++ks) {
+    const uint32_t off = (ks >> 2) * KQ_HALF + (ks & 3) * 32;
+    tc::mma_f16(tmem + COL_D1, tc::sw128_desc(kq + off, 16, 1024), tc::sw128_desc(kq + off, 16, 1024), id, ks > 0);
+  }
+  tc::mma_commit(sm.bar(B_M1));
+}
+
+// Chunk c's [K;Q]K^T, issued by the loader's first thread as soon as the tiles
+// are in (L0 signalled) and the prep group has read chunk c-1's D1 from TMEM, so
+// the MMA role never waits on future tiles before this chunk's products.
+__device__ __forceinline__ bool issue_d1(const Smem& sm, uint32_t tmem, int c, int b, int raw_bf16, unsigned int* err) {
+  if (c >= 1 && !wait_bar(sm, B_E1, (c - 1) & 1, err)) return false;
+  tc::fence_after_sync();
+  issue_m1(sm, tmem, b, raw_bf16);
+  return true;
+}
+
 template <typename TIn>
 __device__ void loader_role(const Smem& sm, const PrefillShape& s, const PrefillArgs& a, const QkvMaps& maps,
-                            int h, int64_t bos, int64_t eos, int nchunks) {
+                            uint32_t tmem, int h, int64_t bos, int64_t eos, int nchunks) {
   constexpr bool kTma = std::is_same<TIn, __nv_bfloat16>::value;
   const int t = threadIdx.x - kLoadWarp0 * 32;  // 0..127
   const bool zero_values = (a.mode == kPrefillTransfer);  // transfer run: V taken as 0
@@ -207,36 +248,32 @@ __device__ void loader_role(const Smem& sm, const PrefillShape& s, const Prefill
   }
   for (int c = 0; c < nchunks; ++c) {
     const int b = c & 1;
-    // chunk c-2 (same tile buffers) no longer reads K, Q or V: its state update,
-    // the last MMA to read them, has completed (so have the earlier ones)
-    if (c >= 2 && !wait_bar(sm, B_M4B, (c - 2) & 1, a.err)) return;
     const int64_t t0 = bos + (int64_t)c * C;
     const int Lc = (int)((eos - t0) < C ? (eos - t0) : C);
     float* vec = sm.vec(c % 3);  // three gate buffers: chunk c-2's output epilogue may still read its own
     uint8_t* kq = sm.base + OFF_KQ + b * KQ_BUF;
     uint8_t* v16 = sm.base + OFF_V + b * V_BUF;
+    // g and beta (zero past the sequence end), into registers first
+    float gv = 0.f, bv = 0.f;
+    if (t < Lc) {
+      const size_t th = (size_t)(t0 + t) * s.H + h;
+      gv = __ldg(a.g + th);
+      bv = __ldg(a.beta + th);
+    }
+    // Chunk c-2 (same tile and gate buffers) must be done with K, Q, V: its state
+    // update, the last MMA to read them, has completed (so have the earlier ones).
+    // With TMA loads the state warps issue chunk c's copies as soon as that update
+    // completes (chunks 0 and 1 are issued here), so the landing of the copies
+    // implies it; the fp32 path waits for it directly.
     if constexpr (kTma) {
       // rows past the sequence end load the next tokens (or zeros past the tensor);
       // they are zeroed once the copies have landed, and their beta and g are 0
-      if (t == 0) {
-        tc::fence_proxy_async_smem();  // the previous generic writes of these tiles precede the copies
-        tc::mbar_arrive_expect_tx(sm.bar(B_T0 + b), (zero_values ? 2u : 3u) * 16384u);
-#pragma unroll
-        for (int hf = 0; hf < 2; ++hf) {
-          tc::tma_load_3d(tc::smem_u32(kq + hf * KQ_HALF), &maps.k, 64 * hf, h, (int)t0, sm.bar(B_T0 + b));
-          tc::tma_load_3d(tc::smem_u32(kq + hf * KQ_HALF + C * 128), &maps.q, 64 * hf, h, (int)t0, sm.bar(B_T0 + b));
-          if (!zero_values)
-            tc::tma_load_3d(tc::smem_u32(v16 + hf * V_HALF), &maps.v, 64 * hf, h, (int)t0, sm.bar(B_T0 + b));
-        }
-      }
+      if (c < 2 && t == 0) issue_tile_loads(sm, maps, b, h, t0, zero_values);
+      if (!wait_bar(sm, B_T0 + b, (c >> 1) & 1, a.err)) return;
+    } else {
+      if (c >= 2 && !wait_bar(sm, B_M4B, (c - 2) & 1, a.err)) return;
     }
-    if (t < C) {  // g and beta (zero past the sequence end)
-      float gv = 0.f, bv = 0.f;
-      if (t < Lc) {
-        const size_t th = (size_t)(t0 + t) * s.H + h;
-        gv = __ldg(a.g + th);
-        bv = __ldg(a.beta + th);
-      }
+    if (t < C) {
       vec[V_G + t] = gv;
       vec[V_BETA + t] = bv;
     }
@@ -266,7 +303,6 @@ __device__ void loader_role(const Smem& sm, const PrefillShape& s, const Prefill
     if constexpr (kTma) {
       // the raw bf16 tiles feed [K;Q] K^T directly (bf16 MMA, exact inputs); they
       // are converted to fp16 in place once that MMA has read them
-      if (!wait_bar(sm, B_T0 + b, (c >> 1) & 1, a.err)) return;
       if (Lc < C) {
         // Rows past the sequence end hold the next sequence's tokens (or zeros past
         // the tensor). They are zeroed before any product reads them: beta = g = 0
@@ -285,6 +321,7 @@ __device__ void loader_role(const Smem& sm, const PrefillShape& s, const Prefill
         }
       }
       group_signal(sm, kBarLoad, B_L0 + b);
+      if (t == 0 && !issue_d1(sm, tmem, c, b, 1, a.err)) return;
       if (!wait_bar(sm, B_M1, c & 1, a.err)) return;
       tc::fence_after_sync();
 #pragma unroll 4
@@ -318,6 +355,7 @@ __device__ void loader_role(const Smem& sm, const PrefillShape& s, const Prefill
         }
       }
       group_signal(sm, kBarLoad, B_L0 + b);
+      if (t == 0 && !issue_d1(sm, tmem, c, b, 0, a.err)) return;
     }
     group_signal(sm, kBarLoad, B_LC0 + b);
   }
@@ -584,9 +622,10 @@ __device__ void prep_role(const Smem& sm, uint32_t tmem, int nchunks, unsigned i
 
 // ---------------------------------------------------------------- state role
 
-template <typename TOut>
+template <typename TIn, typename TOut>
 __device__ void state_role(const Smem& sm, const PrefillShape& s, const PrefillArgs& a, const QkvMaps& maps,
                            uint32_t tmem, int h, int64_t bos, int64_t eos, int nchunks, size_t state_off) {
+  constexpr bool kTmaLoads = std::is_same<TIn, __nv_bfloat16>::value;
   const int j = threadIdx.x;  // TMEM lane == dv row of S^T
   const int warp = threadIdx.x >> 5;
   const uint32_t tl = tmem + ((uint32_t)((warp & 3) * 32) << 16);
@@ -673,6 +712,9 @@ __device__ void state_role(const Smem& sm, const PrefillShape& s, const PrefillA
     // E6a: new state -> fp16 operand; rescale by the next chunk's gamma_C; final state
     if (!wait_bar(sm, B_M4B, c & 1, a.err)) return;
     tc::fence_after_sync();
+    // chunk c's state update was the last reader of tile buffer b: chunk c+2's
+    // copies go out now, well before the loader needs them
+    if (kTmaLoads && j == 0 && c + 2 < nchunks) issue_tile_loads(sm, maps, b, h, t0 + 2 * C, a.mode == kPrefillTransfer);
     const bool last = (c == nchunks - 1);
     float gnext = 1.f;
     if (!last) {
@@ -754,18 +796,6 @@ __device__ void state_role(const Smem& sm, const PrefillShape& s, const PrefillA
 
 // ---------------------------------------------------------------- mma role
 
-// D1 = [K;Q] K^T for chunk buffer b (raw bf16 tiles, or fp16 ones for fp32 inputs).
-__device__ __forceinline__ void issue_m1(const Smem& sm, uint32_t tmem, int b, int raw_bf16) {
-  const uint32_t kq = sm.u32(OFF_KQ + b * KQ_BUF);
-  const uint32_t id = tc::idesc_f16(128, 64, 0, 0, 0, raw_bf16);
-#pragma unroll
-  for (int ks = 0; ks < 8; ++ks) {
-    const uint32_t off = (ks >> 2) * KQ_HALF + (ks & 3) * 32;
-    tc::mma_f16(tmem + COL_D1, tc::sw128_desc(kq + off, 16, 1024), tc::sw128_desc(kq + off, 16, 1024), id, ks > 0);
-  }
-  tc::mma_commit(sm.bar(B_M1));
-}
-
 // W^T = K^T T'^T and U~^T = V^T T''^T for chunk buffer b (A MN-major from the token tiles).
 __device__ __forceinline__ void issue_m2(const Smem& sm, uint32_t tmem, int b) {
   const uint32_t kq = sm.u32(OFF_KQ + b * KQ_BUF), v16 = sm.u32(OFF_V + b * V_BUF);
@@ -782,26 +812,16 @@ __device__ __forceinline__ void issue_m2(const Smem& sm, uint32_t tmem, int b) {
   tc::mma_commit(sm.bar(B_M2));
 }
 
-__device__ void mma_role(const Smem& sm, uint32_t tmem, int nchunks, int raw_bf16, unsigned int* err) {
+__device__ void mma_role(const Smem& sm, uint32_t tmem, int nchunks, unsigned int* err) {
   const uint32_t w16 = sm.u32(OFF_W16), u16 = sm.u32(OFF_U16), udd = sm.u32(OFF_UDD);
   const uint32_t p16 = sm.u32(OFF_P16);
   const uint32_t id_u = tc::idesc_f16(128, 64, 0, 1, 1);
   const uint32_t id_o = tc::idesc_f16(128, 64, 0, 0);
   const uint32_t id_s = tc::idesc_f16(128, 128, 0, 1);
 
-  if (!wait_bar(sm, B_L0, 0, err)) return;
-  tc::fence_after_sync();
-  issue_m1(sm, tmem, 0, raw_bf16);
   for (int c = 0; c < nchunks; ++c) {
     const int b = c & 1;
     const uint32_t kq = sm.u32(OFF_KQ + b * KQ_BUF);
-    // M1 of the next chunk as soon as its tiles are in and this chunk's D1 was read
-    if (c + 1 < nchunks) {
-      if (!wait_bar(sm, B_L0 + (b ^ 1), ((c + 1) >> 1) & 1, err)) return;
-      if (!wait_bar(sm, B_E1, c & 1, err)) return;
-      tc::fence_after_sync();
-      issue_m1(sm, tmem, b ^ 1, raw_bf16);
-    }
     // M2: W^T, U~^T of this chunk
     if (!wait_bar(sm, B_E2, c & 1, err)) return;
     if (!wait_bar(sm, B_LC0 + b, (c >> 1) & 1, err)) return;
@@ -917,13 +937,13 @@ gdn_prefill_fused_kernel(const PrefillShape s, const PrefillArgs a, const __grid
   const uint32_t tmem = *sm.tmem_slot();
 
   if (warp < kPrepWarp0) {
-    state_role<TOut>(sm, s, a, maps, tmem, h, bos, eos, nchunks, state_off);
+    state_role<TIn, TOut>(sm, s, a, maps, tmem, h, bos, eos, nchunks, state_off);
   } else if (warp < kLoadWarp0) {
     prep_role(sm, tmem, nchunks, a.err);
   } else if (warp < kMmaWarp) {
-    loader_role<TIn>(sm, s, a, maps, h, bos, eos, nchunks);
+    loader_role<TIn>(sm, s, a, maps, tmem, h, bos, eos, nchunks);
   } else if ((threadIdx.x & 31) == 0) {
-    mma_role(sm, tmem, nchunks, std::is_same<TIn, __nv_bfloat16>::value ? 1 : 0, a.err);
+    mma_role(sm, tmem, nchunks, a.err);
   }
 
   // teardown: every role finished (all MMAs were waited on by the state role)
