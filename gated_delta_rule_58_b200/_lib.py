@@ -31,6 +31,8 @@ GDN_PREFILL_FUSED = 1
 GDN_PREFILL_TRANSFER = 2
 GDN_PREFILL_SEQUENTIAL = 3
 
+GDN_QK_L2NORM = 0x1
+
 GDN_DEVERR_SLOT_OUT_OF_RANGE = 0x1
 GDN_DEVERR_BAD_CU_SEQLENS = 0x2
 GDN_DEVERR_TIMEOUT = 0x4
@@ -65,16 +67,17 @@ def lib() -> ctypes.CDLL:
             vp, i32, i64, f32, sz = (ctypes.c_void_p, ctypes.c_int, ctypes.c_int64, ctypes.c_float,
                                      ctypes.c_size_t)
             L.gdn_decode.restype = i32
-            L.gdn_decode.argtypes = [vp, vp, vp, vp, vp, vp, i32, vp, vp, i32, i32, i32, i32, i32, i32,
-                                     f32, i32, i32, vp]
+            u32 = ctypes.c_uint32
+            L.gdn_decode.argtypes = [vp, vp, vp, vp, vp, vp, i32, vp, vp, i32, i32, i32, i32, i32, i32, i32,
+                                     f32, u32, i32, i32, vp]
             L.gdn_chunk_prefill_workspace_size.restype = sz
             L.gdn_chunk_prefill_workspace_size.argtypes = [i32, i64, i32, i32, i32, i32, i32]
             L.gdn_chunk_prefill.restype = i32
-            L.gdn_chunk_prefill.argtypes = [vp, vp, vp, vp, vp, vp, i32, i64, vp, vp, vp, i32, i32, i32,
-                                            i32, f32, i32, i32, i32, vp, sz, vp]
+            L.gdn_chunk_prefill.argtypes = [vp, vp, vp, vp, vp, vp, i32, i64, vp, vp, vp, i32, i32, i32, i32,
+                                            i32, f32, u32, i32, i32, i32, vp, sz, vp]
             L.gdn_chunk_prefill_static_scratch.restype = i32
             L.gdn_chunk_prefill_static_scratch.argtypes = [vp, vp, vp, vp, vp, vp, i32, i64, vp, vp, vp, i32,
-                                                           i32, i32, i32, f32, i32, i32, vp]
+                                                           i32, i32, i32, i32, f32, u32, i32, i32, vp]
             L.gdn_last_error.restype = ctypes.c_char_p
             L.gdn_last_error.argtypes = []
             L.gdn_get_device_error.restype = i32
@@ -133,17 +136,19 @@ def _stream_ptr(stream, device):
     return stream.cuda_stream if hasattr(stream, "cuda_stream") else int(stream)
 
 
-def gdn_decode(q, k, v, g, beta, state_pool, slot_ids, o, scale=None, stream=None):
+def gdn_decode(q, k, v, g, beta, state_pool, slot_ids, o, scale=None, stream=None, l2norm=False):
     """One decode step (see include/gdn.h). Shapes:
-    q [B,T,H,dk], k [B,T,H,n_h,dk], v [B,T,H,n_h,dv], g [B,T,H], beta [B,T,H,n_h],
-    state_pool [num_slots,H,dv,dk] fp32 (updated in place), slot_ids [B] int32, o [B,T,H,dv]."""
-    B, T, H, dk = q.shape
-    n_h, dv = k.shape[3], v.shape[4]
+    q [B,T,H_qk,dk], k [B,T,H_qk,n_h,dk], v [B,T,H,n_h,dv], g [B,T,H], beta [B,T,H,n_h],
+    state_pool [num_slots,H,dv,dk] fp32 (updated in place), slot_ids [B] int32, o [B,T,H,dv].
+    l2norm: normalise q and k per token inside the kernel (GDN_QK_L2NORM)."""
+    B, T, H_qk, dk = q.shape
+    H, n_h, dv = v.shape[2], k.shape[3], v.shape[4]
     if scale is None:
         scale = dk ** -0.5
     st = lib().gdn_decode(_ptr(q), _ptr(k), _ptr(v), _ptr(g), _ptr(beta), _ptr(state_pool),
-                          state_pool.shape[0], _ptr(slot_ids), _ptr(o), B, T, H, dk, dv, n_h,
-                          float(scale), _dtype_code(q), _dtype_code(o), _stream_ptr(stream, q.device))
+                          state_pool.shape[0], _ptr(slot_ids), _ptr(o), B, T, H, H_qk, dk, dv, n_h,
+                          float(scale), GDN_QK_L2NORM if l2norm else 0, _dtype_code(q), _dtype_code(o),
+                          _stream_ptr(stream, q.device))
     _check(st)
     return o
 
@@ -156,16 +161,16 @@ def gdn_chunk_prefill_workspace_size(N, total_T, H, dk, dv, chunk, algo=GDN_PREF
 
 
 def gdn_chunk_prefill(q, k, v, g, beta, cu_seqlens, o, initial_state=None, final_state=None,
-                      chunk=64, scale=None, algo=GDN_PREFILL_AUTO, workspace=None, stream=None):
-    """Chunked varlen prefill (see include/gdn.h). Shapes: q,k [total_T,H,dk], v [total_T,H,dv],
+                      chunk=64, scale=None, algo=GDN_PREFILL_AUTO, workspace=None, stream=None, l2norm=False):
+    """Chunked varlen prefill (see include/gdn.h). Shapes: q,k [total_T,H_qk,dk], v [total_T,H,dv],
     g,beta [total_T,H] fp32, cu_seqlens [N+1] int32 (device), initial/final_state [N,H,dv,dk] fp32,
     o [total_T,H,dv]. `workspace` is a uint8 CUDA tensor; when None one of the required size is
     allocated through torch for this call, on `stream` when one is given, so torch orders any
     reuse of that memory after the call's kernels; a raw stream handle needs an explicit
-    `workspace`."""
+    `workspace`. l2norm: normalise q and k per token inside the kernels."""
     import torch
-    total_T, H, dk = q.shape
-    dv = v.shape[-1]
+    total_T, H_qk, dk = q.shape
+    H, dv = v.shape[1], v.shape[-1]
     N = cu_seqlens.numel() - 1
     if scale is None:
         scale = dk ** -0.5
@@ -181,26 +186,26 @@ def gdn_chunk_prefill(q, k, v, g, beta, cu_seqlens, o, initial_state=None, final
     ws_ptr = _ptr(workspace)
     ws_bytes = workspace.numel() if workspace is not None else 0
     st = lib().gdn_chunk_prefill(_ptr(q), _ptr(k), _ptr(v), _ptr(g), _ptr(beta), _ptr(cu_seqlens), N,
-                                 total_T, _ptr(initial_state), _ptr(final_state), _ptr(o), H, dk, dv,
-                                 chunk, float(scale), _dtype_code(q), _dtype_code(o), algo, ws_ptr,
-                                 ws_bytes, _stream_ptr(stream, q.device))
+                                 total_T, _ptr(initial_state), _ptr(final_state), _ptr(o), H, H_qk, dk, dv,
+                                 chunk, float(scale), GDN_QK_L2NORM if l2norm else 0, _dtype_code(q),
+                                 _dtype_code(o), algo, ws_ptr, ws_bytes, _stream_ptr(stream, q.device))
     _check(st)
     return o
 
 
 def gdn_chunk_prefill_static_scratch(q, k, v, g, beta, cu_seqlens, o, initial_state=None, final_state=None,
-                                     chunk=64, scale=None, stream=None):
+                                     chunk=64, scale=None, stream=None, l2norm=False):
     """Transfer prefill whose scratch is the library's own 32 MiB device array, for
     callers that cannot allocate device memory at call time (see include/gdn.h).
     Same shapes as gdn_chunk_prefill; nothing is allocated, here or in the library."""
-    total_T, H, dk = q.shape
-    dv = v.shape[-1]
+    total_T, H_qk, dk = q.shape
+    H, dv = v.shape[1], v.shape[-1]
     N = cu_seqlens.numel() - 1
     if scale is None:
         scale = dk ** -0.5
     st = lib().gdn_chunk_prefill_static_scratch(
         _ptr(q), _ptr(k), _ptr(v), _ptr(g), _ptr(beta), _ptr(cu_seqlens), N, total_T, _ptr(initial_state),
-        _ptr(final_state), _ptr(o), H, dk, dv, chunk, float(scale), _dtype_code(q), _dtype_code(o),
-        _stream_ptr(stream, q.device))
+        _ptr(final_state), _ptr(o), H, H_qk, dk, dv, chunk, float(scale), GDN_QK_L2NORM if l2norm else 0,
+        _dtype_code(q), _dtype_code(o), _stream_ptr(stream, q.device))
     _check(st)
     return o

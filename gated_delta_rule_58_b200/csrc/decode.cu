@@ -60,6 +60,8 @@ struct DecodeParams {
   int B, H, num_slots;
   int n_items;
   float scale;
+  int Hqk;         // query/key heads; value head h reads q/k head h / (H / Hqk)
+  uint32_t flags;  // GDN_QK_L2NORM
 };
 
 // Stage layout for one item (all offsets 16-byte aligned):
@@ -198,11 +200,13 @@ __device__ __forceinline__ void decode_producer(const DecodeParams& p, const CUt
       tc::bulk_load(sst, p.pool + (((size_t)slot * p.H + h) * DK + (size_t)part * L::kRows) * DK, L::kState,
                     &full[s]);
     }
+    const int hq = h / (p.H / p.Hqk);  // the value head's query/key head
 #pragma unroll
     for (int t = 0; t < TT; ++t) {
       const size_t bth = ((size_t)b * TT + t) * p.H + h;
-      tc::bulk_load(sst + L::kKeys + t * NH * L::kRow, kp + bth * NH * DK, NH * L::kRow, &full[s]);
-      tc::bulk_load(sst + L::kQueries + t * L::kRow, qp + bth * DK, L::kRow, &full[s]);
+      const size_t btq = ((size_t)b * TT + t) * p.Hqk + hq;
+      tc::bulk_load(sst + L::kKeys + t * NH * L::kRow, kp + btq * NH * DK, NH * L::kRow, &full[s]);
+      tc::bulk_load(sst + L::kQueries + t * L::kRow, qp + btq * DK, L::kRow, &full[s]);
       tc::bulk_load(sst + L::kValues + t * NH * L::kRow, vp + bth * NH * DK, NH * L::kRow, &full[s]);
     }
   }
@@ -300,9 +304,30 @@ gdn_decode_kernel(const DecodeParams p, const __grid_constant__ CUtensorMap pool
       ks += __shfl_xor_sync(0xffffffffu, ks, 16);
       qs += __shfl_xor_sync(0xffffffffu, qs, 16);
       qkv += __shfl_xor_sync(0xffffffffu, qkv, 16);
+      float rk = 1.f;  // 1 / |k| with the normalisation (the update then adds cm rk k)
+      if (p.flags & GDN_QK_L2NORM) {
+        float kk = 0.f, qq = 0.f;
+#pragma unroll
+        for (int c = 0; c < CPH; ++c) {
+          const int e = half * (DK / TPR) + 4 * c;
+          float wk[4], wq[4];
+          load4_f32<TIn>(st + L::kKeys + e * sizeof(TIn), wk);
+          load4_f32<TIn>(st + L::kQueries + e * sizeof(TIn), wq);
+          kk = fmaf(wk[0], wk[0], fmaf(wk[1], wk[1], fmaf(wk[2], wk[2], fmaf(wk[3], wk[3], kk))));
+          qq = fmaf(wq[0], wq[0], fmaf(wq[1], wq[1], fmaf(wq[2], wq[2], fmaf(wq[3], wq[3], qq))));
+        }
+        kk += __shfl_xor_sync(0xffffffffu, kk, 16);
+        qq += __shfl_xor_sync(0xffffffffu, qq, 16);
+        rk = kk > 0.f ? 1.f / sqrtf(kk) : 0.f;
+        const float rq = qq > 0.f ? 1.f / sqrtf(qq) : 0.f;
+        ks *= rk;
+        qs *= rq;
+        qkv *= rq * rk;
+      }
       const float a = alpha[0];
       const float vj = to_f32(reinterpret_cast<const TIn*>(st + L::kValues)[grow]);
       const float cm = betas[0] * (vj - a * ks);
+      const float cmk = cm * rk;
       if (half == 0) store_out(op + ((size_t)b * p.H + h) * DK + grow, p.scale * fmaf(cm, qkv, a * qs));
 #pragma unroll
       for (int c = 0; c < CPH; ++c) {
@@ -310,10 +335,10 @@ gdn_decode_kernel(const DecodeParams p, const __grid_constant__ CUtensorMap pool
         float wk[4];
         load4_f32<TIn>(st + L::kKeys + e * sizeof(TIn), wk);
         float4 x = sv[c];
-        x.x = fmaf(cm, wk[0], a * x.x);
-        x.y = fmaf(cm, wk[1], a * x.y);
-        x.z = fmaf(cm, wk[2], a * x.z);
-        x.w = fmaf(cm, wk[3], a * x.w);
+        x.x = fmaf(cmk, wk[0], a * x.x);
+        x.y = fmaf(cmk, wk[1], a * x.y);
+        x.z = fmaf(cmk, wk[2], a * x.z);
+        x.w = fmaf(cmk, wk[3], a * x.w);
         reinterpret_cast<float4*>(srow)[(c + grow) & (CPH - 1)] = x;
       }
     } else if (half == 0) {
@@ -418,6 +443,18 @@ gdn_decode_multi_kernel(const DecodeParams p, const __grid_constant__ CUtensorMa
       for (int e = gt * 4; e < NV * DK; e += kGroupThreads * 4)
         load4_f32<TIn>(st + L::kKeys + e * sizeof(TIn), vecf + e);
       tc::named_sync(bar_id, kGroupThreads);
+      if (p.flags & GDN_QK_L2NORM) {  // every key and query to unit length, in place
+        for (int vi = gw; vi < NV; vi += kGroupWarps) {
+          float* x = vecf + vi * DK;
+          float ss = 0.f;
+          for (int e = lane; e < DK; e += 32) ss = fmaf(x[e], x[e], ss);
+#pragma unroll
+          for (int off = 16; off > 0; off >>= 1) ss += __shfl_xor_sync(0xffffffffu, ss, off);
+          const float r = ss > 0.f ? 1.f / sqrtf(ss) : 0.f;
+          for (int e = lane; e < DK; e += 32) x[e] *= r;
+        }
+        tc::named_sync(bar_id, kGroupThreads);
+      }
       // Gram entries: warp w takes pairs w, w + W, ...; a batch of kBatch pairs has
       // its partial sums reduced together (independent shuffles)
       for (int p0 = gw; p0 < kPairs; p0 += kGroupWarps * kBatch) {
@@ -723,10 +760,11 @@ gdn_status_t launch_steps(DecodeParams p, int T, int nh, gdn_dtype_t in, gdn_dty
 
 gdn_status_t decode_launch(const void* q, const void* k, const void* v, const float* g,
                            const float* beta, float* pool, int num_slots, const int32_t* slot_ids,
-                           void* o, int B, int T, int H, int dk, int dv, int nh, float scale,
-                           gdn_dtype_t in, gdn_dtype_t out, unsigned int* err, cudaStream_t stream) {
+                           void* o, int B, int T, int H, int Hqk, int dk, int dv, int nh, float scale,
+                           uint32_t flags, gdn_dtype_t in, gdn_dtype_t out, unsigned int* err,
+                           cudaStream_t stream) {
   (void)dv;
-  DecodeParams p{q, k, v, g, beta, pool, slot_ids, o, err, B, H, num_slots, 0, scale};
+  DecodeParams p{q, k, v, g, beta, pool, slot_ids, o, err, B, H, num_slots, 0, scale, Hqk, flags};
   switch (dk) {
     case 32: return launch_steps<32>(p, T, nh, in, out, stream);
     case 64: return launch_steps<64>(p, T, nh, in, out, stream);

@@ -56,8 +56,9 @@ gdn_status_t device_error_word(unsigned int** word) {
 
 gdn_status_t decode_launch(const void* q, const void* k, const void* v, const float* g,
                            const float* beta, float* pool, int num_slots, const int32_t* slot_ids,
-                           void* o, int B, int T, int H, int dk, int dv, int nh, float scale,
-                           gdn_dtype_t in, gdn_dtype_t out, unsigned int* err, cudaStream_t stream);
+                           void* o, int B, int T, int H, int Hqk, int dk, int dv, int nh, float scale,
+                           uint32_t flags, gdn_dtype_t in, gdn_dtype_t out, unsigned int* err,
+                           cudaStream_t stream);
 
 }  // namespace gdn
 
@@ -105,11 +106,14 @@ gdn_status_t gdn_get_device_error(uint32_t* flags) {
 
 gdn_status_t gdn_decode(const void* q, const void* k, const void* v, const float* g,
                         const float* beta, float* state_pool, int num_slots,
-                        const int32_t* slot_ids, void* o, int B, int T, int H, int dk, int dv,
-                        int n_h, float scale, gdn_dtype_t in_dtype, gdn_dtype_t out_dtype,
-                        void* stream) {
+                        const int32_t* slot_ids, void* o, int B, int T, int H, int H_qk,
+                        int dk, int dv, int n_h, float scale, uint32_t flags,
+                        gdn_dtype_t in_dtype, gdn_dtype_t out_dtype, void* stream) {
   GDN_REQUIRE(B >= 0 && T >= 1 && H >= 1 && n_h >= 1 && num_slots >= 0, GDN_ERR_INVALID_ARG,
               "gdn_decode: need B >= 0, T >= 1, H >= 1, n_h >= 1, num_slots >= 0");
+  GDN_REQUIRE(H_qk >= 1 && H % H_qk == 0, GDN_ERR_INVALID_ARG,
+              "gdn_decode: H_qk must be >= 1 and divide H");
+  GDN_REQUIRE((flags & ~GDN_QK_L2NORM) == 0, GDN_ERR_INVALID_ARG, "gdn_decode: unknown flags");
   GDN_REQUIRE(valid_dtype(in_dtype) && valid_dtype(out_dtype), GDN_ERR_INVALID_ARG,
               "gdn_decode: unknown dtype");
   GDN_REQUIRE(dk == dv, GDN_ERR_UNSUPPORTED, "gdn_decode: dk must equal dv");
@@ -128,30 +132,30 @@ gdn_status_t gdn_decode(const void* q, const void* k, const void* v, const float
   unsigned int* err = nullptr;
   gdn_status_t st = gdn::device_error_word(&err);
   if (st != GDN_OK) return st;
-  return gdn::decode_launch(q, k, v, g, beta, state_pool, num_slots, slot_ids, o, B, T, H, dk, dv,
-                            n_h, scale, in_dtype, out_dtype, err, gdn::as_stream(stream));
+  return gdn::decode_launch(q, k, v, g, beta, state_pool, num_slots, slot_ids, o, B, T, H, H_qk, dk, dv,
+                            n_h, scale, flags, in_dtype, out_dtype, err, gdn::as_stream(stream));
 }
 
 size_t gdn_chunk_prefill_workspace_size(int N, int64_t total_T, int H, int dk, int dv, int chunk,
                                         gdn_prefill_algo_t algo) {
-  gdn::PrefillShape s{N, total_T, H, dk, dv, chunk};
+  gdn::PrefillShape s{N, total_T, H, dk, dv, chunk, H};
   gdn_prefill_algo_t resolved;
-  if (gdn::prefill_resolve(s, GDN_BF16, algo, &resolved) != GDN_OK) return (size_t)-1;
+  if (gdn::prefill_resolve(s, GDN_BF16, 0, algo, &resolved) != GDN_OK) return (size_t)-1;
   return gdn::prefill_workspace_bytes(s, resolved);
 }
 
 gdn_status_t gdn_chunk_prefill(const void* q, const void* k, const void* v, const float* g,
                                const float* beta, const int32_t* cu_seqlens, int N,
                                int64_t total_T, const float* initial_state, float* final_state,
-                               void* o, int H, int dk, int dv, int chunk, float scale,
-                               gdn_dtype_t in_dtype, gdn_dtype_t out_dtype,
+                               void* o, int H, int H_qk, int dk, int dv, int chunk, float scale,
+                               uint32_t flags, gdn_dtype_t in_dtype, gdn_dtype_t out_dtype,
                                gdn_prefill_algo_t algo, void* workspace, size_t workspace_bytes,
                                void* stream) {
   GDN_REQUIRE(valid_dtype(in_dtype) && valid_dtype(out_dtype), GDN_ERR_INVALID_ARG,
               "gdn_chunk_prefill: unknown dtype");
-  gdn::PrefillShape s{N, total_T, H, dk, dv, chunk};
+  gdn::PrefillShape s{N, total_T, H, dk, dv, chunk, H_qk};
   gdn_prefill_algo_t resolved;
-  gdn_status_t st = gdn::prefill_resolve(s, in_dtype, algo, &resolved);
+  gdn_status_t st = gdn::prefill_resolve(s, in_dtype, flags, algo, &resolved);
   if (st != GDN_OK) return st;
   if (N == 0) return gdn::ok();
   GDN_REQUIRE(cu_seqlens != nullptr, GDN_ERR_INVALID_ARG, "gdn_chunk_prefill: cu_seqlens is NULL");
@@ -177,7 +181,7 @@ gdn_status_t gdn_chunk_prefill(const void* q, const void* k, const void* v, cons
   st = gdn::device_error_word(&err);
   if (st != GDN_OK) return st;
   gdn::PrefillArgs a{q, k, v, g, beta, cu_seqlens, initial_state, final_state, o, scale,
-                     in_dtype, out_dtype, workspace, err, gdn::kPrefillOutputs};
+                     in_dtype, out_dtype, workspace, err, gdn::kPrefillOutputs, flags};
   return gdn::prefill_launch(s, a, resolved, gdn::as_stream(stream));
 }
 

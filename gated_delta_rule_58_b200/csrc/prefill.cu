@@ -32,11 +32,14 @@ gdn_prefill_algo_t prefill_auto_tensor_core(const PrefillShape& s) {
   return transfer < 0.8 * fused ? GDN_PREFILL_TRANSFER : GDN_PREFILL_FUSED;
 }
 
-gdn_status_t prefill_resolve(const PrefillShape& s, gdn_dtype_t in, gdn_prefill_algo_t requested,
+gdn_status_t prefill_resolve(const PrefillShape& s, gdn_dtype_t in, uint32_t flags, gdn_prefill_algo_t requested,
                              gdn_prefill_algo_t* resolved) {
   (void)in;
   if (s.N < 0 || s.total_T < 0 || s.H < 1 || s.dk < 1 || s.dv < 1 || s.chunk < 1)
     return fail(GDN_ERR_INVALID_ARG, "gdn_chunk_prefill: need N >= 0, total_T >= 0, H, dk, dv, chunk >= 1");
+  if (s.Hqk < 1 || s.H % s.Hqk != 0)
+    return fail(GDN_ERR_INVALID_ARG, "gdn_chunk_prefill: H_qk must be >= 1 and divide H");
+  if ((flags & ~GDN_QK_L2NORM) != 0) return fail(GDN_ERR_INVALID_ARG, "gdn_chunk_prefill: unknown flags");
   if (s.total_T > (int64_t)INT32_MAX)
     return fail(GDN_ERR_UNSUPPORTED, "gdn_chunk_prefill: total_T must fit int32 (cu_seqlens is int32)");
   const bool seq_ok = s.dk == s.dv && (s.dk == 32 || s.dk == 64 || s.dk == 128);

@@ -9,6 +9,7 @@ struct PrefillShape {
   int N;            // sequences
   int64_t total_T;  // packed tokens
   int H, dk, dv, chunk;
+  int Hqk;          // query/key heads (H is a multiple); value head h reads q/k head h / (H / Hqk)
 };
 
 struct PrefillArgs {
@@ -30,6 +31,7 @@ struct PrefillArgs {
   // sequence). kPrefillTransfer: identity initial state, values taken as zero, no
   // outputs (final state = the transfer matrix M^T of each sequence, K-last).
   int mode;
+  uint32_t flags;  // GDN_QK_L2NORM
 };
 
 constexpr int kPrefillOutputs = 0;
@@ -37,7 +39,7 @@ constexpr int kPrefillLocalState = 1;
 constexpr int kPrefillTransfer = 2;
 
 // Validates the shape for `requested` and resolves GDN_PREFILL_AUTO.
-gdn_status_t prefill_resolve(const PrefillShape& s, gdn_dtype_t in, gdn_prefill_algo_t requested,
+gdn_status_t prefill_resolve(const PrefillShape& s, gdn_dtype_t in, uint32_t flags, gdn_prefill_algo_t requested,
                              gdn_prefill_algo_t* resolved);
 // AUTO choice between the two tensor-core algorithms (dk == dv == 128, chunk == 64).
 gdn_prefill_algo_t prefill_auto_tensor_core(const PrefillShape& s);

@@ -79,7 +79,8 @@ constexpr uint32_t P_BUF = 8192;
 constexpr uint32_t OFF_A = 180224;      // A fp32 [64][64], 16-byte chunks XOR-swizzled by row
 constexpr uint32_t OFF_T = 196608;      // T fp32 [64][64], same swizzle
 constexpr uint32_t OFF_VEC = 212992;    // 3 buffers (chunk % 3) x {G, gamma, dd, beta, beta*gamma} x 64 fp32
-constexpr uint32_t VEC_BUF = 5 * C * 4;
+                                        // + 128 inverse q/k norms
+constexpr uint32_t VEC_BUF = 7 * C * 4;
 constexpr uint32_t OFF_BAR = OFF_VEC + 3 * VEC_BUF;
 constexpr uint32_t SMEM_USED = OFF_BAR + 256;
 constexpr uint32_t SMEM_BYTES = SMEM_USED + 1024;  // slack for the 1024-byte alignment
@@ -145,8 +146,9 @@ struct Smem {
   __device__ uint32_t u32(uint32_t off) const { return tc::smem_u32(base + off); }
 };
 // vec(b) layout: [0,64) G log2(e) (cumulative log gate in base 2), [64,128) gamma,
-// [128,192) dd, [192,256) beta, [256,320) beta*gamma
-constexpr int V_G = 0, V_GAM = 64, V_DD = 128, V_BETA = 192, V_BG = 256;
+// [128,192) dd, [192,256) beta, [256,320) beta*gamma, [320,448) 1/|k_i| then 1/|q_i|
+// (with the q/k normalisation only)
+constexpr int V_G = 0, V_GAM = 64, V_DD = 128, V_BETA = 192, V_BG = 256, V_RN = 320;
 constexpr float kLog2e = 1.4426950408889634f;
 
 // 2^x on the special-function unit (exp(y) = 2^(y log2 e)); results below the
@@ -184,29 +186,34 @@ struct QkvMaps {
 // TMA loads of the raw bf16 K, Q (and V) tiles of the chunk starting at token t0
 // into tile buffer b, completing on B_T0 + b. Issued by one thread, once the
 // buffer's previous chunk (two chunks back) has had its last MMA complete.
-__device__ __forceinline__ void issue_tile_loads(const Smem& sm, const QkvMaps& maps, int b, int h, int64_t t0,
-                                                 bool zero_values) {
+__device__ __forceinline__ void issue_tile_loads(const Smem& sm, const QkvMaps& maps, int b, int h, int hq,
+                                                 int64_t t0, bool zero_values) {
   uint8_t* kq = sm.base + OFF_KQ + b * KQ_BUF;
   uint8_t* v16 = sm.base + OFF_V + b * V_BUF;
   tc::fence_proxy_async_smem();  // the previous generic writes of these tiles precede the copies
   tc::mbar_arrive_expect_tx(sm.bar(B_T0 + b), (zero_values ? 2u : 3u) * 16384u);
 #pragma unroll
   for (int hf = 0; hf < 2; ++hf) {
-    tc::tma_load_3d(tc::smem_u32(kq + hf * KQ_HALF), &maps.k, 64 * hf, h, (int)t0, sm.bar(B_T0 + b));
-    tc::tma_load_3d(tc::smem_u32(kq + hf * KQ_HALF + C * 128), &maps.q, 64 * hf, h, (int)t0, sm.bar(B_T0 + b));
+    tc::tma_load_3d(tc::smem_u32(kq + hf * KQ_HALF), &maps.k, 64 * hf, hq, (int)t0, sm.bar(B_T0 + b));
+    tc::tma_load_3d(tc::smem_u32(kq + hf * KQ_HALF + C * 128), &maps.q, 64 * hf, hq, (int)t0, sm.bar(B_T0 + b));
     if (!zero_values)
       tc::tma_load_3d(tc::smem_u32(v16 + hf * V_HALF), &maps.v, 64 * hf, h, (int)t0, sm.bar(B_T0 + b));
   }
 }
 
-// bf16 -> fp16 of one 16-byte chunk (8 elements) in place.
-__device__ __forceinline__ void convert_chunk_bf16(uint8_t* p) {
+// bf16 -> fp16 of one 16-byte chunk (8 elements) in place, times `sc` if kScale.
+template <bool kScale>
+__device__ __forceinline__ void convert_chunk_bf16(uint8_t* p, float sc = 1.f) {
   uint4* q = reinterpret_cast<uint4*>(p);
   const uint4 raw = *q;
   const __nv_bfloat162* hb = reinterpret_cast<const __nv_bfloat162*>(&raw);
   uint4 u;
-  const float2 f0 = __bfloat1622float2(hb[0]), f1 = __bfloat1622float2(hb[1]);
-  const float2 f2 = __bfloat1622float2(hb[2]), f3 = __bfloat1622float2(hb[3]);
+  float2 f0 = __bfloat1622float2(hb[0]), f1 = __bfloat1622float2(hb[1]);
+  float2 f2 = __bfloat1622float2(hb[2]), f3 = __bfloat1622float2(hb[3]);
+  if (kScale) {
+    f0.x *= sc; f0.y *= sc; f1.x *= sc; f1.y *= sc;
+    f2.x *= sc; f2.y *= sc; f3.x *= sc; f3.y *= sc;
+  }
   u.x = pack_half2(f0.x, f0.y);
   u.y = pack_half2(f1.x, f1.y);
   u.z = pack_half2(f2.x, f2.y);
@@ -242,6 +249,11 @@ __device__ void loader_role(const Smem& sm, const PrefillShape& s, const Prefill
   constexpr bool kTma = std::is_same<TIn, __nv_bfloat16>::value;
   const int t = threadIdx.x - kLoadWarp0 * 32;  // 0..127
   const bool zero_values = (a.mode == kPrefillTransfer);  // transfer run: V taken as 0
+  const int hq = h / (s.H / s.Hqk);                       // the value head's query/key head
+  // With the q/k normalisation K and Q are scaled by their inverse norms while
+  // they are converted to fp16, and the conversion happens before [K;Q]K^T, which
+  // then reads the fp16 tiles (as for fp32 inputs).
+  const bool l2 = (a.flags & GDN_QK_L2NORM) != 0;
   if (zero_values) {  // both V buffers stay zero for the whole run
     for (int i = t; i < 2 * V_BUF / 16; i += 128)
       *reinterpret_cast<uint4*>(sm.base + OFF_V + 16 * i) = make_uint4(0u, 0u, 0u, 0u);
@@ -268,7 +280,7 @@ __device__ void loader_role(const Smem& sm, const PrefillShape& s, const Prefill
     if constexpr (kTma) {
       // rows past the sequence end load the next tokens (or zeros past the tensor);
       // they are zeroed once the copies have landed, and their beta and g are 0
-      if (c < 2 && t == 0) issue_tile_loads(sm, maps, b, h, t0, zero_values);
+      if (c < 2 && t == 0) issue_tile_loads(sm, maps, b, h, hq, t0, zero_values);
       if (!wait_bar(sm, B_T0 + b, (c >> 1) & 1, a.err)) return;
     } else {
       if (c >= 2 && !wait_bar(sm, B_M4B, (c - 2) & 1, a.err)) return;
@@ -320,20 +332,71 @@ __device__ void loader_role(const Smem& sm, const PrefillShape& s, const Prefill
           *reinterpret_cast<uint4*>(base + row * 128 + ch * 16) = make_uint4(0u, 0u, 0u, 0u);
         }
       }
-      group_signal(sm, kBarLoad, B_L0 + b);
-      if (t == 0 && !issue_d1(sm, tmem, c, b, 1, a.err)) return;
-      if (!wait_bar(sm, B_M1, c & 1, a.err)) return;
-      tc::fence_after_sync();
+      if (l2) {
+        // thread t: 1 / |row t| of the [K;Q] tile stack from the raw bf16 row (both
+        // 64-column halves; the chunk order within a row does not matter)
+        tc::named_sync(kBarLoad, 128);  // the zeroed rows are written
+        float ss = 0.f;
+#pragma unroll
+        for (int hf = 0; hf < 2; ++hf)
+#pragma unroll
+          for (int ch = 0; ch < 8; ++ch) {
+            const uint4 raw = *reinterpret_cast<const uint4*>(kq + hf * KQ_HALF + t * 128 + ch * 16);
+            const __nv_bfloat162* hb = reinterpret_cast<const __nv_bfloat162*>(&raw);
+#pragma unroll
+            for (int x = 0; x < 4; ++x) {
+              const float2 f = __bfloat1622float2(hb[x]);
+              ss = fmaf(f.x, f.x, fmaf(f.y, f.y, ss));
+            }
+          }
+        vec[V_RN + t] = ss > 0.f ? 1.f / sqrtf(ss) : 0.f;
+        tc::named_sync(kBarLoad, 128);
 #pragma unroll 4
-      for (int i = t; i < 3 * C * 16; i += 128) {
-        const int mat = i >> 10, rem = i & 1023;  // 0 K, 1 Q, 2 V; 64 rows x 16 chunks each
-        const int row = rem >> 4, ch = rem & 15;
-        if (mat == 2 && zero_values) continue;
-        uint8_t* tile = (mat == 2) ? v16 + (ch >> 3) * V_HALF : kq + (ch >> 3) * KQ_HALF;
-        const int trow = row + (mat == 1 ? C : 0);
-        convert_chunk_bf16(tile + tc::sw128_offset(trow, ch & 7, 1024));
+        for (int i = t; i < 3 * C * 16; i += 128) {
+          const int mat = i >> 10, rem = i & 1023;  // 0 K, 1 Q, 2 V; 64 rows x 16 chunks each
+          const int row = rem >> 4, ch = rem & 15;
+          if (mat == 2 && zero_values) continue;
+          uint8_t* tile = (mat == 2) ? v16 + (ch >> 3) * V_HALF : kq + (ch >> 3) * KQ_HALF;
+          const int trow = row + (mat == 1 ? C : 0);
+          if (mat < 2)  // warp-uniform: the matrices are 1024 chunks apart
+            convert_chunk_bf16<true>(tile + tc::sw128_offset(trow, ch & 7, 1024), vec[V_RN + trow]);
+          else
+            convert_chunk_bf16<false>(tile + tc::sw128_offset(trow, ch & 7, 1024));
+        }
+        group_signal(sm, kBarLoad, B_L0 + b);
+        if (t == 0 && !issue_d1(sm, tmem, c, b, 0, a.err)) return;
+      } else {
+        group_signal(sm, kBarLoad, B_L0 + b);
+        if (t == 0 && !issue_d1(sm, tmem, c, b, 1, a.err)) return;
+        if (!wait_bar(sm, B_M1, c & 1, a.err)) return;
+        tc::fence_after_sync();
+#pragma unroll 4
+        for (int i = t; i < 3 * C * 16; i += 128) {
+          const int mat = i >> 10, rem = i & 1023;  // 0 K, 1 Q, 2 V; 64 rows x 16 chunks each
+          const int row = rem >> 4, ch = rem & 15;
+          if (mat == 2 && zero_values) continue;
+          uint8_t* tile = (mat == 2) ? v16 + (ch >> 3) * V_HALF : kq + (ch >> 3) * KQ_HALF;
+          const int trow = row + (mat == 1 ? C : 0);
+          convert_chunk_bf16<false>(tile + tc::sw128_offset(trow, ch & 7, 1024));
+        }
       }
     } else {
+      if (l2) {  // thread t: 1 / |row t| of [K;Q] (zero past the sequence end)
+        const int row = t & 63;
+        float ss = 0.f;
+        if (row < Lc) {
+          const TIn* src = static_cast<const TIn*>(t < C ? a.k : a.q) + ((size_t)(t0 + row) * s.Hqk + hq) * D;
+#pragma unroll 4
+          for (int e = 0; e < D; e += 8) {
+            float v8[8];
+            load8_f32(src + e, v8);
+#pragma unroll
+            for (int x = 0; x < 8; ++x) ss = fmaf(v8[x], v8[x], ss);
+          }
+        }
+        vec[V_RN + t] = ss > 0.f ? 1.f / sqrtf(ss) : 0.f;
+        tc::named_sync(kBarLoad, 128);
+      }
 #pragma unroll
       for (int mat = 0; mat < 3; ++mat) {
         if (mat == 2 && zero_values) continue;
@@ -346,7 +409,13 @@ __device__ void loader_role(const Smem& sm, const PrefillShape& s, const Prefill
           const int row = i >> 4, ch = i & 15;
           float v8[8];
           if (row < Lc) {
-            load8_f32(src0 + ((size_t)(t0 + row) * s.H + h) * D + ch * 8, v8);
+            const size_t tok = (mat == 2) ? (size_t)(t0 + row) * s.H + h : (size_t)(t0 + row) * s.Hqk + hq;
+            load8_f32(src0 + tok * D + ch * 8, v8);
+            if (l2 && mat < 2) {
+              const float r = vec[V_RN + row + roff];
+#pragma unroll
+              for (int x = 0; x < 8; ++x) v8[x] *= r;
+            }
           } else {
 #pragma unroll
             for (int x = 0; x < 8; ++x) v8[x] = 0.f;
@@ -714,7 +783,8 @@ __device__ void state_role(const Smem& sm, const PrefillShape& s, const PrefillA
     tc::fence_after_sync();
     // chunk c's state update was the last reader of tile buffer b: chunk c+2's
     // copies go out now, well before the loader needs them
-    if (kTmaLoads && j == 0 && c + 2 < nchunks) issue_tile_loads(sm, maps, b, h, t0 + 2 * C, a.mode == kPrefillTransfer);
+    if (kTmaLoads && j == 0 && c + 2 < nchunks)
+      issue_tile_loads(sm, maps, b, h, h / (s.H / s.Hqk), t0 + 2 * C, a.mode == kPrefillTransfer);
     const bool last = (c == nchunks - 1);
     float gnext = 1.f;
     if (!last) {
@@ -970,13 +1040,15 @@ gdn_status_t launch(const PrefillShape& s, const PrefillArgs& a, cudaStream_t st
   QkvMaps maps;
   memset(&maps, 0, sizeof(maps));
   if (std::is_same<TIn, __nv_bfloat16>::value && s.total_T > 0) {
-    // q, k, v as {128, H, total_T} bf16; one box = 64 features x 64 tokens of one head
-    const uint64_t dims[3] = {(uint64_t)D, (uint64_t)s.H, (uint64_t)s.total_T};
-    const uint64_t strides[2] = {(uint64_t)D * 2, (uint64_t)s.H * D * 2};
+    // q, k as {128, H_qk, total_T} and v as {128, H, total_T} bf16; one box = 64
+    // features x 64 tokens of one head
     const uint32_t box[3] = {64, 1, (uint32_t)C};
     const void* src[3] = {a.q, a.k, a.v};
     CUtensorMap* dst[3] = {&maps.q, &maps.k, &maps.v};
     for (int i = 0; i < 3; ++i) {
+      const uint64_t heads = (i == 2) ? (uint64_t)s.H : (uint64_t)s.Hqk;
+      const uint64_t dims[3] = {(uint64_t)D, heads, (uint64_t)s.total_T};
+      const uint64_t strides[2] = {(uint64_t)D * 2, heads * D * 2};
       const gdn_status_t st = make_tensor_map_3d(dst[i], CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, src[i], dims, strides, box,
                                                  "fused prefill");
       if (st != GDN_OK) return st;

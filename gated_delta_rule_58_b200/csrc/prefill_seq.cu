@@ -11,7 +11,8 @@
 //     o_j = scale * q . S[:, j]
 // which is S_t = alpha (I - beta k k^T) S_{t-1} + beta k v^T column by column.
 // k, q, v of the token are staged in double-buffered shared memory (one barrier
-// per token).
+// per token). With GDN_QK_L2NORM, k and q are used divided by their Euclidean
+// norms, which the TPC lanes of a column reduce from their own 32 entries.
 #include "prefill.cuh"
 
 namespace gdn {
@@ -33,6 +34,8 @@ gdn_prefill_sequential_kernel(const PrefillShape s, const PrefillArgs a) {
   const int part = tid % TPC;        // which 32 entries of the column
   const int n = blockIdx.x / s.H;
   const int h = blockIdx.x - n * s.H;
+  const int hq = h / (s.H / s.Hqk);  // the value head's query/key head
+  const bool l2 = (a.flags & GDN_QK_L2NORM) != 0;
   int64_t bos, eos;
   if (!seq_bounds(a.cu_seqlens, n, s.total_T, a.err, &bos, &eos)) return;
 
@@ -56,10 +59,11 @@ gdn_prefill_sequential_kernel(const PrefillShape s, const PrefillArgs a) {
 
   for (int64_t t = bos; t < eos; ++t) {
     const int buf = (int)(t - bos) & 1;
-    const size_t th = (size_t)t * s.H + h;
+    const size_t th = (size_t)t * s.H + h;       // v, g, beta, o
+    const size_t tq = (size_t)t * s.Hqk + hq;    // q, k
     for (int i = tid; i < D; i += NT) {
-      s_k[buf][i] = to_f32(kp[th * D + i]);
-      s_q[buf][i] = to_f32(qp[th * D + i]);
+      s_k[buf][i] = to_f32(kp[tq * D + i]);
+      s_q[buf][i] = to_f32(qp[tq * D + i]);
       s_v[buf][i] = to_f32(vp[th * D + i]);
     }
     if (tid == 0) {
@@ -70,12 +74,28 @@ gdn_prefill_sequential_kernel(const PrefillShape s, const PrefillArgs a) {
     const float alpha = s_ab[buf][0], beta = s_ab[buf][1];
     const float* kv = s_k[buf] + part * PER;
     const float* qv = s_q[buf] + part * PER;
+    float rk = 1.f, rq = 1.f;  // 1 / |k|, 1 / |q| with the normalisation
+    if (l2) {
+      float kk = 0.f, qq = 0.f;
+#pragma unroll
+      for (int i = 0; i < PER; ++i) {
+        kk = fmaf(kv[i], kv[i], kk);
+        qq = fmaf(qv[i], qv[i], qq);
+      }
+#pragma unroll
+      for (int off = 1; off < TPC; off <<= 1) {
+        kk += __shfl_xor_sync(0xffffffffu, kk, off);
+        qq += __shfl_xor_sync(0xffffffffu, qq, off);
+      }
+      rk = kk > 0.f ? 1.f / sqrtf(kk) : 0.f;
+      rq = qq > 0.f ? 1.f / sqrtf(qq) : 0.f;
+    }
     float u = 0.f;
 #pragma unroll
     for (int i = 0; i < PER; ++i) u = fmaf(kv[i], st[i], u);
 #pragma unroll
     for (int off = 1; off < TPC; off <<= 1) u += __shfl_xor_sync(0xffffffffu, u, off);
-    const float c = beta * (s_v[buf][col] - alpha * u);
+    const float c = beta * (s_v[buf][col] - alpha * (u * rk)) * rk;  // the update adds c k
     float o = 0.f;
 #pragma unroll
     for (int i = 0; i < PER; ++i) {
@@ -84,7 +104,7 @@ gdn_prefill_sequential_kernel(const PrefillShape s, const PrefillArgs a) {
     }
 #pragma unroll
     for (int off = 1; off < TPC; off <<= 1) o += __shfl_xor_sync(0xffffffffu, o, off);
-    if (part == 0) store_out(op + th * D + col, a.scale * o);
+    if (part == 0) store_out(op + th * D + col, a.scale * (o * rq));
   }
 
   if (a.final_state) {

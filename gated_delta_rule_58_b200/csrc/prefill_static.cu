@@ -65,14 +65,14 @@ bool ptr_ok(const void* p) { return p != nullptr && aligned16(p); }
 
 extern "C" gdn_status_t gdn_chunk_prefill_static_scratch(
     const void* q, const void* k, const void* v, const float* g, const float* beta, const int32_t* cu_seqlens,
-    int N, int64_t total_T, const float* initial_state, float* final_state, void* o, int H, int dk, int dv,
-    int chunk, float scale, gdn_dtype_t in_dtype, gdn_dtype_t out_dtype, void* stream) {
+    int N, int64_t total_T, const float* initial_state, float* final_state, void* o, int H, int H_qk, int dk,
+    int dv, int chunk, float scale, uint32_t flags, gdn_dtype_t in_dtype, gdn_dtype_t out_dtype, void* stream) {
   using gdn::fail;
   if (!((in_dtype == GDN_BF16 || in_dtype == GDN_F32) && (out_dtype == GDN_BF16 || out_dtype == GDN_F32)))
     return fail(GDN_ERR_INVALID_ARG, "gdn_chunk_prefill_static_scratch: unknown dtype");
-  gdn::PrefillShape s{N, total_T, H, dk, dv, chunk};
+  gdn::PrefillShape s{N, total_T, H, dk, dv, chunk, H_qk};
   gdn_prefill_algo_t resolved;
-  gdn_status_t st = gdn::prefill_resolve(s, in_dtype, GDN_PREFILL_TRANSFER, &resolved);
+  gdn_status_t st = gdn::prefill_resolve(s, in_dtype, flags, GDN_PREFILL_TRANSFER, &resolved);
   if (st != GDN_OK) return st;
   if (N == 0) return gdn::ok();
   if (cu_seqlens == nullptr) return fail(GDN_ERR_INVALID_ARG, "gdn_chunk_prefill_static_scratch: cu_seqlens is NULL");
@@ -95,6 +95,6 @@ extern "C" gdn_status_t gdn_chunk_prefill_static_scratch(
   st = gdn::device_error_word(&err);
   if (st != GDN_OK) return st;
   gdn::PrefillArgs a{q, k, v, g, beta, cu_seqlens, initial_state, final_state, o, scale,
-                     in_dtype, out_dtype, scratch, err, gdn::kPrefillOutputs};
+                     in_dtype, out_dtype, scratch, err, gdn::kPrefillOutputs, flags};
   return gdn::prefill_transfer_launch(s, a, gdn::as_stream(stream));
 }

@@ -69,16 +69,21 @@ class DecodeInputs:
 
 def decode_inputs(B: int, T: int, H: int, dk: int, dv: int, n_h: int, num_slots: int,
                   seed: int = 0, dtype=torch.bfloat16, device="cpu",
-                  g_range=DEFAULT_G_RANGE, state_std: float = 0.1) -> DecodeInputs:
-    """Inputs of one (multi-token, multi-Householder) decode step.
+                  g_range=DEFAULT_G_RANGE, state_std: float = 0.1, H_qk: Optional[int] = None,
+                  normalize_qk: bool = True) -> DecodeInputs:
+    """Inputs of one (multi-token, multi-Householder) decode step. q and k have
+    H_qk heads (default H); with normalize_qk=False they are left as N(0, 1) draws
+    (for the in-kernel normalisation).
 
     Draw order: q, k, v, beta, g, pool, slot permutation.
     """
     if B > num_slots:
         raise ValueError("B must not exceed num_slots (slot ids are distinct)")
+    H_qk = H if H_qk is None else H_qk
+    unit = _unit_rows if normalize_qk else (lambda x: x)
     gen = _gen(seed, device)
-    q = _unit_rows(_draw_normal((B, T, H, dk), gen, device)).to(dtype)
-    k = _unit_rows(_draw_normal((B, T, H, n_h, dk), gen, device)).to(dtype)
+    q = unit(_draw_normal((B, T, H_qk, dk), gen, device)).to(dtype)
+    k = unit(_draw_normal((B, T, H_qk, n_h, dk), gen, device)).to(dtype)
     v = _draw_normal((B, T, H, n_h, dv), gen, device).to(dtype)
     beta = _draw_beta((B, T, H, n_h), gen, device)
     g = _draw_gate((B, T, H), gen, device, g_range)
@@ -114,16 +119,20 @@ def varlen_lengths(n: int, lo: int, hi: int, seed: int = 0) -> list:
 
 def prefill_inputs(seqlens: Sequence[int], H: int, dk: int, dv: int, seed: int = 0,
                    dtype=torch.bfloat16, device="cpu", g_range=DEFAULT_G_RANGE,
-                   with_initial_state: bool = True, state_std: float = 0.1) -> PrefillInputs:
-    """Packed varlen prefill inputs for sequences of the given lengths.
+                   with_initial_state: bool = True, state_std: float = 0.1, H_qk: Optional[int] = None,
+                   normalize_qk: bool = True) -> PrefillInputs:
+    """Packed varlen prefill inputs for sequences of the given lengths. q and k have
+    H_qk heads (default H); with normalize_qk=False they are left as N(0, 1) draws.
 
     Draw order: q, k, v, beta, g, initial state.
     """
     seqlens = [int(x) for x in seqlens]
     total = sum(seqlens)
+    H_qk = H if H_qk is None else H_qk
+    unit = _unit_rows if normalize_qk else (lambda x: x)
     gen = _gen(seed, device)
-    q = _unit_rows(_draw_normal((total, H, dk), gen, device)).to(dtype)
-    k = _unit_rows(_draw_normal((total, H, dk), gen, device)).to(dtype)
+    q = unit(_draw_normal((total, H_qk, dk), gen, device)).to(dtype)
+    k = unit(_draw_normal((total, H_qk, dk), gen, device)).to(dtype)
     v = _draw_normal((total, H, dv), gen, device).to(dtype)
     beta = _draw_beta((total, H), gen, device)
     g = _draw_gate((total, H), gen, device, g_range)

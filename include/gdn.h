@@ -35,6 +35,16 @@
  *    access) and a sticky device error word is set, read by gdn_get_device_error().
  *  - Input dtype: q, k, v are GDN_BF16 or GDN_F32 (same dtype for all three); g
  *    and beta are always fp32; o is GDN_BF16 (round-to-nearest-even) or GDN_F32.
+ *  - Heads. H counts the value heads: v, g, beta, o and the states have H heads.
+ *    q and k may have fewer, H_qk, with H a multiple of H_qk: value head h reads
+ *    query/key head h / (H / H_qk), so consecutive value heads share one q/k head
+ *    (grouped value heads, the layout of models whose q/k projections are repeated
+ *    over value heads). H_qk = H is the one-to-one case. This and the q/k
+ *    normalisation below are plain extensions of the recurrence; the pages do not
+ *    discuss them.
+ *  - flags: GDN_QK_L2NORM scales q and every k to unit Euclidean length per token
+ *    (and per q/k head) inside the kernels before use, in fp32 (a zero vector
+ *    stays zero); without it q and k are used as given.
  */
 #ifndef GDN_H_
 #define GDN_H_
@@ -57,6 +67,9 @@ typedef enum {
 
 typedef enum { GDN_BF16 = 0, GDN_F32 = 1 } gdn_dtype_t;
 
+/* flags of gdn_decode / gdn_chunk_prefill */
+#define GDN_QK_L2NORM 0x1u  /* normalise q and k to unit length per token, in the kernel */
+
 /* Bits of the sticky device error word (gdn_get_device_error). */
 #define GDN_DEVERR_SLOT_OUT_OF_RANGE 0x1u  /* a slot id >= num_slots was skipped */
 #define GDN_DEVERR_BAD_CU_SEQLENS 0x2u     /* cu_seqlens not 0-based / non-decreasing / > total_T */
@@ -72,9 +85,9 @@ typedef enum { GDN_BF16 = 0, GDN_F32 = 1 } gdn_dtype_t;
  * variant of the FlashInfer PR #7156 page); n_h > 1 and/or T > 1 is the gated
  * delta product multi-token step of the same page.
  *
- *   q          [B, T, H, dk]        in_dtype
- *   k          [B, T, H, n_h, dk]   in_dtype
- *   v          [B, T, H, n_h, dv]   in_dtype
+ *   q          [B, T, H_qk, dk]       in_dtype
+ *   k          [B, T, H_qk, n_h, dk]  in_dtype
+ *   v          [B, T, H, n_h, dv]     in_dtype
  *   g          [B, T, H]            fp32, log-space gate (alpha = exp(g); -inf allowed)
  *   beta       [B, T, H, n_h]       fp32
  *   state_pool [num_slots, H, dv, dk] fp32, K-last; read and written in place
@@ -88,9 +101,9 @@ typedef enum { GDN_BF16 = 0, GDN_F32 = 1 } gdn_dtype_t;
  */
 gdn_status_t gdn_decode(const void* q, const void* k, const void* v, const float* g,
                         const float* beta, float* state_pool, int num_slots,
-                        const int32_t* slot_ids, void* o, int B, int T, int H, int dk, int dv,
-                        int n_h, float scale, gdn_dtype_t in_dtype, gdn_dtype_t out_dtype,
-                        void* stream);
+                        const int32_t* slot_ids, void* o, int B, int T, int H, int H_qk,
+                        int dk, int dv, int n_h, float scale, uint32_t flags,
+                        gdn_dtype_t in_dtype, gdn_dtype_t out_dtype, void* stream);
 
 /* Prefill algorithm selection (gdn_chunk_prefill / gdn_chunk_prefill_workspace_size). */
 typedef enum {
@@ -128,7 +141,7 @@ size_t gdn_chunk_prefill_workspace_size(int N, int64_t total_T, int H, int dk, i
  * local state H_c; FlashInfer PR #3866 page, section 2). An empty sequence
  * copies its initial state (or zeros) to final_state.
  *
- *   q, k          [total_T, H, dk]   in_dtype
+ *   q, k          [total_T, H_qk, dk] in_dtype
  *   v             [total_T, H, dv]   in_dtype
  *   g, beta       [total_T, H]       fp32 (g finite)
  *   cu_seqlens    [N + 1] int32, DEVICE; cu[0] = 0, non-decreasing, cu[N] = total_T
@@ -146,8 +159,8 @@ size_t gdn_chunk_prefill_workspace_size(int N, int64_t total_T, int H, int dk, i
 gdn_status_t gdn_chunk_prefill(const void* q, const void* k, const void* v, const float* g,
                                const float* beta, const int32_t* cu_seqlens, int N,
                                int64_t total_T, const float* initial_state, float* final_state,
-                               void* o, int H, int dk, int dv, int chunk, float scale,
-                               gdn_dtype_t in_dtype, gdn_dtype_t out_dtype,
+                               void* o, int H, int H_qk, int dk, int dv, int chunk, float scale,
+                               uint32_t flags, gdn_dtype_t in_dtype, gdn_dtype_t out_dtype,
                                gdn_prefill_algo_t algo, void* workspace, size_t workspace_bytes,
                                void* stream);
 
@@ -173,9 +186,9 @@ gdn_status_t gdn_chunk_prefill(const void* q, const void* k, const void* v, cons
 gdn_status_t gdn_chunk_prefill_static_scratch(const void* q, const void* k, const void* v, const float* g,
                                               const float* beta, const int32_t* cu_seqlens, int N,
                                               int64_t total_T, const float* initial_state,
-                                              float* final_state, void* o, int H, int dk, int dv,
-                                              int chunk, float scale, gdn_dtype_t in_dtype,
-                                              gdn_dtype_t out_dtype, void* stream);
+                                              float* final_state, void* o, int H, int H_qk, int dk,
+                                              int dv, int chunk, float scale, uint32_t flags,
+                                              gdn_dtype_t in_dtype, gdn_dtype_t out_dtype, void* stream);
 
 /* Message for the last non-OK status returned on this host thread ("" if none). */
 const char* gdn_last_error(void);

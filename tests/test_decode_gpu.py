@@ -13,21 +13,21 @@ pytestmark = pytest.mark.gpu
 DEV = "cuda"
 
 
-def _run(inp, out_dtype=torch.bfloat16):
+def _run(inp, out_dtype=torch.bfloat16, l2norm=False):
     pool = inp.pool.to(DEV).clone()
     q, k, v = inp.q.to(DEV), inp.k.to(DEV), inp.v.to(DEV)
     g, beta = inp.g.to(DEV), inp.beta.to(DEV)
     slots = inp.slot_ids.to(DEV)
-    B, T, H, dk = q.shape
+    B, T, H = v.shape[:3]
     o = torch.empty((B, T, H, v.shape[-1]), dtype=out_dtype, device=DEV)
-    gdn.gdn_decode(q, k, v, g, beta, pool, slots, o, scale=inp.scale)
+    gdn.gdn_decode(q, k, v, g, beta, pool, slots, o, scale=inp.scale, l2norm=l2norm)
     torch.cuda.synchronize()
     return o, pool
 
 
-def _check_against_oracle(inp, o, pool, what):
+def _check_against_oracle(inp, o, pool, what, l2norm=False):
     o_ref, pool_ref, _ = oracle.decode(inp.q, inp.k, inp.v, inp.g, inp.beta, inp.pool, inp.slot_ids,
-                                       scale=inp.scale)
+                                       scale=inp.scale, l2norm=l2norm)
     assert_close(o, o_ref, what=f"{what} o")
     used = sorted(set(int(s) for s in inp.slot_ids.tolist() if 0 <= s < inp.pool.shape[0]))
     assert_close(pool[used], pool_ref[used], what=f"{what} state")
@@ -180,3 +180,42 @@ def test_split_v_b1_h4_against_oracle():
         inp = inputs.decode_inputs(1, 1, 4, 128, 128, 1, 3, seed=14)
         o, pool = _run(inp, out_dtype=out_dtype)
         _check_against_oracle(inp, o, pool, f"split-V B=1 H=4 ({out_dtype})")
+
+
+# ---------------------------------------------------------------- grouped q/k heads, q/k normalisation
+
+@pytest.mark.parametrize("l2norm", [False, True])
+@pytest.mark.parametrize("out_dtype", [torch.float32, torch.bfloat16])
+def test_grouped_heads_b64_hv32_hqk8(l2norm, out_dtype):
+    """T=1 decode with 32 value heads over 8 q/k heads (each q/k head shared by four
+    value heads), B=64, 256 slots; with the in-kernel normalisation q and k are
+    un-normalised N(0, 1) draws."""
+    inp = inputs.decode_inputs(64, 1, 32, 128, 128, 1, 256, seed=15, H_qk=8, normalize_qk=not l2norm)
+    o, pool = _run(inp, out_dtype=out_dtype, l2norm=l2norm)
+    _check_against_oracle(inp, o, pool, f"GVA B64 Hv32 Hqk8 l2={l2norm} ({out_dtype})", l2norm=l2norm)
+
+
+@pytest.mark.parametrize("T,nh", [(4, 2), (2, 1), (1, 4)])
+@pytest.mark.parametrize("l2norm", [False, True])
+def test_grouped_heads_multi_token(T, nh, l2norm):
+    inp = inputs.decode_inputs(9, T, 8, 128, 128, nh, 12, seed=16 + T, H_qk=2, normalize_qk=not l2norm)
+    o, pool = _run(inp, out_dtype=torch.float32, l2norm=l2norm)
+    _check_against_oracle(inp, o, pool, f"GVA T={T} nh={nh} l2={l2norm}", l2norm=l2norm)
+
+
+@pytest.mark.parametrize("d", [32, 64, 128])
+def test_grouped_heads_split_v_l2norm(d):
+    """Few heads (the split along V) with one q/k head for all value heads and the
+    normalisation on."""
+    inp = inputs.decode_inputs(2, 1, 4, d, d, 1, 5, seed=17 + d, H_qk=1, normalize_qk=False)
+    o, pool = _run(inp, out_dtype=torch.float32, l2norm=True)
+    _check_against_oracle(inp, o, pool, f"GVA split-V d={d}", l2norm=True)
+
+
+def test_l2norm_of_normalised_inputs_changes_little():
+    """On inputs that are already unit vectors (in bf16) the normalisation only
+    corrects their bf16 rounding of the norm."""
+    inp = inputs.decode_inputs(8, 1, 4, 128, 128, 1, 10, seed=18)
+    o1, p1 = _run(inp, out_dtype=torch.float32)
+    o2, p2 = _run(inp, out_dtype=torch.float32, l2norm=True)
+    assert_close(o2, o1, tol=5e-3, what="l2norm on unit inputs")

@@ -32,11 +32,12 @@ FAKE = 0x10000  # an aligned, never-dereferenced address: validation fails befor
 
 def _decode(L, **kw):
     a = dict(q=FAKE, k=FAKE, v=FAKE, g=FAKE, beta=FAKE, pool=FAKE, num_slots=4, slots=FAKE, o=FAKE,
-             B=2, T=1, H=2, dk=128, dv=128, nh=1, scale=0.1, din=0, dout=0, stream=None)
+             B=2, T=1, H=2, Hqk=None, dk=128, dv=128, nh=1, scale=0.1, flags=0, din=0, dout=0, stream=None)
     a.update(kw)
+    hqk = a["H"] if a["Hqk"] is None else a["Hqk"]
     return L.gdn_decode(a["q"], a["k"], a["v"], a["g"], a["beta"], a["pool"], a["num_slots"], a["slots"],
-                        a["o"], a["B"], a["T"], a["H"], a["dk"], a["dv"], a["nh"], a["scale"], a["din"],
-                        a["dout"], a["stream"])
+                        a["o"], a["B"], a["T"], a["H"], hqk, a["dk"], a["dv"], a["nh"], a["scale"], a["flags"],
+                        a["din"], a["dout"], a["stream"])
 
 
 @pytest.mark.parametrize("kw,status", [
@@ -49,6 +50,9 @@ def _decode(L, **kw):
     (dict(q=None), gdn.GDN_ERR_INVALID_ARG),
     (dict(pool=FAKE + 4), gdn.GDN_ERR_INVALID_ARG),
     (dict(slots=None), gdn.GDN_ERR_INVALID_ARG),
+    (dict(H=4, Hqk=3), gdn.GDN_ERR_INVALID_ARG),
+    (dict(Hqk=0), gdn.GDN_ERR_INVALID_ARG),
+    (dict(flags=0x2), gdn.GDN_ERR_INVALID_ARG),
 ])
 def test_decode_rejects_on_host(L, kw, status):
     assert _decode(L, **kw) == status
@@ -84,12 +88,14 @@ def test_prefill_raw_stream_handle_needs_an_explicit_workspace(L):
 
 def _prefill(L, **kw):
     a = dict(q=FAKE, k=FAKE, v=FAKE, g=FAKE, beta=FAKE, cu=FAKE, N=1, total=64, init=None, fin=FAKE,
-             o=FAKE, H=2, dk=32, dv=32, chunk=16, scale=0.1, din=1, dout=1, algo=0, ws=None, wsb=0,
-             stream=None)
+             o=FAKE, H=2, Hqk=None, dk=32, dv=32, chunk=16, scale=0.1, flags=0, din=1, dout=1, algo=0, ws=None,
+             wsb=0, stream=None)
     a.update(kw)
+    hqk = a["H"] if a["Hqk"] is None else a["Hqk"]
     return L.gdn_chunk_prefill(a["q"], a["k"], a["v"], a["g"], a["beta"], a["cu"], a["N"], a["total"],
-                               a["init"], a["fin"], a["o"], a["H"], a["dk"], a["dv"], a["chunk"],
-                               a["scale"], a["din"], a["dout"], a["algo"], a["ws"], a["wsb"], a["stream"])
+                               a["init"], a["fin"], a["o"], a["H"], hqk, a["dk"], a["dv"], a["chunk"],
+                               a["scale"], a["flags"], a["din"], a["dout"], a["algo"], a["ws"], a["wsb"],
+                               a["stream"])
 
 
 def test_auto_choice_between_fused_and_transfer():
@@ -117,6 +123,9 @@ def test_auto_choice_between_fused_and_transfer():
     (dict(algo=9), gdn.GDN_ERR_INVALID_ARG),
     (dict(dk=128, dv=128, chunk=32, algo=gdn.GDN_PREFILL_FUSED), gdn.GDN_ERR_UNSUPPORTED),
     (dict(dout=5), gdn.GDN_ERR_INVALID_ARG),
+    (dict(H=4, Hqk=3), gdn.GDN_ERR_INVALID_ARG),
+    (dict(Hqk=0), gdn.GDN_ERR_INVALID_ARG),
+    (dict(flags=0x10), gdn.GDN_ERR_INVALID_ARG),
 ])
 def test_prefill_rejects_on_host(L, kw, status):
     assert _prefill(L, **kw) == status

@@ -15,11 +15,11 @@ SEQ = gdn.GDN_PREFILL_SEQUENTIAL
 
 
 def run_prefill(inp, algo, chunk=64, out_dtype=torch.float32, with_final=True, alias=False,
-                workspace=None):
+                workspace=None, l2norm=False):
     q, k, v = inp.q.to(DEV), inp.k.to(DEV), inp.v.to(DEV)
     g, beta, cu = inp.g.to(DEV), inp.beta.to(DEV), inp.cu_seqlens.to(DEV)
-    total, H, dk = q.shape
-    dv = v.shape[-1]
+    total, dk = q.shape[0], q.shape[2]
+    H, dv = v.shape[1], v.shape[-1]
     N = cu.numel() - 1
     init = inp.initial_state.to(DEV).clone() if inp.initial_state is not None else None
     o = torch.full((total, H, dv), float("nan"), dtype=out_dtype, device=DEV)
@@ -27,20 +27,20 @@ def run_prefill(inp, algo, chunk=64, out_dtype=torch.float32, with_final=True, a
     if with_final:
         fin = init if (alias and init is not None) else torch.full((N, H, dv, dk), float("nan"), device=DEV)
     gdn.gdn_chunk_prefill(q, k, v, g, beta, cu, o, initial_state=init, final_state=fin, chunk=chunk,
-                          scale=inp.scale, algo=algo, workspace=workspace)
+                          scale=inp.scale, algo=algo, workspace=workspace, l2norm=l2norm)
     torch.cuda.synchronize()
     return o, fin
 
 
-def oracle_prefill(inp):
+def oracle_prefill(inp, l2norm=False):
     o, fin, _ = oracle.prefill(inp.q, inp.k, inp.v, inp.g, inp.beta, inp.cu_seqlens,
-                               inp.initial_state, scale=inp.scale)
+                               inp.initial_state, scale=inp.scale, l2norm=l2norm)
     return o, fin
 
 
 def check(inp, algo, chunk=64, what="", **kw):
     o, fin = run_prefill(inp, algo, chunk=chunk, **kw)
-    o_ref, f_ref = oracle_prefill(inp)
+    o_ref, f_ref = oracle_prefill(inp, l2norm=kw.get("l2norm", False))
     assert_close(o, o_ref, what=f"{what} o")
     if fin is not None:
         assert_close(fin, f_ref, what=f"{what} final state")
@@ -278,3 +278,41 @@ def test_b1_t65536_h4_full_size(algo, out_dtype):
     o, fin = run_prefill(inp, algo, out_dtype=out_dtype)
     assert_close(o, o_ref, what=f"B1 T65536 H4 o ({out_dtype})")
     assert_close(fin, f_ref, what=f"B1 T65536 H4 final state ({out_dtype})")
+
+
+# ---------------------------------------------------------------- grouped q/k heads, q/k normalisation
+
+@pytest.mark.parametrize("algo", [FUSED, TRANSFER, SEQ])
+@pytest.mark.parametrize("l2norm", [False, True])
+def test_grouped_heads_varlen(algo, l2norm):
+    """8 value heads over 2 q/k heads, lengths around the chunk size; with the
+    normalisation q and k are un-normalised N(0, 1) draws."""
+    lens = [1, 0, 63, 64, 65, 130, 200, 7]
+    inp = inputs.prefill_inputs(lens, 8, 128, 128, seed=51, g_range=(0.0, 0.05), H_qk=2,
+                                normalize_qk=not l2norm)
+    check(inp, algo, what=f"GVA algo={algo} l2={l2norm}", l2norm=l2norm)
+
+
+@pytest.mark.parametrize("in_dtype", [torch.bfloat16, torch.float32])
+def test_l2norm_fused_input_dtypes(in_dtype):
+    inp = inputs.prefill_inputs([300, 65], 4, 128, 128, seed=52, dtype=in_dtype, g_range=(0.0, 0.05),
+                                H_qk=4, normalize_qk=False)
+    check(inp, FUSED, what=f"l2 fused {in_dtype}", l2norm=True)
+
+
+def test_grouped_heads_hv32_hqk8_l2norm():
+    """32 value heads over 8 q/k heads with the normalisation, a few sequences of
+    several chunks (fused and transfer)."""
+    inp = inputs.prefill_inputs([1000, 333, 64], 32, 128, 128, seed=53, H_qk=8, normalize_qk=False)
+    check(inp, FUSED, what="GVA Hv32 Hqk8 fused", l2norm=True)
+    check(inp, TRANSFER, what="GVA Hv32 Hqk8 transfer", l2norm=True)
+
+
+def test_l2norm_neighbour_cannot_leak():
+    """With the normalisation the partial chunk's padded rows are zeroed before the
+    norms are taken: a NaN neighbour leaves the sequence bitwise unchanged."""
+    lens = [100, 37]
+    inp = inputs.prefill_inputs(lens, 2, 128, 128, seed=54, normalize_qk=False)
+    o_ref, f_ref = run_prefill(inp, FUSED, l2norm=True)
+    o, fin = run_prefill(_poisoned(inp, 1, float("nan")), FUSED, l2norm=True)
+    assert torch.equal(o[:100], o_ref[:100]) and torch.equal(fin[0], f_ref[0])

@@ -75,6 +75,6 @@ def test_static_scratch_rejects_shapes_beyond_its_size():
     need = gdn.gdn_chunk_prefill_workspace_size(N, total, H, 128, 128, 64, gdn.GDN_PREFILL_TRANSFER)
     assert need > STATIC_SCRATCH_BYTES
     st = L.gdn_chunk_prefill_static_scratch(fake, fake, fake, fake, fake, fake, N, total, None, None, fake,
-                                            H, 128, 128, 64, 0.1, gdn.GDN_BF16, gdn.GDN_BF16, None)
+                                            H, H, 128, 128, 64, 0.1, 0, gdn.GDN_BF16, gdn.GDN_BF16, None)
     assert st == gdn.GDN_ERR_WORKSPACE
     assert "static scratch" in gdn.gdn_last_error()
