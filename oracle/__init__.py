@@ -55,7 +55,7 @@ def _declare(lib):
     lib.gdn_oracle_decode.argtypes = [dp, dp, dp, dp, dp, dp, ctypes.c_int,
                                       ctypes.POINTER(ctypes.c_int32), dp,
                                       ctypes.c_int, ctypes.c_int, ctypes.c_int, ctypes.c_int, ctypes.c_int,
-                                      ctypes.c_int, ctypes.c_int, ctypes.c_double, ctypes.c_int, ctypes.c_int]
+                                      ctypes.c_int, ctypes.c_int, ctypes.c_double, ctypes.c_int, dp, ctypes.c_int]
 
 
 def _load():
@@ -118,13 +118,15 @@ def prefill(q, k, v, g, beta, cu_seqlens, initial_state=None, scale=None, nthrea
 
 
 def decode(q, k, v, g, beta, pool, slot_ids, scale=None, nthreads=0, lib=None, copy_pool=True,
-           l2norm=False):
+           l2norm=False, token_states=False):
     """Sequential fp64 decode over a slot-indexed pool (the pool copy is updated).
 
     q: [B, T, H_qk, dk]; k: [B, T, H_qk, nh, dk]; v: [B, T, H, nh, dv]; g: [B, T, H];
     beta: [B, T, H, nh]; pool: [num_slots, H, dv, dk]; slot_ids: [B].
     Returns (o [B, T, H, dv], new_pool, threads_used), fp64. With copy_pool=False an
-    fp64 C-contiguous numpy pool is updated in place (no copy).
+    fp64 C-contiguous numpy pool is updated in place (no copy). With token_states=True
+    returns (o, new_pool, threads_used, states [B, T, H, dv, dk]): the state after
+    each token (the rollback points of a speculative verification).
     """
     lib = lib or _load()
     q, k, v, g, beta = (f64(a) for a in (q, k, v, g, beta))
@@ -137,9 +139,13 @@ def decode(q, k, v, g, beta, pool, slot_ids, scale=None, nthreads=0, lib=None, c
     if scale is None:
         scale = 1.0 / np.sqrt(dk)
     o = np.zeros((B, T, H, dv), np.float64)
+    ts = np.zeros((B, T, H, dv, dk), np.float64) if token_states else None
     rc = lib.gdn_oracle_decode(_ptr(q), _ptr(k), _ptr(v), _ptr(g), _ptr(beta), _ptr(pool),
                                pool.shape[0], _ptr(slots, ctypes.c_int32), _ptr(o),
-                               B, T, H, Hqk, dk, dv, nh, float(scale), int(bool(l2norm)), int(nthreads))
+                               B, T, H, Hqk, dk, dv, nh, float(scale), int(bool(l2norm)), _ptr(ts),
+                               int(nthreads))
     if rc < 0:
         raise ValueError("gdn_oracle_decode: bad arguments")
+    if token_states:
+        return o, pool, rc, ts
     return o, pool, rc

@@ -200,6 +200,7 @@ typedef struct {
   double* o;
   int T, H, Hqk, dk, dv, nh, l2norm;
   double scale;
+  double* token_states; /* [B, T, H, dv, dk] or NULL */
 } decode_ctx;
 
 static void decode_item(void* vctx, int item) {
@@ -209,8 +210,12 @@ static void decode_item(void* vctx, int item) {
   const int hq = h / (H / Hqk); /* the value head's query/key head */
   const int slot = c->slot_ids[b];
   if (slot < 0 || slot >= c->num_slots) {
-    for (int t = 0; t < T; ++t)
+    for (int t = 0; t < T; ++t) {
       memset(c->o + (((size_t)b * T + t) * H + h) * dv, 0, (size_t)dv * sizeof(double));
+      if (c->token_states)
+        memset(c->token_states + (((size_t)b * T + t) * H + h) * (size_t)dk * dv, 0,
+               (size_t)dk * dv * sizeof(double));
+    }
     return;
   }
   double* St = c->pool + ((size_t)slot * H + h) * (size_t)dk * dv;
@@ -225,6 +230,8 @@ static void decode_item(void* vctx, int item) {
       apply_householder(St, kt, c->v + km * dv, c->beta[km], dk, dv);
     }
     emit_output(St, maybe_unit(c->q + btq * dk, dk, c->l2norm, buf + dk), c->scale, c->o + bth * dv, dk, dv);
+    if (c->token_states) /* the state after token t (speculative-verify rollback point) */
+      memcpy(c->token_states + bth * (size_t)dk * dv, St, (size_t)dk * dv * sizeof(double));
   }
   free(buf);
 }
@@ -234,16 +241,19 @@ static void decode_item(void* vctx, int item) {
  * beta: [B, T, H, nh]; pool: [num_slots, H, dv, dk], updated in place for the
  * slots named by slot_ids[B] (a negative or out-of-range id leaves the pool
  * untouched and writes zeros to that row of o); o: [B, T, H, dv]. H must be a
- * multiple of Hqk; l2norm != 0 normalises q and every k per token.
+ * multiple of Hqk; l2norm != 0 normalises q and every k per token. token_states
+ * [B, T, H, dv, dk] (or NULL) receives the state after each token (zeros for a
+ * skipped row).
  * Returns the number of threads used, or a negative value on bad arguments.
  */
 int gdn_oracle_decode(const double* q, const double* k, const double* v, const double* g,
                       const double* beta, double* pool, int num_slots, const int32_t* slot_ids,
                       double* o, int B, int T, int H, int Hqk, int dk, int dv, int nh, double scale,
-                      int l2norm, int nthreads) {
+                      int l2norm, double* token_states, int nthreads) {
   if (B < 0 || T <= 0 || H <= 0 || Hqk <= 0 || H % Hqk != 0 || dk <= 0 || dv <= 0 || nh <= 0 ||
       num_slots < 0)
     return -1;
-  decode_ctx c = {q, k, v, g, beta, pool, num_slots, slot_ids, o, T, H, Hqk, dk, dv, nh, l2norm, scale};
+  decode_ctx c = {q, k, v, g, beta, pool, num_slots, slot_ids, o, T, H, Hqk, dk, dv, nh, l2norm, scale,
+                  token_states};
   return run_items(B * H, nthreads, decode_item, &c);
 }

@@ -58,6 +58,15 @@ MUTANTS = {
     # the q/k normalisation applied to the query only
     "l2norm_query_only": [("const double* kt = maybe_unit(c->k + tq * dk, dk, c->l2norm, buf);",
                            "const double* kt = c->k + tq * dk;")],
+    # the per-token state recorded before the token's update instead of after it
+    "token_state_before_update": [(
+        "    if (c->token_states) /* the state after token t (speculative-verify rollback point) */\n"
+        "      memcpy(c->token_states + bth * (size_t)dk * dv, St, (size_t)dk * dv * sizeof(double));\n",
+        ""), (
+        "    apply_gate(St, exp(c->g[bth]), dk, dv);\n    for (int m = 0; m < nh; ++m) {\n",
+        "    if (c->token_states)\n"
+        "      memcpy(c->token_states + bth * (size_t)dk * dv, St, (size_t)dk * dv * sizeof(double));\n"
+        "    apply_gate(St, exp(c->g[bth]), dk, dv);\n    for (int m = 0; m < nh; ++m) {\n")],
     # the normalisation divides by the squared norm
     "l2norm_squared": [("const double inv = ss > 0.0 ? 1.0 / sqrt(ss) : 0.0;",
                         "const double inv = ss > 0.0 ? 1.0 / ss : 0.0;")],

@@ -543,4 +543,42 @@ def test_oracle_rejects_head_counts_that_do_not_divide():
         oracle.prefill(q, q, v, np.zeros((3, 3)), np.ones((3, 3)), [0, 3])
 
 
+# ---------------------------------------------------------------- per-token states (speculative verify)
+
+def check_token_states_are_prefix_decodes(lib=None):
+    """The state recorded after token t equals the pool state left by a decode of
+    the first t + 1 tokens alone (bitwise: the same arithmetic), the last one equals
+    the final pool state, and restoring the state after token t and decoding the
+    remaining tokens reproduces the full step (the rollback use)."""
+    rng = _rng(34)
+    B, T, H, nh, dk, dv, slots = 3, 4, 2, 2, 4, 3, 5
+    q = _unit(rng.standard_normal((B, T, H, dk)))
+    k = _unit(rng.standard_normal((B, T, H, nh, dk)))
+    v = rng.standard_normal((B, T, H, nh, dv))
+    beta = 1 / (1 + np.exp(-rng.standard_normal((B, T, H, nh))))
+    g = -rng.uniform(0.0, 0.4, (B, T, H))
+    pool = 0.1 * rng.standard_normal((slots, H, dv, dk))
+    sid = np.array([4, -1, 1], np.int32)
+    o, fin, _, ts = _decode(lib)(q, k, v, g, beta, pool, sid, scale=0.6, token_states=True)
+    for b in (0, 2):
+        assert np.array_equal(ts[b, T - 1], fin[sid[b]])
+    assert not ts[1].any()
+    for t in range(T):
+        _, pre, _ = _decode(lib)(q[:, :t + 1], k[:, :t + 1], v[:, :t + 1], g[:, :t + 1], beta[:, :t + 1],
+                                 pool, sid, scale=0.6)
+        for b in (0, 2):
+            assert np.array_equal(ts[b, t], pre[sid[b]])
+    t = 1
+    rolled = pool.copy()
+    for b in (0, 2):
+        rolled[sid[b]] = ts[b, t]
+    o2, fin2, _ = _decode(lib)(q[:, t + 1:], k[:, t + 1:], v[:, t + 1:], g[:, t + 1:], beta[:, t + 1:],
+                               rolled, sid, scale=0.6)
+    assert _relerr(o2[[0, 2]], o[[0, 2], t + 1:]) < 1e-14 and _relerr(fin2, fin) < 1e-14
+
+
+def test_token_states_are_prefix_decodes():
+    check_token_states_are_prefix_decodes()
+
+
 PIN_CHECKS.extend(v for k, v in sorted(globals().items()) if k.startswith("check_"))
