@@ -366,7 +366,7 @@ def bench_decode(key, steps, warmup, ws, rank, peaks, e2e=True):
     res["roofline"] = {"bound": "hbm", "achieved": achieved, "peak": peak, "unit": "GB/s",
                        "frac": achieved / peak,
                        "traffic": ncu_traffic(("gdn_decode_multi_kernel" if key == "gdp" else "gdn_decode_kernel")
-                                              + f":{key}", ["gated_delta_rule_58_b200/csrc/decode.cu"])}
+                                              + f":{key}", ["gated_delta_rule_58_b200/csrc/decode_impl.cuh"])}
     res["pct_of_8tbs_state"] = res["state_gbs"] / ws / NOMINAL_HBM_GBS * 100
     return res
 

@@ -70,6 +70,9 @@ def lib() -> ctypes.CDLL:
             u32 = ctypes.c_uint32
             L.gdn_decode.argtypes = [vp, vp, vp, vp, vp, vp, i32, vp, vp, i32, i32, i32, i32, i32, i32, i32,
                                      f32, u32, i32, i32, vp]
+            L.gdn_decode_mtp.restype = i32
+            L.gdn_decode_mtp.argtypes = [vp, vp, vp, vp, vp, vp, i32, vp, vp, vp, i32, i32, i32, i32, i32, i32,
+                                         i32, f32, u32, i32, i32, i32, vp]
             L.gdn_chunk_prefill_workspace_size.restype = sz
             L.gdn_chunk_prefill_workspace_size.argtypes = [i32, i64, i32, i32, i32, i32, i32]
             L.gdn_chunk_prefill.restype = i32
@@ -149,6 +152,23 @@ def gdn_decode(q, k, v, g, beta, state_pool, slot_ids, o, scale=None, stream=Non
                           state_pool.shape[0], _ptr(slot_ids), _ptr(o), B, T, H, H_qk, dk, dv, n_h,
                           float(scale), GDN_QK_L2NORM if l2norm else 0, _dtype_code(q), _dtype_code(o),
                           _stream_ptr(stream, q.device))
+    _check(st)
+    return o
+
+
+def gdn_decode_mtp(q, k, v, g, beta, state_pool, slot_ids, o, token_states, update_pool=True, scale=None,
+                   stream=None, l2norm=False):
+    """gdn_decode that also writes the state after every token into token_states
+    [B,T,H,dv,dk] fp32 (the rollback points of a speculative verification); with
+    update_pool=False the pool is only read. Other shapes as gdn_decode."""
+    B, T, H_qk, dk = q.shape
+    H, n_h, dv = v.shape[2], k.shape[3], v.shape[4]
+    if scale is None:
+        scale = dk ** -0.5
+    st = lib().gdn_decode_mtp(_ptr(q), _ptr(k), _ptr(v), _ptr(g), _ptr(beta), _ptr(state_pool),
+                              state_pool.shape[0], _ptr(slot_ids), _ptr(o), _ptr(token_states), B, T, H, H_qk,
+                              dk, dv, n_h, float(scale), GDN_QK_L2NORM if l2norm else 0, 1 if update_pool else 0,
+                              _dtype_code(q), _dtype_code(o), _stream_ptr(stream, q.device))
     _check(st)
     return o
 

@@ -57,8 +57,8 @@ gdn_status_t device_error_word(unsigned int** word) {
 gdn_status_t decode_launch(const void* q, const void* k, const void* v, const float* g,
                            const float* beta, float* pool, int num_slots, const int32_t* slot_ids,
                            void* o, int B, int T, int H, int Hqk, int dk, int dv, int nh, float scale,
-                           uint32_t flags, gdn_dtype_t in, gdn_dtype_t out, unsigned int* err,
-                           cudaStream_t stream);
+                           uint32_t flags, float* token_states, int update_pool, gdn_dtype_t in,
+                           gdn_dtype_t out, unsigned int* err, cudaStream_t stream);
 
 }  // namespace gdn
 
@@ -104,16 +104,17 @@ gdn_status_t gdn_get_device_error(uint32_t* flags) {
   return gdn::ok();
 }
 
-gdn_status_t gdn_decode(const void* q, const void* k, const void* v, const float* g,
-                        const float* beta, float* state_pool, int num_slots,
-                        const int32_t* slot_ids, void* o, int B, int T, int H, int H_qk,
-                        int dk, int dv, int n_h, float scale, uint32_t flags,
-                        gdn_dtype_t in_dtype, gdn_dtype_t out_dtype, void* stream) {
+gdn_status_t gdn_decode_mtp(const void* q, const void* k, const void* v, const float* g,
+                            const float* beta, float* state_pool, int num_slots,
+                            const int32_t* slot_ids, void* o, float* token_states, int B, int T, int H,
+                            int H_qk, int dk, int dv, int n_h, float scale, uint32_t flags, int update_pool,
+                            gdn_dtype_t in_dtype, gdn_dtype_t out_dtype, void* stream) {
   GDN_REQUIRE(B >= 0 && T >= 1 && H >= 1 && n_h >= 1 && num_slots >= 0, GDN_ERR_INVALID_ARG,
               "gdn_decode: need B >= 0, T >= 1, H >= 1, n_h >= 1, num_slots >= 0");
   GDN_REQUIRE(H_qk >= 1 && H % H_qk == 0, GDN_ERR_INVALID_ARG,
               "gdn_decode: H_qk must be >= 1 and divide H");
   GDN_REQUIRE((flags & ~GDN_QK_L2NORM) == 0, GDN_ERR_INVALID_ARG, "gdn_decode: unknown flags");
+  GDN_REQUIRE(update_pool == 0 || update_pool == 1, GDN_ERR_INVALID_ARG, "gdn_decode_mtp: update_pool must be 0 or 1");
   GDN_REQUIRE(valid_dtype(in_dtype) && valid_dtype(out_dtype), GDN_ERR_INVALID_ARG,
               "gdn_decode: unknown dtype");
   GDN_REQUIRE(dk == dv, GDN_ERR_UNSUPPORTED, "gdn_decode: dk must equal dv");
@@ -127,13 +128,24 @@ gdn_status_t gdn_decode(const void* q, const void* k, const void* v, const float
   GDN_REQUIRE(slot_ids != nullptr, GDN_ERR_INVALID_ARG, "gdn_decode: slot_ids is NULL");
   GDN_REQUIRE_PTR(state_pool, "gdn_decode: state_pool");
   GDN_REQUIRE(o != nullptr, GDN_ERR_INVALID_ARG, "gdn_decode: o is NULL");
+  if (token_states) GDN_REQUIRE_PTR(token_states, "gdn_decode_mtp: token_states");
   GDN_REQUIRE((long long)B * H * ((dv + 63) / 64) < (1LL << 31), GDN_ERR_UNSUPPORTED,
               "gdn_decode: B * H too large for one launch");
   unsigned int* err = nullptr;
   gdn_status_t st = gdn::device_error_word(&err);
   if (st != GDN_OK) return st;
   return gdn::decode_launch(q, k, v, g, beta, state_pool, num_slots, slot_ids, o, B, T, H, H_qk, dk, dv,
-                            n_h, scale, flags, in_dtype, out_dtype, err, gdn::as_stream(stream));
+                            n_h, scale, flags, token_states, update_pool, in_dtype, out_dtype, err,
+                            gdn::as_stream(stream));
+}
+
+gdn_status_t gdn_decode(const void* q, const void* k, const void* v, const float* g,
+                        const float* beta, float* state_pool, int num_slots,
+                        const int32_t* slot_ids, void* o, int B, int T, int H, int H_qk,
+                        int dk, int dv, int n_h, float scale, uint32_t flags,
+                        gdn_dtype_t in_dtype, gdn_dtype_t out_dtype, void* stream) {
+  return gdn_decode_mtp(q, k, v, g, beta, state_pool, num_slots, slot_ids, o, nullptr, B, T, H, H_qk, dk, dv,
+                        n_h, scale, flags, 1, in_dtype, out_dtype, stream);
 }
 
 size_t gdn_chunk_prefill_workspace_size(int N, int64_t total_T, int H, int dk, int dv, int chunk,

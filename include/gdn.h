@@ -105,6 +105,30 @@ gdn_status_t gdn_decode(const void* q, const void* k, const void* v, const float
                         int dk, int dv, int n_h, float scale, uint32_t flags,
                         gdn_dtype_t in_dtype, gdn_dtype_t out_dtype, void* stream);
 
+/*
+ * gdn_decode_mtp — gdn_decode that also records the state after every token, for
+ * speculative (multi-token prediction) verification: the T tokens of a step are
+ * draft tokens, and once the caller knows how many were accepted it restores the
+ * state after the last accepted one (a rollback). The kernel family on the
+ * FlashInfer PR #7156 page (introduction) carries "mtp" in its name; recording the
+ * per-token states is the reading adopted here.
+ *
+ *   token_states [B, T, H, dv, dk] fp32, K-last, or NULL: the state of (b, h) after
+ *                token t (after its gate and all n_h Householder updates). Rows of a
+ *                skipped batch row (slot id < 0 or >= num_slots) are written as zeros.
+ *   update_pool  1: the final state is written back to the pool slot (as gdn_decode);
+ *                0: the pool is only read (verification without committing).
+ *
+ * Everything else, including validation, is as gdn_decode, which is this call with
+ * token_states = NULL and update_pool = 1. The per-token states add T * dk * dv * 4
+ * bytes of writes per (batch row, head).
+ */
+gdn_status_t gdn_decode_mtp(const void* q, const void* k, const void* v, const float* g,
+                            const float* beta, float* state_pool, int num_slots,
+                            const int32_t* slot_ids, void* o, float* token_states, int B, int T, int H,
+                            int H_qk, int dk, int dv, int n_h, float scale, uint32_t flags, int update_pool,
+                            gdn_dtype_t in_dtype, gdn_dtype_t out_dtype, void* stream);
+
 /* Prefill algorithm selection (gdn_chunk_prefill / gdn_chunk_prefill_workspace_size). */
 typedef enum {
   GDN_PREFILL_AUTO = 0,       /* library picks from (N, H, total_T, dims) */

@@ -219,3 +219,68 @@ def test_l2norm_of_normalised_inputs_changes_little():
     o1, p1 = _run(inp, out_dtype=torch.float32)
     o2, p2 = _run(inp, out_dtype=torch.float32, l2norm=True)
     assert_close(o2, o1, tol=5e-3, what="l2norm on unit inputs")
+
+
+# ---------------------------------------------------------------- per-token states (speculative verify)
+
+def _run_mtp(inp, update_pool, out_dtype=torch.float32, l2norm=False):
+    pool = inp.pool.to(DEV).clone()
+    q, k, v = inp.q.to(DEV), inp.k.to(DEV), inp.v.to(DEV)
+    B, T, H = v.shape[:3]
+    dk = q.shape[-1]
+    o = torch.empty((B, T, H, v.shape[-1]), dtype=out_dtype, device=DEV)
+    ts = torch.full((B, T, H, v.shape[-1], dk), float("nan"), device=DEV)
+    gdn.gdn_decode_mtp(q, k, v, inp.g.to(DEV), inp.beta.to(DEV), pool, inp.slot_ids.to(DEV), o, ts,
+                       update_pool=update_pool, scale=inp.scale, l2norm=l2norm)
+    torch.cuda.synchronize()
+    return o, pool, ts
+
+
+@pytest.mark.parametrize("T,nh", [(4, 2), (2, 1), (1, 1), (8, 1), (1, 4)])
+@pytest.mark.parametrize("update_pool", [True, False])
+def test_mtp_token_states_against_oracle(T, nh, update_pool):
+    """The state after every token (and the outputs) against the oracle; a skipped
+    batch row gets zero states; with update_pool=False the pool is bitwise untouched."""
+    inp = inputs.decode_inputs(6, T, 4, 128, 128, nh, 9, seed=60 + T + nh)
+    inp.slot_ids[2] = -1
+    o, pool, ts = _run_mtp(inp, update_pool)
+    o_ref, pool_ref, _, ts_ref = oracle.decode(inp.q, inp.k, inp.v, inp.g, inp.beta, inp.pool, inp.slot_ids,
+                                               scale=inp.scale, token_states=True)
+    assert_close(o, o_ref, what=f"mtp T={T} nh={nh} o")
+    assert_close(ts, ts_ref, what=f"mtp T={T} nh={nh} token states")
+    assert torch.all(ts[2] == 0)
+    used = sorted(int(x) for x in inp.slot_ids.tolist() if x >= 0)
+    if update_pool:
+        assert_close(pool[used], pool_ref[used], what=f"mtp T={T} nh={nh} pool")
+        assert torch.equal(ts[[b for b in range(6) if b != 2], T - 1].cpu(),
+                           pool[[int(inp.slot_ids[b]) for b in range(6) if b != 2]].cpu())
+    else:
+        assert torch.equal(pool.cpu(), inp.pool)
+
+
+def test_mtp_rollback_round_trip():
+    """Verify 4 draft tokens without committing, accept 2: restoring the state after
+    token 1 and decoding tokens 2-3 gives the full step's outputs and final state."""
+    inp = inputs.decode_inputs(16, 4, 8, 128, 128, 2, 20, seed=64, g_range=(0.0, 0.05))
+    o_full, pool_full = _run(inp, out_dtype=torch.float32)
+    o, pool, ts = _run_mtp(inp, update_pool=False)
+    assert_close(o, o_full, tol=1e-6, what="mtp outputs vs decode")
+    rolled = pool.clone()
+    slots = inp.slot_ids.long().to(DEV)
+    rolled[slots] = ts[:, 1]
+    rest = inputs.DecodeInputs(inp.q[:, 2:].contiguous(), inp.k[:, 2:].contiguous(), inp.v[:, 2:].contiguous(),
+                               inp.g[:, 2:].contiguous(), inp.beta[:, 2:].contiguous(), rolled.cpu(),
+                               inp.slot_ids, inp.scale)
+    o2, pool2 = _run(rest, out_dtype=torch.float32)
+    assert_close(o2, o_full[:, 2:], tol=1e-5, what="rollback outputs")
+    assert_close(pool2[slots], pool_full[slots], tol=1e-5, what="rollback final state")
+
+
+def test_mtp_split_v_grouped_l2norm():
+    """T=1 with few heads (split along V), grouped q/k heads and the normalisation."""
+    inp = inputs.decode_inputs(2, 1, 4, 128, 128, 1, 5, seed=65, H_qk=2, normalize_qk=False)
+    o, pool, ts = _run_mtp(inp, update_pool=True, l2norm=True)
+    o_ref, pool_ref, _, ts_ref = oracle.decode(inp.q, inp.k, inp.v, inp.g, inp.beta, inp.pool, inp.slot_ids,
+                                               scale=inp.scale, token_states=True, l2norm=True)
+    assert_close(o, o_ref, what="mtp split-V o")
+    assert_close(ts, ts_ref, what="mtp split-V token states")
