@@ -12,6 +12,6 @@ from ._lib import (  # noqa: F401
     GDN_PREFILL_SEQUENTIAL, GDN_PREFILL_TRANSFER, GDN_QK_L2NORM, GdnError, declared_functions,
     gdn_chunk_prefill, gdn_chunk_prefill_static_scratch, gdn_chunk_prefill_workspace_size, gdn_decode,
     gdn_decode_mtp,
-    gdn_get_device_error,
+    gdn_get_device_error, gdn_selftest_wait_timeout,
     gdn_last_error, gdn_version, lib,
 )

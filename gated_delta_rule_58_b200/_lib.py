@@ -85,6 +85,8 @@ def lib() -> ctypes.CDLL:
             L.gdn_last_error.argtypes = []
             L.gdn_get_device_error.restype = i32
             L.gdn_get_device_error.argtypes = [ctypes.POINTER(ctypes.c_uint32)]
+            L.gdn_selftest_wait_timeout.restype = i32
+            L.gdn_selftest_wait_timeout.argtypes = [u32, vp]
             L.gdn_version.restype = ctypes.c_char_p
             L.gdn_version.argtypes = []
             _lib = L
@@ -111,6 +113,12 @@ def gdn_get_device_error() -> int:
     if st not in (GDN_OK, GDN_ERR_DEVICE_DATA):
         _check(st)
     return int(flags.value)
+
+
+def gdn_selftest_wait_timeout(wait_us: int, stream=None):
+    """Enqueue the bounded-wait self-test kernel (see include/gdn.h); afterwards
+    gdn_get_device_error() reports GDN_DEVERR_TIMEOUT."""
+    _check(lib().gdn_selftest_wait_timeout(int(wait_us), stream))
 
 
 # ---------------------------------------------------------------- torch marshalling

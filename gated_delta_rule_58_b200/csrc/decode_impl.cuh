@@ -139,6 +139,9 @@ __device__ __forceinline__ void decode_producer(const DecodeParams& p, const CUt
     tc::bulk_commit();
   };
   int it = 0;
+  int last_fill[NS];  // per stage: the last item filled into it (-1: none)
+#pragma unroll
+  for (int x = 0; x < NS; ++x) last_fill[x] = -1;
   for (int item = blockIdx.x; item < p.n_items; item += gridDim.x, ++it) {
     const int s = it % NS;
     // the item's scalars are loaded before the stage wait, which hides their latency
@@ -155,8 +158,9 @@ __device__ __forceinline__ void decode_producer(const DecodeParams& p, const CUt
     }
     if (it >= NS && !tc::mbar_wait(&empty[s], ((it / NS) & 1) ^ 1, kDecodeWaitNs)) {
       raise_device_error(p.err, GDN_DEVERR_TIMEOUT);
-      return;
+      break;
     }
+    last_fill[s] = it;
     uint8_t* st = base + s * L::kBytes;
     if constexpr (kStores) {
       if (it >= NS) {
@@ -209,6 +213,12 @@ __device__ __forceinline__ void decode_producer(const DecodeParams& p, const CUt
     }
     tc::bulk_wait_all();
   }
+  // Every fill has landed before the CTA exits: after a timeout some were never
+  // consumed. A stage is only refilled after its previous fill was consumed, so
+  // waiting for each stage's last fill covers all of them (immediate when consumed).
+#pragma unroll
+  for (int x = 0; x < NS; ++x)
+    if (last_fill[x] >= 0) tc::mbar_wait(&full[x], (last_fill[x] / NS) & 1, kDecodeWaitNs);
 }
 
 // Single-token step (T = n_h = 1): 2 threads per state row, all consumers on one item.

@@ -6,6 +6,7 @@
 
 #include "common.cuh"
 #include "prefill.cuh"
+#include "tcgen05.cuh"
 
 namespace gdn {
 
@@ -60,6 +61,23 @@ gdn_status_t decode_launch(const void* q, const void* k, const void* v, const fl
                            uint32_t flags, float* token_states, int update_pool, gdn_dtype_t in,
                            gdn_dtype_t out, unsigned int* err, cudaStream_t stream);
 
+namespace {
+
+// One thread waits, with the kernels' bounded wait, for a phase of a shared-memory
+// mbarrier that nothing completes, then reports the timeout the way every kernel
+// of the library does. No copies or tensor-memory allocations are in flight, so
+// the kernel simply returns.
+__global__ void gdn_selftest_timeout_kernel(unsigned int* err, uint64_t wait_ns) {
+  __shared__ __align__(8) uint64_t bar;
+  if (threadIdx.x == 0) {
+    tc::mbar_init(&bar, 1);
+    tc::fence_mbar_init();
+  }
+  __syncthreads();
+  if (threadIdx.x == 0 && !tc::mbar_wait(&bar, 0, wait_ns)) raise_device_error(err, GDN_DEVERR_TIMEOUT);
+}
+
+}  // namespace
 }  // namespace gdn
 
 using gdn::fail;
@@ -146,6 +164,16 @@ gdn_status_t gdn_decode(const void* q, const void* k, const void* v, const float
                         gdn_dtype_t in_dtype, gdn_dtype_t out_dtype, void* stream) {
   return gdn_decode_mtp(q, k, v, g, beta, state_pool, num_slots, slot_ids, o, nullptr, B, T, H, H_qk, dk, dv,
                         n_h, scale, flags, 1, in_dtype, out_dtype, stream);
+}
+
+gdn_status_t gdn_selftest_wait_timeout(uint32_t wait_us, void* stream) {
+  GDN_REQUIRE(wait_us >= 1 && wait_us <= 10000000u, GDN_ERR_INVALID_ARG,
+              "gdn_selftest_wait_timeout: wait_us must be in [1, 10^7]");
+  unsigned int* err = nullptr;
+  gdn_status_t st = gdn::device_error_word(&err);
+  if (st != GDN_OK) return st;
+  gdn::gdn_selftest_timeout_kernel<<<1, 32, 0, gdn::as_stream(stream)>>>(err, (uint64_t)wait_us * 1000u);
+  return gdn::check_launch("gdn_selftest_wait_timeout");
 }
 
 size_t gdn_chunk_prefill_workspace_size(int N, int64_t total_T, int H, int dk, int dv, int chunk,

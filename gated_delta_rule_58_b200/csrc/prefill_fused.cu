@@ -111,6 +111,8 @@ enum Bar : int {
   B_E5,                // state: U16/UDD ready, U region consumed
   B_E6A,               // state: S16 ready, TMEM state rescaled
   B_E6B,               // state: O1/O2 consumed
+  B_FREE0, B_FREE1,    // state: a tile buffer's last reader (the state update) is done (fp32 inputs)
+  B_DRAIN_M, B_DRAIN_L,  // abort path: the MMA thread's / the loader's MMAs have completed
   B_COUNT
 };
 
@@ -142,6 +144,14 @@ struct Smem {
   __device__ uint32_t* tmem_slot() const { return reinterpret_cast<uint32_t*>(base + OFF_BAR + 8 * B_COUNT); }
   __device__ volatile int* abort_flag() const {
     return reinterpret_cast<volatile int*>(base + OFF_BAR + 8 * B_COUNT + 4);
+  }
+  // per tile buffer: copies issued into it, and copies whose landing the loader saw
+  // (an aborting CTA waits for the difference before it exits)
+  __device__ volatile uint32_t* loads_issued() const {
+    return reinterpret_cast<volatile uint32_t*>(base + OFF_BAR + 8 * B_COUNT + 8);
+  }
+  __device__ volatile uint32_t* loads_landed() const {
+    return reinterpret_cast<volatile uint32_t*>(base + OFF_BAR + 8 * B_COUNT + 16);
   }
   __device__ uint32_t u32(uint32_t off) const { return tc::smem_u32(base + off); }
 };
@@ -191,6 +201,7 @@ __device__ __forceinline__ void issue_tile_loads(const Smem& sm, const QkvMaps& 
   uint8_t* kq = sm.base + OFF_KQ + b * KQ_BUF;
   uint8_t* v16 = sm.base + OFF_V + b * V_BUF;
   tc::fence_proxy_async_smem();  // the previous generic writes of these tiles precede the copies
+  sm.loads_issued()[b] = sm.loads_issued()[b] + 1;
   tc::mbar_arrive_expect_tx(sm.bar(B_T0 + b), (zero_values ? 2u : 3u) * 16384u);
 #pragma unroll
   for (int hf = 0; hf < 2; ++hf) {
@@ -282,8 +293,11 @@ __device__ void loader_role(const Smem& sm, const PrefillShape& s, const Prefill
       // they are zeroed once the copies have landed, and their beta and g are 0
       if (c < 2 && t == 0) issue_tile_loads(sm, maps, b, h, hq, t0, zero_values);
       if (!wait_bar(sm, B_T0 + b, (c >> 1) & 1, a.err)) return;
+      if (t == 0) sm.loads_landed()[b] = sm.loads_landed()[b] + 1;
     } else {
-      if (c >= 2 && !wait_bar(sm, B_M4B, (c - 2) & 1, a.err)) return;
+      // the buffer's release barrier completes once per use of the buffer, so its
+      // parity names the use (chunk c-2) without depending on timing
+      if (c >= 2 && !wait_bar(sm, B_FREE0 + b, ((c - 2) >> 1) & 1, a.err)) return;
     }
     if (t < C) {
       vec[V_G + t] = gv;
@@ -783,8 +797,13 @@ __device__ void state_role(const Smem& sm, const PrefillShape& s, const PrefillA
     tc::fence_after_sync();
     // chunk c's state update was the last reader of tile buffer b: chunk c+2's
     // copies go out now, well before the loader needs them
-    if (kTmaLoads && j == 0 && c + 2 < nchunks)
-      issue_tile_loads(sm, maps, b, h, h / (s.H / s.Hqk), t0 + 2 * C, a.mode == kPrefillTransfer);
+    if (j == 0) {
+      if (kTmaLoads) {
+        if (c + 2 < nchunks) issue_tile_loads(sm, maps, b, h, h / (s.H / s.Hqk), t0 + 2 * C, a.mode == kPrefillTransfer);
+      } else {
+        tc::mbar_arrive(sm.bar(B_FREE0 + b));  // fp32 inputs: the loader refills the buffer itself
+      }
+    }
     const bool last = (c == nchunks - 1);
     float gnext = 1.f;
     if (!last) {
@@ -999,6 +1018,8 @@ gdn_prefill_fused_kernel(const PrefillShape s, const PrefillArgs a, const __grid
   if (threadIdx.x == 0) {
     for (int i = 0; i < B_COUNT; ++i) tc::mbar_init(sm.bar(i), i == B_E1 ? 4 : 1);
     *sm.abort_flag() = 0;
+    sm.loads_issued()[0] = sm.loads_issued()[1] = 0;
+    sm.loads_landed()[0] = sm.loads_landed()[1] = 0;
     tc::fence_mbar_init();
   }
   tc::fence_before_sync();
@@ -1016,7 +1037,27 @@ gdn_prefill_fused_kernel(const PrefillShape s, const PrefillArgs a, const __grid
     mma_role(sm, tmem, nchunks, a.err);
   }
 
-  // teardown: every role finished (all MMAs were waited on by the state role)
+  // teardown: every role finished (all MMAs were waited on by the state role).
+  // After a timeout the roles returned early, so asynchronous work they issued may
+  // still be running: each MMA issuer waits for its own MMAs (a commit arrives once
+  // every earlier MMA of the thread is done), the output stores of the state warps
+  // drain, and outstanding tile copies land, all before TMEM is released and the
+  // CTA exits (each wait bounded again).
+  if (*sm.abort_flag()) {
+    const bool mma_issuer = (warp == kMmaWarp && (threadIdx.x & 31) == 0);
+    const bool d1_issuer = (threadIdx.x == kLoadWarp0 * 32);
+    if (mma_issuer || d1_issuer) {
+      uint64_t* drain = sm.bar(mma_issuer ? B_DRAIN_M : B_DRAIN_L);
+      tc::mma_commit(drain);
+      tc::mbar_wait(drain, 0, kWaitNs);
+    }
+    if (threadIdx.x == 0) {
+      for (int b = 0; b < 2; ++b)
+        for (uint32_t n = sm.loads_landed()[b]; n < sm.loads_issued()[b]; ++n)
+          if (!tc::mbar_wait(sm.bar(B_T0 + b), n & 1, kWaitNs)) break;
+    }
+  }
+  if (warp == 0) tc::bulk_wait_all();  // the state warps' output stores (a no-op when none)
   tc::fence_before_sync();
   __syncthreads();
   tc::fence_after_sync();

@@ -225,6 +225,20 @@ const char* gdn_last_error(void);
  */
 gdn_status_t gdn_get_device_error(uint32_t* flags);
 
+/*
+ * gdn_selftest_wait_timeout — a check of the failure reporting, for tests and
+ * health checks. Every wait inside the library's kernels (on an mbarrier phase) is
+ * bounded; when one gives up the kernel sets GDN_DEVERR_TIMEOUT in the device
+ * error word and unwinds instead of hanging. This call enqueues one small kernel
+ * that performs such a bounded wait, for wait_us microseconds, on a barrier that
+ * nothing completes, so the wait always gives up: afterwards gdn_get_device_error
+ * reports GDN_DEVERR_TIMEOUT and the CUDA context remains usable. wait_us must be in
+ * [1, 10^7]; GDN_ERR_INVALID_ARG otherwise (nothing launched). The pages have no
+ * counterpart (the error conventions follow the checked errors of the FlashInfer
+ * PR #4593 page, section 1, host launcher).
+ */
+gdn_status_t gdn_selftest_wait_timeout(uint32_t wait_us, void* stream);
+
 /* Library version, e.g. "gdn 0.1.0 sm_100a". */
 const char* gdn_version(void);
 

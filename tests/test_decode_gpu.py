@@ -284,3 +284,17 @@ def test_mtp_split_v_grouped_l2norm():
                                                scale=inp.scale, token_states=True, l2norm=True)
     assert_close(o, o_ref, what="mtp split-V o")
     assert_close(ts, ts_ref, what="mtp split-V token states")
+
+
+def test_bounded_wait_gives_up_reports_timeout_and_the_context_stays_usable():
+    """A bounded in-kernel wait on a barrier that nothing completes gives up after
+    its limit, the device error word reports GDN_DEVERR_TIMEOUT (read and cleared
+    once), and later calls on the same context still give the oracle's results."""
+    gdn.gdn_get_device_error()  # clear
+    gdn.gdn_selftest_wait_timeout(2000)  # 2 ms
+    assert gdn.gdn_get_device_error() & gdn.GDN_DEVERR_TIMEOUT
+    assert gdn.gdn_get_device_error() == 0
+    inp = inputs.decode_inputs(3, 2, 2, 64, 64, 2, 5, seed=70)
+    o, pool = _run(inp, out_dtype=torch.float32)
+    _check_against_oracle(inp, o, pool, "after a timeout")
+    assert gdn.gdn_get_device_error() == 0

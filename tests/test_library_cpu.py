@@ -137,3 +137,8 @@ def test_binding_fails_loudly_without_library(monkeypatch, tmp_path):
     monkeypatch.setattr(_lib, "LIB_PATH", str(tmp_path / "missing.so"))
     with pytest.raises(RuntimeError, match="no CPU fallback"):
         _lib.lib()
+
+
+def test_selftest_wait_rejects_bad_limits_on_host(L):
+    assert L.gdn_selftest_wait_timeout(0, None) == gdn.GDN_ERR_INVALID_ARG
+    assert L.gdn_selftest_wait_timeout(10000001, None) == gdn.GDN_ERR_INVALID_ARG
