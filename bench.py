@@ -150,15 +150,17 @@ def source_sha(*rel_paths) -> str:
     return h.hexdigest()[:16]
 
 
-def ncu_traffic(kernel_key: str, sources):
-    """DRAM bytes per launch from the committed ncu summary, if the kernel source is unchanged."""
+def ncu_traffic(part_key: str):
+    """DRAM bytes (read + write) per launch of the part's dominant kernel (for the
+    transfer prefill: of all library kernels of one step) from the committed ncu
+    capture, or None when a source file it names has changed since."""
     path = os.path.join(ROOT, "profiles", "ncu_traffic.json")
     if not os.path.exists(path):
         return None
     with open(path) as f:
         d = json.load(f)
-    e = d.get(kernel_key)
-    if not e or e.get("source_sha") != source_sha(*sources):
+    e = d.get(part_key)
+    if not e or e.get("source_sha") != source_sha(*e.get("sources", [])):
         return None
     return e.get("dram_bytes_per_launch")
 
@@ -365,8 +367,7 @@ def bench_decode(key, steps, warmup, ws, rank, peaks, e2e=True):
     peak = peaks["hbm_gbs"]
     res["roofline"] = {"bound": "hbm", "achieved": achieved, "peak": peak, "unit": "GB/s",
                        "frac": achieved / peak,
-                       "traffic": ncu_traffic(("gdn_decode_multi_kernel" if key == "gdp" else "gdn_decode_kernel")
-                                              + f":{key}", ["gated_delta_rule_58_b200/csrc/decode_impl.cuh"])}
+                       "traffic": ncu_traffic(key)}
     res["pct_of_8tbs_state"] = res["state_gbs"] / ws / NOMINAL_HBM_GBS * 100
     return res
 
@@ -448,8 +449,7 @@ def bench_prefill(key, steps, warmup, ws, rank, peaks, algo=None):
                      "peak": peaks["hbm_gbs"] if bound == "hbm" else peaks["bf16_tflops"],
                      "unit": "GB/s" if bound == "hbm" else "TFLOP/s",
                      "frac": max(hbm_t, tc_t) / t,
-                     "traffic": ncu_traffic(f"gdn_prefill_fused_kernel:{key}",
-                                            ["gated_delta_rule_58_b200/csrc/prefill_fused.cu"])},
+                     "traffic": ncu_traffic(key)},
         "pct_of_nominal_roofline": max(alg_b / (NOMINAL_HBM_GBS * 1e9), flops / 2.25e15) / t * 100,
         "alg_bytes": alg_b,
         "flops": flops,
@@ -598,7 +598,8 @@ def main():
     ap.add_argument("--impl", default="ours", choices=["ours", "reference"])
     ap.add_argument("--parts", default="gdp,decode_b1,decode_b4,decode_b16,prefill,varlen,longseq,tiny",
                     help="comma list of extra workloads to measure ('none' for none)")
-    ap.add_argument("--part-steps", type=int, default=5)
+    ap.add_argument("--part-steps", type=int, default=5,
+                    help="timed steps of each prefill part (decode parts: 20 times this, at least 20)")
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--reference-seconds", type=float, default=120.0,
                     help="wall-time budget of the --impl reference run")

@@ -22,15 +22,14 @@ def test_a_code_change_changes_the_code():
 
 
 def test_committed_traffic_entries_match_the_sources():
-    """Every entry of profiles/ncu_traffic.json names a kernel whose source hashes
-    to the recorded value (else bench.py reports traffic as null)."""
+    """Every entry of profiles/ncu_traffic.json names the sources of its kernel(s),
+    which hash to the recorded value (else bench.py reports traffic as null), and a
+    committed ncu summary."""
     import json
     with open(os.path.join(ROOT, "profiles", "ncu_traffic.json")) as f:
         entries = {k: v for k, v in json.load(f).items() if not k.startswith("_")}
-    src = {"gdn_decode_kernel": "decode.cu", "gdn_decode_multi_kernel": "decode.cu",
-           "gdn_prefill_fused_kernel": "prefill_fused.cu"}
     for key, e in entries.items():
-        path = "gated_delta_rule_58_b200/csrc/" + src[key.split(":")[0]]
-        assert bench.source_sha(path) == e["source_sha"], key
-        assert bench.ncu_traffic(key, [path]) == e["dram_bytes_per_launch"]
+        assert e["sources"], key
+        assert bench.source_sha(*e["sources"]) == e["source_sha"], key
+        assert bench.ncu_traffic(key) == e["dram_bytes_per_launch"]
         assert os.path.exists(os.path.join(ROOT, "profiles", e["profile"]))
