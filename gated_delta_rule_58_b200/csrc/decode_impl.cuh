@@ -720,6 +720,11 @@ gdn_status_t launch_single_rows(DecodeParams p, cudaStream_t stream) {
     int sms = 0, per_sm = 0;
     e = cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, d);
     if (e == cudaSuccess) e = cudaFuncSetAttribute(kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, L::kSmem);
+    // the whole configurable L1/shared split to shared memory, so that several of the
+    // smaller CTAs of a split head fit on an SM (the occupancy query below, and the
+    // launches, use this carveout)
+    if (e == cudaSuccess)
+      e = cudaFuncSetAttribute(kernel, cudaFuncAttributePreferredSharedMemoryCarveout, cudaSharedmemCarveoutMaxShared);
     if (e == cudaSuccess)
       e = cudaOccupancyMaxActiveBlocksPerMultiprocessor(&per_sm, kernel, kThreadsPerCta, L::kSmem);
     *out = sms * (per_sm > 0 ? per_sm : 1);

@@ -626,44 +626,32 @@ __device__ void prep_role(const Smem& sm, uint32_t tmem, int nchunks, unsigned i
     const float* vec = sm.vec(c % 3);
     const float* G = vec + V_G;
     if (t < C) {
-      // A row t (rows 0-63 of D1): beta_t exp(G_t - G_j) k_t.k_j for j < t. Warp 5
-      // (rows 32-63) needs both 32-column halves: the second half's TMEM load is
-      // issued before the first half is processed, so its latency is hidden.
+      // A row t (rows 0-63 of D1): beta_t exp(G_t - G_j) k_t.k_j for j < t; the warp
+      // of rows 32-63 also needs the right 32-column half (warp-uniform, as tcgen05.ld
+      // is warp-collective). One half is loaded and processed at a time.
       const float Gi = G[t], bi = vec[V_BETA + t];
-      const bool two = (t | 31) > 32;  // warp-uniform (tcgen05.ld is warp-collective)
-      float x0[32], x1[32];
-      tc::tmem_ld16(tl + COL_D1, x0);
-      tc::tmem_ld16(tl + COL_D1 + 16, x0 + 16);
-      tc::wait_ld();
-      if (two) {
-        tc::tmem_ld16(tl + COL_D1 + 32, x1);
-        tc::tmem_ld16(tl + COL_D1 + 48, x1 + 16);
-      }
-      a_row_half(sm.A(), t, 0, bi, Gi, G, x0);
-      if (two) {
+      const int halves = ((t | 31) > 32) ? 2 : 1;
+      for (int hq = 0; hq < halves; ++hq) {
+        float x[32];
+        tc::tmem_ld16(tl + COL_D1 + 32 * hq, x);
+        tc::tmem_ld16(tl + COL_D1 + 32 * hq + 16, x + 16);
         tc::wait_ld();
-        a_row_half(sm.A(), t, 1, bi, Gi, G, x1);
+        a_row_half(sm.A(), t, hq, bi, Gi, G, x);
       }
     } else {
-      // P row r (rows 64-127 of D1) into P16[b]; its previous reader (chunk c-2's O2
-      // MMA) completed before this chunk's D1 MMA, whose completion was waited on.
-      // 16-byte chunks entirely above the diagonal keep the zeros written at start.
+      // P row r (rows 64-127 of D1) into P16[b]; its previous reader (chunk c-2's
+      // output MMA) completed before this chunk's D1 MMA, whose completion was waited
+      // on. 16-byte chunks entirely above the diagonal keep the zeros written at start.
       const int r = t - C;
       const float Gr = G[r];
-      const bool two = (r | 31) >= 32;  // warp 7: both halves (warp-uniform)
+      const int halves = ((r | 31) >= 32) ? 2 : 1;
       uint8_t* p16 = sm.base + OFF_P16 + b * P_BUF;
-      float x0[32], x1[32];
-      tc::tmem_ld16(tl + COL_D1, x0);
-      tc::tmem_ld16(tl + COL_D1 + 16, x0 + 16);
-      tc::wait_ld();
-      if (two) {
-        tc::tmem_ld16(tl + COL_D1 + 32, x1);
-        tc::tmem_ld16(tl + COL_D1 + 48, x1 + 16);
-      }
-      p_row_half(p16, r, 0, Gr, G, x0);
-      if (two) {
+      for (int hq = 0; hq < halves; ++hq) {
+        float x[32];
+        tc::tmem_ld16(tl + COL_D1 + 32 * hq, x);
+        tc::tmem_ld16(tl + COL_D1 + 32 * hq + 16, x + 16);
         tc::wait_ld();
-        p_row_half(p16, r, 1, Gr, G, x1);
+        p_row_half(p16, r, hq, Gr, G, x);
       }
     }
     // this warp's reads of D1 are complete: the next chunk's [K;Q]K^T may overwrite it
