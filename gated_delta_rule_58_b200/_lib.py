@@ -85,6 +85,11 @@ def lib() -> ctypes.CDLL:
             L.gdn_last_error.argtypes = []
             L.gdn_get_device_error.restype = i32
             L.gdn_get_device_error.argtypes = [ctypes.POINTER(ctypes.c_uint32)]
+            L.gdn_cp_local_state.restype = i32
+            L.gdn_cp_local_state.argtypes = [vp, vp, vp, vp, vp, vp, i32, i64, vp, vp, i32, i32, i32, i32, i32, u32,
+                                             i32, vp]
+            L.gdn_cp_combine.restype = i32
+            L.gdn_cp_combine.argtypes = [vp, vp, i32, i32, i32, i32, i32, i32, vp, vp, vp]
             L.gdn_selftest_wait_timeout.restype = i32
             L.gdn_selftest_wait_timeout.argtypes = [u32, vp]
             L.gdn_version.restype = ctypes.c_char_p
@@ -113,6 +118,25 @@ def gdn_get_device_error() -> int:
     if st not in (GDN_OK, GDN_ERR_DEVICE_DATA):
         _check(st)
     return int(flags.value)
+
+
+def gdn_cp_local_state(q, k, v, g, beta, cu_seqlens, local_state, transfer, chunk=64, stream=None, l2norm=False):
+    """Context parallelism, step 1 (see include/gdn.h): the slice's local state H and
+    transfer M^T, both [N,H,dv,dk] fp32 K-last."""
+    total_T, H_qk, dk = q.shape
+    H, dv = v.shape[1], v.shape[-1]
+    N = cu_seqlens.numel() - 1
+    _check(lib().gdn_cp_local_state(_ptr(q), _ptr(k), _ptr(v), _ptr(g), _ptr(beta), _ptr(cu_seqlens), N, total_T,
+                                    _ptr(local_state), _ptr(transfer), H, H_qk, dk, dv, chunk,
+                                    GDN_QK_L2NORM if l2norm else 0, _dtype_code(q), _stream_ptr(stream, q.device)))
+
+
+def gdn_cp_combine(local_states, transfers, rank, start_state, initial_state=None, stream=None):
+    """Context parallelism, step 3: rank `rank`'s start state [N,H,dv,dk] from the
+    rank-major pairs [ranks,N,H,dv,dk] of ranks 0..rank-1 and the initial state."""
+    ranks, N, H, dv, dk = local_states.shape
+    _check(lib().gdn_cp_combine(_ptr(local_states), _ptr(transfers), ranks, rank, N, H, dk, dv, _ptr(initial_state),
+                                _ptr(start_state), _stream_ptr(stream, start_state.device)))
 
 
 def gdn_selftest_wait_timeout(wait_us: int, stream=None):

@@ -53,6 +53,11 @@ size_t prefill_transfer_workspace_bytes(const PrefillShape& s);
 // Chunks per segment (G) the transfer algorithm uses for this shape.
 int prefill_transfer_segment_chunks(const PrefillShape& s);
 gdn_status_t prefill_transfer_launch(const PrefillShape& s, const PrefillArgs& a, cudaStream_t stream);
+// Context parallelism: the start state of rank `rank` from the (local state,
+// transfer) pairs of ranks 0..rank-1, rank-major [ranks][N][H][128][128] (K-last).
+gdn_status_t cp_combine_launch(const float* local_states, const float* transfers, int ranks, int rank, int N, int H,
+                               const float* initial_state, float* start_state, unsigned int* err,
+                               cudaStream_t stream);
 
 // Reads cu_seqlens[n], cu_seqlens[n+1] and validates them against total_T; on a bad
 // pair sets GDN_DEVERR_BAD_CU_SEQLENS and returns false (the caller skips the unit).

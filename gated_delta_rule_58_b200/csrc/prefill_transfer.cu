@@ -154,9 +154,14 @@ __device__ __forceinline__ void fixup_issue(float* mt, float* loc, uint64_t* bar
   tc::bulk_load(tc::smem_u32(loc), local + off + (size_t)r0 * D, kFixLocBytes, bar);
 }
 
+// The segments of sequence n: seg_of_seq[n] .. seg_of_seq[n+1]-1 (the transfer
+// path), or, with seg_of_seq null, the context-parallel ranks 0 .. cp_count-1 of a
+// rank-major [ranks][N] list: entries n, n + cp_stride, ... (cp_stride = N). `fixed`
+// may be null (only the final state is wanted).
 __global__ void __launch_bounds__(kFixThreads)
-gdn_fixup_scan_kernel(const int32_t* seg_of_seq, int H, const float* local, const float* transfer,
-                      float* fixed, const float* initial_state, float* final_state, unsigned int* err) {
+gdn_fixup_scan_kernel(const int32_t* seg_of_seq, int cp_stride, int cp_count, int H, const float* local,
+                      const float* transfer, float* fixed, const float* initial_state, float* final_state,
+                      unsigned int* err) {
   extern __shared__ __align__(16) uint8_t fsm[];
   float* mt = reinterpret_cast<float*>(fsm);                 // [2][D][D]
   float* loc = mt + 2 * D * D;                                // [2][kFixRows][D]
@@ -173,7 +178,9 @@ gdn_fixup_scan_kernel(const int32_t* seg_of_seq, int H, const float* local, cons
   const int r0 = rb * kFixRows;
   const size_t ssz = (size_t)D * D;
   const size_t soff = ((size_t)n * H + h) * ssz;
-  const int s0 = seg_of_seq[n], s1 = seg_of_seq[n + 1];
+  const int first = seg_of_seq ? seg_of_seq[n] : n;
+  const int stride = seg_of_seq ? 1 : cp_stride;
+  const int count = seg_of_seq ? seg_of_seq[n + 1] - first : cp_count;
 
   if (tid == 0) {
     tc::mbar_init(&full[0], 1);
@@ -191,17 +198,18 @@ gdn_fixup_scan_kernel(const int32_t* seg_of_seq, int H, const float* local, cons
     for (int x4 = 0; x4 < 4; ++x4) sT[(l0 + x4) * kFixRows + jr + a] = cur[a][x4];
   }
   __syncthreads();
-  if (tid == 0 && s0 < s1)
-    fixup_issue(mt, loc, &full[0], transfer, local, ((size_t)s0 * H + h) * ssz, r0);
+  if (tid == 0 && count > 0)
+    fixup_issue(mt, loc, &full[0], transfer, local, ((size_t)first * H + h) * ssz, r0);
 
   int it = 0;
   bool pending_other = false;  // a prefetch into the other buffer is in flight
-  for (int sg = s0; sg < s1; ++sg, ++it) {
+  for (int i = 0; i < count; ++i, ++it) {
+    const int sg = first + i * stride;
     const int b = it & 1;
     pending_other = false;
-    if (tid == 0 && sg + 1 < s1) {
+    if (tid == 0 && i + 1 < count) {
       fixup_issue(mt + (b ^ 1) * D * D, loc + (b ^ 1) * kFixRows * D, &full[b ^ 1], transfer, local,
-                  ((size_t)(sg + 1) * H + h) * ssz, r0);
+                  ((size_t)(sg + stride) * H + h) * ssz, r0);
       pending_other = true;
     }
     const bool got = tc::mbar_wait(&full[b], (it >> 1) & 1, kFixWaitNs);
@@ -219,8 +227,9 @@ gdn_fixup_scan_kernel(const int32_t* seg_of_seq, int H, const float* local, cons
 #pragma unroll
     for (int a = 0; a < kFixRPT; ++a) {
       // the state at the segment start, then the local state as the accumulator
-      *reinterpret_cast<float4*>(fixed + off + (size_t)(r0 + jr + a) * D + l0) =
-          make_float4(cur[a][0], cur[a][1], cur[a][2], cur[a][3]);
+      if (fixed)
+        *reinterpret_cast<float4*>(fixed + off + (size_t)(r0 + jr + a) * D + l0) =
+            make_float4(cur[a][0], cur[a][1], cur[a][2], cur[a][3]);
       const float4 x = *reinterpret_cast<const float4*>(lr + (jr + a) * D + l0);
       acc[a][0] = x.x; acc[a][1] = x.y; acc[a][2] = x.z; acc[a][3] = x.w;
     }
@@ -304,7 +313,7 @@ gdn_status_t prefill_transfer_launch(const PrefillShape& s, const PrefillArgs& a
                 std::string("transfer prefill: setup: ") +
                     (e != cudaSuccess ? cudaGetErrorString(e) : "device index too large"));
   gdn_fixup_scan_kernel<<<(unsigned)((long long)s.N * s.H * (D / kFixRows)), kFixThreads, kFixSmem, stream>>>(
-      seg_of_seq, s.H, local, transfer, fixed, a.initial_state, a.final_state, a.err);
+      seg_of_seq, 0, 0, s.H, local, transfer, fixed, a.initial_state, a.final_state, a.err);
   st = check_launch("transfer prefill: fixup scan");
   if (st != GDN_OK) return st;
 
@@ -314,6 +323,26 @@ gdn_status_t prefill_transfer_launch(const PrefillShape& s, const PrefillArgs& a
   out.final_state = nullptr;
   out.mode = kPrefillOutputs;
   return prefill_fused_launch(seg, out, stream);
+}
+
+gdn_status_t cp_combine_launch(const float* local_states, const float* transfers, int ranks, int rank, int N, int H,
+                               const float* initial_state, float* start_state, unsigned int* err,
+                               cudaStream_t stream) {
+  static PerDeviceOnce once;  // the shared-memory opt-in applies to the current device only
+  int dev = 0;
+  cudaError_t e = cudaGetDevice(&dev);
+  if (e != cudaSuccess) return fail(GDN_ERR_CUDA, std::string("cp combine: cudaGetDevice: ") + cudaGetErrorString(e));
+  if (!run_once_per_device(once, dev, [&](int, int*) {
+        e = cudaFuncSetAttribute(gdn_fixup_scan_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, kFixSmem);
+        return e == cudaSuccess;
+      }))
+    return fail(e != cudaSuccess ? GDN_ERR_CUDA : GDN_ERR_UNSUPPORTED,
+                std::string("cp combine: setup: ") + (e != cudaSuccess ? cudaGetErrorString(e) : "device index too large"));
+  (void)ranks;
+  if ((long long)N * H * (D / kFixRows) >= (1LL << 31)) return fail(GDN_ERR_UNSUPPORTED, "cp combine: N * H too large");
+  gdn_fixup_scan_kernel<<<(unsigned)((long long)N * H * (D / kFixRows)), kFixThreads, kFixSmem, stream>>>(
+      nullptr, N, rank, H, local_states, transfers, nullptr, initial_state, start_state, err);
+  return check_launch("gdn_cp_combine");
 }
 
 }  // namespace gdn

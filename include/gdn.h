@@ -214,6 +214,34 @@ gdn_status_t gdn_chunk_prefill_static_scratch(const void* q, const void* k, cons
                                               int dv, int chunk, float scale, uint32_t flags,
                                               gdn_dtype_t in_dtype, gdn_dtype_t out_dtype, void* stream);
 
+/*
+ * Context parallelism for long prefills (the chunk/context-parallel state passing
+ * of the FlashInfer PR #3866 page, section 2, generalised from chunks to ranks).
+ * The tokens of each of the N sequences are split into consecutive slices held by
+ * consecutive ranks 0..ranks-1 (one GPU each). The recurrence is affine in the
+ * state over any run of tokens, S_end = M S_start + H, so each rank:
+ *   1. gdn_cp_local_state on its slice: H (from a zero state) and M (from the
+ *      identity with the values taken as zero), both [N, H, dv, dk] fp32 K-last
+ *      (the transfer as M^T row-major, i.e. K-last like a state);
+ *   2. all-gathers both across ranks in rank order (by the caller, e.g. NCCL):
+ *      rank-major [ranks, N, H, dv, dk];
+ *   3. gdn_cp_combine: its start state from the pairs of ranks 0..rank-1 and the
+ *      sequences' initial state (NULL = zero): S^T <- S^T M_r^T + H_r^T in fp32;
+ *   4. gdn_chunk_prefill on its slice with initial_state = that start state; the
+ *      last rank's final state is the sequences' final state.
+ * gdn_cp_local_state: dk == dv == 128, chunk == 64 (the fused tensor-core kernel,
+ * two launches); other arguments as gdn_chunk_prefill. gdn_cp_combine: dk == dv ==
+ * 128; rank 0 copies the initial state (or zeros); start_state may alias
+ * initial_state. Both only enqueue on `stream`.
+ */
+gdn_status_t gdn_cp_local_state(const void* q, const void* k, const void* v, const float* g,
+                                const float* beta, const int32_t* cu_seqlens, int N, int64_t total_T,
+                                float* local_state, float* transfer, int H, int H_qk, int dk, int dv,
+                                int chunk, uint32_t flags, gdn_dtype_t in_dtype, void* stream);
+gdn_status_t gdn_cp_combine(const float* local_states, const float* transfers, int ranks, int rank, int N,
+                            int H, int dk, int dv, const float* initial_state, float* start_state,
+                            void* stream);
+
 /* Message for the last non-OK status returned on this host thread ("" if none). */
 const char* gdn_last_error(void);
 

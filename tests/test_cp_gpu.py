@@ -1,0 +1,77 @@
+"""Context-parallel prefill with the library's kernels, ranks emulated one after
+another in one process on one GPU (nothing waits on another rank: the exchange is
+the stacking of the ranks' pairs). Each rank's slice: gdn_cp_local_state, then
+gdn_cp_combine over the earlier ranks' pairs, then gdn_chunk_prefill from that
+start state. The assembled outputs and the last rank's final state are compared
+with the oracle over whole sequences."""
+import pytest
+import torch
+
+import oracle
+import gated_delta_rule_58_b200 as gdn
+from gated_delta_rule_58_b200 import inputs
+from tests.cp_slices import rank_slice, slice_bounds
+from tests.util import assert_close
+
+pytestmark = pytest.mark.gpu
+DEV = "cuda"
+
+
+def _emulate(inp, ranks, l2norm=False, out_dtype=torch.float32):
+    lengths = inp.seqlens
+    N, H, dk = len(lengths), inp.v.shape[1], inp.q.shape[-1]
+    bounds = slice_bounds(lengths, ranks)
+    slices = [rank_slice(inp, bounds, r) for r in range(ranks)]
+    loc = torch.empty((ranks, N, H, 128, 128), device=DEV)
+    tr = torch.empty_like(loc)
+    for r, ((q, k, v, g, beta), cu, _) in enumerate(slices):
+        gdn.gdn_cp_local_state(q.to(DEV), k.to(DEV), v.to(DEV), g.to(DEV), beta.to(DEV), cu.to(DEV), loc[r], tr[r],
+                               l2norm=l2norm)
+    o = torch.full((inp.q.shape[0], H, 128), float("nan"), dtype=out_dtype, device=DEV)
+    fin = None
+    init = inp.initial_state.to(DEV) if inp.initial_state is not None else None
+    for r, ((q, k, v, g, beta), cu, idx) in enumerate(slices):
+        start = torch.empty((N, H, 128, 128), device=DEV)
+        gdn.gdn_cp_combine(loc, tr, r, start, initial_state=init)
+        o_r = torch.empty((q.shape[0], H, 128), dtype=out_dtype, device=DEV)
+        fin = torch.empty((N, H, 128, 128), device=DEV)
+        gdn.gdn_chunk_prefill(q.to(DEV), k.to(DEV), v.to(DEV), g.to(DEV), beta.to(DEV), cu.to(DEV), o_r,
+                              initial_state=start, final_state=fin, scale=inp.scale, l2norm=l2norm)
+        o[idx.to(DEV)] = o_r
+    torch.cuda.synchronize()
+    return o, fin
+
+
+@pytest.mark.parametrize("ranks", [1, 2, 4])
+@pytest.mark.parametrize("g_range", [(0.01, 0.5), (0.0, 0.01)])
+def test_cp_emulated_ranks_against_oracle(ranks, g_range):
+    inp = inputs.prefill_inputs([3000, 333, 64, 0, 1000], 4, 128, 128, seed=80, g_range=g_range)
+    o, fin = _emulate(inp, ranks)
+    o_r, f_r, _ = oracle.prefill(inp.q, inp.k, inp.v, inp.g, inp.beta, inp.cu_seqlens, inp.initial_state,
+                                 scale=inp.scale)
+    assert_close(o, o_r, what=f"cp ranks={ranks} o")
+    assert_close(fin, f_r, what=f"cp ranks={ranks} final state")
+
+
+def test_cp_one_long_sequence_grouped_heads_l2norm():
+    """One 16384-token sequence over 4 ranks, 8 value heads over 2 q/k heads, with
+    the normalisation and no initial state."""
+    inp = inputs.prefill_inputs([16384], 8, 128, 128, seed=81, g_range=(0.0, 0.02), H_qk=2, normalize_qk=False,
+                                with_initial_state=False)
+    o, fin = _emulate(inp, 4, l2norm=True, out_dtype=torch.bfloat16)
+    o_r, f_r, _ = oracle.prefill(inp.q, inp.k, inp.v, inp.g, inp.beta, inp.cu_seqlens, None, scale=inp.scale,
+                                 l2norm=True)
+    assert_close(o, o_r, what="cp long o")
+    assert_close(fin, f_r, what="cp long final state")
+
+
+def test_cp_single_rank_is_the_plain_prefill_bitwise():
+    inp = inputs.prefill_inputs([700, 65], 2, 128, 128, seed=82, g_range=(0.0, 0.05))
+    o, fin = _emulate(inp, 1)
+    o2 = torch.empty_like(o)
+    fin2 = torch.empty_like(fin)
+    gdn.gdn_chunk_prefill(inp.q.to(DEV), inp.k.to(DEV), inp.v.to(DEV), inp.g.to(DEV), inp.beta.to(DEV),
+                          inp.cu_seqlens.to(DEV), o2, initial_state=inp.initial_state.to(DEV), final_state=fin2,
+                          scale=inp.scale)
+    torch.cuda.synchronize()
+    assert torch.equal(o, o2) and torch.equal(fin, fin2)

@@ -142,3 +142,14 @@ def test_binding_fails_loudly_without_library(monkeypatch, tmp_path):
 def test_selftest_wait_rejects_bad_limits_on_host(L):
     assert L.gdn_selftest_wait_timeout(0, None) == gdn.GDN_ERR_INVALID_ARG
     assert L.gdn_selftest_wait_timeout(10000001, None) == gdn.GDN_ERR_INVALID_ARG
+
+
+def test_cp_entry_points_reject_on_host(L):
+    st = L.gdn_cp_combine(FAKE, FAKE, 2, 2, 1, 2, 128, 128, None, FAKE, None)  # rank >= ranks
+    assert st == gdn.GDN_ERR_INVALID_ARG
+    assert L.gdn_cp_combine(FAKE, FAKE, 2, 1, 1, 2, 64, 64, None, FAKE, None) == gdn.GDN_ERR_UNSUPPORTED
+    assert L.gdn_cp_combine(None, None, 2, 1, 1, 2, 128, 128, None, FAKE, None) == gdn.GDN_ERR_INVALID_ARG
+    assert L.gdn_cp_local_state(FAKE, FAKE, FAKE, FAKE, FAKE, FAKE, 1, 64, FAKE, FAKE, 2, 2, 128, 128, 32, 0,
+                                gdn.GDN_BF16, None) == gdn.GDN_ERR_UNSUPPORTED  # chunk 32
+    assert L.gdn_cp_local_state(FAKE, FAKE, FAKE, FAKE, FAKE, FAKE, 1, 64, None, FAKE, 2, 2, 128, 128, 64, 0,
+                                gdn.GDN_BF16, None) == gdn.GDN_ERR_INVALID_ARG

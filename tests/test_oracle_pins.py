@@ -581,4 +581,40 @@ def test_token_states_are_prefix_decodes():
     check_token_states_are_prefix_decodes()
 
 
+# ---------------------------------------------------------------- affine in the start state (context parallelism)
+
+def check_prefill_is_affine_in_the_initial_state(lib=None):
+    """A sequence's final state is affine in its start state, S_end = M S_0 + H,
+    with H the final state from a zero start and M (K-last: M^T) the final state
+    from the identity with the values set to zero; and running slice after slice
+    equals composing the slices' (M, H) pairs (what context parallelism exchanges).
+    Pinned against direct oracle runs from arbitrary start states."""
+    rng = _rng(35)
+    T, H, d = 23, 2, 4
+    q, k, v, g, beta = _rand_prefill(rng, T, H, d, d, 0.0, 0.3)
+    pref = _prefill(lib)
+    ident = np.broadcast_to(np.eye(d), (1, H, d, d)).copy()
+
+    def pair(sl):
+        _, Ht, _ = pref(q[sl], k[sl], v[sl], g[sl], beta[sl], [0, sl.stop - sl.start], None, scale=0.5)
+        _, Mt, _ = pref(q[sl], k[sl], np.zeros_like(v[sl]), g[sl], beta[sl], [0, sl.stop - sl.start], ident,
+                        scale=0.5)
+        return Mt[0], Ht[0]  # K-last: [H, dv, dk] and [H, dk, dk]
+
+    S0 = 0.1 * rng.standard_normal((1, H, d, d))
+    Mt, Ht = pair(slice(0, T))
+    _, fin, _ = pref(q, k, v, g, beta, [0, T], S0, scale=0.5)
+    assert _relerr(np.einsum("hij,hjk->hik", S0[0], Mt) + Ht, fin[0]) < 1e-13
+    # slices of 7, 9 and 7 tokens, composed in order from S0
+    S = S0[0]
+    for sl in (slice(0, 7), slice(7, 16), slice(16, T)):
+        Mt, Ht = pair(sl)
+        S = np.einsum("hij,hjk->hik", S, Mt) + Ht
+    assert _relerr(S, fin[0]) < 1e-13
+
+
+def test_prefill_is_affine_in_the_initial_state():
+    check_prefill_is_affine_in_the_initial_state()
+
+
 PIN_CHECKS.extend(v for k, v in sorted(globals().items()) if k.startswith("check_"))
