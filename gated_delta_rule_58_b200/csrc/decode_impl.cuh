@@ -368,6 +368,34 @@ gdn_decode_kernel(const DecodeParams p, const __grid_constant__ CUtensorMap pool
   if (tid == 0) tc::bulk_wait_all();
 }
 
+// Packed fp32 arithmetic (sm_100): one instruction does two independent fp32 FMAs
+// (or products), each rounded like its scalar form, so two state elements advance
+// together with the per-element operation sequence of a scalar loop.
+__device__ __forceinline__ float2 lo_pair(const float4& x) { return make_float2(x.x, x.y); }
+__device__ __forceinline__ float2 hi_pair(const float4& x) { return make_float2(x.z, x.w); }
+
+// One 16-byte chunk (4 columns) of two rows: x <- G x + sum_{m < n_terms} c_m k_m, the
+// terms in order m = 0, 1, ...; w points at the chunk's columns of key 0 in the
+// [vectors][DK] fp32 buffer, cc0/cc1 hold each row's c_m twice.
+template <int DK, int M>
+__device__ __forceinline__ void apply_terms(float4& x0, float4& x1, float G, const float2* cc0, const float2* cc1,
+                                            const float* w, int n_terms) {
+  const float2 gg = make_float2(G, G);
+  float2 a0 = __fmul2_rn(gg, lo_pair(x0)), b0 = __fmul2_rn(gg, hi_pair(x0));
+  float2 a1 = __fmul2_rn(gg, lo_pair(x1)), b1 = __fmul2_rn(gg, hi_pair(x1));
+#pragma unroll
+  for (int m = 0; m < M; ++m) {
+    if (m >= n_terms) break;
+    const float4 wv = *reinterpret_cast<const float4*>(w + m * DK);
+    a0 = __ffma2_rn(cc0[m], lo_pair(wv), a0);
+    a1 = __ffma2_rn(cc1[m], lo_pair(wv), a1);
+    b0 = __ffma2_rn(cc0[m], hi_pair(wv), b0);
+    b1 = __ffma2_rn(cc1[m], hi_pair(wv), b1);
+  }
+  x0 = make_float4(a0.x, a0.y, b0.x, b0.y);
+  x1 = make_float4(a1.x, a1.y, b1.x, b1.y);
+}
+
 // Multi-token / product step (M = T n_h > 1). Two consumer groups of DK threads
 // take the CTA's items alternately (group g its items g, g + 2, ...), so one
 // group's phases, which are separated by group barriers, overlap the other's.
@@ -514,9 +542,11 @@ gdn_decode_multi_kernel(const DecodeParams p, const __grid_constant__ CUtensorMa
       // row pass: dot products of both old rows with every key and query
       const uint8_t* srow0 = st + (size_t)r0 * 128;
       const uint8_t* srow1 = st + (size_t)r1 * 128;
-      float d0[NV], d1[NV];
+      // (each dot product as two partial sums, over the even and the odd columns,
+      // advanced together by packed FMAs and added at the end)
+      float2 e0[NV], e1[NV];
 #pragma unroll
-      for (int v = 0; v < NV; ++v) d0[v] = d1[v] = 0.f;
+      for (int v = 0; v < NV; ++v) e0[v] = e1[v] = make_float2(0.f, 0.f);
 #pragma unroll 4
       for (int c = 0; c < CPH; ++c) {
         const int gc = half * CPH + c;
@@ -527,14 +557,17 @@ gdn_decode_multi_kernel(const DecodeParams p, const __grid_constant__ CUtensorMa
 #pragma unroll
         for (int v = 0; v < NV; ++v) {
           const float4 wv = *reinterpret_cast<const float4*>(w + v * DK);
-          float a0 = d0[v], a1 = d1[v];
-          a0 = fmaf(x0.x, wv.x, a0); a1 = fmaf(x1.x, wv.x, a1);
-          a0 = fmaf(x0.y, wv.y, a0); a1 = fmaf(x1.y, wv.y, a1);
-          a0 = fmaf(x0.z, wv.z, a0); a1 = fmaf(x1.z, wv.z, a1);
-          a0 = fmaf(x0.w, wv.w, a0); a1 = fmaf(x1.w, wv.w, a1);
-          d0[v] = a0;
-          d1[v] = a1;
+          e0[v] = __ffma2_rn(lo_pair(x0), lo_pair(wv), e0[v]);
+          e1[v] = __ffma2_rn(lo_pair(x1), lo_pair(wv), e1[v]);
+          e0[v] = __ffma2_rn(hi_pair(x0), hi_pair(wv), e0[v]);
+          e1[v] = __ffma2_rn(hi_pair(x1), hi_pair(wv), e1[v]);
         }
+      }
+      float d0[NV], d1[NV];
+#pragma unroll
+      for (int v = 0; v < NV; ++v) {
+        d0[v] = e0[v].x + e0[v].y;
+        d1[v] = e1[v].x + e1[v].y;
       }
 #pragma unroll
       for (int v = 0; v < NV; ++v) {
@@ -585,24 +618,19 @@ gdn_decode_multi_kernel(const DecodeParams p, const __grid_constant__ CUtensorMa
           const int n_terms = (t + 1) * NH;  // a constant once the token loop is unrolled
           float* ts0 = p.token_states + ((((size_t)b * TT + t) * p.H + h) * DK + r0) * DK;
           float* ts1 = p.token_states + ((((size_t)b * TT + t) * p.H + h) * DK + r1) * DK;
+          float2 cc0[M], cc1[M];
+#pragma unroll
+          for (int m = 0; m < M; ++m) {
+            cc0[m] = make_float2(c0[m], c0[m]);
+            cc1[m] = make_float2(c1[m], c1[m]);
+          }
 #pragma unroll 4
           for (int c = 0; c < CPH; ++c) {
             const int gc = half * CPH + c;
             const uint32_t off = (gc >> 3) * (DK * 128) + (((gc & 7) ^ (r0 & 7)) << 4);
             float4 x0 = *reinterpret_cast<const float4*>(st + (size_t)r0 * 128 + off);
             float4 x1 = *reinterpret_cast<const float4*>(st + (size_t)r1 * 128 + off);
-            x0.x *= G; x0.y *= G; x0.z *= G; x0.w *= G;
-            x1.x *= G; x1.y *= G; x1.z *= G; x1.w *= G;
-            const float* w = vecf + 4 * gc;
-#pragma unroll
-            for (int m = 0; m < M; ++m) {
-              if (m >= n_terms) break;
-              const float4 wv = *reinterpret_cast<const float4*>(w + m * DK);
-              x0.x = fmaf(c0[m], wv.x, x0.x); x1.x = fmaf(c1[m], wv.x, x1.x);
-              x0.y = fmaf(c0[m], wv.y, x0.y); x1.y = fmaf(c1[m], wv.y, x1.y);
-              x0.z = fmaf(c0[m], wv.z, x0.z); x1.z = fmaf(c1[m], wv.z, x1.z);
-              x0.w = fmaf(c0[m], wv.w, x0.w); x1.w = fmaf(c1[m], wv.w, x1.w);
-            }
+            apply_terms<DK, M>(x0, x1, G, cc0, cc1, vecf + 4 * gc, n_terms);
             reinterpret_cast<float4*>(ts0)[gc] = x0;
             reinterpret_cast<float4*>(ts1)[gc] = x1;
           }
@@ -612,23 +640,19 @@ gdn_decode_multi_kernel(const DecodeParams p, const __grid_constant__ CUtensorMa
       // update pass: s_new = Gamma s_0 + sum_m c_m k_m, in place (same swizzled chunks)
       uint8_t* wrow0 = st + (size_t)r0 * 128;
       uint8_t* wrow1 = st + (size_t)r1 * 128;
+      float2 cc0[M], cc1[M];
+#pragma unroll
+      for (int m = 0; m < M; ++m) {
+        cc0[m] = make_float2(c0[m], c0[m]);
+        cc1[m] = make_float2(c1[m], c1[m]);
+      }
 #pragma unroll 4
       for (int c = 0; c < CPH; ++c) {
         const int gc = half * CPH + c;
         const uint32_t off = (gc >> 3) * (DK * 128) + (((gc & 7) ^ (r0 & 7)) << 4);
         float4 x0 = *reinterpret_cast<const float4*>(wrow0 + off);
         float4 x1 = *reinterpret_cast<const float4*>(wrow1 + off);
-        x0.x *= G; x0.y *= G; x0.z *= G; x0.w *= G;
-        x1.x *= G; x1.y *= G; x1.z *= G; x1.w *= G;
-        const float* w = vecf + 4 * gc;
-#pragma unroll
-        for (int m = 0; m < M; ++m) {
-          const float4 wv = *reinterpret_cast<const float4*>(w + m * DK);
-          x0.x = fmaf(c0[m], wv.x, x0.x); x1.x = fmaf(c1[m], wv.x, x1.x);
-          x0.y = fmaf(c0[m], wv.y, x0.y); x1.y = fmaf(c1[m], wv.y, x1.y);
-          x0.z = fmaf(c0[m], wv.z, x0.z); x1.z = fmaf(c1[m], wv.z, x1.z);
-          x0.w = fmaf(c0[m], wv.w, x0.w); x1.w = fmaf(c1[m], wv.w, x1.w);
-        }
+        apply_terms<DK, M>(x0, x1, G, cc0, cc1, vecf + 4 * gc, M);
         *reinterpret_cast<float4*>(wrow0 + off) = x0;
         *reinterpret_cast<float4*>(wrow1 + off) = x1;
       }
