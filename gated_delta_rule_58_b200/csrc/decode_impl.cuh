@@ -227,8 +227,14 @@ __device__ __forceinline__ void decode_producer(const DecodeParams& p, const CUt
 // split along V) otherwise. Rows are independent in this step (each needs only the
 // head's k, q and its own v entry), so every row gets the same arithmetic in the
 // same order whatever ROWS is.
+//
+// Registers are allocated per scheduler (a quarter of the SM's 64K each, in units
+// of 256 per warp). A split head's CTA is small enough that two or more fit in
+// shared memory, so its register use is capped at 168 (5,376 per warp, three warps
+// per scheduler): at 180 a scheduler holds two warps and one CTA of five warps
+// fills the SM.
 template <int DK, int TT, int NH, typename TIn, typename TOut, int ROWS>
-__global__ void __launch_bounds__(threads_per_row<TT, NH>() * ROWS + 32, 1)
+__global__ void __launch_bounds__(threads_per_row<TT, NH>() * ROWS + 32, 1) __maxnreg__(ROWS < DK ? 168 : 255)
 gdn_decode_kernel(const DecodeParams p, const __grid_constant__ CUtensorMap pool_map) {
   using L = StageLayout<DK, TT, NH, TIn, ROWS>;
   static_assert(L::M == 1, "single-token step");
