@@ -51,6 +51,10 @@ def _declare(lib):
     lib.gdn_oracle_prefill.argtypes = [dp, dp, dp, dp, dp, ctypes.POINTER(ctypes.c_int64),
                                        ctypes.c_int, ctypes.c_int, ctypes.c_int, ctypes.c_int, ctypes.c_int,
                                        ctypes.c_double, ctypes.c_int, dp, dp, dp, ctypes.c_int]
+    lib.gdn_oracle_prefill_backward.restype = ctypes.c_int
+    lib.gdn_oracle_prefill_backward.argtypes = [dp, dp, dp, dp, dp, ctypes.POINTER(ctypes.c_int64),
+                                                ctypes.c_int, ctypes.c_int, ctypes.c_int, ctypes.c_int, ctypes.c_int,
+                                                ctypes.c_double, dp, dp, dp, dp, dp, dp, dp, dp, dp, ctypes.c_int]
     lib.gdn_oracle_decode.restype = ctypes.c_int
     lib.gdn_oracle_decode.argtypes = [dp, dp, dp, dp, dp, dp, ctypes.c_int,
                                       ctypes.POINTER(ctypes.c_int32), dp,
@@ -115,6 +119,42 @@ def prefill(q, k, v, g, beta, cu_seqlens, initial_state=None, scale=None, nthrea
     if rc < 0:
         raise ValueError("gdn_oracle_prefill: bad arguments")
     return o, fin, rc
+
+
+def prefill_backward(q, k, v, g, beta, cu_seqlens, d_o, initial_state=None, d_final_state=None, scale=None,
+                     nthreads=0, lib=None):
+    """Reverse-mode derivatives of `prefill` (one Householder per token, no q/k
+    normalisation), fp64, token by token (see gdn_oracle.c).
+
+    d_o: [total_T, H, dv]; d_final_state: [N, H, dv, dk] or None (zero).
+    Returns dict(dq [total_T, H_qk, dk], dk [total_T, H_qk, dk], dv [total_T, H, dv],
+    dg [total_T, H], dbeta [total_T, H], d_initial_state [N, H, dv, dk]). The q/k
+    derivatives of value heads that share a q/k head are summed.
+    """
+    lib = lib or _load()
+    q, k, v, g, beta, d_o = (f64(a) for a in (q, k, v, g, beta, d_o))
+    cu = np.ascontiguousarray(np.asarray(f64(cu_seqlens), dtype=np.int64))
+    init, dfin = f64(initial_state), f64(d_final_state)
+    total_T, Hqk, dk = q.shape
+    H, dv = v.shape[1], v.shape[-1]
+    N = cu.shape[0] - 1
+    if scale is None:
+        scale = 1.0 / np.sqrt(dk)
+    dq = np.zeros((total_T, H, dk), np.float64)
+    dkk = np.zeros((total_T, H, dk), np.float64)
+    dvv = np.zeros((total_T, H, dv), np.float64)
+    dg = np.zeros((total_T, H), np.float64)
+    db = np.zeros((total_T, H), np.float64)
+    dinit = np.zeros((N, H, dv, dk), np.float64)
+    rc = lib.gdn_oracle_prefill_backward(_ptr(q), _ptr(k), _ptr(v), _ptr(g), _ptr(beta), _ptr(cu, ctypes.c_int64),
+                                         N, H, Hqk, dk, dv, float(scale), _ptr(init), _ptr(d_o), _ptr(dfin),
+                                         _ptr(dq), _ptr(dkk), _ptr(dvv), _ptr(dg), _ptr(db), _ptr(dinit),
+                                         int(nthreads))
+    if rc < 0:
+        raise ValueError("gdn_oracle_prefill_backward: bad arguments")
+    grp = H // Hqk
+    return dict(dq=dq.reshape(total_T, Hqk, grp, dk).sum(2), dk=dkk.reshape(total_T, Hqk, grp, dk).sum(2),
+                dv=dvv, dg=dg, dbeta=db, d_initial_state=dinit)
 
 
 def decode(q, k, v, g, beta, pool, slot_ids, scale=None, nthreads=0, lib=None, copy_pool=True,

@@ -257,3 +257,139 @@ int gdn_oracle_decode(const double* q, const double* k, const double* v, const d
                   token_states};
   return run_items(B * H, nthreads, decode_item, &c);
 }
+
+/* ---- prefill backward: reverse-mode derivatives of the gated delta rule ----
+ *
+ * For a loss L with upstream derivatives dO_t = dL/do_t and dS_T = dL/dS_T (the
+ * final state), the token recurrence is walked backwards with D = dL/dS_t, written
+ * out from the chain rule on the two relations of each token (P = I - beta k k^T,
+ * S~ = alpha S_{t-1}):
+ *     S_t = P S~ + beta k v^T,        o_t = scale S_t^T q.
+ * Per token, last to first:
+ *     D    += scale q dO^T                          (o_t reads S_t)
+ *     dq    = scale S_t dO
+ *     u     = S~^T k,   w = D^T k
+ *     dv    = beta w
+ *     dbeta = w . (v - u)
+ *     dk    = beta (D (v - u) - S~ w)
+ *     dg    = <D, S~> - beta (u . w)                 (alpha = exp(g): dg = alpha dL/dalpha)
+ *     D    <- alpha (D - beta k w^T)                 (= alpha P D, dL/dS_{t-1})
+ * and dL/dS_0 = D at the end. Every state S_t is kept from a forward pass first.
+ * Scope: one Householder per token and no q/k normalisation.
+ */
+
+typedef struct {
+  const double *q, *k, *v, *g, *beta;
+  const int64_t* cu;
+  int H, Hqk, dk, dv;
+  double scale;
+  const double *init, *d_o, *d_fin;
+  double *dq, *dkk, *dvv, *dg, *dbeta, *d_init;
+} backward_ctx;
+
+static void backward_item(void* vctx, int item) {
+  backward_ctx* c = (backward_ctx*)vctx;
+  const int H = c->H, Hqk = c->Hqk, dk = c->dk, dv = c->dv;
+  const int n = item / H, h = item % H;
+  const int hq = h / (H / Hqk);
+  const size_t ssz = (size_t)dk * dv;
+  const int64_t t0 = c->cu[n], T = c->cu[n + 1] - c->cu[n];
+  /* states S_0 .. S_T, each S^T [dv][dk] */
+  double* states = (double*)malloc((size_t)(T + 1) * ssz * sizeof(double));
+  double* Dt = (double*)malloc(ssz * sizeof(double));
+  double* u = (double*)malloc((size_t)dv * sizeof(double));
+  double* w = (double*)malloc((size_t)dv * sizeof(double));
+  if (c->init)
+    memcpy(states, c->init + ((size_t)n * H + h) * ssz, ssz * sizeof(double));
+  else
+    memset(states, 0, ssz * sizeof(double));
+  for (int64_t t = 0; t < T; ++t) {
+    const size_t th = (size_t)(t0 + t) * H + h, tq = (size_t)(t0 + t) * Hqk + hq;
+    double* St = states + (size_t)(t + 1) * ssz;
+    memcpy(St, states + (size_t)t * ssz, ssz * sizeof(double));
+    apply_gate(St, exp(c->g[th]), dk, dv);
+    apply_householder(St, c->k + tq * dk, c->v + th * dv, c->beta[th], dk, dv);
+  }
+  if (c->d_fin)
+    memcpy(Dt, c->d_fin + ((size_t)n * H + h) * ssz, ssz * sizeof(double));
+  else
+    memset(Dt, 0, ssz * sizeof(double));
+  for (int64_t t = T - 1; t >= 0; --t) {
+    const size_t th = (size_t)(t0 + t) * H + h, tq = (size_t)(t0 + t) * Hqk + hq;
+    const double* q = c->q + tq * dk;
+    const double* k = c->k + tq * dk;
+    const double* v = c->v + th * dv;
+    const double* dO = c->d_o + th * dv;
+    const double alpha = exp(c->g[th]), beta = c->beta[th];
+    const double* St = states + (size_t)(t + 1) * ssz;  /* S_t */
+    const double* Sp = states + (size_t)t * ssz;        /* S_{t-1} */
+    double* dq = c->dq + th * dk;                       /* per value head */
+    double* dkv = c->dkk + th * dk;
+    /* D += scale q dO^T;  dq = scale S_t dO */
+    for (int j = 0; j < dv; ++j)
+      for (int i = 0; i < dk; ++i) Dt[(size_t)j * dk + i] += c->scale * q[i] * dO[j];
+    for (int i = 0; i < dk; ++i) {
+      double acc = 0.0;
+      for (int j = 0; j < dv; ++j) acc += St[(size_t)j * dk + i] * dO[j];
+      dq[i] = c->scale * acc;
+    }
+    /* u = S~^T k, w = D^T k */
+    for (int j = 0; j < dv; ++j) {
+      double pu = 0.0, pw = 0.0;
+      for (int i = 0; i < dk; ++i) {
+        pu += alpha * Sp[(size_t)j * dk + i] * k[i];
+        pw += Dt[(size_t)j * dk + i] * k[i];
+      }
+      u[j] = pu;
+      w[j] = pw;
+    }
+    double db = 0.0, uw = 0.0, ds = 0.0;
+    for (int j = 0; j < dv; ++j) {
+      c->dvv[th * dv + j] = beta * w[j];
+      db += w[j] * (v[j] - u[j]);
+      uw += u[j] * w[j];
+    }
+    c->dbeta[th] = db;
+    for (int i = 0; i < dk; ++i) {
+      double a = 0.0, b = 0.0;
+      for (int j = 0; j < dv; ++j) {
+        a += Dt[(size_t)j * dk + i] * (v[j] - u[j]);
+        b += alpha * Sp[(size_t)j * dk + i] * w[j];
+      }
+      dkv[i] = beta * (a - b);
+    }
+    for (int j = 0; j < dv; ++j)
+      for (int i = 0; i < dk; ++i) ds += Dt[(size_t)j * dk + i] * alpha * Sp[(size_t)j * dk + i];
+    c->dg[th] = ds - beta * uw;
+    /* D <- alpha (D - beta k w^T) */
+    for (int j = 0; j < dv; ++j)
+      for (int i = 0; i < dk; ++i)
+        Dt[(size_t)j * dk + i] = alpha * (Dt[(size_t)j * dk + i] - beta * k[i] * w[j]);
+  }
+  if (c->d_init) memcpy(c->d_init + ((size_t)n * H + h) * ssz, Dt, ssz * sizeof(double));
+  free(w);
+  free(u);
+  free(Dt);
+  free(states);
+}
+
+/*
+ * Inputs as for gdn_oracle_prefill, plus d_o [total_T, H, dv] and d_final_state
+ * [N, H, dv, dk] or NULL (zero). Outputs: dq, dk [total_T, H, dk] per VALUE head
+ * (the caller sums the heads that share a q/k head), dv [total_T, H, dv], dg and
+ * dbeta [total_T, H], d_initial_state [N, H, dv, dk] or NULL.
+ * Returns the number of threads used, or a negative value on bad arguments.
+ */
+int gdn_oracle_prefill_backward(const double* q, const double* k, const double* v, const double* g,
+                                const double* beta, const int64_t* cu_seqlens, int N, int H, int Hqk,
+                                int dk, int dv, double scale, const double* init, const double* d_o,
+                                const double* d_final_state, double* dq, double* dk_out, double* dv_out,
+                                double* dg, double* dbeta, double* d_init, int nthreads) {
+  if (N < 0 || H <= 0 || Hqk <= 0 || H % Hqk != 0 || dk <= 0 || dv <= 0 || !cu_seqlens || !d_o) return -1;
+  if (cu_seqlens[0] != 0) return -1;
+  for (int n = 0; n < N; ++n)
+    if (cu_seqlens[n + 1] < cu_seqlens[n]) return -1;
+  backward_ctx c = {q, k, v, g, beta, cu_seqlens, H, Hqk, dk, dv, scale, init, d_o, d_final_state,
+                    dq, dk_out, dv_out, dg, dbeta, d_init};
+  return run_items(N * H, nthreads, backward_item, &c);
+}

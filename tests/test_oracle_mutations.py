@@ -68,6 +68,15 @@ MUTANTS = {
         "      memcpy(c->token_states + bth * (size_t)dk * dv, St, (size_t)dk * dv * sizeof(double));\n"
         "    apply_gate(St, exp(c->g[bth]), dk, dv);\n    for (int m = 0; m < nh; ++m) {\n")],
     # the normalisation divides by the squared norm
+    # backward: the key derivative without its state term
+    "backward_dk_without_state_term": [("dkv[i] = beta * (a - b);", "dkv[i] = beta * a;")],
+    # backward: wrong sign of the Householder part of the gate derivative
+    "backward_dg_sign": [("c->dg[th] = ds - beta * uw;", "c->dg[th] = ds + beta * uw;")],
+    # backward: the state derivative carried to the previous token without the gate
+    "backward_carry_without_gate": [("Dt[(size_t)j * dk + i] = alpha * (Dt[(size_t)j * dk + i] - beta * k[i] * w[j]);",
+                                     "Dt[(size_t)j * dk + i] = Dt[(size_t)j * dk + i] - beta * k[i] * w[j];")],
+    # backward: the query derivative read from the previous state
+    "backward_dq_previous_state": [("acc += St[(size_t)j * dk + i] * dO[j];", "acc += Sp[(size_t)j * dk + i] * dO[j];")],
     "l2norm_squared": [("const double inv = ss > 0.0 ? 1.0 / sqrt(ss) : 0.0;",
                         "const double inv = ss > 0.0 ? 1.0 / ss : 0.0;")],
 }
