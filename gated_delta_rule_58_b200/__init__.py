@@ -10,7 +10,8 @@ from ._lib import (  # noqa: F401
     GDN_ERR_UNSUPPORTED, GDN_ERR_WORKSPACE, GDN_DEVERR_BAD_CU_SEQLENS,
     GDN_DEVERR_SLOT_OUT_OF_RANGE, GDN_DEVERR_TIMEOUT, GDN_PREFILL_AUTO, GDN_PREFILL_FUSED,
     GDN_PREFILL_SEQUENTIAL, GDN_PREFILL_TRANSFER, GDN_QK_L2NORM, GdnError, declared_functions,
-    gdn_chunk_prefill, gdn_chunk_prefill_static_scratch, gdn_cp_combine, gdn_cp_local_state, gdn_chunk_prefill_workspace_size, gdn_decode,
+    gdn_chunk_prefill, gdn_chunk_prefill_backward, gdn_chunk_prefill_backward_workspace_size,
+    gdn_chunk_prefill_static_scratch, gdn_cp_combine, gdn_cp_local_state, gdn_chunk_prefill_workspace_size, gdn_decode,
     gdn_decode_mtp,
     gdn_get_device_error, gdn_selftest_wait_timeout,
     gdn_last_error, gdn_version, lib,

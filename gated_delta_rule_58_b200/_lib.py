@@ -90,6 +90,12 @@ def lib() -> ctypes.CDLL:
                                              i32, vp]
             L.gdn_cp_combine.restype = i32
             L.gdn_cp_combine.argtypes = [vp, vp, i32, i32, i32, i32, i32, i32, vp, vp, vp]
+            L.gdn_chunk_prefill_backward_workspace_size.restype = i32
+            L.gdn_chunk_prefill_backward_workspace_size.argtypes = [i32, i64, i32, i32, i32, i32,
+                                                                    ctypes.POINTER(ctypes.c_size_t)]
+            L.gdn_chunk_prefill_backward.restype = i32
+            L.gdn_chunk_prefill_backward.argtypes = [vp, vp, vp, vp, vp, vp, i32, i64, vp, vp, vp, vp, vp, vp, vp,
+                                                     vp, vp, i32, i32, i32, i32, i32, f32, u32, i32, vp, sz, vp]
             L.gdn_selftest_wait_timeout.restype = i32
             L.gdn_selftest_wait_timeout.argtypes = [u32, vp]
             L.gdn_version.restype = ctypes.c_char_p
@@ -243,6 +249,54 @@ def gdn_chunk_prefill(q, k, v, g, beta, cu_seqlens, o, initial_state=None, final
                                  _dtype_code(o), algo, ws_ptr, ws_bytes, _stream_ptr(stream, q.device))
     _check(st)
     return o
+
+
+def gdn_chunk_prefill_backward_workspace_size(N, total_T, H, dk, dv, chunk=64) -> int:
+    out = ctypes.c_size_t(0)
+    _check(lib().gdn_chunk_prefill_backward_workspace_size(N, total_T, H, dk, dv, chunk, ctypes.byref(out)))
+    return int(out.value)
+
+
+def gdn_chunk_prefill_backward(q, k, v, g, beta, cu_seqlens, d_o, initial_state=None, d_final_state=None,
+                               chunk=64, scale=None, workspace=None, stream=None, grads=None):
+    """Derivatives of a loss with respect to the prefill's inputs (see include/gdn.h),
+    given d_o [total_T,H,dv] (q's dtype) and d_final_state [N,H,dv,dk] fp32 or None.
+    Returns dict(dq, dk [total_T,H_qk,dk], dv [total_T,H,dv], dg, dbeta [total_T,H],
+    d_initial_state [N,H,dv,dk]), fp32; `grads` may pass these tensors in. The
+    workspace (uint8 CUDA tensor) is allocated through torch when None."""
+    import torch
+    total_T, H_qk, dk = q.shape
+    H, dv = v.shape[1], v.shape[-1]
+    N = cu_seqlens.numel() - 1
+    if scale is None:
+        scale = dk ** -0.5
+    dev = q.device
+    if d_o.dtype != q.dtype:
+        raise TypeError("gdn_chunk_prefill_backward: d_o must have q's dtype")
+    if grads is None:
+        f = dict(dtype=torch.float32, device=dev)
+        grads = dict(dq=torch.empty((total_T, H_qk, dk), **f), dk=torch.empty((total_T, H_qk, dk), **f),
+                     dv=torch.empty((total_T, H, dv), **f), dg=torch.empty((total_T, H), **f),
+                     dbeta=torch.empty((total_T, H), **f), d_initial_state=torch.empty((N, H, dv, dk), **f))
+    need = gdn_chunk_prefill_backward_workspace_size(N, total_T, H, dk, dv, chunk)
+    if workspace is None:
+        if stream is not None and not isinstance(stream, torch.cuda.Stream):
+            raise ValueError("gdn_chunk_prefill_backward: pass `workspace` when `stream` is a raw handle")
+        ctx = torch.cuda.stream(stream) if stream is not None else _nullcontext()
+        with ctx:
+            workspace = torch.empty(max(need, 1), dtype=torch.uint8, device=dev)
+    st = lib().gdn_chunk_prefill_backward(
+        _ptr(q), _ptr(k), _ptr(v), _ptr(g), _ptr(beta), _ptr(cu_seqlens), N, total_T, _ptr(initial_state),
+        _ptr(d_o), _ptr(d_final_state), _ptr(grads["dq"]), _ptr(grads["dk"]), _ptr(grads["dv"]),
+        _ptr(grads["dg"]), _ptr(grads["dbeta"]), _ptr(grads.get("d_initial_state")), H, H_qk, dk, dv, chunk,
+        float(scale), 0, _dtype_code(q), _ptr(workspace), workspace.numel(), _stream_ptr(stream, dev))
+    _check(st)
+    return grads
+
+
+def _nullcontext():
+    import contextlib
+    return contextlib.nullcontext()
 
 
 def gdn_chunk_prefill_static_scratch(q, k, v, g, beta, cu_seqlens, o, initial_state=None, final_state=None,

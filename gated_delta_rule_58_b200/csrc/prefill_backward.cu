@@ -1,0 +1,389 @@
+// Backward of the prefill: reverse-mode derivatives of the gated delta rule with
+// respect to q, k, v, g, beta and the initial state, given the derivatives of a loss
+// with respect to the outputs and the final state. The pages give no backward pass;
+// this is the chain rule on the two relations of one token (P = I - beta k k^T,
+// S~ = alpha S_{t-1}, alpha = exp(g)):
+//     S_t = P S~ + beta k v^T,        o_t = scale S_t^T q,
+// walked from the last token to the first with D = dL/dS_t:
+//     D    += scale q dO^T;           dq = scale S_t dO
+//     u     = S~^T k;   w = D^T k;    dv = beta w;   dbeta = w . (v - u)
+//     dk    = beta (D (v - u) - S~ w)
+//     dg    = <D, S~> - beta (u . w)
+//     D    <- alpha (D - beta k w^T)  (dL/dS_{t-1});   dL/dS_0 = D at the end.
+//
+// Token-sequential SIMT, one CTA per (sequence, head), laid out like the sequential
+// forward kernel: value column j of S is owned by dk / 32 adjacent lanes, 32 of its
+// dk entries each. The states S_{t-1} the walk needs are recomputed:
+//   1. forward over the sequence, writing the state at the start of every chunk of
+//      C tokens to the workspace (checkpoints);
+//   2. for each chunk, last to first: recompute the chunk's states from its
+//      checkpoint into a per-CTA scratch (C + 1 states), then walk its tokens
+//      backwards reading S_{t-1} and S_t from there (a thread reads back only what it
+//      wrote, so no barrier orders the scratch).
+// Per token the column sums of dq and dk go through shared memory (each thread
+// writes its 32 partial products, then 2 dk threads each add one entry over the dv
+// columns); dg and dbeta are block reductions. dq and dk are accumulated with fp32
+// atomics into zeroed outputs, so value heads that share a q/k head add up.
+#include <string>
+
+#include "device_once.h"
+#include "prefill.cuh"
+
+namespace gdn {
+namespace {
+
+struct BwdArgs {
+  const void* q;
+  const void* k;
+  const void* v;
+  const void* d_o;
+  const float* g;
+  const float* beta;
+  const int32_t* cu;
+  const float* init;
+  const float* d_fin;
+  float* dq;
+  float* dk;
+  float* dv;
+  float* dg;
+  float* dbeta;
+  float* d_init;
+  float* ckpt;     // [H][ck_slots][D][D]
+  float* scratch;  // [N * H][C + 1][D][D]
+  size_t ck_slots;
+  int64_t total_T;
+  int N, H, Hqk, C;
+  float scale;
+  unsigned int* err;
+};
+
+inline size_t align256(size_t x) { return (x + 255) & ~size_t(255); }
+
+struct BwdLayout {
+  size_t ck_slots, scratch_off, bytes;
+};
+
+// Sequence n's checkpoints take slots bos / C + n ... (+ ceil(len / C)), which never
+// overlap the next sequence's and stay below total_T / C + N + 1.
+BwdLayout bwd_layout(int N, int64_t total_T, int H, int D, int C) {
+  BwdLayout L;
+  const size_t st = (size_t)D * D * sizeof(float);
+  L.ck_slots = (size_t)(total_T / C) + (size_t)N + 1;
+  L.scratch_off = align256((size_t)H * L.ck_slots * st);
+  L.bytes = L.scratch_off + (size_t)N * H * (size_t)(C + 1) * st;
+  return L;
+}
+
+template <int D>
+constexpr size_t bwd_smem_bytes() {
+  // token vectors [2][k, q, v, dO][D], gates [2][alpha, beta], column partials of dq
+  // and dk [D][D] each, scalar partials [warps][2]
+  return (8 * D + 4 + 2 * D * D + 2 * (D * (D / 32) / 32)) * sizeof(float);
+}
+
+template <int D, typename TIn>
+__global__ void __launch_bounds__(D * (D / 32))
+gdn_prefill_backward_kernel(const BwdArgs a) {
+  constexpr int TPC = D / 32;  // threads per state column
+  constexpr int NT = D * TPC;
+  constexpr int PER = 32;      // entries of the column per thread
+  constexpr int NW = NT / 32;
+  extern __shared__ __align__(16) float bsm[];
+  float* tok = bsm;              // [2][4][D]
+  float* gates = tok + 8 * D;    // [2][2]
+  float* red_q = gates + 4;      // [D columns][D entries]
+  float* red_k = red_q + D * D;
+  float* red_s = red_k + D * D;  // [NW][2]
+
+  const int tid = threadIdx.x;
+  const int col = tid / TPC, part = tid % TPC;
+  const int n = blockIdx.x / a.H, h = blockIdx.x - n * a.H;
+  const int hq = h / (a.H / a.Hqk);
+  int64_t bos, eos;
+  if (!seq_bounds(a.cu, n, a.total_T, a.err, &bos, &eos)) return;
+  const int nck = (int)((eos - bos + a.C - 1) / a.C);
+  const size_t SS = (size_t)D * D;
+  const size_t mine = (size_t)col * D + part * PER;  // this thread's entries of a K-last state
+  const size_t state_off = ((size_t)n * a.H + h) * SS + mine;
+  float* ck = a.ckpt + ((size_t)h * a.ck_slots + (size_t)(bos / a.C) + n) * SS + mine;
+  float* scr = a.scratch + (size_t)blockIdx.x * (size_t)(a.C + 1) * SS + mine;
+  const TIn* qp = static_cast<const TIn*>(a.q);
+  const TIn* kp = static_cast<const TIn*>(a.k);
+  const TIn* vp = static_cast<const TIn*>(a.v);
+  const TIn* dop = static_cast<const TIn*>(a.d_o);
+
+  // token t's k, q, v, dO and gates into buffer `buf` (two buffers: the barrier of
+  // the token in between orders every read of a buffer before its refill)
+  auto stage = [&](int64_t t, int buf) {
+    const size_t th = (size_t)t * a.H + h, tq = (size_t)t * a.Hqk + hq;
+    float* tb = tok + buf * 4 * D;
+    for (int i = tid; i < D; i += NT) {
+      tb[i] = to_f32(kp[tq * D + i]);
+      tb[D + i] = to_f32(qp[tq * D + i]);
+      tb[2 * D + i] = to_f32(vp[th * D + i]);
+      tb[3 * D + i] = to_f32(dop[th * D + i]);
+    }
+    if (tid == 0) {
+      gates[2 * buf] = expf(a.g[th]);
+      gates[2 * buf + 1] = a.beta[th];
+    }
+  };
+  // one token forward on this thread's entries of column col (as the forward kernel)
+  auto advance = [&](float* st, int buf) {
+    const float* tb = tok + buf * 4 * D;
+    const float* kv = tb + part * PER;
+    const float alpha = gates[2 * buf], beta = gates[2 * buf + 1];
+    float u = 0.f;
+#pragma unroll
+    for (int x = 0; x < PER; ++x) u = fmaf(kv[x], st[x], u);
+#pragma unroll
+    for (int off = 1; off < TPC; off <<= 1) u += __shfl_xor_sync(0xffffffffu, u, off);
+    const float c = beta * (tb[2 * D + col] - alpha * u);
+#pragma unroll
+    for (int x = 0; x < PER; ++x) st[x] = fmaf(alpha, st[x], c * kv[x]);
+  };
+  auto load_state = [&](const float* p, float* st) {
+#pragma unroll
+    for (int x = 0; x < PER; x += 4) {
+      const float4 f = *reinterpret_cast<const float4*>(p + x);
+      st[x] = f.x; st[x + 1] = f.y; st[x + 2] = f.z; st[x + 3] = f.w;
+    }
+  };
+  auto store_state = [&](float* p, const float* st) {
+#pragma unroll
+    for (int x = 0; x < PER; x += 4)
+      *reinterpret_cast<float4*>(p + x) = make_float4(st[x], st[x + 1], st[x + 2], st[x + 3]);
+  };
+
+  // 1. forward with a checkpoint at the start of every chunk
+  int it = 0;  // staged tokens so far (buffer parity)
+  {
+    float st[PER];
+    if (a.init) {
+      load_state(a.init + state_off, st);
+    } else {
+#pragma unroll
+      for (int x = 0; x < PER; ++x) st[x] = 0.f;
+    }
+    for (int64_t t = bos; t < eos; ++t) {
+      const int buf = (it++) & 1;
+      stage(t, buf);
+      __syncthreads();
+      if ((t - bos) % a.C == 0) store_state(ck + (size_t)((t - bos) / a.C) * SS, st);
+      advance(st, buf);
+    }
+  }
+
+  // 2. chunks last to first
+  float Dm[PER];  // dL/dS_t, this thread's entries
+  if (a.d_fin) {
+    load_state(a.d_fin + state_off, Dm);
+  } else {
+#pragma unroll
+    for (int x = 0; x < PER; ++x) Dm[x] = 0.f;
+  }
+  for (int c = nck - 1; c >= 0; --c) {
+    const int64_t t0 = bos + (int64_t)c * a.C;
+    const int64_t t1 = (t0 + a.C < eos) ? t0 + a.C : eos;
+    {
+      // scratch slot x = the state before token t0 + x; slot t1 - t0 = after the chunk
+      float st[PER];
+      load_state(ck + (size_t)c * SS, st);
+      for (int64_t t = t0; t < t1; ++t) {
+        const int buf = (it++) & 1;
+        stage(t, buf);
+        __syncthreads();
+        store_state(scr + (size_t)(t - t0) * SS, st);
+        advance(st, buf);
+      }
+      store_state(scr + (size_t)(t1 - t0) * SS, st);
+    }
+    for (int64_t t = t1 - 1; t >= t0; --t) {
+      const int buf = (it++) & 1;
+      stage(t, buf);
+      __syncthreads();
+      const float* tb = tok + buf * 4 * D;
+      const float* kv = tb + part * PER;
+      const float* qv = tb + D + part * PER;
+      const float vj = tb[2 * D + col], dOj = tb[3 * D + col];
+      const float alpha = gates[2 * buf], beta = gates[2 * buf + 1];
+      const size_t th = (size_t)t * a.H + h, tq = (size_t)t * a.Hqk + hq;
+      float sp[PER];  // S_{t-1}
+      load_state(scr + (size_t)(t - t0) * SS, sp);
+      // D += scale q dO^T
+#pragma unroll
+      for (int x = 0; x < PER; ++x) Dm[x] = fmaf(a.scale * qv[x], dOj, Dm[x]);
+      // u = S~^T k (S~ = alpha S_{t-1}), w = D^T k, column j
+      float pu = 0.f, pw = 0.f;
+#pragma unroll
+      for (int x = 0; x < PER; ++x) {
+        pu = fmaf(kv[x], sp[x], pu);
+        pw = fmaf(kv[x], Dm[x], pw);
+      }
+#pragma unroll
+      for (int off = 1; off < TPC; off <<= 1) {
+        pu += __shfl_xor_sync(0xffffffffu, pu, off);
+        pw += __shfl_xor_sync(0xffffffffu, pw, off);
+      }
+      const float u = alpha * pu, w = pw, vmu = vj - u;
+      // column j's terms of dq (S_t dO) and dk (D (v - u) - S~ w), and of dg
+      const float* sc = scr + (size_t)(t - t0 + 1) * SS;  // S_t
+      float* rq = red_q + (size_t)col * D + part * PER;
+      float* rk = red_k + (size_t)col * D + part * PER;
+      float sdg = 0.f;
+#pragma unroll
+      for (int x = 0; x < PER; x += 4) {
+        const float4 s4 = *reinterpret_cast<const float4*>(sc + x);
+        *reinterpret_cast<float4*>(rq + x) = make_float4(s4.x * dOj, s4.y * dOj, s4.z * dOj, s4.w * dOj);
+        float kk[4];
+#pragma unroll
+        for (int y = 0; y < 4; ++y) {
+          const float stl = alpha * sp[x + y];
+          kk[y] = Dm[x + y] * vmu - stl * w;
+          sdg = fmaf(Dm[x + y], stl, sdg);
+        }
+        *reinterpret_cast<float4*>(rk + x) = make_float4(kk[0], kk[1], kk[2], kk[3]);
+      }
+      float sdb = 0.f;
+      if (part == 0) {
+        sdg -= beta * u * w;
+        sdb = w * vmu;
+        a.dv[th * D + col] = beta * w;
+      }
+      // dL/dS_{t-1}
+#pragma unroll
+      for (int x = 0; x < PER; ++x) Dm[x] = alpha * (Dm[x] - beta * w * kv[x]);
+#pragma unroll
+      for (int off = 16; off > 0; off >>= 1) {
+        sdg += __shfl_xor_sync(0xffffffffu, sdg, off);
+        sdb += __shfl_xor_sync(0xffffffffu, sdb, off);
+      }
+      if ((tid & 31) == 0) {
+        red_s[2 * (tid >> 5)] = sdg;
+        red_s[2 * (tid >> 5) + 1] = sdb;
+      }
+      __syncthreads();
+      for (int o = tid; o < 2 * D; o += NT) {
+        const float* r = (o < D) ? red_q : red_k;
+        const int i = (o < D) ? o : o - D;
+        float s = 0.f;
+        for (int j = 0; j < D; ++j) s += r[(size_t)j * D + i];
+        if (o < D)
+          atomicAdd(a.dq + tq * D + i, a.scale * s);
+        else
+          atomicAdd(a.dk + tq * D + i, beta * s);
+      }
+      if (tid == 0) {
+        float g_sum = 0.f, b_sum = 0.f;
+        for (int wi = 0; wi < NW; ++wi) {
+          g_sum += red_s[2 * wi];
+          b_sum += red_s[2 * wi + 1];
+        }
+        a.dg[th] = g_sum;
+        a.dbeta[th] = b_sum;
+      }
+    }
+  }
+  if (a.d_init) store_state(a.d_init + state_off, Dm);
+}
+
+template <int D, typename TIn>
+gdn_status_t launch_bwd(const BwdArgs& a, cudaStream_t stream) {
+  auto kernel = gdn_prefill_backward_kernel<D, TIn>;
+  constexpr size_t smem = bwd_smem_bytes<D>();
+  static PerDeviceOnce once;  // the shared-memory opt-in applies to the current device only
+  int dev = 0;
+  cudaError_t e = cudaGetDevice(&dev);
+  if (e != cudaSuccess) return fail(GDN_ERR_CUDA, std::string("prefill backward: cudaGetDevice: ") + cudaGetErrorString(e));
+  if (!run_once_per_device(once, dev, [&](int, int*) {
+        e = cudaFuncSetAttribute(kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
+        return e == cudaSuccess;
+      }))
+    return fail(e != cudaSuccess ? GDN_ERR_CUDA : GDN_ERR_UNSUPPORTED,
+                std::string("prefill backward: setup: ") + (e != cudaSuccess ? cudaGetErrorString(e) : "device index too large"));
+  kernel<<<(unsigned)((long long)a.N * a.H), D * (D / 32), smem, stream>>>(a);
+  return check_launch("gdn_chunk_prefill_backward");
+}
+
+}  // namespace
+}  // namespace gdn
+
+using gdn::fail;
+
+namespace {
+
+gdn_status_t bwd_check_shape(int N, int64_t total_T, int H, int dk, int dv, int chunk) {
+  if (N < 0 || total_T < 0 || H < 1 || chunk < 1)
+    return fail(GDN_ERR_INVALID_ARG, "gdn_chunk_prefill_backward: need N >= 0, total_T >= 0, H >= 1, chunk >= 1");
+  if (dk != dv || (dk != 32 && dk != 64 && dk != 128))
+    return fail(GDN_ERR_UNSUPPORTED, "gdn_chunk_prefill_backward: dk == dv in {32, 64, 128}");
+  if (chunk > 4096) return fail(GDN_ERR_UNSUPPORTED, "gdn_chunk_prefill_backward: chunk <= 4096");
+  if ((long long)N * H >= (1LL << 31)) return fail(GDN_ERR_UNSUPPORTED, "gdn_chunk_prefill_backward: N * H too large");
+  return gdn::ok();
+}
+
+bool ptr_ok(const void* p) { return p != nullptr && gdn::aligned16(p); }
+
+}  // namespace
+
+extern "C" gdn_status_t gdn_chunk_prefill_backward_workspace_size(int N, int64_t total_T, int H, int dk, int dv,
+                                                                  int chunk, size_t* bytes) {
+  if (!bytes) return fail(GDN_ERR_INVALID_ARG, "gdn_chunk_prefill_backward_workspace_size: bytes is NULL");
+  const gdn_status_t st = bwd_check_shape(N, total_T, H, dk, dv, chunk);
+  if (st != GDN_OK) return st;
+  *bytes = gdn::bwd_layout(N, total_T, H, dk, chunk).bytes;
+  return gdn::ok();
+}
+
+extern "C" gdn_status_t gdn_chunk_prefill_backward(
+    const void* q, const void* k, const void* v, const float* g, const float* beta, const int32_t* cu_seqlens, int N,
+    int64_t total_T, const float* initial_state, const void* d_o, const float* d_final_state, float* d_q, float* d_k,
+    float* d_v, float* d_g, float* d_beta, float* d_initial_state, int H, int H_qk, int dk, int dv, int chunk,
+    float scale, uint32_t flags, gdn_dtype_t in_dtype, void* workspace, size_t workspace_bytes, void* stream) {
+  gdn_status_t st = bwd_check_shape(N, total_T, H, dk, dv, chunk);
+  if (st != GDN_OK) return st;
+  if (H_qk < 1 || H % H_qk != 0)
+    return fail(GDN_ERR_INVALID_ARG, "gdn_chunk_prefill_backward: H must be a positive multiple of H_qk");
+  if (flags != 0) return fail(GDN_ERR_UNSUPPORTED, "gdn_chunk_prefill_backward: no flags supported (q/k normalisation)");
+  if (!(in_dtype == GDN_BF16 || in_dtype == GDN_F32))
+    return fail(GDN_ERR_INVALID_ARG, "gdn_chunk_prefill_backward: unknown dtype");
+  if (N == 0) return gdn::ok();
+  if (cu_seqlens == nullptr) return fail(GDN_ERR_INVALID_ARG, "gdn_chunk_prefill_backward: cu_seqlens is NULL");
+  if (total_T > 0 && (!ptr_ok(q) || !ptr_ok(k) || !ptr_ok(v) || !ptr_ok(d_o) || g == nullptr || beta == nullptr ||
+                      !ptr_ok(d_q) || !ptr_ok(d_k) || d_v == nullptr || d_g == nullptr || d_beta == nullptr))
+    return fail(GDN_ERR_INVALID_ARG,
+                "gdn_chunk_prefill_backward: q, k, v, d_o, d_q, d_k must be non-NULL and 16-byte aligned; "
+                "g, beta, d_v, d_g, d_beta non-NULL");
+  if ((initial_state && !ptr_ok(initial_state)) || (d_final_state && !ptr_ok(d_final_state)) ||
+      (d_initial_state && !ptr_ok(d_initial_state)))
+    return fail(GDN_ERR_INVALID_ARG, "gdn_chunk_prefill_backward: state pointers must be 16-byte aligned");
+  const gdn::BwdLayout L = gdn::bwd_layout(N, total_T, H, dk, chunk);
+  if (workspace == nullptr || workspace_bytes < L.bytes || !gdn::aligned16(workspace))
+    return fail(GDN_ERR_WORKSPACE, "gdn_chunk_prefill_backward: workspace missing, misaligned or smaller than "
+                                   "gdn_chunk_prefill_backward_workspace_size");
+  unsigned int* err = nullptr;
+  st = gdn::device_error_word(&err);
+  if (st != GDN_OK) return st;
+  cudaStream_t s = gdn::as_stream(stream);
+  if (total_T > 0) {
+    const size_t qk_bytes = (size_t)total_T * H_qk * dk * sizeof(float);
+    cudaError_t e = cudaMemsetAsync(d_q, 0, qk_bytes, s);
+    if (e == cudaSuccess) e = cudaMemsetAsync(d_k, 0, qk_bytes, s);
+    if (e != cudaSuccess)
+      return fail(GDN_ERR_CUDA, std::string("gdn_chunk_prefill_backward: clearing d_q, d_k: ") + cudaGetErrorString(e));
+  }
+  gdn::BwdArgs a;
+  a.q = q; a.k = k; a.v = v; a.d_o = d_o; a.g = g; a.beta = beta; a.cu = cu_seqlens;
+  a.init = initial_state; a.d_fin = d_final_state;
+  a.dq = d_q; a.dk = d_k; a.dv = d_v; a.dg = d_g; a.dbeta = d_beta; a.d_init = d_initial_state;
+  a.ckpt = static_cast<float*>(workspace);
+  a.scratch = reinterpret_cast<float*>(static_cast<uint8_t*>(workspace) + L.scratch_off);
+  a.ck_slots = L.ck_slots;
+  a.total_T = total_T; a.N = N; a.H = H; a.Hqk = H_qk; a.C = chunk; a.scale = scale; a.err = err;
+  const bool bf = in_dtype == GDN_BF16;
+  switch (dk) {
+    case 32: return bf ? gdn::launch_bwd<32, __nv_bfloat16>(a, s) : gdn::launch_bwd<32, float>(a, s);
+    case 64: return bf ? gdn::launch_bwd<64, __nv_bfloat16>(a, s) : gdn::launch_bwd<64, float>(a, s);
+    default: return bf ? gdn::launch_bwd<128, __nv_bfloat16>(a, s) : gdn::launch_bwd<128, float>(a, s);
+  }
+}

@@ -246,6 +246,43 @@ gdn_status_t gdn_cp_combine(const float* local_states, const float* transfers, i
 const char* gdn_last_error(void);
 
 /*
+ * gdn_chunk_prefill_backward — derivatives of a loss L with respect to the inputs
+ * of gdn_chunk_prefill, given dL/do (d_o) and dL/dS_final (d_final_state, NULL =
+ * zero), for training. The pages give no backward pass: this is the chain rule on
+ * the gated delta rule's token relations S_t = alpha_t (I - beta_t k_t k_t^T)
+ * S_{t-1} + beta_t k_t v_t^T, o_t = scale S_t^T q_t, alpha_t = exp(g_t), walked from
+ * the last token to the first (one Householder per token; no q/k normalisation).
+ *
+ * Inputs as gdn_chunk_prefill (q, k [total_T, H_qk, dk]; v [total_T, H, dv]; g, beta
+ * [total_T, H] fp32; cu_seqlens [N+1] int32 on the device; initial_state [N, H, dv,
+ * dk] fp32 K-last or NULL), plus d_o [total_T, H, dv] in in_dtype. Outputs, fp32,
+ * caller-owned: d_q, d_k [total_T, H_qk, dk] (value heads that share a q/k head add
+ * up; both are cleared on `stream` first), d_v [total_T, H, dv], d_g, d_beta
+ * [total_T, H], d_initial_state [N, H, dv, dk] K-last or NULL (not written).
+ * dk == dv in {32, 64, 128}; flags must be 0 (GDN_ERR_UNSUPPORTED otherwise);
+ * q, k, v, d_o, d_q, d_k and the state pointers 16-byte aligned.
+ *
+ * One CTA per (sequence, head), token-sequential: a forward pass writes the state at
+ * the start of every `chunk` tokens to the workspace, then each chunk, last to first,
+ * is recomputed from its checkpoint into the workspace and walked backwards. The
+ * workspace (gdn_chunk_prefill_backward_workspace_size; 16-byte aligned, contents
+ * need no clearing) holds H x (total_T / chunk + N + 1) checkpoints and N x H x
+ * (chunk + 1) recomputed states of dk x dv fp32. Errors: GDN_ERR_INVALID_ARG /
+ * GDN_ERR_UNSUPPORTED / GDN_ERR_WORKSPACE before anything is launched; a malformed
+ * cu_seqlens pair sets GDN_DEVERR_BAD_CU_SEQLENS and skips that sequence. Only
+ * enqueues on `stream` (two memsets and one kernel).
+ */
+gdn_status_t gdn_chunk_prefill_backward_workspace_size(int N, int64_t total_T, int H, int dk, int dv, int chunk,
+                                                       size_t* bytes);
+gdn_status_t gdn_chunk_prefill_backward(const void* q, const void* k, const void* v, const float* g,
+                                        const float* beta, const int32_t* cu_seqlens, int N, int64_t total_T,
+                                        const float* initial_state, const void* d_o, const float* d_final_state,
+                                        float* d_q, float* d_k, float* d_v, float* d_g, float* d_beta,
+                                        float* d_initial_state, int H, int H_qk, int dk, int dv, int chunk,
+                                        float scale, uint32_t flags, gdn_dtype_t in_dtype, void* workspace,
+                                        size_t workspace_bytes, void* stream);
+
+/*
  * gdn_get_device_error — read and clear the sticky device error word of the
  * current CUDA device (GDN_DEVERR_* bits). Synchronous: waits for all prior work
  * on the device. Returns GDN_OK when the word was 0, GDN_ERR_DEVICE_DATA when a

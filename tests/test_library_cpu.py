@@ -153,3 +153,33 @@ def test_cp_entry_points_reject_on_host(L):
                                 gdn.GDN_BF16, None) == gdn.GDN_ERR_UNSUPPORTED  # chunk 32
     assert L.gdn_cp_local_state(FAKE, FAKE, FAKE, FAKE, FAKE, FAKE, 1, 64, None, FAKE, 2, 2, 128, 128, 64, 0,
                                 gdn.GDN_BF16, None) == gdn.GDN_ERR_INVALID_ARG
+
+
+def test_backward_entry_points_reject_on_host(L):
+    size = ctypes.c_size_t(0)
+    assert L.gdn_chunk_prefill_backward_workspace_size(2, 100, 4, 128, 128, 64, ctypes.byref(size)) == gdn.GDN_OK
+    # 4 heads x (100 // 64 + 2 + 1) checkpoints + 2 x 4 x 65 scratch states of 64 KiB
+    assert size.value >= (4 * 4 + 2 * 4 * 65) * 128 * 128 * 4
+    assert L.gdn_chunk_prefill_backward_workspace_size(2, 100, 4, 128, 64, 64, ctypes.byref(size)) == \
+        gdn.GDN_ERR_UNSUPPORTED  # dk != dv
+    assert L.gdn_chunk_prefill_backward_workspace_size(2, 100, 4, 96, 96, 64, ctypes.byref(size)) == \
+        gdn.GDN_ERR_UNSUPPORTED
+    assert L.gdn_chunk_prefill_backward_workspace_size(2, 100, 4, 128, 128, 0, ctypes.byref(size)) == \
+        gdn.GDN_ERR_INVALID_ARG
+
+    def call(**kw):
+        a = dict(q=FAKE, k=FAKE, v=FAKE, g=FAKE, beta=FAKE, cu=FAKE, N=2, T=100, init=None, d_o=FAKE, dfin=None,
+                 dq=FAKE, dk_=FAKE, dv_=FAKE, dg=FAKE, db=FAKE, dinit=None, H=4, Hqk=2, dk=128, dv=128, chunk=64,
+                 scale=0.1, flags=0, dt=gdn.GDN_BF16, ws=FAKE, wsb=1 << 40, stream=None)
+        a.update(kw)
+        return L.gdn_chunk_prefill_backward(a["q"], a["k"], a["v"], a["g"], a["beta"], a["cu"], a["N"], a["T"],
+                                            a["init"], a["d_o"], a["dfin"], a["dq"], a["dk_"], a["dv_"], a["dg"],
+                                            a["db"], a["dinit"], a["H"], a["Hqk"], a["dk"], a["dv"], a["chunk"],
+                                            a["scale"], a["flags"], a["dt"], a["ws"], a["wsb"], a["stream"])
+    assert call(flags=gdn.GDN_QK_L2NORM) == gdn.GDN_ERR_UNSUPPORTED
+    assert call(Hqk=3) == gdn.GDN_ERR_INVALID_ARG
+    assert call(d_o=None) == gdn.GDN_ERR_INVALID_ARG
+    assert call(dq=FAKE + 4) == gdn.GDN_ERR_INVALID_ARG  # misaligned
+    assert call(wsb=16) == gdn.GDN_ERR_WORKSPACE
+    assert call(ws=None) == gdn.GDN_ERR_WORKSPACE
+    assert call(N=0) == gdn.GDN_OK  # nothing to do, nothing launched
