@@ -460,6 +460,71 @@ def bench_prefill(key, steps, warmup, ws, rank, peaks, algo=None):
     return res
 
 
+def backward_alg_bytes(inp):
+    """Algorithmic HBM bytes of one backward step: q, k, v and d_o read (input dtype),
+    g and beta read, dq, dk, dv, dg, dbeta written (fp32), and per (sequence, head) the
+    initial state and the final-state derivative read and the initial-state
+    derivative written (fp32)."""
+    total, Hqk, dk = inp.q.shape
+    H, dv = inp.v.shape[1], inp.v.shape[-1]
+    N = inp.cu_seqlens.numel() - 1
+    es = inp.q.element_size()
+    per_tok = Hqk * 2 * dk * (es + 4) + H * (2 * dv * es + 8 + dv * 4 + 8)
+    return total * per_tok + 3 * N * H * dk * dv * 4
+
+
+def backward_inputs(key, device, seed):
+    """The backward part runs on the chunked-prefill workload with seeded upstream
+    derivatives d_o (bf16, N(0, 1)) and d_final_state (fp32, N(0, 0.1^2))."""
+    inp, chunk, name = prefill_cfg("prefill", device, seed)
+    gen = torch.Generator(device=device).manual_seed(seed + 7)
+    total, H, dv = inp.v.shape
+    N = inp.cu_seqlens.numel() - 1
+    d_o = torch.randn((total, H, dv), generator=gen, device=device).to(inp.q.dtype)
+    d_fin = torch.randn((N, H, dv, inp.q.shape[-1]), generator=gen, device=device) * 0.1
+    return inp, d_o, d_fin, chunk, "prefill backward (dq, dk, dv, dg, dbeta, d_initial_state), " + name
+
+
+def bench_backward(key, steps, warmup, ws, rank, peaks):
+    import gated_delta_rule_58_b200 as gdn
+    dev = torch.device("cuda", torch.cuda.current_device())
+    inp, d_o, d_fin, chunk, name = backward_inputs(key, dev, rank)
+    total, Hqk, dk = inp.q.shape
+    H, dv = inp.v.shape[1], inp.v.shape[-1]
+    N = inp.cu_seqlens.numel() - 1
+    f = dict(dtype=torch.float32, device=dev)
+    grads = dict(dq=torch.empty((total, Hqk, dk), **f), dk=torch.empty((total, Hqk, dk), **f),
+                 dv=torch.empty((total, H, dv), **f), dg=torch.empty((total, H), **f),
+                 dbeta=torch.empty((total, H), **f), d_initial_state=torch.empty((N, H, dv, dk), **f))
+    ws_bytes = gdn.gdn_chunk_prefill_backward_workspace_size(N, total, H, dk, dv, chunk)
+    work = torch.empty(ws_bytes, dtype=torch.uint8, device=dev)
+
+    def step(i):
+        gdn.gdn_chunk_prefill_backward(inp.q, inp.k, inp.v, inp.g, inp.beta, inp.cu_seqlens, d_o,
+                                       initial_state=inp.initial_state, d_final_state=d_fin, chunk=chunk,
+                                       scale=inp.scale, workspace=work, grads=grads)
+
+    total_ms, per = time_launches(step, steps, warmup, ws)
+    ms = total_ms / steps
+    t = ms * 1e-3
+    alg_b = backward_alg_bytes(inp)
+    achieved = alg_b / t / 1e9
+    res = {
+        "workload": name,
+        "algo": "token-sequential with chunk checkpoints",
+        "ms_per_step": ms,
+        "tokens_per_s": total / t * ws,
+        "roofline": {"bound": "hbm", "achieved": achieved, "peak": peaks["hbm_gbs"], "unit": "GB/s",
+                     "frac": achieved / peaks["hbm_gbs"], "traffic": ncu_traffic(key)},
+        "pct_of_nominal_roofline": alg_b / (NOMINAL_HBM_GBS * 1e9) / t * 100,
+        "alg_bytes": alg_b,
+        "workspace_bytes": ws_bytes,
+    }
+    del inp, d_o, d_fin, grads, work
+    torch.cuda.empty_cache()
+    return res
+
+
 # ---------------------------------------------------------------- CPU oracle (baseline / reference arm)
 
 class OracleDecode:
@@ -559,6 +624,39 @@ def oracle_prefill_rate(key, budget_s=4.0, seed=0):
             f"({tokens // reps} tokens{rep}) of '{name}', {dt:.1f} s{note}")
 
 
+def oracle_backward_rate(key, budget_s=4.0, seed=0):
+    """cpu_baseline of the backward part: the fp64 oracle's backward on the first L
+    tokens of every sequence (all heads), L sized from a calibration call so the timed
+    call takes about budget_s. Returns tokens/s, threads used and the sample."""
+    import numpy as np
+    import oracle
+    gen_dev = "cuda" if torch.cuda.is_available() else "cpu"
+    inp, d_o, d_fin, _, name = backward_inputs(key, gen_dev, seed)
+    cu = inp.cu_seqlens.tolist()
+    N = len(cu) - 1
+    H = inp.v.shape[1]
+    longest = max(cu[n + 1] - cu[n] for n in range(N))
+
+    def timed(L):
+        lens = [min(L, cu[n + 1] - cu[n]) for n in range(N)]
+        idx = torch.cat([torch.arange(cu[n], cu[n] + lens[n]) for n in range(N)]).to(inp.q.device)
+        new_cu = np.concatenate([[0], np.cumsum(lens)]).astype(np.int64)
+        args = [oracle.f64(t[idx]) for t in (inp.q, inp.k, inp.v, inp.g, inp.beta)]
+        t0 = time.perf_counter()
+        oracle.prefill_backward(*args, new_cu, oracle.f64(d_o[idx]), oracle.f64(inp.initial_state),
+                                oracle.f64(d_fin), scale=inp.scale)
+        return time.perf_counter() - t0, int(new_cu[-1])
+
+    L = min(16, longest)
+    dt, tokens = timed(L)
+    L = max(L, min(longest, int(L * budget_s / max(dt, 1e-3))))
+    dt, tokens = timed(L)
+    threads = min(os.cpu_count() or 1, N * H)
+    return (tokens / dt, threads,
+            f"oracle backward on the first {L} tokens of each of the {N} sequences x {H} heads "
+            f"({tokens} tokens) of '{name}', {dt:.1f} s")
+
+
 def run_reference(args, ws, rank):
     """The reference arm: the fp64 CPU oracle on the headline workload, on rank 0 only.
     Each step is a bounded sample (the first rows of the batch, all heads), sized so the
@@ -596,7 +694,7 @@ def main():
     ap.add_argument("--steps", type=int, default=2000)
     ap.add_argument("--warmup", type=int, default=20)
     ap.add_argument("--impl", default="ours", choices=["ours", "reference"])
-    ap.add_argument("--parts", default="gdp,decode_b1,decode_b4,decode_b16,prefill,varlen,longseq,tiny",
+    ap.add_argument("--parts", default="gdp,decode_b1,decode_b4,decode_b16,prefill,varlen,longseq,tiny,backward",
                     help="comma list of extra workloads to measure ('none' for none)")
     ap.add_argument("--part-steps", type=int, default=5,
                     help="timed steps of each prefill part (decode parts: 20 times this, at least 20)")
@@ -638,6 +736,9 @@ def main():
                     r = bench_decode(key, max(args.part_steps * 20, 20), args.warmup, ws, rank, peaks,
                                      e2e=False)
                     r["metric"] = "GDP decode state GB/s" if key == "gdp" else "decode state GB/s"
+                elif key == "backward":
+                    r = bench_backward(key, max(args.part_steps // 2, 1), 3, ws, rank, peaks)
+                    r["metric"] = "backward tokens/s"
                 else:
                     r = bench_prefill(key, args.part_steps, 3, ws, rank, peaks, algo=algo)
                     r["metric"] = "prefill tokens/s"
@@ -662,6 +763,10 @@ def main():
                 if r["key"] in DECODE_CFGS:
                     v, threads, sample = oracle_decode_rate(r["key"], budget_s=2.0 if r["key"] != "gdp" else 4.0)
                     r["cpu_baseline"] = {"value": v, "unit": "GB/s", "cores": threads, "kind": "oracle",
+                                         "sample": sample}
+                elif r["key"] == "backward":
+                    v, threads, sample = oracle_backward_rate(r["key"], budget_s=4.0)
+                    r["cpu_baseline"] = {"value": v, "unit": "tokens/s", "cores": threads, "kind": "oracle",
                                          "sample": sample}
                 else:
                     v, threads, sample = oracle_prefill_rate(r["key"], budget_s=4.0)

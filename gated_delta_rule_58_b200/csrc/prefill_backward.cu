@@ -17,13 +17,18 @@
 //   1. forward over the sequence, writing the state at the start of every chunk of
 //      C tokens to the workspace (checkpoints);
 //   2. for each chunk, last to first: recompute the chunk's states from its
-//      checkpoint into a per-CTA scratch (C + 1 states), then walk its tokens
-//      backwards reading S_{t-1} and S_t from there (a thread reads back only what it
-//      wrote, so no barrier orders the scratch).
+//      checkpoint into a per-CTA scratch (the state before each of its tokens), then
+//      walk its tokens backwards reading S_{t-1} from there (a thread reads back only
+//      what it wrote, so no barrier orders the scratch).
 // Per token the column sums of dq and dk go through shared memory (each thread
 // writes its 32 partial products, then 2 dk threads each add one entry over the dv
 // columns); dg and dbeta are block reductions. dq and dk are accumulated with fp32
 // atomics into zeroed outputs, so value heads that share a q/k head add up.
+// Latency: the next token's k, q, v, dO and gates are loaded into registers while
+// the current token computes; in the backward walk S_t is the previous token's
+// S_{t-1} (kept in registers) and the next S_{t-1} is fetched from the scratch into
+// shared memory by cp.async while the current token computes (each thread copies and
+// reads only its own entries).
 #include <string>
 
 #include "device_once.h"
@@ -74,11 +79,25 @@ BwdLayout bwd_layout(int N, int64_t total_T, int H, int D, int C) {
   return L;
 }
 
+// Shared-memory stride of one column in the [D columns][D entries] buffers, padded
+// so that the eight lanes of a quarter warp (two columns x four 16-byte pieces)
+// store to distinct banks.
+template <int D>
+constexpr int bwd_col_stride() { return D + 16; }
+
 template <int D>
 constexpr size_t bwd_smem_bytes() {
   // token vectors [2][k, q, v, dO][D], gates [2][alpha, beta], column partials of dq
-  // and dk [D][D] each, scalar partials [warps][2]
-  return (8 * D + 4 + 2 * D * D + 2 * (D * (D / 32) / 32)) * sizeof(float);
+  // and dk and the prefetched S_{t-1} ([D][stride] each), scalar partials [warps][2]
+  return (8 * D + 4 + 3 * D * bwd_col_stride<D>() + 2 * (D * (D / 32) / 32)) * sizeof(float);
+}
+
+__device__ __forceinline__ void cp_async16(float* dst, const float* src) {
+  const uint32_t d = (uint32_t)__cvta_generic_to_shared(dst);
+  asm volatile("cp.async.cg.shared.global [%0], [%1], 16;" ::"r"(d), "l"(src) : "memory");
+}
+__device__ __forceinline__ void cp_async_wait_all() {
+  asm volatile("cp.async.commit_group;\ncp.async.wait_group 0;" ::: "memory");
 }
 
 template <int D, typename TIn>
@@ -87,52 +106,82 @@ gdn_prefill_backward_kernel(const BwdArgs a) {
   constexpr int TPC = D / 32;  // threads per state column
   constexpr int NT = D * TPC;
   constexpr int PER = 32;      // entries of the column per thread
+  constexpr int NP = PER / 4;  // 16-byte pieces per thread
   constexpr int NW = NT / 32;
+  constexpr int RS = bwd_col_stride<D>();
   extern __shared__ __align__(16) float bsm[];
-  float* tok = bsm;              // [2][4][D]
-  float* gates = tok + 8 * D;    // [2][2]
-  float* red_q = gates + 4;      // [D columns][D entries]
-  float* red_k = red_q + D * D;
-  float* red_s = red_k + D * D;  // [NW][2]
+  float* tok = bsm;               // [2][4][D]
+  float* gates = tok + 8 * D;     // [2][2]
+  float* red_q = gates + 4;       // [D columns][RS]
+  float* red_k = red_q + D * RS;
+  float* sp_buf = red_k + D * RS;  // [D][RS]: the next S_{t-1}, each thread its own entries
+  float* red_s = sp_buf + D * RS;  // [NW][2]
 
   const int tid = threadIdx.x;
   const int col = tid / TPC, part = tid % TPC;
+  // this thread's entries of column col: the 16-byte pieces part, part + TPC, ...,
+  // i.e. entries 4 (part + TPC y) + z, y < NP, z < 4 (local index x = 4 y + z)
+  auto piece = [&](int y) { return 4 * (part + TPC * y); };
   const int n = blockIdx.x / a.H, h = blockIdx.x - n * a.H;
   const int hq = h / (a.H / a.Hqk);
   int64_t bos, eos;
   if (!seq_bounds(a.cu, n, a.total_T, a.err, &bos, &eos)) return;
   const int nck = (int)((eos - bos + a.C - 1) / a.C);
   const size_t SS = (size_t)D * D;
-  const size_t mine = (size_t)col * D + part * PER;  // this thread's entries of a K-last state
-  const size_t state_off = ((size_t)n * a.H + h) * SS + mine;
-  float* ck = a.ckpt + ((size_t)h * a.ck_slots + (size_t)(bos / a.C) + n) * SS + mine;
-  float* scr = a.scratch + (size_t)blockIdx.x * (size_t)(a.C + 1) * SS + mine;
+  const size_t state_off = ((size_t)n * a.H + h) * SS + (size_t)col * D;
+  float* ck = a.ckpt + ((size_t)h * a.ck_slots + (size_t)(bos / a.C) + n) * SS + (size_t)col * D;
+  float* scr = a.scratch + (size_t)blockIdx.x * (size_t)(a.C + 1) * SS + (size_t)col * D;
+  float* spb = sp_buf + col * RS;
   const TIn* qp = static_cast<const TIn*>(a.q);
   const TIn* kp = static_cast<const TIn*>(a.k);
   const TIn* vp = static_cast<const TIn*>(a.v);
   const TIn* dop = static_cast<const TIn*>(a.d_o);
 
-  // token t's k, q, v, dO and gates into buffer `buf` (two buffers: the barrier of
-  // the token in between orders every read of a buffer before its refill)
-  auto stage = [&](int64_t t, int buf) {
+  // A token's k, q, v, dO (thread tid < D holds element tid; NT >= D) and gates are
+  // fetched into registers, then committed to shared-memory buffer `buf` (two
+  // buffers: the barrier of the token in between orders every read of a buffer
+  // before its refill).
+  float fk = 0.f, fq = 0.f, fv = 0.f, fdo = 0.f, fg = 0.f, fb = 0.f;
+  auto fetch = [&](int64_t t) {
     const size_t th = (size_t)t * a.H + h, tq = (size_t)t * a.Hqk + hq;
-    float* tb = tok + buf * 4 * D;
-    for (int i = tid; i < D; i += NT) {
-      tb[i] = to_f32(kp[tq * D + i]);
-      tb[D + i] = to_f32(qp[tq * D + i]);
-      tb[2 * D + i] = to_f32(vp[th * D + i]);
-      tb[3 * D + i] = to_f32(dop[th * D + i]);
+    if (tid < D) {
+      fk = to_f32(kp[tq * D + tid]);
+      fq = to_f32(qp[tq * D + tid]);
+      fv = to_f32(vp[th * D + tid]);
+      fdo = to_f32(dop[th * D + tid]);
     }
     if (tid == 0) {
-      gates[2 * buf] = expf(a.g[th]);
-      gates[2 * buf + 1] = a.beta[th];
+      fg = a.g[th];
+      fb = a.beta[th];
+    }
+  };
+  auto commit = [&](int buf) {
+    float* tb = tok + buf * 4 * D;
+    if (tid < D) {
+      tb[tid] = fk;
+      tb[D + tid] = fq;
+      tb[2 * D + tid] = fv;
+      tb[3 * D + tid] = fdo;
+    }
+    if (tid == 0) {
+      gates[2 * buf] = expf(fg);
+      gates[2 * buf + 1] = fb;
+    }
+  };
+  // this thread's entries of a D-vector in shared memory
+  auto load_vec = [&](const float* v, float* out) {
+#pragma unroll
+    for (int y = 0; y < NP; ++y) {
+      const float4 f = *reinterpret_cast<const float4*>(v + piece(y));
+      out[4 * y] = f.x; out[4 * y + 1] = f.y; out[4 * y + 2] = f.z; out[4 * y + 3] = f.w;
     }
   };
   // one token forward on this thread's entries of column col (as the forward kernel)
   auto advance = [&](float* st, int buf) {
     const float* tb = tok + buf * 4 * D;
-    const float* kv = tb + part * PER;
     const float alpha = gates[2 * buf], beta = gates[2 * buf + 1];
+    float kv[PER];
+    load_vec(tb, kv);
     float u = 0.f;
 #pragma unroll
     for (int x = 0; x < PER; ++x) u = fmaf(kv[x], st[x], u);
@@ -142,17 +191,22 @@ gdn_prefill_backward_kernel(const BwdArgs a) {
 #pragma unroll
     for (int x = 0; x < PER; ++x) st[x] = fmaf(alpha, st[x], c * kv[x]);
   };
+  // a state column's entries of this thread from / to memory (p = the column's base)
   auto load_state = [&](const float* p, float* st) {
 #pragma unroll
-    for (int x = 0; x < PER; x += 4) {
-      const float4 f = *reinterpret_cast<const float4*>(p + x);
-      st[x] = f.x; st[x + 1] = f.y; st[x + 2] = f.z; st[x + 3] = f.w;
+    for (int y = 0; y < NP; ++y) {
+      const float4 f = *reinterpret_cast<const float4*>(p + piece(y));
+      st[4 * y] = f.x; st[4 * y + 1] = f.y; st[4 * y + 2] = f.z; st[4 * y + 3] = f.w;
     }
   };
   auto store_state = [&](float* p, const float* st) {
 #pragma unroll
-    for (int x = 0; x < PER; x += 4)
-      *reinterpret_cast<float4*>(p + x) = make_float4(st[x], st[x + 1], st[x + 2], st[x + 3]);
+    for (int y = 0; y < NP; ++y)
+      *reinterpret_cast<float4*>(p + piece(y)) = make_float4(st[4 * y], st[4 * y + 1], st[4 * y + 2], st[4 * y + 3]);
+  };
+  auto prefetch_state = [&](const float* p) {  // this thread's entries -> sp_buf, asynchronously
+#pragma unroll
+    for (int y = 0; y < NP; ++y) cp_async16(spb + piece(y), p + piece(y));
   };
 
   // 1. forward with a checkpoint at the start of every chunk
@@ -165,9 +219,11 @@ gdn_prefill_backward_kernel(const BwdArgs a) {
 #pragma unroll
       for (int x = 0; x < PER; ++x) st[x] = 0.f;
     }
+    if (bos < eos) fetch(bos);
     for (int64_t t = bos; t < eos; ++t) {
       const int buf = (it++) & 1;
-      stage(t, buf);
+      commit(buf);
+      if (t + 1 < eos) fetch(t + 1);
       __syncthreads();
       if ((t - bos) % a.C == 0) store_state(ck + (size_t)((t - bos) / a.C) * SS, st);
       advance(st, buf);
@@ -185,34 +241,52 @@ gdn_prefill_backward_kernel(const BwdArgs a) {
   for (int c = nck - 1; c >= 0; --c) {
     const int64_t t0 = bos + (int64_t)c * a.C;
     const int64_t t1 = (t0 + a.C < eos) ? t0 + a.C : eos;
+    float sc[PER];  // S_t of the token being walked
     {
-      // scratch slot x = the state before token t0 + x; slot t1 - t0 = after the chunk
-      float st[PER];
-      load_state(ck + (size_t)c * SS, st);
+      // scratch slot x = the state before token t0 + x
+      load_state(ck + (size_t)c * SS, sc);
+      fetch(t0);
       for (int64_t t = t0; t < t1; ++t) {
         const int buf = (it++) & 1;
-        stage(t, buf);
+        commit(buf);
+        if (t + 1 < t1) fetch(t + 1);
         __syncthreads();
-        store_state(scr + (size_t)(t - t0) * SS, st);
-        advance(st, buf);
+        store_state(scr + (size_t)(t - t0) * SS, sc);
+        advance(sc, buf);
       }
-      store_state(scr + (size_t)(t1 - t0) * SS, st);
     }
+    // sc = the state after the chunk's last token; its S_{t-1} goes into sp_buf
+    prefetch_state(scr + (size_t)(t1 - 1 - t0) * SS);
+    fetch(t1 - 1);
     for (int64_t t = t1 - 1; t >= t0; --t) {
       const int buf = (it++) & 1;
-      stage(t, buf);
+      commit(buf);
+      if (t - 1 >= t0) fetch(t - 1);
       __syncthreads();
       const float* tb = tok + buf * 4 * D;
-      const float* kv = tb + part * PER;
-      const float* qv = tb + D + part * PER;
       const float vj = tb[2 * D + col], dOj = tb[3 * D + col];
       const float alpha = gates[2 * buf], beta = gates[2 * buf + 1];
       const size_t th = (size_t)t * a.H + h, tq = (size_t)t * a.Hqk + hq;
-      float sp[PER];  // S_{t-1}
-      load_state(scr + (size_t)(t - t0) * SS, sp);
-      // D += scale q dO^T
+      // column j's terms of dq (S_t dO) first: S_t is not needed after them
+      float* rq = red_q + col * RS;
+      float* rk = red_k + col * RS;
 #pragma unroll
-      for (int x = 0; x < PER; ++x) Dm[x] = fmaf(a.scale * qv[x], dOj, Dm[x]);
+      for (int y = 0; y < NP; ++y)
+        *reinterpret_cast<float4*>(rq + piece(y)) = make_float4(sc[4 * y] * dOj, sc[4 * y + 1] * dOj,
+                                                                sc[4 * y + 2] * dOj, sc[4 * y + 3] * dOj);
+      float sp[PER];  // S_{t-1}
+      cp_async_wait_all();
+      load_vec(spb, sp);
+      if (t - 1 >= t0) prefetch_state(scr + (size_t)(t - 1 - t0) * SS);
+      // D += scale q dO^T
+      {
+        float qv[PER];
+        load_vec(tb + D, qv);
+#pragma unroll
+        for (int x = 0; x < PER; ++x) Dm[x] = fmaf(a.scale * qv[x], dOj, Dm[x]);
+      }
+      float kv[PER];
+      load_vec(tb, kv);
       // u = S~^T k (S~ = alpha S_{t-1}), w = D^T k, column j
       float pu = 0.f, pw = 0.f;
 #pragma unroll
@@ -226,23 +300,19 @@ gdn_prefill_backward_kernel(const BwdArgs a) {
         pw += __shfl_xor_sync(0xffffffffu, pw, off);
       }
       const float u = alpha * pu, w = pw, vmu = vj - u;
-      // column j's terms of dq (S_t dO) and dk (D (v - u) - S~ w), and of dg
-      const float* sc = scr + (size_t)(t - t0 + 1) * SS;  // S_t
-      float* rq = red_q + (size_t)col * D + part * PER;
-      float* rk = red_k + (size_t)col * D + part * PER;
+      // column j's terms of dk (D (v - u) - S~ w) and of dg
       float sdg = 0.f;
 #pragma unroll
-      for (int x = 0; x < PER; x += 4) {
-        const float4 s4 = *reinterpret_cast<const float4*>(sc + x);
-        *reinterpret_cast<float4*>(rq + x) = make_float4(s4.x * dOj, s4.y * dOj, s4.z * dOj, s4.w * dOj);
+      for (int y = 0; y < NP; ++y) {
         float kk[4];
 #pragma unroll
-        for (int y = 0; y < 4; ++y) {
-          const float stl = alpha * sp[x + y];
-          kk[y] = Dm[x + y] * vmu - stl * w;
-          sdg = fmaf(Dm[x + y], stl, sdg);
+        for (int z = 0; z < 4; ++z) {
+          const int x = 4 * y + z;
+          const float stl = alpha * sp[x];
+          kk[z] = Dm[x] * vmu - stl * w;
+          sdg = fmaf(Dm[x], stl, sdg);
         }
-        *reinterpret_cast<float4*>(rk + x) = make_float4(kk[0], kk[1], kk[2], kk[3]);
+        *reinterpret_cast<float4*>(rk + piece(y)) = make_float4(kk[0], kk[1], kk[2], kk[3]);
       }
       float sdb = 0.f;
       if (part == 0) {
@@ -250,9 +320,12 @@ gdn_prefill_backward_kernel(const BwdArgs a) {
         sdb = w * vmu;
         a.dv[th * D + col] = beta * w;
       }
-      // dL/dS_{t-1}
+      // dL/dS_{t-1}; S_{t-1} becomes the next token's S_t
 #pragma unroll
-      for (int x = 0; x < PER; ++x) Dm[x] = alpha * (Dm[x] - beta * w * kv[x]);
+      for (int x = 0; x < PER; ++x) {
+        Dm[x] = alpha * (Dm[x] - beta * w * kv[x]);
+        sc[x] = sp[x];
+      }
 #pragma unroll
       for (int off = 16; off > 0; off >>= 1) {
         sdg += __shfl_xor_sync(0xffffffffu, sdg, off);
@@ -267,7 +340,7 @@ gdn_prefill_backward_kernel(const BwdArgs a) {
         const float* r = (o < D) ? red_q : red_k;
         const int i = (o < D) ? o : o - D;
         float s = 0.f;
-        for (int j = 0; j < D; ++j) s += r[(size_t)j * D + i];
+        for (int j = 0; j < D; ++j) s += r[j * RS + i];
         if (o < D)
           atomicAdd(a.dq + tq * D + i, a.scale * s);
         else
