@@ -11,19 +11,21 @@
 //     dg    = <D, S~> - beta (u . w)
 //     D    <- alpha (D - beta k w^T)  (dL/dS_{t-1});   dL/dS_0 = D at the end.
 //
-// Token-sequential SIMT, one CTA per (sequence, head), laid out like the sequential
-// forward kernel: value column j of S is owned by dk / 32 adjacent lanes, 32 of its
-// dk entries each. The states S_{t-1} the walk needs are recomputed:
+// Token-sequential SIMT. Every value column j of S (and of D) evolves on its own given
+// the token's k, q, v_j, alpha and beta, so one CTA takes 32 columns of one (sequence,
+// head) (dv / 32 CTAs per head); value column j is owned by dk / 32 adjacent lanes, 32
+// of its dk entries each. The states S_{t-1} the walk needs are recomputed:
 //   1. forward over the sequence, writing the state at the start of every chunk of
 //      C tokens to the workspace (checkpoints);
 //   2. for each chunk, last to first: recompute the chunk's states from its
 //      checkpoint into a per-CTA scratch (the state before each of its tokens), then
 //      walk its tokens backwards reading S_{t-1} from there (a thread reads back only
 //      what it wrote, so no barrier orders the scratch).
-// Per token the column sums of dq and dk go through shared memory (each thread
-// writes its 32 partial products, then 2 dk threads each add one entry over the dv
-// columns); dg and dbeta are block reductions. dq and dk are accumulated with fp32
-// atomics into zeroed outputs, so value heads that share a q/k head add up.
+// Per token the sums over columns of dq and dk go through shared memory (each thread
+// writes its 32 partial products, then each of the dk threads adds two entries over
+// the CTA's columns); dg and dbeta are block reductions. All four are accumulated
+// with fp32 atomics into zeroed outputs, so the column blocks of a head and the value
+// heads that share a q/k head add up.
 // Latency: the next token's k, q, v, dO and gates are loaded into registers while
 // the current token computes; in the backward walk S_t is the previous token's
 // S_{t-1} (kept in registers) and the next S_{t-1} is fetched from the scratch into
@@ -54,7 +56,7 @@ struct BwdArgs {
   float* dbeta;
   float* d_init;
   float* ckpt;     // [H][ck_slots][D][D]
-  float* scratch;  // [N * H][C + 1][D][D]
+  float* scratch;  // [N * H][C + 1][D][D] (each CTA its own columns' rows)
   size_t ck_slots;
   int64_t total_T;
   int N, H, Hqk, C;
@@ -79,17 +81,20 @@ BwdLayout bwd_layout(int N, int64_t total_T, int H, int D, int C) {
   return L;
 }
 
-// Shared-memory stride of one column in the [D columns][D entries] buffers, padded
-// so that the eight lanes of a quarter warp (two columns x four 16-byte pieces)
-// store to distinct banks.
+constexpr int kBwdCols = 32;  // value columns per CTA
+
+// Shared-memory stride of one column in the [columns][D entries] buffers, padded so
+// that the eight lanes of a quarter warp (two columns x four 16-byte pieces) store to
+// distinct banks.
 template <int D>
 constexpr int bwd_col_stride() { return D + 16; }
 
 template <int D>
 constexpr size_t bwd_smem_bytes() {
   // token vectors [2][k, q, v, dO][D], gates [2][alpha, beta], column partials of dq
-  // and dk and the prefetched S_{t-1} ([D][stride] each), scalar partials [warps][2]
-  return (8 * D + 4 + 3 * D * bwd_col_stride<D>() + 2 * (D * (D / 32) / 32)) * sizeof(float);
+  // and dk and the prefetched S_{t-1} ([columns][stride] each), scalar partials
+  // [warps][2]; D threads
+  return (8 * D + 4 + 3 * kBwdCols * bwd_col_stride<D>() + 2 * (D / 32)) * sizeof(float);
 }
 
 __device__ __forceinline__ void cp_async16(float* dst, const float* src) {
@@ -101,28 +106,33 @@ __device__ __forceinline__ void cp_async_wait_all() {
 }
 
 template <int D, typename TIn>
-__global__ void __launch_bounds__(D * (D / 32))
+__global__ void __launch_bounds__(D)
 gdn_prefill_backward_kernel(const BwdArgs a) {
   constexpr int TPC = D / 32;  // threads per state column
-  constexpr int NT = D * TPC;
+  constexpr int NT = kBwdCols * TPC;  // == D
+  static_assert(NT == D, "one thread per dk entry of the token vectors");
   constexpr int PER = 32;      // entries of the column per thread
   constexpr int NP = PER / 4;  // 16-byte pieces per thread
   constexpr int NW = NT / 32;
   constexpr int RS = bwd_col_stride<D>();
   extern __shared__ __align__(16) float bsm[];
-  float* tok = bsm;               // [2][4][D]
-  float* gates = tok + 8 * D;     // [2][2]
-  float* red_q = gates + 4;       // [D columns][RS]
-  float* red_k = red_q + D * RS;
-  float* sp_buf = red_k + D * RS;  // [D][RS]: the next S_{t-1}, each thread its own entries
-  float* red_s = sp_buf + D * RS;  // [NW][2]
+  float* tok = bsm;                       // [2][4][D]
+  float* gates = tok + 8 * D;             // [2][2]
+  float* red_q = gates + 4;               // [kBwdCols][RS]
+  float* red_k = red_q + kBwdCols * RS;
+  float* sp_buf = red_k + kBwdCols * RS;  // [kBwdCols][RS]: the next S_{t-1}, each thread its own entries
+  float* red_s = sp_buf + kBwdCols * RS;  // [NW][2]
 
   const int tid = threadIdx.x;
-  const int col = tid / TPC, part = tid % TPC;
+  constexpr int kBlocks = D / kBwdCols;   // column blocks per head
+  const int cb = blockIdx.x % kBlocks;
+  const int item = blockIdx.x / kBlocks;  // (sequence, head)
+  const int lcol = tid / TPC, part = tid % TPC;
+  const int col = cb * kBwdCols + lcol;
   // this thread's entries of column col: the 16-byte pieces part, part + TPC, ...,
   // i.e. entries 4 (part + TPC y) + z, y < NP, z < 4 (local index x = 4 y + z)
   auto piece = [&](int y) { return 4 * (part + TPC * y); };
-  const int n = blockIdx.x / a.H, h = blockIdx.x - n * a.H;
+  const int n = item / a.H, h = item - n * a.H;
   const int hq = h / (a.H / a.Hqk);
   int64_t bos, eos;
   if (!seq_bounds(a.cu, n, a.total_T, a.err, &bos, &eos)) return;
@@ -130,14 +140,14 @@ gdn_prefill_backward_kernel(const BwdArgs a) {
   const size_t SS = (size_t)D * D;
   const size_t state_off = ((size_t)n * a.H + h) * SS + (size_t)col * D;
   float* ck = a.ckpt + ((size_t)h * a.ck_slots + (size_t)(bos / a.C) + n) * SS + (size_t)col * D;
-  float* scr = a.scratch + (size_t)blockIdx.x * (size_t)(a.C + 1) * SS + (size_t)col * D;
-  float* spb = sp_buf + col * RS;
+  float* scr = a.scratch + (size_t)item * (size_t)(a.C + 1) * SS + (size_t)col * D;
+  float* spb = sp_buf + lcol * RS;
   const TIn* qp = static_cast<const TIn*>(a.q);
   const TIn* kp = static_cast<const TIn*>(a.k);
   const TIn* vp = static_cast<const TIn*>(a.v);
   const TIn* dop = static_cast<const TIn*>(a.d_o);
 
-  // A token's k, q, v, dO (thread tid < D holds element tid; NT >= D) and gates are
+  // A token's k, q, v, dO (thread tid holds element tid) and gates are
   // fetched into registers, then committed to shared-memory buffer `buf` (two
   // buffers: the barrier of the token in between orders every read of a buffer
   // before its refill).
@@ -268,8 +278,8 @@ gdn_prefill_backward_kernel(const BwdArgs a) {
       const float alpha = gates[2 * buf], beta = gates[2 * buf + 1];
       const size_t th = (size_t)t * a.H + h, tq = (size_t)t * a.Hqk + hq;
       // column j's terms of dq (S_t dO) first: S_t is not needed after them
-      float* rq = red_q + col * RS;
-      float* rk = red_k + col * RS;
+      float* rq = red_q + lcol * RS;
+      float* rk = red_k + lcol * RS;
 #pragma unroll
       for (int y = 0; y < NP; ++y)
         *reinterpret_cast<float4*>(rq + piece(y)) = make_float4(sc[4 * y] * dOj, sc[4 * y + 1] * dOj,
@@ -336,15 +346,15 @@ gdn_prefill_backward_kernel(const BwdArgs a) {
         red_s[2 * (tid >> 5) + 1] = sdb;
       }
       __syncthreads();
-      for (int o = tid; o < 2 * D; o += NT) {
-        const float* r = (o < D) ? red_q : red_k;
-        const int i = (o < D) ? o : o - D;
-        float s = 0.f;
-        for (int j = 0; j < D; ++j) s += r[j * RS + i];
-        if (o < D)
-          atomicAdd(a.dq + tq * D + i, a.scale * s);
-        else
-          atomicAdd(a.dk + tq * D + i, beta * s);
+      {  // entry tid of dq and of dk over this CTA's columns
+        float sq = 0.f, sk = 0.f;
+#pragma unroll 8
+        for (int j = 0; j < kBwdCols; ++j) {
+          sq += red_q[j * RS + tid];
+          sk += red_k[j * RS + tid];
+        }
+        atomicAdd(a.dq + tq * D + tid, a.scale * sq);
+        atomicAdd(a.dk + tq * D + tid, beta * sk);
       }
       if (tid == 0) {
         float g_sum = 0.f, b_sum = 0.f;
@@ -352,8 +362,8 @@ gdn_prefill_backward_kernel(const BwdArgs a) {
           g_sum += red_s[2 * wi];
           b_sum += red_s[2 * wi + 1];
         }
-        a.dg[th] = g_sum;
-        a.dbeta[th] = b_sum;
+        atomicAdd(a.dg + th, g_sum);
+        atomicAdd(a.dbeta + th, b_sum);
       }
     }
   }
@@ -374,7 +384,7 @@ gdn_status_t launch_bwd(const BwdArgs& a, cudaStream_t stream) {
       }))
     return fail(e != cudaSuccess ? GDN_ERR_CUDA : GDN_ERR_UNSUPPORTED,
                 std::string("prefill backward: setup: ") + (e != cudaSuccess ? cudaGetErrorString(e) : "device index too large"));
-  kernel<<<(unsigned)((long long)a.N * a.H), D * (D / 32), smem, stream>>>(a);
+  kernel<<<(unsigned)((long long)a.N * a.H * (D / kBwdCols)), D, smem, stream>>>(a);
   return check_launch("gdn_chunk_prefill_backward");
 }
 
@@ -391,7 +401,8 @@ gdn_status_t bwd_check_shape(int N, int64_t total_T, int H, int dk, int dv, int 
   if (dk != dv || (dk != 32 && dk != 64 && dk != 128))
     return fail(GDN_ERR_UNSUPPORTED, "gdn_chunk_prefill_backward: dk == dv in {32, 64, 128}");
   if (chunk > 4096) return fail(GDN_ERR_UNSUPPORTED, "gdn_chunk_prefill_backward: chunk <= 4096");
-  if ((long long)N * H >= (1LL << 31)) return fail(GDN_ERR_UNSUPPORTED, "gdn_chunk_prefill_backward: N * H too large");
+  if ((long long)N * H * (dk / 32) >= (1LL << 31))
+    return fail(GDN_ERR_UNSUPPORTED, "gdn_chunk_prefill_backward: N * H too large");
   return gdn::ok();
 }
 
@@ -440,10 +451,14 @@ extern "C" gdn_status_t gdn_chunk_prefill_backward(
   cudaStream_t s = gdn::as_stream(stream);
   if (total_T > 0) {
     const size_t qk_bytes = (size_t)total_T * H_qk * dk * sizeof(float);
+    const size_t gb_bytes = (size_t)total_T * H * sizeof(float);
     cudaError_t e = cudaMemsetAsync(d_q, 0, qk_bytes, s);
     if (e == cudaSuccess) e = cudaMemsetAsync(d_k, 0, qk_bytes, s);
+    if (e == cudaSuccess) e = cudaMemsetAsync(d_g, 0, gb_bytes, s);
+    if (e == cudaSuccess) e = cudaMemsetAsync(d_beta, 0, gb_bytes, s);
     if (e != cudaSuccess)
-      return fail(GDN_ERR_CUDA, std::string("gdn_chunk_prefill_backward: clearing d_q, d_k: ") + cudaGetErrorString(e));
+      return fail(GDN_ERR_CUDA, std::string("gdn_chunk_prefill_backward: clearing the outputs: ") +
+                                    cudaGetErrorString(e));
   }
   gdn::BwdArgs a;
   a.q = q; a.k = k; a.v = v; a.d_o = d_o; a.g = g; a.beta = beta; a.cu = cu_seqlens;

@@ -257,20 +257,25 @@ const char* gdn_last_error(void);
  * [total_T, H] fp32; cu_seqlens [N+1] int32 on the device; initial_state [N, H, dv,
  * dk] fp32 K-last or NULL), plus d_o [total_T, H, dv] in in_dtype. Outputs, fp32,
  * caller-owned: d_q, d_k [total_T, H_qk, dk] (value heads that share a q/k head add
- * up; both are cleared on `stream` first), d_v [total_T, H, dv], d_g, d_beta
- * [total_T, H], d_initial_state [N, H, dv, dk] K-last or NULL (not written).
+ * up), d_v [total_T, H, dv], d_g, d_beta [total_T, H] (d_q, d_k, d_g and d_beta are
+ * cleared on `stream` first), d_initial_state [N, H, dv, dk] K-last or NULL (not
+ * written).
  * dk == dv in {32, 64, 128}; flags must be 0 (GDN_ERR_UNSUPPORTED otherwise);
  * q, k, v, d_o, d_q, d_k and the state pointers 16-byte aligned.
  *
- * One CTA per (sequence, head), token-sequential: a forward pass writes the state at
- * the start of every `chunk` tokens to the workspace, then each chunk, last to first,
- * is recomputed from its checkpoint into the workspace and walked backwards. The
+ * Token-sequential, one CTA per 32 value columns of a (sequence, head) (the columns
+ * of the state evolve independently): a forward pass writes the state at the start of
+ * every `chunk` tokens to the workspace, then each chunk, last to first, is
+ * recomputed from its checkpoint into the workspace and walked backwards. d_q, d_k,
+ * d_g and d_beta are sums over column blocks (and grouped heads) taken with fp32
+ * atomics: their last bits may differ between calls; d_v and d_initial_state are
+ * written directly and are reproducible. The
  * workspace (gdn_chunk_prefill_backward_workspace_size; 16-byte aligned, contents
  * need no clearing) holds H x (total_T / chunk + N + 1) checkpoints and N x H x
  * (chunk + 1) recomputed states of dk x dv fp32. Errors: GDN_ERR_INVALID_ARG /
  * GDN_ERR_UNSUPPORTED / GDN_ERR_WORKSPACE before anything is launched; a malformed
  * cu_seqlens pair sets GDN_DEVERR_BAD_CU_SEQLENS and skips that sequence. Only
- * enqueues on `stream` (two memsets and one kernel).
+ * enqueues on `stream` (four memsets and one kernel).
  */
 gdn_status_t gdn_chunk_prefill_backward_workspace_size(int N, int64_t total_T, int H, int dk, int dv, int chunk,
                                                        size_t* bytes);

@@ -69,11 +69,15 @@ def test_backward_long_sequence_weak_decay():
 
 
 def test_backward_leaves_no_trace_between_calls():
-    """Two calls in a row on the same workspace give bitwise the same derivatives
-    (one q/k head per value head: no atomics race)."""
+    """Two calls in a row on reused memory: dv and the initial-state derivative,
+    written directly, are bitwise equal; dq, dk, dg and dbeta, summed over column
+    blocks with fp32 atomics in whatever order they arrive, agree to rounding."""
     inp = inputs.prefill_inputs([150, 40], 2, 128, 128, seed=98, g_range=(0.0, 0.05))
     d_o, d_fin = _upstream(inp, 99, torch.bfloat16)
     a = _run(inp, d_o, d_fin, 32)
     b = _run(inp, d_o, d_fin, 32)
-    for name in a:
+    for name in ("dv", "d_initial_state"):
         assert torch.equal(a[name], b[name]), name
+    for name in ("dq", "dk", "dg", "dbeta"):
+        err = (a[name] - b[name]).abs().max() / b[name].abs().max()
+        assert err < 1e-5, (name, float(err))
