@@ -476,13 +476,17 @@ def backward_alg_bytes(inp):
 def backward_inputs(key, device, seed):
     """The backward part runs on the chunked-prefill workload with seeded upstream
     derivatives d_o (bf16, N(0, 1)) and d_final_state (fp32, N(0, 0.1^2))."""
-    inp, chunk, name = prefill_cfg("prefill", device, seed)
+    inp, _, name = prefill_cfg("prefill", device, seed)
+    # checkpoints every 16 tokens: a chunk's recomputed states (16 x 64 KiB per head)
+    # then stay in L2 between their write and their read
+    chunk = 16
     gen = torch.Generator(device=device).manual_seed(seed + 7)
     total, H, dv = inp.v.shape
     N = inp.cu_seqlens.numel() - 1
     d_o = torch.randn((total, H, dv), generator=gen, device=device).to(inp.q.dtype)
     d_fin = torch.randn((N, H, dv, inp.q.shape[-1]), generator=gen, device=device) * 0.1
-    return inp, d_o, d_fin, chunk, "prefill backward (dq, dk, dv, dg, dbeta, d_initial_state), " + name
+    return inp, d_o, d_fin, chunk, ("prefill backward (dq, dk, dv, dg, dbeta, d_initial_state), checkpoints every "
+                                     "16 tokens, " + name)
 
 
 def bench_backward(key, steps, warmup, ws, rank, peaks):
