@@ -529,6 +529,82 @@ def bench_backward(key, steps, warmup, ws, rank, peaks):
     return res
 
 
+CP_RANKS = 4
+
+
+def bench_cp(key, steps, warmup, peaks):
+    """Context-parallel prefill of the low-parallelism workload (B=1 x 65536, H=4)
+    over CP_RANKS ranks, emulated one after another on this GPU (no kernel waits on
+    another rank; the exchange, an all-gather of the (local state, transfer) pairs,
+    is a device copy here). Each rank's slice is a contiguous quarter of the
+    sequence; its device time (local state and transfer, combine, finish of the
+    slice) is timed with CUDA events, and the part reports the maximum over ranks:
+    the step time CP_RANKS GPUs would need with a free exchange."""
+    import gated_delta_rule_58_b200 as gdn
+    dev = torch.device("cuda", torch.cuda.current_device())
+    inp, chunk, name = prefill_cfg("longseq", dev, 0)
+    T, H, dk = inp.q.shape
+    dv = inp.v.shape[-1]
+    R = CP_RANKS
+    cuts = [T * r // R for r in range(R + 1)]
+    sl = []
+    for r in range(R):
+        a, b = cuts[r], cuts[r + 1]
+        cu = torch.tensor([0, b - a], dtype=torch.int32, device=dev)
+        sl.append([x[a:b].contiguous() for x in (inp.q, inp.k, inp.v, inp.g, inp.beta)] + [cu])
+    loc = torch.empty((R, 1, H, dv, dk), device=dev)
+    tr = torch.empty_like(loc)
+    start = torch.empty((R, 1, H, dv, dk), device=dev)
+    o = torch.empty((T, H, dv), dtype=torch.bfloat16, device=dev)
+    fin = torch.empty((1, H, dv, dk), device=dev)
+    gathered = torch.empty((2, R, 1, H, dv, dk), device=dev)
+    ws_cp = [torch.empty(gdn.gdn_cp_local_state_workspace_size(1, cuts[r + 1] - cuts[r], H, dk, dv, chunk),
+                         dtype=torch.uint8, device=dev) for r in range(R)]
+
+    def rank_step(r):
+        q, k, v, g, beta, cu = sl[r]
+        gdn.gdn_cp_local_state(q, k, v, g, beta, cu, loc[r], tr[r], chunk=chunk, workspace=ws_cp[r])
+        gathered[0].copy_(loc)  # stands in for the all-gather
+        gathered[1].copy_(tr)
+        gdn.gdn_cp_combine(gathered[0], gathered[1], r, start[r], initial_state=inp.initial_state)
+        gdn.gdn_cp_finish(q, k, v, g, beta, cu, o[cuts[r]:cuts[r + 1]], ws_cp[r], start_state=start[r],
+                          final_state=fin, chunk=chunk, scale=inp.scale)
+
+    for _ in range(warmup):
+        for r in range(R):
+            rank_step(r)
+    torch.cuda.synchronize()
+    per_rank = []
+    for r in range(R):
+        s_, e_ = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        s_.record()
+        for _ in range(steps):
+            rank_step(r)
+        e_.record()
+        torch.cuda.synchronize()
+        per_rank.append(s_.elapsed_time(e_) / steps)
+    ms = max(per_rank)
+    alg_b = prefill_alg_bytes(inp)
+    exchange = 2 * R * H * dv * dk * 4
+    achieved = alg_b / (ms * 1e-3) / 1e9
+    res = {
+        "workload": f"context-parallel prefill over {R} ranks emulated on one GPU, {name}",
+        "algo": "per rank: local state and transfer over segments (fused kernel, two folds in one fixup launch), "
+                "combine (fixup scan), finish (fixup scan from the start state, output pass over the segments)",
+        "ms_per_step": ms,
+        "ms_per_rank": per_rank,
+        "tokens_per_s": T / (ms * 1e-3),
+        "exchange_bytes_per_rank": exchange,
+        "roofline": {"bound": "hbm", "achieved": achieved, "peak": peaks["hbm_gbs"] * R, "unit": "GB/s",
+                     "frac": achieved / (peaks["hbm_gbs"] * R), "traffic": None,
+                     "note": f"peak = {R} GPUs' copy bandwidth; not a multi-GPU measurement"},
+        "alg_bytes": alg_b,
+    }
+    del sl, loc, tr, start, o, fin, gathered, ws_cp, inp
+    torch.cuda.empty_cache()
+    return res
+
+
 # ---------------------------------------------------------------- CPU oracle (baseline / reference arm)
 
 class OracleDecode:
@@ -698,7 +774,7 @@ def main():
     ap.add_argument("--steps", type=int, default=2000)
     ap.add_argument("--warmup", type=int, default=20)
     ap.add_argument("--impl", default="ours", choices=["ours", "reference"])
-    ap.add_argument("--parts", default="gdp,decode_b1,decode_b4,decode_b16,prefill,varlen,longseq,tiny,backward",
+    ap.add_argument("--parts", default="gdp,decode_b1,decode_b4,decode_b16,prefill,varlen,longseq,tiny,backward,cp",
                     help="comma list of extra workloads to measure ('none' for none)")
     ap.add_argument("--part-steps", type=int, default=5,
                     help="timed steps of each prefill part (decode parts: 20 times this, at least 20)")
@@ -743,6 +819,9 @@ def main():
                 elif key == "backward":
                     r = bench_backward(key, max(args.part_steps // 2, 1), 3, ws, rank, peaks)
                     r["metric"] = "backward tokens/s"
+                elif key == "cp":
+                    r = bench_cp(key, args.part_steps, 3, peaks)
+                    r["metric"] = "prefill tokens/s (max over emulated ranks)"
                 else:
                     r = bench_prefill(key, args.part_steps, 3, ws, rank, peaks, algo=algo)
                     r["metric"] = "prefill tokens/s"
@@ -767,6 +846,10 @@ def main():
                 if r["key"] in DECODE_CFGS:
                     v, threads, sample = oracle_decode_rate(r["key"], budget_s=2.0 if r["key"] != "gdp" else 4.0)
                     r["cpu_baseline"] = {"value": v, "unit": "GB/s", "cores": threads, "kind": "oracle",
+                                         "sample": sample}
+                elif r["key"] == "cp":
+                    v, threads, sample = oracle_prefill_rate("longseq", budget_s=4.0)
+                    r["cpu_baseline"] = {"value": v, "unit": "tokens/s", "cores": threads, "kind": "oracle",
                                          "sample": sample}
                 elif r["key"] == "backward":
                     v, threads, sample = oracle_backward_rate(r["key"], budget_s=4.0)

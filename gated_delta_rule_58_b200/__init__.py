@@ -11,7 +11,7 @@ from ._lib import (  # noqa: F401
     GDN_DEVERR_SLOT_OUT_OF_RANGE, GDN_DEVERR_TIMEOUT, GDN_PREFILL_AUTO, GDN_PREFILL_FUSED,
     GDN_PREFILL_SEQUENTIAL, GDN_PREFILL_TRANSFER, GDN_QK_L2NORM, GdnError, declared_functions,
     gdn_chunk_prefill, gdn_chunk_prefill_backward, gdn_chunk_prefill_backward_workspace_size,
-    gdn_chunk_prefill_static_scratch, gdn_cp_combine, gdn_cp_local_state, gdn_chunk_prefill_workspace_size, gdn_decode,
+    gdn_chunk_prefill_static_scratch, gdn_cp_combine, gdn_cp_finish, gdn_cp_local_state, gdn_cp_local_state_workspace_size, gdn_chunk_prefill_workspace_size, gdn_decode,
     gdn_decode_mtp,
     gdn_get_device_error, gdn_selftest_wait_timeout,
     gdn_last_error, gdn_version, lib,

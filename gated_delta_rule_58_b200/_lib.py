@@ -87,7 +87,13 @@ def lib() -> ctypes.CDLL:
             L.gdn_get_device_error.argtypes = [ctypes.POINTER(ctypes.c_uint32)]
             L.gdn_cp_local_state.restype = i32
             L.gdn_cp_local_state.argtypes = [vp, vp, vp, vp, vp, vp, i32, i64, vp, vp, i32, i32, i32, i32, i32, u32,
-                                             i32, vp]
+                                             i32, vp, sz, vp]
+            L.gdn_cp_local_state_workspace_size.restype = i32
+            L.gdn_cp_local_state_workspace_size.argtypes = [i32, i64, i32, i32, i32, i32,
+                                                            ctypes.POINTER(ctypes.c_size_t)]
+            L.gdn_cp_finish.restype = i32
+            L.gdn_cp_finish.argtypes = [vp, vp, vp, vp, vp, vp, i32, i64, vp, vp, vp, i32, i32, i32, i32, i32, f32, u32,
+                                        i32, i32, vp, sz, vp]
             L.gdn_cp_combine.restype = i32
             L.gdn_cp_combine.argtypes = [vp, vp, i32, i32, i32, i32, i32, i32, vp, vp, vp]
             L.gdn_chunk_prefill_backward_workspace_size.restype = i32
@@ -126,15 +132,49 @@ def gdn_get_device_error() -> int:
     return int(flags.value)
 
 
-def gdn_cp_local_state(q, k, v, g, beta, cu_seqlens, local_state, transfer, chunk=64, stream=None, l2norm=False):
+def gdn_cp_local_state_workspace_size(N, total_T, H, dk, dv, chunk=64) -> int:
+    out = ctypes.c_size_t(0)
+    _check(lib().gdn_cp_local_state_workspace_size(N, total_T, H, dk, dv, chunk, ctypes.byref(out)))
+    return int(out.value)
+
+
+def gdn_cp_local_state(q, k, v, g, beta, cu_seqlens, local_state, transfer, chunk=64, stream=None, l2norm=False,
+                       workspace=None):
     """Context parallelism, step 1 (see include/gdn.h): the slice's local state H and
-    transfer M^T, both [N,H,dv,dk] fp32 K-last."""
+    transfer M^T, both [N,H,dv,dk] fp32 K-last. `workspace` (uint8 CUDA tensor) is
+    allocated through torch when None (pass one with a raw stream handle)."""
+    import torch
     total_T, H_qk, dk = q.shape
     H, dv = v.shape[1], v.shape[-1]
     N = cu_seqlens.numel() - 1
+    if workspace is None:
+        if stream is not None and not isinstance(stream, torch.cuda.Stream):
+            raise ValueError("gdn_cp_local_state: pass `workspace` when `stream` is a raw handle")
+        need = gdn_cp_local_state_workspace_size(N, total_T, H, dk, dv, chunk)
+        ctx = torch.cuda.stream(stream) if stream is not None else _nullcontext()
+        with ctx:
+            workspace = torch.empty(max(need, 1), dtype=torch.uint8, device=q.device)
     _check(lib().gdn_cp_local_state(_ptr(q), _ptr(k), _ptr(v), _ptr(g), _ptr(beta), _ptr(cu_seqlens), N, total_T,
                                     _ptr(local_state), _ptr(transfer), H, H_qk, dk, dv, chunk,
-                                    GDN_QK_L2NORM if l2norm else 0, _dtype_code(q), _stream_ptr(stream, q.device)))
+                                    GDN_QK_L2NORM if l2norm else 0, _dtype_code(q), _ptr(workspace),
+                                    workspace.numel(), _stream_ptr(stream, q.device)))
+
+
+def gdn_cp_finish(q, k, v, g, beta, cu_seqlens, o, workspace, start_state=None, final_state=None, chunk=64,
+                  scale=None, stream=None, l2norm=False):
+    """Context parallelism, step 4 (see include/gdn.h): the slice's outputs and final
+    state from the rank's start state, reusing the segments that gdn_cp_local_state
+    left in `workspace` (the same slice, shapes and workspace)."""
+    total_T, H_qk, dk = q.shape
+    H, dv = v.shape[1], v.shape[-1]
+    N = cu_seqlens.numel() - 1
+    if scale is None:
+        scale = dk ** -0.5
+    _check(lib().gdn_cp_finish(_ptr(q), _ptr(k), _ptr(v), _ptr(g), _ptr(beta), _ptr(cu_seqlens), N, total_T,
+                               _ptr(start_state), _ptr(final_state), _ptr(o), H, H_qk, dk, dv, chunk, float(scale),
+                               GDN_QK_L2NORM if l2norm else 0, _dtype_code(q), _dtype_code(o), _ptr(workspace),
+                               workspace.numel(), _stream_ptr(stream, q.device)))
+    return o
 
 
 def gdn_cp_combine(local_states, transfers, rank, start_state, initial_state=None, stream=None):

@@ -7,11 +7,13 @@ the context-parallelism block of include/gdn.h):
   1. the slice's local state H and transfer M (library kernels);
   2. one all-gather of (H, M) over the group, in rank order;
   3. this rank's start state from the pairs of the ranks before it (library kernel);
-  4. the ordinary prefill of the slice from that start state (library kernels).
+  4. the slice's outputs from that start state, reusing step 1's segments (library
+     kernels: gdn_cp_finish).
 
 Only step 2 communicates; this module does the orchestration and the collective
 and none of the method's arithmetic. `ops` replaces the library calls of steps 1,
-3 and 4 (used by the CPU tests of the rank logic, which run without a GPU).
+3 and 4 (used by the CPU tests of the rank logic, which run without a GPU); its
+local_state returns (H, M, context) and its prefill receives that context.
 """
 from __future__ import annotations
 
@@ -28,17 +30,20 @@ def _library_ops():
         dk, dv = q.shape[-1], v.shape[-1]
         loc = torch.empty((N, H, dv, dk), dtype=torch.float32, device=q.device)
         tr = torch.empty_like(loc)
-        _lib.gdn_cp_local_state(q, k, v, g, beta, cu, loc, tr, chunk=chunk, l2norm=l2norm)
-        return loc, tr
+        N, total_T = cu.numel() - 1, q.shape[0]
+        ws = torch.empty(max(_lib.gdn_cp_local_state_workspace_size(N, total_T, H, dk, dv, chunk), 1),
+                         dtype=torch.uint8, device=q.device)
+        _lib.gdn_cp_local_state(q, k, v, g, beta, cu, loc, tr, chunk=chunk, l2norm=l2norm, workspace=ws)
+        return loc, tr, ws
 
     def combine(all_loc, all_tr, rank, initial_state):
         start = torch.empty(all_loc.shape[1:], dtype=torch.float32, device=all_loc.device)
         _lib.gdn_cp_combine(all_loc, all_tr, rank, start, initial_state=initial_state)
         return start
 
-    def prefill(q, k, v, g, beta, cu, o, start, final_state, chunk, scale, l2norm):
-        _lib.gdn_chunk_prefill(q, k, v, g, beta, cu, o, initial_state=start, final_state=final_state, chunk=chunk,
-                               scale=scale, l2norm=l2norm)
+    def prefill(q, k, v, g, beta, cu, o, start, final_state, chunk, scale, l2norm, ctx):
+        _lib.gdn_cp_finish(q, k, v, g, beta, cu, o, ctx, start_state=start, final_state=final_state, chunk=chunk,
+                           scale=scale, l2norm=l2norm)
 
     return types.SimpleNamespace(local_state=local_state, combine=combine, prefill=prefill)
 
@@ -54,7 +59,7 @@ def cp_chunk_prefill(q, k, v, g, beta, cu_seqlens, o, initial_state=None, final_
     ops = ops or _library_ops()
     rank = dist.get_rank(group)
     ranks = dist.get_world_size(group)
-    loc, tr = ops.local_state(q, k, v, g, beta, cu_seqlens, chunk, l2norm)
+    loc, tr, ctx = ops.local_state(q, k, v, g, beta, cu_seqlens, chunk, l2norm)
     parts_loc = [torch.empty_like(loc) for _ in range(ranks)]
     parts_tr = [torch.empty_like(tr) for _ in range(ranks)]
     dist.all_gather(parts_loc, loc.contiguous(), group=group)
@@ -62,5 +67,5 @@ def cp_chunk_prefill(q, k, v, g, beta, cu_seqlens, o, initial_state=None, final_
     all_loc = torch.stack(parts_loc)  # rank-major [ranks, N, H, dv, dk]
     all_tr = torch.stack(parts_tr)
     start = ops.combine(all_loc, all_tr, rank, initial_state)
-    ops.prefill(q, k, v, g, beta, cu_seqlens, o, start, final_state, chunk, scale, l2norm)
+    ops.prefill(q, k, v, g, beta, cu_seqlens, o, start, final_state, chunk, scale, l2norm, ctx)
     return o

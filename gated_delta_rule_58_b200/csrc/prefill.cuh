@@ -53,6 +53,13 @@ size_t prefill_transfer_workspace_bytes(const PrefillShape& s);
 // Chunks per segment (G) the transfer algorithm uses for this shape.
 int prefill_transfer_segment_chunks(const PrefillShape& s);
 gdn_status_t prefill_transfer_launch(const PrefillShape& s, const PrefillArgs& a, cudaStream_t stream);
+// Context parallelism: a slice's local state and transfer over segments (transfer
+// path workspace).
+gdn_status_t cp_local_state_launch(const PrefillShape& s, const PrefillArgs& a, float* local_out, float* transfer_out,
+                                   cudaStream_t stream);
+// Context parallelism: the slice's outputs and final state from the rank's start
+// state, reusing the segments left in the workspace by cp_local_state_launch.
+gdn_status_t cp_finish_launch(const PrefillShape& s, const PrefillArgs& a, cudaStream_t stream);
 // Context parallelism: the start state of rank `rank` from the (local state,
 // transfer) pairs of ranks 0..rank-1, rank-major [ranks][N][H][128][128] (K-last).
 gdn_status_t cp_combine_launch(const float* local_states, const float* transfers, int ranks, int rank, int N, int H,

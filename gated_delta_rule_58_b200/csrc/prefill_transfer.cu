@@ -146,22 +146,39 @@ constexpr uint32_t kFixLocBytes = kFixRows * D * 4;
 constexpr uint32_t kFixSmem = 2 * kFixMtBytes + 2 * kFixLocBytes + D * kFixRows * 4 + 64;
 constexpr uint64_t kFixWaitNs = 2000000000ull;
 
+// `local` may be null: the local states are then zero and only the transfer is copied.
 __device__ __forceinline__ void fixup_issue(float* mt, float* loc, uint64_t* bar, const float* transfer,
                                             const float* local, size_t off, int r0) {
   tc::fence_proxy_async_smem();  // earlier generic reads of this buffer precede the copy
-  tc::mbar_arrive_expect_tx(bar, kFixMtBytes + kFixLocBytes);
+  tc::mbar_arrive_expect_tx(bar, kFixMtBytes + (local ? kFixLocBytes : 0u));
   tc::bulk_load(tc::smem_u32(mt), transfer + off, kFixMtBytes, bar);
-  tc::bulk_load(tc::smem_u32(loc), local + off + (size_t)r0 * D, kFixLocBytes, bar);
+  if (local) tc::bulk_load(tc::smem_u32(loc), local + off + (size_t)r0 * D, kFixLocBytes, bar);
 }
 
 // The segments of sequence n: seg_of_seq[n] .. seg_of_seq[n+1]-1 (the transfer
 // path), or, with seg_of_seq null, the context-parallel ranks 0 .. cp_count-1 of a
-// rank-major [ranks][N] list: entries n, n + cp_stride, ... (cp_stride = N). `fixed`
-// may be null (only the final state is wanted).
+// rank-major [ranks][N] list: entries n, n + cp_stride, ... (cp_stride = N). A launch
+// may carry two folds over the same transfers (blockIdx.y picks the job). In a job,
+// `fixed` may be null (only the final state is wanted); `local` null means zero local
+// states; init_identity starts from the identity instead of initial_state (which is
+// then ignored), so the fold yields the composed transfer.
+struct FixupJob {
+  const float* local;
+  const float* initial_state;
+  int init_identity;
+  float* fixed;
+  float* final_state;
+};
+
 __global__ void __launch_bounds__(kFixThreads)
-gdn_fixup_scan_kernel(const int32_t* seg_of_seq, int cp_stride, int cp_count, int H, const float* local,
-                      const float* transfer, float* fixed, const float* initial_state, float* final_state,
-                      unsigned int* err) {
+gdn_fixup_scan_kernel(const int32_t* seg_of_seq, int cp_stride, int cp_count, int H, const float* transfer,
+                      const FixupJob job0, const FixupJob job1, unsigned int* err) {
+  const FixupJob job = blockIdx.y ? job1 : job0;
+  const float* local = job.local;
+  const float* initial_state = job.initial_state;
+  const int init_identity = job.init_identity;
+  float* fixed = job.fixed;
+  float* final_state = job.final_state;
   extern __shared__ __align__(16) uint8_t fsm[];
   float* mt = reinterpret_cast<float*>(fsm);                 // [2][D][D]
   float* loc = mt + 2 * D * D;                                // [2][kFixRows][D]
@@ -192,7 +209,12 @@ gdn_fixup_scan_kernel(const int32_t* seg_of_seq, int cp_stride, int cp_count, in
 #pragma unroll
   for (int a = 0; a < kFixRPT; ++a) {
     float4 x = make_float4(0.f, 0.f, 0.f, 0.f);
-    if (initial_state) x = *reinterpret_cast<const float4*>(initial_state + soff + (size_t)(r0 + jr + a) * D + l0);
+    const int row = r0 + jr + a;
+    if (init_identity)
+      x = make_float4(row == l0 ? 1.f : 0.f, row == l0 + 1 ? 1.f : 0.f, row == l0 + 2 ? 1.f : 0.f,
+                      row == l0 + 3 ? 1.f : 0.f);
+    else if (initial_state)
+      x = *reinterpret_cast<const float4*>(initial_state + soff + (size_t)row * D + l0);
     cur[a][0] = x.x; cur[a][1] = x.y; cur[a][2] = x.z; cur[a][3] = x.w;
 #pragma unroll
     for (int x4 = 0; x4 < 4; ++x4) sT[(l0 + x4) * kFixRows + jr + a] = cur[a][x4];
@@ -230,7 +252,8 @@ gdn_fixup_scan_kernel(const int32_t* seg_of_seq, int cp_stride, int cp_count, in
       if (fixed)
         *reinterpret_cast<float4*>(fixed + off + (size_t)(r0 + jr + a) * D + l0) =
             make_float4(cur[a][0], cur[a][1], cur[a][2], cur[a][3]);
-      const float4 x = *reinterpret_cast<const float4*>(lr + (jr + a) * D + l0);
+      const float4 x = local ? *reinterpret_cast<const float4*>(lr + (jr + a) * D + l0)
+                             : make_float4(0.f, 0.f, 0.f, 0.f);
       acc[a][0] = x.x; acc[a][1] = x.y; acc[a][2] = x.z; acc[a][3] = x.w;
     }
 #pragma unroll 8
@@ -312,11 +335,105 @@ gdn_status_t prefill_transfer_launch(const PrefillShape& s, const PrefillArgs& a
     return fail(e != cudaSuccess ? GDN_ERR_CUDA : GDN_ERR_UNSUPPORTED,
                 std::string("transfer prefill: setup: ") +
                     (e != cudaSuccess ? cudaGetErrorString(e) : "device index too large"));
+  const FixupJob job{local, a.initial_state, 0, fixed, a.final_state};
   gdn_fixup_scan_kernel<<<(unsigned)((long long)s.N * s.H * (D / kFixRows)), kFixThreads, kFixSmem, stream>>>(
-      seg_of_seq, 0, 0, s.H, local, transfer, fixed, a.initial_state, a.final_state, a.err);
+      seg_of_seq, 0, 0, s.H, transfer, job, job, a.err);
   st = check_launch("transfer prefill: fixup scan");
   if (st != GDN_OK) return st;
 
+  PrefillArgs out = a;
+  out.cu_seqlens = seg_cu;
+  out.initial_state = fixed;
+  out.final_state = nullptr;
+  out.mode = kPrefillOutputs;
+  return prefill_fused_launch(seg, out, stream);
+}
+
+// Context parallelism, step 1, for any number of sequences: the slice's local state
+// H (zero start) and transfer M (identity start, values zero), both K-last, from the
+// transfer path's segment passes and two fixup scans over the segments (one from
+// zero with the local states, one from the identity with zero local states). Uses
+// the transfer prefill's workspace.
+gdn_status_t cp_local_state_launch(const PrefillShape& s, const PrefillArgs& a, float* local_out, float* transfer_out,
+                                   cudaStream_t stream) {
+  const TransferLayout L = layout_for(s);
+  uint8_t* ws = static_cast<uint8_t*>(a.workspace);
+  int32_t* seg_cu = reinterpret_cast<int32_t*>(ws + L.off_seg_cu);
+  int32_t* seg_of_seq = reinterpret_cast<int32_t*>(ws + L.off_seg_of_seq);
+  float* local = reinterpret_cast<float*>(ws + L.off_local);
+  float* transfer = reinterpret_cast<float*>(ws + L.off_transfer);
+  if ((long long)L.max_segments * s.H >= (1LL << 31) || (long long)s.N * s.H * (D / kFixRows) >= (1LL << 31))
+    return fail(GDN_ERR_UNSUPPORTED, "cp local state: too many segments");
+  gdn_segment_map_kernel<<<1, 1024, 0, stream>>>(a.cu_seqlens, s.N, s.total_T, L.seg_chunks * C, L.max_segments,
+                                                  seg_cu, seg_of_seq, a.err);
+  gdn_status_t st = check_launch("cp local state: segment map");
+  if (st != GDN_OK) return st;
+  PrefillShape seg = s;
+  seg.N = L.max_segments;
+  PrefillArgs loc = a;
+  loc.cu_seqlens = seg_cu;
+  loc.initial_state = nullptr;
+  loc.o = nullptr;
+  loc.final_state = local;
+  loc.mode = kPrefillLocalState;
+  st = prefill_fused_launch(seg, loc, stream);
+  if (st != GDN_OK) return st;
+  PrefillArgs tr = loc;
+  tr.final_state = transfer;
+  tr.mode = kPrefillTransfer;
+  st = prefill_fused_launch(seg, tr, stream);
+  if (st != GDN_OK) return st;
+  static PerDeviceOnce once;  // the shared-memory opt-in applies to the current device only
+  int dev = 0;
+  cudaError_t e = cudaGetDevice(&dev);
+  if (e != cudaSuccess) return fail(GDN_ERR_CUDA, std::string("cp local state: cudaGetDevice: ") + cudaGetErrorString(e));
+  if (!run_once_per_device(once, dev, [&](int, int*) {
+        e = cudaFuncSetAttribute(gdn_fixup_scan_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, kFixSmem);
+        return e == cudaSuccess;
+      }))
+    return fail(e != cudaSuccess ? GDN_ERR_CUDA : GDN_ERR_UNSUPPORTED,
+                std::string("cp local state: setup: ") + (e != cudaSuccess ? cudaGetErrorString(e) : "device index too large"));
+  // both folds in one launch: y = 0 the local states from zero, y = 1 the transfers
+  // from the identity with zero local states
+  const dim3 grid((unsigned)((long long)s.N * s.H * (D / kFixRows)), 2);
+  const FixupJob fold_local{local, nullptr, 0, nullptr, local_out};
+  const FixupJob fold_transfer{nullptr, nullptr, 1, nullptr, transfer_out};
+  gdn_fixup_scan_kernel<<<grid, kFixThreads, kFixSmem, stream>>>(seg_of_seq, 0, 0, s.H, transfer, fold_local,
+                                                                  fold_transfer, a.err);
+  return check_launch("cp local state: fixup scans");
+}
+
+// Context parallelism, step 4, after cp_local_state_launch on the same slice and
+// workspace: the segments' start states from the rank's start state (a.initial_state),
+// the final state, and the outputs of every segment, reusing the segment map, local
+// states and transfers left in the workspace.
+gdn_status_t cp_finish_launch(const PrefillShape& s, const PrefillArgs& a, cudaStream_t stream) {
+  const TransferLayout L = layout_for(s);
+  uint8_t* ws = static_cast<uint8_t*>(a.workspace);
+  int32_t* seg_cu = reinterpret_cast<int32_t*>(ws + L.off_seg_cu);
+  int32_t* seg_of_seq = reinterpret_cast<int32_t*>(ws + L.off_seg_of_seq);
+  float* local = reinterpret_cast<float*>(ws + L.off_local);
+  float* transfer = reinterpret_cast<float*>(ws + L.off_transfer);
+  float* fixed = reinterpret_cast<float*>(ws + L.off_fixed);
+  if ((long long)L.max_segments * s.H >= (1LL << 31) || (long long)s.N * s.H * (D / kFixRows) >= (1LL << 31))
+    return fail(GDN_ERR_UNSUPPORTED, "cp finish: too many segments");
+  static PerDeviceOnce once;  // the shared-memory opt-in applies to the current device only
+  int dev = 0;
+  cudaError_t e = cudaGetDevice(&dev);
+  if (e != cudaSuccess) return fail(GDN_ERR_CUDA, std::string("cp finish: cudaGetDevice: ") + cudaGetErrorString(e));
+  if (!run_once_per_device(once, dev, [&](int, int*) {
+        e = cudaFuncSetAttribute(gdn_fixup_scan_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, kFixSmem);
+        return e == cudaSuccess;
+      }))
+    return fail(e != cudaSuccess ? GDN_ERR_CUDA : GDN_ERR_UNSUPPORTED,
+                std::string("cp finish: setup: ") + (e != cudaSuccess ? cudaGetErrorString(e) : "device index too large"));
+  const FixupJob job{local, a.initial_state, 0, fixed, a.final_state};
+  gdn_fixup_scan_kernel<<<(unsigned)((long long)s.N * s.H * (D / kFixRows)), kFixThreads, kFixSmem, stream>>>(
+      seg_of_seq, 0, 0, s.H, transfer, job, job, a.err);
+  gdn_status_t st = check_launch("cp finish: fixup scan");
+  if (st != GDN_OK) return st;
+  PrefillShape seg = s;
+  seg.N = L.max_segments;
   PrefillArgs out = a;
   out.cu_seqlens = seg_cu;
   out.initial_state = fixed;
@@ -340,8 +457,9 @@ gdn_status_t cp_combine_launch(const float* local_states, const float* transfers
                 std::string("cp combine: setup: ") + (e != cudaSuccess ? cudaGetErrorString(e) : "device index too large"));
   (void)ranks;
   if ((long long)N * H * (D / kFixRows) >= (1LL << 31)) return fail(GDN_ERR_UNSUPPORTED, "cp combine: N * H too large");
+  const FixupJob job{local_states, initial_state, 0, nullptr, start_state};
   gdn_fixup_scan_kernel<<<(unsigned)((long long)N * H * (D / kFixRows)), kFixThreads, kFixSmem, stream>>>(
-      nullptr, N, rank, H, local_states, transfers, nullptr, initial_state, start_state, err);
+      nullptr, N, rank, H, transfers, job, job, err);
   return check_launch("gdn_cp_combine");
 }
 

@@ -227,17 +227,39 @@ gdn_status_t gdn_chunk_prefill_static_scratch(const void* q, const void* k, cons
  *      rank-major [ranks, N, H, dv, dk];
  *   3. gdn_cp_combine: its start state from the pairs of ranks 0..rank-1 and the
  *      sequences' initial state (NULL = zero): S^T <- S^T M_r^T + H_r^T in fp32;
- *   4. gdn_chunk_prefill on its slice with initial_state = that start state; the
- *      last rank's final state is the sequences' final state.
- * gdn_cp_local_state: dk == dv == 128, chunk == 64 (the fused tensor-core kernel,
- * two launches); other arguments as gdn_chunk_prefill. gdn_cp_combine: dk == dv ==
- * 128; rank 0 copies the initial state (or zeros); start_state may alias
- * initial_state. Both only enqueue on `stream`.
+ *   4. gdn_chunk_prefill on its slice with initial_state = that start state, or
+ *      gdn_cp_finish (below), which reuses step 1's segments; the last rank's final
+ *      state is the sequences' final state.
+ * gdn_cp_local_state: dk == dv == 128, chunk == 64; the slice's sequences are cut
+ * into segments processed in parallel by the fused tensor-core kernel (local states
+ * and transfers of every segment), then two fixup scans fold the segments' pairs;
+ * workspace: gdn_cp_local_state_workspace_size bytes, 16-byte aligned (the transfer
+ * prefill's), GDN_ERR_WORKSPACE otherwise; other arguments as gdn_chunk_prefill.
+ * gdn_cp_combine: dk == dv == 128; rank 0 copies the initial state (or zeros);
+ * start_state may alias initial_state. Both only enqueue on `stream`.
  */
+gdn_status_t gdn_cp_local_state_workspace_size(int N, int64_t total_T, int H, int dk, int dv, int chunk,
+                                               size_t* bytes);
 gdn_status_t gdn_cp_local_state(const void* q, const void* k, const void* v, const float* g,
                                 const float* beta, const int32_t* cu_seqlens, int N, int64_t total_T,
                                 float* local_state, float* transfer, int H, int H_qk, int dk, int dv,
-                                int chunk, uint32_t flags, gdn_dtype_t in_dtype, void* stream);
+                                int chunk, uint32_t flags, gdn_dtype_t in_dtype, void* workspace,
+                                size_t workspace_bytes, void* stream);
+/*
+ * gdn_cp_finish — step 4 without recomputing step 1: the slice's outputs o and final
+ * state (NULL: not written) from the rank's start state (NULL = zero), reusing the
+ * segments' local states and transfers that gdn_cp_local_state left in `workspace`.
+ * The call must use the same slice (q, k, v, g, beta, cu_seqlens, N, total_T, H,
+ * H_qk, dk, dv, chunk, flags) and the same workspace as that gdn_cp_local_state call,
+ * with nothing else writing the workspace in between; the result then equals
+ * gdn_chunk_prefill with GDN_PREFILL_TRANSFER on the slice. Other arguments and
+ * errors as gdn_chunk_prefill.
+ */
+gdn_status_t gdn_cp_finish(const void* q, const void* k, const void* v, const float* g, const float* beta,
+                           const int32_t* cu_seqlens, int N, int64_t total_T, const float* start_state,
+                           float* final_state, void* o, int H, int H_qk, int dk, int dv, int chunk, float scale,
+                           uint32_t flags, gdn_dtype_t in_dtype, gdn_dtype_t out_dtype, void* workspace,
+                           size_t workspace_bytes, void* stream);
 gdn_status_t gdn_cp_combine(const float* local_states, const float* transfers, int ranks, int rank, int N,
                             int H, int dk, int dv, const float* initial_state, float* start_state,
                             void* stream);

@@ -34,7 +34,7 @@ def _oracle_ops():
         ident = np.broadcast_to(np.eye(dk), (N, H, dk, dk)).copy()
         zero_v = torch.zeros(v.shape[0], H, dk, dtype=torch.float64)
         _, Mt, _ = oracle.prefill(q, k, zero_v, g, beta, cu, ident, scale=0.3, l2norm=l2norm)
-        return torch.from_numpy(Ht), torch.from_numpy(Mt)
+        return torch.from_numpy(Ht), torch.from_numpy(Mt), None
 
     def combine(all_loc, all_tr, rank, initial_state):
         S = torch.zeros_like(all_loc[0]) if initial_state is None else initial_state.clone()
@@ -42,7 +42,7 @@ def _oracle_ops():
             S = torch.einsum("nhij,nhjk->nhik", S, all_tr[r]) + all_loc[r]
         return S
 
-    def prefill(q, k, v, g, beta, cu, o, start, final_state, chunk, scale, l2norm):
+    def prefill(q, k, v, g, beta, cu, o, start, final_state, chunk, scale, l2norm, ctx):
         o_, f_, _ = oracle.prefill(q, k, v, g, beta, cu, start, scale=0.3, l2norm=l2norm)
         o.copy_(torch.from_numpy(o_))
         final_state.copy_(torch.from_numpy(f_))

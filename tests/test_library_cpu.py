@@ -150,9 +150,16 @@ def test_cp_entry_points_reject_on_host(L):
     assert L.gdn_cp_combine(FAKE, FAKE, 2, 1, 1, 2, 64, 64, None, FAKE, None) == gdn.GDN_ERR_UNSUPPORTED
     assert L.gdn_cp_combine(None, None, 2, 1, 1, 2, 128, 128, None, FAKE, None) == gdn.GDN_ERR_INVALID_ARG
     assert L.gdn_cp_local_state(FAKE, FAKE, FAKE, FAKE, FAKE, FAKE, 1, 64, FAKE, FAKE, 2, 2, 128, 128, 32, 0,
-                                gdn.GDN_BF16, None) == gdn.GDN_ERR_UNSUPPORTED  # chunk 32
+                                gdn.GDN_BF16, FAKE, 1 << 40, None) == gdn.GDN_ERR_UNSUPPORTED  # chunk 32
     assert L.gdn_cp_local_state(FAKE, FAKE, FAKE, FAKE, FAKE, FAKE, 1, 64, None, FAKE, 2, 2, 128, 128, 64, 0,
-                                gdn.GDN_BF16, None) == gdn.GDN_ERR_INVALID_ARG
+                                gdn.GDN_BF16, FAKE, 1 << 40, None) == gdn.GDN_ERR_INVALID_ARG
+    size = ctypes.c_size_t(0)
+    assert L.gdn_cp_local_state_workspace_size(1, 64, 2, 128, 128, 64, ctypes.byref(size)) == gdn.GDN_OK
+    assert size.value > 0
+    assert L.gdn_cp_local_state(FAKE, FAKE, FAKE, FAKE, FAKE, FAKE, 1, 64, FAKE, FAKE, 2, 2, 128, 128, 64, 0,
+                                gdn.GDN_BF16, FAKE, size.value - 1, None) == gdn.GDN_ERR_WORKSPACE
+    assert L.gdn_cp_local_state(FAKE, FAKE, FAKE, FAKE, FAKE, FAKE, 1, 64, FAKE, FAKE, 2, 2, 128, 128, 64, 0,
+                                gdn.GDN_BF16, None, size.value, None) == gdn.GDN_ERR_WORKSPACE
 
 
 def test_backward_entry_points_reject_on_host(L):
