@@ -119,3 +119,56 @@ def test_cp_plain_prefill_path_still_matches():
                                  scale=inp.scale)
     assert_close(o, o_r, what="cp plain o")
     assert_close(fin, f_r, what="cp plain final state")
+
+
+def _gpu_rank_main(rank, ranks, port, lengths, out):
+    """One rank of cp_chunk_prefill (the library driver and kernels) on cuda:0; the
+    ranks share the GPU as separate processes, which only exchange through a gloo
+    all-gather between launches (no kernel waits on another process)."""
+    import datetime
+    import os
+    import sys
+    import torch.distributed as dist
+    sys.path.insert(0, os.path.dirname(os.path.dirname(os.path.abspath(__file__))))
+    from gated_delta_rule_58_b200 import inputs as inp_mod
+    from gated_delta_rule_58_b200.cp import cp_chunk_prefill
+    from tests.cp_slices import rank_slice as rs, slice_bounds as sb
+    os.environ.update(MASTER_ADDR="127.0.0.1", MASTER_PORT=str(port))
+    dist.init_process_group("gloo", rank=rank, world_size=ranks, timeout=datetime.timedelta(seconds=120))
+    try:
+        torch.cuda.set_device(0)
+        inp = inp_mod.prefill_inputs(lengths, 4, 128, 128, seed=86, g_range=(0.0, 0.02), H_qk=2)
+        (q, k, v, g, beta), cu, idx = rs(inp, sb(lengths, ranks), rank)
+        q, k, v, g, beta, cu = (x.cuda() for x in (q, k, v, g, beta, cu))
+        o = torch.empty((q.shape[0], 4, 128), dtype=torch.float32, device="cuda")
+        fin = torch.empty((len(lengths), 4, 128, 128), device="cuda")
+        cp_chunk_prefill(q, k, v, g, beta, cu, o, initial_state=inp.initial_state.cuda(), final_state=fin,
+                         scale=inp.scale)
+        torch.cuda.synchronize()
+        out[rank] = (idx.numpy(), o.cpu().numpy(), fin.cpu().numpy())
+    finally:
+        dist.destroy_process_group()
+
+
+def test_cp_driver_over_two_processes_on_one_gpu():
+    import socket
+    import numpy as np
+    import torch.multiprocessing as mp
+    lengths = [2000, 130, 0, 700]
+    with socket.socket() as s:
+        s.bind(("127.0.0.1", 0))
+        port = s.getsockname()[1]
+    ctx = mp.get_context("spawn")
+    with ctx.Manager() as m:
+        out = m.dict()
+        mp.start_processes(_gpu_rank_main, args=(2, port, lengths, out), nprocs=2, join=True, start_method="spawn")
+        res = dict(out)
+    inp = inputs.prefill_inputs(lengths, 4, 128, 128, seed=86, g_range=(0.0, 0.02), H_qk=2)
+    o_ref, f_ref, _ = oracle.prefill(inp.q, inp.k, inp.v, inp.g, inp.beta, inp.cu_seqlens, inp.initial_state,
+                                     scale=inp.scale)
+    o = np.zeros_like(o_ref)
+    for r in range(2):
+        idx, o_r, _ = res[r]
+        o[idx] = o_r
+    assert_close(o, o_ref, what="cp driver o")
+    assert_close(res[1][2], f_ref, what="cp driver final state")
