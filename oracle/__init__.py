@@ -54,7 +54,8 @@ def _declare(lib):
     lib.gdn_oracle_prefill_backward.restype = ctypes.c_int
     lib.gdn_oracle_prefill_backward.argtypes = [dp, dp, dp, dp, dp, ctypes.POINTER(ctypes.c_int64),
                                                 ctypes.c_int, ctypes.c_int, ctypes.c_int, ctypes.c_int, ctypes.c_int,
-                                                ctypes.c_double, dp, dp, dp, dp, dp, dp, dp, dp, dp, ctypes.c_int]
+                                                ctypes.c_double, ctypes.c_int, dp, dp, dp, dp, dp, dp, dp, dp, dp,
+                                                ctypes.c_int]
     lib.gdn_oracle_decode.restype = ctypes.c_int
     lib.gdn_oracle_decode.argtypes = [dp, dp, dp, dp, dp, dp, ctypes.c_int,
                                       ctypes.POINTER(ctypes.c_int32), dp,
@@ -122,9 +123,9 @@ def prefill(q, k, v, g, beta, cu_seqlens, initial_state=None, scale=None, nthrea
 
 
 def prefill_backward(q, k, v, g, beta, cu_seqlens, d_o, initial_state=None, d_final_state=None, scale=None,
-                     nthreads=0, lib=None):
-    """Reverse-mode derivatives of `prefill` (one Householder per token, no q/k
-    normalisation), fp64, token by token (see gdn_oracle.c).
+                     nthreads=0, lib=None, l2norm=False):
+    """Reverse-mode derivatives of `prefill` (one Householder per token; with l2norm,
+    through the per-token q/k normalisation), fp64, token by token (see gdn_oracle.c).
 
     d_o: [total_T, H, dv]; d_final_state: [N, H, dv, dk] or None (zero).
     Returns dict(dq [total_T, H_qk, dk], dk [total_T, H_qk, dk], dv [total_T, H, dv],
@@ -147,7 +148,8 @@ def prefill_backward(q, k, v, g, beta, cu_seqlens, d_o, initial_state=None, d_fi
     db = np.zeros((total_T, H), np.float64)
     dinit = np.zeros((N, H, dv, dk), np.float64)
     rc = lib.gdn_oracle_prefill_backward(_ptr(q), _ptr(k), _ptr(v), _ptr(g), _ptr(beta), _ptr(cu, ctypes.c_int64),
-                                         N, H, Hqk, dk, dv, float(scale), _ptr(init), _ptr(d_o), _ptr(dfin),
+                                         N, H, Hqk, dk, dv, float(scale), int(bool(l2norm)), _ptr(init), _ptr(d_o),
+                                         _ptr(dfin),
                                          _ptr(dq), _ptr(dkk), _ptr(dvv), _ptr(dg), _ptr(db), _ptr(dinit),
                                          int(nthreads))
     if rc < 0:

@@ -275,17 +275,33 @@ int gdn_oracle_decode(const double* q, const double* k, const double* v, const d
  *     dg    = <D, S~> - beta (u . w)                 (alpha = exp(g): dg = alpha dL/dalpha)
  *     D    <- alpha (D - beta k w^T)                 (= alpha P D, dL/dS_{t-1})
  * and dL/dS_0 = D at the end. Every state S_t is kept from a forward pass first.
- * Scope: one Householder per token and no q/k normalisation.
+ * With l2norm the relations read the unit vectors k^ = k / |k|, q^ = q / |q| (a zero
+ * vector stays zero); the walk above gives the derivatives for k^ and q^, and the
+ * chain rule through the normalisation maps them to dk = (dk^ - k^ (k^ . dk^)) / |k|
+ * (zero for a zero vector), likewise for q. Scope: one Householder per token.
  */
 
 typedef struct {
   const double *q, *k, *v, *g, *beta;
   const int64_t* cu;
-  int H, Hqk, dk, dv;
+  int H, Hqk, dk, dv, l2norm;
   double scale;
   const double *init, *d_o, *d_fin;
   double *dq, *dkk, *dvv, *dg, *dbeta, *d_init;
 } backward_ctx;
+
+/* the derivative for x from the one for x^ = x / |x|: (d - x^ (x^ . d)) / |x| */
+static void unit_backward(const double* x, double* d, int n) {
+  double ss = 0.0, dot = 0.0;
+  for (int i = 0; i < n; ++i) ss += x[i] * x[i];
+  if (!(ss > 0.0)) {
+    for (int i = 0; i < n; ++i) d[i] = 0.0;
+    return;
+  }
+  const double inv = 1.0 / sqrt(ss);
+  for (int i = 0; i < n; ++i) dot += x[i] * inv * d[i];
+  for (int i = 0; i < n; ++i) d[i] = (d[i] - x[i] * inv * dot) * inv;
+}
 
 static void backward_item(void* vctx, int item) {
   backward_ctx* c = (backward_ctx*)vctx;
@@ -299,6 +315,7 @@ static void backward_item(void* vctx, int item) {
   double* Dt = (double*)malloc(ssz * sizeof(double));
   double* u = (double*)malloc((size_t)dv * sizeof(double));
   double* w = (double*)malloc((size_t)dv * sizeof(double));
+  double* unit = (double*)malloc(2 * (size_t)dk * sizeof(double));  /* k^, q^ of a token */
   if (c->init)
     memcpy(states, c->init + ((size_t)n * H + h) * ssz, ssz * sizeof(double));
   else
@@ -308,7 +325,7 @@ static void backward_item(void* vctx, int item) {
     double* St = states + (size_t)(t + 1) * ssz;
     memcpy(St, states + (size_t)t * ssz, ssz * sizeof(double));
     apply_gate(St, exp(c->g[th]), dk, dv);
-    apply_householder(St, c->k + tq * dk, c->v + th * dv, c->beta[th], dk, dv);
+    apply_householder(St, maybe_unit(c->k + tq * dk, dk, c->l2norm, unit), c->v + th * dv, c->beta[th], dk, dv);
   }
   if (c->d_fin)
     memcpy(Dt, c->d_fin + ((size_t)n * H + h) * ssz, ssz * sizeof(double));
@@ -316,8 +333,8 @@ static void backward_item(void* vctx, int item) {
     memset(Dt, 0, ssz * sizeof(double));
   for (int64_t t = T - 1; t >= 0; --t) {
     const size_t th = (size_t)(t0 + t) * H + h, tq = (size_t)(t0 + t) * Hqk + hq;
-    const double* q = c->q + tq * dk;
-    const double* k = c->k + tq * dk;
+    const double* q = maybe_unit(c->q + tq * dk, dk, c->l2norm, unit + dk);
+    const double* k = maybe_unit(c->k + tq * dk, dk, c->l2norm, unit);
     const double* v = c->v + th * dv;
     const double* dO = c->d_o + th * dv;
     const double alpha = exp(c->g[th]), beta = c->beta[th];
@@ -365,8 +382,13 @@ static void backward_item(void* vctx, int item) {
     for (int j = 0; j < dv; ++j)
       for (int i = 0; i < dk; ++i)
         Dt[(size_t)j * dk + i] = alpha * (Dt[(size_t)j * dk + i] - beta * k[i] * w[j]);
+    if (c->l2norm) { /* through the normalisation, from the raw vectors */
+      unit_backward(c->q + tq * dk, dq, dk);
+      unit_backward(c->k + tq * dk, dkv, dk);
+    }
   }
   if (c->d_init) memcpy(c->d_init + ((size_t)n * H + h) * ssz, Dt, ssz * sizeof(double));
+  free(unit);
   free(w);
   free(u);
   free(Dt);
@@ -374,7 +396,8 @@ static void backward_item(void* vctx, int item) {
 }
 
 /*
- * Inputs as for gdn_oracle_prefill, plus d_o [total_T, H, dv] and d_final_state
+ * Inputs as for gdn_oracle_prefill (l2norm != 0: q and k normalised per token), plus
+ * d_o [total_T, H, dv] and d_final_state
  * [N, H, dv, dk] or NULL (zero). Outputs: dq, dk [total_T, H, dk] per VALUE head
  * (the caller sums the heads that share a q/k head), dv [total_T, H, dv], dg and
  * dbeta [total_T, H], d_initial_state [N, H, dv, dk] or NULL.
@@ -382,14 +405,14 @@ static void backward_item(void* vctx, int item) {
  */
 int gdn_oracle_prefill_backward(const double* q, const double* k, const double* v, const double* g,
                                 const double* beta, const int64_t* cu_seqlens, int N, int H, int Hqk,
-                                int dk, int dv, double scale, const double* init, const double* d_o,
+                                int dk, int dv, double scale, int l2norm, const double* init, const double* d_o,
                                 const double* d_final_state, double* dq, double* dk_out, double* dv_out,
                                 double* dg, double* dbeta, double* d_init, int nthreads) {
   if (N < 0 || H <= 0 || Hqk <= 0 || H % Hqk != 0 || dk <= 0 || dv <= 0 || !cu_seqlens || !d_o) return -1;
   if (cu_seqlens[0] != 0) return -1;
   for (int n = 0; n < N; ++n)
     if (cu_seqlens[n + 1] < cu_seqlens[n]) return -1;
-  backward_ctx c = {q, k, v, g, beta, cu_seqlens, H, Hqk, dk, dv, scale, init, d_o, d_final_state,
+  backward_ctx c = {q, k, v, g, beta, cu_seqlens, H, Hqk, dk, dv, l2norm, scale, init, d_o, d_final_state,
                     dq, dk_out, dv_out, dg, dbeta, d_init};
   return run_items(N * H, nthreads, backward_item, &c);
 }

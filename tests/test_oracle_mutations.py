@@ -77,6 +77,9 @@ MUTANTS = {
                                      "Dt[(size_t)j * dk + i] = Dt[(size_t)j * dk + i] - beta * k[i] * w[j];")],
     # backward: the query derivative read from the previous state
     "backward_dq_previous_state": [("acc += St[(size_t)j * dk + i] * dO[j];", "acc += Sp[(size_t)j * dk + i] * dO[j];")],
+    # backward: the normalisation's derivative without its projection term
+    "backward_l2norm_without_projection": [("for (int i = 0; i < n; ++i) d[i] = (d[i] - x[i] * inv * dot) * inv;",
+                                            "for (int i = 0; i < n; ++i) d[i] = d[i] * inv;")],
     "l2norm_squared": [("const double inv = ss > 0.0 ? 1.0 / sqrt(ss) : 0.0;",
                         "const double inv = ss > 0.0 ? 1.0 / ss : 0.0;")],
 }

@@ -619,15 +619,18 @@ def test_prefill_is_affine_in_the_initial_state():
 
 # ---------------------------------------------------------------- backward (reverse-mode derivatives)
 
-def _backward_case(seed):
+def _backward_case(seed, l2norm=False):
     """Three sequences (one empty), two value heads over one q/k head, dk != dv, an
     initial state, upstream derivatives R (outputs) and Q (final state) of the loss
-    L = sum(R * o) + sum(Q * S_final)."""
+    L = sum(R * o) + sum(Q * S_final). Keys are unit vectors, except with l2norm,
+    where keys and queries have norms in (0.5, 2) and are normalised by the method."""
     rng = _rng(seed)
     lens, H, Hqk, dk, dv = [4, 0, 3], 2, 1, 3, 2
     T = sum(lens)
     q = rng.standard_normal((T, Hqk, dk))
     k = _unit(rng.standard_normal((T, Hqk, dk)))
+    if l2norm:
+        k = k * rng.uniform(0.5, 2.0, (T, Hqk, 1))
     v = rng.standard_normal((T, H, dv))
     beta = 1 / (1 + np.exp(-rng.standard_normal((T, H))))
     g = -rng.uniform(0.05, 0.6, (T, H))
@@ -638,36 +641,39 @@ def _backward_case(seed):
     return dict(q=q, k=k, v=v, g=g, beta=beta, initial_state=init), cu, R, Q
 
 
-def _loss(lib, x, cu, R, Q):
+def _loss(lib, x, cu, R, Q, l2norm=False):
     o, fin, _ = oracle.prefill(x["q"], x["k"], x["v"], x["g"], x["beta"], cu, x["initial_state"], scale=0.7,
-                               lib=lib)
+                               lib=lib, l2norm=l2norm)
     return float((R * o).sum() + (Q * fin).sum())
 
 
 def check_backward_matches_central_differences(lib=None):
     """Every derivative of the backward pass against central finite differences of
-    the oracle's forward (fp64, step 1e-6) on every input entry."""
-    x, cu, R, Q = _backward_case(40)
-    d = oracle.prefill_backward(x["q"], x["k"], x["v"], x["g"], x["beta"], cu, R, x["initial_state"], Q, scale=0.7,
-                                lib=lib)
-    names = dict(q="dq", k="dk", v="dv", g="dg", beta="dbeta", initial_state="d_initial_state")
-    eps = 1e-6
-    for name, gname in names.items():
-        fd = np.zeros_like(x[name])
-        for idx in np.ndindex(x[name].shape):
-            xp = {kk: vv.copy() for kk, vv in x.items()}
-            xm = {kk: vv.copy() for kk, vv in x.items()}
-            xp[name][idx] += eps
-            xm[name][idx] -= eps
-            fd[idx] = (_loss(lib, xp, cu, R, Q) - _loss(lib, xm, cu, R, Q)) / (2 * eps)
-        assert _relerr(d[gname], fd) < 1e-6, (name, _relerr(d[gname], fd))
+    the oracle's forward (fp64, step 1e-6) on every input entry, without and with the
+    q/k normalisation."""
+    for l2norm in (False, True):
+        x, cu, R, Q = _backward_case(40, l2norm)
+        d = oracle.prefill_backward(x["q"], x["k"], x["v"], x["g"], x["beta"], cu, R, x["initial_state"], Q,
+                                    scale=0.7, lib=lib, l2norm=l2norm)
+        names = dict(q="dq", k="dk", v="dv", g="dg", beta="dbeta", initial_state="d_initial_state")
+        eps = 1e-6
+        for name, gname in names.items():
+            fd = np.zeros_like(x[name])
+            for idx in np.ndindex(x[name].shape):
+                xp = {kk: vv.copy() for kk, vv in x.items()}
+                xm = {kk: vv.copy() for kk, vv in x.items()}
+                xp[name][idx] += eps
+                xm[name][idx] -= eps
+                fd[idx] = (_loss(lib, xp, cu, R, Q, l2norm) - _loss(lib, xm, cu, R, Q, l2norm)) / (2 * eps)
+            assert _relerr(d[gname], fd) < 1e-6, (l2norm, name, _relerr(d[gname], fd))
 
 
 def check_backward_matches_autograd_of_a_plain_torch_forward(lib=None):
     """The derivatives against torch.autograd through a plain fp64 PyTorch forward
-    of the recurrence written here (gate, Householder write, output per token)."""
+    of the recurrence written here (gate, Householder write, output per token), with
+    the q/k normalisation."""
     import torch
-    x, cu, R, Q = _backward_case(41)
+    x, cu, R, Q = _backward_case(41, l2norm=True)
     tx = {kk: torch.tensor(vv, requires_grad=True) for kk, vv in x.items()}
     H, Hqk = x["v"].shape[1], x["q"].shape[1]
     loss = torch.zeros((), dtype=torch.float64)
@@ -677,13 +683,14 @@ def check_backward_matches_autograd_of_a_plain_torch_forward(lib=None):
             S = tx["initial_state"][n, h].T  # dk x dv
             for t in range(int(cu[n]), int(cu[n + 1])):
                 kt, qt, vt = tx["k"][t, hq], tx["q"][t, hq], tx["v"][t, h]
+                kt, qt = kt / torch.linalg.vector_norm(kt), qt / torch.linalg.vector_norm(qt)
                 S = torch.exp(tx["g"][t, h]) * S
                 S = S - tx["beta"][t, h] * torch.outer(kt, kt @ S) + tx["beta"][t, h] * torch.outer(kt, vt)
                 loss = loss + (torch.tensor(R[t, h]) * (0.7 * (S.T @ qt))).sum()
             loss = loss + (torch.tensor(Q[n, h]) * S.T).sum()
     loss.backward()
     d = oracle.prefill_backward(x["q"], x["k"], x["v"], x["g"], x["beta"], cu, R, x["initial_state"], Q, scale=0.7,
-                                lib=lib)
+                                lib=lib, l2norm=True)
     names = dict(q="dq", k="dk", v="dv", g="dg", beta="dbeta", initial_state="d_initial_state")
     for name, gname in names.items():
         ref = tx[name].grad.numpy()
