@@ -298,12 +298,13 @@ def gdn_chunk_prefill_backward_workspace_size(N, total_T, H, dk, dv, chunk=64) -
 
 
 def gdn_chunk_prefill_backward(q, k, v, g, beta, cu_seqlens, d_o, initial_state=None, d_final_state=None,
-                               chunk=64, scale=None, workspace=None, stream=None, grads=None):
+                               chunk=64, scale=None, workspace=None, stream=None, grads=None, l2norm=False):
     """Derivatives of a loss with respect to the prefill's inputs (see include/gdn.h),
     given d_o [total_T,H,dv] (q's dtype) and d_final_state [N,H,dv,dk] fp32 or None.
     Returns dict(dq, dk [total_T,H_qk,dk], dv [total_T,H,dv], dg, dbeta [total_T,H],
     d_initial_state [N,H,dv,dk]), fp32; `grads` may pass these tensors in. The
-    workspace (uint8 CUDA tensor) is allocated through torch when None."""
+    workspace (uint8 CUDA tensor) is allocated through torch when None. l2norm: the
+    forward normalised q and k per token (GDN_QK_L2NORM)."""
     import torch
     total_T, H_qk, dk = q.shape
     H, dv = v.shape[1], v.shape[-1]
@@ -329,7 +330,8 @@ def gdn_chunk_prefill_backward(q, k, v, g, beta, cu_seqlens, d_o, initial_state=
         _ptr(q), _ptr(k), _ptr(v), _ptr(g), _ptr(beta), _ptr(cu_seqlens), N, total_T, _ptr(initial_state),
         _ptr(d_o), _ptr(d_final_state), _ptr(grads["dq"]), _ptr(grads["dk"]), _ptr(grads["dv"]),
         _ptr(grads["dg"]), _ptr(grads["dbeta"]), _ptr(grads.get("d_initial_state")), H, H_qk, dk, dv, chunk,
-        float(scale), 0, _dtype_code(q), _ptr(workspace), workspace.numel(), _stream_ptr(stream, dev))
+        float(scale), GDN_QK_L2NORM if l2norm else 0, _dtype_code(q), _ptr(workspace), workspace.numel(),
+        _stream_ptr(stream, dev))
     _check(st)
     return grads
 

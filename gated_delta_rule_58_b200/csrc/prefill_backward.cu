@@ -10,6 +10,10 @@
 //     dk    = beta (D (v - u) - S~ w)
 //     dg    = <D, S~> - beta (u . w)
 //     D    <- alpha (D - beta k w^T)  (dL/dS_{t-1});   dL/dS_0 = D at the end.
+// With GDN_QK_L2NORM the relations read k^ = k / |k| and q^ = q / |q| (zero stays
+// zero) and the derivatives found for them are mapped back through the
+// normalisation, dk = (dk^ - k^ (k^ . dk^)) / |k| (likewise q), a linear map that is
+// applied to each CTA's partial sums before they are added up.
 //
 // Token-sequential SIMT. Every value column j of S (and of D) evolves on its own given
 // the token's k, q, v_j, alpha and beta, so one CTA takes 32 columns of one (sequence,
@@ -61,6 +65,7 @@ struct BwdArgs {
   int64_t total_T;
   int N, H, Hqk, C;
   float scale;
+  int l2norm;
   unsigned int* err;
 };
 
@@ -93,8 +98,9 @@ template <int D>
 constexpr size_t bwd_smem_bytes() {
   // token vectors [2][k, q, v, dO][D], gates [2][alpha, beta], column partials of dq
   // and dk and the prefetched S_{t-1} ([columns][stride] each), scalar partials
-  // [warps][2]; D threads
-  return (8 * D + 4 + 3 * kBwdCols * bwd_col_stride<D>() + 2 * (D / 32)) * sizeof(float);
+  // [warps][2], per-warp partial squared norms of k and q [2][warps][2] and partial
+  // projections [warps][2]; D threads
+  return (8 * D + 4 + 3 * kBwdCols * bwd_col_stride<D>() + 8 * (D / 32)) * sizeof(float);
 }
 
 __device__ __forceinline__ void cp_async16(float* dst, const float* src) {
@@ -122,6 +128,9 @@ gdn_prefill_backward_kernel(const BwdArgs a) {
   float* red_k = red_q + kBwdCols * RS;
   float* sp_buf = red_k + kBwdCols * RS;  // [kBwdCols][RS]: the next S_{t-1}, each thread its own entries
   float* red_s = sp_buf + kBwdCols * RS;  // [NW][2]
+  float* nrm = red_s + 2 * NW;            // [2][NW][2]: partial |k|^2, |q|^2 of a buffer's token
+  float* jred = nrm + 4 * NW;             // [NW][2]: partial k^ . dk^, q^ . dq^
+  const bool l2 = a.l2norm != 0;
 
   const int tid = threadIdx.x;
   constexpr int kBlocks = D / kBwdCols;   // column blocks per head
@@ -177,6 +186,32 @@ gdn_prefill_backward_kernel(const BwdArgs a) {
       gates[2 * buf] = expf(fg);
       gates[2 * buf + 1] = fb;
     }
+    if (l2) {  // per-warp partial squared norms (every thread holds one element)
+      float kk = fk * fk, qq = fq * fq;
+#pragma unroll
+      for (int off = 16; off > 0; off >>= 1) {
+        kk += __shfl_xor_sync(0xffffffffu, kk, off);
+        qq += __shfl_xor_sync(0xffffffffu, qq, off);
+      }
+      if ((tid & 31) == 0) {
+        nrm[(buf * NW + (tid >> 5)) * 2] = kk;
+        nrm[(buf * NW + (tid >> 5)) * 2 + 1] = qq;
+      }
+    }
+  };
+  // 1 / |k| and 1 / |q| of the token in buffer `buf` (1 without the normalisation)
+  auto inv_norms = [&](int buf, float* rk, float* rq) {
+    *rk = 1.f;
+    *rq = 1.f;
+    if (l2) {
+      float kk = 0.f, qq = 0.f;
+      for (int wi = 0; wi < NW; ++wi) {
+        kk += nrm[(buf * NW + wi) * 2];
+        qq += nrm[(buf * NW + wi) * 2 + 1];
+      }
+      *rk = kk > 0.f ? 1.f / sqrtf(kk) : 0.f;
+      *rq = qq > 0.f ? 1.f / sqrtf(qq) : 0.f;
+    }
   };
   // this thread's entries of a D-vector in shared memory
   auto load_vec = [&](const float* v, float* out) {
@@ -186,10 +221,13 @@ gdn_prefill_backward_kernel(const BwdArgs a) {
       out[4 * y] = f.x; out[4 * y + 1] = f.y; out[4 * y + 2] = f.z; out[4 * y + 3] = f.w;
     }
   };
-  // one token forward on this thread's entries of column col (as the forward kernel)
+  // one token forward on this thread's entries of column col (as the forward kernel;
+  // the update adds c k with c = beta (v_j - alpha (k^ . S_j)) / |k|)
   auto advance = [&](float* st, int buf) {
     const float* tb = tok + buf * 4 * D;
     const float alpha = gates[2 * buf], beta = gates[2 * buf + 1];
+    float rk, rq;
+    inv_norms(buf, &rk, &rq);
     float kv[PER];
     load_vec(tb, kv);
     float u = 0.f;
@@ -197,7 +235,7 @@ gdn_prefill_backward_kernel(const BwdArgs a) {
     for (int x = 0; x < PER; ++x) u = fmaf(kv[x], st[x], u);
 #pragma unroll
     for (int off = 1; off < TPC; off <<= 1) u += __shfl_xor_sync(0xffffffffu, u, off);
-    const float c = beta * (tb[2 * D + col] - alpha * u);
+    const float c = beta * (tb[2 * D + col] - alpha * (u * rk)) * rk;
 #pragma unroll
     for (int x = 0; x < PER; ++x) st[x] = fmaf(alpha, st[x], c * kv[x]);
   };
@@ -276,13 +314,15 @@ gdn_prefill_backward_kernel(const BwdArgs a) {
       const float* tb = tok + buf * 4 * D;
       const float vj = tb[2 * D + col], dOj = tb[3 * D + col];
       const float alpha = gates[2 * buf], beta = gates[2 * buf + 1];
+      float rk, rq;
+      inv_norms(buf, &rk, &rq);
       const size_t th = (size_t)t * a.H + h, tq = (size_t)t * a.Hqk + hq;
       // column j's terms of dq (S_t dO) first: S_t is not needed after them
-      float* rq = red_q + lcol * RS;
-      float* rk = red_k + lcol * RS;
+      float* rowq = red_q + lcol * RS;
+      float* rowk = red_k + lcol * RS;
 #pragma unroll
       for (int y = 0; y < NP; ++y)
-        *reinterpret_cast<float4*>(rq + piece(y)) = make_float4(sc[4 * y] * dOj, sc[4 * y + 1] * dOj,
+        *reinterpret_cast<float4*>(rowq + piece(y)) = make_float4(sc[4 * y] * dOj, sc[4 * y + 1] * dOj,
                                                                 sc[4 * y + 2] * dOj, sc[4 * y + 3] * dOj);
       float sp[PER];  // S_{t-1}
       cp_async_wait_all();
@@ -293,7 +333,7 @@ gdn_prefill_backward_kernel(const BwdArgs a) {
         float qv[PER];
         load_vec(tb + D, qv);
 #pragma unroll
-        for (int x = 0; x < PER; ++x) Dm[x] = fmaf(a.scale * qv[x], dOj, Dm[x]);
+        for (int x = 0; x < PER; ++x) Dm[x] = fmaf(a.scale * rq * qv[x], dOj, Dm[x]);
       }
       float kv[PER];
       load_vec(tb, kv);
@@ -309,7 +349,7 @@ gdn_prefill_backward_kernel(const BwdArgs a) {
         pu += __shfl_xor_sync(0xffffffffu, pu, off);
         pw += __shfl_xor_sync(0xffffffffu, pw, off);
       }
-      const float u = alpha * pu, w = pw, vmu = vj - u;
+      const float u = alpha * pu * rk, w = pw * rk, vmu = vj - u;
       // column j's terms of dk (D (v - u) - S~ w) and of dg
       float sdg = 0.f;
 #pragma unroll
@@ -322,7 +362,7 @@ gdn_prefill_backward_kernel(const BwdArgs a) {
           kk[z] = Dm[x] * vmu - stl * w;
           sdg = fmaf(Dm[x], stl, sdg);
         }
-        *reinterpret_cast<float4*>(rk + piece(y)) = make_float4(kk[0], kk[1], kk[2], kk[3]);
+        *reinterpret_cast<float4*>(rowk + piece(y)) = make_float4(kk[0], kk[1], kk[2], kk[3]);
       }
       float sdb = 0.f;
       if (part == 0) {
@@ -331,9 +371,10 @@ gdn_prefill_backward_kernel(const BwdArgs a) {
         a.dv[th * D + col] = beta * w;
       }
       // dL/dS_{t-1}; S_{t-1} becomes the next token's S_t
+      const float bw = beta * w * rk;
 #pragma unroll
       for (int x = 0; x < PER; ++x) {
-        Dm[x] = alpha * (Dm[x] - beta * w * kv[x]);
+        Dm[x] = alpha * (Dm[x] - bw * kv[x]);
         sc[x] = sp[x];
       }
 #pragma unroll
@@ -353,8 +394,30 @@ gdn_prefill_backward_kernel(const BwdArgs a) {
           sq += red_q[j * RS + tid];
           sk += red_k[j * RS + tid];
         }
-        atomicAdd(a.dq + tq * D + tid, a.scale * sq);
-        atomicAdd(a.dk + tq * D + tid, beta * sk);
+        float gq = a.scale * sq, gk = beta * sk;  // this CTA's part of dq^, dk^
+        if (l2) {  // through the normalisation: (g - x^ (x^ . g)) / |x|
+          const float kh = tb[tid] * rk, qh = tb[D + tid] * rq;
+          float pk = kh * gk, pq = qh * gq;
+#pragma unroll
+          for (int off = 16; off > 0; off >>= 1) {
+            pk += __shfl_xor_sync(0xffffffffu, pk, off);
+            pq += __shfl_xor_sync(0xffffffffu, pq, off);
+          }
+          if ((tid & 31) == 0) {
+            jred[2 * (tid >> 5)] = pk;
+            jred[2 * (tid >> 5) + 1] = pq;
+          }
+          __syncthreads();
+          float dotk = 0.f, dotq = 0.f;
+          for (int wi = 0; wi < NW; ++wi) {
+            dotk += jred[2 * wi];
+            dotq += jred[2 * wi + 1];
+          }
+          gk = (gk - kh * dotk) * rk;
+          gq = (gq - qh * dotq) * rq;
+        }
+        atomicAdd(a.dq + tq * D + tid, gq);
+        atomicAdd(a.dk + tq * D + tid, gk);
       }
       if (tid == 0) {
         float g_sum = 0.f, b_sum = 0.f;
@@ -428,7 +491,7 @@ extern "C" gdn_status_t gdn_chunk_prefill_backward(
   if (st != GDN_OK) return st;
   if (H_qk < 1 || H % H_qk != 0)
     return fail(GDN_ERR_INVALID_ARG, "gdn_chunk_prefill_backward: H must be a positive multiple of H_qk");
-  if (flags != 0) return fail(GDN_ERR_UNSUPPORTED, "gdn_chunk_prefill_backward: no flags supported (q/k normalisation)");
+  if ((flags & ~(uint32_t)GDN_QK_L2NORM) != 0) return fail(GDN_ERR_INVALID_ARG, "gdn_chunk_prefill_backward: unknown flags");
   if (!(in_dtype == GDN_BF16 || in_dtype == GDN_F32))
     return fail(GDN_ERR_INVALID_ARG, "gdn_chunk_prefill_backward: unknown dtype");
   if (N == 0) return gdn::ok();
@@ -467,7 +530,8 @@ extern "C" gdn_status_t gdn_chunk_prefill_backward(
   a.ckpt = static_cast<float*>(workspace);
   a.scratch = reinterpret_cast<float*>(static_cast<uint8_t*>(workspace) + L.scratch_off);
   a.ck_slots = L.ck_slots;
-  a.total_T = total_T; a.N = N; a.H = H; a.Hqk = H_qk; a.C = chunk; a.scale = scale; a.err = err;
+  a.total_T = total_T; a.N = N; a.H = H; a.Hqk = H_qk; a.C = chunk; a.scale = scale;
+  a.l2norm = (flags & GDN_QK_L2NORM) != 0; a.err = err;
   const bool bf = in_dtype == GDN_BF16;
   switch (dk) {
     case 32: return bf ? gdn::launch_bwd<32, __nv_bfloat16>(a, s) : gdn::launch_bwd<32, float>(a, s);

@@ -273,7 +273,9 @@ const char* gdn_last_error(void);
  * zero), for training. The pages give no backward pass: this is the chain rule on
  * the gated delta rule's token relations S_t = alpha_t (I - beta_t k_t k_t^T)
  * S_{t-1} + beta_t k_t v_t^T, o_t = scale S_t^T q_t, alpha_t = exp(g_t), walked from
- * the last token to the first (one Householder per token; no q/k normalisation).
+ * the last token to the first (one Householder per token). With GDN_QK_L2NORM the
+ * relations read k / |k| and q / |q| (as in gdn_chunk_prefill) and the derivatives
+ * are taken through that normalisation (zero for a zero vector).
  *
  * Inputs as gdn_chunk_prefill (q, k [total_T, H_qk, dk]; v [total_T, H, dv]; g, beta
  * [total_T, H] fp32; cu_seqlens [N+1] int32 on the device; initial_state [N, H, dv,
@@ -282,7 +284,7 @@ const char* gdn_last_error(void);
  * up), d_v [total_T, H, dv], d_g, d_beta [total_T, H] (d_q, d_k, d_g and d_beta are
  * cleared on `stream` first), d_initial_state [N, H, dv, dk] K-last or NULL (not
  * written).
- * dk == dv in {32, 64, 128}; flags must be 0 (GDN_ERR_UNSUPPORTED otherwise);
+ * dk == dv in {32, 64, 128}; flags: GDN_QK_L2NORM or 0 (GDN_ERR_INVALID_ARG otherwise);
  * q, k, v, d_o, d_q, d_k and the state pointers 16-byte aligned.
  *
  * Token-sequential, one CTA per 32 value columns of a (sequence, head) (the columns

@@ -22,21 +22,21 @@ def _upstream(inp, seed, dtype):
     return d_o, d_fin
 
 
-def _run(inp, d_o, d_fin, chunk):
+def _run(inp, d_o, d_fin, chunk, l2norm=False):
     dev = [x.to(DEV) if x is not None else None
            for x in (inp.q, inp.k, inp.v, inp.g, inp.beta, inp.cu_seqlens, inp.initial_state, d_o, d_fin)]
     q, k, v, g, beta, cu, init, do, dfin = dev
     out = gdn.gdn_chunk_prefill_backward(q, k, v, g, beta, cu, do, initial_state=init, d_final_state=dfin,
-                                         chunk=chunk, scale=inp.scale)
+                                         chunk=chunk, scale=inp.scale, l2norm=l2norm)
     torch.cuda.synchronize()
     assert gdn.gdn_get_device_error() == 0
     return out
 
 
-def _check(inp, d_o, d_fin, chunk, what):
-    out = _run(inp, d_o, d_fin, chunk)
+def _check(inp, d_o, d_fin, chunk, what, l2norm=False):
+    out = _run(inp, d_o, d_fin, chunk, l2norm)
     ref = oracle.prefill_backward(inp.q, inp.k, inp.v, inp.g, inp.beta, inp.cu_seqlens, d_o, inp.initial_state,
-                                  d_fin, scale=inp.scale)
+                                  d_fin, scale=inp.scale, l2norm=l2norm)
     for name in ("dq", "dk", "dv", "dg", "dbeta", "d_initial_state"):
         assert_close(out[name], ref[name], what=f"{what} {name}")
 
@@ -81,3 +81,19 @@ def test_backward_leaves_no_trace_between_calls():
     for name in ("dq", "dk", "dg", "dbeta"):
         err = (a[name] - b[name]).abs().max() / b[name].abs().max()
         assert err < 1e-5, (name, float(err))
+
+
+@pytest.mark.parametrize("chunk", [16, 64])
+def test_backward_through_the_qk_normalisation(chunk):
+    """Raw (unnormalised) q and k with GDN_QK_L2NORM, grouped heads, varlen."""
+    inp = inputs.prefill_inputs([180, 0, 77], 4, 128, 128, seed=100, g_range=(0.0, 0.05), H_qk=2,
+                                normalize_qk=False)
+    d_o, d_fin = _upstream(inp, 101, torch.bfloat16)
+    _check(inp, d_o, d_fin, chunk, f"bwd l2norm chunk={chunk}", l2norm=True)
+
+
+def test_backward_through_the_qk_normalisation_small_heads_fp32():
+    inp = inputs.prefill_inputs([90, 41], 2, 64, 64, seed=102, dtype=torch.float32, g_range=(0.0, 0.05),
+                                normalize_qk=False)
+    d_o, d_fin = _upstream(inp, 103, torch.float32)
+    _check(inp, d_o, d_fin, 16, "bwd l2norm d=64", l2norm=True)

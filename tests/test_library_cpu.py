@@ -183,7 +183,7 @@ def test_backward_entry_points_reject_on_host(L):
                                             a["init"], a["d_o"], a["dfin"], a["dq"], a["dk_"], a["dv_"], a["dg"],
                                             a["db"], a["dinit"], a["H"], a["Hqk"], a["dk"], a["dv"], a["chunk"],
                                             a["scale"], a["flags"], a["dt"], a["ws"], a["wsb"], a["stream"])
-    assert call(flags=gdn.GDN_QK_L2NORM) == gdn.GDN_ERR_UNSUPPORTED
+    assert call(flags=0x80) == gdn.GDN_ERR_INVALID_ARG  # unknown flag
     assert call(Hqk=3) == gdn.GDN_ERR_INVALID_ARG
     assert call(d_o=None) == gdn.GDN_ERR_INVALID_ARG
     assert call(dq=FAKE + 4) == gdn.GDN_ERR_INVALID_ARG  # misaligned
