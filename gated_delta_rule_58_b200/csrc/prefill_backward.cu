@@ -16,9 +16,9 @@
 // applied to each CTA's partial sums before they are added up.
 //
 // Token-sequential SIMT. Every value column j of S (and of D) evolves on its own given
-// the token's k, q, v_j, alpha and beta, so one CTA takes 32 columns of one (sequence,
-// head) (dv / 32 CTAs per head); value column j is owned by dk / 32 adjacent lanes, 32
-// of its dk entries each. The states S_{t-1} the walk needs are recomputed:
+// the token's k, q, v_j, alpha and beta, so one CTA (one warp) takes 1024 / dk columns
+// of one (sequence, head) (many small CTAs per SM); value column j is owned by dk / 32
+// adjacent lanes, 32 of its dk entries each. The states S_{t-1} the walk needs are recomputed:
 //   1. forward over the sequence, writing the state at the start of every chunk of
 //      C tokens to the workspace (checkpoints);
 //   2. for each chunk, last to first: recompute the chunk's states from its
@@ -86,7 +86,10 @@ BwdLayout bwd_layout(int N, int64_t total_T, int H, int D, int C) {
   return L;
 }
 
-constexpr int kBwdCols = 32;  // value columns per CTA
+// value columns per CTA: one warp per CTA (1024 / dk columns of dk / 32 lanes each),
+// so many small CTAs share an SM and a barrier spans one warp
+template <int D>
+constexpr int bwd_cols() { return 1024 / D; }
 
 // Shared-memory stride of one column in the [columns][D entries] buffers, padded so
 // that the eight lanes of a quarter warp (two columns x four 16-byte pieces) store to
@@ -95,12 +98,17 @@ template <int D>
 constexpr int bwd_col_stride() { return D + 16; }
 
 template <int D>
+constexpr int bwd_threads() { return bwd_cols<D>() * (D / 32); }
+template <int D>
+constexpr int bwd_warps() { return (bwd_threads<D>() + 31) / 32; }
+
+template <int D>
 constexpr size_t bwd_smem_bytes() {
   // token vectors [2][k, q, v, dO][D], gates [2][alpha, beta], column partials of dq
   // and dk and the prefetched S_{t-1} ([columns][stride] each), scalar partials
   // [warps][2], per-warp partial squared norms of k and q [2][warps][2] and partial
-  // projections [warps][2]; D threads
-  return (8 * D + 4 + 3 * kBwdCols * bwd_col_stride<D>() + 8 * (D / 32)) * sizeof(float);
+  // projections [warps][2]; bwd_cols * D / 32 threads
+  return (8 * D + 4 + 3 * bwd_cols<D>() * bwd_col_stride<D>() + 8 * bwd_warps<D>()) * sizeof(float);
 }
 
 __device__ __forceinline__ void cp_async16(float* dst, const float* src) {
@@ -112,11 +120,13 @@ __device__ __forceinline__ void cp_async_wait_all() {
 }
 
 template <int D, typename TIn>
-__global__ void __launch_bounds__(D)
+__global__ void __launch_bounds__(bwd_threads<D>())
 gdn_prefill_backward_kernel(const BwdArgs a) {
   constexpr int TPC = D / 32;  // threads per state column
-  constexpr int NT = kBwdCols * TPC;  // == D
-  static_assert(NT == D, "one thread per dk entry of the token vectors");
+  constexpr int kBwdCols = bwd_cols<D>();
+  constexpr int NT = kBwdCols * TPC;
+  constexpr int EPT = D / NT;  // dk entries of the token vectors per thread
+  static_assert(NT * EPT == D && NT % 32 == 0, "whole warps, whole vectors");
   constexpr int PER = 32;      // entries of the column per thread
   constexpr int NP = PER / 4;  // 16-byte pieces per thread
   constexpr int NW = NT / 32;
@@ -156,18 +166,21 @@ gdn_prefill_backward_kernel(const BwdArgs a) {
   const TIn* vp = static_cast<const TIn*>(a.v);
   const TIn* dop = static_cast<const TIn*>(a.d_o);
 
-  // A token's k, q, v, dO (thread tid holds element tid) and gates are
+  // A token's k, q, v, dO and gates are
   // fetched into registers, then committed to shared-memory buffer `buf` (two
   // buffers: the barrier of the token in between orders every read of a buffer
   // before its refill).
-  float fk = 0.f, fq = 0.f, fv = 0.f, fdo = 0.f, fg = 0.f, fb = 0.f;
+  // (thread tid holds entries tid + NT e, e < EPT)
+  float fk[EPT], fq[EPT], fv[EPT], fdo[EPT], fg = 0.f, fb = 0.f;
   auto fetch = [&](int64_t t) {
     const size_t th = (size_t)t * a.H + h, tq = (size_t)t * a.Hqk + hq;
-    if (tid < D) {
-      fk = to_f32(kp[tq * D + tid]);
-      fq = to_f32(qp[tq * D + tid]);
-      fv = to_f32(vp[th * D + tid]);
-      fdo = to_f32(dop[th * D + tid]);
+#pragma unroll
+    for (int e = 0; e < EPT; ++e) {
+      const int i = tid + NT * e;
+      fk[e] = to_f32(kp[tq * D + i]);
+      fq[e] = to_f32(qp[tq * D + i]);
+      fv[e] = to_f32(vp[th * D + i]);
+      fdo[e] = to_f32(dop[th * D + i]);
     }
     if (tid == 0) {
       fg = a.g[th];
@@ -176,18 +189,25 @@ gdn_prefill_backward_kernel(const BwdArgs a) {
   };
   auto commit = [&](int buf) {
     float* tb = tok + buf * 4 * D;
-    if (tid < D) {
-      tb[tid] = fk;
-      tb[D + tid] = fq;
-      tb[2 * D + tid] = fv;
-      tb[3 * D + tid] = fdo;
+#pragma unroll
+    for (int e = 0; e < EPT; ++e) {
+      const int i = tid + NT * e;
+      tb[i] = fk[e];
+      tb[D + i] = fq[e];
+      tb[2 * D + i] = fv[e];
+      tb[3 * D + i] = fdo[e];
     }
     if (tid == 0) {
       gates[2 * buf] = expf(fg);
       gates[2 * buf + 1] = fb;
     }
-    if (l2) {  // per-warp partial squared norms (every thread holds one element)
-      float kk = fk * fk, qq = fq * fq;
+    if (l2) {  // per-warp partial squared norms
+      float kk = 0.f, qq = 0.f;
+#pragma unroll
+      for (int e = 0; e < EPT; ++e) {
+        kk = fmaf(fk[e], fk[e], kk);
+        qq = fmaf(fq[e], fq[e], qq);
+      }
 #pragma unroll
       for (int off = 16; off > 0; off >>= 1) {
         kk += __shfl_xor_sync(0xffffffffu, kk, off);
@@ -387,17 +407,28 @@ gdn_prefill_backward_kernel(const BwdArgs a) {
         red_s[2 * (tid >> 5) + 1] = sdb;
       }
       __syncthreads();
-      {  // entry tid of dq and of dk over this CTA's columns
-        float sq = 0.f, sk = 0.f;
+      {  // entries tid + NT e of dq and of dk over this CTA's columns
+        float gq[EPT], gk[EPT];  // this CTA's part of dq^, dk^
+#pragma unroll
+        for (int e = 0; e < EPT; ++e) {
+          const int i = tid + NT * e;
+          float sq = 0.f, sk = 0.f;
 #pragma unroll 8
-        for (int j = 0; j < kBwdCols; ++j) {
-          sq += red_q[j * RS + tid];
-          sk += red_k[j * RS + tid];
+          for (int j = 0; j < kBwdCols; ++j) {
+            sq += red_q[j * RS + i];
+            sk += red_k[j * RS + i];
+          }
+          gq[e] = a.scale * sq;
+          gk[e] = beta * sk;
         }
-        float gq = a.scale * sq, gk = beta * sk;  // this CTA's part of dq^, dk^
         if (l2) {  // through the normalisation: (g - x^ (x^ . g)) / |x|
-          const float kh = tb[tid] * rk, qh = tb[D + tid] * rq;
-          float pk = kh * gk, pq = qh * gq;
+          float pk = 0.f, pq = 0.f;
+#pragma unroll
+          for (int e = 0; e < EPT; ++e) {
+            const int i = tid + NT * e;
+            pk = fmaf(tb[i] * rk, gk[e], pk);
+            pq = fmaf(tb[D + i] * rq, gq[e], pq);
+          }
 #pragma unroll
           for (int off = 16; off > 0; off >>= 1) {
             pk += __shfl_xor_sync(0xffffffffu, pk, off);
@@ -413,11 +444,18 @@ gdn_prefill_backward_kernel(const BwdArgs a) {
             dotk += jred[2 * wi];
             dotq += jred[2 * wi + 1];
           }
-          gk = (gk - kh * dotk) * rk;
-          gq = (gq - qh * dotq) * rq;
+#pragma unroll
+          for (int e = 0; e < EPT; ++e) {
+            const int i = tid + NT * e;
+            gk[e] = (gk[e] - tb[i] * rk * dotk) * rk;
+            gq[e] = (gq[e] - tb[D + i] * rq * dotq) * rq;
+          }
         }
-        atomicAdd(a.dq + tq * D + tid, gq);
-        atomicAdd(a.dk + tq * D + tid, gk);
+#pragma unroll
+        for (int e = 0; e < EPT; ++e) {
+          atomicAdd(a.dq + tq * D + tid + NT * e, gq[e]);
+          atomicAdd(a.dk + tq * D + tid + NT * e, gk[e]);
+        }
       }
       if (tid == 0) {
         float g_sum = 0.f, b_sum = 0.f;
@@ -447,7 +485,7 @@ gdn_status_t launch_bwd(const BwdArgs& a, cudaStream_t stream) {
       }))
     return fail(e != cudaSuccess ? GDN_ERR_CUDA : GDN_ERR_UNSUPPORTED,
                 std::string("prefill backward: setup: ") + (e != cudaSuccess ? cudaGetErrorString(e) : "device index too large"));
-  kernel<<<(unsigned)((long long)a.N * a.H * (D / kBwdCols)), D, smem, stream>>>(a);
+  kernel<<<(unsigned)((long long)a.N * a.H * (D / bwd_cols<D>())), bwd_threads<D>(), smem, stream>>>(a);
   return check_launch("gdn_chunk_prefill_backward");
 }
 
@@ -464,7 +502,7 @@ gdn_status_t bwd_check_shape(int N, int64_t total_T, int H, int dk, int dv, int 
   if (dk != dv || (dk != 32 && dk != 64 && dk != 128))
     return fail(GDN_ERR_UNSUPPORTED, "gdn_chunk_prefill_backward: dk == dv in {32, 64, 128}");
   if (chunk > 4096) return fail(GDN_ERR_UNSUPPORTED, "gdn_chunk_prefill_backward: chunk <= 4096");
-  if ((long long)N * H * (dk / 32) >= (1LL << 31))
+  if ((long long)N * H * (dk * dk / 1024) >= (1LL << 31))  // column blocks: dk / (1024 / dk) per head
     return fail(GDN_ERR_UNSUPPORTED, "gdn_chunk_prefill_backward: N * H too large");
   return gdn::ok();
 }

@@ -287,8 +287,8 @@ const char* gdn_last_error(void);
  * dk == dv in {32, 64, 128}; flags: GDN_QK_L2NORM or 0 (GDN_ERR_INVALID_ARG otherwise);
  * q, k, v, d_o, d_q, d_k and the state pointers 16-byte aligned.
  *
- * Token-sequential, one CTA per 32 value columns of a (sequence, head) (the columns
- * of the state evolve independently): a forward pass writes the state at the start of
+ * Token-sequential, one CTA (one warp) per 1024 / dk value columns of a (sequence,
+ * head) (the columns of the state evolve independently): a forward pass writes the state at the start of
  * every `chunk` tokens to the workspace, then each chunk, last to first, is
  * recomputed from its checkpoint into the workspace and walked backwards. d_q, d_k,
  * d_g and d_beta are sums over column blocks (and grouped heads) taken with fp32
