@@ -773,8 +773,15 @@ __device__ void state_role(const Smem& sm, const PrefillShape& s, const PrefillA
 #pragma unroll
       for (int q = 0; q < 4; ++q) {
         float ud[8];
-#pragma unroll
-        for (int x = 0; x < 8; ++x) ud[x] = u[8 * q + x] * vec[V_DD + 32 * hq + 8 * q + x];
+        {  // U diag(dd), two entries per packed multiply (each rounded as a scalar product)
+          const float4 d0 = *reinterpret_cast<const float4*>(vec + V_DD + 32 * hq + 8 * q);
+          const float4 d1 = *reinterpret_cast<const float4*>(vec + V_DD + 32 * hq + 8 * q + 4);
+          const float2 p0 = __fmul2_rn(make_float2(u[8 * q], u[8 * q + 1]), make_float2(d0.x, d0.y));
+          const float2 p1 = __fmul2_rn(make_float2(u[8 * q + 2], u[8 * q + 3]), make_float2(d0.z, d0.w));
+          const float2 p2 = __fmul2_rn(make_float2(u[8 * q + 4], u[8 * q + 5]), make_float2(d1.x, d1.y));
+          const float2 p3 = __fmul2_rn(make_float2(u[8 * q + 6], u[8 * q + 7]), make_float2(d1.z, d1.w));
+          ud[0] = p0.x; ud[1] = p0.y; ud[2] = p1.x; ud[3] = p1.y; ud[4] = p2.x; ud[5] = p2.y; ud[6] = p3.x; ud[7] = p3.y;
+        }
         st_sw128_chunk(sm.base + OFF_U16, j, 4 * hq + q, u + 8 * q);
         st_sw128_chunk(sm.base + OFF_UDD, j, 4 * hq + q, ud);
       }
@@ -810,7 +817,11 @@ __device__ void state_role(const Smem& sm, const PrefillShape& s, const PrefillA
         for (int x = 0; x < 16; ++x) hv[x] = tc::half2_bits(v[2 * x], v[2 * x + 1]);
         tc::tmem_st16_bits(tl + COL_SH + hq * 16, hv);
 #pragma unroll
-        for (int x = 0; x < 32; ++x) v[x] *= gnext;
+        for (int x = 0; x < 32; x += 2) {
+          const float2 p = __fmul2_rn(make_float2(v[x], v[x + 1]), make_float2(gnext, gnext));
+          v[x] = p.x;
+          v[x + 1] = p.y;
+        }
         tc::tmem_st16(tl + COL_S + hq * 32, v);
         tc::tmem_st16(tl + COL_S + hq * 32 + 16, v + 16);
       } else if (a.final_state) {
@@ -844,13 +855,20 @@ __device__ void state_role(const Smem& sm, const PrefillShape& s, const PrefillA
 #pragma unroll
       for (int q = 0; q < 8; ++q) gm[q] = *reinterpret_cast<const float4*>(vec + V_GAM + hq * 32 + 4 * q);
       tc::wait_ld();
+      const float2 sc2 = make_float2(sc, sc);  // rows r, r + 1 per packed FMA / multiply
 #pragma unroll
       for (int q = 0; q < 8; ++q) {
         const int r = hq * 32 + 4 * q;
-        store_out(stage + (r + 0) * D + j, sc * fmaf(gm[q].x, o1[4 * q + 0], o2[4 * q + 0]));
-        store_out(stage + (r + 1) * D + j, sc * fmaf(gm[q].y, o1[4 * q + 1], o2[4 * q + 1]));
-        store_out(stage + (r + 2) * D + j, sc * fmaf(gm[q].z, o1[4 * q + 2], o2[4 * q + 2]));
-        store_out(stage + (r + 3) * D + j, sc * fmaf(gm[q].w, o1[4 * q + 3], o2[4 * q + 3]));
+        const float2 a = __fmul2_rn(sc2, __ffma2_rn(make_float2(gm[q].x, gm[q].y),
+                                                     make_float2(o1[4 * q], o1[4 * q + 1]),
+                                                     make_float2(o2[4 * q], o2[4 * q + 1])));
+        const float2 b = __fmul2_rn(sc2, __ffma2_rn(make_float2(gm[q].z, gm[q].w),
+                                                     make_float2(o1[4 * q + 2], o1[4 * q + 3]),
+                                                     make_float2(o2[4 * q + 2], o2[4 * q + 3])));
+        store_out(stage + (r + 0) * D + j, a.x);
+        store_out(stage + (r + 1) * D + j, a.y);
+        store_out(stage + (r + 2) * D + j, b.x);
+        store_out(stage + (r + 3) * D + j, b.y);
       }
     }
     tc::fence_proxy_async_smem();
