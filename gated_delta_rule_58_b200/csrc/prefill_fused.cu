@@ -618,6 +618,10 @@ __device__ void prep_role(const Smem& sm, uint32_t tmem, int nchunks, unsigned i
   // both P tiles start as zeros: the strictly upper 16-byte chunks are never written
   for (int i = t; i < 2 * P_BUF / 16; i += 128)
     *reinterpret_cast<uint4*>(sm.base + OFF_P16 + 16 * i) = make_uint4(0u, 0u, 0u, 0u);
+  // so does T: the solve writes only its lower blocks (with zeros above the diagonal
+  // inside the 16x16 diagonal blocks), so T's upper triangle stays zero for good
+  for (int i = t; i < C * C / 4; i += 128) reinterpret_cast<float4*>(sm.T())[i] = make_float4(0.f, 0.f, 0.f, 0.f);
+  tc::named_sync(kBarPrep, 128);
   for (int c = 0; c < nchunks; ++c) {
     const int b = c & 1;
     if (!wait_bar(sm, B_L0 + b, (c >> 1) & 1, err)) return;
@@ -665,8 +669,8 @@ __device__ void prep_role(const Smem& sm, uint32_t tmem, int nchunks, unsigned i
     // MMA has read the old ones
     if (c >= 1 && !wait_bar(sm, B_M2, (c - 1) & 1, err)) return;
     {
-      // row i of T times the column scales; the row and the scales are loaded
-      // up front (independent loads), the upper part is written as zeros
+      // row i of T times the column scales (T's upper triangle is zero); the row
+      // and the scales are loaded up front (independent loads)
       const int mat = t >> 6, i = t & 63;
       const float* colscale = vec + (mat ? V_BETA : V_BG);
       uint8_t* tile = sm.base + (mat ? OFF_TPP : OFF_TP);
@@ -679,11 +683,11 @@ __device__ void prep_role(const Smem& sm, uint32_t tmem, int nchunks, unsigned i
 #pragma unroll
       for (int cc = 0; cc < 8; ++cc) {
         const float4 a0 = tr[2 * cc], a1 = tr[2 * cc + 1], s0 = cs[2 * cc], s1 = cs[2 * cc + 1];
-        const float prod[8] = {a0.x * s0.x, a0.y * s0.y, a0.z * s0.z, a0.w * s0.w,
-                               a1.x * s1.x, a1.y * s1.y, a1.z * s1.z, a1.w * s1.w};
-        float v[8];
-#pragma unroll
-        for (int m = 0; m < 8; ++m) v[m] = (cc * 8 + m <= i) ? prod[m] : 0.f;
+        const float2 p0 = __fmul2_rn(make_float2(a0.x, a0.y), make_float2(s0.x, s0.y));
+        const float2 p1 = __fmul2_rn(make_float2(a0.z, a0.w), make_float2(s0.z, s0.w));
+        const float2 p2 = __fmul2_rn(make_float2(a1.x, a1.y), make_float2(s1.x, s1.y));
+        const float2 p3 = __fmul2_rn(make_float2(a1.z, a1.w), make_float2(s1.z, s1.w));
+        const float v[8] = {p0.x, p0.y, p1.x, p1.y, p2.x, p2.y, p3.x, p3.y};
         st_sw128_chunk(tile, i, cc, v);
       }
     }
