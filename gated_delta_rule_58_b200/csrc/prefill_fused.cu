@@ -575,21 +575,23 @@ __device__ __forceinline__ void solve_merge(const Smem& sm, int t) {
 }
 
 // Columns 32 hq .. 32 hq + 31 of A row t: beta_t 2^(G_t - G_j) x_j for j < t (base-2
-// cumulative gates), 16-byte chunks right of the diagonal skipped (the solve never
-// reads them). The decays are computed unconditionally (independent, so they
-// pipeline); entries right of the diagonal may overflow and are masked.
+// cumulative gates), 16-byte chunks right of the diagonal skipped. The entries with
+// j >= t inside the boundary chunk are stored unmasked: the solve masks them itself
+// (the forward substitution reads A_rk only for k < r; every other reader takes
+// blocks strictly below the diagonal). Products two at a time, rounded as
+// (beta 2^dG) x per entry.
 __device__ __forceinline__ void a_row_half(float* A, int t, int hq, float bi, float Gi, const float* G,
                                            const float* x) {
 #pragma unroll
   for (int q = 0; q < 8; ++q) {
     const int j0 = 32 * hq + 4 * q;
     const float4 g4 = *reinterpret_cast<const float4*>(G + j0);
-    float4 v;
-    v.x = (j0 + 0 < t) ? bi * exp2_approx(Gi - g4.x) * x[4 * q + 0] : 0.f;
-    v.y = (j0 + 1 < t) ? bi * exp2_approx(Gi - g4.y) * x[4 * q + 1] : 0.f;
-    v.z = (j0 + 2 < t) ? bi * exp2_approx(Gi - g4.z) * x[4 * q + 2] : 0.f;
-    v.w = (j0 + 3 < t) ? bi * exp2_approx(Gi - g4.w) * x[4 * q + 3] : 0.f;
-    if (j0 < t) *row_chunk(A, t, j0 >> 2) = v;
+    const float2 bb = make_float2(bi, bi);
+    const float2 lo = __fmul2_rn(__fmul2_rn(bb, make_float2(exp2_approx(Gi - g4.x), exp2_approx(Gi - g4.y))),
+                                 make_float2(x[4 * q + 0], x[4 * q + 1]));
+    const float2 hi = __fmul2_rn(__fmul2_rn(bb, make_float2(exp2_approx(Gi - g4.z), exp2_approx(Gi - g4.w))),
+                                 make_float2(x[4 * q + 2], x[4 * q + 3]));
+    if (j0 < t) *row_chunk(A, t, j0 >> 2) = make_float4(lo.x, lo.y, hi.x, hi.y);
   }
 }
 
