@@ -190,3 +190,23 @@ def test_backward_entry_points_reject_on_host(L):
     assert call(wsb=16) == gdn.GDN_ERR_WORKSPACE
     assert call(ws=None) == gdn.GDN_ERR_WORKSPACE
     assert call(N=0) == gdn.GDN_OK  # nothing to do, nothing launched
+
+
+def test_cp_finish_rejects_on_host(L):
+    def call(**kw):
+        a = dict(q=FAKE, k=FAKE, v=FAKE, g=FAKE, beta=FAKE, cu=FAKE, N=1, T=64, start=None, fin=None, o=FAKE, H=2,
+                 Hqk=2, dk=128, dv=128, chunk=64, scale=0.1, flags=0, dt=gdn.GDN_BF16, odt=gdn.GDN_BF16, ws=FAKE,
+                 wsb=1 << 40, stream=None)
+        a.update(kw)
+        return L.gdn_cp_finish(a["q"], a["k"], a["v"], a["g"], a["beta"], a["cu"], a["N"], a["T"], a["start"],
+                               a["fin"], a["o"], a["H"], a["Hqk"], a["dk"], a["dv"], a["chunk"], a["scale"],
+                               a["flags"], a["dt"], a["odt"], a["ws"], a["wsb"], a["stream"])
+    assert call(chunk=32) == gdn.GDN_ERR_UNSUPPORTED      # the segment passes need chunk 64
+    assert call(dk=64, dv=64) == gdn.GDN_ERR_UNSUPPORTED
+    assert call(Hqk=3) == gdn.GDN_ERR_INVALID_ARG
+    assert call(cu=None) == gdn.GDN_ERR_INVALID_ARG
+    assert call(o=FAKE + 8) == gdn.GDN_ERR_INVALID_ARG     # misaligned output
+    assert call(odt=7) == gdn.GDN_ERR_INVALID_ARG
+    assert call(ws=None) == gdn.GDN_ERR_WORKSPACE
+    assert call(wsb=16) == gdn.GDN_ERR_WORKSPACE
+    assert call(N=0) == gdn.GDN_OK
