@@ -37,6 +37,9 @@ if ROOT not in sys.path:
 
 METRIC = "GDN decode state GB/s (% of 8 TB/s); chunked prefill tokens/s (% roofline)"
 NOMINAL_HBM_GBS = 8000.0
+# fp32 FMA peak of a B200 from its unit counts: 148 SMs x 128 fp32 lanes x 2 flops at
+# the 1965 MHz maximum SM clock (TFLOP/s); the roofline of SIMT fp32 arithmetic
+FP32_SIMT_TFLOPS = 148 * 128 * 2 * 1.965e9 / 1e12
 FALLBACK_PEAKS = {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "bf16_tflops_sustained": 1400.0}
 
 
@@ -460,6 +463,17 @@ def bench_prefill(key, steps, warmup, ws, rank, peaks, algo=None):
     return res
 
 
+def backward_alg_flops(inp):
+    """Algorithmic fp32 flops of one backward step, per token and value head and per
+    entry of the dk x dv state: one forward step to regain S_t (u = S~^T k and the
+    update, 2 FMAs) and the reverse step (D += q dO^T, the terms S_t dO of dq, w = D^T k,
+    D (v - u) and S~ w of dk, <D, S~> of dg, D <- alpha (D - beta k w^T): 7.5 FMAs) =
+    19 flops. The recomputation of the states from checkpoints is not counted."""
+    total, _, dk = inp.q.shape
+    H, dv = inp.v.shape[1], inp.v.shape[-1]
+    return 19.0 * total * H * dk * dv
+
+
 def backward_alg_bytes(inp):
     """Algorithmic HBM bytes of one backward step: q, k, v and d_o read (input dtype),
     g and beta read, dq, dk, dv, dg, dbeta written (fp32), and per (sequence, head) the
@@ -512,15 +526,21 @@ def bench_backward(key, steps, warmup, ws, rank, peaks):
     ms = total_ms / steps
     t = ms * 1e-3
     alg_b = backward_alg_bytes(inp)
-    achieved = alg_b / t / 1e9
+    alg_f = backward_alg_flops(inp)
+    # the arithmetic, not the memory, bounds this step: its flops take about 11x as
+    # long at the fp32 peak as its bytes at the copy peak
+    achieved = alg_f / t / 1e12
     res = {
         "workload": name,
         "algo": "token-sequential with chunk checkpoints",
         "ms_per_step": ms,
         "tokens_per_s": total / t * ws,
-        "roofline": {"bound": "hbm", "achieved": achieved, "peak": peaks["hbm_gbs"], "unit": "GB/s",
-                     "frac": achieved / peaks["hbm_gbs"], "traffic": ncu_traffic(key)},
+        "roofline": {"bound": "alu", "achieved": achieved, "peak": FP32_SIMT_TFLOPS, "unit": "TFLOP/s",
+                     "frac": achieved / FP32_SIMT_TFLOPS, "traffic": ncu_traffic(key),
+                     "peak_source": "148 SMs x 128 fp32 lanes x 2 flops x 1965 MHz"},
+        "hbm_frac": alg_b / t / 1e9 / peaks["hbm_gbs"],
         "pct_of_nominal_roofline": alg_b / (NOMINAL_HBM_GBS * 1e9) / t * 100,
+        "alg_flops": alg_f,
         "alg_bytes": alg_b,
         "workspace_bytes": ws_bytes,
     }

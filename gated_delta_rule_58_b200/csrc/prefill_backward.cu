@@ -26,15 +26,18 @@
 //      walk its tokens backwards reading S_{t-1} from there (a thread reads back only
 //      what it wrote, so no barrier orders the scratch).
 // Per token the sums over columns of dq and dk go through shared memory (each thread
-// writes its 32 partial products, then each of the dk threads adds two entries over
-// the CTA's columns); dg and dbeta are block reductions. All four are accumulated
-// with fp32 atomics into zeroed outputs, so the column blocks of a head and the value
-// heads that share a q/k head add up.
-// Latency: the next token's k, q, v, dO and gates are loaded into registers while
-// the current token computes; in the backward walk S_t is the previous token's
+// writes its partial products, then each thread adds dk / 32 consecutive entries over
+// the CTA's columns); dg and dbeta are warp reductions. All four are accumulated
+// with fp32 atomics (vector atomics for dq and dk) into zeroed outputs, so the column
+// blocks of a head and the value heads that share a q/k head add up.
+// Latency: the tokens' k, q, gates and the CTA's columns of v and dO are copied into
+// a shared-memory ring by cp.async several positions ahead of their use (the order
+// in which the three passes visit the tokens is fixed, so an incremental cursor
+// walks it without divisions); in the backward walk S_t is the previous token's
 // S_{t-1} (kept in registers) and the next S_{t-1} is fetched from the scratch into
 // shared memory by cp.async while the current token computes (each thread copies and
-// reads only its own entries).
+// reads only its own entries). Dot products over a thread's entries use four partial
+// sums, which shortens their dependency chains.
 #include <string>
 
 #include "device_once.h"
@@ -86,60 +89,115 @@ BwdLayout bwd_layout(int N, int64_t total_T, int H, int D, int C) {
   return L;
 }
 
-// value columns per CTA: one warp per CTA (1024 / dk columns of dk / 32 lanes each),
-// so many small CTAs share an SM and a barrier spans one warp
+// entries of a state column held by one thread; a column takes D / kBwdPer lanes
+constexpr int kBwdPer = 32;
 template <int D>
-constexpr int bwd_cols() { return 1024 / D; }
+constexpr int bwd_tpc() { return D / kBwdPer; }
+
+// value columns per CTA: one warp per CTA (32 / (D / kBwdPer) columns), so many small
+// CTAs share an SM and a barrier spans one warp
+template <int D>
+constexpr int bwd_cols() { return 32 / bwd_tpc<D>(); }
 
 // Shared-memory stride of one column in the [columns][D entries] buffers, padded so
-// that the eight lanes of a quarter warp (two columns x four 16-byte pieces) store to
-// distinct banks.
+// that the eight lanes of a quarter warp (8 / tpc columns of tpc 16-byte pieces each)
+// store to distinct banks: consecutive columns start 4 tpc banks apart.
 template <int D>
-constexpr int bwd_col_stride() { return D + 16; }
+constexpr int bwd_col_stride() { return D + 4 * bwd_tpc<D>(); }
 
 template <int D>
-constexpr int bwd_threads() { return bwd_cols<D>() * (D / 32); }
-template <int D>
-constexpr int bwd_warps() { return (bwd_threads<D>() + 31) / 32; }
+constexpr int bwd_threads() { return bwd_cols<D>() * bwd_tpc<D>(); }
 
-template <int D>
+// The kernel visits its tokens in a fixed order of 3 len positions: the forward
+// sweep, then for each chunk from the last its tokens forward (recompute) and
+// backward (walk). Each position's k, q, g, beta and the CTA's columns of v and dO
+// are copied, in the input dtype, into a ring of kRing shared-memory slots by cp.async
+// kRing - 1 positions ahead of their use.
+constexpr int kRing = 8;
+
+template <int D, typename TIn>
+struct BwdSlot {
+  static constexpr int kVec = D * (int)sizeof(TIn);               // bytes of k (and of q)
+  static constexpr int kOwn = bwd_cols<D>() * (int)sizeof(TIn);   // bytes of the CTA's columns of v (of dO)
+  static constexpr int kOwnPad = (kOwn + 15) / 16 * 16;
+  static constexpr int kQ = kVec;
+  static constexpr int kV = 2 * kVec;
+  static constexpr int kDO = kV + kOwnPad;
+  static constexpr int kG = kDO + kOwnPad;  // g, then beta (fp32)
+  static constexpr int kBytes = kG + 16;
+  static_assert(kVec % 16 == 0 && (kOwn == 4 || kOwn == 8 || kOwn % 16 == 0), "cp.async sizes");
+};
+
+template <int D, typename TIn>
 constexpr size_t bwd_smem_bytes() {
-  // token vectors [2][k, q, v, dO][D], gates [2][alpha, beta], column partials of dq
-  // and dk and the prefetched S_{t-1} ([columns][stride] each), scalar partials
-  // [warps][2], per-warp partial squared norms of k and q [2][warps][2] and partial
-  // projections [warps][2]; bwd_cols * D / 32 threads
-  return (8 * D + 4 + 3 * bwd_cols<D>() * bwd_col_stride<D>() + 8 * bwd_warps<D>()) * sizeof(float);
+  // the token ring, then (fp32) the column partials of dq and dk and the prefetched
+  // S_{t-1}, [columns][stride] each
+  return (size_t)kRing * BwdSlot<D, TIn>::kBytes + 3 * (size_t)bwd_cols<D>() * bwd_col_stride<D>() * sizeof(float);
 }
 
-__device__ __forceinline__ void cp_async16(float* dst, const float* src) {
+template <int N>
+__device__ __forceinline__ void cp_async(void* dst, const void* src) {
   const uint32_t d = (uint32_t)__cvta_generic_to_shared(dst);
-  asm volatile("cp.async.cg.shared.global [%0], [%1], 16;" ::"r"(d), "l"(src) : "memory");
+  if constexpr (N == 16)
+    asm volatile("cp.async.cg.shared.global [%0], [%1], 16;" ::"r"(d), "l"(src) : "memory");
+  else
+    asm volatile("cp.async.ca.shared.global [%0], [%1], %2;" ::"r"(d), "l"(src), "n"(N) : "memory");
 }
-__device__ __forceinline__ void cp_async_wait_all() {
-  asm volatile("cp.async.commit_group;\ncp.async.wait_group 0;" ::: "memory");
+__device__ __forceinline__ void cp_async_commit() { asm volatile("cp.async.commit_group;" ::: "memory"); }
+template <int N>
+__device__ __forceinline__ void cp_async_wait() { asm volatile("cp.async.wait_group %0;" ::"n"(N) : "memory"); }
+
+// N = 1, 2 or 4 consecutive fp32 entries (aligned to N) from shared memory, and their
+// addition to global memory by one vector atomic
+template <int N>
+__device__ __forceinline__ void ld_vec(const float* p, float* out) {
+  if constexpr (N == 4) {
+    const float4 f = *reinterpret_cast<const float4*>(p);
+    out[0] = f.x; out[1] = f.y; out[2] = f.z; out[3] = f.w;
+  } else if constexpr (N == 2) {
+    const float2 f = *reinterpret_cast<const float2*>(p);
+    out[0] = f.x; out[1] = f.y;
+  } else {
+    out[0] = *p;
+  }
+}
+template <int N>
+__device__ __forceinline__ void atomic_add_vec(float* p, const float* v) {
+  if constexpr (N == 4) {
+    atomicAdd(reinterpret_cast<float4*>(p), make_float4(v[0], v[1], v[2], v[3]));
+  } else if constexpr (N == 2) {
+    atomicAdd(reinterpret_cast<float2*>(p), make_float2(v[0], v[1]));
+  } else {
+    atomicAdd(p, v[0]);
+  }
+}
+
+// four consecutive entries of a token vector in shared memory, as fp32
+__device__ __forceinline__ float4 ld4_f32(const float* p) { return *reinterpret_cast<const float4*>(p); }
+__device__ __forceinline__ float4 ld4_f32(const __nv_bfloat16* p) {
+  const uint2 r = *reinterpret_cast<const uint2*>(p);
+  const float2 lo = __bfloat1622float2(*reinterpret_cast<const __nv_bfloat162*>(&r.x));
+  const float2 hi = __bfloat1622float2(*reinterpret_cast<const __nv_bfloat162*>(&r.y));
+  return make_float4(lo.x, lo.y, hi.x, hi.y);
 }
 
 template <int D, typename TIn>
 __global__ void __launch_bounds__(bwd_threads<D>())
 gdn_prefill_backward_kernel(const BwdArgs a) {
-  constexpr int TPC = D / 32;  // threads per state column
+  constexpr int TPC = bwd_tpc<D>();  // threads per state column
   constexpr int kBwdCols = bwd_cols<D>();
   constexpr int NT = kBwdCols * TPC;
-  constexpr int EPT = D / NT;  // dk entries of the token vectors per thread
-  static_assert(NT * EPT == D && NT % 32 == 0, "whole warps, whole vectors");
-  constexpr int PER = 32;      // entries of the column per thread
-  constexpr int NP = PER / 4;  // 16-byte pieces per thread
-  constexpr int NW = NT / 32;
+  constexpr int EPT = D / NT;  // consecutive dk entries of dq and dk per thread
+  static_assert(NT * EPT == D && NT == 32 && TPC * kBwdPer == D, "one warp, whole vectors");
+  constexpr int PER = kBwdPer;  // entries of the column per thread
+  constexpr int NP = PER / 4;   // 16-byte pieces per thread
   constexpr int RS = bwd_col_stride<D>();
-  extern __shared__ __align__(16) float bsm[];
-  float* tok = bsm;                       // [2][4][D]
-  float* gates = tok + 8 * D;             // [2][2]
-  float* red_q = gates + 4;               // [kBwdCols][RS]
+  using SL = BwdSlot<D, TIn>;
+  extern __shared__ __align__(16) uint8_t bsm[];
+  uint8_t* ring = bsm;                                                    // [kRing][slot]
+  float* red_q = reinterpret_cast<float*>(bsm + kRing * SL::kBytes);      // [kBwdCols][RS]
   float* red_k = red_q + kBwdCols * RS;
   float* sp_buf = red_k + kBwdCols * RS;  // [kBwdCols][RS]: the next S_{t-1}, each thread its own entries
-  float* red_s = sp_buf + kBwdCols * RS;  // [NW][2]
-  float* nrm = red_s + 2 * NW;            // [2][NW][2]: partial |k|^2, |q|^2 of a buffer's token
-  float* jred = nrm + 4 * NW;             // [NW][2]: partial k^ . dk^, q^ . dq^
   const bool l2 = a.l2norm != 0;
 
   const int tid = threadIdx.x;
@@ -155,116 +213,130 @@ gdn_prefill_backward_kernel(const BwdArgs a) {
   const int hq = h / (a.H / a.Hqk);
   int64_t bos, eos;
   if (!seq_bounds(a.cu, n, a.total_T, a.err, &bos, &eos)) return;
-  const int nck = (int)((eos - bos + a.C - 1) / a.C);
+  const int64_t len = eos - bos;
+  const int nck = (int)((len + a.C - 1) / a.C);
   const size_t SS = (size_t)D * D;
   const size_t state_off = ((size_t)n * a.H + h) * SS + (size_t)col * D;
   float* ck = a.ckpt + ((size_t)h * a.ck_slots + (size_t)(bos / a.C) + n) * SS + (size_t)col * D;
   float* scr = a.scratch + (size_t)item * (size_t)(a.C + 1) * SS + (size_t)col * D;
   float* spb = sp_buf + lcol * RS;
-  const TIn* qp = static_cast<const TIn*>(a.q);
-  const TIn* kp = static_cast<const TIn*>(a.k);
-  const TIn* vp = static_cast<const TIn*>(a.v);
-  const TIn* dop = static_cast<const TIn*>(a.d_o);
 
-  // A token's k, q, v, dO and gates are
-  // fetched into registers, then committed to shared-memory buffer `buf` (two
-  // buffers: the barrier of the token in between orders every read of a buffer
-  // before its refill).
-  // (thread tid holds entries tid + NT e, e < EPT)
-  float fk[EPT], fq[EPT], fv[EPT], fdo[EPT], fg = 0.f, fb = 0.f;
-  auto fetch = [&](int64_t t) {
-    const size_t th = (size_t)t * a.H + h, tq = (size_t)t * a.Hqk + hq;
-#pragma unroll
-    for (int e = 0; e < EPT; ++e) {
-      const int i = tid + NT * e;
-      fk[e] = to_f32(kp[tq * D + i]);
-      fq[e] = to_f32(qp[tq * D + i]);
-      fv[e] = to_f32(vp[th * D + i]);
-      fdo[e] = to_f32(dop[th * D + i]);
+  // The issue cursor: the token of the next position to copy, walked through the
+  // visiting order one position at a time (phase 0 forward sweep, 1 recompute of
+  // chunk [ct0, ct1), 2 its walk, 3 past the end), and the ring slot it goes to.
+  int64_t ct = bos, ct0 = 0, ct1 = 0;
+  int cc = 0, cphase = len > 0 ? 0 : 3, islot = 0;
+  auto cursor_next = [&]() {
+    if (cphase == 0) {
+      if (++ct == eos) {
+        cc = nck - 1;
+        ct0 = bos + (int64_t)cc * a.C;
+        ct1 = eos;
+        ct = ct0;
+        cphase = 1;
+      }
+    } else if (cphase == 1) {
+      if (++ct == ct1) {
+        ct = ct1 - 1;
+        cphase = 2;
+      }
+    } else if (cphase == 2) {
+      if (ct == ct0) {
+        if (--cc < 0) {
+          cphase = 3;
+        } else {
+          ct1 = ct0;
+          ct0 -= a.C;
+          ct = ct0;
+          cphase = 1;
+        }
+      } else {
+        --ct;
+      }
     }
-    if (tid == 0) {
-      fg = a.g[th];
-      fb = a.beta[th];
+    islot = islot + 1 == kRing ? 0 : islot + 1;
+  };
+  // copies of the cursor's position into its slot, as one cp.async group (empty past
+  // the end); the cursor moves on
+  auto issue = [&]() {
+    if (cphase != 3) {
+      const int64_t t = ct;
+      uint8_t* sl = ring + islot * SL::kBytes;
+      const size_t th = (size_t)t * a.H + h, tq = (size_t)t * a.Hqk + hq;
+      const char* kr = static_cast<const char*>(a.k) + tq * SL::kVec;
+      const char* qr = static_cast<const char*>(a.q) + tq * SL::kVec;
+      constexpr int n16 = SL::kVec / 16;
+      for (int c = tid; c < 2 * n16; c += NT) cp_async<16>(sl + 16 * c, c < n16 ? kr + 16 * c : qr + 16 * (c - n16));
+      const size_t own = (th * D + (size_t)cb * kBwdCols) * sizeof(TIn);
+      const char* vr = static_cast<const char*>(a.v) + own;
+      const char* dr = static_cast<const char*>(a.d_o) + own;
+      if constexpr (SL::kOwn >= 16) {
+        constexpr int m16 = SL::kOwn / 16;
+        for (int c = tid; c < 2 * m16; c += NT) {
+          const int r = c < m16 ? c : c - m16;
+          cp_async<16>(sl + (c < m16 ? SL::kV : SL::kDO) + 16 * r, (c < m16 ? vr : dr) + 16 * r);
+        }
+      } else {
+        if (tid < 2) cp_async<SL::kOwn>(sl + (tid == 0 ? SL::kV : SL::kDO), tid == 0 ? vr : dr);
+      }
+      if (tid == NT - 1) cp_async<4>(sl + SL::kG, a.g + th);
+      if (tid == NT - 2) cp_async<4>(sl + SL::kG + 4, a.beta + th);
+    }
+    cp_async_commit();
+    cursor_next();
+  };
+  int rslot = 0;  // the slot of the position being computed
+  auto take_slot = [&]() -> const uint8_t* {
+    const uint8_t* sl = ring + rslot * SL::kBytes;
+    rslot = rslot + 1 == kRing ? 0 : rslot + 1;
+    return sl;
+  };
+  // this thread's entries of the slot's k (or q) vector
+  auto load_tok = [&](const uint8_t* v, float* out) {
+    const TIn* e = reinterpret_cast<const TIn*>(v);
+#pragma unroll
+    for (int y = 0; y < NP; ++y) {
+      const float4 f = ld4_f32(e + piece(y));
+      out[4 * y] = f.x; out[4 * y + 1] = f.y; out[4 * y + 2] = f.z; out[4 * y + 3] = f.w;
     }
   };
-  auto commit = [&](int buf) {
-    float* tb = tok + buf * 4 * D;
+  // 1 / |x| from this thread's entries, summed over the column's lanes (1 without the
+  // normalisation; zero stays zero)
+  auto inv_norm = [&](const float* x) {
+    if (!l2) return 1.f;
+    float s4[4] = {0.f, 0.f, 0.f, 0.f};  // four partial sums (shorter dependency chains)
 #pragma unroll
-    for (int e = 0; e < EPT; ++e) {
-      const int i = tid + NT * e;
-      tb[i] = fk[e];
-      tb[D + i] = fq[e];
-      tb[2 * D + i] = fv[e];
-      tb[3 * D + i] = fdo[e];
-    }
-    if (tid == 0) {
-      gates[2 * buf] = expf(fg);
-      gates[2 * buf + 1] = fb;
-    }
-    if (l2) {  // per-warp partial squared norms
-      float kk = 0.f, qq = 0.f;
+    for (int i = 0; i < PER; ++i) s4[i & 3] = fmaf(x[i], x[i], s4[i & 3]);
+    float ss = (s4[0] + s4[1]) + (s4[2] + s4[3]);
 #pragma unroll
-      for (int e = 0; e < EPT; ++e) {
-        kk = fmaf(fk[e], fk[e], kk);
-        qq = fmaf(fq[e], fq[e], qq);
-      }
-#pragma unroll
-      for (int off = 16; off > 0; off >>= 1) {
-        kk += __shfl_xor_sync(0xffffffffu, kk, off);
-        qq += __shfl_xor_sync(0xffffffffu, qq, off);
-      }
-      if ((tid & 31) == 0) {
-        nrm[(buf * NW + (tid >> 5)) * 2] = kk;
-        nrm[(buf * NW + (tid >> 5)) * 2 + 1] = qq;
-      }
-    }
+    for (int off = 1; off < TPC; off <<= 1) ss += __shfl_xor_sync(0xffffffffu, ss, off);
+    return ss > 0.f ? 1.f / sqrtf(ss) : 0.f;
   };
-  // 1 / |k| and 1 / |q| of the token in buffer `buf` (1 without the normalisation)
-  auto inv_norms = [&](int buf, float* rk, float* rq) {
-    *rk = 1.f;
-    *rq = 1.f;
-    if (l2) {
-      float kk = 0.f, qq = 0.f;
-      for (int wi = 0; wi < NW; ++wi) {
-        kk += nrm[(buf * NW + wi) * 2];
-        qq += nrm[(buf * NW + wi) * 2 + 1];
-      }
-      *rk = kk > 0.f ? 1.f / sqrtf(kk) : 0.f;
-      *rq = qq > 0.f ? 1.f / sqrtf(qq) : 0.f;
-    }
+  // one token forward on this thread's entries of column col (as the forward kernel;
+  // the update adds c k with c = beta (v_j - alpha (k^ . S_j)) / |k|)
+  auto advance = [&](float* st, const uint8_t* sl) {
+    const float alpha = expf(*reinterpret_cast<const float*>(sl + SL::kG));
+    const float beta = *reinterpret_cast<const float*>(sl + SL::kG + 4);
+    const float vj = to_f32(reinterpret_cast<const TIn*>(sl + SL::kV)[lcol]);
+    float kv[PER];
+    load_tok(sl, kv);
+    const float rk = inv_norm(kv);
+    float u4[4] = {0.f, 0.f, 0.f, 0.f};
+#pragma unroll
+    for (int x = 0; x < PER; ++x) u4[x & 3] = fmaf(kv[x], st[x], u4[x & 3]);
+    float u = (u4[0] + u4[1]) + (u4[2] + u4[3]);
+#pragma unroll
+    for (int off = 1; off < TPC; off <<= 1) u += __shfl_xor_sync(0xffffffffu, u, off);
+    const float c = beta * (vj - alpha * (u * rk)) * rk;
+#pragma unroll
+    for (int x = 0; x < PER; ++x) st[x] = fmaf(alpha, st[x], c * kv[x]);
   };
-  // this thread's entries of a D-vector in shared memory
+  // a state column's entries of this thread from / to memory (p = the column's base)
   auto load_vec = [&](const float* v, float* out) {
 #pragma unroll
     for (int y = 0; y < NP; ++y) {
       const float4 f = *reinterpret_cast<const float4*>(v + piece(y));
       out[4 * y] = f.x; out[4 * y + 1] = f.y; out[4 * y + 2] = f.z; out[4 * y + 3] = f.w;
-    }
-  };
-  // one token forward on this thread's entries of column col (as the forward kernel;
-  // the update adds c k with c = beta (v_j - alpha (k^ . S_j)) / |k|)
-  auto advance = [&](float* st, int buf) {
-    const float* tb = tok + buf * 4 * D;
-    const float alpha = gates[2 * buf], beta = gates[2 * buf + 1];
-    float rk, rq;
-    inv_norms(buf, &rk, &rq);
-    float kv[PER];
-    load_vec(tb, kv);
-    float u = 0.f;
-#pragma unroll
-    for (int x = 0; x < PER; ++x) u = fmaf(kv[x], st[x], u);
-#pragma unroll
-    for (int off = 1; off < TPC; off <<= 1) u += __shfl_xor_sync(0xffffffffu, u, off);
-    const float c = beta * (tb[2 * D + col] - alpha * (u * rk)) * rk;
-#pragma unroll
-    for (int x = 0; x < PER; ++x) st[x] = fmaf(alpha, st[x], c * kv[x]);
-  };
-  // a state column's entries of this thread from / to memory (p = the column's base)
-  auto load_state = [&](const float* p, float* st) {
-#pragma unroll
-    for (int y = 0; y < NP; ++y) {
-      const float4 f = *reinterpret_cast<const float4*>(p + piece(y));
-      st[4 * y] = f.x; st[4 * y + 1] = f.y; st[4 * y + 2] = f.z; st[4 * y + 3] = f.w;
     }
   };
   auto store_state = [&](float* p, const float* st) {
@@ -274,34 +346,47 @@ gdn_prefill_backward_kernel(const BwdArgs a) {
   };
   auto prefetch_state = [&](const float* p) {  // this thread's entries -> sp_buf, asynchronously
 #pragma unroll
-    for (int y = 0; y < NP; ++y) cp_async16(spb + piece(y), p + piece(y));
+    for (int y = 0; y < NP; ++y) cp_async<16>(spb + piece(y), p + piece(y));
   };
+  // Every step p commits two groups: [the S_{t-1} of the next step when that is a walk
+  // step, else none], then [position p + kRing - 1]. At step p, position p's group is
+  // followed by 2 (kRing - 2) newer ones, a walk step's S_{t-1} by one. The slot
+  // refilled at step p is step p - 1's, which every thread has left at the barrier.
+  constexpr int kWaitSweep = 2 * (kRing - 2);
+  for (int i = 0; i < kRing - 1; ++i) {
+    cp_async_commit();
+    issue();
+  }
 
   // 1. forward with a checkpoint at the start of every chunk
-  int it = 0;  // staged tokens so far (buffer parity)
   {
     float st[PER];
     if (a.init) {
-      load_state(a.init + state_off, st);
+      load_vec(a.init + state_off, st);
     } else {
 #pragma unroll
       for (int x = 0; x < PER; ++x) st[x] = 0.f;
     }
-    if (bos < eos) fetch(bos);
+    float* ckp = ck;  // the next checkpoint
+    int in_chunk = 0;
     for (int64_t t = bos; t < eos; ++t) {
-      const int buf = (it++) & 1;
-      commit(buf);
-      if (t + 1 < eos) fetch(t + 1);
+      cp_async_wait<kWaitSweep>();
       __syncthreads();
-      if ((t - bos) % a.C == 0) store_state(ck + (size_t)((t - bos) / a.C) * SS, st);
-      advance(st, buf);
+      if (in_chunk == 0) {
+        store_state(ckp, st);
+        ckp += SS;
+      }
+      in_chunk = in_chunk + 1 == a.C ? 0 : in_chunk + 1;
+      cp_async_commit();
+      issue();
+      advance(st, take_slot());
     }
   }
 
   // 2. chunks last to first
   float Dm[PER];  // dL/dS_t, this thread's entries
   if (a.d_fin) {
-    load_state(a.d_fin + state_off, Dm);
+    load_vec(a.d_fin + state_off, Dm);
   } else {
 #pragma unroll
     for (int x = 0; x < PER; ++x) Dm[x] = 0.f;
@@ -310,32 +395,26 @@ gdn_prefill_backward_kernel(const BwdArgs a) {
     const int64_t t0 = bos + (int64_t)c * a.C;
     const int64_t t1 = (t0 + a.C < eos) ? t0 + a.C : eos;
     float sc[PER];  // S_t of the token being walked
-    {
-      // scratch slot x = the state before token t0 + x
-      load_state(ck + (size_t)c * SS, sc);
-      fetch(t0);
-      for (int64_t t = t0; t < t1; ++t) {
-        const int buf = (it++) & 1;
-        commit(buf);
-        if (t + 1 < t1) fetch(t + 1);
-        __syncthreads();
-        store_state(scr + (size_t)(t - t0) * SS, sc);
-        advance(sc, buf);
-      }
-    }
-    // sc = the state after the chunk's last token; its S_{t-1} goes into sp_buf
-    prefetch_state(scr + (size_t)(t1 - 1 - t0) * SS);
-    fetch(t1 - 1);
-    for (int64_t t = t1 - 1; t >= t0; --t) {
-      const int buf = (it++) & 1;
-      commit(buf);
-      if (t - 1 >= t0) fetch(t - 1);
+    // recompute: scratch slot x = the state before token t0 + x
+    load_vec(ck + (size_t)c * SS, sc);
+    for (int64_t t = t0; t < t1; ++t) {
+      cp_async_wait<kWaitSweep>();
       __syncthreads();
-      const float* tb = tok + buf * 4 * D;
-      const float vj = tb[2 * D + col], dOj = tb[3 * D + col];
-      const float alpha = gates[2 * buf], beta = gates[2 * buf + 1];
-      float rk, rq;
-      inv_norms(buf, &rk, &rq);
+      store_state(scr + (size_t)(t - t0) * SS, sc);
+      if (t + 1 == t1) prefetch_state(scr + (size_t)(t - t0) * SS);  // the first walk step's S_{t-1}
+      cp_async_commit();
+      issue();
+      advance(sc, take_slot());
+    }
+    // walk: sc = S_t, its S_{t-1} waits in sp_buf
+    for (int64_t t = t1 - 1; t >= t0; --t) {
+      cp_async_wait<1>();
+      __syncthreads();
+      const uint8_t* sl = take_slot();
+      const float vj = to_f32(reinterpret_cast<const TIn*>(sl + SL::kV)[lcol]);
+      const float dOj = to_f32(reinterpret_cast<const TIn*>(sl + SL::kDO)[lcol]);
+      const float alpha = expf(*reinterpret_cast<const float*>(sl + SL::kG));
+      const float beta = *reinterpret_cast<const float*>(sl + SL::kG + 4);
       const size_t th = (size_t)t * a.H + h, tq = (size_t)t * a.Hqk + hq;
       // column j's terms of dq (S_t dO) first: S_t is not needed after them
       float* rowq = red_q + lcol * RS;
@@ -345,25 +424,30 @@ gdn_prefill_backward_kernel(const BwdArgs a) {
         *reinterpret_cast<float4*>(rowq + piece(y)) = make_float4(sc[4 * y] * dOj, sc[4 * y + 1] * dOj,
                                                                 sc[4 * y + 2] * dOj, sc[4 * y + 3] * dOj);
       float sp[PER];  // S_{t-1}
-      cp_async_wait_all();
       load_vec(spb, sp);
       if (t - 1 >= t0) prefetch_state(scr + (size_t)(t - 1 - t0) * SS);
+      cp_async_commit();
+      issue();
+      float kv[PER];
+      load_tok(sl, kv);
+      const float rk = inv_norm(kv);
       // D += scale q dO^T
+      float rq;
       {
         float qv[PER];
-        load_vec(tb + D, qv);
+        load_tok(sl + SL::kQ, qv);
+        rq = inv_norm(qv);
 #pragma unroll
         for (int x = 0; x < PER; ++x) Dm[x] = fmaf(a.scale * rq * qv[x], dOj, Dm[x]);
       }
-      float kv[PER];
-      load_vec(tb, kv);
       // u = S~^T k (S~ = alpha S_{t-1}), w = D^T k, column j
-      float pu = 0.f, pw = 0.f;
+      float pu4[4] = {0.f, 0.f, 0.f, 0.f}, pw4[4] = {0.f, 0.f, 0.f, 0.f};
 #pragma unroll
       for (int x = 0; x < PER; ++x) {
-        pu = fmaf(kv[x], sp[x], pu);
-        pw = fmaf(kv[x], Dm[x], pw);
+        pu4[x & 3] = fmaf(kv[x], sp[x], pu4[x & 3]);
+        pw4[x & 3] = fmaf(kv[x], Dm[x], pw4[x & 3]);
       }
+      float pu = (pu4[0] + pu4[1]) + (pu4[2] + pu4[3]), pw = (pw4[0] + pw4[1]) + (pw4[2] + pw4[3]);
 #pragma unroll
       for (int off = 1; off < TPC; off <<= 1) {
         pu += __shfl_xor_sync(0xffffffffu, pu, off);
@@ -371,7 +455,7 @@ gdn_prefill_backward_kernel(const BwdArgs a) {
       }
       const float u = alpha * pu * rk, w = pw * rk, vmu = vj - u;
       // column j's terms of dk (D (v - u) - S~ w) and of dg
-      float sdg = 0.f;
+      float g4[4] = {0.f, 0.f, 0.f, 0.f};
 #pragma unroll
       for (int y = 0; y < NP; ++y) {
         float kk[4];
@@ -380,10 +464,11 @@ gdn_prefill_backward_kernel(const BwdArgs a) {
           const int x = 4 * y + z;
           const float stl = alpha * sp[x];
           kk[z] = Dm[x] * vmu - stl * w;
-          sdg = fmaf(Dm[x], stl, sdg);
+          g4[z] = fmaf(Dm[x], stl, g4[z]);
         }
         *reinterpret_cast<float4*>(rowk + piece(y)) = make_float4(kk[0], kk[1], kk[2], kk[3]);
       }
+      float sdg = (g4[0] + g4[1]) + (g4[2] + g4[3]);
       float sdb = 0.f;
       if (part == 0) {
         sdg -= beta * u * w;
@@ -397,74 +482,60 @@ gdn_prefill_backward_kernel(const BwdArgs a) {
         Dm[x] = alpha * (Dm[x] - bw * kv[x]);
         sc[x] = sp[x];
       }
+      // dg and dbeta over the CTA's columns (every lane ends with the sums)
 #pragma unroll
       for (int off = 16; off > 0; off >>= 1) {
         sdg += __shfl_xor_sync(0xffffffffu, sdg, off);
         sdb += __shfl_xor_sync(0xffffffffu, sdb, off);
       }
-      if ((tid & 31) == 0) {
-        red_s[2 * (tid >> 5)] = sdg;
-        red_s[2 * (tid >> 5) + 1] = sdb;
-      }
-      __syncthreads();
-      {  // entries tid + NT e of dq and of dk over this CTA's columns
+      __syncthreads();  // the column partials of dq and dk are written
+      {  // entries i0 .. i0 + EPT - 1 of dq and of dk over this CTA's columns
+        const int i0 = EPT * tid;
         float gq[EPT], gk[EPT];  // this CTA's part of dq^, dk^
 #pragma unroll
-        for (int e = 0; e < EPT; ++e) {
-          const int i = tid + NT * e;
-          float sq = 0.f, sk = 0.f;
+        for (int e = 0; e < EPT; ++e) gq[e] = gk[e] = 0.f;
 #pragma unroll 8
-          for (int j = 0; j < kBwdCols; ++j) {
-            sq += red_q[j * RS + i];
-            sk += red_k[j * RS + i];
+        for (int j = 0; j < kBwdCols; ++j) {
+          float xq[EPT], xk[EPT];
+          ld_vec<EPT>(red_q + j * RS + i0, xq);
+          ld_vec<EPT>(red_k + j * RS + i0, xk);
+#pragma unroll
+          for (int e = 0; e < EPT; ++e) {
+            gq[e] += xq[e];
+            gk[e] += xk[e];
           }
-          gq[e] = a.scale * sq;
-          gk[e] = beta * sk;
+        }
+#pragma unroll
+        for (int e = 0; e < EPT; ++e) {
+          gq[e] *= a.scale;
+          gk[e] *= beta;
         }
         if (l2) {  // through the normalisation: (g - x^ (x^ . g)) / |x|
+          const TIn* ke = reinterpret_cast<const TIn*>(sl);
+          const TIn* qe = reinterpret_cast<const TIn*>(sl + SL::kQ);
           float pk = 0.f, pq = 0.f;
 #pragma unroll
           for (int e = 0; e < EPT; ++e) {
-            const int i = tid + NT * e;
-            pk = fmaf(tb[i] * rk, gk[e], pk);
-            pq = fmaf(tb[D + i] * rq, gq[e], pq);
+            pk = fmaf(to_f32(ke[i0 + e]) * rk, gk[e], pk);
+            pq = fmaf(to_f32(qe[i0 + e]) * rq, gq[e], pq);
           }
 #pragma unroll
           for (int off = 16; off > 0; off >>= 1) {
             pk += __shfl_xor_sync(0xffffffffu, pk, off);
             pq += __shfl_xor_sync(0xffffffffu, pq, off);
           }
-          if ((tid & 31) == 0) {
-            jred[2 * (tid >> 5)] = pk;
-            jred[2 * (tid >> 5) + 1] = pq;
-          }
-          __syncthreads();
-          float dotk = 0.f, dotq = 0.f;
-          for (int wi = 0; wi < NW; ++wi) {
-            dotk += jred[2 * wi];
-            dotq += jred[2 * wi + 1];
-          }
 #pragma unroll
           for (int e = 0; e < EPT; ++e) {
-            const int i = tid + NT * e;
-            gk[e] = (gk[e] - tb[i] * rk * dotk) * rk;
-            gq[e] = (gq[e] - tb[D + i] * rq * dotq) * rq;
+            gk[e] = (gk[e] - to_f32(ke[i0 + e]) * rk * pk) * rk;
+            gq[e] = (gq[e] - to_f32(qe[i0 + e]) * rq * pq) * rq;
           }
         }
-#pragma unroll
-        for (int e = 0; e < EPT; ++e) {
-          atomicAdd(a.dq + tq * D + tid + NT * e, gq[e]);
-          atomicAdd(a.dk + tq * D + tid + NT * e, gk[e]);
-        }
+        atomic_add_vec<EPT>(a.dq + tq * D + i0, gq);
+        atomic_add_vec<EPT>(a.dk + tq * D + i0, gk);
       }
       if (tid == 0) {
-        float g_sum = 0.f, b_sum = 0.f;
-        for (int wi = 0; wi < NW; ++wi) {
-          g_sum += red_s[2 * wi];
-          b_sum += red_s[2 * wi + 1];
-        }
-        atomicAdd(a.dg + th, g_sum);
-        atomicAdd(a.dbeta + th, b_sum);
+        atomicAdd(a.dg + th, sdg);
+        atomicAdd(a.dbeta + th, sdb);
       }
     }
   }
@@ -474,7 +545,7 @@ gdn_prefill_backward_kernel(const BwdArgs a) {
 template <int D, typename TIn>
 gdn_status_t launch_bwd(const BwdArgs& a, cudaStream_t stream) {
   auto kernel = gdn_prefill_backward_kernel<D, TIn>;
-  constexpr size_t smem = bwd_smem_bytes<D>();
+  constexpr size_t smem = bwd_smem_bytes<D, TIn>();
   static PerDeviceOnce once;  // the shared-memory opt-in applies to the current device only
   int dev = 0;
   cudaError_t e = cudaGetDevice(&dev);
@@ -502,7 +573,7 @@ gdn_status_t bwd_check_shape(int N, int64_t total_T, int H, int dk, int dv, int 
   if (dk != dv || (dk != 32 && dk != 64 && dk != 128))
     return fail(GDN_ERR_UNSUPPORTED, "gdn_chunk_prefill_backward: dk == dv in {32, 64, 128}");
   if (chunk > 4096) return fail(GDN_ERR_UNSUPPORTED, "gdn_chunk_prefill_backward: chunk <= 4096");
-  if ((long long)N * H * (dk * dk / 1024) >= (1LL << 31))  // column blocks: dk / (1024 / dk) per head
+  if ((long long)N * H * (dk * dk / (32 * gdn::kBwdPer)) >= (1LL << 31))  // column blocks per head: dk / cols
     return fail(GDN_ERR_UNSUPPORTED, "gdn_chunk_prefill_backward: N * H too large");
   return gdn::ok();
 }
