@@ -172,6 +172,13 @@ __device__ __forceinline__ void atomic_add_vec(float* p, const float* v) {
   }
 }
 
+// entries x, x + 1 of a register array as one packed pair, and back
+__device__ __forceinline__ float2 pr(const float* a, int x) { return make_float2(a[x], a[x + 1]); }
+__device__ __forceinline__ void put(float* a, int x, float2 v) {
+  a[x] = v.x;
+  a[x + 1] = v.y;
+}
+
 // four consecutive entries of a token vector in shared memory, as fp32
 __device__ __forceinline__ float4 ld4_f32(const float* p) { return *reinterpret_cast<const float4*>(p); }
 __device__ __forceinline__ float4 ld4_f32(const __nv_bfloat16* p) {
@@ -304,10 +311,15 @@ gdn_prefill_backward_kernel(const BwdArgs a) {
   // normalisation; zero stays zero)
   auto inv_norm = [&](const float* x) {
     if (!l2) return 1.f;
-    float s4[4] = {0.f, 0.f, 0.f, 0.f};  // four partial sums (shorter dependency chains)
+    // four partial sums (entries 0, 1, 2, 3 mod 4: shorter dependency chains), as two
+    // packed pairs
+    float2 sa = make_float2(0.f, 0.f), sb = sa;
 #pragma unroll
-    for (int i = 0; i < PER; ++i) s4[i & 3] = fmaf(x[i], x[i], s4[i & 3]);
-    float ss = (s4[0] + s4[1]) + (s4[2] + s4[3]);
+    for (int i = 0; i < PER; i += 4) {
+      sa = __ffma2_rn(pr(x, i), pr(x, i), sa);
+      sb = __ffma2_rn(pr(x, i + 2), pr(x, i + 2), sb);
+    }
+    float ss = (sa.x + sa.y) + (sb.x + sb.y);
 #pragma unroll
     for (int off = 1; off < TPC; off <<= 1) ss += __shfl_xor_sync(0xffffffffu, ss, off);
     return ss > 0.f ? 1.f / sqrtf(ss) : 0.f;
@@ -321,15 +333,19 @@ gdn_prefill_backward_kernel(const BwdArgs a) {
     float kv[PER];
     load_tok(sl, kv);
     const float rk = inv_norm(kv);
-    float u4[4] = {0.f, 0.f, 0.f, 0.f};
+    float2 ua = make_float2(0.f, 0.f), ub = ua;
 #pragma unroll
-    for (int x = 0; x < PER; ++x) u4[x & 3] = fmaf(kv[x], st[x], u4[x & 3]);
-    float u = (u4[0] + u4[1]) + (u4[2] + u4[3]);
+    for (int x = 0; x < PER; x += 4) {
+      ua = __ffma2_rn(pr(kv, x), pr(st, x), ua);
+      ub = __ffma2_rn(pr(kv, x + 2), pr(st, x + 2), ub);
+    }
+    float u = (ua.x + ua.y) + (ub.x + ub.y);
 #pragma unroll
     for (int off = 1; off < TPC; off <<= 1) u += __shfl_xor_sync(0xffffffffu, u, off);
     const float c = beta * (vj - alpha * (u * rk)) * rk;
+    const float2 a2 = make_float2(alpha, alpha), c2 = make_float2(c, c);
 #pragma unroll
-    for (int x = 0; x < PER; ++x) st[x] = fmaf(alpha, st[x], c * kv[x]);
+    for (int x = 0; x < PER; x += 2) put(st, x, __ffma2_rn(a2, pr(st, x), __fmul2_rn(c2, pr(kv, x))));
   };
   // a state column's entries of this thread from / to memory (p = the column's base)
   auto load_vec = [&](const float* v, float* out) {
@@ -419,10 +435,12 @@ gdn_prefill_backward_kernel(const BwdArgs a) {
       // column j's terms of dq (S_t dO) first: S_t is not needed after them
       float* rowq = red_q + lcol * RS;
       float* rowk = red_k + lcol * RS;
+      const float2 do2 = make_float2(dOj, dOj);
 #pragma unroll
-      for (int y = 0; y < NP; ++y)
-        *reinterpret_cast<float4*>(rowq + piece(y)) = make_float4(sc[4 * y] * dOj, sc[4 * y + 1] * dOj,
-                                                                sc[4 * y + 2] * dOj, sc[4 * y + 3] * dOj);
+      for (int y = 0; y < NP; ++y) {
+        const float2 lo = __fmul2_rn(pr(sc, 4 * y), do2), hi = __fmul2_rn(pr(sc, 4 * y + 2), do2);
+        *reinterpret_cast<float4*>(rowq + piece(y)) = make_float4(lo.x, lo.y, hi.x, hi.y);
+      }
       float sp[PER];  // S_{t-1}
       load_vec(spb, sp);
       if (t - 1 >= t0) prefetch_state(scr + (size_t)(t - 1 - t0) * SS);
@@ -437,17 +455,21 @@ gdn_prefill_backward_kernel(const BwdArgs a) {
         float qv[PER];
         load_tok(sl + SL::kQ, qv);
         rq = inv_norm(qv);
+        const float sr = a.scale * rq;
+        const float2 sr2 = make_float2(sr, sr);
 #pragma unroll
-        for (int x = 0; x < PER; ++x) Dm[x] = fmaf(a.scale * rq * qv[x], dOj, Dm[x]);
+        for (int x = 0; x < PER; x += 2) put(Dm, x, __ffma2_rn(__fmul2_rn(sr2, pr(qv, x)), do2, pr(Dm, x)));
       }
       // u = S~^T k (S~ = alpha S_{t-1}), w = D^T k, column j
-      float pu4[4] = {0.f, 0.f, 0.f, 0.f}, pw4[4] = {0.f, 0.f, 0.f, 0.f};
+      float2 pua = make_float2(0.f, 0.f), pub = pua, pwa = pua, pwb = pua;
 #pragma unroll
-      for (int x = 0; x < PER; ++x) {
-        pu4[x & 3] = fmaf(kv[x], sp[x], pu4[x & 3]);
-        pw4[x & 3] = fmaf(kv[x], Dm[x], pw4[x & 3]);
+      for (int x = 0; x < PER; x += 4) {
+        pua = __ffma2_rn(pr(kv, x), pr(sp, x), pua);
+        pub = __ffma2_rn(pr(kv, x + 2), pr(sp, x + 2), pub);
+        pwa = __ffma2_rn(pr(kv, x), pr(Dm, x), pwa);
+        pwb = __ffma2_rn(pr(kv, x + 2), pr(Dm, x + 2), pwb);
       }
-      float pu = (pu4[0] + pu4[1]) + (pu4[2] + pu4[3]), pw = (pw4[0] + pw4[1]) + (pw4[2] + pw4[3]);
+      float pu = (pua.x + pua.y) + (pub.x + pub.y), pw = (pwa.x + pwa.y) + (pwb.x + pwb.y);
 #pragma unroll
       for (int off = 1; off < TPC; off <<= 1) {
         pu += __shfl_xor_sync(0xffffffffu, pu, off);
@@ -455,20 +477,19 @@ gdn_prefill_backward_kernel(const BwdArgs a) {
       }
       const float u = alpha * pu * rk, w = pw * rk, vmu = vj - u;
       // column j's terms of dk (D (v - u) - S~ w) and of dg
-      float g4[4] = {0.f, 0.f, 0.f, 0.f};
+      const float2 al2 = make_float2(alpha, alpha), vmu2 = make_float2(vmu, vmu), nw2 = make_float2(-w, -w);
+      float2 ga = make_float2(0.f, 0.f), gb = ga;
 #pragma unroll
       for (int y = 0; y < NP; ++y) {
-        float kk[4];
-#pragma unroll
-        for (int z = 0; z < 4; ++z) {
-          const int x = 4 * y + z;
-          const float stl = alpha * sp[x];
-          kk[z] = Dm[x] * vmu - stl * w;
-          g4[z] = fmaf(Dm[x], stl, g4[z]);
-        }
-        *reinterpret_cast<float4*>(rowk + piece(y)) = make_float4(kk[0], kk[1], kk[2], kk[3]);
+        const int x = 4 * y;
+        const float2 s0 = __fmul2_rn(al2, pr(sp, x)), s1 = __fmul2_rn(al2, pr(sp, x + 2));  // S~ entries
+        const float2 k0 = __ffma2_rn(pr(Dm, x), vmu2, __fmul2_rn(s0, nw2));
+        const float2 k1 = __ffma2_rn(pr(Dm, x + 2), vmu2, __fmul2_rn(s1, nw2));
+        ga = __ffma2_rn(pr(Dm, x), s0, ga);
+        gb = __ffma2_rn(pr(Dm, x + 2), s1, gb);
+        *reinterpret_cast<float4*>(rowk + piece(y)) = make_float4(k0.x, k0.y, k1.x, k1.y);
       }
-      float sdg = (g4[0] + g4[1]) + (g4[2] + g4[3]);
+      float sdg = (ga.x + ga.y) + (gb.x + gb.y);
       float sdb = 0.f;
       if (part == 0) {
         sdg -= beta * u * w;
@@ -477,11 +498,11 @@ gdn_prefill_backward_kernel(const BwdArgs a) {
       }
       // dL/dS_{t-1}; S_{t-1} becomes the next token's S_t
       const float bw = beta * w * rk;
+      const float2 nbw2 = make_float2(-bw, -bw);
 #pragma unroll
-      for (int x = 0; x < PER; ++x) {
-        Dm[x] = alpha * (Dm[x] - bw * kv[x]);
-        sc[x] = sp[x];
-      }
+      for (int x = 0; x < PER; x += 2) put(Dm, x, __fmul2_rn(al2, __ffma2_rn(nbw2, pr(kv, x), pr(Dm, x))));
+#pragma unroll
+      for (int x = 0; x < PER; ++x) sc[x] = sp[x];
       // dg and dbeta over the CTA's columns (every lane ends with the sums)
 #pragma unroll
       for (int off = 16; off > 0; off >>= 1) {
