@@ -26,11 +26,10 @@ def _library_ops():
     from . import _lib
 
     def local_state(q, k, v, g, beta, cu, chunk, l2norm):
-        N, H = cu.numel() - 1, v.shape[1]
+        N, H, total_T = cu.numel() - 1, v.shape[1], q.shape[0]
         dk, dv = q.shape[-1], v.shape[-1]
         loc = torch.empty((N, H, dv, dk), dtype=torch.float32, device=q.device)
         tr = torch.empty_like(loc)
-        N, total_T = cu.numel() - 1, q.shape[0]
         ws = torch.empty(max(_lib.gdn_cp_local_state_workspace_size(N, total_T, H, dk, dv, chunk), 1),
                          dtype=torch.uint8, device=q.device)
         _lib.gdn_cp_local_state(q, k, v, g, beta, cu, loc, tr, chunk=chunk, l2norm=l2norm, workspace=ws)
@@ -60,12 +59,13 @@ def cp_chunk_prefill(q, k, v, g, beta, cu_seqlens, o, initial_state=None, final_
     rank = dist.get_rank(group)
     ranks = dist.get_world_size(group)
     loc, tr, ctx = ops.local_state(q, k, v, g, beta, cu_seqlens, chunk, l2norm)
-    parts_loc = [torch.empty_like(loc) for _ in range(ranks)]
-    parts_tr = [torch.empty_like(tr) for _ in range(ranks)]
-    dist.all_gather(parts_loc, loc.contiguous(), group=group)
-    dist.all_gather(parts_tr, tr.contiguous(), group=group)
-    all_loc = torch.stack(parts_loc)  # rank-major [ranks, N, H, dv, dk]
-    all_tr = torch.stack(parts_tr)
+    # this rank's (H, M) as one flat buffer, so that a single all-gather carries both
+    pair = torch.cat((loc.contiguous().view(-1), tr.contiguous().view(-1)))
+    parts = [torch.empty_like(pair) for _ in range(ranks)]
+    dist.all_gather(parts, pair, group=group)
+    gathered = torch.stack(parts)  # rank-major [ranks, |H| + |M|]
+    all_loc = gathered[:, :loc.numel()].reshape((ranks,) + tuple(loc.shape)).contiguous()
+    all_tr = gathered[:, loc.numel():].reshape((ranks,) + tuple(tr.shape)).contiguous()
     start = ops.combine(all_loc, all_tr, rank, initial_state)
     ops.prefill(q, k, v, g, beta, cu_seqlens, o, start, final_state, chunk, scale, l2norm, ctx)
     return o

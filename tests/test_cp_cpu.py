@@ -37,6 +37,8 @@ def _oracle_ops():
         return torch.from_numpy(Ht), torch.from_numpy(Mt), None
 
     def combine(all_loc, all_tr, rank, initial_state):
+        # the library's combine takes contiguous rank-major arrays
+        assert all_loc.is_contiguous() and all_tr.is_contiguous()
         S = torch.zeros_like(all_loc[0]) if initial_state is None else initial_state.clone()
         for r in range(rank):
             S = torch.einsum("nhij,nhjk->nhik", S, all_tr[r]) + all_loc[r]
