@@ -97,3 +97,18 @@ def test_backward_through_the_qk_normalisation_small_heads_fp32():
                                 normalize_qk=False)
     d_o, d_fin = _upstream(inp, 103, torch.float32)
     _check(inp, d_o, d_fin, 16, "bwd l2norm d=64", l2norm=True)
+
+
+@pytest.mark.parametrize("chunk", [3, 7])
+def test_backward_odd_checkpoint_intervals_one_shared_qk_head(chunk):
+    """Checkpoint intervals that divide no sequence length (the staging order then has
+    a short last chunk), all value heads on one q/k head, d=64 bf16."""
+    inp = inputs.prefill_inputs([50, 1, 64, 33], 3, 64, 64, seed=104 + chunk, g_range=(0.0, 0.1), H_qk=1)
+    d_o, d_fin = _upstream(inp, 105, torch.bfloat16)
+    _check(inp, d_o, d_fin, chunk, f"bwd chunk={chunk} H_qk=1")
+
+
+def test_backward_fp32_inputs_full_head_size():
+    inp = inputs.prefill_inputs([129, 64, 5], 2, 128, 128, seed=106, dtype=torch.float32, g_range=(0.0, 0.05))
+    d_o, d_fin = _upstream(inp, 107, torch.float32)
+    _check(inp, d_o, d_fin, 5, "bwd fp32 d=128 chunk=5")
