@@ -112,3 +112,34 @@ def test_backward_fp32_inputs_full_head_size():
     inp = inputs.prefill_inputs([129, 64, 5], 2, 128, 128, seed=106, dtype=torch.float32, g_range=(0.0, 0.05))
     d_o, d_fin = _upstream(inp, 107, torch.float32)
     _check(inp, d_o, d_fin, 5, "bwd fp32 d=128 chunk=5")
+
+
+def test_backward_full_size_bench_workload_sampled_heads():
+    """The bench's backward workload (B=4 x 8192, H=16, bf16, checkpoints every 16
+    tokens) in the launch configuration the bench times; three (sequence, head) pairs,
+    each its own chain (H_qk = H), against the oracle run on that pair alone."""
+    import bench
+    inp, d_o, d_fin, chunk, _ = bench.backward_inputs("backward", torch.device(DEV), 0)
+    assert inp.q.shape[1] == inp.v.shape[1]
+    out = gdn.gdn_chunk_prefill_backward(inp.q, inp.k, inp.v, inp.g, inp.beta, inp.cu_seqlens, d_o,
+                                         initial_state=inp.initial_state, d_final_state=d_fin, chunk=chunk,
+                                         scale=inp.scale)
+    torch.cuda.synchronize()
+    assert gdn.gdn_get_device_error() == 0
+    cu = inp.cu_seqlens.cpu().tolist()
+    for n, h in ((0, 0), (1, 7), (3, 15)):
+        a, b = cu[n], cu[n + 1]
+
+        def tok(x):
+            return x[a:b, h:h + 1].cpu()
+
+        def state(x):
+            return x[n:n + 1, h:h + 1].cpu()
+
+        ref = oracle.prefill_backward(tok(inp.q), tok(inp.k), tok(inp.v), tok(inp.g), tok(inp.beta),
+                                      torch.tensor([0, b - a], dtype=torch.int32), tok(d_o),
+                                      state(inp.initial_state), state(d_fin), scale=inp.scale)
+        got = {name: tok(out[name]) for name in ("dq", "dk", "dv", "dg", "dbeta")}
+        got["d_initial_state"] = state(out["d_initial_state"])
+        for name in ref:
+            assert_close(got[name], ref[name], what=f"bwd full size n={n} h={h} {name}")
