@@ -616,7 +616,7 @@ def bench_cp(key, steps, warmup, peaks):
         "tokens_per_s": T / (ms * 1e-3),
         "exchange_bytes_per_rank": exchange,
         "roofline": {"bound": "hbm", "achieved": achieved, "peak": peaks["hbm_gbs"] * R, "unit": "GB/s",
-                     "frac": achieved / (peaks["hbm_gbs"] * R), "traffic": None,
+                     "frac": achieved / (peaks["hbm_gbs"] * R), "traffic": ncu_traffic(key),
                      "note": f"peak = {R} GPUs' copy bandwidth; not a multi-GPU measurement"},
         "alg_bytes": alg_b,
     }
