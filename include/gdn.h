@@ -29,7 +29,9 @@
  *    of the FlashInfer PR #6291 page, section 3).
  *  - Every host-checkable error (null or misaligned pointer, bad size, unsupported
  *    combination, small workspace) returns a non-OK status BEFORE anything is
- *    launched; gdn_last_error() then gives a message (thread-local). Errors that
+ *    launched; gdn_last_error() then gives a message (thread-local). This follows the
+ *    host launcher of the FlashInfer PR #4593 page (section 1), which checks its
+ *    arguments and reports each failure with a message before any launch. Errors that
  *    only the data can show (slot id out of range, non-monotone cu_seqlens) are
  *    detected on the device: the offending unit is skipped (never an out-of-bounds
  *    access) and a sticky device error word is set, read by gdn_get_device_error().
